@@ -1,0 +1,97 @@
+"""fp64 CPU oracle for the key-axis-gated delta-rule recurrence.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by ``__graft_entry__.smoke()`` and
+by the CPU-baseline / reference legs of ``bench.py``.  The product path (the CUDA
+library and its binding) never imports it.
+
+``gdr_fwd`` and ``gdr_decode_step`` wrap the token-by-token C recurrence in
+``gdr_oracle.c`` (the definition written out; see that file's header for the
+passages it follows).  ``chunk_wy`` and ``chunk_ut`` restate the chunk-parallel
+algebra in fp64 numpy so the tests can check it against the recurrence, as the
+"Semidirect Fourier Delta Attention" page reports doing in its results section
+(numerical verification against brute force).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+GATE_LOGDECAY = 0
+GATE_NEG_SOFTPLUS = 1
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_gdr_fwd.argtypes = [ctypes.c_int] * 7 + [ctypes.c_double] + [dp] * 9
+        lib.oracle_gdr_fwd.restype = None
+        lib.oracle_gdr_decode_step.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [dp] * 8
+        lib.oracle_gdr_decode_step.restype = None
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    if a is None:
+        return None
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return ctypes.POINTER(ctypes.c_double)()
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def gdr_fwd(q, k, v, g, beta, theta=None, S0=None, gate_mode=GATE_LOGDECAY, scale=1.0,
+            want_state=True):
+    """Token-by-token fp64 forward.
+
+    q, k: [B,T,H,dk]; v: [B,T,H,dv]; g: [B,T,H,dk] (or dk/2 with rotation);
+    beta: [B,T,H]; theta: [B,T,H,dk/2] or None; S0: [B,H,dv,dk] or None.
+    Returns (o [B,T,H,dv], S_T [B,H,dv,dk] or None), both float64.
+    """
+    q, k, v, g, beta, theta, S0 = map(_f64, (q, k, v, g, beta, theta, S0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    rotation = theta is not None
+    assert k.shape == q.shape and v.shape == (B, T, H, dv) and beta.shape == (B, T, H)
+    assert g.shape == (B, T, H, dk // 2 if rotation else dk)
+    if rotation:
+        assert dk % 2 == 0 and theta.shape == (B, T, H, dk // 2)
+    if S0 is not None:
+        assert S0.shape == (B, H, dv, dk)
+    o = np.zeros((B, T, H, dv))
+    S_T = np.zeros((B, H, dv, dk)) if want_state else None
+    _load().oracle_gdr_fwd(B, T, H, dk, dv, int(gate_mode), int(rotation), float(scale),
+                           _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(theta),
+                           _ptr(S0), _ptr(o), _ptr(S_T))
+    return o, S_T
+
+
+def gdr_decode_step(q, k, v, g, beta, S, theta=None, gate_mode=GATE_LOGDECAY, scale=1.0):
+    """One fp64 decode step.  S [N,H,dv,dk] is NOT modified; returns (o, S_new)."""
+    q, k, v, g, beta, theta = map(_f64, (q, k, v, g, beta, theta))
+    S_new = np.array(S, dtype=np.float64, copy=True, order="C")
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    rotation = theta is not None
+    assert g.shape == (N, H, dk // 2 if rotation else dk) and beta.shape == (N, H)
+    o = np.zeros((N, H, dv))
+    _load().oracle_gdr_decode_step(N, H, dk, dv, int(gate_mode), int(rotation), float(scale),
+                                   _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                   _ptr(theta), _ptr(S_new), _ptr(o))
+    return o, S_new
