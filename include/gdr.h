@@ -1,0 +1,167 @@
+/*
+ * gdr.h -- C ABI of libgdr.so: the key-axis-gated delta-rule recurrence on B200.
+ *
+ * The operation (one head of one sequence, tokens t = 1..T, state S_t in R^{dv x dk}):
+ *
+ *     S_t = S_{t-1} D_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,     o_t = S_t (scale * q_t)
+ *
+ *   - "Semidirect Fourier Delta Attention" page, section "Core architecture":
+ *     the state is decayed, then erased along k_t, then written with
+ *     beta_t k_t v_t^*.  The page's state is dk x dv and is acted on from the left;
+ *     this library stores its transpose (value rows, key columns), as the
+ *     "CARVE" page does in section 1.
+ *   - "CARVE" page, section 2.3: the decay is a key-axis exponential gate,
+ *     D_t = diag(exp(g_t)), g_t <= 0 (rotation off).
+ *   - "Semidirect Fourier Delta Attention" page, "Core architecture", real
+ *     implementation: with rotation on, D_t is a direct sum of 2x2 rotation-decay
+ *     blocks.  Key pair j = (2j, 2j+1) of every row of S, read as x + i y, is
+ *     multiplied by alpha_{t,j} e^{i theta_{t,j}}, alpha = exp(g_{t,j}).  That is
+ *     the transpose of the page's Lambda_t = diag(alpha_t e^{i theta_t}).
+ *   - The readout uses the post-update state S_t.
+ *
+ * Gate activation (fused in the kernels; "CARVE" page, section 2.3, gate in
+ * kernel): GDR_GATE_LOGDECAY reads g itself; GDR_GATE_NEG_SOFTPLUS reads a raw
+ * gate a and uses g = -softplus(a) = log sigmoid(-a).
+ *
+ * Common conventions
+ *   - Every pointer is a DEVICE pointer unless stated otherwise.  The caller owns
+ *     all buffers and the stream.  The library allocates no memory.
+ *   - All calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream).  Argument checks are synchronous and
+ *     return before anything is launched.
+ *   - Layouts are dense row-major, last index fastest.  Every pointer must be
+ *     16-byte aligned.
+ *   - Element types: q, k, v use `qkv_dtype`; o uses `out_dtype`; g, beta, theta,
+ *     S0, S_T and the decode state S are always fp32.
+ *   - Errors: GDR_ERR_INVALID_ARG / GDR_ERR_UNSUPPORTED mean nothing was
+ *     launched.  GDR_ERR_CUDA means a launch failed (see gdr_last_error_detail).
+ *     No call aborts or throws.
+ */
+#ifndef GDR_H
+#define GDR_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDR_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define GDR_API __attribute__((visibility("default")))
+#else
+#define GDR_API
+#endif
+
+typedef void* gdr_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or enum; nothing launched */
+    GDR_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. dk not in {32,64,128}) */
+    GDR_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    GDR_ERR_TIMEOUT = 4,     /* a kernel gave up on a bounded wait (device status word) */
+    GDR_ERR_WORKSPACE = 5    /* workspace pointer NULL or smaller than required */
+} gdr_status;
+
+typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+
+typedef enum { GDR_GATE_LOGDECAY = 0, GDR_GATE_NEG_SOFTPLUS = 1 } gdr_gate_mode;
+
+typedef enum {
+    GDR_ALGO_AUTO = 0,    /* tensor-core chunk kernel when supported, else SIMT */
+    GDR_ALGO_SIMT = 1,    /* fp32 CUDA-core chunk-WY kernel (every supported shape) */
+    GDR_ALGO_TCGEN05 = 2  /* tcgen05/TMEM chunk-WY kernel: bf16 q/k/v, dk = dv = 128 */
+} gdr_algo;
+
+/* Shape and mode of one chunked forward call. */
+typedef struct {
+    int B, H, T;          /* batch, heads, tokens (T >= 0; T = 0 only copies S0 to S_T) */
+    int dk, dv;           /* key / value head dims, each in {32, 64, 128} */
+    int chunk;            /* chunk length; must be 64 */
+    gdr_dtype qkv_dtype;  /* storage of q, k, v */
+    gdr_dtype out_dtype;  /* storage of o */
+    gdr_gate_mode gate_mode;
+    int rotation;         /* 0: real key-axis decay; 1: 2x2 rotation-decay blocks */
+    float scale;          /* multiplies q (1.0 for none) */
+    gdr_algo algo;
+} gdr_fwd_desc;
+
+/* Shape and mode of one decode step over N independent sequences. */
+typedef struct {
+    int N, H;             /* sequences, heads */
+    int dk, dv;           /* each in {32, 64, 128} */
+    gdr_dtype qkv_dtype, out_dtype;
+    gdr_gate_mode gate_mode;
+    int rotation;
+    float scale;
+} gdr_dec_desc;
+
+/* GDR_ABI_VERSION of the loaded library. */
+GDR_API int gdr_abi_version(void);
+
+/* Static, NUL-terminated name of a status code. */
+GDR_API const char* gdr_status_string(gdr_status s);
+
+/* Detail of the last GDR_ERR_* returned on the calling host thread (static
+ * thread-local string; empty when there is none). */
+GDR_API const char* gdr_last_error_detail(void);
+
+/* Bytes of device workspace gdr_chunk_fwd needs for this descriptor (0 = none;
+ * the workspace argument may then be NULL).  Returns 0 for an invalid desc. */
+GDR_API size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc);
+
+/*
+ * Chunk-parallel forward over whole sequences (chunk-WY / UT-transform solver).
+ *
+ * Source: the WY-form triangular chunk solver that batches a chunk's tokens into
+ * one linear system ("CARVE" page, section 1 item 3, section 3 item 1), in the
+ * constructive form of the "Semidirect Fourier Delta Attention" page (section
+ * "Constructive Chunk-WY Theorem": the in-chunk correction has rank <= chunk;
+ * section "Main contributions": exact affine chunk transfer of the state).
+ *
+ *   q, k  [B,T,H,dk]  qkv_dtype          v  [B,T,H,dv]  qkv_dtype
+ *   g     [B,T,H,dk]  fp32 (rotation: [B,T,H,dk/2], one decay per key pair)
+ *   beta  [B,T,H]     fp32, the write strength (0 <= beta <= 1 expected)
+ *   theta [B,T,H,dk/2] fp32 angles; must be NULL unless rotation
+ *   S0    [B,H,dv,dk] fp32 initial state, or NULL for zeros
+ *   o     [B,T,H,dv]  out_dtype (written)
+ *   S_T   [B,H,dv,dk] fp32 final state, or NULL to skip (may alias S0)
+ *   workspace / workspace_bytes: see gdr_chunk_fwd_workspace_bytes.
+ *
+ * Numerical range: the kernels factor exp(Gamma_r - Gamma_i) through per-chunk
+ * reference points; a key dim whose log-decay over 32 consecutive tokens is
+ * below -80 may overflow the factored form (GDR_ALGO_TCGEN05 only).
+ */
+GDR_API gdr_status gdr_chunk_fwd(const gdr_fwd_desc* desc,
+                         const void* q, const void* k, const void* v,
+                         const float* g, const float* beta, const float* theta,
+                         const float* S0, void* o, float* S_T,
+                         void* workspace, size_t workspace_bytes,
+                         gdr_stream_t stream);
+
+/*
+ * One recurrent decode step: the token update above applied once to each of
+ * N*H states, in place.  Reads and writes S exactly once.
+ *
+ *   q, k [N,H,dk] qkv_dtype;  v [N,H,dv] qkv_dtype;  g [N,H,dk] (rotation: [N,H,dk/2]);
+ *   beta [N,H];  theta [N,H,dk/2] or NULL;  S [N,H,dv,dk] fp32, in/out;  o [N,H,dv] out_dtype.
+ */
+GDR_API gdr_status gdr_decode_step(const gdr_dec_desc* desc,
+                           const void* q, const void* k, const void* v,
+                           const float* g, const float* beta, const float* theta,
+                           float* S, void* o, gdr_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word that
+ * kernels set when a bounded wait gives up.  Returns GDR_OK, GDR_ERR_TIMEOUT or
+ * GDR_ERR_CUDA (a sticky CUDA error on the context).  Uses the current device.
+ */
+GDR_API gdr_status gdr_query_device_status(gdr_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H */

@@ -1,0 +1,157 @@
+// decode.cuh -- one recurrent decode step, HBM-bound: S is read once and written once.
+//
+// Per value row s (one row of S, dk wide), with X = S D_t:
+//   x_k = (s D_t) . k,   x_q = (s D_t) . q,   e = beta (v_row - x_k)
+//   s  <- s D_t + e k^T,   o_row = x_q + e (k . q)
+// which is the token update of the "Semidirect Fourier Delta Attention" page
+// ("Core architecture": decay, erase along k, write v) transposed to value rows,
+// with the readout o = S_t q taken from the updated row without a second pass.
+//
+// Layout: one warp owns a row at a time; lane l holds dims [VEC*l, VEC*l + VEC)
+// (VEC = dk/32), so a row is one coalesced 128-bit (dk = 128) access per lane.
+// Each warp keeps ROWS rows in flight; CTAs are ROWS*8 rows of one head.
+#pragma once
+
+#include "common.cuh"
+
+namespace gdr {
+namespace dec {
+
+struct DecParams {
+    int N, H, dv;
+    int gate_mode;
+    float scale;
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    const float* theta;
+    float* S;
+    void* o;
+};
+
+constexpr int WARPS = 8;
+constexpr int ROWS = 8;                       // rows per warp per CTA
+constexpr int ROWS_PER_CTA = WARPS * ROWS;    // 64
+
+template <int VEC> struct Vec;
+template <> struct Vec<4> { using T = float4; };
+template <> struct Vec<2> { using T = float2; };
+template <> struct Vec<1> { using T = float; };
+
+template <int VEC>
+__device__ __forceinline__ void unpack(const typename Vec<VEC>::T& x, float (&a)[VEC]) {
+    if constexpr (VEC == 4) { a[0] = x.x; a[1] = x.y; a[2] = x.z; a[3] = x.w; }
+    else if constexpr (VEC == 2) { a[0] = x.x; a[1] = x.y; }
+    else { a[0] = x; }
+}
+template <int VEC>
+__device__ __forceinline__ typename Vec<VEC>::T pack(const float (&a)[VEC]) {
+    if constexpr (VEC == 4) return make_float4(a[0], a[1], a[2], a[3]);
+    else if constexpr (VEC == 2) return make_float2(a[0], a[1]);
+    else return a[0];
+}
+
+template <int DK, bool ROT, typename QT, typename OT>
+__global__ void __launch_bounds__(WARPS * 32) decode_kernel(DecParams p) {
+    constexpr int VEC = DK / 32;
+    static_assert(!ROT || VEC % 2 == 0 || VEC == 1, "pairs");
+    using VT = typename Vec<VEC>::T;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int row_blocks = (p.dv + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
+    const int nh = blockIdx.x / row_blocks;
+    const int row0 = (blockIdx.x % row_blocks) * ROWS_PER_CTA + warp * ROWS;
+    const QT* q = static_cast<const QT*>(p.q) + (size_t)nh * DK;
+    const QT* k = static_cast<const QT*>(p.k) + (size_t)nh * DK;
+    const QT* v = static_cast<const QT*>(p.v) + (size_t)nh * p.dv;
+    OT* o = static_cast<OT*>(p.o) + (size_t)nh * p.dv;
+    float* S = p.S + (size_t)nh * p.dv * DK;
+
+    // Issue the state loads first: they are the only large traffic.
+    VT sv[ROWS];
+#pragma unroll
+    for (int rr = 0; rr < ROWS; ++rr) {
+        const int row = row0 + rr;
+        if (row < p.dv) sv[rr] = __ldcs(reinterpret_cast<const VT*>(S + (size_t)row * DK) + lane);
+    }
+
+    // This lane's slice of k, q and the decay (real: per dim; rotation: per pair).
+    float kk[VEC], qq[VEC], al[VEC], cs[VEC], sn[VEC];
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) {
+        const int d = lane * VEC + u;
+        kk[u] = ld_f32(k + d);
+        qq[u] = p.scale * ld_f32(q + d);
+    }
+    if constexpr (!ROT) {
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) al[u] = decay_factor(p.g[(size_t)nh * DK + lane * VEC + u], p.gate_mode);
+    } else if constexpr (VEC >= 2) {
+#pragma unroll
+        for (int u = 0; u < VEC; u += 2) {
+            const int jp = (lane * VEC + u) / 2;
+            const float a = decay_factor(p.g[(size_t)nh * (DK / 2) + jp], p.gate_mode);
+            float s_, c_;
+            sincosf(p.theta[(size_t)nh * (DK / 2) + jp], &s_, &c_);
+            al[u] = a; cs[u] = c_; sn[u] = s_;
+        }
+    }
+    // Rotation with one dim per lane (dk = 32): a pair spans lanes 2m, 2m+1.
+    float pair_c = 0.f, pair_s = 0.f, pair_a = 0.f;
+    if constexpr (ROT && VEC == 1) {
+        const int jp = lane / 2;
+        pair_a = decay_factor(p.g[(size_t)nh * (DK / 2) + jp], p.gate_mode);
+        sincosf(p.theta[(size_t)nh * (DK / 2) + jp], &pair_s, &pair_c);
+    }
+    float kq = 0.f;
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) kq = fmaf(kk[u], qq[u], kq);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    const float bt = p.beta[nh];
+    const float vrow = (row0 + lane < p.dv && lane < ROWS) ? ld_f32(v + row0 + lane) : 0.f;
+
+    float orow = 0.f;
+#pragma unroll
+    for (int rr = 0; rr < ROWS; ++rr) {
+        const int row = row0 + rr;
+        if (row >= p.dv) break;
+        float s[VEC];
+        unpack<VEC>(sv[rr], s);
+        // X = s D_t
+        if constexpr (!ROT) {
+#pragma unroll
+            for (int u = 0; u < VEC; ++u) s[u] *= al[u];
+        } else if constexpr (VEC >= 2) {
+#pragma unroll
+            for (int u = 0; u < VEC; u += 2) {
+                const float x = s[u], y = s[u + 1];
+                s[u] = al[u] * (cs[u] * x - sn[u] * y);
+                s[u + 1] = al[u] * (sn[u] * x + cs[u] * y);
+            }
+        } else {
+            const float other = __shfl_xor_sync(0xffffffffu, s[0], 1);
+            const float x = (lane & 1) ? other : s[0];
+            const float y = (lane & 1) ? s[0] : other;
+            s[0] = pair_a * ((lane & 1) ? (pair_s * x + pair_c * y) : (pair_c * x - pair_s * y));
+        }
+        float xk = 0.f, xq = 0.f;
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) { xk = fmaf(s[u], kk[u], xk); xq = fmaf(s[u], qq[u], xq); }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            xk += __shfl_xor_sync(0xffffffffu, xk, off);
+            xq += __shfl_xor_sync(0xffffffffu, xq, off);
+        }
+        const float e = bt * (__shfl_sync(0xffffffffu, vrow, rr) - xk);
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) s[u] = fmaf(e, kk[u], s[u]);
+        __stcs(reinterpret_cast<VT*>(S + (size_t)row * DK) + lane, pack<VEC>(s));
+        if (lane == rr) orow = fmaf(e, kq, xq);
+    }
+    if (lane < ROWS && row0 + lane < p.dv) st_from_f32(o + row0 + lane, orow);
+}
+
+}  // namespace dec
+}  // namespace gdr

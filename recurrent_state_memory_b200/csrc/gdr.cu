@@ -1,0 +1,221 @@
+// gdr.cu -- the C ABI declared in include/gdr.h: argument checks and kernel dispatch.
+//
+// All kernels are compiled into this one translation unit so that the device
+// status word below is a single symbol per loaded module.
+#include <cstdio>
+#include <cstring>
+
+#include "gdr.h"
+#include "common.cuh"
+#include "simt_fwd.cuh"
+#include "decode.cuh"
+
+namespace gdr {
+
+// Set by kernels that give up on a bounded wait (GDR_ERR_TIMEOUT); read and
+// cleared by gdr_query_device_status.
+__device__ unsigned int g_device_status = 0;
+
+static thread_local char t_detail[256] = "";
+
+static gdr_status fail(gdr_status s, const char* fmt, const char* what = "") {
+    snprintf(t_detail, sizeof(t_detail), fmt, what);
+    return s;
+}
+
+static gdr_status cuda_fail(cudaError_t e, const char* where) {
+    snprintf(t_detail, sizeof(t_detail), "%s: %s", where, cudaGetErrorString(e));
+    return GDR_ERR_CUDA;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+static bool dtype_ok(gdr_dtype t) { return t == GDR_F32 || t == GDR_BF16; }
+
+// ---------------------------------------------------------------- forward ----
+
+template <int DK, bool ROT, typename QT, typename OT>
+static gdr_status launch_simt(const FwdParams& p, cudaStream_t st) {
+    using L = simt::Smem<DK, ROT>;
+    auto kern = simt::chunk_fwd_kernel<DK, ROT, QT, OT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(simt chunk kernel)");
+    dim3 grid(p.B * p.H, p.dv / simt::DVT);
+    kern<<<grid, simt::NT, L::bytes, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch(simt chunk kernel)");
+    return GDR_OK;
+}
+
+template <int DK, bool ROT>
+static gdr_status dispatch_simt_types(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st) {
+    const bool qb = d->qkv_dtype == GDR_BF16, ob = d->out_dtype == GDR_BF16;
+    if (qb && ob) return launch_simt<DK, ROT, __nv_bfloat16, __nv_bfloat16>(p, st);
+    if (qb && !ob) return launch_simt<DK, ROT, __nv_bfloat16, float>(p, st);
+    if (!qb && ob) return launch_simt<DK, ROT, float, __nv_bfloat16>(p, st);
+    return launch_simt<DK, ROT, float, float>(p, st);
+}
+
+template <bool ROT>
+static gdr_status dispatch_simt_dk(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st) {
+    switch (d->dk) {
+        case 32: return dispatch_simt_types<32, ROT>(d, p, st);
+        case 64: return dispatch_simt_types<64, ROT>(d, p, st);
+        default: return dispatch_simt_types<128, ROT>(d, p, st);
+    }
+}
+
+static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
+    if (!d) return fail(GDR_ERR_INVALID_ARG, "desc is NULL%s");
+    if (d->B < 0 || d->H < 0 || d->T < 0) return fail(GDR_ERR_INVALID_ARG, "B, H, T must be >= 0%s");
+    if (!head_dim_ok(d->dk) || !head_dim_ok(d->dv))
+        return fail(GDR_ERR_UNSUPPORTED, "dk and dv must each be 32, 64 or 128%s");
+    if (d->chunk != 64) return fail(GDR_ERR_UNSUPPORTED, "chunk must be 64%s");
+    if (!dtype_ok(d->qkv_dtype) || !dtype_ok(d->out_dtype)) return fail(GDR_ERR_INVALID_ARG, "bad dtype%s");
+    if (d->gate_mode != GDR_GATE_LOGDECAY && d->gate_mode != GDR_GATE_NEG_SOFTPLUS)
+        return fail(GDR_ERR_INVALID_ARG, "bad gate_mode%s");
+    if (d->rotation != 0 && d->rotation != 1) return fail(GDR_ERR_INVALID_ARG, "rotation must be 0 or 1%s");
+    if (d->algo != GDR_ALGO_AUTO && d->algo != GDR_ALGO_SIMT && d->algo != GDR_ALGO_TCGEN05)
+        return fail(GDR_ERR_INVALID_ARG, "bad algo%s");
+    if ((long long)d->B * d->H > 0x7fffffffLL) return fail(GDR_ERR_INVALID_ARG, "B*H too large%s");
+    if (d->algo == GDR_ALGO_TCGEN05) return fail(GDR_ERR_UNSUPPORTED, "tcgen05 kernel not built in this library%s");
+    return GDR_OK;
+}
+
+// ----------------------------------------------------------------- decode ----
+
+template <int DK, bool ROT, typename QT, typename OT>
+static gdr_status launch_decode(const dec::DecParams& p, cudaStream_t st) {
+    const int row_blocks = (p.dv + dec::ROWS_PER_CTA - 1) / dec::ROWS_PER_CTA;
+    const long long grid = (long long)p.N * p.H * row_blocks;
+    if (grid > 0x7fffffffLL) return fail(GDR_ERR_INVALID_ARG, "N*H too large%s");
+    dec::decode_kernel<DK, ROT, QT, OT><<<(unsigned)grid, dec::WARPS * 32, 0, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch(decode kernel)");
+    return GDR_OK;
+}
+
+template <int DK, bool ROT>
+static gdr_status decode_types(const gdr_dec_desc* d, const dec::DecParams& p, cudaStream_t st) {
+    const bool qb = d->qkv_dtype == GDR_BF16, ob = d->out_dtype == GDR_BF16;
+    if (qb && ob) return launch_decode<DK, ROT, __nv_bfloat16, __nv_bfloat16>(p, st);
+    if (qb && !ob) return launch_decode<DK, ROT, __nv_bfloat16, float>(p, st);
+    if (!qb && ob) return launch_decode<DK, ROT, float, __nv_bfloat16>(p, st);
+    return launch_decode<DK, ROT, float, float>(p, st);
+}
+
+}  // namespace gdr
+
+using namespace gdr;
+
+extern "C" {
+
+int gdr_abi_version(void) { return GDR_ABI_VERSION; }
+
+const char* gdr_status_string(gdr_status s) {
+    switch (s) {
+        case GDR_OK: return "GDR_OK";
+        case GDR_ERR_INVALID_ARG: return "GDR_ERR_INVALID_ARG";
+        case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED";
+        case GDR_ERR_CUDA: return "GDR_ERR_CUDA";
+        case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
+        case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE";
+    }
+    return "GDR_ERR_UNKNOWN";
+}
+
+const char* gdr_last_error_detail(void) { return t_detail; }
+
+size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc) {
+    if (check_fwd_desc(desc) != GDR_OK) return 0;
+    return 0;
+}
+
+gdr_status gdr_chunk_fwd(const gdr_fwd_desc* d, const void* q, const void* k, const void* v,
+                         const float* g, const float* beta, const float* theta, const float* S0,
+                         void* o, float* S_T, void* workspace, size_t workspace_bytes,
+                         gdr_stream_t stream) {
+    t_detail[0] = 0;
+    gdr_status s = check_fwd_desc(d);
+    if (s != GDR_OK) return s;
+    if (d->B == 0 || d->H == 0) return GDR_OK;
+    if (d->T > 0) {
+        if (!q || !k || !v || !g || !beta || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta and o are required%s");
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) || !aligned16(o))
+            return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
+        if (d->rotation && !theta) return fail(GDR_ERR_INVALID_ARG, "theta is required with rotation%s");
+    }
+    if (!d->rotation && theta) return fail(GDR_ERR_INVALID_ARG, "theta must be NULL without rotation%s");
+    if ((theta && !aligned16(theta)) || (S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
+        return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
+    const size_t need = gdr_chunk_fwd_workspace_bytes(d);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return fail(GDR_ERR_WORKSPACE, "workspace too small%s");
+
+    FwdParams p;
+    p.B = d->B; p.H = d->H; p.T = d->T; p.dv = d->dv;
+    p.gate_mode = (int)d->gate_mode;
+    p.scale = d->scale;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.theta = theta;
+    p.S0 = S0; p.o = o; p.S_T = S_T;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (d->T == 0 && !S_T) return GDR_OK;
+    return d->rotation ? dispatch_simt_dk<true>(d, p, st) : dispatch_simt_dk<false>(d, p, st);
+}
+
+gdr_status gdr_decode_step(const gdr_dec_desc* d, const void* q, const void* k, const void* v,
+                           const float* g, const float* beta, const float* theta, float* S,
+                           void* o, gdr_stream_t stream) {
+    t_detail[0] = 0;
+    if (!d) return fail(GDR_ERR_INVALID_ARG, "desc is NULL%s");
+    if (d->N < 0 || d->H < 0) return fail(GDR_ERR_INVALID_ARG, "N, H must be >= 0%s");
+    if (!head_dim_ok(d->dk) || !head_dim_ok(d->dv))
+        return fail(GDR_ERR_UNSUPPORTED, "dk and dv must each be 32, 64 or 128%s");
+    if (!dtype_ok(d->qkv_dtype) || !dtype_ok(d->out_dtype)) return fail(GDR_ERR_INVALID_ARG, "bad dtype%s");
+    if (d->gate_mode != GDR_GATE_LOGDECAY && d->gate_mode != GDR_GATE_NEG_SOFTPLUS)
+        return fail(GDR_ERR_INVALID_ARG, "bad gate_mode%s");
+    if (d->rotation != 0 && d->rotation != 1) return fail(GDR_ERR_INVALID_ARG, "rotation must be 0 or 1%s");
+    if (d->N == 0 || d->H == 0) return GDR_OK;
+    if (!q || !k || !v || !g || !beta || !S || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta, S and o are required%s");
+    if (d->rotation && !theta) return fail(GDR_ERR_INVALID_ARG, "theta is required with rotation%s");
+    if (!d->rotation && theta) return fail(GDR_ERR_INVALID_ARG, "theta must be NULL without rotation%s");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) ||
+        !aligned16(S) || !aligned16(o) || (theta && !aligned16(theta)))
+        return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
+    dec::DecParams p;
+    p.N = d->N; p.H = d->H; p.dv = d->dv;
+    p.gate_mode = (int)d->gate_mode;
+    p.scale = d->scale;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.theta = theta; p.S = S; p.o = o;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (d->rotation) {
+        switch (d->dk) {
+            case 32: return decode_types<32, true>(d, p, st);
+            case 64: return decode_types<64, true>(d, p, st);
+            default: return decode_types<128, true>(d, p, st);
+        }
+    }
+    switch (d->dk) {
+        case 32: return decode_types<32, false>(d, p, st);
+        case 64: return decode_types<64, false>(d, p, st);
+        default: return decode_types<128, false>(d, p, st);
+    }
+}
+
+gdr_status gdr_query_device_status(gdr_stream_t stream) {
+    t_detail[0] = 0;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int word = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&word, g_device_status, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol(status)");
+    if (word != 0) {
+        e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(status)");
+        snprintf(t_detail, sizeof(t_detail), "device status word 0x%08x", word);
+        return GDR_ERR_TIMEOUT;
+    }
+    return GDR_OK;
+}
+
+}  // extern "C"

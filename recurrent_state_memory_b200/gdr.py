@@ -1,0 +1,223 @@
+"""Thin ctypes binding over libgdr.so (C ABI in include/gdr.h).
+
+Argument marshalling only: every step of the recurrence runs in the library's
+CUDA kernels.  torch is used for device memory and streams.  There is no CPU
+fallback: if the library is missing or a call fails, an exception is raised.
+
+Layouts follow include/gdr.h: q, k [B,T,H,dk]; v, o [B,T,H,dv]; g [B,T,H,dk]
+([B,T,H,dk/2] with rotation); beta [B,T,H]; theta [B,T,H,dk/2]; S [B,H,dv,dk].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdr.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gdr.h")
+
+GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT, GDR_ERR_WORKSPACE = range(6)
+GDR_F32, GDR_BF16 = 0, 1
+GATE_LOGDECAY, GATE_NEG_SOFTPLUS = 0, 1
+ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2}
+
+
+class FwdDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("qkv_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+                ("gate_mode", ctypes.c_int), ("rotation", ctypes.c_int),
+                ("scale", ctypes.c_float), ("algo", ctypes.c_int)]
+
+
+class DecDesc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int), ("H", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int),
+                ("qkv_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+                ("gate_mode", ctypes.c_int), ("rotation", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+class GdrError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: {status_string(status)} ({detail})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdr.so; raise if it has not been built (no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m recurrent_state_memory_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t
+        L.gdr_abi_version.restype = ctypes.c_int
+        L.gdr_status_string.restype = ctypes.c_char_p
+        L.gdr_status_string.argtypes = [ctypes.c_int]
+        L.gdr_last_error_detail.restype = ctypes.c_char_p
+        L.gdr_chunk_fwd_workspace_bytes.restype = sz
+        L.gdr_chunk_fwd_workspace_bytes.argtypes = [ctypes.POINTER(FwdDesc)]
+        L.gdr_chunk_fwd.restype = ctypes.c_int
+        L.gdr_chunk_fwd.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp, vp, sz, vp]
+        L.gdr_decode_step.restype = ctypes.c_int
+        L.gdr_decode_step.argtypes = [ctypes.POINTER(DecDesc), vp, vp, vp, fp, fp, fp, fp, vp, vp]
+        L.gdr_query_device_status.restype = ctypes.c_int
+        L.gdr_query_device_status.argtypes = [vp]
+        if L.gdr_abi_version() != 1:
+            raise RuntimeError("libgdr.so ABI version mismatch")
+        _lib = L
+    return _lib
+
+
+def header_symbols() -> list:
+    """Names of the entry points include/gdr.h declares."""
+    text = open(HEADER_PATH).read()
+    return re.findall(r"GDR_API\s+[\w\s\*]+?\b(gdr_\w+)\s*\(", text)
+
+
+def status_string(s: int) -> str:
+    return lib().gdr_status_string(int(s)).decode()
+
+
+def _check(status: int, where: str):
+    if status != GDR_OK:
+        raise GdrError(status, where, lib().gdr_last_error_detail().decode())
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return GDR_BF16
+    if t == torch.float32:
+        return GDR_F32
+    raise TypeError(f"unsupported dtype {t} (bf16 or fp32)")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream], device) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, device=None):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def fwd_desc(B, H, T, dk, dv, qkv_dtype, out_dtype, gate_mode=GATE_NEG_SOFTPLUS, rotation=False,
+             scale=1.0, algo="auto", chunk=64) -> FwdDesc:
+    return FwdDesc(B, H, T, dk, dv, chunk, _dtype_code(qkv_dtype), _dtype_code(out_dtype),
+                   int(gate_mode), int(bool(rotation)), float(scale), ALGOS[algo])
+
+
+def workspace_bytes(desc: FwdDesc) -> int:
+    return int(lib().gdr_chunk_fwd_workspace_bytes(ctypes.byref(desc)))
+
+
+def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
+              algo="auto", out_dtype=None, want_state=True, o=None, S_T=None, workspace=None,
+              stream=None, chunk=64) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunk-parallel forward.  Returns (o, S_T).
+
+    With CUDA tensors the call is asynchronous on `stream` (default: the current
+    stream).  With host tensors the inputs are copied to the current device,
+    the library is called, and o / S_T are copied back (synchronising).
+    """
+    if not q.is_cuda:
+        return _chunk_fwd_host(q, k, v, g, beta, theta, S0, gate_mode=gate_mode, scale=scale,
+                               algo=algo, out_dtype=out_dtype, want_state=want_state, chunk=chunk)
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    rotation = theta is not None
+    out_dtype = out_dtype or q.dtype
+    _need(q, "q", device=dev)
+    _need(k, "k", q.dtype, dev)
+    _need(v, "v", q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    if tuple(k.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv):
+        raise ValueError("q, k, v shapes disagree")
+    if tuple(g.shape) != (B, T, H, dk // 2 if rotation else dk) or tuple(beta.shape) != (B, T, H):
+        raise ValueError("g or beta has the wrong shape")
+    if theta is not None:
+        _need(theta, "theta", torch.float32, dev)
+        if tuple(theta.shape) != (B, T, H, dk // 2):
+            raise ValueError("theta has the wrong shape")
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (B, H, dv, dk):
+            raise ValueError("S0 has the wrong shape")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=out_dtype, device=dev)
+    _need(o, "o", out_dtype, dev)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, dev)
+    desc = fwd_desc(B, H, T, dk, dv, q.dtype, out_dtype, gate_mode, rotation, scale, algo, chunk)
+    need = workspace_bytes(desc)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().gdr_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                             _ptr(theta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
+                             _stream_handle(stream, dev))
+    _check(st, "gdr_chunk_fwd")
+    return o, S_T
+
+
+def _chunk_fwd_host(q, k, v, g, beta, theta, S0, **kw):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    to = lambda t: None if t is None else t.to(dev, non_blocking=True)
+    o, S_T = chunk_fwd(to(q), to(k), to(v), to(g), to(beta), to(theta), to(S0), **kw)
+    o_h = o.to("cpu")
+    S_h = None if S_T is None else S_T.to("cpu")
+    return o_h, S_h
+
+
+def decode_step(q, k, v, g, beta, S, theta=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
+                out_dtype=None, o=None, stream=None) -> torch.Tensor:
+    """One decode step; S [N,H,dv,dk] (fp32) is updated in place.  Returns o [N,H,dv]."""
+    dev = S.device
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    rotation = theta is not None
+    out_dtype = out_dtype or q.dtype
+    _need(q, "q", device=dev)
+    _need(k, "k", q.dtype, dev)
+    _need(v, "v", q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(S, "S", torch.float32, dev)
+    if tuple(S.shape) != (N, H, dv, dk) or tuple(g.shape) != (N, H, dk // 2 if rotation else dk):
+        raise ValueError("S or g has the wrong shape")
+    if theta is not None:
+        _need(theta, "theta", torch.float32, dev)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=out_dtype, device=dev)
+    desc = DecDesc(N, H, dk, dv, _dtype_code(q.dtype), _dtype_code(out_dtype), int(gate_mode),
+                   int(rotation), float(scale))
+    st = lib().gdr_decode_step(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                               _ptr(theta), _ptr(S), _ptr(o), _stream_handle(stream, dev))
+    _check(st, "gdr_decode_step")
+    return o
+
+
+def query_device_status(stream=None) -> int:
+    """Synchronise and read/clear the device status word (GDR_OK or GDR_ERR_TIMEOUT)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    return int(lib().gdr_query_device_status(_stream_handle(stream, dev)))

@@ -1,0 +1,94 @@
+"""The C-ABI library: it loads, exports every entry point include/gdr.h declares,
+and rejects bad arguments before launching anything (no GPU needed)."""
+import ctypes
+
+import pytest
+
+from recurrent_state_memory_b200 import build as gdr_build
+
+
+@pytest.fixture(scope="module")
+def G():
+    gdr_build.build()
+    from recurrent_state_memory_b200 import gdr
+    gdr.lib()
+    return gdr
+
+
+def test_exports_every_declared_symbol(G):
+    names = G.header_symbols()
+    assert {"gdr_chunk_fwd", "gdr_decode_step", "gdr_query_device_status",
+            "gdr_chunk_fwd_workspace_bytes", "gdr_status_string", "gdr_abi_version",
+            "gdr_last_error_detail"} <= set(names)
+    for n in names:
+        assert hasattr(G.lib(), n), n
+
+
+def test_status_strings(G):
+    assert G.status_string(0) == "GDR_OK"
+    assert G.status_string(4) == "GDR_ERR_TIMEOUT"
+    assert G.status_string(99) == "GDR_ERR_UNKNOWN"
+
+
+def _call_fwd(G, desc, ptrs=None, ws=None, ws_bytes=0):
+    p = ptrs or {}
+    get = lambda n: ctypes.c_void_p(p[n]) if n in p else None
+    return G.lib().gdr_chunk_fwd(ctypes.byref(desc) if desc is not None else None,
+                                 get("q"), get("k"), get("v"), get("g"), get("beta"), get("theta"),
+                                 get("S0"), get("o"), get("S_T"), ws, ws_bytes, None)
+
+
+FAKE = {n: 0x10000 * (i + 1) for i, n in enumerate(["q", "k", "v", "g", "beta", "o", "S_T"])}
+
+
+def _desc(G, **kw):
+    import torch
+    base = dict(B=1, H=2, T=128, dk=64, dv=64, qkv_dtype=torch.bfloat16, out_dtype=torch.bfloat16)
+    base.update(kw)
+    return G.fwd_desc(**base)
+
+
+def test_rejects_bad_arguments_without_launching(G):
+    import torch
+    L = G.lib()
+    assert L.gdr_chunk_fwd(None, *([None] * 10), 0, None) == G.GDR_ERR_INVALID_ARG
+    assert _call_fwd(G, _desc(G, dk=48), FAKE) == G.GDR_ERR_UNSUPPORTED
+    assert _call_fwd(G, _desc(G, chunk=32), FAKE) == G.GDR_ERR_UNSUPPORTED
+    assert _call_fwd(G, _desc(G, B=-1), FAKE) == G.GDR_ERR_INVALID_ARG
+    d = _desc(G)
+    d.gate_mode = 7
+    assert _call_fwd(G, d, FAKE) == G.GDR_ERR_INVALID_ARG
+    d = _desc(G)
+    d.qkv_dtype = 5
+    assert _call_fwd(G, d, FAKE) == G.GDR_ERR_INVALID_ARG
+    missing = dict(FAKE)
+    del missing["q"]
+    assert _call_fwd(G, _desc(G), missing) == G.GDR_ERR_INVALID_ARG
+    assert b"required" in L.gdr_last_error_detail()
+    misaligned = dict(FAKE, k=FAKE["k"] + 8)
+    assert _call_fwd(G, _desc(G), misaligned) == G.GDR_ERR_INVALID_ARG
+    assert b"aligned" in L.gdr_last_error_detail()
+    assert _call_fwd(G, _desc(G), dict(FAKE, theta=0x900000)) == G.GDR_ERR_INVALID_ARG
+    assert _call_fwd(G, _desc(G, rotation=True), FAKE) == G.GDR_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op(G):
+    assert _call_fwd(G, _desc(G, B=0), {}) == G.GDR_OK
+    assert _call_fwd(G, _desc(G, H=0), {}) == G.GDR_OK
+
+
+def test_decode_rejects_bad_arguments(G):
+    import torch
+    L = G.lib()
+    d = G.DecDesc(4, 2, 128, 128, 1, 1, 1, 0, 1.0)
+    assert L.gdr_decode_step(None, *([None] * 8), None) == G.GDR_ERR_INVALID_ARG
+    assert L.gdr_decode_step(ctypes.byref(d), *([None] * 8), None) == G.GDR_ERR_INVALID_ARG
+    d.dk = 96
+    assert L.gdr_decode_step(ctypes.byref(d), *([None] * 8), None) == G.GDR_ERR_UNSUPPORTED
+    d0 = G.DecDesc(0, 2, 128, 128, 1, 1, 1, 0, 1.0)
+    assert L.gdr_decode_step(ctypes.byref(d0), *([None] * 8), None) == G.GDR_OK
+
+
+def test_workspace_query(G):
+    assert G.workspace_bytes(_desc(G)) >= 0
+    assert G.workspace_bytes(_desc(G, dk=48)) == 0

@@ -1,0 +1,154 @@
+"""GPU parity of the chunk-WY forward against the fp64 oracle (same seeded bytes)."""
+import numpy as np
+import pytest
+
+from recurrent_state_memory_b200 import inputs as I
+
+import parity_util as U
+
+pytestmark = pytest.mark.gpu
+
+ALGOS_ALL = ["simt"]
+
+
+@pytest.fixture(scope="module")
+def G():
+    from recurrent_state_memory_b200 import gdr
+    gdr.lib()
+    return gdr
+
+
+@pytest.mark.parametrize("algo", ALGOS_ALL)
+def test_tiny_fp32_config(G, algo):
+    """The tiny fp32 workload: B=1, H=2, T=256, dk=dv=32, chunk 64, seed 0."""
+    p = I.make_config("tiny_f32")
+    o, S = U.run_gpu_fwd(p, algo)
+    o_ref, S_ref = U.oracle_fwd(p)
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref, tol_o=1e-4, tol_s=1e-4)
+
+
+CASES = [
+    # (B, H, T, dk, dv, dtype, rotation, s0, scale)
+    (2, 3, 200, 32, 32, "f32", False, True, 1.0),
+    (1, 2, 130, 64, 64, "f32", True, True, 0.5),
+    (2, 2, 193, 128, 128, "f32", False, False, 1.0),
+    (1, 2, 257, 128, 128, "f32", True, True, 1.0),
+    (2, 2, 150, 64, 128, "f32", False, True, 1.0),
+    (1, 3, 100, 128, 32, "f32", True, False, 2.0),
+    (2, 2, 321, 128, 128, "bf16", False, True, 1.0),
+    (1, 2, 190, 128, 128, "bf16", True, True, 1.0),
+    (1, 2, 64, 128, 128, "bf16", False, False, 1.0),
+]
+
+
+@pytest.mark.parametrize("algo", ALGOS_ALL)
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B{}H{}T{}k{}v{}_{}{}{}".format(
+    c[0], c[1], c[2], c[3], c[4], c[5], "_rot" if c[6] else "", "_s0" if c[7] else ""))
+def test_parity_small(G, algo, case):
+    B, H, T, dk, dv, dtype, rot, s0, scale = case
+    p = I.make_fwd(B, T, H, dk, dv, dtype=dtype, seed=1000 + T + dk, rotation=rot,
+                   s0_std=0.5 if s0 else None, scale=scale)
+    o, S = U.run_gpu_fwd(p, algo)
+    o_ref, S_ref = U.oracle_fwd(p)
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref, tol_s=1e-4 if dtype == "f32" else U.TOL_S)
+
+
+@pytest.mark.parametrize("algo", ALGOS_ALL)
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 128, 129])
+def test_chunk_edges(G, algo, T):
+    p = I.make_fwd(2, T, 2, 64, 64, dtype="f32", seed=77 + T, rotation=(T % 2 == 1), s0_std=0.3)
+    o, S = U.run_gpu_fwd(p, algo)
+    o_ref, S_ref = U.oracle_fwd(p)
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref, tol_s=1e-4)
+
+
+def test_logdecay_gate_mode(G):
+    """g passed directly (gate_mode LOGDECAY) including g = 0 (no decay) tokens."""
+    import torch
+    p = I.make_fwd(1, 150, 2, 64, 64, dtype="f32", seed=5, s0_std=0.3)
+    g = -np.logaddexp(0.0, p.g.astype(np.float64)).astype(np.float32)
+    g[:, ::7] = 0.0
+    p.g = g
+    p.gate_mode = I.GATE_LOGDECAY
+    o, S = U.run_gpu_fwd(p, "auto")
+    o_ref, S_ref = U.oracle_fwd(p)
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref, tol_s=1e-4)
+
+
+def test_empty_sequence_copies_state(G):
+    import torch
+    p = I.make_fwd(2, 1, 3, 64, 32, dtype="bf16", seed=9, s0_std=0.5)
+    S0 = U.to_torch(p.S0, "cuda")
+    z = lambda *s: torch.zeros(*s, device="cuda")
+    q = torch.zeros((2, 0, 3, 64), dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros((2, 0, 3, 32), dtype=torch.bfloat16, device="cuda")
+    o, S_T = G.chunk_fwd(q, q, v, z(2, 0, 3, 64), z(2, 0, 3), None, S0)
+    torch.cuda.synchronize()
+    assert o.numel() == 0
+    assert torch.equal(S_T, S0)
+    o, S_T = G.chunk_fwd(q, q, v, z(2, 0, 3, 64), z(2, 0, 3), None, None)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(S_T) == 0
+
+
+def test_split_resume_and_in_place_state(G):
+    """fwd(0..T) == fwd(0..t0) then fwd(t0..T) from its final state, with S_T
+    written over S0 in place for the second half."""
+    import torch
+    p = I.make_fwd(2, 300, 2, 128, 128, dtype="f32", seed=21, s0_std=0.3, rotation=True)
+    o_full, S_full = U.run_gpu_fwd(p)
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "g", "beta", "theta", "S0")}
+    t0 = 100
+    sl = lambda x: x[:, :t0].contiguous()
+    sr = lambda x: x[:, t0:].contiguous()
+    oa, Sa = G.chunk_fwd(sl(t["q"]), sl(t["k"]), sl(t["v"]), sl(t["g"]), sl(t["beta"]), sl(t["theta"]), t["S0"])
+    ob, Sb = G.chunk_fwd(sr(t["q"]), sr(t["k"]), sr(t["v"]), sr(t["g"]), sr(t["beta"]), sr(t["theta"]), Sa,
+                         S_T=Sa)
+    torch.cuda.synchronize()
+    assert Sb.data_ptr() == Sa.data_ptr()
+    o_cat = torch.cat([oa, ob], dim=1)
+    assert U.max_rel(U.o_to_f64(o_cat), U.o_to_f64(o_full)) < 1e-4
+    assert U.rel_l2(Sb.cpu().numpy(), S_full.cpu().numpy()) < 1e-4
+
+
+def test_deterministic(G):
+    import torch
+    p = I.make_fwd(2, 200, 2, 128, 128, dtype="bf16", seed=31, s0_std=0.1)
+    o1, S1 = U.run_gpu_fwd(p)
+    o2, S2 = U.run_gpu_fwd(p)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_host_buffers_round_trip(G):
+    """Host (CPU) tensors go through the same library call with copies around it."""
+    import torch
+    p = I.make_fwd(1, 130, 2, 64, 64, dtype="bf16", seed=41, s0_std=0.2)
+    t = {key: U.to_torch(getattr(p, key), "cpu") for key in ("q", "k", "v", "g", "beta", "S0")}
+    o, S = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], None, t["S0"])
+    assert o.device.type == "cpu" and S.device.type == "cpu"
+    o_ref, S_ref = U.oracle_fwd(p)
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref)
+
+
+FULL = ["b4_h16_t4096_d128", "b16_h12_t4096_d128_slow_s0", "b2_h16_t8192_d128_rot"]
+
+
+@pytest.mark.parametrize("algo", ALGOS_ALL)
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_configs_sampled(G, algo, name):
+    """Full-size workloads in the benchmark's launch configuration; the oracle
+    recomputes a sample of whole heads (every token of each sampled head)."""
+    p = I.make_config(name)
+    o, S = U.run_gpu_fwd(p, algo)
+    rng = np.random.default_rng(0)
+    heads = [(int(b), int(h)) for b, h in zip(rng.integers(0, p.B, 4), rng.integers(0, p.H, 4))]
+    heads += [(0, 0), (p.B - 1, p.H - 1)]
+    og = o
+    for (b, h) in heads:
+        ps = p.head_slice(b, h)
+        o_ref, S_ref = U.oracle_fwd(ps)
+        o_bh = og[b:b + 1, :, h:h + 1]
+        S_bh = S[b:b + 1, h:h + 1]
+        U.assert_fwd_parity(ps, o_bh, S_bh, o_ref, S_ref)
+    import torch
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
