@@ -30,7 +30,7 @@ if ROOT not in sys.path:
 
 METRIC = "gated delta-rule fwd Mtokens/s and % roofline at H=16,dk=dv=128; decode GB/s"
 WORKLOAD = "b4_h16_t4096_d128"
-L2_BYTES = 126 * 1024 * 1024
+L2_BYTES = 126e6
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -78,14 +78,23 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
-    """Hash of the CUDA sources: a stored ncu traffic figure is only valid for it."""
+KERNEL_SOURCES = {
+    "gdr_chunk_fwd_simt": ["simt_fwd.cuh", "common.cuh"],
+    "gdr_chunk_fwd_tcgen05": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
+    "gdr_decode_step": ["decode.cuh", "common.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of one kernel's CUDA sources: a stored ncu traffic figure is only valid for it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "recurrent_state_memory_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
-            h.update(f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        path = os.path.join(csrc, name)
+        if os.path.exists(path):
+            with open(path, "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -98,7 +107,7 @@ def stored_traffic(kernel: str, workload: str):
     with open(path) as f:
         tab = json.load(f)
     ent = tab.get(f"{kernel}@{workload}")
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 
