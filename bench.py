@@ -235,7 +235,9 @@ def run_ours(args):
     algo_bytes = p.nbytes_algorithmic
     avg_launch_s = statistics.mean(per_launch_ms) * 1e-3
     achieved_gbs = algo_bytes / avg_launch_s / 1e9
-    kernel_name = "gdr_chunk_fwd_" + ("tcgen05" if args.algo == "tcgen05" else "simt")
+    resolved = gdr.resolved_algo(gdr.fwd_desc(p.B, p.H, p.T, p.dk, p.dv, dv_t["q"].dtype, o.dtype,
+                                              p.gate_mode, p.rotation, p.scale, args.algo))
+    kernel_name = "gdr_chunk_fwd_" + resolved
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
                 "traffic": stored_traffic(kernel_name, args.workload),
@@ -328,11 +330,11 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 3), "unit": "Mtokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms_max / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if args.algo == "tcgen05" else "f32",
+        "dtype": "bf16" if resolved == "tcgen05" else "f32",
         "data": "synthetic (seeded SplitMix64; q,k L2-normalised, bf16)",
         "config": {"workload": f"{args.workload}: B={p.B} H={p.H} T={p.T} dk={p.dk} dv={p.dv} chunk={p.chunk}, "
                                "bf16 q/k/v, fp32 g (raw gate, -softplus fused) and beta, S0=0",
-                   "B": p.B, "H": p.H, "T": p.T, "dk": p.dk, "dv": p.dv, "chunk": p.chunk, "algo": args.algo,
+                   "B": p.B, "H": p.H, "T": p.T, "dk": p.dk, "dv": p.dv, "chunk": p.chunk, "algo": resolved,
                    "per_rank_batch": p.B, "parallelism": f"replicas x{ws} (independent batches)",
                    "l2": f"inputs {algo_bytes / 1e6:.0f} MB > L2 {L2_BYTES / 1e6:.0f} MB; no flush"},
         "tflops_algorithmic": round(tflops, 2),

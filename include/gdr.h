@@ -62,7 +62,8 @@ typedef enum {
     GDR_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. dk not in {32,64,128}) */
     GDR_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
     GDR_ERR_TIMEOUT = 4,     /* a kernel gave up on a bounded wait (device status word) */
-    GDR_ERR_WORKSPACE = 5    /* workspace pointer NULL or smaller than required */
+    GDR_ERR_WORKSPACE = 5,   /* workspace pointer NULL or smaller than required */
+    GDR_ERR_RANGE = 6        /* a decay factor left the factored range (device status word) */
 } gdr_status;
 
 typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
@@ -155,10 +156,26 @@ GDR_API gdr_status gdr_decode_step(const gdr_dec_desc* desc,
 
 /*
  * Synchronises `stream`, then reads and clears the device status word that
- * kernels set when a bounded wait gives up.  Returns GDR_OK, GDR_ERR_TIMEOUT or
- * GDR_ERR_CUDA (a sticky CUDA error on the context).  Uses the current device.
+ * kernels set when a bounded wait gives up (GDR_ERR_TIMEOUT) or when the tensor-core
+ * kernel meets a decay outside its factored range (GDR_ERR_RANGE; the outputs of that
+ * call are not valid).  Returns GDR_OK, GDR_ERR_TIMEOUT, GDR_ERR_RANGE or GDR_ERR_CUDA
+ * (a sticky CUDA error on the context).  Uses the current device.
  */
 GDR_API gdr_status gdr_query_device_status(gdr_stream_t stream);
+
+/* The gdr_algo a descriptor would run with (GDR_ALGO_AUTO resolved), or -1 if the
+ * descriptor is invalid.  No GPU work. */
+GDR_API int gdr_chunk_fwd_algo(const gdr_fwd_desc* desc);
+
+/*
+ * Test hook for the bounded waits of the tensor-core kernel (process-wide, not
+ * thread-safe).  wait_limit_ns bounds every mbarrier wait (0 restores the 2 s
+ * default).  With skip_first_commit != 0, each later launch never signals its first
+ * MMA completion: the wait gives up after wait_limit_ns, the kernel frees its tensor
+ * memory and returns, and gdr_query_device_status reports GDR_ERR_TIMEOUT.  Outputs of
+ * such a launch are not valid.  Nothing faults or traps.
+ */
+GDR_API void gdr_debug_set_tc_fault(int skip_first_commit, unsigned long long wait_limit_ns);
 
 #ifdef __cplusplus
 }

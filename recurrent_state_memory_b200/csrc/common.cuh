@@ -7,6 +7,11 @@
 
 namespace gdr {
 
+// Device status word: kernels OR in a bit when a bounded wait gives up (bit 0) or a
+// decay factor leaves the range of the factored tensor-core form (bit 1).  Read and
+// cleared by gdr_query_device_status.  (All kernels live in one translation unit.)
+__device__ unsigned int g_device_status = 0;
+
 // Element loads/stores with the storage type chosen at compile time.
 template <typename T> __device__ __forceinline__ float ld_f32(const T* p);
 template <> __device__ __forceinline__ float ld_f32<float>(const float* p) { return *p; }

@@ -9,12 +9,14 @@
 #include "common.cuh"
 #include "simt_fwd.cuh"
 #include "decode.cuh"
+#include "tc_fwd.cuh"
 
 namespace gdr {
 
-// Set by kernels that give up on a bounded wait (GDR_ERR_TIMEOUT); read and
-// cleared by gdr_query_device_status.
-__device__ unsigned int g_device_status = 0;
+// Test hook state (gdr_debug_set_tc_fault): bound of every mbarrier wait in the
+// tensor-core kernel, and whether its first MMA completion is never signalled.
+static unsigned long long s_wait_limit_ns = 2000000000ull;
+static int s_fault_skip_commit = 0;
 
 static thread_local char t_detail[256] = "";
 
@@ -65,6 +67,17 @@ static gdr_status dispatch_simt_dk(const gdr_fwd_desc* d, const FwdParams& p, cu
     }
 }
 
+static bool tc_supported(const gdr_fwd_desc* d) {
+    return d->qkv_dtype == GDR_BF16 && d->dk == 128 && d->dv == 128 && d->chunk == 64;
+}
+
+// The algorithm a descriptor runs with: AUTO takes the tensor-core kernel when it
+// supports the shape and dtype.
+static gdr_algo resolve_algo(const gdr_fwd_desc* d) {
+    if (d->algo == GDR_ALGO_AUTO) return tc_supported(d) ? GDR_ALGO_TCGEN05 : GDR_ALGO_SIMT;
+    return d->algo;
+}
+
 static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
     if (!d) return fail(GDR_ERR_INVALID_ARG, "desc is NULL%s");
     if (d->B < 0 || d->H < 0 || d->T < 0) return fail(GDR_ERR_INVALID_ARG, "B, H, T must be >= 0%s");
@@ -78,8 +91,29 @@ static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
     if (d->algo != GDR_ALGO_AUTO && d->algo != GDR_ALGO_SIMT && d->algo != GDR_ALGO_TCGEN05)
         return fail(GDR_ERR_INVALID_ARG, "bad algo%s");
     if ((long long)d->B * d->H > 0x7fffffffLL) return fail(GDR_ERR_INVALID_ARG, "B*H too large%s");
-    if (d->algo == GDR_ALGO_TCGEN05) return fail(GDR_ERR_UNSUPPORTED, "tcgen05 kernel not built in this library%s");
+    if (d->algo == GDR_ALGO_TCGEN05 && !tc_supported(d))
+        return fail(GDR_ERR_UNSUPPORTED, "the tcgen05 kernel needs bf16 q/k/v and dk = dv = 128%s");
     return GDR_OK;
+}
+
+template <bool ROT, typename OT>
+static gdr_status launch_tc(const FwdParams& p, cudaStream_t st) {
+    auto kern = tcf::chunk_fwd_tc_kernel<ROT, OT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tcgen05 chunk kernel)");
+    tcf::TcExtra x;
+    x.wait_limit_ns = s_wait_limit_ns;
+    x.fault_skip_commit = s_fault_skip_commit;
+    kern<<<p.B * p.H, tcf::NT, tcf::SMEM_BYTES, st>>>(p, x);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
+    return GDR_OK;
+}
+
+static gdr_status dispatch_tc(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st) {
+    const bool ob = d->out_dtype == GDR_BF16;
+    if (d->rotation) return ob ? launch_tc<true, __nv_bfloat16>(p, st) : launch_tc<true, float>(p, st);
+    return ob ? launch_tc<false, __nv_bfloat16>(p, st) : launch_tc<false, float>(p, st);
 }
 
 // ----------------------------------------------------------------- decode ----
@@ -120,6 +154,7 @@ const char* gdr_status_string(gdr_status s) {
         case GDR_ERR_CUDA: return "GDR_ERR_CUDA";
         case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
         case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE";
+        case GDR_ERR_RANGE: return "GDR_ERR_RANGE";
     }
     return "GDR_ERR_UNKNOWN";
 }
@@ -159,6 +194,7 @@ gdr_status gdr_chunk_fwd(const gdr_fwd_desc* d, const void* q, const void* k, co
     p.S0 = S0; p.o = o; p.S_T = S_T;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d->T == 0 && !S_T) return GDR_OK;
+    if (resolve_algo(d) == GDR_ALGO_TCGEN05) return dispatch_tc(d, p, st);
     return d->rotation ? dispatch_simt_dk<true>(d, p, st) : dispatch_simt_dk<false>(d, p, st);
 }
 
@@ -213,9 +249,19 @@ gdr_status gdr_query_device_status(gdr_stream_t stream) {
         e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(status)");
         snprintf(t_detail, sizeof(t_detail), "device status word 0x%08x", word);
-        return GDR_ERR_TIMEOUT;
+        return (word & tcf::STATUS_TIMEOUT) ? GDR_ERR_TIMEOUT : GDR_ERR_RANGE;
     }
     return GDR_OK;
+}
+
+int gdr_chunk_fwd_algo(const gdr_fwd_desc* desc) {
+    if (check_fwd_desc(desc) != GDR_OK) return -1;
+    return (int)resolve_algo(desc);
+}
+
+void gdr_debug_set_tc_fault(int skip_first_commit, unsigned long long wait_limit_ns) {
+    s_fault_skip_commit = skip_first_commit ? 1 : 0;
+    s_wait_limit_ns = wait_limit_ns ? wait_limit_ns : 2000000000ull;
 }
 
 }  // extern "C"

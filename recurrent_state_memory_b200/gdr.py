@@ -20,10 +20,12 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdr.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gdr.h")
 
-GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT, GDR_ERR_WORKSPACE = range(6)
+(GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT, GDR_ERR_WORKSPACE,
+ GDR_ERR_RANGE) = range(7)
 GDR_F32, GDR_BF16 = 0, 1
 GATE_LOGDECAY, GATE_NEG_SOFTPLUS = 0, 1
 ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2}
+ALGO_NAMES = {v: k for k, v in ALGOS.items()}
 
 
 class FwdDesc(ctypes.Structure):
@@ -70,6 +72,10 @@ def lib() -> ctypes.CDLL:
         L.gdr_decode_step.argtypes = [ctypes.POINTER(DecDesc), vp, vp, vp, fp, fp, fp, fp, vp, vp]
         L.gdr_query_device_status.restype = ctypes.c_int
         L.gdr_query_device_status.argtypes = [vp]
+        L.gdr_chunk_fwd_algo.restype = ctypes.c_int
+        L.gdr_chunk_fwd_algo.argtypes = [ctypes.POINTER(FwdDesc)]
+        L.gdr_debug_set_tc_fault.restype = None
+        L.gdr_debug_set_tc_fault.argtypes = [ctypes.c_int, ctypes.c_ulonglong]
         if L.gdr_abi_version() != 1:
             raise RuntimeError("libgdr.so ABI version mismatch")
         _lib = L
@@ -121,6 +127,19 @@ def fwd_desc(B, H, T, dk, dv, qkv_dtype, out_dtype, gate_mode=GATE_NEG_SOFTPLUS,
              scale=1.0, algo="auto", chunk=64) -> FwdDesc:
     return FwdDesc(B, H, T, dk, dv, chunk, _dtype_code(qkv_dtype), _dtype_code(out_dtype),
                    int(gate_mode), int(bool(rotation)), float(scale), ALGOS[algo])
+
+
+def resolved_algo(desc: FwdDesc) -> str:
+    """Name of the kernel a descriptor runs with ("simt" or "tcgen05")."""
+    a = int(lib().gdr_chunk_fwd_algo(ctypes.byref(desc)))
+    if a < 0:
+        raise ValueError("invalid descriptor")
+    return ALGO_NAMES[a]
+
+
+def debug_set_tc_fault(skip_first_commit: bool, wait_limit_ns: int = 0):
+    """Test hook: make the tensor-core kernel's first MMA wait run out (see gdr.h)."""
+    lib().gdr_debug_set_tc_fault(int(bool(skip_first_commit)), int(wait_limit_ns))
 
 
 def workspace_bytes(desc: FwdDesc) -> int:

@@ -27,6 +27,7 @@ def test_exports_every_declared_symbol(G):
 def test_status_strings(G):
     assert G.status_string(0) == "GDR_OK"
     assert G.status_string(4) == "GDR_ERR_TIMEOUT"
+    assert G.status_string(6) == "GDR_ERR_RANGE"
     assert G.status_string(99) == "GDR_ERR_UNKNOWN"
 
 

@@ -8,7 +8,12 @@ import parity_util as U
 
 pytestmark = pytest.mark.gpu
 
-ALGOS_ALL = ["simt"]
+ALGOS_ALL = ["simt", "tcgen05"]
+
+
+def _skip_unsupported(algo, dtype, dk, dv):
+    if algo == "tcgen05" and not (dtype == "bf16" and dk == 128 and dv == 128):
+        pytest.skip("tcgen05 kernel: bf16 q/k/v with dk = dv = 128 only")
 
 
 @pytest.fixture(scope="module")
@@ -18,7 +23,7 @@ def G():
     return gdr
 
 
-@pytest.mark.parametrize("algo", ALGOS_ALL)
+@pytest.mark.parametrize("algo", ["simt"])
 def test_tiny_fp32_config(G, algo):
     """The tiny fp32 workload: B=1, H=2, T=256, dk=dv=32, chunk 64, seed 0."""
     p = I.make_config("tiny_f32")
@@ -46,6 +51,7 @@ CASES = [
     c[0], c[1], c[2], c[3], c[4], c[5], "_rot" if c[6] else "", "_s0" if c[7] else ""))
 def test_parity_small(G, algo, case):
     B, H, T, dk, dv, dtype, rot, s0, scale = case
+    _skip_unsupported(algo, dtype, dk, dv)
     p = I.make_fwd(B, T, H, dk, dv, dtype=dtype, seed=1000 + T + dk, rotation=rot,
                    s0_std=0.5 if s0 else None, scale=scale)
     o, S = U.run_gpu_fwd(p, algo)
@@ -53,7 +59,7 @@ def test_parity_small(G, algo, case):
     U.assert_fwd_parity(p, o, S, o_ref, S_ref, tol_s=1e-4 if dtype == "f32" else U.TOL_S)
 
 
-@pytest.mark.parametrize("algo", ALGOS_ALL)
+@pytest.mark.parametrize("algo", ["simt"])
 @pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 128, 129])
 def test_chunk_edges(G, algo, T):
     p = I.make_fwd(2, T, 2, 64, 64, dtype="f32", seed=77 + T, rotation=(T % 2 == 1), s0_std=0.3)
@@ -152,3 +158,48 @@ def test_full_size_configs_sampled(G, algo, name):
         U.assert_fwd_parity(ps, o_bh, S_bh, o_ref, S_ref)
     import torch
     assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
+
+
+TC_CASES = [
+    # (B, H, T, rotation, s0, out_dtype, gate_mode, scale)
+    (1, 2, 1, False, True, "bf16", 1, 1.0),
+    (1, 2, 31, True, False, "bf16", 1, 1.0),
+    (2, 1, 32, False, True, "f32", 1, 1.0),
+    (1, 3, 63, False, False, "bf16", 1, 0.75),
+    (2, 2, 64, True, True, "f32", 1, 1.0),
+    (1, 2, 65, False, True, "bf16", 0, 1.0),
+    (2, 3, 200, True, True, "bf16", 0, 1.0),
+    (3, 2, 511, False, True, "f32", 1, 1.0),
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: "B{}H{}T{}{}{}_{}_g{}".format(
+    c[0], c[1], c[2], "_rot" if c[3] else "", "_s0" if c[4] else "", c[5], c[6]))
+def test_tcgen05_parity(G, case):
+    """The tensor-core kernel against the oracle: ragged tails, rotation, initial state,
+    both output dtypes and both gate modes."""
+    import torch
+    B, H, T, rot, s0, odt, gm, scale = case
+    p = I.make_fwd(B, T, H, 128, 128, dtype="bf16", seed=500 + T + 7 * B, rotation=rot,
+                   s0_std=0.3 if s0 else None, scale=scale)
+    if gm == 0:
+        p.g = (-np.logaddexp(0.0, p.g.astype(np.float64))).astype(np.float32)
+        p.gate_mode = I.GATE_LOGDECAY
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "g", "beta", "theta", "S0")}
+    o, S = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["theta"], t["S0"], gate_mode=p.gate_mode,
+                       scale=p.scale, algo="tcgen05",
+                       out_dtype=torch.float32 if odt == "f32" else torch.bfloat16)
+    torch.cuda.synchronize()
+    assert G.query_device_status() == G.GDR_OK
+    o_ref, S_ref = U.oracle_fwd(p)
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref)
+
+
+def test_auto_picks_tensor_cores_for_bf16_d128(G):
+    import torch
+    d = G.fwd_desc(1, 1, 64, 128, 128, torch.bfloat16, torch.bfloat16)
+    assert G.resolved_algo(d) == "tcgen05"
+    d = G.fwd_desc(1, 1, 64, 64, 64, torch.bfloat16, torch.bfloat16)
+    assert G.resolved_algo(d) == "simt"
+    d = G.fwd_desc(1, 1, 64, 128, 128, torch.float32, torch.float32)
+    assert G.resolved_algo(d) == "simt"
