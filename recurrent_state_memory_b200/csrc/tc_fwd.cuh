@@ -6,7 +6,7 @@
 // dk = dv = 128, chunk C = 64.  One CTA owns one (batch, head); the state S (dv x dk,
 // fp32) stays resident in tensor memory for the whole sequence.
 //
-// Per chunk, with P_r = D_1 ... D_r and a reference token m = 31 (the middle of the
+// Per chunk, with P_r = D_1 ... D_r and the reference token m = 31 (the middle of the
 // chunk), every decay factor is split around P_m so that no factor exceeds the decay
 // of half a chunk:
 //   Ktil_r = (P_m^{-1} P_r) k_r,  Qtil_r = (P_m^{-1} P_r) q_r,  Khat_i = (P_i^{-1} P_m)^T k_i
@@ -17,13 +17,25 @@
 //   E^T = U^T - Stil Wm^T,   O^T = Stil Qtil^T                      (MMA, 128 x 64 x 128)
 //   O^T += E^T Pm^T,   S_acc = Stil + E^T Khat                      (MMA, K = 64)
 //   S <- S_acc (P_m^{-1} P_C)
-// which is the same algebra as the SIMT kernel with the reference moved from the chunk
-// start to its middle.  A tail chunk is padded with identity tokens (g = 0, beta = 0).
+// A tail chunk is padded with identity tokens (g = 0, beta = 0, k = q = v = 0).
 //
-// Shared-memory tiles use the 128-byte swizzle; every tile is either K-major (rows of
-// 128 B along K) or MN-major (rows of 128 B along M/N), and the K-major Khat tile doubles
-// as the MN-major B operand of the state update.  TMEM columns (lane = row):
-//   [0,128) S   [128,192) O^T   [192,256) U^T / E^T   [256,320) [A' ; Pmat]   [320,384) Wm^T
+// Warp roles (384 threads):
+//   warps 0-7  "prep": gate activation and decay factors (register-prefetched inputs),
+//              the operand tiles, MMA1, the triangular solve, U^T / Wm^T.  They run up
+//              to two chunks ahead of the chain, through double-buffered tiles.
+//   warps 8-11 "chain": one thread per TMEM lane (value row of S); issue the state MMAs,
+//              convert E^T to bf16 in TMEM, rescale S, write o and S_T.
+// Hand-offs use mbarriers in pairs indexed by chunk parity (full: prep -> chain,
+// empty: chain -> prep), so no barrier ever runs two phases ahead of its waiter.
+// Every mbarrier wait is bounded; a group that gives up stops at a point where all of
+// its warps agree, and the other group then gives up on its own bounded waits.
+//
+// Tensor memory (512 columns, lane = row):
+//   [0,128) S fp32 | [128,192) Stil bf16 (A operand) | [192,320) O^T x 2 |
+//   [320,448) U^T -> E^T x 2 (fp32, then bf16 in the first 32 columns) | [448,512) A'/Wm^T
+// Shared-memory tiles use the 128-byte swizzle; K-major tiles have rows of 128 B along K,
+// MN-major tiles rows of 128 B along M/N; the K-major Khat tile doubles as the MN-major
+// B operand of the state update.
 #pragma once
 
 #include "common.cuh"
@@ -33,26 +45,28 @@ namespace gdr {
 namespace tcf {
 
 constexpr int C = 64;
-constexpr int D = 128;          // dk = dv
-constexpr int NT = 256;
-constexpr uint32_t COL_S = 0, COL_O = 128, COL_E = 192, COL_A1 = 256, COL_W = 320;
+constexpr int D = 128;           // dk = dv
+constexpr int NT = 384;
+constexpr int NPREP = 256;       // threads of the prep group
+constexpr uint32_t COL_S = 0, COL_SB = 128, COL_O = 192, COL_E = 320, COL_AW = 448;
 constexpr uint32_t TMEM_COLS = 512;
 
 // Shared memory map (bytes from a 1024-aligned base).
-constexpr uint32_t OFF_KQ = 0;                      // [Ktil ; Qtil] K-major: 2 kblocks x 128 rows x 128 B
-constexpr uint32_t OFF_KH = OFF_KQ + 32768;         // Khat K-major: 2 kblocks x 64 rows x 128 B
-constexpr uint32_t OFF_V = OFF_KH + 16384;          // V, MN-major for V^T: 2 groups x 64 tokens x 128 B
-constexpr uint32_t OFF_S = OFF_V + 16384;           // Stil bf16 K-major: 2 kblocks x 128 rows x 128 B
-constexpr uint32_t OFF_E = OFF_S + 32768;           // E^T bf16 K-major: 128 rows x 128 B
-constexpr uint32_t OFF_W = OFF_E + 16384;           // Wm^T bf16 MN-major: 128 dk rows x 128 B
-constexpr uint32_t OFF_TB = OFF_W + 16384;          // Tb K-major: 64 rows x 128 B
-constexpr uint32_t OFF_PM = OFF_TB + 8192;          // Pm K-major: 64 rows x 128 B
-constexpr uint32_t OFF_AF = OFF_PM + 8192;          // fp32 A [64][65]
-constexpr uint32_t OFF_TF = OFF_AF + 64 * 65 * 4;   // fp32 Tm [64][65]
-constexpr uint32_t OFF_XF = OFF_TF + 64 * 65 * 4;   // fp32 scratch [3][16][17]
-constexpr uint32_t OFF_VEC = OFF_XF + 3 * 16 * 17 * 4;  // beta[64], rho_ref[2][128], rho_C[2][128]
-constexpr uint32_t OFF_BAR = (OFF_VEC + (64 + 4 * 128) * 4 + 15) & ~15u;
-constexpr uint32_t SMEM_USED = OFF_BAR + 32;
+constexpr uint32_t OFF_KQ = 0;                       // [Ktil ; Qtil] K-major, x2: 2 kblocks x 128 rows x 128 B
+constexpr uint32_t OFF_KH = OFF_KQ + 2 * 32768;      // Khat K-major, x2: 2 kblocks x 64 rows x 128 B
+constexpr uint32_t OFF_W = OFF_KH + 2 * 16384;       // Wm^T bf16 MN-major, x2: 128 dk rows x 128 B
+constexpr uint32_t OFF_PM = OFF_W + 2 * 16384;       // Pm K-major, x2: 64 rows x 128 B
+constexpr uint32_t OFF_V = OFF_PM + 2 * 8192;        // V, MN-major for V^T: 2 groups x 64 tokens x 128 B
+constexpr uint32_t OFF_TB = OFF_V + 16384;           // Tb K-major: 64 rows x 128 B
+constexpr int AS = 68;                               // row stride (floats) of the fp32 solve matrices
+constexpr uint32_t OFF_AF = OFF_TB + 8192;           // fp32 A [64][68]
+constexpr uint32_t OFF_TF = OFF_AF + 64 * AS * 4;    // fp32 Tm [64][68]
+constexpr uint32_t OFF_XF = OFF_TF + 64 * AS * 4;    // fp32 scratch [3][16][17]
+constexpr uint32_t OFF_QT = OFF_XF + 3 * 16 * 17 * 4;   // quarter products [4][64][4]
+constexpr uint32_t VEC_FLOATS = 64 + 4 * 128;        // beta[64], rho_ref[2][128], rho_C[2][128]
+constexpr uint32_t OFF_VEC = OFF_QT + 4 * 64 * 4 * 4;   // x2
+constexpr uint32_t OFF_BAR = (OFF_VEC + 2 * VEC_FLOATS * 4 + 63) & ~63u;
+constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // slack for 1024-byte alignment
 
 // Device status bits (gdr_query_device_status).
@@ -64,6 +78,33 @@ struct TcExtra {
     int fault_skip_commit;              // test hook: 1 = never signal the first MMA barrier
 };
 
+__device__ __forceinline__ void named_bar(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 pack8(const float* m8) {
+    using tc::pack_bf16x2;
+    return make_uint4(pack_bf16x2(m8[0], m8[1]), pack_bf16x2(m8[2], m8[3]),
+                      pack_bf16x2(m8[4], m8[5]), pack_bf16x2(m8[6], m8[7]));
+}
+
 template <bool ROT, typename OT>
 __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtra x) {
     using namespace tc;
@@ -74,31 +115,44 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
     float* Af = reinterpret_cast<float*>(base + OFF_AF);
     float* Tf = reinterpret_cast<float*>(base + OFF_TF);
     float* Xf = reinterpret_cast<float*>(base + OFF_XF);
-    float* sbeta = reinterpret_cast<float*>(base + OFF_VEC);
-    float* rho_ref = sbeta + 64;          // [2][128]: re, im (real mode uses re only)
-    float* rho_C = rho_ref + 256;         // [2][128]
-    uint64_t* bar = reinterpret_cast<uint64_t*>(base + OFF_BAR);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_BAR + 8);
-    int* abort_flag = reinterpret_cast<int*>(base + OFF_BAR + 12);
-    int* range_flag = reinterpret_cast<int*>(base + OFF_BAR + 16);
+    float* QT = reinterpret_cast<float*>(base + OFF_QT);
+    uint64_t* bar_pmma = reinterpret_cast<uint64_t*>(base + OFF_BAR);
+    uint64_t* bar_cmma = bar_pmma + 1;
+    uint64_t* bar_full = bar_pmma + 2;       // [2] prep -> chain: tiles of a chunk ready
+    uint64_t* bar_empty = bar_pmma + 4;      // [2] chain -> prep: buffers of a chunk free
+    uint64_t* bar_rho = bar_pmma + 6;        // [2] prep -> chain: decay vectors of a chunk ready
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_BAR + 64);
+    int* abort_p = reinterpret_cast<int*>(base + OFF_BAR + 68);
+    int* abort_c = reinterpret_cast<int*>(base + OFF_BAR + 72);
+    int* range_flag = reinterpret_cast<int*>(base + OFF_BAR + 76);
+    auto vecs = [&](int c) -> float* { return reinterpret_cast<float*>(base + OFF_VEC) + (c & 1) * VEC_FLOATS; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
-    const int row = quad * 32 + lane;                        // TMEM lane owned by this thread
+    const int quad = warp & 3;
     const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
     const __nv_bfloat16* __restrict__ q = static_cast<const __nv_bfloat16*>(p.q);
     const __nv_bfloat16* __restrict__ k = static_cast<const __nv_bfloat16*>(p.k);
     const __nv_bfloat16* __restrict__ v = static_cast<const __nv_bfloat16*>(p.v);
     OT* __restrict__ o = static_cast<OT*>(p.o);
+    const int nchunks = (p.T + C - 1) / C;
+    auto chunk_len = [&](int c) -> int { return min(C, p.T - c * C); };
+    auto tok = [&](int c, int r) -> size_t { return ((size_t)b * p.T + (c * C + r)) * p.H + h; };
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(bar_pmma, 1);
+        mbar_init(bar_cmma, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_full + i, NPREP);
+            mbar_init(bar_empty + i, NT - NPREP);
+            mbar_init(bar_rho + i, NPREP);
+        }
         fence_mbar_init();
-        *abort_flag = 0;
+        *abort_p = 0;
+        *abort_c = 0;
         *range_flag = 0;
     }
     tc_fence_before();
@@ -106,406 +160,545 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const uint32_t tq = tbase + ((uint32_t)(quad * 32) << 16);   // this warp's lane quadrant
-    uint32_t phase = 0;
-    bool skip_commit = x.fault_skip_commit != 0;
 
-    // Issue-side helper: one thread commits, every thread waits (bounded).
-    auto commit_and_wait = [&]() -> bool {
-        if (tid == 0) {
-            if (!skip_commit) mma_commit(bar);
-            skip_commit = false;
-        }
-        bool ok = mbar_wait_bounded(bar, phase, x.wait_limit_ns);
-        phase ^= 1u;
-        if (!ok) atomicExch(abort_flag, 1);
-        tc_fence_after();
-        __syncthreads();
-        return *abort_flag == 0;
-    };
-    // Make generic smem writes and TMEM stores visible to the MMA issued next.
-    auto publish = [&]() {
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-    };
+    if (nchunks > 0 && tid < NPREP) {
+        // =========================== prep group ===================================
+        const int pp = tid & 63;           // key pair: dims 2pp, 2pp+1
+        const int qt = tid >> 6;           // token quarter: tokens 16 qt .. 16 qt + 15
+        const int half = warp >> 2;        // TMEM column half for readbacks
+        const int row = quad * 32 + lane;  // TMEM lane for readbacks
+        const uint32_t kb = (uint32_t)(pp >> 5);
+        const uint32_t ch = (uint32_t)((pp & 31) >> 2);
+        const uint32_t in_ch = (uint32_t)(pp & 3) * 4u;
+        uint32_t mma_phase = 0;
+        bool skip_commit = x.fault_skip_commit != 0;
+        bool bad = false;
 
-    const uint32_t ID_128x64_KK = idesc_bf16(128, 64, 0, 0, 0);
-    const uint32_t ID_128x64_MK = idesc_bf16(128, 64, 1, 0, 0);
-    const uint32_t ID_128x64_KMneg = idesc_bf16(128, 64, 0, 1, 1);
-    const uint32_t ID_128x128_KM = idesc_bf16(128, 128, 0, 1, 0);
-
-    const int nchunks = (p.T + C - 1) / C;
-    bool failed = false;
-    for (int c = 0; c < nchunks && !failed; ++c) {
-        const int t0 = c * C;
-        const int Lc = min(C, p.T - t0);
-        auto tok = [&](int r) -> size_t { return ((size_t)b * p.T + (t0 + r)) * p.H + h; };
-
-        // ---------------- prep: gate, decay factors, operand tiles -------------
-        if (tid < 128) {
-            const int pp = tid & 63;                 // key pair: dims 2pp, 2pp+1
-            const int hf = tid >> 6;                 // 0: tokens 31..0 (backward), 1: 32..63
-            const uint32_t kb = (uint32_t)(pp >> 5);
-            const uint32_t ch = (uint32_t)((pp & 31) >> 2);
-            const uint32_t in_ch = (uint32_t)(pp & 3) * 4u;
-            bool bad = false;
-            float P0 = 1.f, P1 = 1.f, Q0 = 1.f, Q1 = 1.f;    // alpha / (1/alpha) products
-            float Rre = 1.f, Rim = 0.f;                     // rotation phase product
-            for (int s = 0; s < 32; ++s) {
-                const int r = hf ? 32 + s : 31 - s;
-                float k0 = 0.f, k1 = 0.f, q0 = 0.f, q1 = 0.f;
-                float al0 = 1.f, al1 = 1.f, iv0 = 1.f, iv1 = 1.f, cth = 1.f, sth = 0.f;
+        // Register prefetch of this thread's raw inputs for one chunk.
+        uint32_t rk[16], rq[16];
+        float ra0[16], ra1[16];            // real: gate dims 2pp, 2pp+1; rotation: gate, angle
+        auto prefetch = [&](int c) {
+            const int Lc = chunk_len(c);
+#pragma unroll
+            for (int s = 0; s < 16; ++s) {
+                const int r = 16 * qt + s;
+                rk[s] = 0u; rq[s] = 0u; ra0[s] = 0.f; ra1[s] = 0.f;
                 if (r < Lc) {
-                    const size_t tk = tok(r);
-                    const __nv_bfloat162 kk = *reinterpret_cast<const __nv_bfloat162*>(k + tk * D + 2 * pp);
-                    const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162*>(q + tk * D + 2 * pp);
-                    k0 = __low2float(kk); k1 = __high2float(kk);
-                    q0 = p.scale * __low2float(qq); q1 = p.scale * __high2float(qq);
+                    const size_t tk = tok(c, r);
+                    rk[s] = __ldg(reinterpret_cast<const unsigned int*>(k + tk * D + 2 * pp));
+                    rq[s] = __ldg(reinterpret_cast<const unsigned int*>(q + tk * D + 2 * pp));
                     if (!ROT) {
-                        const float2 a2 = *reinterpret_cast<const float2*>(p.g + tk * D + 2 * pp);
-                        if (p.gate_mode == 1) {
-                            const float e0 = __expf(a2.x), e1 = __expf(a2.y);
-                            iv0 = 1.f + e0; iv1 = 1.f + e1;
-                            al0 = __frcp_rn(iv0); al1 = __frcp_rn(iv1);
-                        } else {
-                            al0 = __expf(a2.x); al1 = __expf(a2.y);
-                            iv0 = __expf(-a2.x); iv1 = __expf(-a2.y);
-                        }
+                        const float2 a2 = __ldg(reinterpret_cast<const float2*>(p.g + tk * D + 2 * pp));
+                        ra0[s] = a2.x; ra1[s] = a2.y;
                     } else {
-                        const float a1 = p.g[tk * (D / 2) + pp];
+                        ra0[s] = __ldg(p.g + tk * (D / 2) + pp);
+                        ra1[s] = __ldg(p.theta + tk * (D / 2) + pp);
+                    }
+                }
+            }
+        };
+        auto mma_wait = [&]() -> bool {
+            const bool ok = mbar_wait_bounded(bar_pmma, mma_phase, x.wait_limit_ns);
+            mma_phase ^= 1u;
+            if (!ok) atomicExch(abort_p, 1);
+            tc_fence_after();
+            named_bar(1, NPREP);
+            return *abort_p == 0;
+        };
+        auto publish = [&]() {
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(1, NPREP);
+            tc_fence_after();
+        };
+
+        prefetch(0);
+        for (int c = 0; c < nchunks; ++c) {
+            const int Lc = chunk_len(c);
+            const int bufi = c & 1;
+            float* vec = vecs(c);
+            float* sbeta = vec;
+            float* rho_ref = vec + 64;
+            float* rho_C = vec + 64 + 256;
+            uint8_t* KQ = base + OFF_KQ + bufi * 32768;
+            uint8_t* KH = base + OFF_KH + bufi * 16384;
+
+            // V tile of this chunk (MN-major for V^T), asynchronously; done before the U MMA.
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int id = tid * 4 + j;
+                const int i = id >> 4, c16 = id & 15;
+                const bool ok = i < Lc;
+                const void* src = ok ? (const void*)(v + tok(c, i) * D + c16 * 8) : (const void*)v;
+                cp_async16(sb + OFF_V + (uint32_t)(c16 >> 3) * 8192u + sw128_off(i, c16 & 7), src, ok ? 16u : 0u);
+            }
+            cp_async_commit();
+
+            // ---- pass 1: per-token decays; quarter products -------------------------
+            float al0[16], al1[16], iv0[16], iv1[16];
+            // real: products of alpha and 1/alpha per dim; rotation: (PA0, PI0) magnitudes and
+            // (PA1, PI1) the complex product of e^{+i theta}, starting at 1 + 0i.
+            float PA0 = 1.f, PA1 = 1.f, PI0 = 1.f, PI1 = ROT ? 0.f : 1.f;
+            const float L2E = 1.4426950408889634f;
+#pragma unroll
+            for (int s = 0; s < 16; ++s) {
+                const bool ok = 16 * qt + s < Lc;
+                if (!ROT) {
+                    float a0 = 1.f, a1 = 1.f, i0 = 1.f, i1 = 1.f;
+                    if (ok) {
                         if (p.gate_mode == 1) {
-                            const float e0 = __expf(a1);
-                            iv0 = 1.f + e0;
-                            al0 = __frcp_rn(iv0);
+                            i0 = 1.f + ex2_approx(ra0[s] * L2E);
+                            i1 = 1.f + ex2_approx(ra1[s] * L2E);
+                            a0 = rcp_approx(i0);
+                            a1 = rcp_approx(i1);
                         } else {
-                            al0 = __expf(a1);
-                            iv0 = __expf(-a1);
+                            a0 = ex2_approx(ra0[s] * L2E);
+                            a1 = ex2_approx(ra1[s] * L2E);
+                            i0 = ex2_approx(-ra0[s] * L2E);
+                            i1 = ex2_approx(-ra1[s] * L2E);
                         }
-                        al1 = al0; iv1 = iv0;
-                        sincosf(p.theta[tk * (D / 2) + pp], &sth, &cth);
                     }
-                }
-                float F0, F1, G0, G1, Fim = 0.f, Gim = 0.f;
-                if (hf) {   // include token r, then use it
-                    P0 *= al0; P1 *= al1; Q0 *= iv0; Q1 *= iv1;
-                    if (ROT) {   // R *= e^{-i theta}
-                        const float nre = Rre * cth + Rim * sth, nim = Rim * cth - Rre * sth;
-                        Rre = nre; Rim = nim;
-                    }
-                    F0 = P0; F1 = P1; G0 = Q0; G1 = Q1;
-                } else {    // use the product over tokens r+1..31, then include r
-                    F0 = Q0; F1 = Q1; G0 = P0; G1 = P1;
-                }
-                float kt0, kt1, qt0, qt1, kh0, kh1;
-                if (!ROT) {
-                    kt0 = k0 * F0; kt1 = k1 * F1; qt0 = q0 * F0; qt1 = q1 * F1;
-                    kh0 = k0 * G0; kh1 = k1 * G1;
+                    al0[s] = a0; al1[s] = a1; iv0[s] = i0; iv1[s] = i1;
+                    PA0 *= a0; PA1 *= a1; PI0 *= i0; PI1 *= i1;
                 } else {
-                    // F = |F| R, G = |G| R (complex), applied to kappa = k0 + i k1
-                    const float fr = F0 * Rre, fi = F0 * Rim, gr = G0 * Rre, gi = G0 * Rim;
-                    kt0 = fr * k0 - fi * k1; kt1 = fr * k1 + fi * k0;
-                    qt0 = fr * q0 - fi * q1; qt1 = fr * q1 + fi * q0;
-                    kh0 = gr * k0 - gi * k1; kh1 = gr * k1 + gi * k0;
-                    (void)Fim; (void)Gim;
-                }
-                if (!(isfinite(kt0) && isfinite(kt1) && isfinite(kh0) && isfinite(kh1) &&
-                      isfinite(qt0) && isfinite(qt1))) bad = true;
-                *reinterpret_cast<uint32_t*>(base + OFF_KQ + kb * 16384u + sw128_off(r, ch) + in_ch) = pack_bf16x2(kt0, kt1);
-                *reinterpret_cast<uint32_t*>(base + OFF_KQ + kb * 16384u + sw128_off(64 + r, ch) + in_ch) = pack_bf16x2(qt0, qt1);
-                *reinterpret_cast<uint32_t*>(base + OFF_KH + kb * 8192u + sw128_off(r, ch) + in_ch) = pack_bf16x2(kh0, kh1);
-                if (!hf) {
-                    P0 *= al0; P1 *= al1; Q0 *= iv0; Q1 *= iv1;
-                    if (ROT) {   // Rb *= e^{+i theta}
-                        const float nre = Rre * cth - Rim * sth, nim = Rim * cth + Rre * sth;
-                        Rre = nre; Rim = nim;
-                    }
-                }
-            }
-            if (bad) atomicExch(range_flag, 1);
-            // hf = 0 ends with prod_{0..31} alpha = e^{Gamma_m} (and e^{i Theta_m});
-            // hf = 1 ends with prod_{32..63} alpha = e^{Gamma_C - Gamma_m} (and e^{-i(...)}).
-            float* dst = hf ? rho_C : rho_ref;
-            if (!ROT) {
-                dst[2 * pp] = P0; dst[2 * pp + 1] = P1;
-            } else {
-                dst[pp] = P0 * Rre;
-                dst[128 + pp] = hf ? -P0 * Rim : P0 * Rim;   // forward product holds conj
-            }
-        } else {
-            // V tile (MN-major: rows = tokens, 64 dv per group) and beta.
-            const int u = tid - 128;
-            const int j = u & 15;                    // 16-byte chunk of the 256-byte row
-            for (int pass = 0; pass < 8; ++pass) {
-                const int i = pass * 8 + (u >> 4);
-                uint4 val = make_uint4(0, 0, 0, 0);
-                if (i < Lc) val = *reinterpret_cast<const uint4*>(v + tok(i) * D + j * 8);
-                *reinterpret_cast<uint4*>(base + OFF_V + (uint32_t)(j >> 3) * 8192u + sw128_off(i, j & 7)) = val;
-            }
-            if (u < 64) sbeta[u] = u < Lc ? p.beta[tok(u)] : 0.f;
-        }
-        publish();
-
-        // ---------------- MMA1: [Ktil ; Qtil] Khat^T -> TMEM ----------------------
-        if (tid == 0) {
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t kb = ks >> 2, kin = (ks & 3) * 32;
-                mma_bf16_ss(tbase + COL_A1, sdesc_sw128(sb + OFF_KQ + kb * 16384 + kin, 16, 1024),
-                            sdesc_sw128(sb + OFF_KH + kb * 8192 + kin, 16, 1024), ID_128x64_KK, ks > 0);
-            }
-        }
-        // Meanwhile: Stil = S P_m into TMEM (fp32) and shared memory (bf16 operand).
-        {
-            const int j = row;
-            for (int g = 0; g < 4; ++g) {
-                const int col0 = half * 64 + g * 16;
-                float s[16];
-                if (c == 0) {
-                    if (p.S0) {
-                        const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)bh * D + j) * D + col0);
-#pragma unroll
-                        for (int u4 = 0; u4 < 4; ++u4) {
-                            const float4 t4 = src[u4];
-                            s[4 * u4] = t4.x; s[4 * u4 + 1] = t4.y; s[4 * u4 + 2] = t4.z; s[4 * u4 + 3] = t4.w;
+                    float a0 = 1.f, i0 = 1.f, cs = 1.f, sn = 0.f;
+                    if (ok) {
+                        if (p.gate_mode == 1) {
+                            i0 = 1.f + ex2_approx(ra0[s] * L2E);
+                            a0 = rcp_approx(i0);
+                        } else {
+                            a0 = ex2_approx(ra0[s] * L2E);
+                            i0 = ex2_approx(-ra0[s] * L2E);
                         }
+                        __sincosf(ra1[s], &sn, &cs);
+                    }
+                    al0[s] = a0; iv0[s] = i0; al1[s] = cs; iv1[s] = sn;
+                    PA0 *= a0; PI0 *= i0;
+                    const float zr = PA1 * cs - PI1 * sn, zi = PI1 * cs + PA1 * sn;
+                    PA1 = zr; PI1 = zi;
+                }
+            }
+            {
+                float* qtp = QT + (qt * 64 + pp) * 4;
+                qtp[0] = PA0; qtp[1] = PA1; qtp[2] = PI0; qtp[3] = PI1;
+            }
+            if (tid < 64) sbeta[tid] = tid < Lc ? __ldg(p.beta + tok(c, tid)) : 0.f;
+            named_bar(1, NPREP);
+            // Buffers of chunk c - 2 must be released by the chain before they are rewritten.
+            if (c >= 2) {
+                const bool ok = mbar_wait_bounded(bar_empty + bufi, ((c - 2) >> 1) & 1, x.wait_limit_ns);
+                if (!ok) atomicExch(abort_p, 1);
+            }
+            named_bar(1, NPREP);
+            if (*abort_p) break;
+
+            // ---- pass 2: factors around the reference token 31; operand tiles ----------
+            {
+                float P0, P1, Q0, Q1, Rre, Rim;          // real: P/Q per dim; rotation: P0/Q0, R
+                if (!ROT) {
+                    P0 = P1 = Q0 = Q1 = 1.f; Rre = 1.f; Rim = 0.f;
+                    if (qt == 0) { const float* t1 = QT + (64 + pp) * 4; P0 = t1[0]; P1 = t1[1]; Q0 = t1[2]; Q1 = t1[3]; }
+                    if (qt == 3) { const float* t2 = QT + (128 + pp) * 4; P0 = t2[0]; P1 = t2[1]; Q0 = t2[2]; Q1 = t2[3]; }
+                } else {
+                    P0 = Q0 = 1.f; P1 = Q1 = 0.f; Rre = 1.f; Rim = 0.f;
+                    if (qt == 0) { const float* t1 = QT + (64 + pp) * 4; P0 = t1[0]; Q0 = t1[2]; Rre = t1[1]; Rim = t1[3]; }
+                    if (qt == 3) { const float* t2 = QT + (128 + pp) * 4; P0 = t2[0]; Q0 = t2[2]; Rre = t2[1]; Rim = -t2[3]; }
+                }
+                auto emit = [&](int r, float F0, float F1, float G0, float G1, uint32_t kraw, uint32_t qraw) {
+                    const float k0 = __uint_as_float(kraw << 16), k1 = __uint_as_float(kraw & 0xFFFF0000u);
+                    const float q0 = p.scale * __uint_as_float(qraw << 16), q1 = p.scale * __uint_as_float(qraw & 0xFFFF0000u);
+                    float kt0, kt1, qt0, qt1, kh0, kh1;
+                    if (!ROT) {
+                        kt0 = k0 * F0; kt1 = k1 * F1; qt0 = q0 * F0; qt1 = q1 * F1;
+                        kh0 = k0 * G0; kh1 = k1 * G1;
                     } else {
+                        // F = F0 R, G = G0 R (complex), applied to k0 + i k1 and q0 + i q1
+                        const float fr = F0 * Rre, fi = F0 * Rim, gr = G0 * Rre, gi = G0 * Rim;
+                        kt0 = fr * k0 - fi * k1; kt1 = fr * k1 + fi * k0;
+                        qt0 = fr * q0 - fi * q1; qt1 = fr * q1 + fi * q0;
+                        kh0 = gr * k0 - gi * k1; kh1 = gr * k1 + gi * k0;
+                    }
+                    if (!(fabsf(kt0) < 3e38f && fabsf(kt1) < 3e38f && fabsf(kh0) < 3e38f &&
+                          fabsf(kh1) < 3e38f && fabsf(qt0) < 3e38f && fabsf(qt1) < 3e38f)) bad = true;
+                    *reinterpret_cast<uint32_t*>(KQ + kb * 16384u + sw128_off(r, ch) + in_ch) = pack_bf16x2(kt0, kt1);
+                    *reinterpret_cast<uint32_t*>(KQ + kb * 16384u + sw128_off(64 + r, ch) + in_ch) = pack_bf16x2(qt0, qt1);
+                    *reinterpret_cast<uint32_t*>(KH + kb * 8192u + sw128_off(r, ch) + in_ch) = pack_bf16x2(kh0, kh1);
+                };
+                if (qt < 2) {
+                    // backward from token 31: factors over tokens r+1..31, then include r
 #pragma unroll
-                        for (int u = 0; u < 16; ++u) s[u] = 0.f;
+                    for (int s = 15; s >= 0; --s) {
+                        const int r = 16 * qt + s;
+                        emit(r, Q0, ROT ? Q0 : Q1, P0, ROT ? P0 : P1, rk[s], rq[s]);
+                        if (!ROT) {
+                            P0 *= al0[s]; P1 *= al1[s]; Q0 *= iv0[s]; Q1 *= iv1[s];
+                        } else {
+                            P0 *= al0[s]; Q0 *= iv0[s];
+                            const float cs = al1[s], sn = iv1[s];          // R *= e^{+i theta}
+                            const float nr = Rre * cs - Rim * sn, ni = Rim * cs + Rre * sn;
+                            Rre = nr; Rim = ni;
+                        }
+                    }
+                    if (qt == 0) {   // prod over tokens 0..31: e^{Gamma_m} (and e^{i Theta_m})
+                        if (!ROT) { rho_ref[2 * pp] = P0; rho_ref[2 * pp + 1] = P1; }
+                        else { rho_ref[pp] = P0 * Rre; rho_ref[128 + pp] = P0 * Rim; }
                     }
                 } else {
-                    tmem_ld16(tq + COL_S + col0, s);
-                }
-                if (!ROT) {
+                    // forward from token 32: include r, then use
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) s[u] *= rho_ref[col0 + u];
-                } else {
-#pragma unroll
-                    for (int u = 0; u < 16; u += 2) {
-                        const int pr = (col0 + u) >> 1;
-                        const float cr = rho_ref[pr], ci = rho_ref[128 + pr];
-                        const float xr = s[u], xi = s[u + 1];
-                        s[u] = xr * cr - xi * ci;
-                        s[u + 1] = xr * ci + xi * cr;
+                    for (int s = 0; s < 16; ++s) {
+                        const int r = 16 * qt + s;
+                        if (!ROT) {
+                            P0 *= al0[s]; P1 *= al1[s]; Q0 *= iv0[s]; Q1 *= iv1[s];
+                        } else {
+                            P0 *= al0[s]; Q0 *= iv0[s];
+                            const float cs = al1[s], sn = iv1[s];          // R *= e^{-i theta}
+                            const float nr = Rre * cs + Rim * sn, ni = Rim * cs - Rre * sn;
+                            Rre = nr; Rim = ni;
+                        }
+                        emit(r, P0, ROT ? P0 : P1, Q0, ROT ? Q0 : Q1, rk[s], rq[s]);
+                    }
+                    if (qt == 3) {   // prod over tokens 32..63: e^{Gamma_C - Gamma_m} (R holds the conjugate phase)
+                        if (!ROT) { rho_C[2 * pp] = P0; rho_C[2 * pp + 1] = P1; }
+                        else { rho_C[pp] = P0 * Rre; rho_C[128 + pp] = -P0 * Rim; }
                     }
                 }
-                tmem_st16(tq + COL_S + col0, s);
-                const uint32_t kb = (uint32_t)col0 >> 6, c0 = ((uint32_t)col0 & 63u) >> 3;
-                uint4 w0 = make_uint4(pack_bf16x2(s[0], s[1]), pack_bf16x2(s[2], s[3]),
-                                      pack_bf16x2(s[4], s[5]), pack_bf16x2(s[6], s[7]));
-                uint4 w1 = make_uint4(pack_bf16x2(s[8], s[9]), pack_bf16x2(s[10], s[11]),
-                                      pack_bf16x2(s[12], s[13]), pack_bf16x2(s[14], s[15]));
-                *reinterpret_cast<uint4*>(base + OFF_S + kb * 16384u + sw128_off(j, c0)) = w0;
-                *reinterpret_cast<uint4*>(base + OFF_S + kb * 16384u + sw128_off(j, c0 + 1)) = w1;
             }
-            tmem_wait_st();
-        }
-        if (!commit_and_wait()) { failed = true; break; }
+            fence_proxy_async_smem();
+            named_bar(1, NPREP);
+            mbar_arrive(bar_rho + bufi);
+            if (c + 1 < nchunks) prefetch(c + 1);
 
-        // ---------------- solve: Tm = (I + A)^{-1}, Pm masked --------------------
-        {
-            float vals[32];
-            tmem_ld16(tq + COL_A1 + half * 32, *reinterpret_cast<float(*)[16]>(vals));
-            tmem_ld16(tq + COL_A1 + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
-            if (row < 64) {
-                const int r = row;
-                const float br = sbeta[r];
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const int i = half * 32 + u;
-                    Af[r * 65 + i] = (i < r) ? br * vals[u] : 0.f;
+            // ---- MMA1: [Ktil ; Qtil] Khat^T -> TMEM ------------------------------------
+            tc_fence_after();
+            if (tid == 0) {
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t kbk = ks >> 2, kin = (ks & 3) * 32;
+                    mma_bf16_ss(tbase + COL_AW, sdesc_sw128(sb + OFF_KQ + bufi * 32768 + kbk * 16384 + kin, 16, 1024),
+                                sdesc_sw128(sb + OFF_KH + bufi * 16384 + kbk * 8192 + kin, 16, 1024),
+                                idesc_bf16(128, 64, 0, 0, 0), ks > 0);
                 }
-            } else {
-                const int r = row - 64;
+                if (!skip_commit) mma_commit(bar_pmma);
+                skip_commit = false;
+            }
+            if (!mma_wait()) break;
+
+            // ---- solve: Tm = (I + A)^{-1}; Pm masked -> bf16 ---------------------------
+            {
+                float vals[32];
+                tmem_ld16(tq + COL_AW + half * 32, *reinterpret_cast<float(*)[16]>(vals));
+                tmem_ld16(tq + COL_AW + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
+                if (row < 64) {
+                    const int r = row;
+                    const float br = sbeta[r];
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                    for (int u = 0; u < 32; u += 4) {
+                        float4 w;
+                        const int i = half * 32 + u;
+                        w.x = (i < r) ? br * vals[u] : 0.f;
+                        w.y = (i + 1 < r) ? br * vals[u + 1] : 0.f;
+                        w.z = (i + 2 < r) ? br * vals[u + 2] : 0.f;
+                        w.w = (i + 3 < r) ? br * vals[u + 3] : 0.f;
+                        *reinterpret_cast<float4*>(Af + r * AS + i) = w;
+                    }
+                } else {
+                    const int r = row - 64;
+                    uint8_t* PM = base + OFF_PM + bufi * 8192;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float m8[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int i = half * 32 + cc * 8 + u;
+                            m8[u] = (i <= r) ? vals[cc * 8 + u] : 0.f;
+                        }
+                        *reinterpret_cast<uint4*>(PM + sw128_off(r, half * 4 + cc)) = pack8(m8);
+                    }
+                }
+            }
+            named_bar(1, NPREP);
+            // 16x16 diagonal blocks by forward substitution (lane = column of one block).
+            if (tid < 64) {
+                const int bb = (tid >> 4) * 16, jj = tid & 15;
+                float t[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    float s_ = (r == jj) ? 1.f : 0.f;
+#pragma unroll
+                    for (int i = 0; i < r; ++i) s_ = fmaf(-Af[(bb + r) * AS + bb + i], t[i], s_);
+                    t[r] = s_;
+                }
+#pragma unroll
+                for (int r = 0; r < 16; ++r) Tf[(bb + r) * AS + bb + jj] = t[r];
+            }
+            named_bar(1, NPREP);
+            // Off-diagonal blocks, by block distance: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ.
+            // 2x2 register tiles: 64 threads per 16x16 block.
+#pragma unroll 1
+            for (int dist = 1; dist < 4; ++dist) {
+                const int nb = 4 - dist;
+                const int blk = tid >> 6, ti = (tid >> 3) & 7, tj = tid & 7;
+                const bool act = blk < nb;
+                const int J = blk, I = blk + dist;
+                if (act) {
+                    float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+                    const float* a0p = Af + (16 * I + 2 * ti) * AS;
+                    const float* a1p = a0p + AS;
+                    const float* tp = Tf + 16 * J + 2 * tj;
+#pragma unroll 4
+                    for (int kk = 16 * J; kk < 16 * I; ++kk) {
+                        const float a0 = a0p[kk], a1 = a1p[kk];
+                        const float2 t2 = *reinterpret_cast<const float2*>(tp + kk * AS);
+                        x00 = fmaf(a0, t2.x, x00); x01 = fmaf(a0, t2.y, x01);
+                        x10 = fmaf(a1, t2.x, x10); x11 = fmaf(a1, t2.y, x11);
+                    }
+                    float* xp = Xf + blk * 272 + (2 * ti) * 17 + 2 * tj;
+                    xp[0] = x00; xp[1] = x01; xp[17] = x10; xp[18] = x11;
+                }
+                named_bar(1, NPREP);
+                if (act) {
+                    float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+                    const float* d0p = Tf + (16 * I + 2 * ti) * AS + 16 * I;
+                    const float* d1p = d0p + AS;
+                    const float* xp = Xf + blk * 272 + 2 * tj;
+#pragma unroll 4
+                    for (int s_ = 0; s_ < 16; ++s_) {
+                        const float d0 = (s_ <= 2 * ti) ? d0p[s_] : 0.f;
+                        const float d1 = (s_ <= 2 * ti + 1) ? d1p[s_] : 0.f;
+                        const float xa = xp[s_ * 17], xb = xp[s_ * 17 + 1];
+                        y00 = fmaf(d0, xa, y00); y01 = fmaf(d0, xb, y01);
+                        y10 = fmaf(d1, xa, y10); y11 = fmaf(d1, xb, y11);
+                    }
+                    float* tp = Tf + (16 * I + 2 * ti) * AS + 16 * J + 2 * tj;
+                    tp[0] = -y00; tp[1] = -y01; tp[AS] = -y10; tp[AS + 1] = -y11;
+                }
+                named_bar(1, NPREP);
+            }
+            // Tb = Tm diag(beta), zero above the block diagonal, -> bf16 K-major [r][i].
+            {
+                const int r = tid >> 2, qq = tid & 3;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
                     float m8[8];
+                    const int i0 = qq * 16 + hh * 8;
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        const int i = half * 32 + cc * 8 + u;
-                        m8[u] = (i <= r) ? vals[cc * 8 + u] : 0.f;
+                        const int i = i0 + u;
+                        m8[u] = ((i >> 4) <= (r >> 4)) ? Tf[r * AS + i] * sbeta[i] : 0.f;
                     }
-                    *reinterpret_cast<uint4*>(base + OFF_PM + sw128_off(r, half * 4 + cc)) =
-                        make_uint4(pack_bf16x2(m8[0], m8[1]), pack_bf16x2(m8[2], m8[3]),
-                                   pack_bf16x2(m8[4], m8[5]), pack_bf16x2(m8[6], m8[7]));
+                    *reinterpret_cast<uint4*>(base + OFF_TB + sw128_off(r, qq * 2 + hh)) = pack8(m8);
                 }
             }
-            for (int e = tid; e < 64 * 65; e += NT) Tf[e] = 0.f;
-        }
-        __syncthreads();
-        // 16x16 diagonal blocks by forward substitution (one warp per block, lane = column).
-        if (warp < 4 && lane < 16) {
-            const int bb = warp * 16, jj = lane;
-            float t[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float s_ = (r == jj) ? 1.f : 0.f;
-#pragma unroll
-                for (int i = 0; i < r; ++i) s_ = fmaf(-Af[(bb + r) * 65 + bb + i], t[i], s_);
-                t[r] = s_;
-            }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) Tf[(bb + r) * 65 + bb + jj] = t[r];
-        }
-        __syncthreads();
-        // Off-diagonal blocks: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ, by block distance.
-        for (int dist = 1; dist < 4; ++dist) {
-            const int nb = 4 - dist;
-            for (int e = tid; e < nb * 256; e += NT) {
-                const int J = e >> 8, I = J + dist, rr = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
-                for (int kk = 16 * J; kk < 16 * I; ++kk)
-                    acc = fmaf(Af[(16 * I + rr) * 65 + kk], Tf[kk * 65 + 16 * J + cc], acc);
-                Xf[J * 272 + rr * 17 + cc] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nb * 256; e += NT) {
-                const int J = e >> 8, I = J + dist, rr = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
-                for (int s_ = 0; s_ <= rr; ++s_)
-                    acc = fmaf(Tf[(16 * I + rr) * 65 + 16 * I + s_], Xf[J * 272 + s_ * 17 + cc], acc);
-                Tf[(16 * I + rr) * 65 + 16 * J + cc] = -acc;
-            }
-            __syncthreads();
-        }
-        // Tb = Tm diag(beta) -> bf16, K-major [r][i].
-        {
-            const int r = tid >> 2, qq = tid & 3;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float m8[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int i = qq * 16 + hh * 8 + u;
-                    m8[u] = Tf[r * 65 + i] * sbeta[i];
+            cp_async_wait_all();
+            publish();
+
+            // ---- U^T = V^T Tb^T -> E[c&1];  Wm^T = Ktil^T Tb^T -> A'/W columns -------------
+            if (tid == 0) {
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t bdesc = sdesc_sw128(sb + OFF_TB + ks * 32, 16, 1024);
+                    mma_bf16_ss(tbase + COL_E + bufi * 64, sdesc_sw128(sb + OFF_V + ks * 2048, 8192, 1024), bdesc,
+                                idesc_bf16(128, 64, 1, 0, 0), ks > 0);
+                    mma_bf16_ss(tbase + COL_AW, sdesc_sw128(sb + OFF_KQ + bufi * 32768 + ks * 2048, 16384, 1024), bdesc,
+                                idesc_bf16(128, 64, 1, 0, 0), ks > 0);
                 }
-                *reinterpret_cast<uint4*>(base + OFF_TB + sw128_off(r, qq * 2 + hh)) =
-                    make_uint4(pack_bf16x2(m8[0], m8[1]), pack_bf16x2(m8[2], m8[3]),
-                               pack_bf16x2(m8[4], m8[5]), pack_bf16x2(m8[6], m8[7]));
+                mma_commit(bar_pmma);
             }
-        }
-        publish();
+            if (!mma_wait()) break;
 
-        // ---------------- U^T = V^T Tb^T and Wm^T = Ktil^T Tb^T -------------------
-        if (tid == 0) {
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t bdesc = sdesc_sw128(sb + OFF_TB + ks * 32, 16, 1024);
-                mma_bf16_ss(tbase + COL_E, sdesc_sw128(sb + OFF_V + ks * 2048, 8192, 1024), bdesc, ID_128x64_MK, ks > 0);
-                mma_bf16_ss(tbase + COL_W, sdesc_sw128(sb + OFF_KQ + ks * 2048, 16384, 1024), bdesc, ID_128x64_MK, ks > 0);
-            }
-        }
-        if (!commit_and_wait()) { failed = true; break; }
-
-        // Wm^T -> bf16 MN-major tile (row = dk, 64 tokens per row).
-        {
-            float vals[32];
-            tmem_ld16(tq + COL_W + half * 32, *reinterpret_cast<float(*)[16]>(vals));
-            tmem_ld16(tq + COL_W + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
+            // Wm^T -> bf16 MN-major tile (row = dk, 64 tokens per row).
+            {
+                float vals[32];
+                tmem_ld16(tq + COL_AW + half * 32, *reinterpret_cast<float(*)[16]>(vals));
+                tmem_ld16(tq + COL_AW + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
+                uint8_t* W = base + OFF_W + bufi * 16384;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const float* m8 = vals + cc * 8;
-                *reinterpret_cast<uint4*>(base + OFF_W + sw128_off(row, half * 4 + cc)) =
-                    make_uint4(pack_bf16x2(m8[0], m8[1]), pack_bf16x2(m8[2], m8[3]),
-                               pack_bf16x2(m8[4], m8[5]), pack_bf16x2(m8[6], m8[7]));
+                for (int cc = 0; cc < 4; ++cc)
+                    *reinterpret_cast<uint4*>(W + sw128_off(row, half * 4 + cc)) = pack8(vals + cc * 8);
             }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(1, NPREP);
+            mbar_arrive(bar_full + bufi);
         }
-        publish();
-
-        // ---------------- E^T = U^T - Stil Wm^T ;  O^T = Stil Qtil^T ---------------
-        if (tid == 0) {
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t kb = ks >> 2, kin = (ks & 3) * 32;
-                const uint64_t adesc = sdesc_sw128(sb + OFF_S + kb * 16384 + kin, 16, 1024);
-                mma_bf16_ss(tbase + COL_E, adesc, sdesc_sw128(sb + OFF_W + ks * 2048, 8192, 1024), ID_128x64_KMneg, 1);
-                mma_bf16_ss(tbase + COL_O, adesc, sdesc_sw128(sb + OFF_KQ + kb * 16384 + 8192 + kin, 16, 1024),
-                            ID_128x64_KK, ks > 0);
-            }
-        }
-        if (!commit_and_wait()) { failed = true; break; }
-
-        // E^T -> bf16 K-major tile (row = dv, 64 tokens per row).
-        {
-            float vals[32];
-            tmem_ld16(tq + COL_E + half * 32, *reinterpret_cast<float(*)[16]>(vals));
-            tmem_ld16(tq + COL_E + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
+        if (bad) atomicExch(range_flag, 1);
+    } else if (nchunks > 0) {
+        // =========================== chain group ==================================
+        const int row = tid - NPREP;          // TMEM lane = value row of S (quad = warp & 3)
+        uint32_t mma_phase = 0;
+        auto cbar = [&]() { named_bar(2, NT - NPREP); };
+        auto mma_wait = [&]() -> bool {
+            const bool ok = mbar_wait_bounded(bar_cmma, mma_phase, x.wait_limit_ns);
+            mma_phase ^= 1u;
+            if (!ok) atomicExch(abort_c, 1);
+            tc_fence_after();
+            cbar();
+            return *abort_c == 0;
+        };
+        auto bounded = [&](uint64_t* bar, uint32_t parity) -> bool {
+            const bool ok = mbar_wait_bounded(bar, parity, x.wait_limit_ns);
+            if (!ok) atomicExch(abort_c, 1);
+            cbar();
+            return *abort_c == 0;
+        };
+        // Write 16 state columns as fp32 (S) and bf16 (Stil); s holds S * rho.
+        auto store_state = [&](int col0, const float (&s)[16]) {
+            tmem_st16(tq + COL_S + col0, s);
+            uint32_t w[8];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const float* m8 = vals + cc * 8;
-                *reinterpret_cast<uint4*>(base + OFF_E + sw128_off(row, half * 4 + cc)) =
-                    make_uint4(pack_bf16x2(m8[0], m8[1]), pack_bf16x2(m8[2], m8[3]),
-                               pack_bf16x2(m8[4], m8[5]), pack_bf16x2(m8[6], m8[7]));
-            }
-        }
-        publish();
-
-        // ---------------- O^T += E^T Pm^T ;  S_acc += E^T Khat ----------------------
-        if (tid == 0) {
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t adesc = sdesc_sw128(sb + OFF_E + ks * 32, 16, 1024);
-                mma_bf16_ss(tbase + COL_O, adesc, sdesc_sw128(sb + OFF_PM + ks * 32, 16, 1024), ID_128x64_KK, 1);
-                mma_bf16_ss(tbase + COL_S, adesc, sdesc_sw128(sb + OFF_KH + ks * 2048, 8192, 1024), ID_128x128_KM, 1);
-            }
-        }
-        if (!commit_and_wait()) { failed = true; break; }
-
-        // ---------------- epilogue: o, and S <- S_acc (P_m^{-1} P_C) ---------------
-        {
-            const int j = row;
-            float vals[32];
-            tmem_ld16(tq + COL_O + half * 32, *reinterpret_cast<float(*)[16]>(vals));
-            tmem_ld16(tq + COL_O + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
+            for (int u = 0; u < 8; ++u) w[u] = pack_bf16x2(s[2 * u], s[2 * u + 1]);
+            tmem_st8u(tq + COL_SB + (col0 >> 1), w);
+        };
+        auto scale_cols = [&](int col0, float (&s)[16], const float* rho) {
+            if (!ROT) {
 #pragma unroll
-            for (int u = 0; u < 32; ++u) {
-                const int r = half * 32 + u;
-                if (r < Lc) st_from_f32(o + tok(r) * D + j, vals[u]);
+                for (int u = 0; u < 16; ++u) s[u] *= rho[col0 + u];
+            } else {
+#pragma unroll
+                for (int u = 0; u < 16; u += 2) {
+                    const int pr = (col0 + u) >> 1;
+                    const float cr = rho[pr], ci = rho[128 + pr];
+                    const float xr = s[u], xi = s[u + 1];
+                    s[u] = xr * cr - xi * ci;
+                    s[u + 1] = xr * ci + xi * cr;
+                }
             }
-            const bool last = (c == nchunks - 1);
+        };
+        auto o_epilogue = [&](int c) {
+            const int Lc = chunk_len(c);
+            const uint32_t col = COL_O + (c & 1) * 64;
+#pragma unroll 1
             for (int g = 0; g < 4; ++g) {
-                const int col0 = half * 64 + g * 16;
+                float vals[16];
+                tmem_ld16(tq + col + g * 16, vals);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int r = g * 16 + u;
+                    if (r < Lc) st_from_f32(o + tok(c, r) * D + row, vals[u]);
+                }
+            }
+        };
+
+        // Initial state, prescaled by the first chunk's reference decay.
+        bool alive = bounded(bar_rho + 0, 0);
+        if (alive) {
+            const float* rho_ref0 = vecs(0) + 64;
+#pragma unroll 1
+            for (int g = 0; g < 8; ++g) {
+                const int col0 = g * 16;
                 float s[16];
-                tmem_ld16(tq + COL_S + col0, s);
-                if (!ROT) {
+                if (p.S0) {
+                    const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)bh * D + row) * D + col0);
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) s[u] *= rho_C[col0 + u];
-                } else {
-#pragma unroll
-                    for (int u = 0; u < 16; u += 2) {
-                        const int pr = (col0 + u) >> 1;
-                        const float cr = rho_C[pr], ci = rho_C[128 + pr];
-                        const float xr = s[u], xi = s[u + 1];
-                        s[u] = xr * cr - xi * ci;
-                        s[u + 1] = xr * ci + xi * cr;
-                    }
-                }
-                if (last) {
-                    if (p.S_T) {
-                        float4* dst = reinterpret_cast<float4*>(p.S_T + ((size_t)bh * D + j) * D + col0);
-#pragma unroll
-                        for (int u4 = 0; u4 < 4; ++u4)
-                            dst[u4] = make_float4(s[4 * u4], s[4 * u4 + 1], s[4 * u4 + 2], s[4 * u4 + 3]);
+                    for (int u4 = 0; u4 < 4; ++u4) {
+                        const float4 t4 = src[u4];
+                        s[4 * u4] = t4.x; s[4 * u4 + 1] = t4.y; s[4 * u4 + 2] = t4.z; s[4 * u4 + 3] = t4.w;
                     }
                 } else {
-                    tmem_st16(tq + COL_S + col0, s);
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) s[u] = 0.f;
                 }
+                scale_cols(col0, s, rho_ref0);
+                store_state(col0, s);
             }
             tmem_wait_st();
+            tc_fence_before();
         }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+        for (int c = 0; c < nchunks && alive; ++c) {
+            const int bufi = c & 1;
+            const bool last = (c == nchunks - 1);
+            if (!bounded(bar_full + bufi, (c >> 1) & 1)) break;
+            tc_fence_after();
+            // ---- E^T += -Stil Wm^T ;  O^T = Stil Qtil^T --------------------------------
+            if (row == 0) {
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t kbk = ks >> 2, kin = (ks & 3) * 32;
+                    const uint32_t a_t = tbase + COL_SB + ks * 8;
+                    mma_bf16_ts(tbase + COL_E + bufi * 64, a_t,
+                                sdesc_sw128(sb + OFF_W + bufi * 16384 + ks * 2048, 8192, 1024),
+                                idesc_bf16(128, 64, 0, 1, 1), 1);
+                    mma_bf16_ts(tbase + COL_O + bufi * 64, a_t,
+                                sdesc_sw128(sb + OFF_KQ + bufi * 32768 + kbk * 16384 + 8192 + kin, 16, 1024),
+                                idesc_bf16(128, 64, 0, 0, 0), ks > 0);
+                }
+                mma_commit(bar_cmma);
+            }
+            if (c > 0) o_epilogue(c - 1);          // overlaps the MMAs above
+            if (!mma_wait()) break;
+
+            // ---- E^T (fp32) -> bf16 in place, as the A operand ---------------------------
+            {
+                const uint32_t col = COL_E + bufi * 64;
+                uint32_t w[32];
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    float vals[16];
+                    tmem_ld16(tq + col + g * 16, vals);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) w[g * 8 + u] = pack_bf16x2(vals[2 * u], vals[2 * u + 1]);
+                }
+#pragma unroll
+                for (int g = 0; g < 4; ++g) tmem_st8u(tq + col + g * 8, *reinterpret_cast<uint32_t(*)[8]>(w + g * 8));
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            cbar();
+            tc_fence_after();
+            // ---- O^T += E^T Pm^T ;  S_acc += E^T Khat ---------------------------------------
+            if (row == 0) {
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint32_t a_t = tbase + COL_E + bufi * 64 + ks * 8;
+                    mma_bf16_ts(tbase + COL_O + bufi * 64, a_t, sdesc_sw128(sb + OFF_PM + bufi * 8192 + ks * 32, 16, 1024),
+                                idesc_bf16(128, 64, 0, 0, 0), 1);
+                    mma_bf16_ts(tbase + COL_S, a_t, sdesc_sw128(sb + OFF_KH + bufi * 16384 + ks * 2048, 8192, 1024),
+                                idesc_bf16(128, 128, 0, 1, 0), 1);
+                }
+                mma_commit(bar_cmma);
+            }
+            if (!mma_wait()) break;
+
+            // ---- S <- S_acc (P_m^{-1} P_C), then prescale by the next reference ----------
+            if (!last && !bounded(bar_rho + ((c + 1) & 1), ((c + 1) >> 1) & 1)) break;
+            {
+                const float* rho_C = vecs(c) + 64 + 256;
+                const float* rho_nx = vecs(c + 1) + 64;
+#pragma unroll 1
+                for (int g = 0; g < 8; ++g) {
+                    const int col0 = g * 16;
+                    float s[16];
+                    tmem_ld16(tq + COL_S + col0, s);
+                    scale_cols(col0, s, rho_C);
+                    if (last) {
+                        if (p.S_T) {
+                            float4* dst = reinterpret_cast<float4*>(p.S_T + ((size_t)bh * D + row) * D + col0);
+#pragma unroll
+                            for (int u4 = 0; u4 < 4; ++u4)
+                                dst[u4] = make_float4(s[4 * u4], s[4 * u4 + 1], s[4 * u4 + 2], s[4 * u4 + 3]);
+                        }
+                    } else {
+                        scale_cols(col0, s, rho_nx);
+                        store_state(col0, s);
+                    }
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(bar_empty + bufi);
+            if (last) o_epilogue(c);
+        }
     }
 
     if (nchunks == 0 && p.S_T) {
         for (int e = tid; e < D * D; e += NT)
             p.S_T[(size_t)bh * D * D + e] = p.S0 ? p.S0[(size_t)bh * D * D + e] : 0.f;
     }
+    tc_fence_before();
+    __syncthreads();
     if (tid == 0) {
         unsigned bits = 0;
-        if (*abort_flag) bits |= STATUS_TIMEOUT;
+        if (*abort_p || *abort_c) bits |= STATUS_TIMEOUT;
         if (*range_flag) bits |= STATUS_RANGE;
         if (bits) atomicOr(&g_device_status, bits);
     }
-    tc_fence_before();
-    __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tbase, TMEM_COLS);
