@@ -61,10 +61,11 @@ constexpr uint32_t OFF_TB = OFF_V + 16384;           // Tb K-major: 64 rows x 12
 constexpr int AS = 68;                               // row stride (floats) of the fp32 solve matrices
 constexpr uint32_t OFF_AF = OFF_TB + 8192;           // fp32 A [64][68]
 constexpr uint32_t OFF_TF = OFF_AF + 64 * AS * 4;    // fp32 Tm [64][68]
-constexpr uint32_t OFF_XF = OFF_TF + 64 * AS * 4;    // fp32 scratch [3][16][17]
-constexpr uint32_t OFF_QT = OFF_XF + 3 * 16 * 17 * 4;   // quarter products [4][64][4]
+constexpr int XS = 16 * 20;                          // one 16x16 scratch block, rows of 20 floats
+constexpr uint32_t OFF_XF = OFF_TF + 64 * AS * 4;    // fp32 scratch [3][16][20]
+constexpr uint32_t OFF_QT = OFF_XF + 3 * XS * 4;     // segment products [8 segments][32 dim groups][8]
 constexpr uint32_t VEC_FLOATS = 64 + 4 * 128;        // beta[64], rho_ref[2][128], rho_C[2][128]
-constexpr uint32_t OFF_VEC = OFF_QT + 4 * 64 * 4 * 4;   // x2
+constexpr uint32_t OFF_VEC = OFF_QT + 8 * 32 * 8 * 4;   // x2
 constexpr uint32_t OFF_BAR = (OFF_VEC + 2 * VEC_FLOATS * 4 + 63) & ~63u;
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // slack for 1024-byte alignment
@@ -98,6 +99,23 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// In-register transpose of an 8x8 block held by 8 consecutive lanes: lane j (j = lane & 7)
+// enters with row j in v[0..7] and leaves with column j.
+__device__ __forceinline__ void transpose8(float (&v)[8], int j) {
+#pragma unroll
+    for (int st = 4; st >= 1; st >>= 1) {
+        const bool up = (j & st) != 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if ((e & st) == 0) {
+                const float send = up ? v[e] : v[e | st];
+                const float recv = __shfl_xor_sync(0xffffffffu, send, st);
+                if (up) v[e] = recv; else v[e | st] = recv;
+            }
+        }
+    }
+}
 
 __device__ __forceinline__ uint4 pack8(const float* m8) {
     using tc::pack_bf16x2;
@@ -163,36 +181,44 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
 
     if (nchunks > 0 && tid < NPREP) {
         // =========================== prep group ===================================
-        const int pp = tid & 63;           // key pair: dims 2pp, 2pp+1
-        const int qt = tid >> 6;           // token quarter: tokens 16 qt .. 16 qt + 15
-        const int half = warp >> 2;        // TMEM column half for readbacks
-        const int row = quad * 32 + lane;  // TMEM lane for readbacks
-        const uint32_t kb = (uint32_t)(pp >> 5);
-        const uint32_t ch = (uint32_t)((pp & 31) >> 2);
-        const uint32_t in_ch = (uint32_t)(pp & 3) * 4u;
+        // Decay passes: each thread owns 4 key dims (two key pairs) of one 8-token segment;
+        // warp w handles tokens 8w .. 8w+7.  The reference token 31 is the last token of
+        // segment 3, so segments 0-3 run backward from it and segments 4-7 forward.
+        const int dg = tid & 31;                 // dims 4dg .. 4dg+3 (pairs 2dg, 2dg+1)
+        const int sg = tid >> 5;                 // token segment
+        const int half = warp >> 2;              // TMEM column half for readbacks
+        const int row = quad * 32 + lane;        // TMEM lane for readbacks
+        const uint32_t kb = (uint32_t)(dg >> 4);             // K block of the 4 dims
+        const uint32_t ch = (uint32_t)((dg & 15) >> 1);      // 16-byte chunk in the 128-byte row
+        const uint32_t in_ch = (uint32_t)(dg & 1) * 8u;      // byte offset in the chunk
+        const size_t tstride = (size_t)p.H * D;              // elements between consecutive tokens
         uint32_t mma_phase = 0;
         bool skip_commit = x.fault_skip_commit != 0;
         bool bad = false;
 
         // Register prefetch of this thread's raw inputs for one chunk.
-        uint32_t rk[16], rq[16];
-        float ra0[16], ra1[16];            // real: gate dims 2pp, 2pp+1; rotation: gate, angle
+        uint2 rk[8], rq[8];
+        float4 ra[8];       // real: 4 gates; rotation: gates of the 2 pairs, then their 2 angles
         auto prefetch = [&](int c) {
             const int Lc = chunk_len(c);
+            const size_t t0 = tok(c, 8 * sg);
+            const __nv_bfloat16* kp = k + t0 * D + 4 * dg;
+            const __nv_bfloat16* qp = q + t0 * D + 4 * dg;
 #pragma unroll
-            for (int s = 0; s < 16; ++s) {
-                const int r = 16 * qt + s;
-                rk[s] = 0u; rq[s] = 0u; ra0[s] = 0.f; ra1[s] = 0.f;
-                if (r < Lc) {
-                    const size_t tk = tok(c, r);
-                    rk[s] = __ldg(reinterpret_cast<const unsigned int*>(k + tk * D + 2 * pp));
-                    rq[s] = __ldg(reinterpret_cast<const unsigned int*>(q + tk * D + 2 * pp));
+            for (int s_ = 0; s_ < 8; ++s_) {
+                rk[s_] = make_uint2(0u, 0u);
+                rq[s_] = make_uint2(0u, 0u);
+                ra[s_] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (8 * sg + s_ < Lc) {
+                    rk[s_] = __ldg(reinterpret_cast<const uint2*>(kp + s_ * tstride));
+                    rq[s_] = __ldg(reinterpret_cast<const uint2*>(qp + s_ * tstride));
                     if (!ROT) {
-                        const float2 a2 = __ldg(reinterpret_cast<const float2*>(p.g + tk * D + 2 * pp));
-                        ra0[s] = a2.x; ra1[s] = a2.y;
+                        ra[s_] = __ldg(reinterpret_cast<const float4*>(p.g + (t0 + (size_t)s_ * p.H) * D + 4 * dg));
                     } else {
-                        ra0[s] = __ldg(p.g + tk * (D / 2) + pp);
-                        ra1[s] = __ldg(p.theta + tk * (D / 2) + pp);
+                        const size_t e = (t0 + (size_t)s_ * p.H) * (D / 2) + 2 * dg;
+                        const float2 g2 = __ldg(reinterpret_cast<const float2*>(p.g + e));
+                        const float2 t2 = __ldg(reinterpret_cast<const float2*>(p.theta + e));
+                        ra[s_] = make_float4(g2.x, g2.y, t2.x, t2.y);
                     }
                 }
             }
@@ -211,6 +237,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             named_bar(1, NPREP);
             tc_fence_after();
         };
+        const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
 
         prefetch(0);
         for (int c = 0; c < nchunks; ++c) {
@@ -234,53 +261,47 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             }
             cp_async_commit();
 
-            // ---- pass 1: per-token decays; quarter products -------------------------
-            float al0[16], al1[16], iv0[16], iv1[16];
-            // real: products of alpha and 1/alpha per dim; rotation: (PA0, PI0) magnitudes and
-            // (PA1, PI1) the complex product of e^{+i theta}, starting at 1 + 0i.
-            float PA0 = 1.f, PA1 = 1.f, PI0 = 1.f, PI1 = ROT ? 0.f : 1.f;
+            // ---- pass 1: per-token decays and segment products ---------------------------
+            // real:     al/iv[s][d] = alpha and 1/alpha of dim 4dg+d;
+            // rotation: al/iv[s][j] = alpha and 1/alpha of pair 2dg+j, al[s][2+j] = cos, iv[s][2+j] = sin.
+            float al[8][4], iv[8][4];
+            float PA[4] = {1.f, 1.f, 1.f, 1.f}, PI[4] = {1.f, 1.f, 1.f, 1.f};
+            if (ROT) { PI[2] = 0.f; PI[3] = 0.f; }           // (PA[2+j], PI[2+j]) = prod e^{+i theta}, from 1 + 0i
             const float L2E = 1.4426950408889634f;
 #pragma unroll
-            for (int s = 0; s < 16; ++s) {
-                const bool ok = 16 * qt + s < Lc;
-                if (!ROT) {
-                    float a0 = 1.f, a1 = 1.f, i0 = 1.f, i1 = 1.f;
+            for (int s_ = 0; s_ < 8; ++s_) {
+                const bool ok = 8 * sg + s_ < Lc;
+                const float ga[4] = {ra[s_].x, ra[s_].y, ra[s_].z, ra[s_].w};
+#pragma unroll
+                for (int d = 0; d < (ROT ? 2 : 4); ++d) {
+                    float a_ = 1.f, i_ = 1.f;
                     if (ok) {
                         if (p.gate_mode == 1) {
-                            i0 = 1.f + ex2_approx(ra0[s] * L2E);
-                            i1 = 1.f + ex2_approx(ra1[s] * L2E);
-                            a0 = rcp_approx(i0);
-                            a1 = rcp_approx(i1);
+                            i_ = 1.f + ex2_approx(ga[d] * L2E);
+                            a_ = rcp_approx(i_);
                         } else {
-                            a0 = ex2_approx(ra0[s] * L2E);
-                            a1 = ex2_approx(ra1[s] * L2E);
-                            i0 = ex2_approx(-ra0[s] * L2E);
-                            i1 = ex2_approx(-ra1[s] * L2E);
+                            a_ = ex2_approx(ga[d] * L2E);
+                            i_ = ex2_approx(-ga[d] * L2E);
                         }
                     }
-                    al0[s] = a0; al1[s] = a1; iv0[s] = i0; iv1[s] = i1;
-                    PA0 *= a0; PA1 *= a1; PI0 *= i0; PI1 *= i1;
-                } else {
-                    float a0 = 1.f, i0 = 1.f, cs = 1.f, sn = 0.f;
-                    if (ok) {
-                        if (p.gate_mode == 1) {
-                            i0 = 1.f + ex2_approx(ra0[s] * L2E);
-                            a0 = rcp_approx(i0);
-                        } else {
-                            a0 = ex2_approx(ra0[s] * L2E);
-                            i0 = ex2_approx(-ra0[s] * L2E);
-                        }
-                        __sincosf(ra1[s], &sn, &cs);
+                    al[s_][d] = a_; iv[s_][d] = i_;
+                    PA[d] *= a_; PI[d] *= i_;
+                }
+                if (ROT) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        float cs = 1.f, sn = 0.f;
+                        if (ok) __sincosf(ga[2 + j], &sn, &cs);
+                        al[s_][2 + j] = cs; iv[s_][2 + j] = sn;
+                        const float zr = PA[2 + j] * cs - PI[2 + j] * sn, zi = PI[2 + j] * cs + PA[2 + j] * sn;
+                        PA[2 + j] = zr; PI[2 + j] = zi;
                     }
-                    al0[s] = a0; iv0[s] = i0; al1[s] = cs; iv1[s] = sn;
-                    PA0 *= a0; PI0 *= i0;
-                    const float zr = PA1 * cs - PI1 * sn, zi = PI1 * cs + PA1 * sn;
-                    PA1 = zr; PI1 = zi;
                 }
             }
             {
-                float* qtp = QT + (qt * 64 + pp) * 4;
-                qtp[0] = PA0; qtp[1] = PA1; qtp[2] = PI0; qtp[3] = PI1;
+                float4* qtp = reinterpret_cast<float4*>(QT + (sg * 32 + dg) * 8);
+                qtp[0] = make_float4(PA[0], PA[1], PA[2], PA[3]);
+                qtp[1] = make_float4(PI[0], PI[1], PI[2], PI[3]);
             }
             if (tid < 64) sbeta[tid] = tid < Lc ? __ldg(p.beta + tok(c, tid)) : 0.f;
             named_bar(1, NPREP);
@@ -292,77 +313,107 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             named_bar(1, NPREP);
             if (*abort_p) break;
 
-            // ---- pass 2: factors around the reference token 31; operand tiles ----------
+            // ---- pass 2: factors around the reference token 31; operand tiles -----------
             {
-                float P0, P1, Q0, Q1, Rre, Rim;          // real: P/Q per dim; rotation: P0/Q0, R
-                if (!ROT) {
-                    P0 = P1 = Q0 = Q1 = 1.f; Rre = 1.f; Rim = 0.f;
-                    if (qt == 0) { const float* t1 = QT + (64 + pp) * 4; P0 = t1[0]; P1 = t1[1]; Q0 = t1[2]; Q1 = t1[3]; }
-                    if (qt == 3) { const float* t2 = QT + (128 + pp) * 4; P0 = t2[0]; P1 = t2[1]; Q0 = t2[2]; Q1 = t2[3]; }
-                } else {
-                    P0 = Q0 = 1.f; P1 = Q1 = 0.f; Rre = 1.f; Rim = 0.f;
-                    if (qt == 0) { const float* t1 = QT + (64 + pp) * 4; P0 = t1[0]; Q0 = t1[2]; Rre = t1[1]; Rim = t1[3]; }
-                    if (qt == 3) { const float* t2 = QT + (128 + pp) * 4; P0 = t2[0]; Q0 = t2[2]; Rre = t2[1]; Rim = -t2[3]; }
-                }
-                auto emit = [&](int r, float F0, float F1, float G0, float G1, uint32_t kraw, uint32_t qraw) {
-                    const float k0 = __uint_as_float(kraw << 16), k1 = __uint_as_float(kraw & 0xFFFF0000u);
-                    const float q0 = p.scale * __uint_as_float(qraw << 16), q1 = p.scale * __uint_as_float(qraw & 0xFFFF0000u);
-                    float kt0, kt1, qt0, qt1, kh0, kh1;
+                // P: products of alpha, Q: products of 1/alpha (per dim, or per pair magnitude);
+                // R: phase of a pair, as a complex number.
+                float P[4] = {1.f, 1.f, 1.f, 1.f}, Q[4] = {1.f, 1.f, 1.f, 1.f};
+                float Rre[2] = {1.f, 1.f}, Rim[2] = {0.f, 0.f};
+                const int lo = sg < 4 ? sg + 1 : 4, hi = sg < 4 ? 4 : sg;   // segments between me and token 31
+                for (int s2 = lo; s2 < hi; ++s2) {
+                    const float4* t = reinterpret_cast<const float4*>(QT + (s2 * 32 + dg) * 8);
+                    const float4 a4 = t[0], i4 = t[1];
                     if (!ROT) {
-                        kt0 = k0 * F0; kt1 = k1 * F1; qt0 = q0 * F0; qt1 = q1 * F1;
-                        kh0 = k0 * G0; kh1 = k1 * G1;
+                        P[0] *= a4.x; P[1] *= a4.y; P[2] *= a4.z; P[3] *= a4.w;
+                        Q[0] *= i4.x; Q[1] *= i4.y; Q[2] *= i4.z; Q[3] *= i4.w;
                     } else {
-                        // F = F0 R, G = G0 R (complex), applied to k0 + i k1 and q0 + i q1
-                        const float fr = F0 * Rre, fi = F0 * Rim, gr = G0 * Rre, gi = G0 * Rim;
-                        kt0 = fr * k0 - fi * k1; kt1 = fr * k1 + fi * k0;
-                        qt0 = fr * q0 - fi * q1; qt1 = fr * q1 + fi * q0;
-                        kh0 = gr * k0 - gi * k1; kh1 = gr * k1 + gi * k0;
-                    }
-                    if (!(fabsf(kt0) < 3e38f && fabsf(kt1) < 3e38f && fabsf(kh0) < 3e38f &&
-                          fabsf(kh1) < 3e38f && fabsf(qt0) < 3e38f && fabsf(qt1) < 3e38f)) bad = true;
-                    *reinterpret_cast<uint32_t*>(KQ + kb * 16384u + sw128_off(r, ch) + in_ch) = pack_bf16x2(kt0, kt1);
-                    *reinterpret_cast<uint32_t*>(KQ + kb * 16384u + sw128_off(64 + r, ch) + in_ch) = pack_bf16x2(qt0, qt1);
-                    *reinterpret_cast<uint32_t*>(KH + kb * 8192u + sw128_off(r, ch) + in_ch) = pack_bf16x2(kh0, kh1);
-                };
-                if (qt < 2) {
-                    // backward from token 31: factors over tokens r+1..31, then include r
+                        P[0] *= a4.x; P[1] *= a4.y; Q[0] *= i4.x; Q[1] *= i4.y;
+                        const float zr[2] = {a4.z, a4.w};
+                        const float zi[2] = {sg < 4 ? i4.z : -i4.z, sg < 4 ? i4.w : -i4.w};   // forward: conjugate
 #pragma unroll
-                    for (int s = 15; s >= 0; --s) {
-                        const int r = 16 * qt + s;
-                        emit(r, Q0, ROT ? Q0 : Q1, P0, ROT ? P0 : P1, rk[s], rq[s]);
-                        if (!ROT) {
-                            P0 *= al0[s]; P1 *= al1[s]; Q0 *= iv0[s]; Q1 *= iv1[s];
-                        } else {
-                            P0 *= al0[s]; Q0 *= iv0[s];
-                            const float cs = al1[s], sn = iv1[s];          // R *= e^{+i theta}
-                            const float nr = Rre * cs - Rim * sn, ni = Rim * cs + Rre * sn;
-                            Rre = nr; Rim = ni;
+                        for (int j = 0; j < 2; ++j) {
+                            const float nr = Rre[j] * zr[j] - Rim[j] * zi[j], ni = Rim[j] * zr[j] + Rre[j] * zi[j];
+                            Rre[j] = nr; Rim[j] = ni;
                         }
                     }
-                    if (qt == 0) {   // prod over tokens 0..31: e^{Gamma_m} (and e^{i Theta_m})
-                        if (!ROT) { rho_ref[2 * pp] = P0; rho_ref[2 * pp + 1] = P1; }
-                        else { rho_ref[pp] = P0 * Rre; rho_ref[128 + pp] = P0 * Rim; }
+                }
+                const float sc = p.scale;
+                auto emit = [&](int r, const float (&F)[4], const float (&G)[4], uint2 kraw, uint2 qraw) {
+                    const float kk[4] = {__uint_as_float(kraw.x << 16), __uint_as_float(kraw.x & 0xFFFF0000u),
+                                         __uint_as_float(kraw.y << 16), __uint_as_float(kraw.y & 0xFFFF0000u)};
+                    const float qv[4] = {__uint_as_float(qraw.x << 16), __uint_as_float(qraw.x & 0xFFFF0000u),
+                                         __uint_as_float(qraw.y << 16), __uint_as_float(qraw.y & 0xFFFF0000u)};
+                    float kt[4], qt[4], kh[4];
+                    if (!ROT) {
+#pragma unroll
+                        for (int d = 0; d < 4; ++d) {
+                            kt[d] = kk[d] * F[d]; qt[d] = qv[d] * (sc * F[d]); kh[d] = kk[d] * G[d];
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            // F = |F| R, G = |G| R, applied to (x + i y) = (v[2j] + i v[2j+1])
+                            const float fr = F[j] * Rre[j], fi = F[j] * Rim[j];
+                            const float gr = G[j] * Rre[j], gi = G[j] * Rim[j];
+                            const float k0 = kk[2 * j], k1 = kk[2 * j + 1], q0 = sc * qv[2 * j], q1 = sc * qv[2 * j + 1];
+                            kt[2 * j] = fr * k0 - fi * k1; kt[2 * j + 1] = fr * k1 + fi * k0;
+                            qt[2 * j] = fr * q0 - fi * q1; qt[2 * j + 1] = fr * q1 + fi * q0;
+                            kh[2 * j] = gr * k0 - gi * k1; kh[2 * j + 1] = gr * k1 + gi * k0;
+                        }
+                    }
+                    const uint32_t off = sw128_off(r, ch) + in_ch;
+                    *reinterpret_cast<uint2*>(KQ + kb * 16384u + off) = make_uint2(pack_bf16x2(kt[0], kt[1]), pack_bf16x2(kt[2], kt[3]));
+                    *reinterpret_cast<uint2*>(KQ + kb * 16384u + 8192u + off) = make_uint2(pack_bf16x2(qt[0], qt[1]), pack_bf16x2(qt[2], qt[3]));
+                    *reinterpret_cast<uint2*>(KH + kb * 8192u + off) = make_uint2(pack_bf16x2(kh[0], kh[1]), pack_bf16x2(kh[2], kh[3]));
+                };
+                auto include = [&](int s_, bool forward) {
+#pragma unroll
+                    for (int d = 0; d < (ROT ? 2 : 4); ++d) { P[d] *= al[s_][d]; Q[d] *= iv[s_][d]; }
+                    if (ROT) {
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const float cs = al[s_][2 + j], sn = forward ? -iv[s_][2 + j] : iv[s_][2 + j];
+                            const float nr = Rre[j] * cs - Rim[j] * sn, ni = Rim[j] * cs + Rre[j] * sn;
+                            Rre[j] = nr; Rim[j] = ni;
+                        }
+                    }
+                };
+                if (sg < 4) {
+                    // backward from token 31: factors over tokens r+1..31, then include r
+#pragma unroll
+                    for (int s_ = 7; s_ >= 0; --s_) {
+                        emit(8 * sg + s_, Q, P, rk[s_], rq[s_]);
+                        include(s_, false);
+                    }
+                    if (sg == 0) {   // prod over tokens 0..31: e^{Gamma_m} (and e^{i Theta_m})
+                        if (!ROT) {
+                            *reinterpret_cast<float4*>(rho_ref + 4 * dg) = make_float4(P[0], P[1], P[2], P[3]);
+                        } else {
+                            rho_ref[2 * dg] = P[0] * Rre[0]; rho_ref[2 * dg + 1] = P[1] * Rre[1];
+                            rho_ref[128 + 2 * dg] = P[0] * Rim[0]; rho_ref[128 + 2 * dg + 1] = P[1] * Rim[1];
+                        }
                     }
                 } else {
                     // forward from token 32: include r, then use
 #pragma unroll
-                    for (int s = 0; s < 16; ++s) {
-                        const int r = 16 * qt + s;
-                        if (!ROT) {
-                            P0 *= al0[s]; P1 *= al1[s]; Q0 *= iv0[s]; Q1 *= iv1[s];
-                        } else {
-                            P0 *= al0[s]; Q0 *= iv0[s];
-                            const float cs = al1[s], sn = iv1[s];          // R *= e^{-i theta}
-                            const float nr = Rre * cs + Rim * sn, ni = Rim * cs - Rre * sn;
-                            Rre = nr; Rim = ni;
-                        }
-                        emit(r, P0, ROT ? P0 : P1, Q0, ROT ? Q0 : Q1, rk[s], rq[s]);
+                    for (int s_ = 0; s_ < 8; ++s_) {
+                        include(s_, true);
+                        emit(8 * sg + s_, P, Q, rk[s_], rq[s_]);
                     }
-                    if (qt == 3) {   // prod over tokens 32..63: e^{Gamma_C - Gamma_m} (R holds the conjugate phase)
-                        if (!ROT) { rho_C[2 * pp] = P0; rho_C[2 * pp + 1] = P1; }
-                        else { rho_C[pp] = P0 * Rre; rho_C[128 + pp] = -P0 * Rim; }
+                    if (sg == 7) {   // prod over tokens 32..63: e^{Gamma_C - Gamma_m}; R holds the conjugate phase
+                        if (!ROT) {
+                            *reinterpret_cast<float4*>(rho_C + 4 * dg) = make_float4(P[0], P[1], P[2], P[3]);
+                        } else {
+                            rho_C[2 * dg] = P[0] * Rre[0]; rho_C[2 * dg + 1] = P[1] * Rre[1];
+                            rho_C[128 + 2 * dg] = -P[0] * Rim[0]; rho_C[128 + 2 * dg + 1] = -P[1] * Rim[1];
+                        }
                     }
                 }
+                // The products grow monotonically away from token 31: checking the final ones
+                // covers every factor this thread used.
+#pragma unroll
+                for (int d = 0; d < 4; ++d)
+                    if (!(fabsf(Q[d]) < 3e38f && fabsf(P[d]) < 3e38f)) bad = true;
             }
             fence_proxy_async_smem();
             named_bar(1, NPREP);
@@ -375,8 +426,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kbk = ks >> 2, kin = (ks & 3) * 32;
                     mma_bf16_ss(tbase + COL_AW, sdesc_sw128(sb + OFF_KQ + bufi * 32768 + kbk * 16384 + kin, 16, 1024),
-                                sdesc_sw128(sb + OFF_KH + bufi * 16384 + kbk * 8192 + kin, 16, 1024),
-                                idesc_bf16(128, 64, 0, 0, 0), ks > 0);
+                                sdesc_sw128(sb + OFF_KH + bufi * 16384 + kbk * 8192 + kin, 16, 1024), ID_KK, ks > 0);
                 }
                 if (!skip_commit) mma_commit(bar_pmma);
                 skip_commit = false;
@@ -433,44 +483,36 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             }
             named_bar(1, NPREP);
             // Off-diagonal blocks, by block distance: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ.
-            // 2x2 register tiles: 64 threads per 16x16 block.
+            // 64 threads per 16x16 block, each owning a 1x4 strip (row rr, columns c4..c4+3).
 #pragma unroll 1
             for (int dist = 1; dist < 4; ++dist) {
                 const int nb = 4 - dist;
-                const int blk = tid >> 6, ti = (tid >> 3) & 7, tj = tid & 7;
+                const int blk = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
                 const bool act = blk < nb;
                 const int J = blk, I = blk + dist;
                 if (act) {
-                    float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
-                    const float* a0p = Af + (16 * I + 2 * ti) * AS;
-                    const float* a1p = a0p + AS;
-                    const float* tp = Tf + 16 * J + 2 * tj;
-#pragma unroll 4
+                    float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+                    const float* ap = Af + (16 * I + rr) * AS;
+                    const float* tp = Tf + 16 * J + c4;
+#pragma unroll 8
                     for (int kk = 16 * J; kk < 16 * I; ++kk) {
-                        const float a0 = a0p[kk], a1 = a1p[kk];
-                        const float2 t2 = *reinterpret_cast<const float2*>(tp + kk * AS);
-                        x00 = fmaf(a0, t2.x, x00); x01 = fmaf(a0, t2.y, x01);
-                        x10 = fmaf(a1, t2.x, x10); x11 = fmaf(a1, t2.y, x11);
+                        const float a = ap[kk];
+                        const float4 t4 = *reinterpret_cast<const float4*>(tp + kk * AS);
+                        x0 = fmaf(a, t4.x, x0); x1 = fmaf(a, t4.y, x1); x2 = fmaf(a, t4.z, x2); x3 = fmaf(a, t4.w, x3);
                     }
-                    float* xp = Xf + blk * 272 + (2 * ti) * 17 + 2 * tj;
-                    xp[0] = x00; xp[1] = x01; xp[17] = x10; xp[18] = x11;
+                    *reinterpret_cast<float4*>(Xf + blk * XS + rr * 20 + c4) = make_float4(x0, x1, x2, x3);
                 }
                 named_bar(1, NPREP);
                 if (act) {
-                    float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-                    const float* d0p = Tf + (16 * I + 2 * ti) * AS + 16 * I;
-                    const float* d1p = d0p + AS;
-                    const float* xp = Xf + blk * 272 + 2 * tj;
+                    float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+                    const float* dp = Tf + (16 * I + rr) * AS + 16 * I;
 #pragma unroll 4
-                    for (int s_ = 0; s_ < 16; ++s_) {
-                        const float d0 = (s_ <= 2 * ti) ? d0p[s_] : 0.f;
-                        const float d1 = (s_ <= 2 * ti + 1) ? d1p[s_] : 0.f;
-                        const float xa = xp[s_ * 17], xb = xp[s_ * 17 + 1];
-                        y00 = fmaf(d0, xa, y00); y01 = fmaf(d0, xb, y01);
-                        y10 = fmaf(d1, xa, y10); y11 = fmaf(d1, xb, y11);
+                    for (int s_ = 0; s_ <= rr; ++s_) {
+                        const float d = dp[s_];
+                        const float4 x4 = *reinterpret_cast<const float4*>(Xf + blk * XS + s_ * 20 + c4);
+                        y0 = fmaf(d, x4.x, y0); y1 = fmaf(d, x4.y, y1); y2 = fmaf(d, x4.z, y2); y3 = fmaf(d, x4.w, y3);
                     }
-                    float* tp = Tf + (16 * I + 2 * ti) * AS + 16 * J + 2 * tj;
-                    tp[0] = -y00; tp[1] = -y01; tp[AS] = -y10; tp[AS + 1] = -y11;
+                    *reinterpret_cast<float4*>(Tf + (16 * I + rr) * AS + 16 * J + c4) = make_float4(-y0, -y1, -y2, -y3);
                 }
                 named_bar(1, NPREP);
             }
@@ -497,9 +539,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint64_t bdesc = sdesc_sw128(sb + OFF_TB + ks * 32, 16, 1024);
                     mma_bf16_ss(tbase + COL_E + bufi * 64, sdesc_sw128(sb + OFF_V + ks * 2048, 8192, 1024), bdesc,
-                                idesc_bf16(128, 64, 1, 0, 0), ks > 0);
+                                ID_MK, ks > 0);
                     mma_bf16_ss(tbase + COL_AW, sdesc_sw128(sb + OFF_KQ + bufi * 32768 + ks * 2048, 16384, 1024), bdesc,
-                                idesc_bf16(128, 64, 1, 0, 0), ks > 0);
+                                ID_MK, ks > 0);
                 }
                 mma_commit(bar_pmma);
             }
@@ -525,6 +567,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         // =========================== chain group ==================================
         const int row = tid - NPREP;          // TMEM lane = value row of S (quad = warp & 3)
         uint32_t mma_phase = 0;
+        const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_NEG = idesc_bf16(128, 64, 0, 1, 1);
+        const uint32_t ID_KM128 = idesc_bf16(128, 128, 0, 1, 0);
         auto cbar = [&]() { named_bar(2, NT - NPREP); };
         auto mma_wait = [&]() -> bool {
             const bool ok = mbar_wait_bounded(bar_cmma, mma_phase, x.wait_limit_ns);
@@ -551,7 +595,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         auto scale_cols = [&](int col0, float (&s)[16], const float* rho) {
             if (!ROT) {
 #pragma unroll
-                for (int u = 0; u < 16; ++u) s[u] *= rho[col0 + u];
+                for (int u4 = 0; u4 < 4; ++u4) {
+                    const float4 f = *reinterpret_cast<const float4*>(rho + col0 + 4 * u4);
+                    s[4 * u4] *= f.x; s[4 * u4 + 1] *= f.y; s[4 * u4 + 2] *= f.z; s[4 * u4 + 3] *= f.w;
+                }
             } else {
 #pragma unroll
                 for (int u = 0; u < 16; u += 2) {
@@ -563,17 +610,35 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                 }
             }
         };
+        // o for one chunk: O^T sits in TMEM with lane = value row, column = token.  Each 8x8
+        // block (8 value rows of this warp x 8 tokens) is transposed across 8 lanes so that
+        // every lane stores 8 consecutive value columns of one token (16 bytes in bf16).
         auto o_epilogue = [&](int c) {
             const int Lc = chunk_len(c);
             const uint32_t col = COL_O + (c & 1) * 64;
+            const int j8 = lane & 7, grp = lane >> 3;
+            OT* obase = o + tok(c, 0) * D + quad * 32 + grp * 8;
+            const size_t tstride = (size_t)p.H * D;
 #pragma unroll 1
-            for (int g = 0; g < 4; ++g) {
-                float vals[16];
-                tmem_ld16(tq + col + g * 16, vals);
+            for (int g = 0; g < 2; ++g) {
+                float vals[32];
+                tmem_ld32(tq + col + g * 32, vals);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int r = g * 16 + u;
-                    if (r < Lc) st_from_f32(o + tok(c, r) * D + row, vals[u]);
+                for (int blk8 = 0; blk8 < 4; ++blk8) {
+                    float v8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v8[e] = vals[blk8 * 8 + e];
+                    transpose8(v8, j8);
+                    const int r = g * 32 + blk8 * 8 + j8;
+                    if (r < Lc) {
+                        OT* dst = obase + (size_t)r * tstride;
+                        if constexpr (sizeof(OT) == 2) {
+                            *reinterpret_cast<uint4*>(dst) = pack8(v8);
+                        } else {
+                            reinterpret_cast<float4*>(dst)[0] = make_float4(v8[0], v8[1], v8[2], v8[3]);
+                            reinterpret_cast<float4*>(dst)[1] = make_float4(v8[4], v8[5], v8[6], v8[7]);
+                        }
+                    }
                 }
             }
         };
@@ -610,15 +675,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             tc_fence_after();
             // ---- E^T += -Stil Wm^T ;  O^T = Stil Qtil^T --------------------------------
             if (row == 0) {
+                const uint64_t dW = sdesc_sw128(sb + OFF_W + bufi * 16384, 8192, 1024);
+                const uint64_t dQ = sdesc_sw128(sb + OFF_KQ + bufi * 32768 + 8192, 16, 1024);
+#pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t kbk = ks >> 2, kin = (ks & 3) * 32;
                     const uint32_t a_t = tbase + COL_SB + ks * 8;
-                    mma_bf16_ts(tbase + COL_E + bufi * 64, a_t,
-                                sdesc_sw128(sb + OFF_W + bufi * 16384 + ks * 2048, 8192, 1024),
-                                idesc_bf16(128, 64, 0, 1, 1), 1);
+                    // descriptor start addresses advance in 16-byte units
+                    mma_bf16_ts(tbase + COL_E + bufi * 64, a_t, dW + (uint64_t)(ks * 2048 / 16), ID_NEG, 1);
                     mma_bf16_ts(tbase + COL_O + bufi * 64, a_t,
-                                sdesc_sw128(sb + OFF_KQ + bufi * 32768 + kbk * 16384 + 8192 + kin, 16, 1024),
-                                idesc_bf16(128, 64, 0, 0, 0), ks > 0);
+                                dQ + (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) / 16), ID_KK, ks > 0);
                 }
                 mma_commit(bar_cmma);
             }
@@ -630,11 +695,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                 const uint32_t col = COL_E + bufi * 64;
                 uint32_t w[32];
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float vals[16];
-                    tmem_ld16(tq + col + g * 16, vals);
+                for (int g = 0; g < 2; ++g) {
+                    float vals[32];
+                    tmem_ld32(tq + col + g * 32, vals);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) w[g * 8 + u] = pack_bf16x2(vals[2 * u], vals[2 * u + 1]);
+                    for (int u = 0; u < 16; ++u) w[g * 16 + u] = pack_bf16x2(vals[2 * u], vals[2 * u + 1]);
                 }
 #pragma unroll
                 for (int g = 0; g < 4; ++g) tmem_st8u(tq + col + g * 8, *reinterpret_cast<uint32_t(*)[8]>(w + g * 8));
@@ -645,12 +710,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             tc_fence_after();
             // ---- O^T += E^T Pm^T ;  S_acc += E^T Khat ---------------------------------------
             if (row == 0) {
+                const uint64_t dP = sdesc_sw128(sb + OFF_PM + bufi * 8192, 16, 1024);
+                const uint64_t dH = sdesc_sw128(sb + OFF_KH + bufi * 16384, 8192, 1024);
+#pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint32_t a_t = tbase + COL_E + bufi * 64 + ks * 8;
-                    mma_bf16_ts(tbase + COL_O + bufi * 64, a_t, sdesc_sw128(sb + OFF_PM + bufi * 8192 + ks * 32, 16, 1024),
-                                idesc_bf16(128, 64, 0, 0, 0), 1);
-                    mma_bf16_ts(tbase + COL_S, a_t, sdesc_sw128(sb + OFF_KH + bufi * 16384 + ks * 2048, 8192, 1024),
-                                idesc_bf16(128, 128, 0, 1, 0), 1);
+                    mma_bf16_ts(tbase + COL_O + bufi * 64, a_t, dP + (uint64_t)(ks * 32 / 16), ID_KK, 1);
+                    mma_bf16_ts(tbase + COL_S, a_t, dH + (uint64_t)(ks * 2048 / 16), ID_KM128, 1);
                 }
                 mma_commit(bar_cmma);
             }
@@ -662,21 +728,28 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                 const float* rho_C = vecs(c) + 64 + 256;
                 const float* rho_nx = vecs(c + 1) + 64;
 #pragma unroll 1
-                for (int g = 0; g < 8; ++g) {
-                    const int col0 = g * 16;
-                    float s[16];
-                    tmem_ld16(tq + COL_S + col0, s);
-                    scale_cols(col0, s, rho_C);
-                    if (last) {
-                        if (p.S_T) {
-                            float4* dst = reinterpret_cast<float4*>(p.S_T + ((size_t)bh * D + row) * D + col0);
+                for (int g = 0; g < 4; ++g) {
+                    const int col0 = g * 32;
+                    float s32[32];
+                    tmem_ld32(tq + COL_S + col0, s32);
 #pragma unroll
-                            for (int u4 = 0; u4 < 4; ++u4)
-                                dst[u4] = make_float4(s[4 * u4], s[4 * u4 + 1], s[4 * u4 + 2], s[4 * u4 + 3]);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float s[16];
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) s[u] = s32[hh * 16 + u];
+                        const int c16 = col0 + hh * 16;
+                        scale_cols(c16, s, rho_C);
+                        if (last) {
+                            if (p.S_T) {
+                                float4* dst = reinterpret_cast<float4*>(p.S_T + ((size_t)bh * D + row) * D + c16);
+#pragma unroll
+                                for (int u4 = 0; u4 < 4; ++u4)
+                                    dst[u4] = make_float4(s[4 * u4], s[4 * u4 + 1], s[4 * u4 + 2], s[4 * u4 + 3]);
+                            }
+                        } else {
+                            scale_cols(c16, s, rho_nx);
+                            store_state(c16, s);
                         }
-                    } else {
-                        scale_cols(col0, s, rho_nx);
-                        store_state(col0, s);
                     }
                 }
                 tmem_wait_st();
