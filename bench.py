@@ -81,6 +81,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "gdr_chunk_fwd_simt": ["simt_fwd.cuh", "common.cuh"],
     "gdr_chunk_fwd_tcgen05": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
+    "gdr_chunk_fwd_tcgen05_split": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
     "gdr_decode_step": ["decode.cuh", "common.cuh"],
 }
 
@@ -199,10 +200,15 @@ def run_ours(args):
     o = torch.empty((p.B, p.T, p.H, p.dv), dtype=dv_t["q"].dtype, device=dev)
     S_T = torch.empty((p.B, p.H, p.dv, p.dk), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    desc = gdr.fwd_desc(p.B, p.H, p.T, p.dk, p.dv, dv_t["q"].dtype, o.dtype, p.gate_mode, p.rotation,
+                        p.scale, args.algo)
+    ws_bytes = gdr.workspace_bytes(desc)
+    wsp = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
 
     def step():
         gdr.chunk_fwd(dv_t["q"], dv_t["k"], dv_t["v"], dv_t["g"], dv_t["beta"], dv_t["theta"], dv_t["S0"],
-                      gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o, S_T=S_T, stream=stream)
+                      gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o, S_T=S_T, stream=stream,
+                      workspace=wsp)
 
     for _ in range(args.warmup):
         step()
@@ -235,8 +241,7 @@ def run_ours(args):
     algo_bytes = p.nbytes_algorithmic
     avg_launch_s = statistics.mean(per_launch_ms) * 1e-3
     achieved_gbs = algo_bytes / avg_launch_s / 1e9
-    resolved = gdr.resolved_algo(gdr.fwd_desc(p.B, p.H, p.T, p.dk, p.dv, dv_t["q"].dtype, o.dtype,
-                                              p.gate_mode, p.rotation, p.scale, args.algo))
+    resolved = gdr.resolved_algo(desc)
     kernel_name = "gdr_chunk_fwd_" + resolved
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
@@ -258,7 +263,8 @@ def run_ours(args):
         def e2e_step():
             d = {k: (None if t is None else dv_t[k].copy_(t, non_blocking=True)) for k, t in pinned.items()}
             gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["theta"], d["S0"],
-                          gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o, S_T=S_T, stream=stream)
+                          gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o, S_T=S_T, stream=stream,
+                          workspace=wsp)
             o_h.copy_(o, non_blocking=True)
             S_h.copy_(S_T, non_blocking=True)
 
@@ -330,7 +336,7 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 3), "unit": "Mtokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms_max / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if resolved == "tcgen05" else "f32",
+        "dtype": "bf16" if resolved.startswith("tcgen05") else "f32",
         "data": "synthetic (seeded SplitMix64; q,k L2-normalised, bf16)",
         "config": {"workload": f"{args.workload}: B={p.B} H={p.H} T={p.T} dk={p.dk} dv={p.dv} chunk={p.chunk}, "
                                "bf16 q/k/v, fp32 g (raw gate, -softplus fused) and beta, S0=0",
@@ -421,7 +427,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
-    ap.add_argument("--algo", choices=["auto", "simt", "tcgen05"], default="auto")
+    ap.add_argument("--algo", choices=["auto", "simt", "tcgen05", "tcgen05_split"], default="auto")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-decode", action="store_true")

@@ -73,7 +73,11 @@ typedef enum { GDR_GATE_LOGDECAY = 0, GDR_GATE_NEG_SOFTPLUS = 1 } gdr_gate_mode;
 typedef enum {
     GDR_ALGO_AUTO = 0,    /* tensor-core chunk kernel when supported, else SIMT */
     GDR_ALGO_SIMT = 1,    /* fp32 CUDA-core chunk-WY kernel (every supported shape) */
-    GDR_ALGO_TCGEN05 = 2  /* tcgen05/TMEM chunk-WY kernel: bf16 q/k/v, dk = dv = 128 */
+    GDR_ALGO_TCGEN05 = 2, /* tcgen05/TMEM chunk-WY kernel, one CTA per (batch, head):
+                             bf16 q/k/v, dk = dv = 128 */
+    GDR_ALGO_TCGEN05_SPLIT = 3 /* same arithmetic; one CTA per head runs only the state chain
+                             while every other SM prepares chunks, handed over through a
+                             ring in the workspace (needs B*H < SM count; cooperative launch) */
 } gdr_algo;
 
 /* Shape and mode of one chunked forward call. */
@@ -110,7 +114,11 @@ GDR_API const char* gdr_status_string(gdr_status s);
 GDR_API const char* gdr_last_error_detail(void);
 
 /* Bytes of device workspace gdr_chunk_fwd needs for this descriptor (0 = none;
- * the workspace argument may then be NULL).  Returns 0 for an invalid desc. */
+ * the workspace argument may then be NULL).  Returns 0 for an invalid desc.  The split
+ * tensor-core kernel needs B*H*3 ring slots of 84,224 bytes plus 16 bytes of flags per
+ * head; it resets the flags itself (on the call's stream) and the buffer may be reused
+ * by later calls on the same stream.  Uses the current device's SM count when
+ * desc->algo is GDR_ALGO_AUTO. */
 GDR_API size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc);
 
 /*

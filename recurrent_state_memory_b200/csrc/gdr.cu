@@ -71,11 +71,36 @@ static bool tc_supported(const gdr_fwd_desc* d) {
     return d->qkv_dtype == GDR_BF16 && d->dk == 128 && d->dv == 128 && d->chunk == 64;
 }
 
-// The algorithm a descriptor runs with: AUTO takes the tensor-core kernel when it
-// supports the shape and dtype.
+static int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return 148; }
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) { cudaGetLastError(); return 148; }
+    return n;
+}
+
+// The split kernel pays off while the heads leave at least a third of the SMs for prep
+// workers and there is more than one chunk; it needs at least one worker.
+static bool split_fits(const gdr_fwd_desc* d, int sms) {
+    const long long nh = (long long)d->B * d->H;
+    return nh >= 1 && 3 * nh <= 2LL * sms && d->T > 64;
+}
+
+// The algorithm a descriptor runs with: AUTO takes a tensor-core kernel when it supports
+// the shape and dtype, the split one when the heads leave room for prep workers.
 static gdr_algo resolve_algo(const gdr_fwd_desc* d) {
-    if (d->algo == GDR_ALGO_AUTO) return tc_supported(d) ? GDR_ALGO_TCGEN05 : GDR_ALGO_SIMT;
+    if (d->algo == GDR_ALGO_AUTO) {
+        if (!tc_supported(d)) return GDR_ALGO_SIMT;
+        return split_fits(d, device_sm_count()) ? GDR_ALGO_TCGEN05_SPLIT : GDR_ALGO_TCGEN05;
+    }
     return d->algo;
+}
+
+static size_t split_ring_bytes(const gdr_fwd_desc* d) {
+    return (size_t)d->B * d->H * tcf::RING * tcf::SLOT_BYTES;
+}
+static size_t split_workspace_bytes(const gdr_fwd_desc* d) {
+    const size_t nh = (size_t)d->B * d->H;
+    return split_ring_bytes(d) + (nh * tcf::RING + nh) * sizeof(unsigned int);
 }
 
 static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
@@ -88,32 +113,57 @@ static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
     if (d->gate_mode != GDR_GATE_LOGDECAY && d->gate_mode != GDR_GATE_NEG_SOFTPLUS)
         return fail(GDR_ERR_INVALID_ARG, "bad gate_mode%s");
     if (d->rotation != 0 && d->rotation != 1) return fail(GDR_ERR_INVALID_ARG, "rotation must be 0 or 1%s");
-    if (d->algo != GDR_ALGO_AUTO && d->algo != GDR_ALGO_SIMT && d->algo != GDR_ALGO_TCGEN05)
+    if (d->algo != GDR_ALGO_AUTO && d->algo != GDR_ALGO_SIMT && d->algo != GDR_ALGO_TCGEN05 &&
+        d->algo != GDR_ALGO_TCGEN05_SPLIT)
         return fail(GDR_ERR_INVALID_ARG, "bad algo%s");
     if ((long long)d->B * d->H > 0x7fffffffLL) return fail(GDR_ERR_INVALID_ARG, "B*H too large%s");
-    if (d->algo == GDR_ALGO_TCGEN05 && !tc_supported(d))
-        return fail(GDR_ERR_UNSUPPORTED, "the tcgen05 kernel needs bf16 q/k/v and dk = dv = 128%s");
+    if ((d->algo == GDR_ALGO_TCGEN05 || d->algo == GDR_ALGO_TCGEN05_SPLIT) && !tc_supported(d))
+        return fail(GDR_ERR_UNSUPPORTED, "the tcgen05 kernels need bf16 q/k/v and dk = dv = 128%s");
     return GDR_OK;
 }
 
-template <bool ROT, typename OT>
-static gdr_status launch_tc(const FwdParams& p, cudaStream_t st) {
-    auto kern = tcf::chunk_fwd_tc_kernel<ROT, OT>;
+template <int MODE, bool ROT, typename OT>
+static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
+    auto kern = tcf::chunk_fwd_tc_kernel<MODE, ROT, OT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tcgen05 chunk kernel)");
     tcf::TcExtra x;
     x.wait_limit_ns = s_wait_limit_ns;
     x.fault_skip_commit = s_fault_skip_commit;
-    kern<<<p.B * p.H, tcf::NT, tcf::SMEM_BYTES, st>>>(p, x);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
+    tcf::SplitArgs sa{nullptr, nullptr, nullptr};
+    if (MODE == 0) {
+        kern<<<p.B * p.H, tcf::NT, tcf::SMEM_BYTES, st>>>(p, x, sa);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
+        return GDR_OK;
+    }
+    // Split: the whole grid must be resident at once (one CTA per SM), which a cooperative
+    // launch guarantees or refuses.
+    const int nh = p.B * p.H;
+    const int sms = device_sm_count();
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, tcf::NT, tcf::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    const int grid = sms * (per_sm < 1 ? 1 : per_sm > 1 ? 1 : per_sm);
+    if (per_sm < 1 || grid <= nh) return fail(GDR_ERR_UNSUPPORTED, "split kernel: B*H must be below the SM count%s");
+    const size_t nring = (size_t)nh * tcf::RING * tcf::SLOT_BYTES;
+    sa.ring = static_cast<uint8_t*>(ws);
+    sa.ready = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + nring);
+    sa.consumed = sa.ready + (size_t)nh * tcf::RING;
+    e = cudaMemsetAsync(sa.ready, 0, ((size_t)nh * tcf::RING + nh) * sizeof(unsigned int), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split flags)");
+    void* args[] = {const_cast<FwdParams*>(&p), &x, &sa};
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(tcf::NT), args,
+                                    tcf::SMEM_BYTES, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cooperative launch(tcgen05 split kernel)");
     return GDR_OK;
 }
 
-static gdr_status dispatch_tc(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st) {
+template <int MODE>
+static gdr_status dispatch_tc_mode(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws) {
     const bool ob = d->out_dtype == GDR_BF16;
-    if (d->rotation) return ob ? launch_tc<true, __nv_bfloat16>(p, st) : launch_tc<true, float>(p, st);
-    return ob ? launch_tc<false, __nv_bfloat16>(p, st) : launch_tc<false, float>(p, st);
+    if (d->rotation) return ob ? launch_tc<MODE, true, __nv_bfloat16>(p, st, ws) : launch_tc<MODE, true, float>(p, st, ws);
+    return ob ? launch_tc<MODE, false, __nv_bfloat16>(p, st, ws) : launch_tc<MODE, false, float>(p, st, ws);
 }
 
 // ----------------------------------------------------------------- decode ----
@@ -163,6 +213,7 @@ const char* gdr_last_error_detail(void) { return t_detail; }
 
 size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc) {
     if (check_fwd_desc(desc) != GDR_OK) return 0;
+    if (resolve_algo(desc) == GDR_ALGO_TCGEN05_SPLIT) return split_workspace_bytes(desc);
     return 0;
 }
 
@@ -194,7 +245,12 @@ gdr_status gdr_chunk_fwd(const gdr_fwd_desc* d, const void* q, const void* k, co
     p.S0 = S0; p.o = o; p.S_T = S_T;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d->T == 0 && !S_T) return GDR_OK;
-    if (resolve_algo(d) == GDR_ALGO_TCGEN05) return dispatch_tc(d, p, st);
+    const gdr_algo algo = resolve_algo(d);
+    if (algo == GDR_ALGO_TCGEN05_SPLIT && d->T > 0) {
+        if (!aligned16(workspace)) return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned%s");
+        return dispatch_tc_mode<1>(d, p, st, workspace);
+    }
+    if (algo == GDR_ALGO_TCGEN05 || algo == GDR_ALGO_TCGEN05_SPLIT) return dispatch_tc_mode<0>(d, p, st, nullptr);
     return d->rotation ? dispatch_simt_dk<true>(d, p, st) : dispatch_simt_dk<false>(d, p, st);
 }
 

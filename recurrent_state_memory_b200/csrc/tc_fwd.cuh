@@ -70,6 +70,26 @@ constexpr uint32_t OFF_BAR = (OFF_VEC + 2 * VEC_FLOATS * 4 + 63) & ~63u;
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // slack for 1024-byte alignment
 
+// Split mode: a per-head ring in global memory carries each chunk's operands from the prep
+// workers to the chain CTA.  Slot layout (bytes), identical to the chain's shared-memory copy:
+constexpr uint32_t SL_Q = 0;          // Qtil K-major: 2 kblocks x 64 rows x 128 B
+constexpr uint32_t SL_KH = 16384;     // Khat K-major: 2 kblocks x 64 rows x 128 B
+constexpr uint32_t SL_W = 32768;      // Wm^T bf16 MN-major: 128 dk rows x 128 B
+constexpr uint32_t SL_PM = 49152;     // Pm K-major: 64 rows x 128 B
+constexpr uint32_t SL_TB = 57344;     // Tb K-major: 64 rows x 128 B
+constexpr uint32_t SL_V = 65536;      // V, MN-major: 2 groups x 64 tokens x 128 B
+constexpr uint32_t SL_VEC = 81920;    // beta, rho_ref, rho_C (VEC_FLOATS floats)
+constexpr uint32_t SLOT_BYTES = SL_VEC + VEC_FLOATS * 4;
+constexpr uint32_t SLOT_STRIDE = (SLOT_BYTES + 1023) & ~1023u;   // slot buffers in the chain CTA
+constexpr int RING = 3;               // ring slots per head
+static_assert(2 * SLOT_STRIDE <= OFF_BAR, "chain slot buffers overlap the barriers");
+
+struct SplitArgs {
+    uint8_t* ring;            // [B*H][RING][SLOT_BYTES]
+    unsigned int* ready;      // [B*H][RING]: index + 1 of the chunk a slot holds
+    unsigned int* consumed;   // [B*H]: chunks the chain has copied out of the ring
+};
+
 // Device status bits (gdr_query_device_status).
 constexpr unsigned STATUS_TIMEOUT = 1u;
 constexpr unsigned STATUS_RANGE = 2u;
@@ -123,8 +143,13 @@ __device__ __forceinline__ uint4 pack8(const float* m8) {
                       pack_bf16x2(m8[4], m8[5]), pack_bf16x2(m8[6], m8[7]));
 }
 
-template <bool ROT, typename OT>
-__global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtra x) {
+// MODE 0 (fused): one CTA per (batch, head) runs both groups.
+// MODE 1 (split): CTAs [0, B*H) run the chain of head blockIdx.x (warps 8-11) with a loader
+// warp that copies ring slots into shared memory; every other CTA is a prep worker whose
+// warps 0-7 compute chunks in chunk-major task order and whose warps 8-11 copy finished
+// operands into the ring.  The grid must be co-resident (cooperative launch).
+template <int MODE, bool ROT, typename OT>
+__global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtra x, SplitArgs sa) {
     using namespace tc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -147,14 +172,25 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3;
-    const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+    const int NH = p.B * p.H;
+    const bool chain_cta = (MODE == 0) || ((int)blockIdx.x < NH);
+    const int bh = chain_cta ? (int)blockIdx.x : 0;
     const __nv_bfloat16* __restrict__ q = static_cast<const __nv_bfloat16*>(p.q);
     const __nv_bfloat16* __restrict__ k = static_cast<const __nv_bfloat16*>(p.k);
     const __nv_bfloat16* __restrict__ v = static_cast<const __nv_bfloat16*>(p.v);
     OT* __restrict__ o = static_cast<OT*>(p.o);
     const int nchunks = (p.T + C - 1) / C;
     auto chunk_len = [&](int c) -> int { return min(C, p.T - c * C); };
-    auto tok = [&](int c, int r) -> size_t { return ((size_t)b * p.T + (c * C + r)) * p.H + h; };
+    auto tokh = [&](int bhx, int c, int r) -> size_t {
+        return ((size_t)(bhx / p.H) * p.T + (c * C + r)) * p.H + (bhx % p.H);
+    };
+    auto tok = [&](int c, int r) -> size_t { return tokh(bh, c, r); };
+    // Chain-side buffers of chunk c: fused mode reads the prep group's double buffers, split
+    // mode the slot copied from the ring.
+    auto slot_base = [&](int c) -> uint32_t { return (uint32_t)(c & 1) * SLOT_STRIDE; };
+    auto chain_vec = [&](int c) -> const float* {
+        return MODE == 0 ? vecs(c) : reinterpret_cast<const float*>(base + slot_base(c) + SL_VEC);
+    };
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -164,7 +200,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         mbar_init(bar_pmma, 1);
         mbar_init(bar_cmma, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(bar_full + i, NPREP);
+            // split chain CTAs: one arrival (the loader's expect_tx) plus the copied bytes
+            mbar_init(bar_full + i, (MODE == 1 && chain_cta) ? 1 : NPREP);
             mbar_init(bar_empty + i, NT - NPREP);
             mbar_init(bar_rho + i, NPREP);
         }
@@ -179,8 +216,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
     const uint32_t tbase = *tmem_slot;
     const uint32_t tq = tbase + ((uint32_t)(quad * 32) << 16);   // this warp's lane quadrant
 
-    if (nchunks > 0 && tid < NPREP) {
+    if (nchunks > 0 && tid < NPREP && (MODE == 0 || !chain_cta)) {
         // =========================== prep group ===================================
+        // Tasks: fused mode, chunk it of this CTA's head; split mode, task wk + it * W in
+        // chunk-major order (chunk = task / NH, head = task % NH).
+        const int W = (MODE == 0) ? 1 : (int)gridDim.x - NH;
+        const int wk = (MODE == 0) ? 0 : (int)blockIdx.x - NH;
+        const int ntasks = (MODE == 0) ? nchunks : (NH * nchunks - wk + W - 1) / W;
+        auto task_bh = [&](int it) -> int { return MODE == 0 ? bh : (wk + it * W) % NH; };
+        auto task_c = [&](int it) -> int { return MODE == 0 ? it : (wk + it * W) / NH; };
         // Decay passes: each thread owns 4 key dims (two key pairs) of one 8-token segment;
         // warp w handles tokens 8w .. 8w+7.  The reference token 31 is the last token of
         // segment 3, so segments 0-3 run backward from it and segments 4-7 forward.
@@ -199,9 +243,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         // Register prefetch of this thread's raw inputs for one chunk.
         uint2 rk[8], rq[8];
         float4 ra[8];       // real: 4 gates; rotation: gates of the 2 pairs, then their 2 angles
-        auto prefetch = [&](int c) {
+        auto prefetch = [&](int bhx, int c) {
             const int Lc = chunk_len(c);
-            const size_t t0 = tok(c, 8 * sg);
+            const size_t t0 = tokh(bhx, c, 8 * sg);
             const __nv_bfloat16* kp = k + t0 * D + 4 * dg;
             const __nv_bfloat16* qp = q + t0 * D + 4 * dg;
 #pragma unroll
@@ -239,11 +283,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         };
         const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
 
-        prefetch(0);
-        for (int c = 0; c < nchunks; ++c) {
+        if (ntasks > 0) prefetch(task_bh(0), task_c(0));
+        for (int it = 0; it < ntasks; ++it) {
+            const int c = task_c(it), bhx = task_bh(it);
             const int Lc = chunk_len(c);
-            const int bufi = c & 1;
-            float* vec = vecs(c);
+            const int bufi = it & 1;
+            float* vec = vecs(it);
             float* sbeta = vec;
             float* rho_ref = vec + 64;
             float* rho_C = vec + 64 + 256;
@@ -251,15 +296,18 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             uint8_t* KH = base + OFF_KH + bufi * 16384;
 
             // V tile of this chunk (MN-major for V^T), asynchronously; done before the U MMA.
+            // (Split mode: the copy-out warps move V straight into the ring.)
+            if (MODE == 0) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int id = tid * 4 + j;
                 const int i = id >> 4, c16 = id & 15;
                 const bool ok = i < Lc;
-                const void* src = ok ? (const void*)(v + tok(c, i) * D + c16 * 8) : (const void*)v;
+                const void* src = ok ? (const void*)(v + tokh(bhx, c, i) * D + c16 * 8) : (const void*)v;
                 cp_async16(sb + OFF_V + (uint32_t)(c16 >> 3) * 8192u + sw128_off(i, c16 & 7), src, ok ? 16u : 0u);
             }
             cp_async_commit();
+            }
 
             // ---- pass 1: per-token decays and segment products ---------------------------
             // real:     al/iv[s][d] = alpha and 1/alpha of dim 4dg+d;
@@ -303,11 +351,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                 qtp[0] = make_float4(PA[0], PA[1], PA[2], PA[3]);
                 qtp[1] = make_float4(PI[0], PI[1], PI[2], PI[3]);
             }
-            if (tid < 64) sbeta[tid] = tid < Lc ? __ldg(p.beta + tok(c, tid)) : 0.f;
+            if (tid < 64) sbeta[tid] = tid < Lc ? __ldg(p.beta + tokh(bhx, c, tid)) : 0.f;
             named_bar(1, NPREP);
-            // Buffers of chunk c - 2 must be released by the chain before they are rewritten.
-            if (c >= 2) {
-                const bool ok = mbar_wait_bounded(bar_empty + bufi, ((c - 2) >> 1) & 1, x.wait_limit_ns);
+            // Buffers of task it - 2 must be released (by the chain, or by the copy-out warps)
+            // before they are rewritten.
+            if (it >= 2) {
+                const bool ok = mbar_wait_bounded(bar_empty + bufi, ((it - 2) >> 1) & 1, x.wait_limit_ns);
                 if (!ok) atomicExch(abort_p, 1);
             }
             named_bar(1, NPREP);
@@ -417,8 +466,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             }
             fence_proxy_async_smem();
             named_bar(1, NPREP);
-            mbar_arrive(bar_rho + bufi);
-            if (c + 1 < nchunks) prefetch(c + 1);
+            if (MODE == 0) mbar_arrive(bar_rho + bufi);
+            if (it + 1 < ntasks) prefetch(task_bh(it + 1), task_c(it + 1));
 
             // ---- MMA1: [Ktil ; Qtil] Khat^T -> TMEM ------------------------------------
             tc_fence_after();
@@ -517,6 +566,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                 named_bar(1, NPREP);
             }
             // Tb = Tm diag(beta), zero above the block diagonal, -> bf16 K-major [r][i].
+            // (Split mode keeps two Tb tiles in the unused V area, one per buffer.)
+            const uint32_t tb_off = (MODE == 0) ? OFF_TB : OFF_V + (uint32_t)bufi * 8192u;
             {
                 const int r = tid >> 2, qq = tid & 3;
 #pragma unroll
@@ -528,18 +579,19 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                         const int i = i0 + u;
                         m8[u] = ((i >> 4) <= (r >> 4)) ? Tf[r * AS + i] * sbeta[i] : 0.f;
                     }
-                    *reinterpret_cast<uint4*>(base + OFF_TB + sw128_off(r, qq * 2 + hh)) = pack8(m8);
+                    *reinterpret_cast<uint4*>(base + tb_off + sw128_off(r, qq * 2 + hh)) = pack8(m8);
                 }
             }
-            cp_async_wait_all();
+            if (MODE == 0) cp_async_wait_all();
             publish();
 
             // ---- U^T = V^T Tb^T -> E[c&1];  Wm^T = Ktil^T Tb^T -> A'/W columns -------------
             if (tid == 0) {
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t bdesc = sdesc_sw128(sb + OFF_TB + ks * 32, 16, 1024);
-                    mma_bf16_ss(tbase + COL_E + bufi * 64, sdesc_sw128(sb + OFF_V + ks * 2048, 8192, 1024), bdesc,
-                                ID_MK, ks > 0);
+                    const uint64_t bdesc = sdesc_sw128(sb + tb_off + ks * 32, 16, 1024);
+                    if (MODE == 0)
+                        mma_bf16_ss(tbase + COL_E + bufi * 64, sdesc_sw128(sb + OFF_V + ks * 2048, 8192, 1024), bdesc,
+                                    ID_MK, ks > 0);
                     mma_bf16_ss(tbase + COL_AW, sdesc_sw128(sb + OFF_KQ + bufi * 32768 + ks * 2048, 16384, 1024), bdesc,
                                 ID_MK, ks > 0);
                 }
@@ -563,12 +615,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             mbar_arrive(bar_full + bufi);
         }
         if (bad) atomicExch(range_flag, 1);
-    } else if (nchunks > 0) {
+    } else if (nchunks > 0 && tid >= NPREP && chain_cta) {
         // =========================== chain group ==================================
         const int row = tid - NPREP;          // TMEM lane = value row of S (quad = warp & 3)
         uint32_t mma_phase = 0;
         const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_NEG = idesc_bf16(128, 64, 0, 1, 1);
-        const uint32_t ID_KM128 = idesc_bf16(128, 128, 0, 1, 0);
+        const uint32_t ID_KM128 = idesc_bf16(128, 128, 0, 1, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
         auto cbar = [&]() { named_bar(2, NT - NPREP); };
         auto mma_wait = [&]() -> bool {
             const bool ok = mbar_wait_bounded(bar_cmma, mma_phase, x.wait_limit_ns);
@@ -644,9 +696,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         };
 
         // Initial state, prescaled by the first chunk's reference decay.
-        bool alive = bounded(bar_rho + 0, 0);
+        bool alive = bounded(MODE == 0 ? bar_rho + 0 : bar_full + 0, 0);
         if (alive) {
-            const float* rho_ref0 = vecs(0) + 64;
+            const float* rho_ref0 = chain_vec(0) + 64;
 #pragma unroll 1
             for (int g = 0; g < 8; ++g) {
                 const int col0 = g * 16;
@@ -675,15 +727,26 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             tc_fence_after();
             // ---- E^T += -Stil Wm^T ;  O^T = Stil Qtil^T --------------------------------
             if (row == 0) {
-                const uint64_t dW = sdesc_sw128(sb + OFF_W + bufi * 16384, 8192, 1024);
-                const uint64_t dQ = sdesc_sw128(sb + OFF_KQ + bufi * 32768 + 8192, 16, 1024);
+                const uint32_t sl = sb + slot_base(c);
+                if (MODE == 1) {
+                    // U^T = V^T Tb^T from the slot (the fused prep group does this itself)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ss(tbase + COL_E + bufi * 64, sdesc_sw128(sl + SL_V + ks * 2048, 8192, 1024),
+                                    sdesc_sw128(sl + SL_TB + ks * 32, 16, 1024), ID_MK, ks > 0);
+                }
+                const uint64_t dW = MODE == 0 ? sdesc_sw128(sb + OFF_W + bufi * 16384, 8192, 1024)
+                                              : sdesc_sw128(sl + SL_W, 8192, 1024);
+                const uint64_t dQ = MODE == 0 ? sdesc_sw128(sb + OFF_KQ + bufi * 32768 + 8192, 16, 1024)
+                                              : sdesc_sw128(sl + SL_Q, 16, 1024);
+                const uint32_t qkb = MODE == 0 ? 16384u : 8192u;   // K-block stride of the Qtil tile
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t a_t = tbase + COL_SB + ks * 8;
                     // descriptor start addresses advance in 16-byte units
                     mma_bf16_ts(tbase + COL_E + bufi * 64, a_t, dW + (uint64_t)(ks * 2048 / 16), ID_NEG, 1);
                     mma_bf16_ts(tbase + COL_O + bufi * 64, a_t,
-                                dQ + (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) / 16), ID_KK, ks > 0);
+                                dQ + (uint64_t)(((ks >> 2) * qkb + (ks & 3) * 32) / 16), ID_KK, ks > 0);
                 }
                 mma_commit(bar_cmma);
             }
@@ -710,8 +773,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             tc_fence_after();
             // ---- O^T += E^T Pm^T ;  S_acc += E^T Khat ---------------------------------------
             if (row == 0) {
-                const uint64_t dP = sdesc_sw128(sb + OFF_PM + bufi * 8192, 16, 1024);
-                const uint64_t dH = sdesc_sw128(sb + OFF_KH + bufi * 16384, 8192, 1024);
+                const uint32_t sl = sb + slot_base(c);
+                const uint64_t dP = MODE == 0 ? sdesc_sw128(sb + OFF_PM + bufi * 8192, 16, 1024)
+                                              : sdesc_sw128(sl + SL_PM, 16, 1024);
+                const uint64_t dH = MODE == 0 ? sdesc_sw128(sb + OFF_KH + bufi * 16384, 8192, 1024)
+                                              : sdesc_sw128(sl + SL_KH, 8192, 1024);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint32_t a_t = tbase + COL_E + bufi * 64 + ks * 8;
@@ -723,10 +789,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             if (!mma_wait()) break;
 
             // ---- S <- S_acc (P_m^{-1} P_C), then prescale by the next reference ----------
-            if (!last && !bounded(bar_rho + ((c + 1) & 1), ((c + 1) >> 1) & 1)) break;
+            if (!last && !bounded((MODE == 0 ? bar_rho : bar_full) + ((c + 1) & 1), ((c + 1) >> 1) & 1)) break;
             {
-                const float* rho_C = vecs(c) + 64 + 256;
-                const float* rho_nx = vecs(c + 1) + 64;
+                const float* rho_C = chain_vec(c) + 64 + 256;
+                const float* rho_nx = chain_vec(c + 1) + 64;
 #pragma unroll 1
                 for (int g = 0; g < 4; ++g) {
                     const int col0 = g * 32;
@@ -760,7 +826,81 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         }
     }
 
-    if (nchunks == 0 && p.S_T) {
+    if (MODE == 1 && nchunks > 0 && chain_cta && warp == 0) {
+        // ============ split mode: loader of the chain CTA (one warp, lane 0 issues) ============
+        for (int c = 0; c < nchunks; ++c) {
+            const int bufi = c & 1;
+            bool ok = true;
+            if (lane == 0) {
+                // the chain must be done with chunk c - 2 before its buffer is refilled
+                if (c >= 2) ok = mbar_wait_bounded(bar_empty + bufi, ((c - 2) >> 1) & 1, x.wait_limit_ns);
+                const int slot = c % RING;
+                if (ok) ok = spin_until_ge(sa.ready + (size_t)bh * RING + slot, (unsigned)(c + 1), x.wait_limit_ns);
+                if (ok) {
+                    fence_proxy_async_global();
+                    const uint8_t* src = sa.ring + ((size_t)bh * RING + slot) * SLOT_BYTES;
+                    mbar_arrive_expect_tx(bar_full + bufi, SLOT_BYTES);
+                    for (uint32_t off = 0; off < SLOT_BYTES; off += 16384u) {
+                        const uint32_t n = SLOT_BYTES - off < 16384u ? SLOT_BYTES - off : 16384u;
+                        bulk_g2s(sb + slot_base(c) + off, src + off, n, bar_full + bufi);
+                    }
+                    // the ring slot may be reused once its bytes have landed here
+                    ok = mbar_wait_bounded(bar_full + bufi, (c >> 1) & 1, x.wait_limit_ns);
+                    if (ok) st_release_gpu(sa.consumed + bh, (unsigned)(c + 1));
+                }
+                if (!ok) atomicExch(abort_p, 1);
+            }
+            if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
+        }
+    }
+    if (MODE == 1 && nchunks > 0 && !chain_cta && tid >= NPREP) {
+        // ============ split mode: copy-out warps of a prep worker ==============================
+        const int ct = tid - NPREP;
+        const int W = (int)gridDim.x - NH, wk = (int)blockIdx.x - NH;
+        const int ntasks = (NH * nchunks - wk + W - 1) / W;
+        auto cbar = [&]() { named_bar(2, NT - NPREP); };
+        for (int it = 0; it < ntasks; ++it) {
+            const int bufi = it & 1;
+            const int task = wk + it * W, c = task / NH, bhx = task % NH, slot = c % RING;
+            const int Lc = chunk_len(c);
+            bool ok = mbar_wait_bounded(bar_full + bufi, (it >> 1) & 1, x.wait_limit_ns);
+            // the chain must have copied chunk c - RING out of this slot
+            if (ok && ct == 0 && c >= RING)
+                ok = spin_until_ge(sa.consumed + bhx, (unsigned)(c - RING + 1), x.wait_limit_ns);
+            if (!ok) atomicExch(abort_c, 1);
+            cbar();
+            if (*abort_c) break;
+            uint8_t* dst = sa.ring + ((size_t)bhx * RING + slot) * SLOT_BYTES;
+            // shared-memory tiles of this task -> ring slot (16-byte pieces)
+            auto copy16 = [&](uint32_t src_off, uint32_t dst_off, uint32_t bytes) {
+                for (uint32_t o16 = (uint32_t)ct * 16u; o16 < bytes; o16 += (NT - NPREP) * 16u)
+                    *reinterpret_cast<uint4*>(dst + dst_off + o16) = *reinterpret_cast<const uint4*>(base + src_off + o16);
+            };
+            copy16(OFF_KQ + bufi * 32768 + 8192, SL_Q, 8192);
+            copy16(OFF_KQ + bufi * 32768 + 16384 + 8192, SL_Q + 8192, 8192);
+            copy16(OFF_KH + bufi * 16384, SL_KH, 16384);
+            copy16(OFF_W + bufi * 16384, SL_W, 16384);
+            copy16(OFF_PM + bufi * 8192, SL_PM, 8192);
+            copy16(OFF_V + bufi * 8192, SL_TB, 8192);
+            copy16(OFF_VEC + bufi * VEC_FLOATS * 4, SL_VEC, VEC_FLOATS * 4);
+            // the shared buffers may be refilled by the prep warps now
+            mbar_arrive(bar_empty + bufi);
+            // V of this chunk straight from the input into the slot's MN-major layout
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int id = ct * 8 + j;
+                const int i = id >> 4, c16 = id & 15;
+                uint4 val = make_uint4(0u, 0u, 0u, 0u);
+                if (i < Lc) val = __ldg(reinterpret_cast<const uint4*>(v + tokh(bhx, c, i) * D + c16 * 8));
+                *reinterpret_cast<uint4*>(dst + SL_V + (uint32_t)(c16 >> 3) * 8192u + sw128_off(i, c16 & 7)) = val;
+            }
+            __threadfence();
+            cbar();
+            if (ct == 0) st_release_gpu(sa.ready + (size_t)bhx * RING + slot, (unsigned)(c + 1));
+        }
+    }
+
+    if (nchunks == 0 && p.S_T && chain_cta) {
         for (int e = tid; e < D * D; e += NT)
             p.S_T[(size_t)bh * D * D + e] = p.S0 ? p.S0[(size_t)bh * D * D + e] : 0.f;
     }

@@ -18,18 +18,19 @@ def G():
     gdr.debug_set_tc_fault(False, 0)
 
 
-def test_bounded_wait_gives_up_and_reports(G):
+@pytest.mark.parametrize("algo", ["tcgen05", "tcgen05_split"])
+def test_bounded_wait_gives_up_and_reports(G, algo):
     """A barrier that nothing signals: the wait runs out after 5 ms, the kernel frees
     its tensor memory and returns, the status word says GDR_ERR_TIMEOUT; the next
     normal call on the same context is correct."""
     import torch
     p = I.make_fwd(1, 128, 2, 128, 128, dtype="bf16", seed=7, s0_std=0.2)
     G.debug_set_tc_fault(True, 5_000_000)
-    U.run_gpu_fwd(p, "tcgen05")
+    U.run_gpu_fwd(p, algo)
     assert G.query_device_status() == G.GDR_ERR_TIMEOUT
     assert G.query_device_status() == G.GDR_OK            # read-and-clear
     G.debug_set_tc_fault(False, 0)
-    o, S = U.run_gpu_fwd(p, "tcgen05")
+    o, S = U.run_gpu_fwd(p, algo)
     assert G.query_device_status() == G.GDR_OK
     o_ref, S_ref = U.oracle_fwd(p)
     U.assert_fwd_parity(p, o, S, o_ref, S_ref)

@@ -8,12 +8,17 @@ import parity_util as U
 
 pytestmark = pytest.mark.gpu
 
-ALGOS_ALL = ["simt", "tcgen05"]
+ALGOS_ALL = ["simt", "tcgen05", "tcgen05_split"]
+TC_ALGOS = ["tcgen05", "tcgen05_split"]
 
 
-def _skip_unsupported(algo, dtype, dk, dv):
-    if algo == "tcgen05" and not (dtype == "bf16" and dk == 128 and dv == 128):
-        pytest.skip("tcgen05 kernel: bf16 q/k/v with dk = dv = 128 only")
+def _skip_unsupported(algo, dtype, dk, dv, nh=1):
+    if algo.startswith("tcgen05") and not (dtype == "bf16" and dk == 128 and dv == 128):
+        pytest.skip("tcgen05 kernels: bf16 q/k/v with dk = dv = 128 only")
+    if algo == "tcgen05_split":
+        import torch
+        if nh >= torch.cuda.get_device_properties(0).multi_processor_count:
+            pytest.skip("split kernel: B*H must be below the SM count")
 
 
 @pytest.fixture(scope="module")
@@ -51,7 +56,7 @@ CASES = [
     c[0], c[1], c[2], c[3], c[4], c[5], "_rot" if c[6] else "", "_s0" if c[7] else ""))
 def test_parity_small(G, algo, case):
     B, H, T, dk, dv, dtype, rot, s0, scale = case
-    _skip_unsupported(algo, dtype, dk, dv)
+    _skip_unsupported(algo, dtype, dk, dv, B * H)
     p = I.make_fwd(B, T, H, dk, dv, dtype=dtype, seed=1000 + T + dk, rotation=rot,
                    s0_std=0.5 if s0 else None, scale=scale)
     o, S = U.run_gpu_fwd(p, algo)
@@ -144,6 +149,8 @@ FULL = ["b4_h16_t4096_d128", "b16_h12_t4096_d128_slow_s0", "b2_h16_t8192_d128_ro
 def test_full_size_configs_sampled(G, algo, name):
     """Full-size workloads in the benchmark's launch configuration; the oracle
     recomputes a sample of whole heads (every token of each sampled head)."""
+    cfg = I.FWD_CONFIGS[name]
+    _skip_unsupported(algo, cfg["dtype"], cfg["dk"], cfg["dv"], cfg["B"] * cfg["H"])
     p = I.make_config(name)
     o, S = U.run_gpu_fwd(p, algo)
     rng = np.random.default_rng(0)
@@ -173,9 +180,10 @@ TC_CASES = [
 ]
 
 
+@pytest.mark.parametrize("algo", TC_ALGOS)
 @pytest.mark.parametrize("case", TC_CASES, ids=lambda c: "B{}H{}T{}{}{}_{}_g{}".format(
     c[0], c[1], c[2], "_rot" if c[3] else "", "_s0" if c[4] else "", c[5], c[6]))
-def test_tcgen05_parity(G, case):
+def test_tcgen05_parity(G, case, algo):
     """The tensor-core kernel against the oracle: ragged tails, rotation, initial state,
     both output dtypes and both gate modes."""
     import torch
@@ -187,7 +195,7 @@ def test_tcgen05_parity(G, case):
         p.gate_mode = I.GATE_LOGDECAY
     t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "g", "beta", "theta", "S0")}
     o, S = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["theta"], t["S0"], gate_mode=p.gate_mode,
-                       scale=p.scale, algo="tcgen05",
+                       scale=p.scale, algo=algo,
                        out_dtype=torch.float32 if odt == "f32" else torch.bfloat16)
     torch.cuda.synchronize()
     assert G.query_device_status() == G.GDR_OK
@@ -198,8 +206,22 @@ def test_tcgen05_parity(G, case):
 def test_auto_picks_tensor_cores_for_bf16_d128(G):
     import torch
     d = G.fwd_desc(1, 1, 64, 128, 128, torch.bfloat16, torch.bfloat16)
-    assert G.resolved_algo(d) == "tcgen05"
+    assert G.resolved_algo(d) == "tcgen05"                    # a single chunk: fused
+    d = G.fwd_desc(4, 16, 4096, 128, 128, torch.bfloat16, torch.bfloat16)
+    assert G.resolved_algo(d) == "tcgen05_split"              # few heads: chain + prep workers
+    assert G.workspace_bytes(d) >= 64 * 3 * 84224
+    d = G.fwd_desc(16, 12, 4096, 128, 128, torch.bfloat16, torch.bfloat16)
+    assert G.resolved_algo(d) == "tcgen05"                    # many heads: fused
     d = G.fwd_desc(1, 1, 64, 64, 64, torch.bfloat16, torch.bfloat16)
     assert G.resolved_algo(d) == "simt"
     d = G.fwd_desc(1, 1, 64, 128, 128, torch.float32, torch.float32)
     assert G.resolved_algo(d) == "simt"
+
+
+def test_split_matches_fused_bitwise_state_free_parts(G):
+    """The split kernel runs the same arithmetic as the fused one: identical outputs."""
+    import torch
+    p = I.make_fwd(2, 700, 3, 128, 128, dtype="bf16", seed=61, s0_std=0.2, rotation=True)
+    o1, S1 = U.run_gpu_fwd(p, "tcgen05")
+    o2, S2 = U.run_gpu_fwd(p, "tcgen05_split")
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
