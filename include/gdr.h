@@ -171,6 +171,37 @@ GDR_API gdr_status gdr_decode_step(const gdr_dec_desc* desc,
  */
 GDR_API gdr_status gdr_query_device_status(gdr_stream_t stream);
 
+/*
+ * gdr_chunk_fwd without a workspace argument: the library allocates nothing, ever.
+ *
+ * The pages have no counterpart to this call; it serves callers that cannot hand the
+ * library device memory.  Examples: plain-C hosts whose own memory manager owns all of
+ * the GPU's memory and forbids further cudaMalloc, and serving loops that must not
+ * call cudaMalloc or cudaFree on their latency path, because those calls can
+ * synchronise the device.
+ *
+ * It runs the split tensor-core kernel (same arithmetic and results as
+ * gdr_chunk_fwd with GDR_ALGO_TCGEN05_SPLIT) with the kernel's hand-off ring in a scratch
+ * array compiled into the library: GDR_NOALLOC_MAX_HEADS * 3 slots of 84,224 bytes plus
+ * flags (about 7.7 MiB), which every GPU that loads the library holds until the process
+ * exits.
+ *   - desc->algo must be GDR_ALGO_AUTO or GDR_ALGO_TCGEN05_SPLIT; q, k, v must be bf16 with
+ *     dk = dv = 128; B*H must not exceed GDR_NOALLOC_MAX_HEADS, else GDR_ERR_UNSUPPORTED with
+ *     a message (nothing launched).  Other arguments as for gdr_chunk_fwd.
+ *   - The first call on each device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any stream capture.
+ *   - Every call shares the one scratch array, which keeps the last call's contents; each
+ *     call clears the flags it needs on its own stream first.  Calls that overlap on the
+ *     GPU (other streams, other host threads) race on the array and must be serialised by
+ *     the caller.
+ */
+#define GDR_NOALLOC_MAX_HEADS 32
+GDR_API gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* desc,
+                                         const void* q, const void* k, const void* v,
+                                         const float* g, const float* beta, const float* theta,
+                                         const float* S0, void* o, float* S_T,
+                                         gdr_stream_t stream);
+
 /* The gdr_algo a descriptor would run with (GDR_ALGO_AUTO resolved), or -1 if the
  * descriptor is invalid.  No GPU work. */
 GDR_API int gdr_chunk_fwd_algo(const gdr_fwd_desc* desc);

@@ -4,6 +4,7 @@
 // status word below is a single symbol per loaded module.
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "gdr.h"
 #include "common.cuh"
@@ -101,6 +102,37 @@ static size_t split_ring_bytes(const gdr_fwd_desc* d) {
 static size_t split_workspace_bytes(const gdr_fwd_desc* d) {
     const size_t nh = (size_t)d->B * d->H;
     return split_ring_bytes(d) + (nh * tcf::RING + nh) * sizeof(unsigned int);
+}
+
+// ---- scratch for gdr_chunk_fwd_noalloc ---------------------------------------------------
+// The split kernel's ring and flags for at most NOALLOC_MAX_HEADS heads, as a file-scope
+// device array: every GPU that loads this library holds these bytes until the process exits.
+constexpr int NOALLOC_MAX_HEADS = GDR_NOALLOC_MAX_HEADS;
+constexpr size_t NOALLOC_BYTES =
+    (size_t)NOALLOC_MAX_HEADS * tcf::RING * tcf::SLOT_BYTES +
+    ((size_t)NOALLOC_MAX_HEADS * tcf::RING + NOALLOC_MAX_HEADS) * sizeof(unsigned int);
+static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_BYTES];
+
+// In host code g_noalloc_scratch names a host-side stand-in, not device memory; the device
+// address is looked up once per device (with that device current) and cached here.
+constexpr int NOALLOC_MAX_DEVICES = 64;
+static void* s_noalloc_ptr[NOALLOC_MAX_DEVICES] = {};
+static std::mutex s_noalloc_mu;
+
+static gdr_status noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return fail(GDR_ERR_UNSUPPORTED, "device index too large%s");
+    std::lock_guard<std::mutex> lock(s_noalloc_mu);
+    if (!s_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || ptr == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+        s_noalloc_ptr[dev] = ptr;
+    }
+    *out = s_noalloc_ptr[dev];
+    return GDR_OK;
 }
 
 static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
@@ -313,6 +345,46 @@ gdr_status gdr_query_device_status(gdr_stream_t stream) {
 int gdr_chunk_fwd_algo(const gdr_fwd_desc* desc) {
     if (check_fwd_desc(desc) != GDR_OK) return -1;
     return (int)resolve_algo(desc);
+}
+
+gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* d, const void* q, const void* k, const void* v,
+                                 const float* g, const float* beta, const float* theta, const float* S0,
+                                 void* o, float* S_T, gdr_stream_t stream) {
+    t_detail[0] = 0;
+    gdr_status s = check_fwd_desc(d);
+    if (s != GDR_OK) return s;
+    if (d->algo != GDR_ALGO_AUTO && d->algo != GDR_ALGO_TCGEN05_SPLIT)
+        return fail(GDR_ERR_INVALID_ARG, "gdr_chunk_fwd_noalloc runs the split tensor-core kernel: algo must be AUTO or TCGEN05_SPLIT%s");
+    if (!tc_supported(d))
+        return fail(GDR_ERR_UNSUPPORTED, "gdr_chunk_fwd_noalloc needs bf16 q/k/v and dk = dv = 128%s");
+    if ((long long)d->B * d->H > NOALLOC_MAX_HEADS) {
+        snprintf(t_detail, sizeof(t_detail),
+                 "gdr_chunk_fwd_noalloc: B*H = %lld exceeds the built-in scratch limit of %d heads; "
+                 "use gdr_chunk_fwd with a caller workspace", (long long)d->B * d->H, NOALLOC_MAX_HEADS);
+        return GDR_ERR_UNSUPPORTED;
+    }
+    if (d->B == 0 || d->H == 0) return GDR_OK;
+    if (d->T > 0) {
+        if (!q || !k || !v || !g || !beta || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta and o are required%s");
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) || !aligned16(o))
+            return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
+        if (d->rotation && !theta) return fail(GDR_ERR_INVALID_ARG, "theta is required with rotation%s");
+    }
+    if (!d->rotation && theta) return fail(GDR_ERR_INVALID_ARG, "theta must be NULL without rotation%s");
+    if ((theta && !aligned16(theta)) || (S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
+        return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
+    FwdParams p;
+    p.B = d->B; p.H = d->H; p.T = d->T; p.dv = d->dv;
+    p.gate_mode = (int)d->gate_mode;
+    p.scale = d->scale;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.theta = theta;
+    p.S0 = S0; p.o = o; p.S_T = S_T;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (d->T == 0) return S_T ? dispatch_tc_mode<0>(d, p, st, nullptr) : GDR_OK;
+    void* scratch = nullptr;
+    s = noalloc_scratch(&scratch);
+    if (s != GDR_OK) return s;
+    return dispatch_tc_mode<1>(d, p, st, scratch);
 }
 
 void gdr_debug_set_tc_fault(int skip_first_commit, unsigned long long wait_limit_ns) {

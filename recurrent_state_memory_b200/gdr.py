@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_query_device_status.argtypes = [vp]
         L.gdr_chunk_fwd_algo.restype = ctypes.c_int
         L.gdr_chunk_fwd_algo.argtypes = [ctypes.POINTER(FwdDesc)]
+        L.gdr_chunk_fwd_noalloc.restype = ctypes.c_int
+        L.gdr_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp, vp]
         L.gdr_debug_set_tc_fault.restype = None
         L.gdr_debug_set_tc_fault.argtypes = [ctypes.c_int, ctypes.c_ulonglong]
         if L.gdr_abi_version() != 1:
