@@ -79,11 +79,11 @@ static int device_sm_count() {
     return n;
 }
 
-// The split kernel pays off while the heads leave at least a third of the SMs for prep
-// workers and there is more than one chunk; it needs at least one worker.
+// The split kernel pays off while the heads leave most SMs to prep workers (each head's
+// chain needs about three workers to keep up) and there is more than one chunk.
 static bool split_fits(const gdr_fwd_desc* d, int sms) {
     const long long nh = (long long)d->B * d->H;
-    return nh >= 1 && 3 * nh <= 2LL * sms && d->T > 64;
+    return nh >= 1 && 4 * nh <= (long long)sms && d->T > 64;
 }
 
 // The algorithm a descriptor runs with: AUTO takes a tensor-core kernel when it supports
@@ -154,6 +154,66 @@ static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
     return GDR_OK;
 }
 
+// ---- tensor maps of the split kernel ---------------------------------------------------
+// cuTensorMapEncodeTiled is a driver call; it is looked up through the runtime so that the
+// library does not link libcuda itself.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static gdr_status encode_fn(EncodeTiledFn* out) {
+    static std::mutex mu;
+    static EncodeTiledFn fn = nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+        if (q != cudaDriverEntryPointSuccess || !ptr)
+            return fail(GDR_ERR_CUDA, "the driver has no cuTensorMapEncodeTiled%s");
+        fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    *out = fn;
+    return GDR_OK;
+}
+
+// A [B][T][H][inner] row-major tensor as the 4-D map {inner, H, T, B}; boxes cover `box_inner`
+// elements of one head for 64 consecutive tokens.  Out-of-range tokens read as zero and are
+// not written by stores.
+static gdr_status encode_bthd(EncodeTiledFn fn, CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                              size_t esize, const FwdParams& p, int inner, int box_inner, bool swizzle128) {
+    const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)p.H, (cuuint64_t)p.T, (cuuint64_t)p.B};
+    const cuuint64_t strides[3] = {(cuuint64_t)inner * esize, (cuuint64_t)p.H * inner * esize,
+                                   (cuuint64_t)p.T * p.H * inner * esize};
+    const cuuint32_t box[4] = {(cuuint32_t)box_inner, 1u, (cuuint32_t)tcf::C, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    CUresult r = fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(t_detail, sizeof(t_detail), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return GDR_ERR_CUDA;
+    }
+    return GDR_OK;
+}
+
+template <bool ROT, typename OT>
+static gdr_status encode_split_maps(const FwdParams& p, tcf::TmaMaps* tm) {
+    EncodeTiledFn fn = nullptr;
+    gdr_status s = encode_fn(&fn);
+    if (s != GDR_OK) return s;
+    const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const int D = tcf::D, NG = ROT ? tcf::D / 2 : tcf::D;
+    if ((s = encode_bthd(fn, &tm->q, p.q, bf, 2, p, D, D, false)) != GDR_OK) return s;
+    if ((s = encode_bthd(fn, &tm->k, p.k, bf, 2, p, D, D, false)) != GDR_OK) return s;
+    if ((s = encode_bthd(fn, &tm->g, p.g, f32, 4, p, NG, NG, false)) != GDR_OK) return s;
+    if (ROT && (s = encode_bthd(fn, &tm->th, p.theta, f32, 4, p, NG, NG, false)) != GDR_OK) return s;
+    if ((s = encode_bthd(fn, &tm->v, p.v, bf, 2, p, D, 64, true)) != GDR_OK) return s;
+    const bool ob = sizeof(OT) == 2;
+    return encode_bthd(fn, &tm->o, p.o, ob ? bf : f32, sizeof(OT), p, D, D, false);
+}
+
 template <int MODE, bool ROT, typename OT>
 static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
     auto kern = tcf::chunk_fwd_tc_kernel<MODE, ROT, OT>;
@@ -163,8 +223,10 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
     x.wait_limit_ns = s_wait_limit_ns;
     x.fault_skip_commit = s_fault_skip_commit;
     tcf::SplitArgs sa{nullptr, nullptr, nullptr};
+    tcf::TmaMaps tm;
+    memset(&tm, 0, sizeof(tm));
     if (MODE == 0) {
-        kern<<<p.B * p.H, tcf::NT, tcf::SMEM_BYTES, st>>>(p, x, sa);
+        kern<<<p.B * p.H, tcf::NT, tcf::SMEM_BYTES, st>>>(p, x, sa, tm);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
         return GDR_OK;
@@ -178,13 +240,15 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     const int grid = sms * (per_sm < 1 ? 1 : per_sm > 1 ? 1 : per_sm);
     if (per_sm < 1 || grid <= nh) return fail(GDR_ERR_UNSUPPORTED, "split kernel: B*H must be below the SM count%s");
+    gdr_status s = encode_split_maps<ROT, OT>(p, &tm);
+    if (s != GDR_OK) return s;
     const size_t nring = (size_t)nh * tcf::RING * tcf::SLOT_BYTES;
     sa.ring = static_cast<uint8_t*>(ws);
     sa.ready = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + nring);
     sa.consumed = sa.ready + (size_t)nh * tcf::RING;
     e = cudaMemsetAsync(sa.ready, 0, ((size_t)nh * tcf::RING + nh) * sizeof(unsigned int), st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split flags)");
-    void* args[] = {const_cast<FwdParams*>(&p), &x, &sa};
+    void* args[] = {const_cast<FwdParams*>(&p), &x, &sa, &tm};
     e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(tcf::NT), args,
                                     tcf::SMEM_BYTES, st);
     if (e != cudaSuccess) return cuda_fail(e, "cooperative launch(tcgen05 split kernel)");

@@ -38,6 +38,8 @@
 // B operand of the state update.
 #pragma once
 
+#include <cuda.h>   // CUtensorMap
+
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -77,12 +79,30 @@ constexpr uint32_t SL_KH = 16384;     // Khat K-major: 2 kblocks x 64 rows x 128
 constexpr uint32_t SL_W = 32768;      // Wm^T bf16 MN-major: 128 dk rows x 128 B
 constexpr uint32_t SL_PM = 49152;     // Pm K-major: 64 rows x 128 B
 constexpr uint32_t SL_TB = 57344;     // Tb K-major: 64 rows x 128 B
-constexpr uint32_t SL_V = 65536;      // V, MN-major: 2 groups x 64 tokens x 128 B
-constexpr uint32_t SL_VEC = 81920;    // beta, rho_ref, rho_C (VEC_FLOATS floats)
-constexpr uint32_t SLOT_BYTES = SL_VEC + VEC_FLOATS * 4;
-constexpr uint32_t SLOT_STRIDE = (SLOT_BYTES + 1023) & ~1023u;   // slot buffers in the chain CTA
+constexpr uint32_t SL_VEC = 65536;    // beta, rho_ref, rho_C (VEC_FLOATS floats)
+constexpr uint32_t SLOT_BYTES = SL_VEC + VEC_FLOATS * 4;        // bytes of one ring slot
+// The chain CTA's copy of a slot is followed by the chunk's V tile, which the chain loads
+// itself from the input (MN-major: 2 groups x 64 tokens x 128 B).
+constexpr uint32_t SL_V = (SLOT_BYTES + 1023) & ~1023u;
+constexpr uint32_t SLOT_STRIDE = SL_V + 16384;                  // slot buffers in the chain CTA
 constexpr int RING = 3;               // ring slots per head
-static_assert(2 * SLOT_STRIDE <= OFF_BAR, "chain slot buffers overlap the barriers");
+// Split chain CTAs stage each chunk's o here ([64 tokens][128] in the output type) and
+// bulk-store it row by row.
+constexpr uint32_t OFF_OSTG = 2 * SLOT_STRIDE;
+static_assert(2 * SLOT_STRIDE + 64 * 128 * 4 <= OFF_BAR, "chain slot buffers overlap the barriers");
+// Split-mode prep workers keep one set of tiles and stage the next task's raw inputs in the
+// second set's place: gates (and angles) in KQ[1], q in KH[1], k in W[1].
+constexpr uint32_t STG_A = OFF_KQ + 32768;   // [64][128] fp32 gates; rotation: [64][64] gates + [64][64] angles
+constexpr uint32_t STG_Q = OFF_KH + 16384;   // [64][128] bf16
+constexpr uint32_t STG_K = OFF_W + 16384;    // [64][128] bf16
+
+// 4-D tensor maps {inner dim, H, T, B} with boxes of 64 tokens (split mode only).
+// q, k: bf16 box {128,1,64,1}; g: fp32 box {128,...} ({64,...} with rotation); th: fp32
+// {64,...} (rotation); v: bf16 box {64,1,64,1}, 128-byte swizzle (the MN-major V tile);
+// o: output type, box {128,1,64,1}.
+struct TmaMaps {
+    CUtensorMap q, k, g, th, v, o;
+};
 
 struct SplitArgs {
     uint8_t* ring;            // [B*H][RING][SLOT_BYTES]
@@ -137,6 +157,21 @@ __device__ __forceinline__ void transpose8(float (&v)[8], int j) {
     }
 }
 
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// D (16x8, fp32) += A (16x8, tf32, row-major fragment) * B (8x8, tf32, column fragment),
+// one warp (mma.sync m16n8k8).
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 __device__ __forceinline__ uint4 pack8(const float* m8) {
     using tc::pack_bf16x2;
     return make_uint4(pack_bf16x2(m8[0], m8[1]), pack_bf16x2(m8[2], m8[3]),
@@ -149,7 +184,8 @@ __device__ __forceinline__ uint4 pack8(const float* m8) {
 // warps 0-7 compute chunks in chunk-major task order and whose warps 8-11 copy finished
 // operands into the ring.  The grid must be co-resident (cooperative launch).
 template <int MODE, bool ROT, typename OT>
-__global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtra x, SplitArgs sa) {
+__global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtra x, SplitArgs sa,
+                                                              const __grid_constant__ TmaMaps tm) {
     using namespace tc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -200,10 +236,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         mbar_init(bar_pmma, 1);
         mbar_init(bar_cmma, 1);
         for (int i = 0; i < 2; ++i) {
-            // split chain CTAs: one arrival (the loader's expect_tx) plus the copied bytes
+            // split chain CTAs: the loader's expect_tx arrival (plus the slot's and V's bytes)
             mbar_init(bar_full + i, (MODE == 1 && chain_cta) ? 1 : NPREP);
-            mbar_init(bar_empty + i, NT - NPREP);
-            mbar_init(bar_rho + i, NPREP);
+            // split workers: bar_empty[0] = tiles copied out (one issuing thread)
+            mbar_init(bar_empty + i, (MODE == 1 && !chain_cta) ? 1 : NT - NPREP);
+            // split workers: bar_rho[0] = staged inputs ready (one expect_tx arrival plus the
+            // bytes), bar_rho[1] = staging consumed (prep warps arrive)
+            mbar_init(bar_rho + i, (MODE == 1 && !chain_cta && i == 0) ? 1 : NPREP);
         }
         fence_mbar_init();
         *abort_p = 0;
@@ -283,12 +322,38 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         };
         const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
 
-        if (ntasks > 0) prefetch(task_bh(0), task_c(0));
+        if (MODE == 0 && ntasks > 0) prefetch(task_bh(0), task_c(0));
         for (int it = 0; it < ntasks; ++it) {
             const int c = task_c(it), bhx = task_bh(it);
             const int Lc = chunk_len(c);
-            const int bufi = it & 1;
-            float* vec = vecs(it);
+            const int bufi = (MODE == 0) ? (it & 1) : 0;      // split workers: single tile buffers
+            float* vec = vecs(bufi);
+            if (MODE == 1) {
+                // raw inputs of this task, staged by the copy-out warps
+                const bool ok = mbar_wait_bounded(bar_rho + 0, it & 1, x.wait_limit_ns);
+                if (!ok) atomicExch(abort_p, 1);
+                named_bar(1, NPREP);
+                if (*abort_p) break;
+#pragma unroll
+                for (int s_ = 0; s_ < 8; ++s_) {
+                    const int r = 8 * sg + s_;
+                    // rows past the chunk's end are not staged: they are identity tokens
+                    rk[s_] = make_uint2(0u, 0u);
+                    rq[s_] = make_uint2(0u, 0u);
+                    ra[s_] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (r >= Lc) continue;
+                    rk[s_] = *reinterpret_cast<const uint2*>(base + STG_K + (uint32_t)(r * D + 4 * dg) * 2u);
+                    rq[s_] = *reinterpret_cast<const uint2*>(base + STG_Q + (uint32_t)(r * D + 4 * dg) * 2u);
+                    if (!ROT) {
+                        ra[s_] = *reinterpret_cast<const float4*>(base + STG_A + (uint32_t)(r * D + 4 * dg) * 4u);
+                    } else {
+                        const float2 g2 = *reinterpret_cast<const float2*>(base + STG_A + (uint32_t)(r * 64 + 2 * dg) * 4u);
+                        const float2 t2 = *reinterpret_cast<const float2*>(base + STG_A + 16384u + (uint32_t)(r * 64 + 2 * dg) * 4u);
+                        ra[s_] = make_float4(g2.x, g2.y, t2.x, t2.y);
+                    }
+                }
+                mbar_arrive(bar_rho + 1);
+            }
             float* sbeta = vec;
             float* rho_ref = vec + 64;
             float* rho_C = vec + 64 + 256;
@@ -355,8 +420,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             named_bar(1, NPREP);
             // Buffers of task it - 2 must be released (by the chain, or by the copy-out warps)
             // before they are rewritten.
-            if (it >= 2) {
+            if (MODE == 0 && it >= 2) {
                 const bool ok = mbar_wait_bounded(bar_empty + bufi, ((it - 2) >> 1) & 1, x.wait_limit_ns);
+                if (!ok) atomicExch(abort_p, 1);
+            }
+            if (MODE == 1 && it >= 1) {     // the copy-out warps must have copied the previous tiles
+                const bool ok = mbar_wait_bounded(bar_empty + 0, (it - 1) & 1, x.wait_limit_ns);
                 if (!ok) atomicExch(abort_p, 1);
             }
             named_bar(1, NPREP);
@@ -467,7 +536,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             fence_proxy_async_smem();
             named_bar(1, NPREP);
             if (MODE == 0) mbar_arrive(bar_rho + bufi);
-            if (it + 1 < ntasks) prefetch(task_bh(it + 1), task_c(it + 1));
+            if (MODE == 0 && it + 1 < ntasks) prefetch(task_bh(it + 1), task_c(it + 1));
 
             // ---- MMA1: [Ktil ; Qtil] Khat^T -> TMEM ------------------------------------
             tc_fence_after();
@@ -532,38 +601,55 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             }
             named_bar(1, NPREP);
             // Off-diagonal blocks, by block distance: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ.
-            // 64 threads per 16x16 block, each owning a 1x4 strip (row rr, columns c4..c4+3).
+            // One warp per 16x16 block, on m16n8k8 tf32 tensor-core MMAs (the result is rounded
+            // to bf16 for the UT transform anyway): X = sum A_IK T_KJ, then T_IJ = -T_II X.
+            {
+                const int gid = lane >> 2, tig = lane & 3;
+                float* Xw = Xf + warp * XS;                   // this warp's 16 x 20 scratch
 #pragma unroll 1
-            for (int dist = 1; dist < 4; ++dist) {
-                const int nb = 4 - dist;
-                const int blk = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
-                const bool act = blk < nb;
-                const int J = blk, I = blk + dist;
-                if (act) {
-                    float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-                    const float* ap = Af + (16 * I + rr) * AS;
-                    const float* tp = Tf + 16 * J + c4;
-#pragma unroll 8
-                    for (int kk = 16 * J; kk < 16 * I; ++kk) {
-                        const float a = ap[kk];
-                        const float4 t4 = *reinterpret_cast<const float4*>(tp + kk * AS);
-                        x0 = fmaf(a, t4.x, x0); x1 = fmaf(a, t4.y, x1); x2 = fmaf(a, t4.z, x2); x3 = fmaf(a, t4.w, x3);
+                for (int dist = 1; dist < 4; ++dist) {
+                    if (warp < 4 - dist) {
+                        const int J = warp, I = warp + dist;
+                        float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+                        const float* ar0 = Af + (16 * I + gid) * AS;
+                        const float* ar1 = ar0 + 8 * AS;
+#pragma unroll 2
+                        for (int kb8 = 16 * J; kb8 < 16 * I; kb8 += 8) {
+                            const uint32_t a[4] = {to_tf32(ar0[kb8 + tig]), to_tf32(ar1[kb8 + tig]),
+                                                   to_tf32(ar0[kb8 + tig + 4]), to_tf32(ar1[kb8 + tig + 4])};
+                            const float* tr0 = Tf + (kb8 + tig) * AS + 16 * J + gid;
+                            const float* tr1 = tr0 + 4 * AS;
+                            const uint32_t b0[2] = {to_tf32(tr0[0]), to_tf32(tr1[0])};
+                            const uint32_t b1[2] = {to_tf32(tr0[8]), to_tf32(tr1[8])};
+                            mma_tf32_16x8x8(x0, a, b0);
+                            mma_tf32_16x8x8(x1, a, b1);
+                        }
+                        Xw[gid * 20 + 2 * tig] = x0[0];       Xw[gid * 20 + 2 * tig + 1] = x0[1];
+                        Xw[(gid + 8) * 20 + 2 * tig] = x0[2]; Xw[(gid + 8) * 20 + 2 * tig + 1] = x0[3];
+                        Xw[gid * 20 + 8 + 2 * tig] = x1[0];       Xw[gid * 20 + 9 + 2 * tig] = x1[1];
+                        Xw[(gid + 8) * 20 + 8 + 2 * tig] = x1[2]; Xw[(gid + 8) * 20 + 9 + 2 * tig] = x1[3];
+                        __syncwarp();
+                        float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+                        const float* dr0 = Tf + (16 * I + gid) * AS + 16 * I;
+                        const float* dr1 = dr0 + 8 * AS;
+#pragma unroll
+                        for (int kb8 = 0; kb8 < 16; kb8 += 8) {
+                            const uint32_t a[4] = {to_tf32(dr0[kb8 + tig]), to_tf32(dr1[kb8 + tig]),
+                                                   to_tf32(dr0[kb8 + tig + 4]), to_tf32(dr1[kb8 + tig + 4])};
+                            const float* xr0 = Xw + (kb8 + tig) * 20 + gid;
+                            const float* xr1 = xr0 + 4 * 20;
+                            const uint32_t b0[2] = {to_tf32(xr0[0]), to_tf32(xr1[0])};
+                            const uint32_t b1[2] = {to_tf32(xr0[8]), to_tf32(xr1[8])};
+                            mma_tf32_16x8x8(y0, a, b0);
+                            mma_tf32_16x8x8(y1, a, b1);
+                        }
+                        float* t0 = Tf + (16 * I + gid) * AS + 16 * J;
+                        float* t1 = t0 + 8 * AS;
+                        t0[2 * tig] = -y0[0]; t0[2 * tig + 1] = -y0[1]; t1[2 * tig] = -y0[2]; t1[2 * tig + 1] = -y0[3];
+                        t0[8 + 2 * tig] = -y1[0]; t0[9 + 2 * tig] = -y1[1]; t1[8 + 2 * tig] = -y1[2]; t1[9 + 2 * tig] = -y1[3];
                     }
-                    *reinterpret_cast<float4*>(Xf + blk * XS + rr * 20 + c4) = make_float4(x0, x1, x2, x3);
+                    named_bar(1, NPREP);
                 }
-                named_bar(1, NPREP);
-                if (act) {
-                    float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
-                    const float* dp = Tf + (16 * I + rr) * AS + 16 * I;
-#pragma unroll 4
-                    for (int s_ = 0; s_ <= rr; ++s_) {
-                        const float d = dp[s_];
-                        const float4 x4 = *reinterpret_cast<const float4*>(Xf + blk * XS + s_ * 20 + c4);
-                        y0 = fmaf(d, x4.x, y0); y1 = fmaf(d, x4.y, y1); y2 = fmaf(d, x4.z, y2); y3 = fmaf(d, x4.w, y3);
-                    }
-                    *reinterpret_cast<float4*>(Tf + (16 * I + rr) * AS + 16 * J + c4) = make_float4(-y0, -y1, -y2, -y3);
-                }
-                named_bar(1, NPREP);
             }
             // Tb = Tm diag(beta), zero above the block diagonal, -> bf16 K-major [r][i].
             // (Split mode keeps two Tb tiles in the unused V area, one per buffer.)
@@ -668,6 +754,27 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         auto o_epilogue = [&](int c) {
             const int Lc = chunk_len(c);
             const uint32_t col = COL_O + (c & 1) * 64;
+            if (MODE == 1) {
+                // stage o as [token][value] in shared memory, then one thread bulk-stores rows
+                if (row == 0) bulk_wait_read_all();            // the previous chunk's stores have read it
+                cbar();
+                OT* stg = reinterpret_cast<OT*>(base + OFF_OSTG);
+#pragma unroll 1
+                for (int g = 0; g < 2; ++g) {
+                    float vals[32];
+                    tmem_ld32(tq + col + g * 32, vals);
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) st_from_f32(stg + (g * 32 + u) * D + row, vals[u]);
+                }
+                fence_proxy_async_smem();
+                cbar();
+                if (row == 0) {
+                    tma_store_4d(&tm.o, 0, bh % p.H, c * C, bh / p.H, sb + OFF_OSTG);   // rows past T clipped
+                    bulk_commit();
+                }
+                (void)Lc;
+                return;
+            }
             const int j8 = lane & 7, grp = lane >> 3;
             OT* obase = o + tok(c, 0) * D + quad * 32 + grp * 8;
             const size_t tstride = (size_t)p.H * D;
@@ -824,6 +931,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             mbar_arrive(bar_empty + bufi);
             if (last) o_epilogue(c);
         }
+        if (MODE == 1 && row == 0) bulk_wait_all();     // o stores complete before the CTA exits
     }
 
     if (MODE == 1 && nchunks > 0 && chain_cta && warp == 0) {
@@ -839,11 +947,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                 if (ok) {
                     fence_proxy_async_global();
                     const uint8_t* src = sa.ring + ((size_t)bh * RING + slot) * SLOT_BYTES;
-                    mbar_arrive_expect_tx(bar_full + bufi, SLOT_BYTES);
+                    mbar_arrive_expect_tx(bar_full + bufi, SLOT_BYTES + 16384u);
                     for (uint32_t off = 0; off < SLOT_BYTES; off += 16384u) {
                         const uint32_t n = SLOT_BYTES - off < 16384u ? SLOT_BYTES - off : 16384u;
                         bulk_g2s(sb + slot_base(c) + off, src + off, n, bar_full + bufi);
                     }
+                    // V of this chunk, two 64-column boxes straight into the MN-major layout
+                    const int bb = bh / p.H, hh = bh % p.H;
+                    tma_load_4d(sb + slot_base(c) + SL_V, &tm.v, 0, hh, c * C, bb, bar_full + bufi);
+                    tma_load_4d(sb + slot_base(c) + SL_V + 8192u, &tm.v, 64, hh, c * C, bb, bar_full + bufi);
                     // the ring slot may be reused once its bytes have landed here
                     ok = mbar_wait_bounded(bar_full + bufi, (c >> 1) & 1, x.wait_limit_ns);
                     if (ok) st_release_gpu(sa.consumed + bh, (unsigned)(c + 1));
@@ -854,49 +966,50 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         }
     }
     if (MODE == 1 && nchunks > 0 && !chain_cta && tid >= NPREP) {
-        // ============ split mode: copy-out warps of a prep worker ==============================
-        const int ct = tid - NPREP;
-        const int W = (int)gridDim.x - NH, wk = (int)blockIdx.x - NH;
-        const int ntasks = (NH * nchunks - wk + W - 1) / W;
-        auto cbar = [&]() { named_bar(2, NT - NPREP); };
-        for (int it = 0; it < ntasks; ++it) {
-            const int bufi = it & 1;
-            const int task = wk + it * W, c = task / NH, bhx = task % NH, slot = c % RING;
-            const int Lc = chunk_len(c);
-            bool ok = mbar_wait_bounded(bar_full + bufi, (it >> 1) & 1, x.wait_limit_ns);
-            // the chain must have copied chunk c - RING out of this slot
-            if (ok && ct == 0 && c >= RING)
-                ok = spin_until_ge(sa.consumed + bhx, (unsigned)(c - RING + 1), x.wait_limit_ns);
-            if (!ok) atomicExch(abort_c, 1);
-            cbar();
-            if (*abort_c) break;
-            uint8_t* dst = sa.ring + ((size_t)bhx * RING + slot) * SLOT_BYTES;
-            // shared-memory tiles of this task -> ring slot (16-byte pieces)
-            auto copy16 = [&](uint32_t src_off, uint32_t dst_off, uint32_t bytes) {
-                for (uint32_t o16 = (uint32_t)ct * 16u; o16 < bytes; o16 += (NT - NPREP) * 16u)
-                    *reinterpret_cast<uint4*>(dst + dst_off + o16) = *reinterpret_cast<const uint4*>(base + src_off + o16);
+        // ============ split mode: transfer thread of a prep worker =============================
+        // One thread stages each task's raw inputs with bulk copies (one per token row) for the
+        // prep warps, then bulk-stores the finished tiles into the ring slot and publishes it.
+        if (tid == NPREP) {
+            const int W = (int)gridDim.x - NH, wk = (int)blockIdx.x - NH;
+            const int ntasks = (NH * nchunks - wk + W - 1) / W;
+            auto stage_task = [&](int itx) {
+                const int task = wk + itx * W, c = task / NH, bhx = task % NH;
+                const int bb = bhx / p.H, hh = bhx % p.H;
+                // tokens past the sequence end arrive as zeros; 64 KB in every case
+                mbar_arrive_expect_tx(bar_rho + 0, 65536u);
+                tma_load_4d(sb + STG_Q, &tm.q, 0, hh, c * C, bb, bar_rho + 0);
+                tma_load_4d(sb + STG_K, &tm.k, 0, hh, c * C, bb, bar_rho + 0);
+                tma_load_4d(sb + STG_A, &tm.g, 0, hh, c * C, bb, bar_rho + 0);
+                if (ROT) tma_load_4d(sb + STG_A + 16384u, &tm.th, 0, hh, c * C, bb, bar_rho + 0);
             };
-            copy16(OFF_KQ + bufi * 32768 + 8192, SL_Q, 8192);
-            copy16(OFF_KQ + bufi * 32768 + 16384 + 8192, SL_Q + 8192, 8192);
-            copy16(OFF_KH + bufi * 16384, SL_KH, 16384);
-            copy16(OFF_W + bufi * 16384, SL_W, 16384);
-            copy16(OFF_PM + bufi * 8192, SL_PM, 8192);
-            copy16(OFF_V + bufi * 8192, SL_TB, 8192);
-            copy16(OFF_VEC + bufi * VEC_FLOATS * 4, SL_VEC, VEC_FLOATS * 4);
-            // the shared buffers may be refilled by the prep warps now
-            mbar_arrive(bar_empty + bufi);
-            // V of this chunk straight from the input into the slot's MN-major layout
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int id = ct * 8 + j;
-                const int i = id >> 4, c16 = id & 15;
-                uint4 val = make_uint4(0u, 0u, 0u, 0u);
-                if (i < Lc) val = __ldg(reinterpret_cast<const uint4*>(v + tokh(bhx, c, i) * D + c16 * 8));
-                *reinterpret_cast<uint4*>(dst + SL_V + (uint32_t)(c16 >> 3) * 8192u + sw128_off(i, c16 & 7)) = val;
+            if (ntasks > 0) stage_task(0);
+            for (int it = 0; it < ntasks; ++it) {
+                const int task = wk + it * W, c = task / NH, bhx = task % NH, slot = c % RING;
+                bool ok = true;
+                if (it + 1 < ntasks) {
+                    // once the prep warps have read this task's staging, stage the next task
+                    ok = mbar_wait_bounded(bar_rho + 1, it & 1, x.wait_limit_ns);
+                    if (ok) stage_task(it + 1);
+                }
+                if (ok) ok = mbar_wait_bounded(bar_full + 0, it & 1, x.wait_limit_ns);
+                // the chain must have copied chunk c - RING out of this slot
+                if (ok && c >= RING) ok = spin_until_ge(sa.consumed + bhx, (unsigned)(c - RING + 1), x.wait_limit_ns);
+                if (!ok) { atomicExch(abort_c, 1); break; }
+                uint8_t* dst = sa.ring + ((size_t)bhx * RING + slot) * SLOT_BYTES;
+                bulk_s2g(dst + SL_Q, sb + OFF_KQ + 8192, 8192);
+                bulk_s2g(dst + SL_Q + 8192, sb + OFF_KQ + 16384 + 8192, 8192);
+                bulk_s2g(dst + SL_KH, sb + OFF_KH, 16384);
+                bulk_s2g(dst + SL_W, sb + OFF_W, 16384);
+                bulk_s2g(dst + SL_PM, sb + OFF_PM, 8192);
+                bulk_s2g(dst + SL_TB, sb + OFF_V, 8192);
+                bulk_s2g(dst + SL_VEC, sb + OFF_VEC, VEC_FLOATS * 4);
+                bulk_commit();
+                bulk_wait_read_all();
+                mbar_arrive(bar_empty + 0);          // the tiles may be rewritten now
+                bulk_wait_all();
+                fence_proxy_async_global();
+                st_release_gpu(sa.ready + (size_t)bhx * RING + slot, (unsigned)(c + 1));
             }
-            __threadfence();
-            cbar();
-            if (ct == 0) st_release_gpu(sa.ready + (size_t)bhx * RING + slot, (unsigned)(c + 1));
         }
     }
 
