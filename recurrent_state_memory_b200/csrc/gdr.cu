@@ -217,7 +217,9 @@ static gdr_status encode_split_maps(const FwdParams& p, tcf::TmaMaps* tm) {
 template <int MODE, bool ROT, typename OT>
 static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
     auto kern = tcf::chunk_fwd_tc_kernel<MODE, ROT, OT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::SMEM_BYTES);
+    constexpr int nt = tcf::nthreads<MODE>();
+    constexpr uint32_t smem = tcf::smem_bytes<MODE>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tcgen05 chunk kernel)");
     tcf::TcExtra x;
     x.wait_limit_ns = s_wait_limit_ns;
@@ -226,7 +228,7 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
     tcf::TmaMaps tm;
     memset(&tm, 0, sizeof(tm));
     if (MODE == 0) {
-        kern<<<p.B * p.H, tcf::NT, tcf::SMEM_BYTES, st>>>(p, x, sa, tm);
+        kern<<<p.B * p.H, nt, smem, st>>>(p, x, sa, tm);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
         return GDR_OK;
@@ -236,7 +238,7 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
     const int nh = p.B * p.H;
     const int sms = device_sm_count();
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, tcf::NT, tcf::SMEM_BYTES);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     const int grid = sms * (per_sm < 1 ? 1 : per_sm > 1 ? 1 : per_sm);
     if (per_sm < 1 || grid <= nh) return fail(GDR_ERR_UNSUPPORTED, "split kernel: B*H must be below the SM count%s");
@@ -249,8 +251,7 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
     e = cudaMemsetAsync(sa.ready, 0, ((size_t)nh * tcf::RING + nh) * sizeof(unsigned int), st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split flags)");
     void* args[] = {const_cast<FwdParams*>(&p), &x, &sa, &tm};
-    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(tcf::NT), args,
-                                    tcf::SMEM_BYTES, st);
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(nt), args, smem, st);
     if (e != cudaSuccess) return cuda_fail(e, "cooperative launch(tcgen05 split kernel)");
     return GDR_OK;
 }

@@ -49,7 +49,8 @@ namespace tcf {
 constexpr int C = 64;
 constexpr int D = 128;           // dk = dv
 constexpr int NT = 384;
-constexpr int NPREP = 256;       // threads of the prep group
+constexpr int NPREP = 256;       // threads of a prep group
+constexpr int CHAIN_THREADS = 128;   // threads of the chain group (one per TMEM lane)
 constexpr uint32_t COL_S = 0, COL_SB = 128, COL_O = 192, COL_E = 320, COL_AW = 448;
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -63,14 +64,11 @@ constexpr uint32_t OFF_TB = OFF_V + 16384;           // Tb K-major: 64 rows x 12
 constexpr int AS = 68;                               // row stride (floats) of the fp32 solve matrices
 constexpr uint32_t OFF_AF = OFF_TB + 8192;           // fp32 A [64][68]
 constexpr uint32_t OFF_TF = OFF_AF + 64 * AS * 4;    // fp32 Tm [64][68]
-constexpr int XS = 16 * 20;                          // one 16x16 scratch block, rows of 20 floats
-constexpr uint32_t OFF_XF = OFF_TF + 64 * AS * 4;    // fp32 scratch [3][16][20]
-constexpr uint32_t OFF_QT = OFF_XF + 3 * XS * 4;     // segment products [8 segments][32 dim groups][8]
+constexpr uint32_t OFF_QT = OFF_TF + 64 * AS * 4;    // segment products [8 segments][32 dim groups][8]
 constexpr uint32_t VEC_FLOATS = 64 + 4 * 128;        // beta[64], rho_ref[2][128], rho_C[2][128]
 constexpr uint32_t OFF_VEC = OFF_QT + 8 * 32 * 8 * 4;   // x2
 constexpr uint32_t OFF_BAR = (OFF_VEC + 2 * VEC_FLOATS * 4 + 63) & ~63u;
-constexpr uint32_t SMEM_USED = OFF_BAR + 128;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // slack for 1024-byte alignment
+constexpr uint32_t BAR_BYTES = 256;                  // mbarriers, TMEM address, flags
 
 // Split mode: a per-head ring in global memory carries each chunk's operands from the prep
 // workers to the chain CTA.  Slot layout (bytes), identical to the chain's shared-memory copy:
@@ -85,16 +83,32 @@ constexpr uint32_t SLOT_BYTES = SL_VEC + VEC_FLOATS * 4;        // bytes of one 
 // itself from the input (MN-major: 2 groups x 64 tokens x 128 B).
 constexpr uint32_t SL_V = (SLOT_BYTES + 1023) & ~1023u;
 constexpr uint32_t SLOT_STRIDE = SL_V + 16384;                  // slot buffers in the chain CTA
-constexpr int RING = 3;               // ring slots per head
+constexpr int RING = 4;               // ring slots per head
 // Split chain CTAs stage each chunk's o here ([64 tokens][128] in the output type) and
-// bulk-store it row by row.
+// store it with one tensor-map tile store.
 constexpr uint32_t OFF_OSTG = 2 * SLOT_STRIDE;
-static_assert(2 * SLOT_STRIDE + 64 * 128 * 4 <= OFF_BAR, "chain slot buffers overlap the barriers");
-// Split-mode prep workers keep one set of tiles and stage the next task's raw inputs in the
-// second set's place: gates (and angles) in KQ[1], q in KH[1], k in W[1].
-constexpr uint32_t STG_A = OFF_KQ + 32768;   // [64][128] fp32 gates; rotation: [64][64] gates + [64][64] angles
-constexpr uint32_t STG_Q = OFF_KH + 16384;   // [64][128] bf16
-constexpr uint32_t STG_K = OFF_W + 16384;    // [64][128] bf16
+// Split-mode prep workers run two independent groups of 8 warps, each with its own tiles
+// (bytes from the group's base, group g at g * G_STRIDE).  A group stages the raw inputs of
+// its next task into tiles that the current task no longer needs: q into G_KH (free after
+// MMA1), the gates (and angles) into G_AF..G_TF (free after the solve), k into G_TB..G_QT
+// (free after the Wm MMA).
+constexpr uint32_t G_KQ = 0;         // [Ktil ; Qtil] K-major: 2 kblocks x 128 rows x 128 B
+constexpr uint32_t G_KH = 32768;     // Khat K-major: 2 kblocks x 64 rows x 128 B
+constexpr uint32_t G_TB = 49152;     // Tb K-major: 64 rows x 128 B
+constexpr uint32_t G_QT = 57344;     // segment products [8][32][8]
+constexpr uint32_t G_AF = 65536;     // fp32 A [64][68]
+constexpr uint32_t G_TF = G_AF + 64 * AS * 4;   // fp32 Tm [64][68]
+constexpr uint32_t G_VEC = G_TF + 64 * AS * 4;  // beta, rho_ref, rho_C
+constexpr uint32_t G_STRIDE = (G_VEC + VEC_FLOATS * 4 + 1023) & ~1023u;
+constexpr int NT_SPLIT = 2 * NPREP + 64;        // two prep groups and one publishing warp each
+constexpr uint32_t OFF_BAR_SPLIT = 2 * G_STRIDE;
+static_assert(2 * SLOT_STRIDE + 64 * 128 * 4 <= OFF_BAR_SPLIT, "chain slot buffers overlap the barriers");
+static_assert(G_TF + 64 * AS * 4 >= G_AF + 32768, "gate staging does not fit in A and Tm");
+
+template <int MODE> __host__ __device__ constexpr int nthreads() { return MODE == 0 ? NT : NT_SPLIT; }
+template <int MODE> __host__ __device__ constexpr uint32_t off_bar() { return MODE == 0 ? OFF_BAR : OFF_BAR_SPLIT; }
+// dynamic shared memory, with slack for the 1024-byte alignment of the base
+template <int MODE> __host__ __device__ constexpr uint32_t smem_bytes() { return off_bar<MODE>() + BAR_BYTES + 1024; }
 
 // 4-D tensor maps {inner dim, H, T, B} with boxes of 64 tokens (split mode only).
 // q, k: bf16 box {128,1,64,1}; g: fp32 box {128,...} ({64,...} with rotation); th: fp32
@@ -157,10 +171,11 @@ __device__ __forceinline__ void transpose8(float (&v)[8], int j) {
     }
 }
 
+// fp32 -> tf32 bits, rounded to nearest with ties away from zero, with two integer
+// operations (the conversion instruction issues at a fraction of the ALU rate).  Finite
+// inputs only: a NaN payload may round into another encoding.
 __device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
 }
 
 // D (16x8, fp32) += A (16x8, tf32, row-major fragment) * B (8x8, tf32, column fragment),
@@ -184,26 +199,25 @@ __device__ __forceinline__ uint4 pack8(const float* m8) {
 // warps 0-7 compute chunks in chunk-major task order and whose warps 8-11 copy finished
 // operands into the ring.  The grid must be co-resident (cooperative launch).
 template <int MODE, bool ROT, typename OT>
-__global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtra x, SplitArgs sa,
+__global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdParams p, TcExtra x, SplitArgs sa,
                                                               const __grid_constant__ TmaMaps tm) {
     using namespace tc;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
     const uint32_t sb = (raw_u32 + 1023u) & ~1023u;          // shared-window base address
     uint8_t* base = smem_raw + (sb - raw_u32);               // generic pointer to the same byte
-    float* Af = reinterpret_cast<float*>(base + OFF_AF);
-    float* Tf = reinterpret_cast<float*>(base + OFF_TF);
-    float* Xf = reinterpret_cast<float*>(base + OFF_XF);
-    float* QT = reinterpret_cast<float*>(base + OFF_QT);
-    uint64_t* bar_pmma = reinterpret_cast<uint64_t*>(base + OFF_BAR);
-    uint64_t* bar_cmma = bar_pmma + 1;
-    uint64_t* bar_full = bar_pmma + 2;       // [2] prep -> chain: tiles of a chunk ready
-    uint64_t* bar_empty = bar_pmma + 4;      // [2] chain -> prep: buffers of a chunk free
-    uint64_t* bar_rho = bar_pmma + 6;        // [2] prep -> chain: decay vectors of a chunk ready
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_BAR + 64);
-    int* abort_p = reinterpret_cast<int*>(base + OFF_BAR + 68);
-    int* abort_c = reinterpret_cast<int*>(base + OFF_BAR + 72);
-    int* range_flag = reinterpret_cast<int*>(base + OFF_BAR + 76);
+    uint8_t* bar_base = base + off_bar<MODE>();
+    uint64_t* bar_pmma = reinterpret_cast<uint64_t*>(bar_base);   // [2] prep MMAs done (per group)
+    uint64_t* bar_cmma = bar_pmma + 2;       // chain MMAs done
+    uint64_t* bar_full = bar_pmma + 3;       // [2] prep -> chain: tiles of a chunk ready;
+                                             //     split workers: group g's task done
+    uint64_t* bar_empty = bar_pmma + 5;      // [2] chain -> prep: buffers of a chunk free
+    uint64_t* bar_rho = bar_pmma + 7;        // [2] prep -> chain: decay vectors of a chunk ready;
+                                             //     split workers: group g's staged inputs landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_base + 96);
+    int* abort_p = reinterpret_cast<int*>(bar_base + 100);
+    int* abort_c = reinterpret_cast<int*>(bar_base + 104);
+    int* range_flag = reinterpret_cast<int*>(bar_base + 108);
     auto vecs = [&](int c) -> float* { return reinterpret_cast<float*>(base + OFF_VEC) + (c & 1) * VEC_FLOATS; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -233,16 +247,14 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(bar_pmma, 1);
         mbar_init(bar_cmma, 1);
         for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_pmma + i, 1);
             // split chain CTAs: the loader's expect_tx arrival (plus the slot's and V's bytes)
             mbar_init(bar_full + i, (MODE == 1 && chain_cta) ? 1 : NPREP);
-            // split workers: bar_empty[0] = tiles copied out (one issuing thread)
-            mbar_init(bar_empty + i, (MODE == 1 && !chain_cta) ? 1 : NT - NPREP);
-            // split workers: bar_rho[0] = staged inputs ready (one expect_tx arrival plus the
-            // bytes), bar_rho[1] = staging consumed (prep warps arrive)
-            mbar_init(bar_rho + i, (MODE == 1 && !chain_cta && i == 0) ? 1 : NPREP);
+            mbar_init(bar_empty + i, CHAIN_THREADS);
+            // split workers: one expect_tx arrival plus the staged bytes
+            mbar_init(bar_rho + i, (MODE == 1) ? 1 : NPREP);
         }
         fence_mbar_init();
         *abort_p = 0;
@@ -255,12 +267,25 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
     const uint32_t tbase = *tmem_slot;
     const uint32_t tq = tbase + ((uint32_t)(quad * 32) << 16);   // this warp's lane quadrant
 
-    if (nchunks > 0 && tid < NPREP && (MODE == 0 || !chain_cta)) {
+    if (nchunks > 0 && (MODE == 0 ? tid < NPREP : (!chain_cta && tid < 2 * NPREP))) {
         // =========================== prep group ===================================
         // Tasks: fused mode, chunk it of this CTA's head; split mode, task wk + it * W in
-        // chunk-major order (chunk = task / NH, head = task % NH).
-        const int W = (MODE == 0) ? 1 : (int)gridDim.x - NH;
-        const int wk = (MODE == 0) ? 0 : (int)blockIdx.x - NH;
+        // chunk-major order (chunk = task / NH, head = task % NH), where the workers' groups
+        // count as 2 (gridDim.x - NH) independent workers.
+        const int grp = (MODE == 1) ? (int)threadIdx.x / NPREP : 0;
+        const int tid = (int)threadIdx.x - grp * NPREP;      // thread within the group
+        const int warp = tid >> 5;
+        const int gbar = 1 + 2 * grp;                        // the group's named barrier
+        uint8_t* gb = base + (uint32_t)grp * G_STRIDE;      // split: the group's tiles
+        const uint32_t gsb = sb + (uint32_t)grp * G_STRIDE;
+        uint64_t* g_pmma = bar_pmma + grp;
+        uint64_t* g_stage = bar_rho + grp;
+        const uint32_t col_aw = (MODE == 0) ? COL_AW : (uint32_t)grp * 64u;
+        float* Af = reinterpret_cast<float*>(MODE == 0 ? base + OFF_AF : gb + G_AF);
+        float* Tf = reinterpret_cast<float*>(MODE == 0 ? base + OFF_TF : gb + G_TF);
+        float* QT = reinterpret_cast<float*>(MODE == 0 ? base + OFF_QT : gb + G_QT);
+        const int W = (MODE == 0) ? 1 : 2 * ((int)gridDim.x - NH);
+        const int wk = (MODE == 0) ? 0 : 2 * ((int)blockIdx.x - NH) + grp;
         const int ntasks = (MODE == 0) ? nchunks : (NH * nchunks - wk + W - 1) / W;
         auto task_bh = [&](int it) -> int { return MODE == 0 ? bh : (wk + it * W) % NH; };
         auto task_c = [&](int it) -> int { return MODE == 0 ? it : (wk + it * W) / NH; };
@@ -307,58 +332,85 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             }
         };
         auto mma_wait = [&]() -> bool {
-            const bool ok = mbar_wait_bounded(bar_pmma, mma_phase, x.wait_limit_ns);
+            const bool ok = mbar_wait_bounded(g_pmma, mma_phase, x.wait_limit_ns);
             mma_phase ^= 1u;
             if (!ok) atomicExch(abort_p, 1);
             tc_fence_after();
-            named_bar(1, NPREP);
+            named_bar(gbar, NPREP);
             return *abort_p == 0;
         };
         auto publish = [&]() {
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar(1, NPREP);
+            named_bar(gbar, NPREP);
             tc_fence_after();
+        };
+        // split: stage part `part` of task itx's raw inputs (tokens past the sequence end
+        // arrive as zeros); part 0 also arms the barrier for all 64 KB
+        int staged = 0, landed = 0;     // split: tasks whose staging was issued / has landed
+        auto stage_part = [&](int itx, int part) {
+            const int c2 = task_c(itx), b2 = task_bh(itx);
+            const int bb = b2 / p.H, hh = b2 % p.H;
+            if (part == 0) {
+                staged = itx + 1;
+                mbar_arrive_expect_tx(g_stage, 65536u);
+                tma_load_4d(gsb + G_KH, &tm.q, 0, hh, c2 * C, bb, g_stage);
+            } else if (part == 1) {
+                tma_load_4d(gsb + G_AF, &tm.g, 0, hh, c2 * C, bb, g_stage);
+                if (ROT) tma_load_4d(gsb + G_AF + 16384u, &tm.th, 0, hh, c2 * C, bb, g_stage);
+            } else {
+                tma_load_4d(gsb + G_TB, &tm.k, 0, hh, c2 * C, bb, g_stage);
+            }
         };
         const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
 
         if (MODE == 0 && ntasks > 0) prefetch(task_bh(0), task_c(0));
+        if (MODE == 1 && tid == 0 && ntasks > 0) {
+            stage_part(0, 0);
+            stage_part(0, 1);
+            stage_part(0, 2);
+        }
         for (int it = 0; it < ntasks; ++it) {
             const int c = task_c(it), bhx = task_bh(it);
             const int Lc = chunk_len(c);
             const int bufi = (MODE == 0) ? (it & 1) : 0;      // split workers: single tile buffers
-            float* vec = vecs(bufi);
+            float* vec = (MODE == 0) ? vecs(bufi) : reinterpret_cast<float*>(gb + G_VEC);
+            // split mode: this task's ring slot, written directly by the prep warps
+            uint8_t* ring = (MODE == 1) ? sa.ring + ((size_t)bhx * RING + c % RING) * SLOT_BYTES : nullptr;
+            float* rvec = reinterpret_cast<float*>(ring + SL_VEC);
+            // beta of this task, consumed after pass 1
+            float beta_r = 0.f;
+            if (tid < 64 && tid < Lc) beta_r = __ldg(p.beta + tokh(bhx, c, tid));
             if (MODE == 1) {
-                // raw inputs of this task, staged by the copy-out warps
-                const bool ok = mbar_wait_bounded(bar_rho + 0, it & 1, x.wait_limit_ns);
+                // raw inputs of this task, staged by the transfer thread (tokens past the
+                // sequence end arrive as zeros)
+                const bool ok = mbar_wait_bounded(g_stage, it & 1, x.wait_limit_ns);
                 if (!ok) atomicExch(abort_p, 1);
-                named_bar(1, NPREP);
+                landed = it + 1;
+                named_bar(gbar, NPREP);
                 if (*abort_p) break;
 #pragma unroll
                 for (int s_ = 0; s_ < 8; ++s_) {
                     const int r = 8 * sg + s_;
-                    // rows past the chunk's end are not staged: they are identity tokens
-                    rk[s_] = make_uint2(0u, 0u);
-                    rq[s_] = make_uint2(0u, 0u);
-                    ra[s_] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (r >= Lc) continue;
-                    rk[s_] = *reinterpret_cast<const uint2*>(base + STG_K + (uint32_t)(r * D + 4 * dg) * 2u);
-                    rq[s_] = *reinterpret_cast<const uint2*>(base + STG_Q + (uint32_t)(r * D + 4 * dg) * 2u);
+                    rk[s_] = *reinterpret_cast<const uint2*>(gb + G_TB + (uint32_t)(r * D + 4 * dg) * 2u);
+                    rq[s_] = *reinterpret_cast<const uint2*>(gb + G_KH + (uint32_t)(r * D + 4 * dg) * 2u);
                     if (!ROT) {
-                        ra[s_] = *reinterpret_cast<const float4*>(base + STG_A + (uint32_t)(r * D + 4 * dg) * 4u);
+                        ra[s_] = *reinterpret_cast<const float4*>(gb + G_AF + (uint32_t)(r * D + 4 * dg) * 4u);
                     } else {
-                        const float2 g2 = *reinterpret_cast<const float2*>(base + STG_A + (uint32_t)(r * 64 + 2 * dg) * 4u);
-                        const float2 t2 = *reinterpret_cast<const float2*>(base + STG_A + 16384u + (uint32_t)(r * 64 + 2 * dg) * 4u);
+                        const float2 g2 = *reinterpret_cast<const float2*>(gb + G_AF + (uint32_t)(r * 64 + 2 * dg) * 4u);
+                        const float2 t2 = *reinterpret_cast<const float2*>(gb + G_AF + 16384u + (uint32_t)(r * 64 + 2 * dg) * 4u);
                         ra[s_] = make_float4(g2.x, g2.y, t2.x, t2.y);
                     }
                 }
-                mbar_arrive(bar_rho + 1);
+                named_bar(gbar, NPREP);      // pass 1 rewrites the k staging area (G_QT)
             }
             float* sbeta = vec;
             float* rho_ref = vec + 64;
             float* rho_C = vec + 64 + 256;
-            uint8_t* KQ = base + OFF_KQ + bufi * 32768;
-            uint8_t* KH = base + OFF_KH + bufi * 16384;
+            uint8_t* KQ = (MODE == 0) ? base + OFF_KQ + bufi * 32768 : gb + G_KQ;
+            uint8_t* KH = (MODE == 0) ? base + OFF_KH + bufi * 16384 : gb + G_KH;
+            const uint32_t kq_s = (MODE == 0) ? sb + OFF_KQ + bufi * 32768 : gsb + G_KQ;
+            const uint32_t kh_s = (MODE == 0) ? sb + OFF_KH + bufi * 16384 : gsb + G_KH;
 
             // V tile of this chunk (MN-major for V^T), asynchronously; done before the U MMA.
             // (Split mode: the copy-out warps move V straight into the ring.)
@@ -375,9 +427,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             }
 
             // ---- pass 1: per-token decays and segment products ---------------------------
-            // real:     al/iv[s][d] = alpha and 1/alpha of dim 4dg+d;
-            // rotation: al/iv[s][j] = alpha and 1/alpha of pair 2dg+j, al[s][2+j] = cos, iv[s][2+j] = sin.
-            float al[8][4], iv[8][4];
+            // real:     al[s][d] = alpha of dim 4dg+d;
+            // rotation: al[s][j] = alpha of pair 2dg+j, al[s][2+j] = cos, sn[s][j] = sin.
+            // (1/alpha is formed again where pass 2 needs it.)
+            float al[8][4], sn[8][2];
             float PA[4] = {1.f, 1.f, 1.f, 1.f}, PI[4] = {1.f, 1.f, 1.f, 1.f};
             if (ROT) { PI[2] = 0.f; PI[3] = 0.f; }           // (PA[2+j], PI[2+j]) = prod e^{+i theta}, from 1 + 0i
             const float L2E = 1.4426950408889634f;
@@ -397,16 +450,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                             i_ = ex2_approx(-ga[d] * L2E);
                         }
                     }
-                    al[s_][d] = a_; iv[s_][d] = i_;
+                    al[s_][d] = a_;
                     PA[d] *= a_; PI[d] *= i_;
                 }
                 if (ROT) {
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        float cs = 1.f, sn = 0.f;
-                        if (ok) __sincosf(ga[2 + j], &sn, &cs);
-                        al[s_][2 + j] = cs; iv[s_][2 + j] = sn;
-                        const float zr = PA[2 + j] * cs - PI[2 + j] * sn, zi = PI[2 + j] * cs + PA[2 + j] * sn;
+                        float cs = 1.f, sn_ = 0.f;
+                        if (ok) __sincosf(ga[2 + j], &sn_, &cs);
+                        al[s_][2 + j] = cs; sn[s_][j] = sn_;
+                        const float zr = PA[2 + j] * cs - PI[2 + j] * sn_, zi = PI[2 + j] * cs + PA[2 + j] * sn_;
                         PA[2 + j] = zr; PI[2 + j] = zi;
                     }
                 }
@@ -416,20 +469,22 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                 qtp[0] = make_float4(PA[0], PA[1], PA[2], PA[3]);
                 qtp[1] = make_float4(PI[0], PI[1], PI[2], PI[3]);
             }
-            if (tid < 64) sbeta[tid] = tid < Lc ? __ldg(p.beta + tokh(bhx, c, tid)) : 0.f;
-            named_bar(1, NPREP);
+            if (tid < 64) sbeta[tid] = beta_r;
+            named_bar(gbar, NPREP);
             // Buffers of task it - 2 must be released (by the chain, or by the copy-out warps)
             // before they are rewritten.
             if (MODE == 0 && it >= 2) {
                 const bool ok = mbar_wait_bounded(bar_empty + bufi, ((it - 2) >> 1) & 1, x.wait_limit_ns);
                 if (!ok) atomicExch(abort_p, 1);
             }
-            if (MODE == 1 && it >= 1) {     // the copy-out warps must have copied the previous tiles
-                const bool ok = mbar_wait_bounded(bar_empty + 0, (it - 1) & 1, x.wait_limit_ns);
+            if (MODE == 1 && tid == 0 && c >= RING) {
+                // the chain must have copied chunk c - RING out of this ring slot
+                const bool ok = spin_until_ge(sa.consumed + bhx, (unsigned)(c - RING + 1), x.wait_limit_ns);
                 if (!ok) atomicExch(abort_p, 1);
             }
-            named_bar(1, NPREP);
+            named_bar(gbar, NPREP);
             if (*abort_p) break;
+            if (MODE == 1 && tid < 64) rvec[tid] = beta_r;
 
             // ---- pass 2: factors around the reference token 31; operand tiles -----------
             {
@@ -480,18 +535,24 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                         }
                     }
                     const uint32_t off = sw128_off(r, ch) + in_ch;
+                    const uint2 qtv = make_uint2(pack_bf16x2(qt[0], qt[1]), pack_bf16x2(qt[2], qt[3]));
+                    const uint2 khv = make_uint2(pack_bf16x2(kh[0], kh[1]), pack_bf16x2(kh[2], kh[3]));
                     *reinterpret_cast<uint2*>(KQ + kb * 16384u + off) = make_uint2(pack_bf16x2(kt[0], kt[1]), pack_bf16x2(kt[2], kt[3]));
-                    *reinterpret_cast<uint2*>(KQ + kb * 16384u + 8192u + off) = make_uint2(pack_bf16x2(qt[0], qt[1]), pack_bf16x2(qt[2], qt[3]));
-                    *reinterpret_cast<uint2*>(KH + kb * 8192u + off) = make_uint2(pack_bf16x2(kh[0], kh[1]), pack_bf16x2(kh[2], kh[3]));
+                    *reinterpret_cast<uint2*>(KQ + kb * 16384u + 8192u + off) = qtv;
+                    *reinterpret_cast<uint2*>(KH + kb * 8192u + off) = khv;
+                    if (MODE == 1) {        // the ring slot has the tiles' shared-memory layout
+                        *reinterpret_cast<uint2*>(ring + SL_Q + kb * 8192u + off) = qtv;
+                        *reinterpret_cast<uint2*>(ring + SL_KH + kb * 8192u + off) = khv;
+                    }
                 };
                 auto include = [&](int s_, bool forward) {
 #pragma unroll
-                    for (int d = 0; d < (ROT ? 2 : 4); ++d) { P[d] *= al[s_][d]; Q[d] *= iv[s_][d]; }
+                    for (int d = 0; d < (ROT ? 2 : 4); ++d) { P[d] *= al[s_][d]; Q[d] *= rcp_approx(al[s_][d]); }
                     if (ROT) {
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
-                            const float cs = al[s_][2 + j], sn = forward ? -iv[s_][2 + j] : iv[s_][2 + j];
-                            const float nr = Rre[j] * cs - Rim[j] * sn, ni = Rim[j] * cs + Rre[j] * sn;
+                            const float cs = al[s_][2 + j], sv = forward ? -sn[s_][j] : sn[s_][j];
+                            const float nr = Rre[j] * cs - Rim[j] * sv, ni = Rim[j] * cs + Rre[j] * sv;
                             Rre[j] = nr; Rim[j] = ni;
                         }
                     }
@@ -534,7 +595,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                     if (!(fabsf(Q[d]) < 3e38f && fabsf(P[d]) < 3e38f)) bad = true;
             }
             fence_proxy_async_smem();
-            named_bar(1, NPREP);
+            named_bar(gbar, NPREP);
+            if (MODE == 1 && tid < 128)     // rho_ref, rho_C -> ring
+                reinterpret_cast<float4*>(rvec + 64)[tid] = reinterpret_cast<const float4*>(vec + 64)[tid];
             if (MODE == 0) mbar_arrive(bar_rho + bufi);
             if (MODE == 0 && it + 1 < ntasks) prefetch(task_bh(it + 1), task_c(it + 1));
 
@@ -543,19 +606,20 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             if (tid == 0) {
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kbk = ks >> 2, kin = (ks & 3) * 32;
-                    mma_bf16_ss(tbase + COL_AW, sdesc_sw128(sb + OFF_KQ + bufi * 32768 + kbk * 16384 + kin, 16, 1024),
-                                sdesc_sw128(sb + OFF_KH + bufi * 16384 + kbk * 8192 + kin, 16, 1024), ID_KK, ks > 0);
+                    mma_bf16_ss(tbase + col_aw, sdesc_sw128(kq_s + kbk * 16384 + kin, 16, 1024),
+                                sdesc_sw128(kh_s + kbk * 8192 + kin, 16, 1024), ID_KK, ks > 0);
                 }
-                if (!skip_commit) mma_commit(bar_pmma);
+                if (!skip_commit) mma_commit(g_pmma);
                 skip_commit = false;
             }
             if (!mma_wait()) break;
+            if (MODE == 1 && tid == 0 && it + 1 < ntasks) stage_part(it + 1, 0);   // Khat tile read
 
             // ---- solve: Tm = (I + A)^{-1}; Pm masked -> bf16 ---------------------------
             {
                 float vals[32];
-                tmem_ld16(tq + COL_AW + half * 32, *reinterpret_cast<float(*)[16]>(vals));
-                tmem_ld16(tq + COL_AW + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
+                tmem_ld16(tq + col_aw + half * 32, *reinterpret_cast<float(*)[16]>(vals));
+                tmem_ld16(tq + col_aw + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
                 if (row < 64) {
                     const int r = row;
                     const float br = sbeta[r];
@@ -571,7 +635,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                     }
                 } else {
                     const int r = row - 64;
-                    uint8_t* PM = base + OFF_PM + bufi * 8192;
+                    uint8_t* PM = (MODE == 0) ? base + OFF_PM + bufi * 8192 : ring + SL_PM;
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc) {
                         float m8[8];
@@ -584,7 +648,18 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                     }
                 }
             }
-            named_bar(1, NPREP);
+            {   // Tb: blocks above the diagonal stay zero (the area may hold staged k)
+                uint4* tbz = reinterpret_cast<uint4*>((MODE == 0) ? base + OFF_TB : gb + G_TB);
+                tbz[tid] = make_uint4(0u, 0u, 0u, 0u);
+                tbz[tid + NPREP] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            named_bar(gbar, NPREP);
+            // Tb = Tm diag(beta) as bf16 K-major [r][i] (blocks above the diagonal stay zero).
+            uint8_t* TB = (MODE == 0) ? base + OFF_TB : gb + G_TB;
+            auto tb_put2 = [&](int r, int i, float x0, float x1) {      // columns i, i + 1
+                *reinterpret_cast<uint32_t*>(TB + sw128_off(r, i >> 3) + (i & 7) * 2) =
+                    pack_bf16x2(x0 * sbeta[i], x1 * sbeta[i + 1]);
+            };
             // 16x16 diagonal blocks by forward substitution (lane = column of one block).
             if (tid < 64) {
                 const int bb = (tid >> 4) * 16, jj = tid & 15;
@@ -596,118 +671,144 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
                     for (int i = 0; i < r; ++i) s_ = fmaf(-Af[(bb + r) * AS + bb + i], t[i], s_);
                     t[r] = s_;
                 }
+                const float bj = sbeta[bb + jj];
+                const int ib = bb + jj;
 #pragma unroll
-                for (int r = 0; r < 16; ++r) Tf[(bb + r) * AS + bb + jj] = t[r];
-            }
-            named_bar(1, NPREP);
-            // Off-diagonal blocks, by block distance: T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ.
-            // One warp per 16x16 block, on m16n8k8 tf32 tensor-core MMAs (the result is rounded
-            // to bf16 for the UT transform anyway): X = sum A_IK T_KJ, then T_IJ = -T_II X.
-            {
-                const int gid = lane >> 2, tig = lane & 3;
-                float* Xw = Xf + warp * XS;                   // this warp's 16 x 20 scratch
-#pragma unroll 1
-                for (int dist = 1; dist < 4; ++dist) {
-                    if (warp < 4 - dist) {
-                        const int J = warp, I = warp + dist;
-                        float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
-                        const float* ar0 = Af + (16 * I + gid) * AS;
-                        const float* ar1 = ar0 + 8 * AS;
-#pragma unroll 2
-                        for (int kb8 = 16 * J; kb8 < 16 * I; kb8 += 8) {
-                            const uint32_t a[4] = {to_tf32(ar0[kb8 + tig]), to_tf32(ar1[kb8 + tig]),
-                                                   to_tf32(ar0[kb8 + tig + 4]), to_tf32(ar1[kb8 + tig + 4])};
-                            const float* tr0 = Tf + (kb8 + tig) * AS + 16 * J + gid;
-                            const float* tr1 = tr0 + 4 * AS;
-                            const uint32_t b0[2] = {to_tf32(tr0[0]), to_tf32(tr1[0])};
-                            const uint32_t b1[2] = {to_tf32(tr0[8]), to_tf32(tr1[8])};
-                            mma_tf32_16x8x8(x0, a, b0);
-                            mma_tf32_16x8x8(x1, a, b1);
-                        }
-                        Xw[gid * 20 + 2 * tig] = x0[0];       Xw[gid * 20 + 2 * tig + 1] = x0[1];
-                        Xw[(gid + 8) * 20 + 2 * tig] = x0[2]; Xw[(gid + 8) * 20 + 2 * tig + 1] = x0[3];
-                        Xw[gid * 20 + 8 + 2 * tig] = x1[0];       Xw[gid * 20 + 9 + 2 * tig] = x1[1];
-                        Xw[(gid + 8) * 20 + 8 + 2 * tig] = x1[2]; Xw[(gid + 8) * 20 + 9 + 2 * tig] = x1[3];
-                        __syncwarp();
-                        float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-                        const float* dr0 = Tf + (16 * I + gid) * AS + 16 * I;
-                        const float* dr1 = dr0 + 8 * AS;
-#pragma unroll
-                        for (int kb8 = 0; kb8 < 16; kb8 += 8) {
-                            const uint32_t a[4] = {to_tf32(dr0[kb8 + tig]), to_tf32(dr1[kb8 + tig]),
-                                                   to_tf32(dr0[kb8 + tig + 4]), to_tf32(dr1[kb8 + tig + 4])};
-                            const float* xr0 = Xw + (kb8 + tig) * 20 + gid;
-                            const float* xr1 = xr0 + 4 * 20;
-                            const uint32_t b0[2] = {to_tf32(xr0[0]), to_tf32(xr1[0])};
-                            const uint32_t b1[2] = {to_tf32(xr0[8]), to_tf32(xr1[8])};
-                            mma_tf32_16x8x8(y0, a, b0);
-                            mma_tf32_16x8x8(y1, a, b1);
-                        }
-                        float* t0 = Tf + (16 * I + gid) * AS + 16 * J;
-                        float* t1 = t0 + 8 * AS;
-                        t0[2 * tig] = -y0[0]; t0[2 * tig + 1] = -y0[1]; t1[2 * tig] = -y0[2]; t1[2 * tig + 1] = -y0[3];
-                        t0[8 + 2 * tig] = -y1[0]; t0[9 + 2 * tig] = -y1[1]; t1[8 + 2 * tig] = -y1[2]; t1[9 + 2 * tig] = -y1[3];
-                    }
-                    named_bar(1, NPREP);
+                for (int r = 0; r < 16; ++r) {
+                    Tf[(bb + r) * AS + bb + jj] = t[r];
+                    *reinterpret_cast<__nv_bfloat16*>(TB + sw128_off(bb + r, ib >> 3) + (ib & 7) * 2) =
+                        __float2bfloat16_rn(t[r] * bj);
                 }
             }
-            // Tb = Tm diag(beta), zero above the block diagonal, -> bf16 K-major [r][i].
-            // (Split mode keeps two Tb tiles in the unused V area, one per buffer.)
-            const uint32_t tb_off = (MODE == 0) ? OFF_TB : OFF_V + (uint32_t)bufi * 8192u;
-            {
-                const int r = tid >> 2, qq = tid & 3;
+            named_bar(gbar, NPREP);
+            // Blocks below the diagonal in one phase, one warp per block, with the 2x2 block
+            // recursion T_lo,hi-split: T_hi,lo = -T_hi A_hi,lo T_lo for the halves {0,1}, {2,3}:
+            //   T10 = -D1 A10 D0,  T21 = -D2 A21 D1,  T32 = -D3 A32 D2,
+            //   T20 = -D2 X20,     T31 = -(T32 A21 + D3 A31) D1,   T30 = -(T32 X20 + D3 X30),
+            //   X20 = A20 D0 + A21 T10,  X30 = A30 D0 + A31 T10   (D_I: diagonal blocks).
+            // Each warp forms the blocks it depends on itself, in 16x16 scratch taken from the
+            // unused upper triangles of A and Tm, on m16n8k8 tf32 tensor-core MMAs (the result
+            // is rounded to bf16 for the UT transform anyway).
+            if (warp < 6) {
+                const int gid = lane >> 2, tig = lane & 3;
+                auto Ab = [&](int I, int J) { return Af + 16 * I * AS + 16 * J; };
+                auto Tb_ = [&](int I, int J) { return Tf + 16 * I * AS + 16 * J; };
+                // acc += L R for 16x16 fp32 blocks (row stride AS)
+                auto mm = [&](float (&acc)[2][4], const float* L, const float* R) {
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float m8[8];
-                    const int i0 = qq * 16 + hh * 8;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int i = i0 + u;
-                        m8[u] = ((i >> 4) <= (r >> 4)) ? Tf[r * AS + i] * sbeta[i] : 0.f;
+                    for (int kb8 = 0; kb8 < 16; kb8 += 8) {
+                        const uint32_t a[4] = {to_tf32(L[gid * AS + kb8 + tig]), to_tf32(L[(gid + 8) * AS + kb8 + tig]),
+                                               to_tf32(L[gid * AS + kb8 + tig + 4]),
+                                               to_tf32(L[(gid + 8) * AS + kb8 + tig + 4])};
+                        const uint32_t b0[2] = {to_tf32(R[(kb8 + tig) * AS + gid]), to_tf32(R[(kb8 + tig + 4) * AS + gid])};
+                        const uint32_t b1[2] = {to_tf32(R[(kb8 + tig) * AS + 8 + gid]),
+                                                to_tf32(R[(kb8 + tig + 4) * AS + 8 + gid])};
+                        mma_tf32_16x8x8(acc[0], a, b0);
+                        mma_tf32_16x8x8(acc[1], a, b1);
                     }
-                    *reinterpret_cast<uint4*>(base + tb_off + sw128_off(r, qq * 2 + hh)) = pack8(m8);
+                };
+                auto zero = [&](float (&acc)[2][4]) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+                };
+                auto put = [&](float* Dst, const float (&acc)[2][4], float sg) {   // Dst = sg * acc
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        *reinterpret_cast<float2*>(Dst + gid * AS + 8 * h + 2 * tig) = make_float2(sg * acc[h][0], sg * acc[h][1]);
+                        *reinterpret_cast<float2*>(Dst + (gid + 8) * AS + 8 * h + 2 * tig) =
+                            make_float2(sg * acc[h][2], sg * acc[h][3]);
+                    }
+                    __syncwarp();
+                };
+                auto out = [&](int I, int J, const float (&acc)[2][4]) {     // Tb block (I, J) = -acc
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int i = 16 * J + 8 * h + 2 * tig;
+                        tb_put2(16 * I + gid, i, -acc[h][0], -acc[h][1]);
+                        tb_put2(16 * I + gid + 8, i, -acc[h][2], -acc[h][3]);
+                    }
+                };
+                float x[2][4], y[2][4];
+                if (warp < 3) {                 // T(w+1, w) = -D(w+1) A(w+1, w) D(w)
+                    const int J = warp, I = warp + 1;
+                    float* S0 = Ab(0, warp + 1);
+                    zero(x); mm(x, Ab(I, J), Tb_(J, J)); put(S0, x, 1.f);
+                    zero(y); mm(y, Tb_(I, I), S0); out(I, J, y);
+                } else if (warp == 3) {         // T20
+                    float* S0 = Ab(1, 2); float* S1 = Ab(1, 3);
+                    zero(x); mm(x, Ab(1, 0), Tb_(0, 0)); put(S0, x, 1.f);
+                    zero(y); mm(y, Tb_(1, 1), S0); put(S1, y, -1.f);                       // T10
+                    zero(x); mm(x, Ab(2, 0), Tb_(0, 0)); mm(x, Ab(2, 1), S1); put(S0, x, 1.f);   // X20
+                    zero(y); mm(y, Tb_(2, 2), S0); out(2, 0, y);
+                } else if (warp == 4) {         // T31
+                    float* S0 = Ab(2, 3); float* S1 = Tb_(0, 1);
+                    zero(x); mm(x, Ab(3, 2), Tb_(2, 2)); put(S0, x, 1.f);
+                    zero(y); mm(y, Tb_(3, 3), S0); put(S1, y, -1.f);                       // T32
+                    zero(x); mm(x, S1, Ab(2, 1)); mm(x, Tb_(3, 3), Ab(3, 1)); put(S0, x, 1.f);
+                    zero(y); mm(y, S0, Tb_(1, 1)); out(3, 1, y);
+                } else {                        // T30
+                    float* S0 = Tb_(0, 2); float* S1 = Tb_(0, 3); float* S2 = Tb_(1, 2); float* S3 = Tb_(1, 3);
+                    zero(x); mm(x, Ab(1, 0), Tb_(0, 0));
+                    zero(y); mm(y, Ab(3, 2), Tb_(2, 2));
+                    put(S0, x, 1.f); put(S1, y, 1.f);
+                    zero(x); mm(x, Tb_(1, 1), S0);
+                    zero(y); mm(y, Tb_(3, 3), S1);
+                    put(S2, x, -1.f); put(S3, y, -1.f);                                   // T10, T32
+                    zero(x); mm(x, Ab(2, 0), Tb_(0, 0)); mm(x, Ab(2, 1), S2);             // X20
+                    zero(y); mm(y, Ab(3, 0), Tb_(0, 0)); mm(y, Ab(3, 1), S2);             // X30
+                    put(S0, x, 1.f); put(S1, y, 1.f);
+                    zero(x); mm(x, S3, S0); mm(x, Tb_(3, 3), S1); out(3, 0, x);
                 }
             }
             if (MODE == 0) cp_async_wait_all();
             publish();
+            if (MODE == 1) {                // Tb -> ring
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+                    reinterpret_cast<uint4*>(ring + SL_TB)[tid + e * NPREP] = reinterpret_cast<const uint4*>(TB)[tid + e * NPREP];
+                if (tid == 0 && it + 1 < ntasks) stage_part(it + 1, 1);          // A and Tm done
+            }
 
             // ---- U^T = V^T Tb^T -> E[c&1];  Wm^T = Ktil^T Tb^T -> A'/W columns -------------
             if (tid == 0) {
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t bdesc = sdesc_sw128(sb + tb_off + ks * 32, 16, 1024);
+                    const uint64_t bdesc = sdesc_sw128(((MODE == 0) ? sb + OFF_TB : gsb + G_TB) + ks * 32, 16, 1024);
                     if (MODE == 0)
                         mma_bf16_ss(tbase + COL_E + bufi * 64, sdesc_sw128(sb + OFF_V + ks * 2048, 8192, 1024), bdesc,
                                     ID_MK, ks > 0);
-                    mma_bf16_ss(tbase + COL_AW, sdesc_sw128(sb + OFF_KQ + bufi * 32768 + ks * 2048, 16384, 1024), bdesc,
+                    mma_bf16_ss(tbase + col_aw, sdesc_sw128(kq_s + ks * 2048, 16384, 1024), bdesc,
                                 ID_MK, ks > 0);
                 }
-                mma_commit(bar_pmma);
+                mma_commit(g_pmma);
             }
             if (!mma_wait()) break;
+            if (MODE == 1 && tid == 0 && it + 1 < ntasks) stage_part(it + 1, 2);   // Tb tile read
 
             // Wm^T -> bf16 MN-major tile (row = dk, 64 tokens per row).
             {
                 float vals[32];
-                tmem_ld16(tq + COL_AW + half * 32, *reinterpret_cast<float(*)[16]>(vals));
-                tmem_ld16(tq + COL_AW + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
-                uint8_t* W = base + OFF_W + bufi * 16384;
+                tmem_ld16(tq + col_aw + half * 32, *reinterpret_cast<float(*)[16]>(vals));
+                tmem_ld16(tq + col_aw + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
+                uint8_t* W = (MODE == 0) ? base + OFF_W + bufi * 16384 : ring + SL_W;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc)
                     *reinterpret_cast<uint4*>(W + sw128_off(row, half * 4 + cc)) = pack8(vals + cc * 8);
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar(1, NPREP);
-            mbar_arrive(bar_full + bufi);
+            named_bar(gbar, NPREP);
+            mbar_arrive(bar_full + (MODE == 0 ? bufi : grp));
         }
         if (bad) atomicExch(range_flag, 1);
-    } else if (nchunks > 0 && tid >= NPREP && chain_cta) {
+        // after an early exit, let staging copies still in flight land before the CTA ends
+        if (MODE == 1 && tid == 0 && staged > landed) (void)mbar_wait_bounded(g_stage, landed & 1, x.wait_limit_ns);
+    } else if (nchunks > 0 && tid >= NPREP && tid < NPREP + CHAIN_THREADS && chain_cta) {
         // =========================== chain group ==================================
         const int row = tid - NPREP;          // TMEM lane = value row of S (quad = warp & 3)
         uint32_t mma_phase = 0;
         const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_NEG = idesc_bf16(128, 64, 0, 1, 1);
         const uint32_t ID_KM128 = idesc_bf16(128, 128, 0, 1, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
-        auto cbar = [&]() { named_bar(2, NT - NPREP); };
+        auto cbar = [&]() { named_bar(2, CHAIN_THREADS); };
         auto mma_wait = [&]() -> bool {
             const bool ok = mbar_wait_bounded(bar_cmma, mma_phase, x.wait_limit_ns);
             mma_phase ^= 1u;
@@ -965,56 +1066,23 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(FwdParams p, TcExtr
             if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
         }
     }
-    if (MODE == 1 && nchunks > 0 && !chain_cta && tid >= NPREP) {
-        // ============ split mode: transfer thread of a prep worker =============================
-        // One thread stages each task's raw inputs with bulk copies (one per token row) for the
-        // prep warps, then bulk-stores the finished tiles into the ring slot and publishes it.
-        if (tid == NPREP) {
-            const int W = (int)gridDim.x - NH, wk = (int)blockIdx.x - NH;
-            const int ntasks = (NH * nchunks - wk + W - 1) / W;
-            auto stage_task = [&](int itx) {
-                const int task = wk + itx * W, c = task / NH, bhx = task % NH;
-                const int bb = bhx / p.H, hh = bhx % p.H;
-                // tokens past the sequence end arrive as zeros; 64 KB in every case
-                mbar_arrive_expect_tx(bar_rho + 0, 65536u);
-                tma_load_4d(sb + STG_Q, &tm.q, 0, hh, c * C, bb, bar_rho + 0);
-                tma_load_4d(sb + STG_K, &tm.k, 0, hh, c * C, bb, bar_rho + 0);
-                tma_load_4d(sb + STG_A, &tm.g, 0, hh, c * C, bb, bar_rho + 0);
-                if (ROT) tma_load_4d(sb + STG_A + 16384u, &tm.th, 0, hh, c * C, bb, bar_rho + 0);
-            };
-            if (ntasks > 0) stage_task(0);
-            for (int it = 0; it < ntasks; ++it) {
-                const int task = wk + it * W, c = task / NH, bhx = task % NH, slot = c % RING;
-                bool ok = true;
-                if (it + 1 < ntasks) {
-                    // once the prep warps have read this task's staging, stage the next task
-                    ok = mbar_wait_bounded(bar_rho + 1, it & 1, x.wait_limit_ns);
-                    if (ok) stage_task(it + 1);
-                }
-                if (ok) ok = mbar_wait_bounded(bar_full + 0, it & 1, x.wait_limit_ns);
-                // the chain must have copied chunk c - RING out of this slot
-                if (ok && c >= RING) ok = spin_until_ge(sa.consumed + bhx, (unsigned)(c - RING + 1), x.wait_limit_ns);
-                if (!ok) { atomicExch(abort_c, 1); break; }
-                uint8_t* dst = sa.ring + ((size_t)bhx * RING + slot) * SLOT_BYTES;
-                bulk_s2g(dst + SL_Q, sb + OFF_KQ + 8192, 8192);
-                bulk_s2g(dst + SL_Q + 8192, sb + OFF_KQ + 16384 + 8192, 8192);
-                bulk_s2g(dst + SL_KH, sb + OFF_KH, 16384);
-                bulk_s2g(dst + SL_W, sb + OFF_W, 16384);
-                bulk_s2g(dst + SL_PM, sb + OFF_PM, 8192);
-                bulk_s2g(dst + SL_TB, sb + OFF_V, 8192);
-                bulk_s2g(dst + SL_VEC, sb + OFF_VEC, VEC_FLOATS * 4);
-                bulk_commit();
-                bulk_wait_read_all();
-                mbar_arrive(bar_empty + 0);          // the tiles may be rewritten now
-                bulk_wait_all();
-                fence_proxy_async_global();
-                st_release_gpu(sa.ready + (size_t)bhx * RING + slot, (unsigned)(c + 1));
-            }
+    if (MODE == 1 && nchunks > 0 && !chain_cta && tid >= 2 * NPREP && (tid & 31) == 0) {
+        // ============ split mode: publisher of a prep group (one thread per group) ============
+        // The group's stores to a ring slot precede its bar_full arrival, so a gpu-scope fence
+        // here orders them before the release of the slot's ready flag.
+        const int grp = (tid - 2 * NPREP) >> 5;
+        const int W = 2 * ((int)gridDim.x - NH), wk = 2 * ((int)blockIdx.x - NH) + grp;
+        const int ntasks = (NH * nchunks - wk + W - 1) / W;
+        for (int it = 0; it < ntasks; ++it) {
+            const int task = wk + it * W, c = task / NH, bhx = task % NH;
+            if (!mbar_wait_bounded(bar_full + grp, it & 1, x.wait_limit_ns)) { atomicExch(abort_c, 1); break; }
+            __threadfence();
+            st_release_gpu(sa.ready + (size_t)bhx * RING + c % RING, (unsigned)(c + 1));
         }
     }
 
     if (nchunks == 0 && p.S_T && chain_cta) {
-        for (int e = tid; e < D * D; e += NT)
+        for (int e = tid; e < D * D; e += nthreads<MODE>())
             p.S_T[(size_t)bh * D * D + e] = p.S0 ? p.S0[(size_t)bh * D * D + e] : 0.f;
     }
     tc_fence_before();
