@@ -182,8 +182,8 @@ GDR_API gdr_status gdr_query_device_status(gdr_stream_t stream);
  *
  * It runs the split tensor-core kernel (same arithmetic and results as
  * gdr_chunk_fwd with GDR_ALGO_TCGEN05_SPLIT) with the kernel's hand-off ring in a scratch
- * array compiled into the library: GDR_NOALLOC_MAX_HEADS * 3 slots of 84,224 bytes plus
- * flags (about 7.7 MiB), which every GPU that loads the library holds until the process
+ * array compiled into the library: GDR_NOALLOC_MAX_HEADS * 6 slots of 67,840 bytes plus
+ * flags (about 12.4 MiB), which every GPU that loads the library holds until the process
  * exits.
  *   - desc->algo must be GDR_ALGO_AUTO or GDR_ALGO_TCGEN05_SPLIT; q, k, v must be bf16 with
  *     dk = dv = 128; B*H must not exceed GDR_NOALLOC_MAX_HEADS, else GDR_ERR_UNSUPPORTED with

@@ -83,7 +83,7 @@ constexpr uint32_t SLOT_BYTES = SL_VEC + VEC_FLOATS * 4;        // bytes of one 
 // itself from the input (MN-major: 2 groups x 64 tokens x 128 B).
 constexpr uint32_t SL_V = (SLOT_BYTES + 1023) & ~1023u;
 constexpr uint32_t SLOT_STRIDE = SL_V + 16384;                  // slot buffers in the chain CTA
-constexpr int RING = 4;               // ring slots per head
+constexpr int RING = 6;               // ring slots per head
 // Split chain CTAs stage each chunk's o here ([64 tokens][128] in the output type) and
 // store it with one tensor-map tile store.
 constexpr uint32_t OFF_OSTG = 2 * SLOT_STRIDE;
@@ -100,7 +100,7 @@ constexpr uint32_t G_AF = 65536;     // fp32 A [64][68]
 constexpr uint32_t G_TF = G_AF + 64 * AS * 4;   // fp32 Tm [64][68]
 constexpr uint32_t G_VEC = G_TF + 64 * AS * 4;  // beta, rho_ref, rho_C
 constexpr uint32_t G_STRIDE = (G_VEC + VEC_FLOATS * 4 + 1023) & ~1023u;
-constexpr int NT_SPLIT = 2 * NPREP + 64;        // two prep groups and one publishing warp each
+constexpr int NT_SPLIT = 2 * NPREP;             // two prep groups (16 warps: 128 registers a thread)
 constexpr uint32_t OFF_BAR_SPLIT = 2 * G_STRIDE;
 static_assert(2 * SLOT_STRIDE + 64 * 128 * 4 <= OFF_BAR_SPLIT, "chain slot buffers overlap the barriers");
 static_assert(G_TF + 64 * AS * 4 >= G_AF + 32768, "gate staging does not fit in A and Tm");
@@ -214,6 +214,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
     uint64_t* bar_empty = bar_pmma + 5;      // [2] chain -> prep: buffers of a chunk free
     uint64_t* bar_rho = bar_pmma + 7;        // [2] prep -> chain: decay vectors of a chunk ready;
                                              //     split workers: group g's staged inputs landed
+    uint64_t* bar_o = bar_pmma + 9;          // [2] split chain: O^T of a chunk complete (per buffer)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_base + 96);
     int* abort_p = reinterpret_cast<int*>(bar_base + 100);
     int* abort_c = reinterpret_cast<int*>(bar_base + 104);
@@ -250,9 +251,10 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         mbar_init(bar_cmma, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_pmma + i, 1);
+            mbar_init(bar_o + i, 1);
             // split chain CTAs: the loader's expect_tx arrival (plus the slot's and V's bytes)
             mbar_init(bar_full + i, (MODE == 1 && chain_cta) ? 1 : NPREP);
-            mbar_init(bar_empty + i, CHAIN_THREADS);
+            mbar_init(bar_empty + i, (MODE == 1) ? 1 : CHAIN_THREADS);
             // split workers: one expect_tx arrival plus the staged bytes
             mbar_init(bar_rho + i, (MODE == 1) ? 1 : NPREP);
         }
@@ -348,6 +350,17 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         // split: stage part `part` of task itx's raw inputs (tokens past the sequence end
         // arrive as zeros); part 0 also arms the barrier for all 64 KB
         int staged = 0, landed = 0;     // split: tasks whose staging was issued / has landed
+        // Split: the ring slot of a finished task is published by the group's thread 32 once
+        // the next task's inputs have been read (or after the last task), while the other warps
+        // run pass 1; the named barriers order every thread's stores to the slot before its
+        // gpu-scope fence and release.  Publishing before the next task's ring-slot wait keeps
+        // the workers free of waits on one another.
+        int pub_c = -1, pub_bh = 0;
+        auto publish_slot = [&]() {
+            __threadfence();
+            st_release_gpu(sa.ready + (size_t)pub_bh * RING + pub_c % RING, (unsigned)(pub_c + 1));
+            pub_c = -1;
+        };
         auto stage_part = [&](int itx, int part) {
             const int c2 = task_c(itx), b2 = task_bh(itx);
             const int bb = b2 / p.H, hh = b2 % p.H;
@@ -403,6 +416,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     }
                 }
                 named_bar(gbar, NPREP);      // pass 1 rewrites the k staging area (G_QT)
+                if (tid == 32 && pub_c >= 0) publish_slot();   // overlaps pass 1 of the other warps
             }
             float* sbeta = vec;
             float* rho_ref = vec + 64;
@@ -511,6 +525,43 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     }
                 }
                 const float sc = p.scale;
+                // Split: the ring carries Qtil2 = Qtil P_m^T and Khat2 = Khat (P_m^{-1} P_C), the
+                // reference decay folded in, so that the chain can keep the plain state.  rr / rc:
+                // P_m and P_m^{-1} P_C of this thread's dims (rotation: [j] real, [2+j] imaginary
+                // part of pair 2dg+j), from the segment products.
+                float rr[4] = {1.f, 1.f, 1.f, 1.f}, rc[4] = {1.f, 1.f, 1.f, 1.f};
+                if (MODE == 1) {
+                    float mr[4] = {1.f, 1.f, 0.f, 0.f}, mc[4] = {1.f, 1.f, 0.f, 0.f};   // rotation: magnitudes, phases
+                    float pr_re[2] = {1.f, 1.f}, pr_im[2] = {0.f, 0.f}, pc_re[2] = {1.f, 1.f}, pc_im[2] = {0.f, 0.f};
+#pragma unroll
+                    for (int s2 = 0; s2 < 8; ++s2) {
+                        const float4* t = reinterpret_cast<const float4*>(QT + (s2 * 32 + dg) * 8);
+                        const float4 a4 = t[0];
+                        if (!ROT) {
+                            float* f = s2 < 4 ? rr : rc;
+                            f[0] *= a4.x; f[1] *= a4.y; f[2] *= a4.z; f[3] *= a4.w;
+                        } else {
+                            const float4 i4 = t[1];
+                            float* m = s2 < 4 ? mr : mc;
+                            float* zre = s2 < 4 ? pr_re : pc_re;
+                            float* zim = s2 < 4 ? pr_im : pc_im;
+                            m[0] *= a4.x; m[1] *= a4.y;
+                            const float zr[2] = {a4.z, a4.w}, zi[2] = {i4.z, i4.w};
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                const float nr = zre[j] * zr[j] - zim[j] * zi[j], ni = zim[j] * zr[j] + zre[j] * zi[j];
+                                zre[j] = nr; zim[j] = ni;
+                            }
+                        }
+                    }
+                    if (ROT) {
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            rr[j] = mr[j] * pr_re[j]; rr[2 + j] = mr[j] * pr_im[j];
+                            rc[j] = mc[j] * pc_re[j]; rc[2 + j] = mc[j] * pc_im[j];
+                        }
+                    }
+                }
                 auto emit = [&](int r, const float (&F)[4], const float (&G)[4], uint2 kraw, uint2 qraw) {
                     const float kk[4] = {__uint_as_float(kraw.x << 16), __uint_as_float(kraw.x & 0xFFFF0000u),
                                          __uint_as_float(kraw.y << 16), __uint_as_float(kraw.y & 0xFFFF0000u)};
@@ -541,8 +592,24 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     *reinterpret_cast<uint2*>(KQ + kb * 16384u + 8192u + off) = qtv;
                     *reinterpret_cast<uint2*>(KH + kb * 8192u + off) = khv;
                     if (MODE == 1) {        // the ring slot has the tiles' shared-memory layout
-                        *reinterpret_cast<uint2*>(ring + SL_Q + kb * 8192u + off) = qtv;
-                        *reinterpret_cast<uint2*>(ring + SL_KH + kb * 8192u + off) = khv;
+                        float q2[4], k2[4];
+                        if (!ROT) {
+#pragma unroll
+                            for (int d = 0; d < 4; ++d) { q2[d] = qt[d] * rr[d]; k2[d] = kh[d] * rc[d]; }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                const float a = qt[2 * j], b = qt[2 * j + 1], e = kh[2 * j], f = kh[2 * j + 1];
+                                q2[2 * j] = a * rr[j] + b * rr[2 + j];        // times conj(P_m)
+                                q2[2 * j + 1] = b * rr[j] - a * rr[2 + j];
+                                k2[2 * j] = e * rc[j] - f * rc[2 + j];        // times P_m^{-1} P_C
+                                k2[2 * j + 1] = e * rc[2 + j] + f * rc[j];
+                            }
+                        }
+                        *reinterpret_cast<uint2*>(ring + SL_Q + kb * 8192u + off) =
+                            make_uint2(pack_bf16x2(q2[0], q2[1]), pack_bf16x2(q2[2], q2[3]));
+                        *reinterpret_cast<uint2*>(ring + SL_KH + kb * 8192u + off) =
+                            make_uint2(pack_bf16x2(k2[0], k2[1]), pack_bf16x2(k2[2], k2[3]));
                     }
                 };
                 auto include = [&](int s_, bool forward) {
@@ -596,8 +663,15 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             }
             fence_proxy_async_smem();
             named_bar(gbar, NPREP);
-            if (MODE == 1 && tid < 128)     // rho_ref, rho_C -> ring
-                reinterpret_cast<float4*>(rvec + 64)[tid] = reinterpret_cast<const float4*>(vec + 64)[tid];
+            if (MODE == 1 && tid < 128) {   // P_C = P_m (P_m^{-1} P_C) -> ring
+                if (!ROT) {
+                    rvec[64 + tid] = vec[64 + tid] * vec[64 + 256 + tid];
+                } else if (tid < 64) {
+                    const float a = vec[64 + tid], b = vec[64 + 128 + tid], cc = vec[64 + 256 + tid], d = vec[64 + 384 + tid];
+                    rvec[64 + tid] = a * cc - b * d;
+                    rvec[64 + 128 + tid] = a * d + b * cc;
+                }
+            }
             if (MODE == 0) mbar_arrive(bar_rho + bufi);
             if (MODE == 0 && it + 1 < ntasks) prefetch(task_bh(it + 1), task_c(it + 1));
 
@@ -790,6 +864,21 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 tmem_ld16(tq + col_aw + half * 32, *reinterpret_cast<float(*)[16]>(vals));
                 tmem_ld16(tq + col_aw + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
                 uint8_t* W = (MODE == 0) ? base + OFF_W + bufi * 16384 : ring + SL_W;
+                if (MODE == 1) {        // Wm2^T = P_m Wm^T (row = dk index)
+                    if (!ROT) {
+                        const float f = vec[64 + row];
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) vals[u] *= f;
+                    } else {            // rows 2j, 2j+1: (w0 + i w1) conj(P_m)
+                        const float cr = vec[64 + (row >> 1)], ci = vec[64 + 128 + (row >> 1)];
+                        const float sgn = (row & 1) ? -1.f : 1.f;
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const float other = __shfl_xor_sync(0xffffffffu, vals[u], 1);
+                            vals[u] = vals[u] * cr + sgn * other * ci;
+                        }
+                    }
+                }
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc)
                     *reinterpret_cast<uint4*>(W + sw128_off(row, half * 4 + cc)) = pack8(vals + cc * 8);
@@ -797,12 +886,249 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(gbar, NPREP);
-            mbar_arrive(bar_full + (MODE == 0 ? bufi : grp));
+            if (MODE == 0) mbar_arrive(bar_full + bufi);
+            if (MODE == 1) { pub_c = c; pub_bh = bhx; }
         }
+        if (MODE == 1 && tid == 32 && pub_c >= 0) publish_slot();
         if (bad) atomicExch(range_flag, 1);
         // after an early exit, let staging copies still in flight land before the CTA ends
         if (MODE == 1 && tid == 0 && staged > landed) (void)mbar_wait_bounded(g_stage, landed & 1, x.wait_limit_ns);
-    } else if (nchunks > 0 && tid >= NPREP && tid < NPREP + CHAIN_THREADS && chain_cta) {
+    } else if (MODE == 1 && nchunks > 0 && chain_cta && tid >= NPREP - 128 && tid < NPREP + CHAIN_THREADS) {
+        // ============ split mode: chain (warps 8-11) and o epilogue (warps 4-7) ==================
+        // The chain keeps the plain state S (fp32) in TMEM and its bf16 copy in one of two column
+        // blocks (chunk parity); the workers fold the reference decay into the ring's tiles
+        // (Qtil2 = Qtil P_m^T, Wm2^T = P_m Wm^T, Khat2 = Khat P_m^{-1} P_C), so per chunk
+        //   E^T = U^T - S Wm2^T,   O^T = S Qtil2^T + E^T Pm^T,   S <- S P_C + E^T Khat2,
+        // and the decay S P_C runs while the E^T MMAs do, off the state's critical path.
+        // MMA completions: bar_cmma (E^T), bar_pmma[0] (state), bar_o[b] (O^T of buffer b);
+        // the epilogue frees O^T buffer b through bar_rho[b] and ring slot b through bar_empty[b].
+        const int row = quad * 32 + lane;
+        uint64_t* bar_e = bar_cmma;
+        uint64_t* bar_s = bar_pmma;
+        uint64_t* bar_ofree = bar_rho;
+        const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_NEG = idesc_bf16(128, 64, 0, 1, 1);
+        const uint32_t ID_KM128 = idesc_bf16(128, 128, 0, 1, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
+        auto sbcol = [](int c) -> uint32_t { return (c & 1) ? COL_AW : COL_SB; };
+        auto scale_cols = [&](int col0, float (&s)[16], const float* rho) {
+            if (!ROT) {
+#pragma unroll
+                for (int u4 = 0; u4 < 4; ++u4) {
+                    const float4 f = *reinterpret_cast<const float4*>(rho + col0 + 4 * u4);
+                    s[4 * u4] *= f.x; s[4 * u4 + 1] *= f.y; s[4 * u4 + 2] *= f.z; s[4 * u4 + 3] *= f.w;
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < 16; u += 2) {
+                    const int pr = (col0 + u) >> 1;
+                    const float cr = rho[pr], ci = rho[128 + pr];
+                    const float xr = s[u], xi = s[u + 1];
+                    s[u] = xr * cr - xi * ci;
+                    s[u + 1] = xr * ci + xi * cr;
+                }
+            }
+        };
+        if (tid >= NPREP) {
+            // ---------------- chain: one thread per TMEM lane, tid NPREP issues the MMAs ----------
+            const bool issuer = (tid == NPREP);
+            auto cbar = [&]() { named_bar(2, CHAIN_THREADS); };
+            auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+                const bool ok = mbar_wait_bounded(bar, parity, x.wait_limit_ns);
+                if (!ok) atomicExch(abort_c, 1);
+                cbar();
+                tc_fence_after();
+                return *abort_c == 0;
+            };
+            auto issue_u = [&](int c) {       // U^T = V^T Tb^T -> E^T buffer of chunk c
+                const uint32_t sl = sb + slot_base(c);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(tbase + COL_E + (c & 1) * 64, sdesc_sw128(sl + SL_V + ks * 2048, 8192, 1024),
+                                sdesc_sw128(sl + SL_TB + ks * 32, 16, 1024), ID_MK, ks > 0);
+            };
+            bool alive = wait_all(bar_full + 0, 0);
+            if (alive) {
+                // S_0 (fp32) and its bf16 copy
+#pragma unroll 1
+                for (int g = 0; g < 8; ++g) {
+                    const int col0 = g * 16;
+                    float s[16];
+                    if (p.S0) {
+                        const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)bh * D + row) * D + col0);
+#pragma unroll
+                        for (int u4 = 0; u4 < 4; ++u4) {
+                            const float4 t4 = src[u4];
+                            s[4 * u4] = t4.x; s[4 * u4 + 1] = t4.y; s[4 * u4 + 2] = t4.z; s[4 * u4 + 3] = t4.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) s[u] = 0.f;
+                    }
+                    tmem_st16(tq + COL_S + col0, s);
+                    uint32_t w[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) w[u] = pack_bf16x2(s[2 * u], s[2 * u + 1]);
+                    tmem_st8u(tq + COL_SB + (col0 >> 1), w);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                cbar();
+                if (issuer) {
+                    tc_fence_after();
+                    issue_u(0);
+                }
+            }
+            int u_issued = 1;                 // chunks whose U^T MMAs have been issued
+            for (int c = 0; c < nchunks && alive; ++c) {
+                const int b = c & 1;
+                const bool last = (c == nchunks - 1);
+                const uint32_t sl = sb + slot_base(c);
+                // ---- E^T = U^T - S Wm2^T (commit), O^T = S Qtil2^T ----------------------------
+                if (issuer) {
+                    bool ok = true;
+                    if (u_issued <= c) {
+                        ok = mbar_wait_bounded(bar_full + b, (c >> 1) & 1, x.wait_limit_ns);
+                        if (ok) {
+                            tc_fence_after();
+                            issue_u(c);
+                            u_issued = c + 1;
+                        }
+                    }
+                    // the epilogue must have read O^T buffer b (chunk c - 2)
+                    if (ok && c >= 2) ok = mbar_wait_bounded(bar_ofree + b, ((c - 2) >> 1) & 1, x.wait_limit_ns);
+                    if (!ok) {
+                        atomicExch(abort_c, 1);
+                    } else {
+                        tc_fence_after();
+                        const uint32_t a0 = tbase + sbcol(c);
+                        const uint64_t dW = sdesc_sw128(sl + SL_W, 8192, 1024), dQ = sdesc_sw128(sl + SL_Q, 16, 1024);
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks)
+                            mma_bf16_ts(tbase + COL_E + b * 64, a0 + ks * 8, dW + (uint64_t)(ks * 2048 / 16), ID_NEG, 1);
+                        mma_commit(bar_e);
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks)
+                            mma_bf16_ts(tbase + COL_O + b * 64, a0 + ks * 8,
+                                        dQ + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) / 16), ID_KK, ks > 0);
+                    }
+                }
+                // ---- S <- S P_C while they run (no MMA reads or writes S now) ------------------
+                if (!mbar_wait_bounded(bar_full + b, (c >> 1) & 1, x.wait_limit_ns)) atomicExch(abort_c, 1);
+                {
+                    const float* rt = reinterpret_cast<const float*>(base + slot_base(c) + SL_VEC) + 64;
+#pragma unroll 1
+                    for (int g = 0; g < 4; ++g) {
+                        float s32[32];
+                        tmem_ld32(tq + COL_S + g * 32, s32);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            float s16[16];
+#pragma unroll
+                            for (int u = 0; u < 16; ++u) s16[u] = s32[hh * 16 + u];
+                            scale_cols(g * 32 + hh * 16, s16, rt);
+                            tmem_st16(tq + COL_S + g * 32 + hh * 16, s16);
+                        }
+                    }
+                    tmem_wait_st();
+                }
+                if (!wait_all(bar_e, c & 1)) break;
+                // ---- E^T (fp32) -> bf16 in place, as the A operand ----------------------------
+                {
+                    const uint32_t col = COL_E + b * 64;
+                    uint32_t w[32];
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        float vals[32];
+                        tmem_ld32(tq + col + g * 32, vals);
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) w[g * 16 + u] = pack_bf16x2(vals[2 * u], vals[2 * u + 1]);
+                    }
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) tmem_st8u(tq + col + g * 8, *reinterpret_cast<uint32_t(*)[8]>(w + g * 8));
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                cbar();
+                // ---- S += E^T Khat2 (commit), O^T += E^T Pm^T (commit) -------------------------
+                if (issuer) {
+                    tc_fence_after();
+                    const uint64_t dH = sdesc_sw128(sl + SL_KH, 8192, 1024), dP = sdesc_sw128(sl + SL_PM, 16, 1024);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ts(tbase + COL_S, tbase + COL_E + b * 64 + ks * 8, dH + (uint64_t)(ks * 2048 / 16),
+                                    ID_KM128, 1);
+                    mma_commit(bar_s);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ts(tbase + COL_O + b * 64, tbase + COL_E + b * 64 + ks * 8, dP + (uint64_t)(ks * 32 / 16),
+                                    ID_KK, 1);
+                    mma_commit(bar_o + b);
+                    // the next chunk's U^T, if its slot is already here
+                    if (!last && mbar_test_wait(bar_full + (b ^ 1), ((c + 1) >> 1) & 1)) {
+                        tc_fence_after();
+                        issue_u(c + 1);
+                        u_issued = c + 2;
+                    }
+                }
+                if (!wait_all(bar_s, c & 1)) break;
+                // ---- S -> bf16 copy for the next chunk; the last chunk writes S_T --------------
+#pragma unroll 1
+                for (int g = 0; g < 4; ++g) {
+                    float s32[32];
+                    tmem_ld32(tq + COL_S + g * 32, s32);
+                    if (last) {
+                        if (p.S_T) {
+                            float4* dst = reinterpret_cast<float4*>(p.S_T + ((size_t)bh * D + row) * D + g * 32);
+#pragma unroll
+                            for (int u4 = 0; u4 < 8; ++u4)
+                                dst[u4] = make_float4(s32[4 * u4], s32[4 * u4 + 1], s32[4 * u4 + 2], s32[4 * u4 + 3]);
+                        }
+                    } else {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) w[u] = pack_bf16x2(s32[2 * u], s32[2 * u + 1]);
+                        tmem_st8u(tq + sbcol(c + 1) + g * 16, *reinterpret_cast<uint32_t(*)[8]>(w));
+                        tmem_st8u(tq + sbcol(c + 1) + g * 16 + 8, *reinterpret_cast<uint32_t(*)[8]>(w + 8));
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                cbar();
+            }
+        } else {
+            // ---------------- o epilogue: O^T (lane = value row, column = token) -> o ---------------
+            const int et = tid - (NPREP - 128);
+            auto ebar = [&]() { named_bar(4, 128); };
+            OT* stg = reinterpret_cast<OT*>(base + OFF_OSTG);
+            for (int c = 0; c < nchunks; ++c) {
+                const int b = c & 1;
+                if (!mbar_wait_bounded(bar_o + b, (c >> 1) & 1, x.wait_limit_ns)) atomicExch(abort_c, 1);
+                ebar();
+                if (*abort_c) break;
+                tc_fence_after();
+                if (et == 0) {
+                    mbar_arrive(bar_empty + b);     // every MMA that read ring slot b is done
+                    bulk_wait_read_all();           // the previous o store has read the staging
+                }
+                ebar();
+#pragma unroll 1
+                for (int g = 0; g < 2; ++g) {
+                    float vals[32];
+                    tmem_ld32(tq + COL_O + b * 64 + g * 32, vals);
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) st_from_f32(stg + (g * 32 + u) * D + row, vals[u]);
+                }
+                tc_fence_before();
+                fence_proxy_async_smem();
+                ebar();
+                if (et == 0) {
+                    mbar_arrive(bar_ofree + b);
+                    tma_store_4d(&tm.o, 0, bh % p.H, c * C, bh / p.H, sb + OFF_OSTG);   // rows past T clipped
+                    bulk_commit();
+                }
+            }
+            if (et == 0) bulk_wait_all();
+        }
+    } else if (MODE == 0 && nchunks > 0 && tid >= NPREP && tid < NPREP + CHAIN_THREADS && chain_cta) {
         // =========================== chain group ==================================
         const int row = tid - NPREP;          // TMEM lane = value row of S (quad = warp & 3)
         uint32_t mma_phase = 0;
@@ -1066,21 +1392,6 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
         }
     }
-    if (MODE == 1 && nchunks > 0 && !chain_cta && tid >= 2 * NPREP && (tid & 31) == 0) {
-        // ============ split mode: publisher of a prep group (one thread per group) ============
-        // The group's stores to a ring slot precede its bar_full arrival, so a gpu-scope fence
-        // here orders them before the release of the slot's ready flag.
-        const int grp = (tid - 2 * NPREP) >> 5;
-        const int W = 2 * ((int)gridDim.x - NH), wk = 2 * ((int)blockIdx.x - NH) + grp;
-        const int ntasks = (NH * nchunks - wk + W - 1) / W;
-        for (int it = 0; it < ntasks; ++it) {
-            const int task = wk + it * W, c = task / NH, bhx = task % NH;
-            if (!mbar_wait_bounded(bar_full + grp, it & 1, x.wait_limit_ns)) { atomicExch(abort_c, 1); break; }
-            __threadfence();
-            st_release_gpu(sa.ready + (size_t)bhx * RING + c % RING, (unsigned)(c + 1));
-        }
-    }
-
     if (nchunks == 0 && p.S_T && chain_cta) {
         for (int e = tid; e < D * D; e += nthreads<MODE>())
             p.S_T[(size_t)bh * D * D + e] = p.S0 ? p.S0[(size_t)bh * D * D + e] : 0.f;

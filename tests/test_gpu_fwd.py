@@ -221,10 +221,12 @@ def test_auto_picks_tensor_cores_for_bf16_d128(G):
     assert G.resolved_algo(d) == "simt"
 
 
-def test_split_matches_fused_bitwise_state_free_parts(G):
-    """The split kernel runs the same arithmetic as the fused one: identical outputs."""
-    import torch
-    p = I.make_fwd(2, 700, 3, 128, 128, dtype="bf16", seed=61, s0_std=0.2, rotation=True)
+@pytest.mark.parametrize("rotation", [False, True])
+def test_split_agrees_with_fused(G, rotation):
+    """The split kernel folds the reference decay into its ring tiles and keeps the plain
+    state, the fused one keeps the state prescaled: the same result up to rounding."""
+    p = I.make_fwd(2, 700, 3, 128, 128, dtype="bf16", seed=61, s0_std=0.2, rotation=rotation)
     o1, S1 = U.run_gpu_fwd(p, "tcgen05")
     o2, S2 = U.run_gpu_fwd(p, "tcgen05_split")
-    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    assert U.max_rel(U.o_to_f64(o2), U.o_to_f64(o1)) <= U.TOL_O["bf16"]
+    assert U.rel_l2(S2.cpu().numpy(), S1.cpu().numpy()) <= U.TOL_S
