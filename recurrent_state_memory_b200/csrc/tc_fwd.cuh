@@ -214,7 +214,8 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
     uint64_t* bar_empty = bar_pmma + 5;      // [2] chain -> prep: buffers of a chunk free
     uint64_t* bar_rho = bar_pmma + 7;        // [2] prep -> chain: decay vectors of a chunk ready;
                                              //     split workers: group g's staged inputs landed
-    uint64_t* bar_o = bar_pmma + 9;          // [2] split chain: O^T of a chunk complete (per buffer)
+    uint64_t* bar_o = bar_pmma + 9;          // split chain: O^T of a chunk complete
+    uint64_t* bar_wready = bar_pmma + 11;    // split chain: P_m Wm^T of a chunk converted into its slot
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_base + 96);
     int* abort_p = reinterpret_cast<int*>(bar_base + 100);
     int* abort_c = reinterpret_cast<int*>(bar_base + 104);
@@ -252,6 +253,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_pmma + i, 1);
             mbar_init(bar_o + i, 1);
+            if (i == 0) mbar_init(bar_wready, 1);
             // split chain CTAs: the loader's expect_tx arrival (plus the slot's and V's bytes)
             mbar_init(bar_full + i, (MODE == 1 && chain_cta) ? 1 : NPREP);
             mbar_init(bar_empty + i, (MODE == 1) ? 1 : CHAIN_THREADS);
@@ -333,12 +335,13 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 }
             }
         };
+        // One thread waits for the MMAs; the others wait at the named barrier (no issue slots)
+        // and order their tensor-memory reads after it with the fence.
         auto mma_wait = [&]() -> bool {
-            const bool ok = mbar_wait_bounded(g_pmma, mma_phase, x.wait_limit_ns);
+            if (tid == 0 && !mbar_wait_bounded(g_pmma, mma_phase, x.wait_limit_ns)) atomicExch(abort_p, 1);
             mma_phase ^= 1u;
-            if (!ok) atomicExch(abort_p, 1);
-            tc_fence_after();
             named_bar(gbar, NPREP);
+            tc_fence_after();
             return *abort_p == 0;
         };
         auto publish = [&]() {
@@ -608,6 +611,20 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                         }
                         *reinterpret_cast<uint2*>(ring + SL_Q + kb * 8192u + off) =
                             make_uint2(pack_bf16x2(q2[0], q2[1]), pack_bf16x2(q2[2], q2[3]));
+                        // Ktil2 = Ktil P_m^T, from which the chain CTA forms P_m Wm^T = Ktil2^T Tb^T
+                        if (!ROT) {
+#pragma unroll
+                            for (int d = 0; d < 4; ++d) q2[d] = kt[d] * rr[d];
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                const float a = kt[2 * j], b = kt[2 * j + 1];
+                                q2[2 * j] = a * rr[j] + b * rr[2 + j];
+                                q2[2 * j + 1] = b * rr[j] - a * rr[2 + j];
+                            }
+                        }
+                        *reinterpret_cast<uint2*>(ring + SL_W + kb * 8192u + off) =
+                            make_uint2(pack_bf16x2(q2[0], q2[1]), pack_bf16x2(q2[2], q2[3]));
                         *reinterpret_cast<uint2*>(ring + SL_KH + kb * 8192u + off) =
                             make_uint2(pack_bf16x2(k2[0], k2[1]), pack_bf16x2(k2[2], k2[3]));
                     }
@@ -843,49 +860,37 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 if (tid == 0 && it + 1 < ntasks) stage_part(it + 1, 1);          // A and Tm done
             }
 
-            // ---- U^T = V^T Tb^T -> E[c&1];  Wm^T = Ktil^T Tb^T -> A'/W columns -------------
-            if (tid == 0) {
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t bdesc = sdesc_sw128(((MODE == 0) ? sb + OFF_TB : gsb + G_TB) + ks * 32, 16, 1024);
-                    if (MODE == 0)
+            if (MODE == 1) {
+                // the Tb tile has been copied out: stage the next task's k over it
+                named_bar(gbar, NPREP);
+                if (tid == 0 && it + 1 < ntasks) stage_part(it + 1, 2);
+            }
+            if (MODE == 0) {
+                // ---- U^T = V^T Tb^T -> E[c&1];  Wm^T = Ktil^T Tb^T -> A'/W columns ---------
+                if (tid == 0) {
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t bdesc = sdesc_sw128(sb + OFF_TB + ks * 32, 16, 1024);
                         mma_bf16_ss(tbase + COL_E + bufi * 64, sdesc_sw128(sb + OFF_V + ks * 2048, 8192, 1024), bdesc,
                                     ID_MK, ks > 0);
-                    mma_bf16_ss(tbase + col_aw, sdesc_sw128(kq_s + ks * 2048, 16384, 1024), bdesc,
-                                ID_MK, ks > 0);
-                }
-                mma_commit(g_pmma);
-            }
-            if (!mma_wait()) break;
-            if (MODE == 1 && tid == 0 && it + 1 < ntasks) stage_part(it + 1, 2);   // Tb tile read
-
-            // Wm^T -> bf16 MN-major tile (row = dk, 64 tokens per row).
-            {
-                float vals[32];
-                tmem_ld16(tq + col_aw + half * 32, *reinterpret_cast<float(*)[16]>(vals));
-                tmem_ld16(tq + col_aw + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
-                uint8_t* W = (MODE == 0) ? base + OFF_W + bufi * 16384 : ring + SL_W;
-                if (MODE == 1) {        // Wm2^T = P_m Wm^T (row = dk index)
-                    if (!ROT) {
-                        const float f = vec[64 + row];
-#pragma unroll
-                        for (int u = 0; u < 32; ++u) vals[u] *= f;
-                    } else {            // rows 2j, 2j+1: (w0 + i w1) conj(P_m)
-                        const float cr = vec[64 + (row >> 1)], ci = vec[64 + 128 + (row >> 1)];
-                        const float sgn = (row & 1) ? -1.f : 1.f;
-#pragma unroll
-                        for (int u = 0; u < 32; ++u) {
-                            const float other = __shfl_xor_sync(0xffffffffu, vals[u], 1);
-                            vals[u] = vals[u] * cr + sgn * other * ci;
-                        }
+                        mma_bf16_ss(tbase + col_aw, sdesc_sw128(kq_s + ks * 2048, 16384, 1024), bdesc, ID_MK, ks > 0);
                     }
+                    mma_commit(g_pmma);
                 }
+                if (!mma_wait()) break;
+                // Wm^T -> bf16 MN-major tile (row = dk, 64 tokens per row).
+                {
+                    float vals[32];
+                    tmem_ld16(tq + col_aw + half * 32, *reinterpret_cast<float(*)[16]>(vals));
+                    tmem_ld16(tq + col_aw + half * 32 + 16, *reinterpret_cast<float(*)[16]>(vals + 16));
+                    uint8_t* W = base + OFF_W + bufi * 16384;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc)
-                    *reinterpret_cast<uint4*>(W + sw128_off(row, half * 4 + cc)) = pack8(vals + cc * 8);
+                    for (int cc = 0; cc < 4; ++cc)
+                        *reinterpret_cast<uint4*>(W + sw128_off(row, half * 4 + cc)) = pack8(vals + cc * 8);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(gbar, NPREP);
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(gbar, NPREP);
             if (MODE == 0) mbar_arrive(bar_full + bufi);
             if (MODE == 1) { pub_c = c; pub_bh = bhx; }
         }
@@ -894,18 +899,24 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         // after an early exit, let staging copies still in flight land before the CTA ends
         if (MODE == 1 && tid == 0 && staged > landed) (void)mbar_wait_bounded(g_stage, landed & 1, x.wait_limit_ns);
     } else if (MODE == 1 && nchunks > 0 && chain_cta && tid >= NPREP - 128 && tid < NPREP + CHAIN_THREADS) {
-        // ============ split mode: chain (warps 8-11) and o epilogue (warps 4-7) ==================
+        // ============ split mode: chain (warps 8-11) and helper warps 4-7 ======================
         // The chain keeps the plain state S (fp32) in TMEM and its bf16 copy in one of two column
         // blocks (chunk parity); the workers fold the reference decay into the ring's tiles
-        // (Qtil2 = Qtil P_m^T, Wm2^T = P_m Wm^T, Khat2 = Khat P_m^{-1} P_C), so per chunk
-        //   E^T = U^T - S Wm2^T,   O^T = S Qtil2^T + E^T Pm^T,   S <- S P_C + E^T Khat2,
-        // and the decay S P_C runs while the E^T MMAs do, off the state's critical path.
-        // MMA completions: bar_cmma (E^T), bar_pmma[0] (state), bar_o[b] (O^T of buffer b);
-        // the epilogue frees O^T buffer b through bar_rho[b] and ring slot b through bar_empty[b].
+        // (Qtil2 = Qtil P_m^T, Ktil2 = Ktil P_m^T, Khat2 = Khat P_m^{-1} P_C), so per chunk
+        //   Wm2^T = Ktil2^T Tb^T,   E^T = U^T - S Wm2^T,   O^T = S Qtil2^T + E^T Pm^T,
+        //   S <- S P_C + E^T Khat2,
+        // and the decay S P_C runs while the E^T MMAs do, off the state's critical path.  The
+        // helper warps turn each chunk's Wm2^T (TMEM) into the bf16 tile the E^T MMA reads (in
+        // the slot, over Ktil2) and write o.
+        // MMA completions: bar_cmma (E^T), bar_pmma[0] (state), bar_o (O^T), bar_rho[1] (Wm2^T);
+        // the helpers free O^T through bar_rho[0], ring slot b through bar_empty[b], and report
+        // a converted Wm2^T tile through bar_wready.
         const int row = quad * 32 + lane;
+        constexpr uint32_t COL_WS = COL_O + 64;     // Wm2^T scratch (O^T is single-buffered here)
         uint64_t* bar_e = bar_cmma;
         uint64_t* bar_s = bar_pmma;
         uint64_t* bar_ofree = bar_rho;
+        uint64_t* bar_w = bar_rho + 1;
         const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_NEG = idesc_bf16(128, 64, 0, 1, 1);
         const uint32_t ID_KM128 = idesc_bf16(128, 128, 0, 1, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
         auto sbcol = [](int c) -> uint32_t { return (c & 1) ? COL_AW : COL_SB; };
@@ -931,21 +942,28 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             // ---------------- chain: one thread per TMEM lane, tid NPREP issues the MMAs ----------
             const bool issuer = (tid == NPREP);
             auto cbar = [&]() { named_bar(2, CHAIN_THREADS); };
+            // MMA completions: one thread waits, the others at the named barrier
             auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-                const bool ok = mbar_wait_bounded(bar, parity, x.wait_limit_ns);
-                if (!ok) atomicExch(abort_c, 1);
+                if (issuer && !mbar_wait_bounded(bar, parity, x.wait_limit_ns)) atomicExch(abort_c, 1);
                 cbar();
                 tc_fence_after();
                 return *abort_c == 0;
             };
-            auto issue_u = [&](int c) {       // U^T = V^T Tb^T -> E^T buffer of chunk c
+            // U^T = V^T Tb^T -> E^T buffer of chunk c;  Wm2^T = Ktil2^T Tb^T -> scratch (commit)
+            auto issue_slot_mmas = [&](int c) {
                 const uint32_t sl = sb + slot_base(c);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tbase + COL_E + (c & 1) * 64, sdesc_sw128(sl + SL_V + ks * 2048, 8192, 1024),
-                                sdesc_sw128(sl + SL_TB + ks * 32, 16, 1024), ID_MK, ks > 0);
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t dTb = sdesc_sw128(sl + SL_TB + ks * 32, 16, 1024);
+                    mma_bf16_ss(tbase + COL_E + (c & 1) * 64, sdesc_sw128(sl + SL_V + ks * 2048, 8192, 1024), dTb,
+                                ID_MK, ks > 0);
+                    mma_bf16_ss(tbase + COL_WS, sdesc_sw128(sl + SL_W + ks * 2048, 8192, 1024), dTb, ID_MK, ks > 0);
+                }
+                mma_commit(bar_w);
             };
-            bool alive = wait_all(bar_full + 0, 0);
+            if (!mbar_wait_bounded(bar_full + 0, 0, x.wait_limit_ns)) atomicExch(abort_c, 1);
+            cbar();
+            bool alive = *abort_c == 0;
             if (alive) {
                 // S_0 (fp32) and its bf16 copy
 #pragma unroll 1
@@ -974,10 +992,10 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 cbar();
                 if (issuer) {
                     tc_fence_after();
-                    issue_u(0);
+                    issue_slot_mmas(0);
                 }
             }
-            int u_issued = 1;                 // chunks whose U^T MMAs have been issued
+            int u_issued = 1;                 // chunks whose U^T / Wm2^T MMAs have been issued
             for (int c = 0; c < nchunks && alive; ++c) {
                 const int b = c & 1;
                 const bool last = (c == nchunks - 1);
@@ -989,12 +1007,13 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                         ok = mbar_wait_bounded(bar_full + b, (c >> 1) & 1, x.wait_limit_ns);
                         if (ok) {
                             tc_fence_after();
-                            issue_u(c);
+                            issue_slot_mmas(c);
                             u_issued = c + 1;
                         }
                     }
-                    // the epilogue must have read O^T buffer b (chunk c - 2)
-                    if (ok && c >= 2) ok = mbar_wait_bounded(bar_ofree + b, ((c - 2) >> 1) & 1, x.wait_limit_ns);
+                    // the helpers must have written this chunk's Wm2^T tile, and read O^T of c - 1
+                    if (ok) ok = mbar_wait_bounded(bar_wready, c & 1, x.wait_limit_ns);
+                    if (ok && c >= 1) ok = mbar_wait_bounded(bar_ofree, (c - 1) & 1, x.wait_limit_ns);
                     if (!ok) {
                         atomicExch(abort_c, 1);
                     } else {
@@ -1007,7 +1026,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                         mma_commit(bar_e);
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks)
-                            mma_bf16_ts(tbase + COL_O + b * 64, a0 + ks * 8,
+                            mma_bf16_ts(tbase + COL_O, a0 + ks * 8,
                                         dQ + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) / 16), ID_KK, ks > 0);
                     }
                 }
@@ -1059,13 +1078,12 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     mma_commit(bar_s);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16_ts(tbase + COL_O + b * 64, tbase + COL_E + b * 64 + ks * 8, dP + (uint64_t)(ks * 32 / 16),
-                                    ID_KK, 1);
-                    mma_commit(bar_o + b);
-                    // the next chunk's U^T, if its slot is already here
+                        mma_bf16_ts(tbase + COL_O, tbase + COL_E + b * 64 + ks * 8, dP + (uint64_t)(ks * 32 / 16), ID_KK, 1);
+                    mma_commit(bar_o);
+                    // the next chunk's U^T and Wm2^T, if its slot is already here
                     if (!last && mbar_test_wait(bar_full + (b ^ 1), ((c + 1) >> 1) & 1)) {
                         tc_fence_after();
-                        issue_u(c + 1);
+                        issue_slot_mmas(c + 1);
                         u_issued = c + 2;
                     }
                 }
@@ -1095,13 +1113,35 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 cbar();
             }
         } else {
-            // ---------------- o epilogue: O^T (lane = value row, column = token) -> o ---------------
+            // ---------------- helpers: Wm2^T tiles and o --------------------------------------------
             const int et = tid - (NPREP - 128);
             auto ebar = [&]() { named_bar(4, 128); };
             OT* stg = reinterpret_cast<OT*>(base + OFF_OSTG);
-            for (int c = 0; c < nchunks; ++c) {
+            // Wm2^T of chunk c (lane = dk row, 64 token columns) -> bf16 MN-major tile over Ktil2
+            auto convert_w = [&](int c) -> bool {
+                if (et == 0 && !mbar_wait_bounded(bar_w, c & 1, x.wait_limit_ns)) atomicExch(abort_c, 1);
+                ebar();
+                if (*abort_c) return false;
+                tc_fence_after();
+                uint8_t* W = base + slot_base(c) + SL_W;
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    float vals[32];
+                    tmem_ld32(tq + COL_WS + g * 32, vals);
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+                        *reinterpret_cast<uint4*>(W + sw128_off(row, g * 4 + cc)) = pack8(vals + cc * 8);
+                }
+                tc_fence_before();
+                fence_proxy_async_smem();
+                ebar();
+                if (et == 0) mbar_arrive(bar_wready);
+                return true;
+            };
+            bool ok = convert_w(0);
+            for (int c = 0; c < nchunks && ok; ++c) {
                 const int b = c & 1;
-                if (!mbar_wait_bounded(bar_o + b, (c >> 1) & 1, x.wait_limit_ns)) atomicExch(abort_c, 1);
+                if (et == 0 && !mbar_wait_bounded(bar_o, c & 1, x.wait_limit_ns)) atomicExch(abort_c, 1);
                 ebar();
                 if (*abort_c) break;
                 tc_fence_after();
@@ -1113,7 +1153,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
 #pragma unroll 1
                 for (int g = 0; g < 2; ++g) {
                     float vals[32];
-                    tmem_ld32(tq + COL_O + b * 64 + g * 32, vals);
+                    tmem_ld32(tq + COL_O + g * 32, vals);
 #pragma unroll
                     for (int u = 0; u < 32; ++u) st_from_f32(stg + (g * 32 + u) * D + row, vals[u]);
                 }
@@ -1121,10 +1161,11 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 fence_proxy_async_smem();
                 ebar();
                 if (et == 0) {
-                    mbar_arrive(bar_ofree + b);
+                    mbar_arrive(bar_ofree);
                     tma_store_4d(&tm.o, 0, bh % p.H, c * C, bh / p.H, sb + OFF_OSTG);   // rows past T clipped
                     bulk_commit();
                 }
+                if (c + 1 < nchunks) ok = convert_w(c + 1);
             }
             if (et == 0) bulk_wait_all();
         }
@@ -1135,12 +1176,11 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_NEG = idesc_bf16(128, 64, 0, 1, 1);
         const uint32_t ID_KM128 = idesc_bf16(128, 128, 0, 1, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
         auto cbar = [&]() { named_bar(2, CHAIN_THREADS); };
-        auto mma_wait = [&]() -> bool {
-            const bool ok = mbar_wait_bounded(bar_cmma, mma_phase, x.wait_limit_ns);
+        auto mma_wait = [&]() -> bool {      // one thread waits, the others at the barrier
+            if (row == 0 && !mbar_wait_bounded(bar_cmma, mma_phase, x.wait_limit_ns)) atomicExch(abort_c, 1);
             mma_phase ^= 1u;
-            if (!ok) atomicExch(abort_c, 1);
-            tc_fence_after();
             cbar();
+            tc_fence_after();
             return *abort_c == 0;
         };
         auto bounded = [&](uint64_t* bar, uint32_t parity) -> bool {
