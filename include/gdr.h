@@ -71,13 +71,16 @@ typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
 typedef enum { GDR_GATE_LOGDECAY = 0, GDR_GATE_NEG_SOFTPLUS = 1 } gdr_gate_mode;
 
 typedef enum {
-    GDR_ALGO_AUTO = 0,    /* tensor-core chunk kernel when supported, else SIMT */
+    GDR_ALGO_AUTO = 0,    /* tensor-core chunk kernel when supported (the split one when
+                             2*B*H <= SM count and T > 64), else SIMT */
     GDR_ALGO_SIMT = 1,    /* fp32 CUDA-core chunk-WY kernel (every supported shape) */
     GDR_ALGO_TCGEN05 = 2, /* tcgen05/TMEM chunk-WY kernel, one CTA per (batch, head):
                              bf16 q/k/v, dk = dv = 128 */
-    GDR_ALGO_TCGEN05_SPLIT = 3 /* same arithmetic; one CTA per head runs only the state chain
-                             while every other SM prepares chunks, handed over through a
-                             ring in the workspace (needs B*H < SM count; cooperative launch) */
+    GDR_ALGO_TCGEN05_SPLIT = 3 /* same method; one CTA per head runs only the state chain
+                             while every other SM prepares chunks (two at a time), handed
+                             over through a ring in the workspace (needs B*H < SM count;
+                             cooperative launch); results agree with GDR_ALGO_TCGEN05 to
+                             rounding */
 } gdr_algo;
 
 /* Shape and mode of one chunked forward call. */
@@ -115,7 +118,7 @@ GDR_API const char* gdr_last_error_detail(void);
 
 /* Bytes of device workspace gdr_chunk_fwd needs for this descriptor (0 = none;
  * the workspace argument may then be NULL).  Returns 0 for an invalid desc.  The split
- * tensor-core kernel needs B*H*3 ring slots of 84,224 bytes plus 16 bytes of flags per
+ * tensor-core kernel needs B*H*6 ring slots of 67,840 bytes plus 28 bytes of flags per
  * head; it resets the flags itself (on the call's stream) and the buffer may be reused
  * by later calls on the same stream.  Uses the current device's SM count when
  * desc->algo is GDR_ALGO_AUTO. */

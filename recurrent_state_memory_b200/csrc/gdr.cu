@@ -81,9 +81,12 @@ static int device_sm_count() {
 
 // The split kernel pays off while the heads leave most SMs to prep workers (each head's
 // chain needs about three workers to keep up) and there is more than one chunk.
+// The split kernel gives each head one chain CTA and shares the remaining SMs among prep
+// workers; with more than half of the SMs taken by chains, too few workers are left and the
+// fused kernel (prep and chain of a head in one CTA) is faster.
 static bool split_fits(const gdr_fwd_desc* d, int sms) {
     const long long nh = (long long)d->B * d->H;
-    return nh >= 1 && 4 * nh <= (long long)sms && d->T > 64;
+    return nh >= 1 && 2 * nh <= (long long)sms && d->T > 64;
 }
 
 // The algorithm a descriptor runs with: AUTO takes a tensor-core kernel when it supports

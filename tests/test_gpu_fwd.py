@@ -208,11 +208,12 @@ def test_auto_picks_tensor_cores_for_bf16_d128(G):
     d = G.fwd_desc(1, 1, 64, 128, 128, torch.bfloat16, torch.bfloat16)
     assert G.resolved_algo(d) == "tcgen05"                    # a single chunk: fused
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    d = G.fwd_desc(2, 16, 8192, 128, 128, torch.bfloat16, torch.bfloat16)
-    expect = "tcgen05_split" if 4 * 32 <= sms else "tcgen05"   # few heads: chain + prep workers
-    assert G.resolved_algo(d) == expect
-    if expect == "tcgen05_split":
-        assert G.workspace_bytes(d) >= 32 * 3 * 67840
+    for B, H in ((2, 16), (4, 16)):
+        d = G.fwd_desc(B, H, 8192, 128, 128, torch.bfloat16, torch.bfloat16)
+        expect = "tcgen05_split" if 2 * B * H <= sms else "tcgen05"   # chains + prep workers
+        assert G.resolved_algo(d) == expect
+        if expect == "tcgen05_split":
+            assert G.workspace_bytes(d) >= B * H * 6 * 67840
     d = G.fwd_desc(16, 12, 4096, 128, 128, torch.bfloat16, torch.bfloat16)
     assert G.resolved_algo(d) == "tcgen05"                    # many heads: fused
     d = G.fwd_desc(1, 1, 64, 64, 64, torch.bfloat16, torch.bfloat16)
