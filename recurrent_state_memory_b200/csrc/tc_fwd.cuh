@@ -216,10 +216,12 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                                              //     split workers: group g's staged inputs landed
     uint64_t* bar_o = bar_pmma + 9;          // split chain: O^T of a chunk complete
     uint64_t* bar_wready = bar_pmma + 11;    // split chain: P_m Wm^T of a chunk converted into its slot
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_base + 96);
-    int* abort_p = reinterpret_cast<int*>(bar_base + 100);
-    int* abort_c = reinterpret_cast<int*>(bar_base + 104);
-    int* range_flag = reinterpret_cast<int*>(bar_base + 108);
+    uint64_t* bar_sbr = bar_pmma + 10;       // split chain: bf16 state of the next chunk written
+    uint64_t* bar_ecv = bar_pmma + 12;       // split chain: E^T converted and S decayed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_base + 112);
+    int* abort_p = reinterpret_cast<int*>(bar_base + 116);
+    int* abort_c = reinterpret_cast<int*>(bar_base + 120);
+    int* range_flag = reinterpret_cast<int*>(bar_base + 124);
     auto vecs = [&](int c) -> float* { return reinterpret_cast<float*>(base + OFF_VEC) + (c & 1) * VEC_FLOATS; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -253,7 +255,10 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_pmma + i, 1);
             mbar_init(bar_o + i, 1);
-            if (i == 0) mbar_init(bar_wready, 1);
+            if (i == 0) {
+                mbar_init(bar_wready, 1);
+                mbar_init(bar_ecv, 1);
+            }
             // split chain CTAs: the loader's expect_tx arrival (plus the slot's and V's bytes)
             mbar_init(bar_full + i, (MODE == 1 && chain_cta) ? 1 : NPREP);
             mbar_init(bar_empty + i, (MODE == 1) ? 1 : CHAIN_THREADS);
@@ -898,7 +903,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         if (bad) atomicExch(range_flag, 1);
         // after an early exit, let staging copies still in flight land before the CTA ends
         if (MODE == 1 && tid == 0 && staged > landed) (void)mbar_wait_bounded(g_stage, landed & 1, x.wait_limit_ns);
-    } else if (MODE == 1 && nchunks > 0 && chain_cta && tid >= NPREP - 128 && tid < NPREP + CHAIN_THREADS) {
+    } else if (MODE == 1 && nchunks > 0 && chain_cta && tid >= NPREP - 128 && tid <= NPREP + CHAIN_THREADS) {
         // ============ split mode: chain (warps 8-11) and helper warps 4-7 ======================
         // The chain keeps the plain state S (fp32) in TMEM and its bf16 copy in one of two column
         // blocks (chunk parity); the workers fold the reference decay into the ring's tiles
@@ -908,9 +913,12 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         // and the decay S P_C runs while the E^T MMAs do, off the state's critical path.  The
         // helper warps turn each chunk's Wm2^T (TMEM) into the bf16 tile the E^T MMA reads (in
         // the slot, over Ktil2) and write o.
-        // MMA completions: bar_cmma (E^T), bar_pmma[0] (state), bar_o (O^T), bar_rho[1] (Wm2^T);
-        // the helpers free O^T through bar_rho[0], ring slot b through bar_empty[b], and report
-        // a converted Wm2^T tile through bar_wready.
+        // One thread (warp 12, lane 0) issues every MMA, so that the state warps never wait for
+        // an issue queue.  MMA completions: bar_cmma (E^T), bar_pmma[0] (state), bar_o (O^T),
+        // bar_rho[1] (Wm2^T); the state warps report the next bf16 state through bar_sbr and a
+        // converted E^T (with S decayed) through bar_ecv; the helpers free O^T through
+        // bar_rho[0], ring slot b through bar_empty[b], and report a converted Wm2^T tile
+        // through bar_wready.
         const int row = quad * 32 + lane;
         constexpr uint32_t COL_WS = COL_O + 64;     // Wm2^T scratch (O^T is single-buffered here)
         uint64_t* bar_e = bar_cmma;
@@ -938,30 +946,85 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 }
             }
         };
-        if (tid >= NPREP) {
-            // ---------------- chain: one thread per TMEM lane, tid NPREP issues the MMAs ----------
-            const bool issuer = (tid == NPREP);
+        // U^T = V^T Tb^T -> E^T buffer of chunk c;  Wm2^T = Ktil2^T Tb^T -> scratch (commit)
+        auto issue_slot_mmas = [&](int c) {
+            const uint32_t sl = sb + slot_base(c);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t dTb = sdesc_sw128(sl + SL_TB + ks * 32, 16, 1024);
+                mma_bf16_ss(tbase + COL_E + (c & 1) * 64, sdesc_sw128(sl + SL_V + ks * 2048, 8192, 1024), dTb,
+                            ID_MK, ks > 0);
+                mma_bf16_ss(tbase + COL_WS, sdesc_sw128(sl + SL_W + ks * 2048, 8192, 1024), dTb, ID_MK, ks > 0);
+            }
+            mma_commit(bar_w);
+        };
+        if (tid == NPREP + CHAIN_THREADS) {
+            // ---------------- MMA issuer ------------------------------------------------------------
+            auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+                if (mbar_wait_bounded(bar, parity, x.wait_limit_ns) && *abort_c == 0) return true;
+                atomicExch(abort_c, 1);
+                return false;
+            };
+            int u_issued = 0;                 // chunks whose U^T / Wm2^T MMAs have been issued
+            for (int c = 0; c < nchunks; ++c) {
+                const int b = c & 1;
+                const bool last = (c == nchunks - 1);
+                const uint32_t sl = sb + slot_base(c);
+                if (u_issued <= c) {
+                    if (!wait(bar_full + b, (c >> 1) & 1)) break;
+                    tc_fence_after();
+                    issue_slot_mmas(c);
+                    u_issued = c + 1;
+                }
+                // the state's bf16 copy, this chunk's Wm2^T tile, and O^T read by the helpers
+                if (!wait(bar_sbr, c & 1) || !wait(bar_wready, c & 1)) break;
+                if (c >= 1 && !wait(bar_ofree, (c - 1) & 1)) break;
+                tc_fence_after();
+                {   // E^T = U^T - S Wm2^T (commit), O^T = S Qtil2^T
+                    const uint32_t a0 = tbase + sbcol(c);
+                    const uint64_t dW = sdesc_sw128(sl + SL_W, 8192, 1024), dQ = sdesc_sw128(sl + SL_Q, 16, 1024);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16_ts(tbase + COL_E + b * 64, a0 + ks * 8, dW + (uint64_t)(ks * 2048 / 16), ID_NEG, 1);
+                    mma_commit(bar_e);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16_ts(tbase + COL_O, a0 + ks * 8, dQ + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) / 16),
+                                    ID_KK, ks > 0);
+                }
+                if (!wait(bar_ecv, c & 1)) break;
+                tc_fence_after();
+                {   // S += E^T Khat2 (commit), O^T += E^T Pm^T (commit)
+                    const uint64_t dH = sdesc_sw128(sl + SL_KH, 8192, 1024), dP = sdesc_sw128(sl + SL_PM, 16, 1024);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ts(tbase + COL_S, tbase + COL_E + b * 64 + ks * 8, dH + (uint64_t)(ks * 2048 / 16),
+                                    ID_KM128, 1);
+                    mma_commit(bar_s);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ts(tbase + COL_O, tbase + COL_E + b * 64 + ks * 8, dP + (uint64_t)(ks * 32 / 16), ID_KK, 1);
+                    mma_commit(bar_o);
+                }
+                // the next chunk's U^T and Wm2^T, if its slot is already here
+                if (!last && mbar_test_wait(bar_full + (b ^ 1), ((c + 1) >> 1) & 1)) {
+                    tc_fence_after();
+                    issue_slot_mmas(c + 1);
+                    u_issued = c + 2;
+                }
+            }
+        } else if (tid >= NPREP) {
+            // ---------------- state warps: one thread per TMEM lane -----------------------------------
+            const bool lead = (tid == NPREP);
             auto cbar = [&]() { named_bar(2, CHAIN_THREADS); };
             // MMA completions: one thread waits, the others at the named barrier
             auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-                if (issuer && !mbar_wait_bounded(bar, parity, x.wait_limit_ns)) atomicExch(abort_c, 1);
+                if (lead && !mbar_wait_bounded(bar, parity, x.wait_limit_ns)) atomicExch(abort_c, 1);
                 cbar();
                 tc_fence_after();
                 return *abort_c == 0;
             };
-            // U^T = V^T Tb^T -> E^T buffer of chunk c;  Wm2^T = Ktil2^T Tb^T -> scratch (commit)
-            auto issue_slot_mmas = [&](int c) {
-                const uint32_t sl = sb + slot_base(c);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t dTb = sdesc_sw128(sl + SL_TB + ks * 32, 16, 1024);
-                    mma_bf16_ss(tbase + COL_E + (c & 1) * 64, sdesc_sw128(sl + SL_V + ks * 2048, 8192, 1024), dTb,
-                                ID_MK, ks > 0);
-                    mma_bf16_ss(tbase + COL_WS, sdesc_sw128(sl + SL_W + ks * 2048, 8192, 1024), dTb, ID_MK, ks > 0);
-                }
-                mma_commit(bar_w);
-            };
-            if (!mbar_wait_bounded(bar_full + 0, 0, x.wait_limit_ns)) atomicExch(abort_c, 1);
+            if (lead && !mbar_wait_bounded(bar_full + 0, 0, x.wait_limit_ns)) atomicExch(abort_c, 1);
             cbar();
             bool alive = *abort_c == 0;
             if (alive) {
@@ -990,47 +1053,12 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 tmem_wait_st();
                 tc_fence_before();
                 cbar();
-                if (issuer) {
-                    tc_fence_after();
-                    issue_slot_mmas(0);
-                }
+                if (lead) mbar_arrive(bar_sbr);
             }
-            int u_issued = 1;                 // chunks whose U^T / Wm2^T MMAs have been issued
             for (int c = 0; c < nchunks && alive; ++c) {
                 const int b = c & 1;
                 const bool last = (c == nchunks - 1);
-                const uint32_t sl = sb + slot_base(c);
-                // ---- E^T = U^T - S Wm2^T (commit), O^T = S Qtil2^T ----------------------------
-                if (issuer) {
-                    bool ok = true;
-                    if (u_issued <= c) {
-                        ok = mbar_wait_bounded(bar_full + b, (c >> 1) & 1, x.wait_limit_ns);
-                        if (ok) {
-                            tc_fence_after();
-                            issue_slot_mmas(c);
-                            u_issued = c + 1;
-                        }
-                    }
-                    // the helpers must have written this chunk's Wm2^T tile, and read O^T of c - 1
-                    if (ok) ok = mbar_wait_bounded(bar_wready, c & 1, x.wait_limit_ns);
-                    if (ok && c >= 1) ok = mbar_wait_bounded(bar_ofree, (c - 1) & 1, x.wait_limit_ns);
-                    if (!ok) {
-                        atomicExch(abort_c, 1);
-                    } else {
-                        tc_fence_after();
-                        const uint32_t a0 = tbase + sbcol(c);
-                        const uint64_t dW = sdesc_sw128(sl + SL_W, 8192, 1024), dQ = sdesc_sw128(sl + SL_Q, 16, 1024);
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks)
-                            mma_bf16_ts(tbase + COL_E + b * 64, a0 + ks * 8, dW + (uint64_t)(ks * 2048 / 16), ID_NEG, 1);
-                        mma_commit(bar_e);
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks)
-                            mma_bf16_ts(tbase + COL_O, a0 + ks * 8,
-                                        dQ + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) / 16), ID_KK, ks > 0);
-                    }
-                }
-                // ---- S <- S P_C while they run (no MMA reads or writes S now) ------------------
+                // ---- S <- S P_C while E^T is formed (no MMA reads or writes S now) ------------
                 if (!mbar_wait_bounded(bar_full + b, (c >> 1) & 1, x.wait_limit_ns)) atomicExch(abort_c, 1);
                 {
                     const float* rt = reinterpret_cast<const float*>(base + slot_base(c) + SL_VEC) + 64;
@@ -1067,26 +1095,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 }
                 tc_fence_before();
                 cbar();
-                // ---- S += E^T Khat2 (commit), O^T += E^T Pm^T (commit) -------------------------
-                if (issuer) {
-                    tc_fence_after();
-                    const uint64_t dH = sdesc_sw128(sl + SL_KH, 8192, 1024), dP = sdesc_sw128(sl + SL_PM, 16, 1024);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16_ts(tbase + COL_S, tbase + COL_E + b * 64 + ks * 8, dH + (uint64_t)(ks * 2048 / 16),
-                                    ID_KM128, 1);
-                    mma_commit(bar_s);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16_ts(tbase + COL_O, tbase + COL_E + b * 64 + ks * 8, dP + (uint64_t)(ks * 32 / 16), ID_KK, 1);
-                    mma_commit(bar_o);
-                    // the next chunk's U^T and Wm2^T, if its slot is already here
-                    if (!last && mbar_test_wait(bar_full + (b ^ 1), ((c + 1) >> 1) & 1)) {
-                        tc_fence_after();
-                        issue_slot_mmas(c + 1);
-                        u_issued = c + 2;
-                    }
-                }
+                if (lead) mbar_arrive(bar_ecv);
                 if (!wait_all(bar_s, c & 1)) break;
                 // ---- S -> bf16 copy for the next chunk; the last chunk writes S_T --------------
 #pragma unroll 1
@@ -1111,6 +1120,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 tmem_wait_st();
                 tc_fence_before();
                 cbar();
+                if (lead && !last) mbar_arrive(bar_sbr);
             }
         } else {
             // ---------------- helpers: Wm2^T tiles and o --------------------------------------------
