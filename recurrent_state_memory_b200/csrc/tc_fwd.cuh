@@ -83,15 +83,14 @@ constexpr uint32_t SLOT_BYTES = SL_VEC + VEC_FLOATS * 4;        // bytes of one 
 // itself from the input (MN-major: 2 groups x 64 tokens x 128 B).
 constexpr uint32_t SL_V = (SLOT_BYTES + 1023) & ~1023u;
 constexpr uint32_t SLOT_STRIDE = SL_V + 16384;                  // slot buffers in the chain CTA
-constexpr int RING = 6;               // ring slots per head
+constexpr int RING = 8;               // ring slots per head
 // Split chain CTAs stage each chunk's o here ([64 tokens][128] in the output type) and
 // store it with one tensor-map tile store.
 constexpr uint32_t OFF_OSTG = 2 * SLOT_STRIDE;
 // Split-mode prep workers run two independent groups of 8 warps, each with its own tiles
 // (bytes from the group's base, group g at g * G_STRIDE).  A group stages the raw inputs of
-// its next task into tiles that the current task no longer needs: q into G_KH (free after
-// MMA1), the gates (and angles) into G_AF..G_TF (free after the solve), k into G_TB..G_QT
-// (free after the Wm MMA).
+// its next task into tiles that the current task no longer needs: q into G_KH and the gates
+// (and angles) into G_KQ once MMA1 has read them, k into G_AF once the solve is done.
 constexpr uint32_t G_KQ = 0;         // [Ktil ; Qtil] K-major: 2 kblocks x 128 rows x 128 B
 constexpr uint32_t G_KH = 32768;     // Khat K-major: 2 kblocks x 64 rows x 128 B
 constexpr uint32_t G_TB = 49152;     // Tb K-major: 64 rows x 128 B
@@ -103,7 +102,7 @@ constexpr uint32_t G_STRIDE = (G_VEC + VEC_FLOATS * 4 + 1023) & ~1023u;
 constexpr int NT_SPLIT = 2 * NPREP;             // two prep groups (16 warps: 128 registers a thread)
 constexpr uint32_t OFF_BAR_SPLIT = 2 * G_STRIDE;
 static_assert(2 * SLOT_STRIDE + 64 * 128 * 4 <= OFF_BAR_SPLIT, "chain slot buffers overlap the barriers");
-static_assert(G_TF + 64 * AS * 4 >= G_AF + 32768, "gate staging does not fit in A and Tm");
+static_assert(G_KH - G_KQ >= 32768 && 64 * AS * 4 >= 16384, "staging does not fit");
 
 template <int MODE> __host__ __device__ constexpr int nthreads() { return MODE == 0 ? NT : NT_SPLIT; }
 template <int MODE> __host__ __device__ constexpr uint32_t off_bar() { return MODE == 0 ? OFF_BAR : OFF_BAR_SPLIT; }
@@ -361,11 +360,10 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         // Split: the ring slot of a finished task is published by the group's thread 32 once
         // the next task's inputs have been read (or after the last task), while the other warps
         // run pass 1; the named barriers order every thread's stores to the slot before its
-        // gpu-scope fence and release.  Publishing before the next task's ring-slot wait keeps
-        // the workers free of waits on one another.
+        // gpu-scope release (cumulative over what the thread has observed).  Publishing before
+        // the next task's ring-slot wait keeps the workers free of waits on one another.
         int pub_c = -1, pub_bh = 0;
         auto publish_slot = [&]() {
-            __threadfence();
             st_release_gpu(sa.ready + (size_t)pub_bh * RING + pub_c % RING, (unsigned)(pub_c + 1));
             pub_c = -1;
         };
@@ -377,10 +375,10 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 mbar_arrive_expect_tx(g_stage, 65536u);
                 tma_load_4d(gsb + G_KH, &tm.q, 0, hh, c2 * C, bb, g_stage);
             } else if (part == 1) {
-                tma_load_4d(gsb + G_AF, &tm.g, 0, hh, c2 * C, bb, g_stage);
-                if (ROT) tma_load_4d(gsb + G_AF + 16384u, &tm.th, 0, hh, c2 * C, bb, g_stage);
+                tma_load_4d(gsb + G_KQ, &tm.g, 0, hh, c2 * C, bb, g_stage);
+                if (ROT) tma_load_4d(gsb + G_KQ + 16384u, &tm.th, 0, hh, c2 * C, bb, g_stage);
             } else {
-                tma_load_4d(gsb + G_TB, &tm.k, 0, hh, c2 * C, bb, g_stage);
+                tma_load_4d(gsb + G_AF, &tm.k, 0, hh, c2 * C, bb, g_stage);
             }
         };
         const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
@@ -413,17 +411,16 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
 #pragma unroll
                 for (int s_ = 0; s_ < 8; ++s_) {
                     const int r = 8 * sg + s_;
-                    rk[s_] = *reinterpret_cast<const uint2*>(gb + G_TB + (uint32_t)(r * D + 4 * dg) * 2u);
+                    rk[s_] = *reinterpret_cast<const uint2*>(gb + G_AF + (uint32_t)(r * D + 4 * dg) * 2u);
                     rq[s_] = *reinterpret_cast<const uint2*>(gb + G_KH + (uint32_t)(r * D + 4 * dg) * 2u);
                     if (!ROT) {
-                        ra[s_] = *reinterpret_cast<const float4*>(gb + G_AF + (uint32_t)(r * D + 4 * dg) * 4u);
+                        ra[s_] = *reinterpret_cast<const float4*>(gb + G_KQ + (uint32_t)(r * D + 4 * dg) * 4u);
                     } else {
-                        const float2 g2 = *reinterpret_cast<const float2*>(gb + G_AF + (uint32_t)(r * 64 + 2 * dg) * 4u);
-                        const float2 t2 = *reinterpret_cast<const float2*>(gb + G_AF + 16384u + (uint32_t)(r * 64 + 2 * dg) * 4u);
+                        const float2 g2 = *reinterpret_cast<const float2*>(gb + G_KQ + (uint32_t)(r * 64 + 2 * dg) * 4u);
+                        const float2 t2 = *reinterpret_cast<const float2*>(gb + G_KQ + 16384u + (uint32_t)(r * 64 + 2 * dg) * 4u);
                         ra[s_] = make_float4(g2.x, g2.y, t2.x, t2.y);
                     }
                 }
-                named_bar(gbar, NPREP);      // pass 1 rewrites the k staging area (G_QT)
                 if (tid == 32 && pub_c >= 0) publish_slot();   // overlaps pass 1 of the other warps
             }
             float* sbeta = vec;
@@ -709,7 +706,10 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 skip_commit = false;
             }
             if (!mma_wait()) break;
-            if (MODE == 1 && tid == 0 && it + 1 < ntasks) stage_part(it + 1, 0);   // Khat tile read
+            if (MODE == 1 && tid == 0 && it + 1 < ntasks) {     // MMA1 has read the operand tiles
+                stage_part(it + 1, 0);
+                stage_part(it + 1, 1);
+            }
 
             // ---- solve: Tm = (I + A)^{-1}; Pm masked -> bf16 ---------------------------
             {
@@ -862,14 +862,9 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
 #pragma unroll
                 for (int e = 0; e < 2; ++e)
                     reinterpret_cast<uint4*>(ring + SL_TB)[tid + e * NPREP] = reinterpret_cast<const uint4*>(TB)[tid + e * NPREP];
-                if (tid == 0 && it + 1 < ntasks) stage_part(it + 1, 1);          // A and Tm done
+                if (tid == 0 && it + 1 < ntasks) stage_part(it + 1, 2);          // A and Tm done
             }
 
-            if (MODE == 1) {
-                // the Tb tile has been copied out: stage the next task's k over it
-                named_bar(gbar, NPREP);
-                if (tid == 0 && it + 1 < ntasks) stage_part(it + 1, 2);
-            }
             if (MODE == 0) {
                 // ---- U^T = V^T Tb^T -> E[c&1];  Wm^T = Ktil^T Tb^T -> A'/W columns ---------
                 if (tid == 0) {

@@ -213,7 +213,7 @@ def test_auto_picks_tensor_cores_for_bf16_d128(G):
         expect = "tcgen05_split" if 2 * B * H <= sms else "tcgen05"   # chains + prep workers
         assert G.resolved_algo(d) == expect
         if expect == "tcgen05_split":
-            assert G.workspace_bytes(d) >= B * H * 6 * 67840
+            assert G.workspace_bytes(d) >= B * H * 8 * 67840
     d = G.fwd_desc(16, 12, 4096, 128, 128, torch.bfloat16, torch.bfloat16)
     assert G.resolved_algo(d) == "tcgen05"                    # many heads: fused
     d = G.fwd_desc(1, 1, 64, 64, 64, torch.bfloat16, torch.bfloat16)
