@@ -3,8 +3,8 @@
 // The WY/UT-transform triangular chunk solver ("CARVE" page, section 1 item 3 and
 // section 3 item 1; "Semidirect Fourier Delta Attention" page, "Constructive Chunk-WY
 // Theorem" and the exact affine chunk transfer), bf16 operands, fp32 accumulation,
-// dk = dv = 128, chunk C = 64.  One CTA owns one (batch, head); the state S (dv x dk,
-// fp32) stays resident in tensor memory for the whole sequence.
+// dk = dv = 128, chunk C = 64.  One CTA owns the state chain of one (batch, head); the state
+// S (dv x dk, fp32) stays resident in tensor memory for the whole sequence.
 //
 // Per chunk, with P_r = D_1 ... D_r and the reference token m = 31 (the middle of the
 // chunk), every decay factor is split around P_m so that no factor exceeds the decay
@@ -18,8 +18,12 @@
 //   O^T += E^T Pm^T,   S_acc = Stil + E^T Khat                      (MMA, K = 64)
 //   S <- S_acc (P_m^{-1} P_C)
 // A tail chunk is padded with identity tokens (g = 0, beta = 0, k = q = v = 0).
+// The split kernel (MODE 1) evaluates the same chunk with the reference decay folded into the
+// operands its chain reads (Qtil2 = Qtil P_m^T, Ktil2 = Ktil P_m^T, Khat2 = Khat P_m^{-1} P_C),
+// so its chain keeps the plain state:
+//   Wm2^T = Ktil2^T Tb^T,  E^T = U^T - S Wm2^T,  O^T = S Qtil2^T + E^T Pm^T,  S <- S P_C + E^T Khat2.
 //
-// Warp roles (384 threads):
+// Warp roles of the fused kernel (384 threads):
 //   warps 0-7  "prep": gate activation and decay factors (register-prefetched inputs),
 //              the operand tiles, MMA1, the triangular solve, U^T / Wm^T.  They run up
 //              to two chunks ahead of the chain, through double-buffered tiles.
@@ -192,11 +196,12 @@ __device__ __forceinline__ uint4 pack8(const float* m8) {
                       pack_bf16x2(m8[4], m8[5]), pack_bf16x2(m8[6], m8[7]));
 }
 
-// MODE 0 (fused): one CTA per (batch, head) runs both groups.
-// MODE 1 (split): CTAs [0, B*H) run the chain of head blockIdx.x (warps 8-11) with a loader
-// warp that copies ring slots into shared memory; every other CTA is a prep worker whose
-// warps 0-7 compute chunks in chunk-major task order and whose warps 8-11 copy finished
-// operands into the ring.  The grid must be co-resident (cooperative launch).
+// MODE 0 (fused): one CTA per (batch, head) runs both groups (384 threads).
+// MODE 1 (split, 512 threads): CTAs [0, B*H) run the chain of head blockIdx.x: warp 0 copies
+// ring slots into shared memory, warp 12 lane 0 issues the MMAs, warps 8-11 run the state and
+// warps 4-7 convert the Wm tiles and write o.  Every other CTA is a prep worker with two
+// independent 8-warp groups that compute chunks in chunk-major task order and write their
+// operand tiles into the ring.  The grid must be co-resident (cooperative launch).
 template <int MODE, bool ROT, typename OT>
 __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdParams p, TcExtra x, SplitArgs sa,
                                                               const __grid_constant__ TmaMaps tm) {
