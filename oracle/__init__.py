@@ -30,9 +30,9 @@ def _load():
         path = _build.build()
         lib = ctypes.CDLL(path)
         dp = ctypes.POINTER(ctypes.c_double)
-        lib.oracle_gdr_fwd.argtypes = [ctypes.c_int] * 7 + [ctypes.c_double] + [dp] * 9
+        lib.oracle_gdr_fwd.argtypes = [ctypes.c_int] * 7 + [ctypes.c_double] + [dp] * 10
         lib.oracle_gdr_fwd.restype = None
-        lib.oracle_gdr_decode_step.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [dp] * 8
+        lib.oracle_gdr_decode_step.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [dp] * 9
         lib.oracle_gdr_decode_step.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -57,18 +57,20 @@ def num_threads() -> int:
 
 
 def gdr_fwd(q, k, v, g, beta, theta=None, S0=None, gate_mode=GATE_LOGDECAY, scale=1.0,
-            want_state=True):
+            want_state=True, w=None):
     """Token-by-token fp64 forward.
 
     q, k: [B,T,H,dk]; v: [B,T,H,dv]; g: [B,T,H,dk] (or dk/2 with rotation);
-    beta: [B,T,H]; theta: [B,T,H,dk/2] or None; S0: [B,H,dv,dk] or None.
+    beta: [B,T,H] erase strength; w: [B,T,H] write strength or None (w = beta);
+    theta: [B,T,H,dk/2] or None; S0: [B,H,dv,dk] or None.
     Returns (o [B,T,H,dv], S_T [B,H,dv,dk] or None), both float64.
     """
-    q, k, v, g, beta, theta, S0 = map(_f64, (q, k, v, g, beta, theta, S0))
+    q, k, v, g, beta, w, theta, S0 = map(_f64, (q, k, v, g, beta, w, theta, S0))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     rotation = theta is not None
     assert k.shape == q.shape and v.shape == (B, T, H, dv) and beta.shape == (B, T, H)
+    assert w is None or w.shape == (B, T, H)
     assert g.shape == (B, T, H, dk // 2 if rotation else dk)
     if rotation:
         assert dk % 2 == 0 and theta.shape == (B, T, H, dk // 2)
@@ -77,14 +79,15 @@ def gdr_fwd(q, k, v, g, beta, theta=None, S0=None, gate_mode=GATE_LOGDECAY, scal
     o = np.zeros((B, T, H, dv))
     S_T = np.zeros((B, H, dv, dk)) if want_state else None
     _load().oracle_gdr_fwd(B, T, H, dk, dv, int(gate_mode), int(rotation), float(scale),
-                           _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(theta),
+                           _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(w), _ptr(theta),
                            _ptr(S0), _ptr(o), _ptr(S_T))
     return o, S_T
 
 
-def gdr_decode_step(q, k, v, g, beta, S, theta=None, gate_mode=GATE_LOGDECAY, scale=1.0):
-    """One fp64 decode step.  S [N,H,dv,dk] is NOT modified; returns (o, S_new)."""
-    q, k, v, g, beta, theta = map(_f64, (q, k, v, g, beta, theta))
+def gdr_decode_step(q, k, v, g, beta, S, theta=None, gate_mode=GATE_LOGDECAY, scale=1.0, w=None):
+    """One fp64 decode step (w: write strength [N,H] or None for w = beta).
+    S [N,H,dv,dk] is NOT modified; returns (o, S_new)."""
+    q, k, v, g, beta, w, theta = map(_f64, (q, k, v, g, beta, w, theta))
     S_new = np.array(S, dtype=np.float64, copy=True, order="C")
     N, H, dk = q.shape
     dv = v.shape[-1]
@@ -92,6 +95,6 @@ def gdr_decode_step(q, k, v, g, beta, S, theta=None, gate_mode=GATE_LOGDECAY, sc
     assert g.shape == (N, H, dk // 2 if rotation else dk) and beta.shape == (N, H)
     o = np.zeros((N, H, dv))
     _load().oracle_gdr_decode_step(N, H, dk, dv, int(gate_mode), int(rotation), float(scale),
-                                   _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                   _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(w),
                                    _ptr(theta), _ptr(S_new), _ptr(o))
     return o, S_new

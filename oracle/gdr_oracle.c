@@ -8,9 +8,10 @@
  *
  * What it computes (one head of one sequence, tokens t = 1..T):
  *
- *   S_t = S_{t-1} D_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t (scale q_t)
+ *   S_t = S_{t-1} D_t (I - beta_t k_t k_t^T) + w_t v_t k_t^T,   o_t = S_t (scale q_t)
  *
- * with S_t in R^{dv x dk} (value rows, key columns).  Sources:
+ * with S_t in R^{dv x dk} (value rows, key columns), erase strength beta_t and write
+ * strength w_t (w_t = beta_t, the tied delta rule, unless a separate w is given).  Sources:
  *   - "Semidirect Fourier Delta Attention" page, section "Core architecture":
  *     the update decays first, then erases along k_t, then writes beta_t k_t v_t^*;
  *     the state there is the transpose of ours (dk x dv, acting from the left).
@@ -21,6 +22,10 @@
  *     D_t = diag(exp(g_t)) with g_t <= 0.
  *   - the readout o_t = S_t q_t uses the post-update state (the CARVE page
  *     writes S_{t-1} q_t in section 2.1; the benchmark spec fixes S_t).
+ *   - "CARVE" page, sections 2.1-2.2: an erase gate b_t and a separate scalar value
+ *     write gate w_{h,t} per head and token.  Read here as the erase strength that
+ *     multiplies the removal along k_t and the write strength that multiplies v_t k_t^T;
+ *     with both equal the update is the original delta rule (section 3, Theorem 1).
  *
  * The token step, in the order the SFDA page gives it (decay, erase, write):
  *   1. alpha = exp(g_t) per key dim (rotation mode: per key pair j, with angle
@@ -28,7 +33,7 @@
  *      number x + i y and multiplied by alpha e^{i theta}).  This is the
  *      transpose of Lambda_t acting on the left of the SFDA state.
  *   2. X = S D_t.
- *   3. e = beta_t (v_t - X k_t)                 (erase along k_t)
+ *   3. e = w_t v_t - beta_t X k_t              (erase along k_t, write v_t)
  *   4. S = X + e k_t^T                          (write)
  *   5. o_t = S (scale q_t)
  *
@@ -38,7 +43,7 @@
  *
  * Layouts (row-major, last index fastest):
  *   q, k [B,T,H,dk]; v, o [B,T,H,dv]; g [B,T,H,dk] ([B,T,H,dk/2] in rotation
- *   mode); beta [B,T,H]; theta [B,T,H,dk/2]; S0, S_T [B,H,dv,dk].
+ *   mode); beta, w [B,T,H]; theta [B,T,H,dk/2]; S0, S_T [B,H,dv,dk].
  * All arrays are double; bf16 or fp32 inputs are widened exactly by the caller.
  */
 #include <math.h>
@@ -62,7 +67,7 @@ static double oracle_log_decay(double g_in, int gate_mode)
  */
 static void oracle_token_step(int dk, int dv, int gate_mode, int rotation, double scale,
                               const double* q, const double* k, const double* v,
-                              const double* g, double beta, const double* theta,
+                              const double* g, double beta, double w, const double* theta,
                               double* S, double* o)
 {
     /* 1-2: X = S D_t, in place. */
@@ -88,7 +93,7 @@ static void oracle_token_step(int dk, int dv, int gate_mode, int rotation, doubl
         double* row = S + (size_t)i * dk;
         double xk = 0.0;
         for (int d = 0; d < dk; ++d) xk += row[d] * k[d];
-        double e = beta * (v[i] - xk);
+        double e = w * v[i] - beta * xk;
         for (int d = 0; d < dk; ++d) row[d] += e * k[d];
         double oq = 0.0;
         for (int d = 0; d < dk; ++d) oq += row[d] * (scale * q[d]);
@@ -97,12 +102,13 @@ static void oracle_token_step(int dk, int dv, int gate_mode, int rotation, doubl
 }
 
 /*
- * Whole-sequence forward, token by token.  S0 may be NULL (zero state);
- * S_T may be NULL (final state not wanted).  Heads run in parallel with OpenMP.
+ * Whole-sequence forward, token by token.  w may be NULL (w = beta); S0 may be
+ * NULL (zero state); S_T may be NULL (final state not wanted).  Heads run in
+ * parallel with OpenMP.
  */
 void oracle_gdr_fwd(int B, int T, int H, int dk, int dv, int gate_mode, int rotation,
                     double scale, const double* q, const double* k, const double* v,
-                    const double* g, const double* beta, const double* theta,
+                    const double* g, const double* beta, const double* w, const double* theta,
                     const double* S0, double* o, double* S_T)
 {
     const int ng = rotation ? dk / 2 : dk;
@@ -116,7 +122,7 @@ void oracle_gdr_fwd(int B, int T, int H, int dk, int dv, int gate_mode, int rota
             const size_t tok = ((size_t)b * T + t) * H + h;
             oracle_token_step(dk, dv, gate_mode, rotation, scale,
                               q + tok * dk, k + tok * dk, v + tok * dv,
-                              g + tok * ng, beta[tok],
+                              g + tok * ng, beta[tok], w ? w[tok] : beta[tok],
                               rotation ? theta + tok * (dk / 2) : NULL,
                               S, o + tok * dv);
         }
@@ -128,19 +134,20 @@ void oracle_gdr_fwd(int B, int T, int H, int dk, int dv, int gate_mode, int rota
 /*
  * One recurrent decode step for N independent sequences: S [N,H,dv,dk] is
  * updated in place; q, k [N,H,dk]; v, o [N,H,dv]; g [N,H,dk] (or dk/2);
- * beta [N,H]; theta [N,H,dk/2].  It is the same token step as the forward.
+ * beta, w [N,H] (w may be NULL: w = beta); theta [N,H,dk/2].  It is the same
+ * token step as the forward.
  */
 void oracle_gdr_decode_step(int N, int H, int dk, int dv, int gate_mode, int rotation,
                             double scale, const double* q, const double* k, const double* v,
-                            const double* g, const double* beta, const double* theta,
-                            double* S, double* o)
+                            const double* g, const double* beta, const double* w,
+                            const double* theta, double* S, double* o)
 {
     const int ng = rotation ? dk / 2 : dk;
 #pragma omp parallel for schedule(static)
     for (int nh = 0; nh < N * H; ++nh) {
         oracle_token_step(dk, dv, gate_mode, rotation, scale,
                           q + (size_t)nh * dk, k + (size_t)nh * dk, v + (size_t)nh * dv,
-                          g + (size_t)nh * ng, beta[nh],
+                          g + (size_t)nh * ng, beta[nh], w ? w[nh] : beta[nh],
                           rotation ? theta + (size_t)nh * (dk / 2) : NULL,
                           S + (size_t)nh * dv * dk, o + (size_t)nh * dv);
     }

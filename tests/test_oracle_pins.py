@@ -50,9 +50,11 @@ def _decay_by_complex(a_t, theta_t, dk):
     return D
 
 
-def _brute_head(q, k, v, a, beta, theta, S0, scale):
-    """S_t = S_0 prod_{s<=t} M_s + sum_{i<=t} beta_i v_i k_i^T prod_{i<s<=t} M_s with
-    M_s = D_s (I - beta_s k_s k_s^T), every product formed explicitly."""
+def _brute_head(q, k, v, a, beta, theta, S0, scale, w=None):
+    """S_t = S_0 prod_{s<=t} M_s + sum_{i<=t} w_i v_i k_i^T prod_{i<s<=t} M_s with
+    M_s = D_s (I - beta_s k_s k_s^T), every product formed explicitly (w = beta: the
+    tied delta rule; otherwise beta erases and w writes)."""
+    w = beta if w is None else w
     T, dk = q.shape
     dv = v.shape[1]
     M = []
@@ -72,7 +74,7 @@ def _brute_head(q, k, v, a, beta, theta, S0, scale):
     for t in range(T):
         S_t = S0 @ prod(0, t + 1)
         for i in range(t + 1):
-            S_t = S_t + beta[i] * np.outer(v[i], k[i]) @ prod(i + 1, t + 1)
+            S_t = S_t + w[i] * np.outer(v[i], k[i]) @ prod(i + 1, t + 1)
         o[t] = S_t @ (scale * q[t])
     return o, S_t
 
@@ -355,3 +357,75 @@ def test_decode_steps_equal_forward(rotation):
                                        oracle.GATE_NEG_SOFTPLUS, 0.8)
         assert np.array_equal(od, o[:, t])
     assert np.array_equal(S, S_T)
+
+
+# ---- separate erase and write strengths ("CARVE" page, sections 2.1-2.2) ----------------
+
+def _write_gate(rng, shape):
+    return 1.0 / (1.0 + np.exp(-rng.standard_normal(shape)))
+
+
+@pytest.mark.parametrize("rotation", [False, True])
+def test_untied_oracle_matches_brute_force_products(rotation):
+    rng = np.random.default_rng(71 + rotation)
+    B, T, H, dk, dv = 2, 11, 2, 8, 6
+    q, k, v, a, beta, theta, S0 = _rand_problem(rng, B, T, H, dk, dv, rotation)
+    w = _write_gate(rng, (B, T, H))
+    o, S_T = oracle.gdr_fwd(q, k, v, a, beta, theta, S0, oracle.GATE_NEG_SOFTPLUS, scale=0.9, w=w)
+    for b in range(B):
+        for h in range(H):
+            ob, Sb = _brute_head(q[b, :, h], k[b, :, h], v[b, :, h], a[b, :, h], beta[b, :, h],
+                                 None if theta is None else theta[b, :, h], S0[b, h], 0.9, w=w[b, :, h])
+            assert _rel(o[b, :, h], ob) < 1e-12
+            assert _rel(S_T[b, h], Sb) < 1e-12
+    # the pin separates the two gates: exchanging them moves the result far
+    o_x, _ = _brute_head(q[0, :, 0], k[0, :, 0], v[0, :, 0], a[0, :, 0], w[0, :, 0],
+                         None if theta is None else theta[0, :, 0], S0[0, 0], 0.9, w=beta[0, :, 0])
+    assert _rel(o_x, o[0, :, 0]) > 1e-3
+
+
+def test_untied_with_write_equal_to_erase_is_the_delta_rule():
+    rng = np.random.default_rng(72)
+    q, k, v, a, beta, theta, S0 = _rand_problem(rng, 1, 20, 2, 8, 5)
+    o1, S1 = oracle.gdr_fwd(q, k, v, a, beta, theta, S0, oracle.GATE_NEG_SOFTPLUS)
+    o2, S2 = oracle.gdr_fwd(q, k, v, a, beta, theta, S0, oracle.GATE_NEG_SOFTPLUS, w=beta.copy())
+    assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
+
+
+def test_write_only_without_decay_is_a_running_sum():
+    """beta = 0, g = 0: nothing is erased or decayed, so S_t = S_0 + sum_{i<=t} w_i v_i k_i^T
+    and o_t = S_t q_t, written out as cumulative sums."""
+    rng = np.random.default_rng(73)
+    q, k, v, a, beta, theta, S0 = _rand_problem(rng, 1, 17, 1, 6, 4, unit_k=False)
+    w = rng.standard_normal((1, 17, 1))
+    zero = np.zeros_like(beta)
+    o, S_T = oracle.gdr_fwd(q, k, v, np.zeros_like(a), zero, None, S0, oracle.GATE_LOGDECAY, w=w)
+    terms = w[0, :, 0, None, None] * v[0, :, 0, :, None] * k[0, :, 0, None, :]
+    S_run = S0[0, 0][None] + np.cumsum(terms, axis=0)
+    assert _rel(S_T[0, 0], S_run[-1]) < 1e-13
+    assert _rel(o[0, :, 0], np.einsum("tij,tj->ti", S_run, q[0, :, 0])) < 1e-13
+
+
+def test_erase_only_annihilates_the_key():
+    """w = 0, beta = 1, unit keys, no decay: each step projects the state off k_t, so
+    S_t k_t = 0 and nothing of v is written."""
+    rng = np.random.default_rng(74)
+    q, k, v, a, beta, theta, S0 = _rand_problem(rng, 1, 6, 1, 8, 5)
+    ones, zero = np.ones_like(beta), np.zeros_like(beta)
+    for t in range(1, 7):
+        _, S = oracle.gdr_fwd(q[:, :t], k[:, :t], v[:, :t], np.zeros_like(a[:, :t]), ones[:, :t], None, S0,
+                              oracle.GATE_LOGDECAY, w=zero[:, :t])
+        assert np.max(np.abs(S[0, 0] @ k[0, t - 1, 0])) < 1e-13
+
+
+def test_untied_decode_steps_equal_forward():
+    rng = np.random.default_rng(75)
+    q, k, v, a, beta, theta, S0 = _rand_problem(rng, 1, 9, 3, 8, 6, rotation=True)
+    w = _write_gate(rng, (1, 9, 3))
+    o_f, S_f = oracle.gdr_fwd(q, k, v, a, beta, theta, S0, oracle.GATE_NEG_SOFTPLUS, w=w)
+    S = S0.copy()
+    for t in range(9):
+        o_t, S = oracle.gdr_decode_step(q[:, t], k[:, t], v[:, t], a[:, t], beta[:, t], S, theta[:, t],
+                                        oracle.GATE_NEG_SOFTPLUS, w=w[:, t])
+        assert _rel(o_t, o_f[:, t]) < 1e-12
+    assert _rel(S, S_f) < 1e-12
