@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define GDR_ABI_VERSION 1
+#define GDR_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define GDR_API __attribute__((visibility("default")))
@@ -164,6 +164,32 @@ GDR_API gdr_status gdr_decode_step(const gdr_dec_desc* desc,
                            const void* q, const void* k, const void* v,
                            const float* g, const float* beta, const float* theta,
                            float* S, void* o, gdr_stream_t stream);
+
+/*
+ * Separate erase and write strengths ("CARVE" page, sections 2.1-2.2: an erase gate and a
+ * scalar value write gate per head and token).  The token update becomes
+ *
+ *   S_t = S_{t-1} D_t (I - beta_t k_t k_t^T) + w_t v_t k_t^T,     o_t = S_t (scale q_t)
+ *
+ * with beta the erase strength and w [B,T,H] (decode: [N,H]) fp32 the write strength,
+ * 16-byte aligned.  w = NULL is the tied rule above (w = beta): gdr_chunk_fwd and
+ * gdr_decode_step are these calls with w = NULL.  Every kernel supports it; the chunk solver
+ * is unchanged (A still uses beta), only U = (I + A)^{-1} diag(w) V changes.  The
+ * content-aware erase of that page (beta modulated by the previous chunk's mean output)
+ * is left to the caller, which passes the resulting beta.  Other arguments, layouts, errors
+ * and ownership as for gdr_chunk_fwd / gdr_decode_step.  (gdr_chunk_fwd_noalloc is tied only.)
+ */
+GDR_API gdr_status gdr_chunk_fwd_untied(const gdr_fwd_desc* desc,
+                                        const void* q, const void* k, const void* v,
+                                        const float* g, const float* beta, const float* w,
+                                        const float* theta, const float* S0, void* o, float* S_T,
+                                        void* workspace, size_t workspace_bytes,
+                                        gdr_stream_t stream);
+GDR_API gdr_status gdr_decode_step_untied(const gdr_dec_desc* desc,
+                                          const void* q, const void* k, const void* v,
+                                          const float* g, const float* beta, const float* w,
+                                          const float* theta, float* S, void* o,
+                                          gdr_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word that

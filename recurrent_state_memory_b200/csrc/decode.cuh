@@ -1,7 +1,7 @@
 // decode.cuh -- one recurrent decode step, HBM-bound: S is read once and written once.
 //
 // Per value row s (one row of S, dk wide), with X = S D_t:
-//   x_k = (s D_t) . k,   x_q = (s D_t) . q,   e = beta (v_row - x_k)
+//   x_k = (s D_t) . k,   x_q = (s D_t) . q,   e = w v_row - beta x_k  (w = beta unless given)
 //   s  <- s D_t + e k^T,   o_row = x_q + e (k . q)
 // which is the token update of the "Semidirect Fourier Delta Attention" page
 // ("Core architecture": decay, erase along k, write v) transposed to value rows,
@@ -26,6 +26,7 @@ struct DecParams {
     const void* v;
     const float* g;
     const float* beta;
+    const float* w;         // write strength [N,H], or nullptr: w = beta
     const float* theta;
     float* S;
     void* o;
@@ -110,6 +111,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_kernel(DecParams p) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
     const float bt = p.beta[nh];
+    const float wt = p.w ? p.w[nh] : bt;
     const float vrow = (row0 + lane < p.dv && lane < ROWS) ? ld_f32(v + row0 + lane) : 0.f;
 
     float orow = 0.f;
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_kernel(DecParams p) {
             xk += __shfl_xor_sync(0xffffffffu, xk, off);
             xq += __shfl_xor_sync(0xffffffffu, xq, off);
         }
-        const float e = bt * (__shfl_sync(0xffffffffu, vrow, rr) - xk);
+        const float e = wt * __shfl_sync(0xffffffffu, vrow, rr) - bt * xk;
 #pragma unroll
         for (int u = 0; u < VEC; ++u) s[u] = fmaf(e, kk[u], s[u]);
         __stcs(reinterpret_cast<VT*>(S + (size_t)row * DK) + lane, pack<VEC>(s));

@@ -321,6 +321,14 @@ gdr_status gdr_chunk_fwd(const gdr_fwd_desc* d, const void* q, const void* k, co
                          const float* g, const float* beta, const float* theta, const float* S0,
                          void* o, float* S_T, void* workspace, size_t workspace_bytes,
                          gdr_stream_t stream) {
+    return gdr_chunk_fwd_untied(d, q, k, v, g, beta, nullptr, theta, S0, o, S_T, workspace, workspace_bytes,
+                                stream);
+}
+
+gdr_status gdr_chunk_fwd_untied(const gdr_fwd_desc* d, const void* q, const void* k, const void* v,
+                                const float* g, const float* beta, const float* w, const float* theta,
+                                const float* S0, void* o, float* S_T, void* workspace,
+                                size_t workspace_bytes, gdr_stream_t stream) {
     t_detail[0] = 0;
     gdr_status s = check_fwd_desc(d);
     if (s != GDR_OK) return s;
@@ -332,7 +340,8 @@ gdr_status gdr_chunk_fwd(const gdr_fwd_desc* d, const void* q, const void* k, co
         if (d->rotation && !theta) return fail(GDR_ERR_INVALID_ARG, "theta is required with rotation%s");
     }
     if (!d->rotation && theta) return fail(GDR_ERR_INVALID_ARG, "theta must be NULL without rotation%s");
-    if ((theta && !aligned16(theta)) || (S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
+    if ((theta && !aligned16(theta)) || (S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)) ||
+        (w && !aligned16(w)))
         return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
     const size_t need = gdr_chunk_fwd_workspace_bytes(d);
     if (need > 0 && (!workspace || workspace_bytes < need)) return fail(GDR_ERR_WORKSPACE, "workspace too small%s");
@@ -341,7 +350,7 @@ gdr_status gdr_chunk_fwd(const gdr_fwd_desc* d, const void* q, const void* k, co
     p.B = d->B; p.H = d->H; p.T = d->T; p.dv = d->dv;
     p.gate_mode = (int)d->gate_mode;
     p.scale = d->scale;
-    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.theta = theta;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.theta = theta;
     p.S0 = S0; p.o = o; p.S_T = S_T;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d->T == 0 && !S_T) return GDR_OK;
@@ -357,6 +366,12 @@ gdr_status gdr_chunk_fwd(const gdr_fwd_desc* d, const void* q, const void* k, co
 gdr_status gdr_decode_step(const gdr_dec_desc* d, const void* q, const void* k, const void* v,
                            const float* g, const float* beta, const float* theta, float* S,
                            void* o, gdr_stream_t stream) {
+    return gdr_decode_step_untied(d, q, k, v, g, beta, nullptr, theta, S, o, stream);
+}
+
+gdr_status gdr_decode_step_untied(const gdr_dec_desc* d, const void* q, const void* k, const void* v,
+                                  const float* g, const float* beta, const float* w, const float* theta,
+                                  float* S, void* o, gdr_stream_t stream) {
     t_detail[0] = 0;
     if (!d) return fail(GDR_ERR_INVALID_ARG, "desc is NULL%s");
     if (d->N < 0 || d->H < 0) return fail(GDR_ERR_INVALID_ARG, "N, H must be >= 0%s");
@@ -371,13 +386,13 @@ gdr_status gdr_decode_step(const gdr_dec_desc* d, const void* q, const void* k, 
     if (d->rotation && !theta) return fail(GDR_ERR_INVALID_ARG, "theta is required with rotation%s");
     if (!d->rotation && theta) return fail(GDR_ERR_INVALID_ARG, "theta must be NULL without rotation%s");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) ||
-        !aligned16(S) || !aligned16(o) || (theta && !aligned16(theta)))
+        !aligned16(S) || !aligned16(o) || (theta && !aligned16(theta)) || (w && !aligned16(w)))
         return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
     dec::DecParams p;
     p.N = d->N; p.H = d->H; p.dv = d->dv;
     p.gate_mode = (int)d->gate_mode;
     p.scale = d->scale;
-    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.theta = theta; p.S = S; p.o = o;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.theta = theta; p.S = S; p.o = o;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d->rotation) {
         switch (d->dk) {
@@ -445,7 +460,7 @@ gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* d, const void* q, const voi
     p.B = d->B; p.H = d->H; p.T = d->T; p.dv = d->dv;
     p.gate_mode = (int)d->gate_mode;
     p.scale = d->scale;
-    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.theta = theta;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = nullptr; p.theta = theta;
     p.S0 = S0; p.o = o; p.S_T = S_T;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d->T == 0) return S_T ? dispatch_tc_mode<0>(d, p, st, nullptr) : GDR_OK;

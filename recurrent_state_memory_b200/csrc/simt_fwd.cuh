@@ -12,7 +12,8 @@
 // mode), P_r = D_1 ... D_r:
 //   A[r,i]  = beta_r k_i^T P_i^{-1} P_r k_r        (i < r)
 //   Pm[r,i] = k_i^T P_i^{-1} P_r q_r               (i <= r)
-//   E       = (I + A)^{-1} diag(beta) (V - Ktil S^T),   Ktil_r = P_r k_r
+//   E       = (I + A)^{-1} (diag(w) V - diag(beta) Ktil S^T),   Ktil_r = P_r k_r
+//             (w: the write strength, w = beta unless given; beta erases)
 //   O       = Qtil S^T + Pm E,                          Qtil_r = P_r q_r
 //   S      <- S P_C + E^T Kdec,                         Kdec_i = P_C^T P_i^{-T} k_i
 // A and Pm are formed with exp(Gamma_r - Gamma_i) inside the sum (no factoring),
@@ -32,6 +33,7 @@ struct FwdParams {
     const void* v;
     const float* g;
     const float* beta;
+    const float* w;         // write strength [B,T,H], or nullptr: w = beta
     const float* theta;
     const float* S0;
     void* o;
@@ -54,7 +56,8 @@ struct Smem {
     static constexpr int off_G = off_kt + C * KS;           // cumulative log-decay   [C][NG]
     static constexpr int off_Th = off_G + C * NG;           // cumulative angle       [C][DK/2] (ROT)
     static constexpr int off_b = off_Th + (ROT ? C * (DK / 2) : 0);   // beta   [C]
-    static constexpr int off_A = off_b + C;                 // A (strict lower)       [C][C+1]
+    static constexpr int off_w = off_b + C;                 // write strength         [C]
+    static constexpr int off_A = off_w + C;                 // A (strict lower)       [C][C+1]
     static constexpr int off_P = off_A + C * (C + 1);       // Pm (lower, inclusive)  [C][C+1]
     static constexpr int off_S = off_P + C * (C + 1);       // state slice            [DVT][KS]
     static constexpr int off_R = off_S + DVT * KS;          // RHS, then E            [C][DVT+1]
@@ -76,6 +79,7 @@ __global__ void __launch_bounds__(NT) chunk_fwd_kernel(FwdParams p) {
     float* Gc = sm + L::off_G;
     float* Th = sm + L::off_Th;
     float* bc = sm + L::off_b;
+    float* wc = sm + L::off_w;
     float* Am = sm + L::off_A;
     float* Pm = sm + L::off_P;
     float* S = sm + L::off_S;
@@ -123,6 +127,7 @@ __global__ void __launch_bounds__(NT) chunk_fwd_kernel(FwdParams p) {
             if (ROT) Th[idx] = r < Lc ? p.theta[tok(r) * (DK / 2) + jg] : 0.f;
         }
         if (tid < C) bc[tid] = tid < Lc ? p.beta[tok(tid)] : 0.f;
+        if (tid < C) wc[tid] = tid < Lc ? (p.w ? p.w[tok(tid)] : p.beta[tok(tid)]) : 0.f;
         __syncthreads();
 
         // 2. In-chunk prefix sums: Gamma_r (and Theta_r, kept in [-pi, pi]).
@@ -221,7 +226,7 @@ __global__ void __launch_bounds__(NT) chunk_fwd_kernel(FwdParams p) {
         }
         __syncthreads();
 
-        // 5. R = diag(beta) (V - Ktil S^T) and QS = Qtil S^T.
+        // 5. R = diag(w) V - diag(beta) Ktil S^T and QS = Qtil S^T.
         for (int idx = tid; idx < C * DVT; idx += NT) {
             const int r = idx / DVT, j = idx % DVT;
             float ks = 0.f, qs = 0.f;
@@ -235,7 +240,7 @@ __global__ void __launch_bounds__(NT) chunk_fwd_kernel(FwdParams p) {
                     qs = fmaf(qr[d], Sj[d], qs);
                 }
                 const float vv = ld_f32(v + tok(r) * dv + j0 + j);
-                R[r * (DVT + 1) + j] = bc[r] * (vv - ks);
+                R[r * (DVT + 1) + j] = wc[r] * vv - bc[r] * ks;
             } else {
                 R[r * (DVT + 1) + j] = 0.f;
             }

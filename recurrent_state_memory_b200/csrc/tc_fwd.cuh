@@ -69,19 +69,24 @@ constexpr int AS = 68;                               // row stride (floats) of t
 constexpr uint32_t OFF_AF = OFF_TB + 8192;           // fp32 A [64][68]
 constexpr uint32_t OFF_TF = OFF_AF + 64 * AS * 4;    // fp32 Tm [64][68]
 constexpr uint32_t OFF_QT = OFF_TF + 64 * AS * 4;    // segment products [8 segments][32 dim groups][8]
-constexpr uint32_t VEC_FLOATS = 64 + 4 * 128;        // beta[64], rho_ref[2][128], rho_C[2][128]
+constexpr uint32_t VEC_FLOATS = 64 + 4 * 128 + 64;   // beta[64], rho_ref[2][128], rho_C[2][128], w[64]
+constexpr uint32_t VEC_W = 64 + 4 * 128;             // offset of the write strengths in a vector block
 constexpr uint32_t OFF_VEC = OFF_QT + 8 * 32 * 8 * 4;   // x2
 constexpr uint32_t OFF_BAR = (OFF_VEC + 2 * VEC_FLOATS * 4 + 63) & ~63u;
 constexpr uint32_t BAR_BYTES = 256;                  // mbarriers, TMEM address, flags
+// Tw = Tm diag(w) K-major, for a write strength w separate from the erase strength beta
+constexpr uint32_t OFF_TW = (OFF_BAR + BAR_BYTES + 1023) & ~1023u;
 
 // Split mode: a per-head ring in global memory carries each chunk's operands from the prep
 // workers to the chain CTA.  Slot layout (bytes), identical to the chain's shared-memory copy:
 constexpr uint32_t SL_Q = 0;          // Qtil K-major: 2 kblocks x 64 rows x 128 B
 constexpr uint32_t SL_KH = 16384;     // Khat K-major: 2 kblocks x 64 rows x 128 B
-constexpr uint32_t SL_W = 32768;      // Wm^T bf16 MN-major: 128 dk rows x 128 B
+constexpr uint32_t SL_W = 32768;      // Ktil2 (2 kblocks x 64 rows x 128 B); in the chain CTA then
+                                      // Wm2^T bf16 MN-major (128 dk rows x 128 B)
 constexpr uint32_t SL_PM = 49152;     // Pm K-major: 64 rows x 128 B
 constexpr uint32_t SL_TB = 57344;     // Tb K-major: 64 rows x 128 B
-constexpr uint32_t SL_VEC = 65536;    // beta, rho_ref, rho_C (VEC_FLOATS floats)
+constexpr uint32_t SL_TW = 65536;     // Tw K-major (only with a separate write strength)
+constexpr uint32_t SL_VEC = 73728;    // beta, P_C, ... (VEC_FLOATS floats)
 constexpr uint32_t SLOT_BYTES = SL_VEC + VEC_FLOATS * 4;        // bytes of one ring slot
 // The chain CTA's copy of a slot is followed by the chunk's V tile, which the chain loads
 // itself from the input (MN-major: 2 groups x 64 tokens x 128 B).
@@ -99,7 +104,8 @@ constexpr uint32_t G_KQ = 0;         // [Ktil ; Qtil] K-major: 2 kblocks x 128 r
 constexpr uint32_t G_KH = 32768;     // Khat K-major: 2 kblocks x 64 rows x 128 B
 constexpr uint32_t G_TB = 49152;     // Tb K-major: 64 rows x 128 B
 constexpr uint32_t G_QT = 57344;     // segment products [8][32][8]
-constexpr uint32_t G_AF = 65536;     // fp32 A [64][68]
+constexpr uint32_t G_TW = 65536;     // Tw K-major (separate write strength only)
+constexpr uint32_t G_AF = 73728;     // fp32 A [64][68]
 constexpr uint32_t G_TF = G_AF + 64 * AS * 4;   // fp32 Tm [64][68]
 constexpr uint32_t G_VEC = G_TF + 64 * AS * 4;  // beta, rho_ref, rho_C
 constexpr uint32_t G_STRIDE = (G_VEC + VEC_FLOATS * 4 + 1023) & ~1023u;
@@ -111,7 +117,11 @@ static_assert(G_KH - G_KQ >= 32768 && 64 * AS * 4 >= 16384, "staging does not fi
 template <int MODE> __host__ __device__ constexpr int nthreads() { return MODE == 0 ? NT : NT_SPLIT; }
 template <int MODE> __host__ __device__ constexpr uint32_t off_bar() { return MODE == 0 ? OFF_BAR : OFF_BAR_SPLIT; }
 // dynamic shared memory, with slack for the 1024-byte alignment of the base
-template <int MODE> __host__ __device__ constexpr uint32_t smem_bytes() { return off_bar<MODE>() + BAR_BYTES + 1024; }
+template <int MODE> __host__ __device__ constexpr uint32_t smem_bytes() {
+    return (MODE == 0 ? OFF_TW + 8192 : OFF_BAR_SPLIT + BAR_BYTES) + 1024;
+}
+static_assert(OFF_TW + 8192 + 1024 <= 232448 && OFF_BAR_SPLIT + BAR_BYTES + 1024 <= 232448,
+              "shared memory exceeds 227 KB");
 
 // 4-D tensor maps {inner dim, H, T, B} with boxes of 64 tokens (split mode only).
 // q, k: bf16 box {128,1,64,1}; g: fp32 box {128,...} ({64,...} with rotation); th: fp32
@@ -238,6 +248,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
     const __nv_bfloat16* __restrict__ v = static_cast<const __nv_bfloat16*>(p.v);
     OT* __restrict__ o = static_cast<OT*>(p.o);
     const int nchunks = (p.T + C - 1) / C;
+    const bool untied = p.w != nullptr;     // a write strength w separate from beta
     auto chunk_len = [&](int c) -> int { return min(C, p.T - c * C); };
     auto tokh = [&](int bhx, int c, int r) -> size_t {
         return ((size_t)(bhx / p.H) * p.T + (c * C + r)) * p.H + (bhx % p.H);
@@ -403,8 +414,11 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             uint8_t* ring = (MODE == 1) ? sa.ring + ((size_t)bhx * RING + c % RING) * SLOT_BYTES : nullptr;
             float* rvec = reinterpret_cast<float*>(ring + SL_VEC);
             // beta of this task, consumed after pass 1
-            float beta_r = 0.f;
-            if (tid < 64 && tid < Lc) beta_r = __ldg(p.beta + tokh(bhx, c, tid));
+            float beta_r = 0.f, w_r = 0.f;
+            if (tid < 64 && tid < Lc) {
+                beta_r = __ldg(p.beta + tokh(bhx, c, tid));
+                w_r = untied ? __ldg(p.w + tokh(bhx, c, tid)) : beta_r;
+            }
             if (MODE == 1) {
                 // raw inputs of this task, staged by the transfer thread (tokens past the
                 // sequence end arrive as zeros)
@@ -493,7 +507,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 qtp[0] = make_float4(PA[0], PA[1], PA[2], PA[3]);
                 qtp[1] = make_float4(PI[0], PI[1], PI[2], PI[3]);
             }
-            if (tid < 64) sbeta[tid] = beta_r;
+            if (tid < 64) { sbeta[tid] = beta_r; vec[VEC_W + tid] = w_r; }
             named_bar(gbar, NPREP);
             // Buffers of task it - 2 must be released (by the chain, or by the copy-out warps)
             // before they are rewritten.
@@ -749,17 +763,26 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     }
                 }
             }
-            {   // Tb: blocks above the diagonal stay zero (the area may hold staged k)
-                uint4* tbz = reinterpret_cast<uint4*>((MODE == 0) ? base + OFF_TB : gb + G_TB);
+            uint8_t* TB = (MODE == 0) ? base + OFF_TB : gb + G_TB;
+            uint8_t* TW = (MODE == 0) ? base + OFF_TW : gb + G_TW;
+            const float* sw = vec + VEC_W;
+            {   // Tb (and Tw): blocks above the diagonal stay zero
+                uint4* tbz = reinterpret_cast<uint4*>(TB);
                 tbz[tid] = make_uint4(0u, 0u, 0u, 0u);
                 tbz[tid + NPREP] = make_uint4(0u, 0u, 0u, 0u);
+                if (untied) {
+                    uint4* twz = reinterpret_cast<uint4*>(TW);
+                    twz[tid] = make_uint4(0u, 0u, 0u, 0u);
+                    twz[tid + NPREP] = make_uint4(0u, 0u, 0u, 0u);
+                }
             }
             named_bar(gbar, NPREP);
-            // Tb = Tm diag(beta) as bf16 K-major [r][i] (blocks above the diagonal stay zero).
-            uint8_t* TB = (MODE == 0) ? base + OFF_TB : gb + G_TB;
+            // Tb = Tm diag(beta) as bf16 K-major [r][i] (blocks above the diagonal stay zero);
+            // with a separate write strength also Tw = Tm diag(w), for U = Tw V.
             auto tb_put2 = [&](int r, int i, float x0, float x1) {      // columns i, i + 1
-                *reinterpret_cast<uint32_t*>(TB + sw128_off(r, i >> 3) + (i & 7) * 2) =
-                    pack_bf16x2(x0 * sbeta[i], x1 * sbeta[i + 1]);
+                const uint32_t off = sw128_off(r, i >> 3) + (i & 7) * 2;
+                *reinterpret_cast<uint32_t*>(TB + off) = pack_bf16x2(x0 * sbeta[i], x1 * sbeta[i + 1]);
+                if (untied) *reinterpret_cast<uint32_t*>(TW + off) = pack_bf16x2(x0 * sw[i], x1 * sw[i + 1]);
             };
             // 16x16 diagonal blocks by forward substitution (lane = column of one block).
             if (tid < 64) {
@@ -772,13 +795,14 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     for (int i = 0; i < r; ++i) s_ = fmaf(-Af[(bb + r) * AS + bb + i], t[i], s_);
                     t[r] = s_;
                 }
-                const float bj = sbeta[bb + jj];
+                const float bj = sbeta[bb + jj], wj = sw[bb + jj];
                 const int ib = bb + jj;
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
                     Tf[(bb + r) * AS + bb + jj] = t[r];
-                    *reinterpret_cast<__nv_bfloat16*>(TB + sw128_off(bb + r, ib >> 3) + (ib & 7) * 2) =
-                        __float2bfloat16_rn(t[r] * bj);
+                    const uint32_t off = sw128_off(bb + r, ib >> 3) + (ib & 7) * 2;
+                    *reinterpret_cast<__nv_bfloat16*>(TB + off) = __float2bfloat16_rn(t[r] * bj);
+                    if (untied) *reinterpret_cast<__nv_bfloat16*>(TW + off) = __float2bfloat16_rn(t[r] * wj);
                 }
             }
             named_bar(gbar, NPREP);
@@ -865,8 +889,11 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             publish();
             if (MODE == 1) {                // Tb -> ring
 #pragma unroll
-                for (int e = 0; e < 2; ++e)
+                for (int e = 0; e < 2; ++e) {
                     reinterpret_cast<uint4*>(ring + SL_TB)[tid + e * NPREP] = reinterpret_cast<const uint4*>(TB)[tid + e * NPREP];
+                    if (untied)
+                        reinterpret_cast<uint4*>(ring + SL_TW)[tid + e * NPREP] = reinterpret_cast<const uint4*>(TW)[tid + e * NPREP];
+                }
                 if (tid == 0 && it + 1 < ntasks) stage_part(it + 1, 2);          // A and Tm done
             }
 
@@ -875,7 +902,8 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 if (tid == 0) {
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t bdesc = sdesc_sw128(sb + OFF_TB + ks * 32, 16, 1024);
-                        mma_bf16_ss(tbase + COL_E + bufi * 64, sdesc_sw128(sb + OFF_V + ks * 2048, 8192, 1024), bdesc,
+                        const uint64_t wdesc = sdesc_sw128(sb + (untied ? OFF_TW : OFF_TB) + ks * 32, 16, 1024);
+                        mma_bf16_ss(tbase + COL_E + bufi * 64, sdesc_sw128(sb + OFF_V + ks * 2048, 8192, 1024), wdesc,
                                     ID_MK, ks > 0);
                         mma_bf16_ss(tbase + col_aw, sdesc_sw128(kq_s + ks * 2048, 16384, 1024), bdesc, ID_MK, ks > 0);
                     }
@@ -952,7 +980,8 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t dTb = sdesc_sw128(sl + SL_TB + ks * 32, 16, 1024);
-                mma_bf16_ss(tbase + COL_E + (c & 1) * 64, sdesc_sw128(sl + SL_V + ks * 2048, 8192, 1024), dTb,
+                const uint64_t dTw = sdesc_sw128(sl + (untied ? SL_TW : SL_TB) + ks * 32, 16, 1024);
+                mma_bf16_ss(tbase + COL_E + (c & 1) * 64, sdesc_sw128(sl + SL_V + ks * 2048, 8192, 1024), dTw,
                             ID_MK, ks > 0);
                 mma_bf16_ss(tbase + COL_WS, sdesc_sw128(sl + SL_W + ks * 2048, 8192, 1024), dTb, ID_MK, ks > 0);
             }
@@ -1424,11 +1453,14 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 if (ok) {
                     fence_proxy_async_global();
                     const uint8_t* src = sa.ring + ((size_t)bh * RING + slot) * SLOT_BYTES;
-                    mbar_arrive_expect_tx(bar_full + bufi, SLOT_BYTES + 16384u);
-                    for (uint32_t off = 0; off < SLOT_BYTES; off += 16384u) {
-                        const uint32_t n = SLOT_BYTES - off < 16384u ? SLOT_BYTES - off : 16384u;
+                    // the tiles (Tw only with a separate write strength), the vectors, and V
+                    const uint32_t tiles = untied ? SL_VEC : SL_TW;
+                    mbar_arrive_expect_tx(bar_full + bufi, tiles + (SLOT_BYTES - SL_VEC) + 16384u);
+                    for (uint32_t off = 0; off < tiles; off += 16384u) {
+                        const uint32_t n = tiles - off < 16384u ? tiles - off : 16384u;
                         bulk_g2s(sb + slot_base(c) + off, src + off, n, bar_full + bufi);
                     }
+                    bulk_g2s(sb + slot_base(c) + SL_VEC, src + SL_VEC, SLOT_BYTES - SL_VEC, bar_full + bufi);
                     // V of this chunk, two 64-column boxes straight into the MN-major layout
                     const int bb = bh / p.H, hh = bh % p.H;
                     tma_load_4d(sb + slot_base(c) + SL_V, &tm.v, 0, hh, c * C, bb, bar_full + bufi);

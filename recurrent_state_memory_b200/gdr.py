@@ -70,6 +70,10 @@ def lib() -> ctypes.CDLL:
         L.gdr_chunk_fwd.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp, vp, sz, vp]
         L.gdr_decode_step.restype = ctypes.c_int
         L.gdr_decode_step.argtypes = [ctypes.POINTER(DecDesc), vp, vp, vp, fp, fp, fp, fp, vp, vp]
+        L.gdr_chunk_fwd_untied.restype = ctypes.c_int
+        L.gdr_chunk_fwd_untied.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, fp, vp, sz, vp]
+        L.gdr_decode_step_untied.restype = ctypes.c_int
+        L.gdr_decode_step_untied.argtypes = [ctypes.POINTER(DecDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, vp]
         L.gdr_query_device_status.restype = ctypes.c_int
         L.gdr_query_device_status.argtypes = [vp]
         L.gdr_chunk_fwd_algo.restype = ctypes.c_int
@@ -78,7 +82,7 @@ def lib() -> ctypes.CDLL:
         L.gdr_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp, vp]
         L.gdr_debug_set_tc_fault.restype = None
         L.gdr_debug_set_tc_fault.argtypes = [ctypes.c_int, ctypes.c_ulonglong]
-        if L.gdr_abi_version() != 1:
+        if L.gdr_abi_version() != 2:
             raise RuntimeError("libgdr.so ABI version mismatch")
         _lib = L
     return _lib
@@ -150,16 +154,17 @@ def workspace_bytes(desc: FwdDesc) -> int:
 
 def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
               algo="auto", out_dtype=None, want_state=True, o=None, S_T=None, workspace=None,
-              stream=None, chunk=64) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              stream=None, chunk=64, w=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunk-parallel forward.  Returns (o, S_T).
 
-    With CUDA tensors the call is asynchronous on `stream` (default: the current
-    stream).  With host tensors the inputs are copied to the current device,
-    the library is called, and o / S_T are copied back (synchronising).
+    beta is the erase strength; w [B,T,H] (fp32) a separate write strength, or None for
+    the tied rule (w = beta).  With CUDA tensors the call is asynchronous on `stream`
+    (default: the current stream).  With host tensors the inputs are copied to the current
+    device, the library is called, and o / S_T are copied back (synchronising).
     """
     if not q.is_cuda:
         return _chunk_fwd_host(q, k, v, g, beta, theta, S0, gate_mode=gate_mode, scale=scale,
-                               algo=algo, out_dtype=out_dtype, want_state=want_state, chunk=chunk)
+                               algo=algo, out_dtype=out_dtype, want_state=want_state, chunk=chunk, w=w)
     dev = q.device
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -174,6 +179,10 @@ def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTP
         raise ValueError("q, k, v shapes disagree")
     if tuple(g.shape) != (B, T, H, dk // 2 if rotation else dk) or tuple(beta.shape) != (B, T, H):
         raise ValueError("g or beta has the wrong shape")
+    if w is not None:
+        _need(w, "w", torch.float32, dev)
+        if tuple(w.shape) != (B, T, H):
+            raise ValueError("w has the wrong shape")
     if theta is not None:
         _need(theta, "theta", torch.float32, dev)
         if tuple(theta.shape) != (B, T, H, dk // 2):
@@ -194,25 +203,31 @@ def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTP
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().gdr_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                             _ptr(theta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
-                             _stream_handle(stream, dev))
+    if w is None:
+        st = lib().gdr_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                 _ptr(theta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
+                                 _stream_handle(stream, dev))
+    else:
+        st = lib().gdr_chunk_fwd_untied(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                        _ptr(w), _ptr(theta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                                        ws_bytes, _stream_handle(stream, dev))
     _check(st, "gdr_chunk_fwd")
     return o, S_T
 
 
-def _chunk_fwd_host(q, k, v, g, beta, theta, S0, **kw):
+def _chunk_fwd_host(q, k, v, g, beta, theta, S0, w=None, **kw):
     dev = torch.device("cuda", torch.cuda.current_device())
     to = lambda t: None if t is None else t.to(dev, non_blocking=True)
-    o, S_T = chunk_fwd(to(q), to(k), to(v), to(g), to(beta), to(theta), to(S0), **kw)
+    o, S_T = chunk_fwd(to(q), to(k), to(v), to(g), to(beta), to(theta), to(S0), w=to(w), **kw)
     o_h = o.to("cpu")
     S_h = None if S_T is None else S_T.to("cpu")
     return o_h, S_h
 
 
 def decode_step(q, k, v, g, beta, S, theta=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
-                out_dtype=None, o=None, stream=None) -> torch.Tensor:
-    """One decode step; S [N,H,dv,dk] (fp32) is updated in place.  Returns o [N,H,dv]."""
+                out_dtype=None, o=None, stream=None, w=None) -> torch.Tensor:
+    """One decode step; S [N,H,dv,dk] (fp32) is updated in place.  Returns o [N,H,dv].
+    beta erases; w [N,H] (fp32) is a separate write strength, or None for w = beta."""
     dev = S.device
     N, H, dk = q.shape
     dv = v.shape[-1]
@@ -232,8 +247,12 @@ def decode_step(q, k, v, g, beta, S, theta=None, *, gate_mode=GATE_NEG_SOFTPLUS,
         o = torch.empty((N, H, dv), dtype=out_dtype, device=dev)
     desc = DecDesc(N, H, dk, dv, _dtype_code(q.dtype), _dtype_code(out_dtype), int(gate_mode),
                    int(rotation), float(scale))
-    st = lib().gdr_decode_step(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                               _ptr(theta), _ptr(S), _ptr(o), _stream_handle(stream, dev))
+    if w is not None:
+        _need(w, "w", torch.float32, dev)
+        if tuple(w.shape) != (N, H):
+            raise ValueError("w has the wrong shape")
+    st = lib().gdr_decode_step_untied(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                      _ptr(w), _ptr(theta), _ptr(S), _ptr(o), _stream_handle(stream, dev))
     _check(st, "gdr_decode_step")
     return o
 

@@ -251,6 +251,11 @@ class DecodeInputs:
         return a.astype(np.float64)
 
 
+def make_write_strength(seed, shape) -> np.ndarray:
+    """A write strength w = sigmoid(N(0,1)) separate from beta (fp32), for the untied rule."""
+    return (1.0 / (1.0 + np.exp(-normal(seed, "w", shape)))).astype(np.float32)
+
+
 def make_decode(N, H, dk, dv, steps, dtype="bf16", seed=4, s_std=0.02, rotation=False,
                 scale=1.0) -> DecodeInputs:
     """Per-step single-token inputs for N independent sequences, plus the state S."""

@@ -93,3 +93,19 @@ def test_decode_rejects_bad_arguments(G):
 def test_workspace_query(G):
     assert G.workspace_bytes(_desc(G)) >= 0
     assert G.workspace_bytes(_desc(G, dk=48)) == 0
+
+
+def test_untied_entry_points_check_the_write_strength(G):
+    """gdr_chunk_fwd_untied / gdr_decode_step_untied take a write strength w; a misaligned
+    w is rejected before any launch, and the tied calls are the untied ones with w = NULL."""
+    L = G.lib()
+    d = _desc(G)
+    get = lambda n: ctypes.c_void_p(FAKE[n])
+    st = L.gdr_chunk_fwd_untied(ctypes.byref(d), get("q"), get("k"), get("v"), get("g"), get("beta"),
+                                ctypes.c_void_p(0x10004), None, None, get("o"), get("S_T"), None, 0, None)
+    assert st == G.GDR_ERR_INVALID_ARG
+    import torch
+    dd = G.DecDesc(2, 2, 64, 64, 1, 1, 1, 0, 1.0)
+    st = L.gdr_decode_step_untied(ctypes.byref(dd), get("q"), get("k"), get("v"), get("g"), get("beta"),
+                                  ctypes.c_void_p(0x10004), None, get("S_T"), get("o"), None)
+    assert st == G.GDR_ERR_INVALID_ARG

@@ -90,3 +90,25 @@ def test_decode_steps_match_forward(G):
     o_dec = torch.stack(outs, dim=1)
     assert U.max_rel(U.o_to_f64(o_dec), U.o_to_f64(o_fwd)) < 1e-4
     assert U.rel_l2(S.cpu().numpy(), S_fwd.cpu().numpy()) < 1e-4
+
+
+@pytest.mark.parametrize("dk,rot", [(128, False), (64, True), (32, True)])
+def test_decode_untied_parity(G, dk, rot):
+    """Separate erase (beta) and write (w) strengths against the fp64 oracle."""
+    import torch
+    d = I.make_decode(N=5, H=3, dk=dk, dv=dk, steps=3, dtype="bf16", seed=91 + dk, rotation=rot)
+    w = I.make_write_strength(93 + dk, (3, 5, 3))
+    S = U.to_torch(d.S, "cuda").clone()
+    S_ref = d.widened("S")
+    for s in range(3):
+        t = {key: U.to_torch(getattr(d, key)[s], "cuda") for key in ("q", "k", "v", "g", "beta")}
+        th = None if d.theta is None else U.to_torch(d.theta[s], "cuda")
+        o = G.decode_step(t["q"], t["k"], t["v"], t["g"], t["beta"], S, th, gate_mode=d.gate_mode,
+                          scale=d.scale, w=torch.from_numpy(w[s]).cuda())
+        o_ref, S_ref = oracle.gdr_decode_step(d.widened("q", s), d.widened("k", s), d.widened("v", s),
+                                              d.widened("g", s), d.widened("beta", s), S_ref,
+                                              d.widened("theta", s), d.gate_mode, d.scale,
+                                              w=w[s].astype(np.float64))
+        torch.cuda.synchronize()
+        assert U.max_rel(U.o_to_f64(o), o_ref) <= U.TOL_O["bf16"]
+    assert U.rel_l2(S.cpu().numpy(), S_ref) <= U.TOL_S

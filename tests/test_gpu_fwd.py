@@ -2,6 +2,7 @@
 import numpy as np
 import pytest
 
+import oracle
 from recurrent_state_memory_b200 import inputs as I
 
 import parity_util as U
@@ -231,3 +232,39 @@ def test_split_agrees_with_fused(G, rotation):
     o2, S2 = U.run_gpu_fwd(p, "tcgen05_split")
     assert U.max_rel(U.o_to_f64(o2), U.o_to_f64(o1)) <= U.TOL_O["bf16"]
     assert U.rel_l2(S2.cpu().numpy(), S1.cpu().numpy()) <= U.TOL_S
+
+
+UNTIED_CASES = [
+    # (algo, dtype, B, H, T, rotation, s0)
+    ("simt", "f32", 1, 2, 133, False, True),
+    ("simt", "bf16", 1, 2, 200, True, False),
+    ("tcgen05", "bf16", 2, 2, 333, False, True),
+    ("tcgen05", "bf16", 1, 3, 200, True, True),
+    ("tcgen05_split", "bf16", 2, 3, 333, False, True),
+    ("tcgen05_split", "bf16", 2, 2, 450, True, True),
+]
+
+
+@pytest.mark.parametrize("case", UNTIED_CASES, ids=lambda c: "{}_{}_B{}H{}T{}{}{}".format(
+    c[0], c[1], c[2], c[3], c[4], "_rot" if c[5] else "", "_s0" if c[6] else ""))
+def test_untied_parity(G, case):
+    """Separate erase (beta) and write (w) strengths: every kernel against the fp64 oracle."""
+    import torch
+    algo, dtype, B, H, T, rot, s0 = case
+    dk = 128 if algo != "simt" else 64
+    p = I.make_fwd(B, T, H, dk, dk, dtype=dtype, seed=700 + T, rotation=rot, s0_std=0.2 if s0 else None)
+    w = I.make_write_strength(701 + T, (B, T, H))
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "g", "beta", "theta", "S0")}
+    o, S = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["theta"], t["S0"], gate_mode=p.gate_mode,
+                       algo=algo, w=torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    assert G.query_device_status() == G.GDR_OK
+    o_ref, S_ref = oracle.gdr_fwd(p.widened("q"), p.widened("k"), p.widened("v"), p.widened("g"),
+                                  p.widened("beta"), p.widened("theta"), p.widened("S0"),
+                                  gate_mode=p.gate_mode, scale=p.scale, w=w.astype(np.float64))
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref)
+    # and it is not the tied result
+    o_t, _ = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["theta"], t["S0"], gate_mode=p.gate_mode,
+                         algo=algo)
+    torch.cuda.synchronize()
+    assert U.max_rel(U.o_to_f64(o_t), o_ref) > 10 * U.TOL_O[dtype]
