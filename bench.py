@@ -283,6 +283,36 @@ def run_ours(args):
         e2e = {"value": round(e_tok / (e_ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
 
+    # ---- separate erase / write strengths (CARVE): the same workload with a write strength w ----
+    untied = None
+    if not args.no_untied:
+        w_dev = torch.from_numpy(I.make_write_strength(rank_seed(cfg["seed"], rank) + 17, (p.B, p.T, p.H))).to(dev)
+
+        def ustep():
+            gdr.chunk_fwd(dv_t["q"], dv_t["k"], dv_t["v"], dv_t["g"], dv_t["beta"], dv_t["theta"], dv_t["S0"],
+                          gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o, S_T=S_T, stream=stream,
+                          workspace=wsp, w=w_dev)
+
+        for _ in range(3):
+            ustep()
+        torch.cuda.synchronize()
+        n_u = max(3, min(args.steps, 10))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_u):
+            ustep()
+        b.record(stream)
+        torch.cuda.synchronize()
+        u_ms = max_over_ranks(a.elapsed_time(b), dev)
+        u_tok = sum_over_ranks(float(tokens * n_u), dev)
+        u_bytes = algo_bytes + p.B * p.T * p.H * 4            # plus w
+        u_gbs = u_bytes / (a.elapsed_time(b) / n_u * 1e-3) / 1e9
+        untied = {"value": round(u_tok / (u_ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s",
+                  "ms_per_step": round(u_ms / n_u, 4), "steps": n_u, "kernel": kernel_name,
+                  "roofline": {"bound": "hbm", "achieved": round(u_gbs, 1), "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": round(u_gbs / peaks["hbm_gbs"], 4),
+                               "algorithmic_bytes_per_launch": int(u_bytes)}}
+
     # ---- decode: 256 sequences x 16 heads, fp32 state, one launch per step ----
     decode = None
     if not args.no_decode:
@@ -348,6 +378,7 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": args.steps * 1,
         "decode": decode,
+        "untied": untied,
         "cpu_baseline": cpu,
         "clocks": clk.summary(),
     }
@@ -433,6 +464,7 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-untied", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
