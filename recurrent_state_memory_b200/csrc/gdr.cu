@@ -217,9 +217,9 @@ static gdr_status encode_split_maps(const FwdParams& p, tcf::TmaMaps* tm) {
     return encode_bthd(fn, &tm->o, p.o, ob ? bf : f32, sizeof(OT), p, D, D, false);
 }
 
-template <int MODE, bool ROT, typename OT>
+template <int MODE, bool ROT, typename OT, bool UNT>
 static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
-    auto kern = tcf::chunk_fwd_tc_kernel<MODE, ROT, OT>;
+    auto kern = tcf::chunk_fwd_tc_kernel<MODE, ROT, OT, UNT>;
     constexpr int nt = tcf::nthreads<MODE>();
     constexpr uint32_t smem = tcf::smem_bytes<MODE>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -262,8 +262,14 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
 template <int MODE>
 static gdr_status dispatch_tc_mode(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws) {
     const bool ob = d->out_dtype == GDR_BF16;
-    if (d->rotation) return ob ? launch_tc<MODE, true, __nv_bfloat16>(p, st, ws) : launch_tc<MODE, true, float>(p, st, ws);
-    return ob ? launch_tc<MODE, false, __nv_bfloat16>(p, st, ws) : launch_tc<MODE, false, float>(p, st, ws);
+    if (p.w) {
+        if (d->rotation)
+            return ob ? launch_tc<MODE, true, __nv_bfloat16, true>(p, st, ws) : launch_tc<MODE, true, float, true>(p, st, ws);
+        return ob ? launch_tc<MODE, false, __nv_bfloat16, true>(p, st, ws) : launch_tc<MODE, false, float, true>(p, st, ws);
+    }
+    if (d->rotation)
+        return ob ? launch_tc<MODE, true, __nv_bfloat16, false>(p, st, ws) : launch_tc<MODE, true, float, false>(p, st, ws);
+    return ob ? launch_tc<MODE, false, __nv_bfloat16, false>(p, st, ws) : launch_tc<MODE, false, float, false>(p, st, ws);
 }
 
 // ----------------------------------------------------------------- decode ----

@@ -212,7 +212,9 @@ __device__ __forceinline__ uint4 pack8(const float* m8) {
 // warps 4-7 convert the Wm tiles and write o.  Every other CTA is a prep worker with two
 // independent 8-warp groups that compute chunks in chunk-major task order and write their
 // operand tiles into the ring.  The grid must be co-resident (cooperative launch).
-template <int MODE, bool ROT, typename OT>
+// UNT: a write strength w separate from beta (p.w set); a compile-time switch so that the
+// tied kernel carries none of its cost.
+template <int MODE, bool ROT, typename OT, bool UNT>
 __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdParams p, TcExtra x, SplitArgs sa,
                                                               const __grid_constant__ TmaMaps tm) {
     using namespace tc;
@@ -248,7 +250,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
     const __nv_bfloat16* __restrict__ v = static_cast<const __nv_bfloat16*>(p.v);
     OT* __restrict__ o = static_cast<OT*>(p.o);
     const int nchunks = (p.T + C - 1) / C;
-    const bool untied = p.w != nullptr;     // a write strength w separate from beta
+    constexpr bool untied = UNT;            // a write strength w separate from beta
     auto chunk_len = [&](int c) -> int { return min(C, p.T - c * C); };
     auto tokh = [&](int bhx, int c, int r) -> size_t {
         return ((size_t)(bhx / p.H) * p.T + (c * C + r)) * p.H + (bhx % p.H);
