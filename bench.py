@@ -82,6 +82,7 @@ KERNEL_SOURCES = {
     "gdr_chunk_fwd_simt": ["simt_fwd.cuh", "common.cuh"],
     "gdr_chunk_fwd_tcgen05": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
     "gdr_chunk_fwd_tcgen05_split": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
+    "gdr_chunk_fwd_tcgen05_waves": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
     "gdr_decode_step": ["decode.cuh", "common.cuh"],
 }
 
@@ -376,7 +377,7 @@ def run_ours(args):
         "tflops_algorithmic": round(tflops, 2),
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": args.steps * 1,
+        "gpu_launches": args.steps * (2 if resolved == "tcgen05_waves" else 1),
         "decode": decode,
         "untied": untied,
         "cpu_baseline": cpu,
@@ -458,7 +459,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
-    ap.add_argument("--algo", choices=["auto", "simt", "tcgen05", "tcgen05_split"], default="auto")
+    ap.add_argument("--algo", choices=["auto", "simt", "tcgen05", "tcgen05_split", "tcgen05_waves"], default="auto")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-decode", action="store_true")

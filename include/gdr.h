@@ -72,7 +72,8 @@ typedef enum { GDR_GATE_LOGDECAY = 0, GDR_GATE_NEG_SOFTPLUS = 1 } gdr_gate_mode;
 
 typedef enum {
     GDR_ALGO_AUTO = 0,    /* tensor-core chunk kernel when supported (the split one when
-                             2*B*H <= SM count and T > 64), else SIMT */
+                             2*B*H <= SM count and T > 64, the waves mix when B*H exceeds the SM
+                             count and its remainder would take the split kernel), else SIMT */
     GDR_ALGO_SIMT = 1,    /* fp32 CUDA-core chunk-WY kernel (every supported shape) */
     GDR_ALGO_TCGEN05 = 2, /* tcgen05/TMEM chunk-WY kernel, one CTA per (batch, head):
                              bf16 q/k/v, dk = dv = 128 */
@@ -80,7 +81,11 @@ typedef enum {
                              while every other SM prepares chunks (two at a time), handed
                              over through a ring in the workspace (needs B*H < SM count;
                              cooperative launch); results agree with GDR_ALGO_TCGEN05 to
-                             rounding */
+                             rounding */,
+    GDR_ALGO_TCGEN05_WAVES = 4 /* more heads than SMs: the fused kernel for whole waves of
+                             SM-count heads, then the split kernel for the last partial wave
+                             when it is at most half the SM count (else fused throughout);
+                             workspace for the split part */
 } gdr_algo;
 
 /* Shape and mode of one chunked forward call. */

@@ -79,33 +79,41 @@ static int device_sm_count() {
     return n;
 }
 
-// The split kernel pays off while the heads leave most SMs to prep workers (each head's
-// chain needs about three workers to keep up) and there is more than one chunk.
 // The split kernel gives each head one chain CTA and shares the remaining SMs among prep
 // workers; with more than half of the SMs taken by chains, too few workers are left and the
 // fused kernel (prep and chain of a head in one CTA) is faster.
+static bool split_fits_heads(long long nh, int sms, int T) { return nh >= 1 && 2 * nh <= (long long)sms && T > 64; }
 static bool split_fits(const gdr_fwd_desc* d, int sms) {
+    return split_fits_heads((long long)d->B * d->H, sms, d->T);
+}
+// More heads than SMs: the fused kernel runs whole waves of SM-count heads; a last partial
+// wave that would leave more than half of the SMs idle goes to the split kernel instead.
+static long long waves_remainder(const gdr_fwd_desc* d, int sms) {
     const long long nh = (long long)d->B * d->H;
-    return nh >= 1 && 2 * nh <= (long long)sms && d->T > 64;
+    return nh > sms ? nh % sms : 0;
+}
+static bool waves_fit(const gdr_fwd_desc* d, int sms) {
+    const long long rem = waves_remainder(d, sms);
+    return rem > 0 && split_fits_heads(rem, sms, d->T);
 }
 
 // The algorithm a descriptor runs with: AUTO takes a tensor-core kernel when it supports
-// the shape and dtype, the split one when the heads leave room for prep workers.
+// the shape and dtype, the split one when the heads leave room for prep workers, the waves
+// mix when a partial last wave would leave most SMs idle.
 static gdr_algo resolve_algo(const gdr_fwd_desc* d) {
     if (d->algo == GDR_ALGO_AUTO) {
         if (!tc_supported(d)) return GDR_ALGO_SIMT;
-        return split_fits(d, device_sm_count()) ? GDR_ALGO_TCGEN05_SPLIT : GDR_ALGO_TCGEN05;
+        const int sms = device_sm_count();
+        if (split_fits(d, sms)) return GDR_ALGO_TCGEN05_SPLIT;
+        return waves_fit(d, sms) ? GDR_ALGO_TCGEN05_WAVES : GDR_ALGO_TCGEN05;
     }
     return d->algo;
 }
 
-static size_t split_ring_bytes(const gdr_fwd_desc* d) {
-    return (size_t)d->B * d->H * tcf::RING * tcf::SLOT_BYTES;
+static size_t split_workspace_heads(size_t nh) {
+    return nh * tcf::RING * tcf::SLOT_BYTES + (nh * tcf::RING + nh) * sizeof(unsigned int);
 }
-static size_t split_workspace_bytes(const gdr_fwd_desc* d) {
-    const size_t nh = (size_t)d->B * d->H;
-    return split_ring_bytes(d) + (nh * tcf::RING + nh) * sizeof(unsigned int);
-}
+static size_t split_workspace_bytes(const gdr_fwd_desc* d) { return split_workspace_heads((size_t)d->B * d->H); }
 
 // ---- scratch for gdr_chunk_fwd_noalloc ---------------------------------------------------
 // The split kernel's ring and flags for at most NOALLOC_MAX_HEADS heads, as a file-scope
@@ -149,10 +157,11 @@ static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
         return fail(GDR_ERR_INVALID_ARG, "bad gate_mode%s");
     if (d->rotation != 0 && d->rotation != 1) return fail(GDR_ERR_INVALID_ARG, "rotation must be 0 or 1%s");
     if (d->algo != GDR_ALGO_AUTO && d->algo != GDR_ALGO_SIMT && d->algo != GDR_ALGO_TCGEN05 &&
-        d->algo != GDR_ALGO_TCGEN05_SPLIT)
+        d->algo != GDR_ALGO_TCGEN05_SPLIT && d->algo != GDR_ALGO_TCGEN05_WAVES)
         return fail(GDR_ERR_INVALID_ARG, "bad algo%s");
     if ((long long)d->B * d->H > 0x7fffffffLL) return fail(GDR_ERR_INVALID_ARG, "B*H too large%s");
-    if ((d->algo == GDR_ALGO_TCGEN05 || d->algo == GDR_ALGO_TCGEN05_SPLIT) && !tc_supported(d))
+    if ((d->algo == GDR_ALGO_TCGEN05 || d->algo == GDR_ALGO_TCGEN05_SPLIT || d->algo == GDR_ALGO_TCGEN05_WAVES) &&
+        !tc_supported(d))
         return fail(GDR_ERR_UNSUPPORTED, "the tcgen05 kernels need bf16 q/k/v and dk = dv = 128%s");
     return GDR_OK;
 }
@@ -231,14 +240,14 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
     tcf::TmaMaps tm;
     memset(&tm, 0, sizeof(tm));
     if (MODE == 0) {
-        kern<<<p.B * p.H, nt, smem, st>>>(p, x, sa, tm);
+        kern<<<p.nheads, nt, smem, st>>>(p, x, sa, tm);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
         return GDR_OK;
     }
     // Split: the whole grid must be resident at once (one CTA per SM), which a cooperative
     // launch guarantees or refuses.
-    const int nh = p.B * p.H;
+    const int nh = p.nheads;
     const int sms = device_sm_count();
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem);
@@ -319,7 +328,9 @@ const char* gdr_last_error_detail(void) { return t_detail; }
 
 size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc) {
     if (check_fwd_desc(desc) != GDR_OK) return 0;
-    if (resolve_algo(desc) == GDR_ALGO_TCGEN05_SPLIT) return split_workspace_bytes(desc);
+    const gdr_algo a = resolve_algo(desc);
+    if (a == GDR_ALGO_TCGEN05_SPLIT) return split_workspace_bytes(desc);
+    if (a == GDR_ALGO_TCGEN05_WAVES) return split_workspace_heads((size_t)waves_remainder(desc, device_sm_count()));
     return 0;
 }
 
@@ -354,6 +365,7 @@ gdr_status gdr_chunk_fwd_untied(const gdr_fwd_desc* d, const void* q, const void
 
     FwdParams p;
     p.B = d->B; p.H = d->H; p.T = d->T; p.dv = d->dv;
+    p.head0 = 0; p.nheads = d->B * d->H;
     p.gate_mode = (int)d->gate_mode;
     p.scale = d->scale;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.theta = theta;
@@ -365,7 +377,22 @@ gdr_status gdr_chunk_fwd_untied(const gdr_fwd_desc* d, const void* q, const void
         if (!aligned16(workspace)) return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned%s");
         return dispatch_tc_mode<1>(d, p, st, workspace);
     }
-    if (algo == GDR_ALGO_TCGEN05 || algo == GDR_ALGO_TCGEN05_SPLIT) return dispatch_tc_mode<0>(d, p, st, nullptr);
+    if (algo == GDR_ALGO_TCGEN05_WAVES && d->T > 0) {
+        const long long rem = waves_remainder(d, device_sm_count());
+        if (rem > 0 && split_fits_heads(rem, device_sm_count(), d->T)) {
+            if (!aligned16(workspace)) return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned%s");
+            FwdParams pf = p, ps = p;
+            pf.nheads = (int)(p.nheads - rem);
+            ps.head0 = pf.nheads;
+            ps.nheads = (int)rem;
+            s = dispatch_tc_mode<0>(d, pf, st, nullptr);           // whole waves, fused
+            if (s != GDR_OK) return s;
+            return dispatch_tc_mode<1>(d, ps, st, workspace);      // the last partial wave, split
+        }
+        return dispatch_tc_mode<0>(d, p, st, nullptr);
+    }
+    if (algo == GDR_ALGO_TCGEN05 || algo == GDR_ALGO_TCGEN05_SPLIT || algo == GDR_ALGO_TCGEN05_WAVES)
+        return dispatch_tc_mode<0>(d, p, st, nullptr);
     return d->rotation ? dispatch_simt_dk<true>(d, p, st) : dispatch_simt_dk<false>(d, p, st);
 }
 
@@ -464,6 +491,7 @@ gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* d, const void* q, const voi
         return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
     FwdParams p;
     p.B = d->B; p.H = d->H; p.T = d->T; p.dv = d->dv;
+    p.head0 = 0; p.nheads = d->B * d->H;
     p.gate_mode = (int)d->gate_mode;
     p.scale = d->scale;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = nullptr; p.theta = theta;

@@ -26,6 +26,7 @@ namespace gdr {
 
 struct FwdParams {
     int B, H, T, dv;
+    int head0, nheads;      // tensor-core kernels: heads [head0, head0 + nheads) of b*H + h
     int gate_mode;
     float scale;
     const void* q;

@@ -242,9 +242,12 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3;
-    const int NH = p.B * p.H;
+    // Heads [p.head0, p.head0 + p.nheads) of the flattened b*H + h; indices below are local
+    // (ring slots, task numbers) unless named global.
+    const int NH = p.nheads;
     const bool chain_cta = (MODE == 0) || ((int)blockIdx.x < NH);
     const int bh = chain_cta ? (int)blockIdx.x : 0;
+    const int gbh = p.head0 + bh;           // this chain's global head
     const __nv_bfloat16* __restrict__ q = static_cast<const __nv_bfloat16*>(p.q);
     const __nv_bfloat16* __restrict__ k = static_cast<const __nv_bfloat16*>(p.k);
     const __nv_bfloat16* __restrict__ v = static_cast<const __nv_bfloat16*>(p.v);
@@ -252,8 +255,9 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
     const int nchunks = (p.T + C - 1) / C;
     constexpr bool untied = UNT;            // a write strength w separate from beta
     auto chunk_len = [&](int c) -> int { return min(C, p.T - c * C); };
-    auto tokh = [&](int bhx, int c, int r) -> size_t {
-        return ((size_t)(bhx / p.H) * p.T + (c * C + r)) * p.H + (bhx % p.H);
+    auto tokh = [&](int bhx, int c, int r) -> size_t {      // bhx: local head
+        const int gx = p.head0 + bhx;
+        return ((size_t)(gx / p.H) * p.T + (c * C + r)) * p.H + (gx % p.H);
     };
     auto tok = [&](int c, int r) -> size_t { return tokh(bh, c, r); };
     // Chain-side buffers of chunk c: fused mode reads the prep group's double buffers, split
@@ -386,7 +390,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             pub_c = -1;
         };
         auto stage_part = [&](int itx, int part) {
-            const int c2 = task_c(itx), b2 = task_bh(itx);
+            const int c2 = task_c(itx), b2 = p.head0 + task_bh(itx);     // global head
             const int bb = b2 / p.H, hh = b2 % p.H;
             if (part == 0) {
                 staged = itx + 1;
@@ -1065,7 +1069,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     const int col0 = g * 16;
                     float s[16];
                     if (p.S0) {
-                        const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)bh * D + row) * D + col0);
+                        const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)gbh * D + row) * D + col0);
 #pragma unroll
                         for (int u4 = 0; u4 < 4; ++u4) {
                             const float4 t4 = src[u4];
@@ -1135,7 +1139,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     tmem_ld32(tq + COL_S + g * 32, s32);
                     if (last) {
                         if (p.S_T) {
-                            float4* dst = reinterpret_cast<float4*>(p.S_T + ((size_t)bh * D + row) * D + g * 32);
+                            float4* dst = reinterpret_cast<float4*>(p.S_T + ((size_t)gbh * D + row) * D + g * 32);
 #pragma unroll
                             for (int u4 = 0; u4 < 8; ++u4)
                                 dst[u4] = make_float4(s32[4 * u4], s32[4 * u4 + 1], s32[4 * u4 + 2], s32[4 * u4 + 3]);
@@ -1203,7 +1207,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 ebar();
                 if (et == 0) {
                     mbar_arrive(bar_ofree);
-                    tma_store_4d(&tm.o, 0, bh % p.H, c * C, bh / p.H, sb + OFF_OSTG);   // rows past T clipped
+                    tma_store_4d(&tm.o, 0, gbh % p.H, c * C, gbh / p.H, sb + OFF_OSTG);   // rows past T clipped
                     bulk_commit();
                 }
                 if (c + 1 < nchunks) ok = convert_w(c + 1);
@@ -1277,7 +1281,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 fence_proxy_async_smem();
                 cbar();
                 if (row == 0) {
-                    tma_store_4d(&tm.o, 0, bh % p.H, c * C, bh / p.H, sb + OFF_OSTG);   // rows past T clipped
+                    tma_store_4d(&tm.o, 0, gbh % p.H, c * C, gbh / p.H, sb + OFF_OSTG);   // rows past T clipped
                     bulk_commit();
                 }
                 (void)Lc;
@@ -1319,7 +1323,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 const int col0 = g * 16;
                 float s[16];
                 if (p.S0) {
-                    const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)bh * D + row) * D + col0);
+                    const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)gbh * D + row) * D + col0);
 #pragma unroll
                     for (int u4 = 0; u4 < 4; ++u4) {
                         const float4 t4 = src[u4];
@@ -1422,7 +1426,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                         scale_cols(c16, s, rho_C);
                         if (last) {
                             if (p.S_T) {
-                                float4* dst = reinterpret_cast<float4*>(p.S_T + ((size_t)bh * D + row) * D + c16);
+                                float4* dst = reinterpret_cast<float4*>(p.S_T + ((size_t)gbh * D + row) * D + c16);
 #pragma unroll
                                 for (int u4 = 0; u4 < 4; ++u4)
                                     dst[u4] = make_float4(s[4 * u4], s[4 * u4 + 1], s[4 * u4 + 2], s[4 * u4 + 3]);
@@ -1464,7 +1468,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     }
                     bulk_g2s(sb + slot_base(c) + SL_VEC, src + SL_VEC, SLOT_BYTES - SL_VEC, bar_full + bufi);
                     // V of this chunk, two 64-column boxes straight into the MN-major layout
-                    const int bb = bh / p.H, hh = bh % p.H;
+                    const int bb = gbh / p.H, hh = gbh % p.H;
                     tma_load_4d(sb + slot_base(c) + SL_V, &tm.v, 0, hh, c * C, bb, bar_full + bufi);
                     tma_load_4d(sb + slot_base(c) + SL_V + 8192u, &tm.v, 64, hh, c * C, bb, bar_full + bufi);
                     // the ring slot may be reused once its bytes have landed here
@@ -1478,7 +1482,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
     }
     if (nchunks == 0 && p.S_T && chain_cta) {
         for (int e = tid; e < D * D; e += nthreads<MODE>())
-            p.S_T[(size_t)bh * D * D + e] = p.S0 ? p.S0[(size_t)bh * D * D + e] : 0.f;
+            p.S_T[(size_t)gbh * D * D + e] = p.S0 ? p.S0[(size_t)gbh * D * D + e] : 0.f;
     }
     tc_fence_before();
     __syncthreads();

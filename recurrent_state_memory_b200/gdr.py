@@ -24,7 +24,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gdr.h")
  GDR_ERR_RANGE) = range(7)
 GDR_F32, GDR_BF16 = 0, 1
 GATE_LOGDECAY, GATE_NEG_SOFTPLUS = 0, 1
-ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_split": 3}
+ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_split": 3, "tcgen05_waves": 4}
 ALGO_NAMES = {v: k for k, v in ALGOS.items()}
 
 

@@ -216,7 +216,11 @@ def test_auto_picks_tensor_cores_for_bf16_d128(G):
         if expect == "tcgen05_split":
             assert G.workspace_bytes(d) >= B * H * 8 * 67840
     d = G.fwd_desc(16, 12, 4096, 128, 128, torch.bfloat16, torch.bfloat16)
-    assert G.resolved_algo(d) == "tcgen05"                    # many heads: fused
+    rem = (16 * 12) % sms if 16 * 12 > sms else 0
+    expect = "tcgen05_waves" if 0 < rem and 2 * rem <= sms else "tcgen05"   # many heads
+    assert G.resolved_algo(d) == expect
+    if expect == "tcgen05_waves":
+        assert G.workspace_bytes(d) >= rem * 8 * 67840
     d = G.fwd_desc(1, 1, 64, 64, 64, torch.bfloat16, torch.bfloat16)
     assert G.resolved_algo(d) == "simt"
     d = G.fwd_desc(1, 1, 64, 128, 128, torch.float32, torch.float32)
@@ -268,3 +272,20 @@ def test_untied_parity(G, case):
                          algo=algo)
     torch.cuda.synchronize()
     assert U.max_rel(U.o_to_f64(o_t), o_ref) > 10 * U.TOL_O[dtype]
+
+
+@pytest.mark.parametrize("B,rotation", [(1, False), (2, True)])
+def test_waves_split_remainder_parity(G, B, rotation):
+    """More heads than SMs: whole waves on the fused kernel, the remainder on the split
+    kernel (heads offset into the batch), every head against the oracle."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    nh = sms + 12 + (B - 1) * 2                       # a remainder of 12-14 heads
+    H = nh // B
+    p = I.make_fwd(B, 130, H, 128, 128, dtype="bf16", seed=801 + B, rotation=rotation, s0_std=0.2)
+    d = G.fwd_desc(B, H, 130, 128, 128, torch.bfloat16, torch.bfloat16, p.gate_mode, rotation)
+    assert G.resolved_algo(d) == "tcgen05_waves"
+    o, S = U.run_gpu_fwd(p, "auto")
+    assert G.query_device_status() == G.GDR_OK
+    o_ref, S_ref = U.oracle_fwd(p)
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref)
