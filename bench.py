@@ -314,6 +314,33 @@ def run_ours(args):
                                "unit": "GB/s", "frac": round(u_gbs / peaks["hbm_gbs"], 4),
                                "algorithmic_bytes_per_launch": int(u_bytes)}}
 
+    # ---- fused L2 normalisation of q and k: the same workload with the prologue on ----
+    l2norm = None
+    if not args.no_untied:
+        def nstep():
+            gdr.chunk_fwd(dv_t["q"], dv_t["k"], dv_t["v"], dv_t["g"], dv_t["beta"], dv_t["theta"], dv_t["S0"],
+                          gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o, S_T=S_T, stream=stream,
+                          workspace=wsp, qk_l2norm=True)
+
+        for _ in range(3):
+            nstep()
+        torch.cuda.synchronize()
+        n_n = max(3, min(args.steps, 10))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_n):
+            nstep()
+        b.record(stream)
+        torch.cuda.synchronize()
+        n_ms = max_over_ranks(a.elapsed_time(b), dev)
+        n_tok = sum_over_ranks(float(tokens * n_n), dev)
+        n_gbs = algo_bytes / (a.elapsed_time(b) / n_n * 1e-3) / 1e9
+        l2norm = {"value": round(n_tok / (n_ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s",
+                  "ms_per_step": round(n_ms / n_n, 4), "steps": n_n, "kernel": kernel_name,
+                  "roofline": {"bound": "hbm", "achieved": round(n_gbs, 1), "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": round(n_gbs / peaks["hbm_gbs"], 4),
+                               "algorithmic_bytes_per_launch": int(algo_bytes)}}
+
     # ---- decode: 256 sequences x 16 heads, fp32 state, one launch per step ----
     decode = None
     if not args.no_decode:
@@ -380,6 +407,7 @@ def run_ours(args):
         "gpu_launches": args.steps * (2 if resolved == "tcgen05_waves" else 1),
         "decode": decode,
         "untied": untied,
+        "qk_l2norm": l2norm,
         "cpu_baseline": cpu,
         "clocks": clk.summary(),
     }
@@ -465,7 +493,8 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--no-untied", action="store_true")
+    ap.add_argument("--no-untied", action="store_true", help="skip the separate-write-strength and "
+                    "fused-L2-norm measurements")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -99,6 +99,8 @@ typedef struct {
     int rotation;         /* 0: real key-axis decay; 1: 2x2 rotation-decay blocks */
     float scale;          /* multiplies q (1.0 for none) */
     gdr_algo algo;
+    int qk_l2norm;        /* 1: the kernels L2-normalise q_t and k_t per token and head first,
+                             x / sqrt(sum x^2 + 1e-6) in fp32, before the scale (0: as given) */
 } gdr_fwd_desc;
 
 /* Shape and mode of one decode step over N independent sequences. */
@@ -109,6 +111,7 @@ typedef struct {
     gdr_gate_mode gate_mode;
     int rotation;
     float scale;
+    int qk_l2norm;        /* as in gdr_fwd_desc */
 } gdr_dec_desc;
 
 /* GDR_ABI_VERSION of the loaded library. */

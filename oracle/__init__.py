@@ -56,8 +56,19 @@ def num_threads() -> int:
     return int(_load().oracle_num_threads())
 
 
+L2NORM_EPS = 1e-6
+
+
+def l2_normalise(x):
+    """x / sqrt(sum x^2 + 1e-6) over the last axis, in fp64: the L2 normalisation of q and k
+    that the layer applies before the recurrence (task statement; CARVE / KDA mixers),
+    with a small epsilon so that a zero vector stays zero."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + L2NORM_EPS)
+
+
 def gdr_fwd(q, k, v, g, beta, theta=None, S0=None, gate_mode=GATE_LOGDECAY, scale=1.0,
-            want_state=True, w=None):
+            want_state=True, w=None, qk_l2norm=False):
     """Token-by-token fp64 forward.
 
     q, k: [B,T,H,dk]; v: [B,T,H,dv]; g: [B,T,H,dk] (or dk/2 with rotation);
@@ -66,6 +77,8 @@ def gdr_fwd(q, k, v, g, beta, theta=None, S0=None, gate_mode=GATE_LOGDECAY, scal
     Returns (o [B,T,H,dv], S_T [B,H,dv,dk] or None), both float64.
     """
     q, k, v, g, beta, w, theta, S0 = map(_f64, (q, k, v, g, beta, w, theta, S0))
+    if qk_l2norm:
+        q, k = l2_normalise(q), l2_normalise(k)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     rotation = theta is not None
@@ -84,10 +97,13 @@ def gdr_fwd(q, k, v, g, beta, theta=None, S0=None, gate_mode=GATE_LOGDECAY, scal
     return o, S_T
 
 
-def gdr_decode_step(q, k, v, g, beta, S, theta=None, gate_mode=GATE_LOGDECAY, scale=1.0, w=None):
+def gdr_decode_step(q, k, v, g, beta, S, theta=None, gate_mode=GATE_LOGDECAY, scale=1.0, w=None,
+                    qk_l2norm=False):
     """One fp64 decode step (w: write strength [N,H] or None for w = beta).
     S [N,H,dv,dk] is NOT modified; returns (o, S_new)."""
     q, k, v, g, beta, w, theta = map(_f64, (q, k, v, g, beta, w, theta))
+    if qk_l2norm:
+        q, k = l2_normalise(q), l2_normalise(k)
     S_new = np.array(S, dtype=np.float64, copy=True, order="C")
     N, H, dk = q.shape
     dv = v.shape[-1]

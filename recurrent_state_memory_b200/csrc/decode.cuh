@@ -27,6 +27,7 @@ struct DecParams {
     const float* g;
     const float* beta;
     const float* w;         // write strength [N,H], or nullptr: w = beta
+    int qk_norm;            // 1: L2-normalise q and k first (x / sqrt(sum x^2 + 1e-6))
     const float* theta;
     float* S;
     void* o;
@@ -83,7 +84,24 @@ __global__ void __launch_bounds__(WARPS * 32) decode_kernel(DecParams p) {
     for (int u = 0; u < VEC; ++u) {
         const int d = lane * VEC + u;
         kk[u] = ld_f32(k + d);
-        qq[u] = p.scale * ld_f32(q + d);
+        qq[u] = ld_f32(q + d);
+    }
+    {
+        float ik = 1.f, iq = p.scale;
+        if (p.qk_norm) {
+            float sk = 0.f, sq = 0.f;
+#pragma unroll
+            for (int u = 0; u < VEC; ++u) { sk = fmaf(kk[u], kk[u], sk); sq = fmaf(qq[u], qq[u], sq); }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            }
+            ik = rsqrtf(sk + 1e-6f);
+            iq = p.scale * rsqrtf(sq + 1e-6f);
+        }
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) { kk[u] *= ik; qq[u] *= iq; }
     }
     if constexpr (!ROT) {
 #pragma unroll

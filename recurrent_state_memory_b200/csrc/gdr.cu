@@ -156,6 +156,7 @@ static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
     if (d->gate_mode != GDR_GATE_LOGDECAY && d->gate_mode != GDR_GATE_NEG_SOFTPLUS)
         return fail(GDR_ERR_INVALID_ARG, "bad gate_mode%s");
     if (d->rotation != 0 && d->rotation != 1) return fail(GDR_ERR_INVALID_ARG, "rotation must be 0 or 1%s");
+    if (d->qk_l2norm != 0 && d->qk_l2norm != 1) return fail(GDR_ERR_INVALID_ARG, "qk_l2norm must be 0 or 1%s");
     if (d->algo != GDR_ALGO_AUTO && d->algo != GDR_ALGO_SIMT && d->algo != GDR_ALGO_TCGEN05 &&
         d->algo != GDR_ALGO_TCGEN05_SPLIT && d->algo != GDR_ALGO_TCGEN05_WAVES)
         return fail(GDR_ERR_INVALID_ARG, "bad algo%s");
@@ -226,9 +227,9 @@ static gdr_status encode_split_maps(const FwdParams& p, tcf::TmaMaps* tm) {
     return encode_bthd(fn, &tm->o, p.o, ob ? bf : f32, sizeof(OT), p, D, D, false);
 }
 
-template <int MODE, bool ROT, typename OT, bool UNT>
+template <int MODE, bool ROT, typename OT, bool EXT>
 static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
-    auto kern = tcf::chunk_fwd_tc_kernel<MODE, ROT, OT, UNT>;
+    auto kern = tcf::chunk_fwd_tc_kernel<MODE, ROT, OT, EXT>;
     constexpr int nt = tcf::nthreads<MODE>();
     constexpr uint32_t smem = tcf::smem_bytes<MODE>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -271,7 +272,7 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
 template <int MODE>
 static gdr_status dispatch_tc_mode(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws) {
     const bool ob = d->out_dtype == GDR_BF16;
-    if (p.w) {
+    if (p.w || p.qk_norm) {      // the kernel with the optional features
         if (d->rotation)
             return ob ? launch_tc<MODE, true, __nv_bfloat16, true>(p, st, ws) : launch_tc<MODE, true, float, true>(p, st, ws);
         return ob ? launch_tc<MODE, false, __nv_bfloat16, true>(p, st, ws) : launch_tc<MODE, false, float, true>(p, st, ws);
@@ -366,6 +367,7 @@ gdr_status gdr_chunk_fwd_untied(const gdr_fwd_desc* d, const void* q, const void
     FwdParams p;
     p.B = d->B; p.H = d->H; p.T = d->T; p.dv = d->dv;
     p.head0 = 0; p.nheads = d->B * d->H;
+    p.qk_norm = d->qk_l2norm;
     p.gate_mode = (int)d->gate_mode;
     p.scale = d->scale;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.theta = theta;
@@ -414,6 +416,7 @@ gdr_status gdr_decode_step_untied(const gdr_dec_desc* d, const void* q, const vo
     if (d->gate_mode != GDR_GATE_LOGDECAY && d->gate_mode != GDR_GATE_NEG_SOFTPLUS)
         return fail(GDR_ERR_INVALID_ARG, "bad gate_mode%s");
     if (d->rotation != 0 && d->rotation != 1) return fail(GDR_ERR_INVALID_ARG, "rotation must be 0 or 1%s");
+    if (d->qk_l2norm != 0 && d->qk_l2norm != 1) return fail(GDR_ERR_INVALID_ARG, "qk_l2norm must be 0 or 1%s");
     if (d->N == 0 || d->H == 0) return GDR_OK;
     if (!q || !k || !v || !g || !beta || !S || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta, S and o are required%s");
     if (d->rotation && !theta) return fail(GDR_ERR_INVALID_ARG, "theta is required with rotation%s");
@@ -426,6 +429,7 @@ gdr_status gdr_decode_step_untied(const gdr_dec_desc* d, const void* q, const vo
     p.gate_mode = (int)d->gate_mode;
     p.scale = d->scale;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.theta = theta; p.S = S; p.o = o;
+    p.qk_norm = d->qk_l2norm;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d->rotation) {
         switch (d->dk) {
@@ -492,6 +496,7 @@ gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* d, const void* q, const voi
     FwdParams p;
     p.B = d->B; p.H = d->H; p.T = d->T; p.dv = d->dv;
     p.head0 = 0; p.nheads = d->B * d->H;
+    p.qk_norm = d->qk_l2norm;
     p.gate_mode = (int)d->gate_mode;
     p.scale = d->scale;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = nullptr; p.theta = theta;

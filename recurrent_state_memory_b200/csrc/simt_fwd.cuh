@@ -27,6 +27,7 @@ namespace gdr {
 struct FwdParams {
     int B, H, T, dv;
     int head0, nheads;      // tensor-core kernels: heads [head0, head0 + nheads) of b*H + h
+    int qk_norm;            // 1: L2-normalise q_t and k_t first (x / sqrt(sum x^2 + 1e-6))
     int gate_mode;
     float scale;
     const void* q;
@@ -117,10 +118,33 @@ __global__ void __launch_bounds__(NT) chunk_fwd_kernel(FwdParams p) {
             float kv = 0.f, qv = 0.f;
             if (r < Lc) {
                 kv = ld_f32(k + tok(r) * DK + d);
-                qv = p.scale * ld_f32(q + tok(r) * DK + d);
+                qv = ld_f32(q + tok(r) * DK + d);
+                if (!p.qk_norm) qv *= p.scale;
             }
             kc[r * KS + d] = kv;
             qc[r * KS + d] = qv;
+        }
+        if (p.qk_norm) {
+            // L2-normalise every token's k and q (one warp per row), then scale q
+            __syncthreads();
+            const int wid = tid >> 5, ln = tid & 31;
+            for (int r = wid; r < C; r += NT / 32) {
+                float sk = 0.f, sq = 0.f;
+                for (int d = ln; d < DK; d += 32) {
+                    sk = fmaf(kc[r * KS + d], kc[r * KS + d], sk);
+                    sq = fmaf(qc[r * KS + d], qc[r * KS + d], sq);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                }
+                const float ik = rsqrtf(sk + 1e-6f), iq = p.scale * rsqrtf(sq + 1e-6f);
+                for (int d = ln; d < DK; d += 32) {
+                    kc[r * KS + d] *= ik;
+                    qc[r * KS + d] *= iq;
+                }
+            }
         }
         for (int idx = tid; idx < C * NG; idx += NT) {
             const int r = idx / NG, jg = idx % NG;

@@ -76,6 +76,8 @@ constexpr uint32_t OFF_BAR = (OFF_VEC + 2 * VEC_FLOATS * 4 + 63) & ~63u;
 constexpr uint32_t BAR_BYTES = 256;                  // mbarriers, TMEM address, flags
 // Tw = Tm diag(w) K-major, for a write strength w separate from the erase strength beta
 constexpr uint32_t OFF_TW = (OFF_BAR + BAR_BYTES + 1023) & ~1023u;
+// per-token inverse L2 norms of k and q (fused L2-normalisation only): [64][2] fp32
+constexpr uint32_t OFF_NRM = OFF_TW + 8192;
 
 // Split mode: a per-head ring in global memory carries each chunk's operands from the prep
 // workers to the chain CTA.  Slot layout (bytes), identical to the chain's shared-memory copy:
@@ -108,7 +110,8 @@ constexpr uint32_t G_TW = 65536;     // Tw K-major (separate write strength only
 constexpr uint32_t G_AF = 73728;     // fp32 A [64][68]
 constexpr uint32_t G_TF = G_AF + 64 * AS * 4;   // fp32 Tm [64][68]
 constexpr uint32_t G_VEC = G_TF + 64 * AS * 4;  // beta, rho_ref, rho_C
-constexpr uint32_t G_STRIDE = (G_VEC + VEC_FLOATS * 4 + 1023) & ~1023u;
+constexpr uint32_t G_NRM = G_VEC + VEC_FLOATS * 4;   // inverse L2 norms [64][2] fp32
+constexpr uint32_t G_STRIDE = (G_NRM + 512 + 1023) & ~1023u;
 constexpr int NT_SPLIT = 2 * NPREP;             // two prep groups (16 warps: 128 registers a thread)
 constexpr uint32_t OFF_BAR_SPLIT = 2 * G_STRIDE;
 static_assert(2 * SLOT_STRIDE + 64 * 128 * 4 <= OFF_BAR_SPLIT, "chain slot buffers overlap the barriers");
@@ -118,9 +121,9 @@ template <int MODE> __host__ __device__ constexpr int nthreads() { return MODE =
 template <int MODE> __host__ __device__ constexpr uint32_t off_bar() { return MODE == 0 ? OFF_BAR : OFF_BAR_SPLIT; }
 // dynamic shared memory, with slack for the 1024-byte alignment of the base
 template <int MODE> __host__ __device__ constexpr uint32_t smem_bytes() {
-    return (MODE == 0 ? OFF_TW + 8192 : OFF_BAR_SPLIT + BAR_BYTES) + 1024;
+    return (MODE == 0 ? OFF_NRM + 512 : OFF_BAR_SPLIT + BAR_BYTES) + 1024;
 }
-static_assert(OFF_TW + 8192 + 1024 <= 232448 && OFF_BAR_SPLIT + BAR_BYTES + 1024 <= 232448,
+static_assert(OFF_NRM + 512 + 1024 <= 232448 && OFF_BAR_SPLIT + BAR_BYTES + 1024 <= 232448,
               "shared memory exceeds 227 KB");
 
 // 4-D tensor maps {inner dim, H, T, B} with boxes of 64 tokens (split mode only).
@@ -212,9 +215,10 @@ __device__ __forceinline__ uint4 pack8(const float* m8) {
 // warps 4-7 convert the Wm tiles and write o.  Every other CTA is a prep worker with two
 // independent 8-warp groups that compute chunks in chunk-major task order and write their
 // operand tiles into the ring.  The grid must be co-resident (cooperative launch).
-// UNT: a write strength w separate from beta (p.w set); a compile-time switch so that the
-// tied kernel carries none of its cost.
-template <int MODE, bool ROT, typename OT, bool UNT>
+// EXT: the kernel with the optional features (a write strength w separate from beta when
+// p.w is set; the fused L2 normalisation of q and k when p.qk_norm is set), switched on at
+// run time; the plain kernel carries none of their cost.
+template <int MODE, bool ROT, typename OT, bool EXT>
 __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdParams p, TcExtra x, SplitArgs sa,
                                                               const __grid_constant__ TmaMaps tm) {
     using namespace tc;
@@ -253,7 +257,8 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
     const __nv_bfloat16* __restrict__ v = static_cast<const __nv_bfloat16*>(p.v);
     OT* __restrict__ o = static_cast<OT*>(p.o);
     const int nchunks = (p.T + C - 1) / C;
-    constexpr bool untied = UNT;            // a write strength w separate from beta
+    const bool untied = EXT && p.w != nullptr;    // a write strength w separate from beta
+    const bool qkn = EXT && p.qk_norm != 0;       // fused L2 normalisation of q and k
     auto chunk_len = [&](int c) -> int { return min(C, p.T - c * C); };
     auto tokh = [&](int bhx, int c, int r) -> size_t {      // bhx: local head
         const int gx = p.head0 + bhx;
@@ -470,6 +475,27 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             cp_async_commit();
             }
 
+            // ---- fused L2 normalisation: inverse norms of this warp's 8 tokens' k and q ----
+            float2* nrm = reinterpret_cast<float2*>((MODE == 0) ? base + OFF_NRM : gb + G_NRM);
+            if (qkn) {
+#pragma unroll
+                for (int s_ = 0; s_ < 8; ++s_) {
+                    const uint2 kr = rk[s_], qr = rq[s_];
+                    const float k0 = __uint_as_float(kr.x << 16), k1 = __uint_as_float(kr.x & 0xFFFF0000u);
+                    const float k2 = __uint_as_float(kr.y << 16), k3 = __uint_as_float(kr.y & 0xFFFF0000u);
+                    const float q0 = __uint_as_float(qr.x << 16), q1 = __uint_as_float(qr.x & 0xFFFF0000u);
+                    const float q2 = __uint_as_float(qr.y << 16), q3 = __uint_as_float(qr.y & 0xFFFF0000u);
+                    float sk = k0 * k0 + k1 * k1 + k2 * k2 + k3 * k3;
+                    float sq = q0 * q0 + q1 * q1 + q2 * q2 + q3 * q3;
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) {      // the warp holds all 128 dims
+                        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                    }
+                    if (lane == 0) nrm[8 * sg + s_] = make_float2(rsqrtf(sk + 1e-6f), rsqrtf(sq + 1e-6f));
+                }
+            }
+
             // ---- pass 1: per-token decays and segment products ---------------------------
             // real:     al[s][d] = alpha of dim 4dg+d;
             // rotation: al[s][j] = alpha of pair 2dg+j, al[s][2+j] = cos, sn[s][j] = sin.
@@ -593,10 +619,15 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     }
                 }
                 auto emit = [&](int r, const float (&F)[4], const float (&G)[4], uint2 kraw, uint2 qraw) {
-                    const float kk[4] = {__uint_as_float(kraw.x << 16), __uint_as_float(kraw.x & 0xFFFF0000u),
-                                         __uint_as_float(kraw.y << 16), __uint_as_float(kraw.y & 0xFFFF0000u)};
-                    const float qv[4] = {__uint_as_float(qraw.x << 16), __uint_as_float(qraw.x & 0xFFFF0000u),
-                                         __uint_as_float(qraw.y << 16), __uint_as_float(qraw.y & 0xFFFF0000u)};
+                    float kk[4] = {__uint_as_float(kraw.x << 16), __uint_as_float(kraw.x & 0xFFFF0000u),
+                                   __uint_as_float(kraw.y << 16), __uint_as_float(kraw.y & 0xFFFF0000u)};
+                    float qv[4] = {__uint_as_float(qraw.x << 16), __uint_as_float(qraw.x & 0xFFFF0000u),
+                                   __uint_as_float(qraw.y << 16), __uint_as_float(qraw.y & 0xFFFF0000u)};
+                    if (qkn) {
+                        const float2 nn = nrm[r];
+#pragma unroll
+                        for (int d = 0; d < 4; ++d) { kk[d] *= nn.x; qv[d] *= nn.y; }
+                    }
                     float kt[4], qt[4], kh[4];
                     if (!ROT) {
 #pragma unroll

@@ -33,13 +33,14 @@ class FwdDesc(ctypes.Structure):
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("chunk", ctypes.c_int),
                 ("qkv_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
                 ("gate_mode", ctypes.c_int), ("rotation", ctypes.c_int),
-                ("scale", ctypes.c_float), ("algo", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("algo", ctypes.c_int), ("qk_l2norm", ctypes.c_int)]
 
 
 class DecDesc(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int), ("H", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int),
                 ("qkv_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
-                ("gate_mode", ctypes.c_int), ("rotation", ctypes.c_int), ("scale", ctypes.c_float)]
+                ("gate_mode", ctypes.c_int), ("rotation", ctypes.c_int), ("scale", ctypes.c_float),
+                ("qk_l2norm", ctypes.c_int)]
 
 
 class GdrError(RuntimeError):
@@ -130,9 +131,9 @@ def _need(t: torch.Tensor, name: str, dtype=None, device=None):
 
 
 def fwd_desc(B, H, T, dk, dv, qkv_dtype, out_dtype, gate_mode=GATE_NEG_SOFTPLUS, rotation=False,
-             scale=1.0, algo="auto", chunk=64) -> FwdDesc:
+             scale=1.0, algo="auto", chunk=64, qk_l2norm=False) -> FwdDesc:
     return FwdDesc(B, H, T, dk, dv, chunk, _dtype_code(qkv_dtype), _dtype_code(out_dtype),
-                   int(gate_mode), int(bool(rotation)), float(scale), ALGOS[algo])
+                   int(gate_mode), int(bool(rotation)), float(scale), ALGOS[algo], int(bool(qk_l2norm)))
 
 
 def resolved_algo(desc: FwdDesc) -> str:
@@ -154,7 +155,7 @@ def workspace_bytes(desc: FwdDesc) -> int:
 
 def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
               algo="auto", out_dtype=None, want_state=True, o=None, S_T=None, workspace=None,
-              stream=None, chunk=64, w=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              stream=None, chunk=64, w=None, qk_l2norm=False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunk-parallel forward.  Returns (o, S_T).
 
     beta is the erase strength; w [B,T,H] (fp32) a separate write strength, or None for
@@ -164,7 +165,8 @@ def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTP
     """
     if not q.is_cuda:
         return _chunk_fwd_host(q, k, v, g, beta, theta, S0, gate_mode=gate_mode, scale=scale,
-                               algo=algo, out_dtype=out_dtype, want_state=want_state, chunk=chunk, w=w)
+                               algo=algo, out_dtype=out_dtype, want_state=want_state, chunk=chunk, w=w,
+                               qk_l2norm=qk_l2norm)
     dev = q.device
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -198,7 +200,7 @@ def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTP
         S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
     if S_T is not None:
         _need(S_T, "S_T", torch.float32, dev)
-    desc = fwd_desc(B, H, T, dk, dv, q.dtype, out_dtype, gate_mode, rotation, scale, algo, chunk)
+    desc = fwd_desc(B, H, T, dk, dv, q.dtype, out_dtype, gate_mode, rotation, scale, algo, chunk, qk_l2norm)
     need = workspace_bytes(desc)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -225,7 +227,7 @@ def _chunk_fwd_host(q, k, v, g, beta, theta, S0, w=None, **kw):
 
 
 def decode_step(q, k, v, g, beta, S, theta=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
-                out_dtype=None, o=None, stream=None, w=None) -> torch.Tensor:
+                out_dtype=None, o=None, stream=None, w=None, qk_l2norm=False) -> torch.Tensor:
     """One decode step; S [N,H,dv,dk] (fp32) is updated in place.  Returns o [N,H,dv].
     beta erases; w [N,H] (fp32) is a separate write strength, or None for w = beta."""
     dev = S.device
@@ -246,7 +248,7 @@ def decode_step(q, k, v, g, beta, S, theta=None, *, gate_mode=GATE_NEG_SOFTPLUS,
     if o is None:
         o = torch.empty((N, H, dv), dtype=out_dtype, device=dev)
     desc = DecDesc(N, H, dk, dv, _dtype_code(q.dtype), _dtype_code(out_dtype), int(gate_mode),
-                   int(rotation), float(scale))
+                   int(rotation), float(scale), int(bool(qk_l2norm)))
     if w is not None:
         _need(w, "w", torch.float32, dev)
         if tuple(w.shape) != (N, H):

@@ -109,3 +109,11 @@ def test_untied_entry_points_check_the_write_strength(G):
     st = L.gdr_decode_step_untied(ctypes.byref(dd), get("q"), get("k"), get("v"), get("g"), get("beta"),
                                   ctypes.c_void_p(0x10004), None, get("S_T"), get("o"), None)
     assert st == G.GDR_ERR_INVALID_ARG
+
+
+def test_qk_l2norm_flag_is_checked(G):
+    d = _desc(G)
+    d.qk_l2norm = 2
+    assert _call_fwd(G, d, FAKE) == G.GDR_ERR_INVALID_ARG
+    d.qk_l2norm = 1
+    assert G.lib().gdr_chunk_fwd_workspace_bytes(ctypes.byref(d)) == 0     # SIMT shape here

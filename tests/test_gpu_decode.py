@@ -112,3 +112,25 @@ def test_decode_untied_parity(G, dk, rot):
         torch.cuda.synchronize()
         assert U.max_rel(U.o_to_f64(o), o_ref) <= U.TOL_O["bf16"]
     assert U.rel_l2(S.cpu().numpy(), S_ref) <= U.TOL_S
+
+
+@pytest.mark.parametrize("dk,rot", [(128, False), (32, True)])
+def test_decode_l2norm_prologue_parity(G, dk, rot):
+    """q and k stored with per-token norms far from 1, normalised in the kernel."""
+    import torch
+    d = I.make_decode(N=4, H=3, dk=dk, dv=dk, steps=2, dtype="f32", seed=95 + dk, rotation=rot, scale=0.7)
+    f = np.exp(I.normal(96 + dk, "qkscale", (2, 2, 4, 3, 1)) * 0.7).astype(np.float32)
+    S = U.to_torch(d.S, "cuda").clone()
+    S_ref = d.widened("S")
+    for s in range(2):
+        qs, ks = (d.q[s] * f[0, s]).astype(np.float32), (d.k[s] * f[1, s]).astype(np.float32)
+        t = {key: U.to_torch(getattr(d, key)[s], "cuda") for key in ("v", "g", "beta")}
+        th = None if d.theta is None else U.to_torch(d.theta[s], "cuda")
+        o = G.decode_step(U.to_torch(qs, "cuda"), U.to_torch(ks, "cuda"), t["v"], t["g"], t["beta"], S, th,
+                          gate_mode=d.gate_mode, scale=d.scale, qk_l2norm=True)
+        o_ref, S_ref = oracle.gdr_decode_step(qs.astype(np.float64), ks.astype(np.float64), d.widened("v", s),
+                                              d.widened("g", s), d.widened("beta", s), S_ref,
+                                              d.widened("theta", s), d.gate_mode, d.scale, qk_l2norm=True)
+        torch.cuda.synchronize()
+        assert U.max_rel(U.o_to_f64(o), o_ref) <= U.TOL_O["f32"]
+    assert U.rel_l2(S.cpu().numpy(), S_ref) <= 1e-4

@@ -289,3 +289,40 @@ def test_waves_split_remainder_parity(G, B, rotation):
     assert G.query_device_status() == G.GDR_OK
     o_ref, S_ref = U.oracle_fwd(p)
     U.assert_fwd_parity(p, o, S, o_ref, S_ref)
+
+
+L2NORM_CASES = [
+    # (algo, dtype, B, H, T, rotation)
+    ("simt", "f32", 1, 2, 150, False),
+    ("tcgen05", "bf16", 2, 2, 257, True),
+    ("tcgen05_split", "bf16", 2, 3, 333, False),
+]
+
+
+@pytest.mark.parametrize("case", L2NORM_CASES, ids=lambda c: "{}_{}_B{}H{}T{}{}".format(
+    c[0], c[1], c[2], c[3], c[4], "_rot" if c[5] else ""))
+def test_l2norm_prologue_parity(G, case):
+    """q and k stored un-normalised (per-token norms in [0.25, 4]), normalised in the kernel:
+    against the oracle with its own fp64 normalisation of the same stored values."""
+    import torch
+    algo, dtype, B, H, T, rot = case
+    dk = 128 if algo != "simt" else 64
+    p = I.make_fwd(B, T, H, dk, dk, dtype="f32", seed=900 + T, rotation=rot, s0_std=0.2, scale=0.8)
+    f = np.exp(I.normal(901 + T, "qkscale", (2, B, T, H, 1)) * 0.5).astype(np.float32)
+    q = (p.q * f[0]).astype(np.float32)
+    k = (p.k * f[1]).astype(np.float32)
+    if dtype == "bf16":
+        q, k, v = I.to_bf16_bits(q), I.to_bf16_bits(k), I.to_bf16_bits(p.v)
+        p = I.FwdInputs(p.B, p.T, p.H, p.dk, p.dv, p.chunk, "bf16", p.gate_mode, p.rotation, q, k, v,
+                        p.g, p.beta, p.theta, p.S0, p.scale)
+    else:
+        p.q, p.k = q, k
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "g", "beta", "theta", "S0")}
+    o, S = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["theta"], t["S0"], gate_mode=p.gate_mode,
+                       scale=p.scale, algo=algo, qk_l2norm=True)
+    torch.cuda.synchronize()
+    assert G.query_device_status() == G.GDR_OK
+    o_ref, S_ref = oracle.gdr_fwd(p.widened("q"), p.widened("k"), p.widened("v"), p.widened("g"),
+                                  p.widened("beta"), p.widened("theta"), p.widened("S0"),
+                                  gate_mode=p.gate_mode, scale=p.scale, qk_l2norm=True)
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref)

@@ -429,3 +429,42 @@ def test_untied_decode_steps_equal_forward():
                                         oracle.GATE_NEG_SOFTPLUS, w=w[:, t])
         assert _rel(o_t, o_f[:, t]) < 1e-12
     assert _rel(S, S_f) < 1e-12
+
+
+# ---- fused L2 normalisation of q and k (NEXT-4 prologue) ---------------------------------
+
+def test_l2norm_prologue_makes_the_layer_blind_to_key_and_query_scale():
+    """With the prologue on, rescaling each token's q and k by arbitrary positive factors
+    changes nothing (up to the 1e-6 epsilon); with it off, the same rescaling changes the
+    result a lot."""
+    rng = np.random.default_rng(81)
+    q, k, v, a, beta, theta, S0 = _rand_problem(rng, 1, 23, 2, 8, 5, rotation=True)
+    fq = np.exp(rng.uniform(0, 2, q.shape[:-1] + (1,)))       # norms >= 1: epsilon below 1e-6
+    fk = np.exp(rng.uniform(0, 2, k.shape[:-1] + (1,)))
+    o1, S1 = oracle.gdr_fwd(q, k, v, a, beta, theta, S0, oracle.GATE_NEG_SOFTPLUS, qk_l2norm=True)
+    o2, S2 = oracle.gdr_fwd(q * fq, k * fk, v, a, beta, theta, S0, oracle.GATE_NEG_SOFTPLUS, qk_l2norm=True)
+    assert _rel(o2, o1) < 1e-5 and _rel(S2, S1) < 1e-5
+    o3, _ = oracle.gdr_fwd(q * fq, k * fk, v, a, beta, theta, S0, oracle.GATE_NEG_SOFTPLUS)
+    assert _rel(o3, o1) > 1e-2
+
+
+def test_l2norm_prologue_on_unit_inputs_changes_only_by_epsilon():
+    rng = np.random.default_rng(82)
+    q, k, v, a, beta, theta, S0 = _rand_problem(rng, 2, 15, 2, 8, 6)       # unit q, k
+    o1, S1 = oracle.gdr_fwd(q, k, v, a, beta, theta, S0, oracle.GATE_NEG_SOFTPLUS)
+    o2, S2 = oracle.gdr_fwd(q, k, v, a, beta, theta, S0, oracle.GATE_NEG_SOFTPLUS, qk_l2norm=True)
+    assert _rel(o2, o1) < 1e-5 and _rel(S2, S1) < 1e-5
+
+
+def test_l2norm_prologue_keeps_zero_vectors_zero_and_decode_agrees():
+    rng = np.random.default_rng(83)
+    q, k, v, a, beta, theta, S0 = _rand_problem(rng, 1, 7, 3, 8, 4, unit_k=False)
+    q[0, 3] = 0.0                                   # a zero query reads nothing
+    o, S_f = oracle.gdr_fwd(q, k, v, a, beta, None, S0, oracle.GATE_NEG_SOFTPLUS, qk_l2norm=True)
+    assert np.all(o[0, 3] == 0.0)
+    S = S0.copy()
+    for t in range(7):
+        o_t, S = oracle.gdr_decode_step(q[:, t], k[:, t], v[:, t], a[:, t], beta[:, t], S, None,
+                                        oracle.GATE_NEG_SOFTPLUS, qk_l2norm=True)
+        assert _rel(o_t + 1e-300, o[:, t] + 1e-300) < 1e-12 or np.all(o[:, t] == o_t)
+    assert _rel(S, S_f) < 1e-12
