@@ -268,9 +268,6 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
     // Chain-side buffers of chunk c: fused mode reads the prep group's double buffers, split
     // mode the slot copied from the ring.
     auto slot_base = [&](int c) -> uint32_t { return (uint32_t)(c & 1) * SLOT_STRIDE; };
-    auto chain_vec = [&](int c) -> const float* {
-        return MODE == 0 ? vecs(c) : reinterpret_cast<const float*>(base + slot_base(c) + SL_VEC);
-    };
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -1250,7 +1247,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         const int row = tid - NPREP;          // TMEM lane = value row of S (quad = warp & 3)
         uint32_t mma_phase = 0;
         const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_NEG = idesc_bf16(128, 64, 0, 1, 1);
-        const uint32_t ID_KM128 = idesc_bf16(128, 128, 0, 1, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
+        const uint32_t ID_KM128 = idesc_bf16(128, 128, 0, 1, 0);
         auto cbar = [&]() { named_bar(2, CHAIN_THREADS); };
         auto mma_wait = [&]() -> bool {      // one thread waits, the others at the barrier
             if (row == 0 && !mbar_wait_bounded(bar_cmma, mma_phase, x.wait_limit_ns)) atomicExch(abort_c, 1);
@@ -1297,27 +1294,6 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         auto o_epilogue = [&](int c) {
             const int Lc = chunk_len(c);
             const uint32_t col = COL_O + (c & 1) * 64;
-            if (MODE == 1) {
-                // stage o as [token][value] in shared memory, then one thread bulk-stores rows
-                if (row == 0) bulk_wait_read_all();            // the previous chunk's stores have read it
-                cbar();
-                OT* stg = reinterpret_cast<OT*>(base + OFF_OSTG);
-#pragma unroll 1
-                for (int g = 0; g < 2; ++g) {
-                    float vals[32];
-                    tmem_ld32(tq + col + g * 32, vals);
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) st_from_f32(stg + (g * 32 + u) * D + row, vals[u]);
-                }
-                fence_proxy_async_smem();
-                cbar();
-                if (row == 0) {
-                    tma_store_4d(&tm.o, 0, gbh % p.H, c * C, gbh / p.H, sb + OFF_OSTG);   // rows past T clipped
-                    bulk_commit();
-                }
-                (void)Lc;
-                return;
-            }
             const int j8 = lane & 7, grp = lane >> 3;
             OT* obase = o + tok(c, 0) * D + quad * 32 + grp * 8;
             const size_t tstride = (size_t)p.H * D;
@@ -1346,9 +1322,9 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         };
 
         // Initial state, prescaled by the first chunk's reference decay.
-        bool alive = bounded(MODE == 0 ? bar_rho + 0 : bar_full + 0, 0);
+        bool alive = bounded(bar_rho + 0, 0);
         if (alive) {
-            const float* rho_ref0 = chain_vec(0) + 64;
+            const float* rho_ref0 = vecs(0) + 64;
 #pragma unroll 1
             for (int g = 0; g < 8; ++g) {
                 const int col0 = g * 16;
@@ -1377,19 +1353,9 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             tc_fence_after();
             // ---- E^T += -Stil Wm^T ;  O^T = Stil Qtil^T --------------------------------
             if (row == 0) {
-                const uint32_t sl = sb + slot_base(c);
-                if (MODE == 1) {
-                    // U^T = V^T Tb^T from the slot (the fused prep group does this itself)
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16_ss(tbase + COL_E + bufi * 64, sdesc_sw128(sl + SL_V + ks * 2048, 8192, 1024),
-                                    sdesc_sw128(sl + SL_TB + ks * 32, 16, 1024), ID_MK, ks > 0);
-                }
-                const uint64_t dW = MODE == 0 ? sdesc_sw128(sb + OFF_W + bufi * 16384, 8192, 1024)
-                                              : sdesc_sw128(sl + SL_W, 8192, 1024);
-                const uint64_t dQ = MODE == 0 ? sdesc_sw128(sb + OFF_KQ + bufi * 32768 + 8192, 16, 1024)
-                                              : sdesc_sw128(sl + SL_Q, 16, 1024);
-                const uint32_t qkb = MODE == 0 ? 16384u : 8192u;   // K-block stride of the Qtil tile
+                const uint64_t dW = sdesc_sw128(sb + OFF_W + bufi * 16384, 8192, 1024);
+                const uint64_t dQ = sdesc_sw128(sb + OFF_KQ + bufi * 32768 + 8192, 16, 1024);
+                const uint32_t qkb = 16384u;                         // K-block stride of the Qtil tile
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t a_t = tbase + COL_SB + ks * 8;
@@ -1423,11 +1389,8 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             tc_fence_after();
             // ---- O^T += E^T Pm^T ;  S_acc += E^T Khat ---------------------------------------
             if (row == 0) {
-                const uint32_t sl = sb + slot_base(c);
-                const uint64_t dP = MODE == 0 ? sdesc_sw128(sb + OFF_PM + bufi * 8192, 16, 1024)
-                                              : sdesc_sw128(sl + SL_PM, 16, 1024);
-                const uint64_t dH = MODE == 0 ? sdesc_sw128(sb + OFF_KH + bufi * 16384, 8192, 1024)
-                                              : sdesc_sw128(sl + SL_KH, 8192, 1024);
+                const uint64_t dP = sdesc_sw128(sb + OFF_PM + bufi * 8192, 16, 1024);
+                const uint64_t dH = sdesc_sw128(sb + OFF_KH + bufi * 16384, 8192, 1024);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint32_t a_t = tbase + COL_E + bufi * 64 + ks * 8;
@@ -1439,10 +1402,10 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             if (!mma_wait()) break;
 
             // ---- S <- S_acc (P_m^{-1} P_C), then prescale by the next reference ----------
-            if (!last && !bounded((MODE == 0 ? bar_rho : bar_full) + ((c + 1) & 1), ((c + 1) >> 1) & 1)) break;
+            if (!last && !bounded(bar_rho + ((c + 1) & 1), ((c + 1) >> 1) & 1)) break;
             {
-                const float* rho_C = chain_vec(c) + 64 + 256;
-                const float* rho_nx = chain_vec(c + 1) + 64;
+                const float* rho_C = vecs(c) + 64 + 256;
+                const float* rho_nx = vecs(c + 1) + 64;
 #pragma unroll 1
                 for (int g = 0; g < 4; ++g) {
                     const int col0 = g * 32;
@@ -1474,7 +1437,6 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             mbar_arrive(bar_empty + bufi);
             if (last) o_epilogue(c);
         }
-        if (MODE == 1 && row == 0) bulk_wait_all();     // o stores complete before the CTA exits
     }
 
     if (MODE == 1 && nchunks > 0 && chain_cta && warp == 0) {

@@ -145,7 +145,7 @@ def test_host_buffers_round_trip(G):
 FULL = ["b4_h16_t4096_d128", "b16_h12_t4096_d128_slow_s0", "b2_h16_t8192_d128_rot"]
 
 
-@pytest.mark.parametrize("algo", ALGOS_ALL)
+@pytest.mark.parametrize("algo", ALGOS_ALL + ["auto"])
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_configs_sampled(G, algo, name):
     """Full-size workloads in the benchmark's launch configuration; the oracle
@@ -326,3 +326,29 @@ def test_l2norm_prologue_parity(G, case):
                                   p.widened("beta"), p.widened("theta"), p.widened("S0"),
                                   gate_mode=p.gate_mode, scale=p.scale, qk_l2norm=True)
     U.assert_fwd_parity(p, o, S, o_ref, S_ref)
+
+
+def test_full_size_with_both_optional_features_sampled(G):
+    """The bench workload with a separate write strength and the fused L2 normalisation
+    together (q and k stored at norms far from 1), AUTO's launch configuration, sampled
+    whole heads against the oracle."""
+    import torch
+    p = I.make_config("b4_h16_t4096_d128")
+    w = I.make_write_strength(77, (p.B, p.T, p.H))
+    f = np.exp(I.normal(78, "qkscale", (2, p.B, p.T, p.H, 1)) * 0.5).astype(np.float32)
+    q32 = U.to_torch(p.q, "cuda").float() * torch.from_numpy(f[0]).cuda()
+    k32 = U.to_torch(p.k, "cuda").float() * torch.from_numpy(f[1]).cuda()
+    q16, k16 = q32.to(torch.bfloat16), k32.to(torch.bfloat16)
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("v", "g", "beta", "theta", "S0")}
+    o, S = G.chunk_fwd(q16, k16, t["v"], t["g"], t["beta"], t["theta"], t["S0"], gate_mode=p.gate_mode,
+                       scale=p.scale, w=torch.from_numpy(w).cuda(), qk_l2norm=True)
+    torch.cuda.synchronize()
+    assert G.query_device_status() == G.GDR_OK
+    qh, kh = q16.float().cpu().numpy(), k16.float().cpu().numpy()
+    for (b, h) in [(0, 0), (1, 7), (p.B - 1, p.H - 1)]:
+        ps = p.head_slice(b, h)
+        o_ref, S_ref = oracle.gdr_fwd(qh[b:b + 1, :, h:h + 1], kh[b:b + 1, :, h:h + 1], ps.widened("v"),
+                                      ps.widened("g"), ps.widened("beta"), ps.widened("theta"), ps.widened("S0"),
+                                      gate_mode=p.gate_mode, scale=p.scale, w=w[b:b + 1, :, h:h + 1].astype(np.float64),
+                                      qk_l2norm=True)
+        U.assert_fwd_parity(ps, o[b:b + 1, :, h:h + 1], S[b:b + 1, h:h + 1], o_ref, S_ref)
