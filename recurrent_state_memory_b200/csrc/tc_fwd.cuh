@@ -265,8 +265,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         return ((size_t)(gx / p.H) * p.T + (c * C + r)) * p.H + (gx % p.H);
     };
     auto tok = [&](int c, int r) -> size_t { return tokh(bh, c, r); };
-    // Chain-side buffers of chunk c: fused mode reads the prep group's double buffers, split
-    // mode the slot copied from the ring.
+    // Split chain CTAs: the shared-memory buffer that holds chunk c's ring slot.
     auto slot_base = [&](int c) -> uint32_t { return (uint32_t)(c & 1) * SLOT_STRIDE; };
 
     if (warp == 0) {
