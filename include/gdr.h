@@ -126,8 +126,8 @@ GDR_API const char* gdr_last_error_detail(void);
 
 /* Bytes of device workspace gdr_chunk_fwd needs for this descriptor (0 = none;
  * the workspace argument may then be NULL).  Returns 0 for an invalid desc.  The split
- * tensor-core kernel needs B*H*8 ring slots of 67,840 bytes plus 36 bytes of flags per
- * head; it resets the flags itself (on the call's stream) and the buffer may be reused
+ * tensor-core kernel needs B*H*8 ring slots of 76,288 bytes plus 36 bytes of flags per
+ * head and one 4-byte task counter; it resets the flags itself (on the call's stream) and the buffer may be reused
  * by later calls on the same stream.  Uses the current device's SM count when
  * desc->algo is GDR_ALGO_AUTO. */
 GDR_API size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc);
@@ -219,8 +219,8 @@ GDR_API gdr_status gdr_query_device_status(gdr_stream_t stream);
  *
  * It runs the split tensor-core kernel (same arithmetic and results as
  * gdr_chunk_fwd with GDR_ALGO_TCGEN05_SPLIT) with the kernel's hand-off ring in a scratch
- * array compiled into the library: GDR_NOALLOC_MAX_HEADS * 8 slots of 67,840 bytes plus
- * flags (about 16.6 MiB), which every GPU that loads the library holds until the process
+ * array compiled into the library: GDR_NOALLOC_MAX_HEADS * 8 slots of 76,288 bytes plus
+ * flags (about 18.6 MiB), which every GPU that loads the library holds until the process
  * exits.
  *   - desc->algo must be GDR_ALGO_AUTO or GDR_ALGO_TCGEN05_SPLIT; q, k, v must be bf16 with
  *     dk = dv = 128; B*H must not exceed GDR_NOALLOC_MAX_HEADS, else GDR_ERR_UNSUPPORTED with

@@ -111,7 +111,7 @@ static gdr_algo resolve_algo(const gdr_fwd_desc* d) {
 }
 
 static size_t split_workspace_heads(size_t nh) {
-    return nh * tcf::RING * tcf::SLOT_BYTES + (nh * tcf::RING + nh) * sizeof(unsigned int);
+    return nh * tcf::RING * tcf::SLOT_BYTES + tcf::split_flag_words(nh) * sizeof(unsigned int);
 }
 static size_t split_workspace_bytes(const gdr_fwd_desc* d) { return split_workspace_heads((size_t)d->B * d->H); }
 
@@ -121,7 +121,7 @@ static size_t split_workspace_bytes(const gdr_fwd_desc* d) { return split_worksp
 constexpr int NOALLOC_MAX_HEADS = GDR_NOALLOC_MAX_HEADS;
 constexpr size_t NOALLOC_BYTES =
     (size_t)NOALLOC_MAX_HEADS * tcf::RING * tcf::SLOT_BYTES +
-    ((size_t)NOALLOC_MAX_HEADS * tcf::RING + NOALLOC_MAX_HEADS) * sizeof(unsigned int);
+    tcf::split_flag_words(NOALLOC_MAX_HEADS) * sizeof(unsigned int);
 static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_BYTES];
 
 // In host code g_noalloc_scratch names a host-side stand-in, not device memory; the device
@@ -261,7 +261,12 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
     sa.ring = static_cast<uint8_t*>(ws);
     sa.ready = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + nring);
     sa.consumed = sa.ready + (size_t)nh * tcf::RING;
-    e = cudaMemsetAsync(sa.ready, 0, ((size_t)nh * tcf::RING + nh) * sizeof(unsigned int), st);
+    sa.next_task = sa.consumed + nh;
+    // Worker order: from the counter while the worker groups fill at most half the ring's
+    // slots (the workers are then the bound and the counter evens out their load); at a
+    // fixed stride otherwise (measured faster there: it paces each group to the chains).
+    sa.dynamic = (2 * (grid - nh) <= nh * tcf::RING / 2) ? 1 : 0;
+    e = cudaMemsetAsync(sa.ready, 0, tcf::split_flag_words(nh) * sizeof(unsigned int), st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split flags)");
     void* args[] = {const_cast<FwdParams*>(&p), &x, &sa, &tm};
     e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(nt), args, smem, st);

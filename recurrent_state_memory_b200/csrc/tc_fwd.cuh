@@ -138,7 +138,14 @@ struct SplitArgs {
     uint8_t* ring;            // [B*H][RING][SLOT_BYTES]
     unsigned int* ready;      // [B*H][RING]: index + 1 of the chunk a slot holds
     unsigned int* consumed;   // [B*H]: chunks the chain has copied out of the ring
+    unsigned int* next_task;  // [1]: the next worker task to hand out (dynamic order)
+    int dynamic;              // 1: tasks from the counter; 0: group i takes tasks i, i + G, ...
+                              //    (G worker groups)
 };
+
+// Flag words of the split workspace after the ring: ready, consumed, next_task (zeroed
+// before every launch).
+__host__ __device__ constexpr size_t split_flag_words(size_t nh) { return nh * RING + nh + 1; }
 
 // Device status bits (gdr_query_device_status).
 constexpr unsigned STATUS_TIMEOUT = 1u;
@@ -300,9 +307,12 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
 
     if (nchunks > 0 && (MODE == 0 ? tid < NPREP : (!chain_cta && tid < 2 * NPREP))) {
         // =========================== prep group ===================================
-        // Tasks: fused mode, chunk it of this CTA's head; split mode, task wk + it * W in
-        // chunk-major order (chunk = task / NH, head = task % NH), where the workers' groups
-        // count as 2 (gridDim.x - NH) independent workers.
+        // Tasks: fused mode, the chunks of this CTA's head in order; split mode, tasks in
+        // chunk-major order (chunk = task / NH, head = task % NH), either handed out one at a
+        // time by a global counter (a group that ran fast takes the next task) or at a fixed
+        // stride of the number of groups (which paces each group to the chains once the
+        // stride nears the ring's depth in tasks).  A group claims its next task while it
+        // works on the current one.
         const int grp = (MODE == 1) ? (int)threadIdx.x / NPREP : 0;
         const int tid = (int)threadIdx.x - grp * NPREP;      // thread within the group
         const int warp = tid >> 5;
@@ -315,11 +325,8 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         float* Af = reinterpret_cast<float*>(MODE == 0 ? base + OFF_AF : gb + G_AF);
         float* Tf = reinterpret_cast<float*>(MODE == 0 ? base + OFF_TF : gb + G_TF);
         float* QT = reinterpret_cast<float*>(MODE == 0 ? base + OFF_QT : gb + G_QT);
-        const int W = (MODE == 0) ? 1 : 2 * ((int)gridDim.x - NH);
-        const int wk = (MODE == 0) ? 0 : 2 * ((int)blockIdx.x - NH) + grp;
-        const int ntasks = (MODE == 0) ? nchunks : (NH * nchunks - wk + W - 1) / W;
-        auto task_bh = [&](int it) -> int { return MODE == 0 ? bh : (wk + it * W) % NH; };
-        auto task_c = [&](int it) -> int { return MODE == 0 ? it : (wk + it * W) / NH; };
+        const int total = (MODE == 0) ? nchunks : NH * nchunks;
+        int* s_task = reinterpret_cast<int*>(bar_base + 128) + grp;   // split: the group's next task
         // Decay passes: each thread owns 4 key dims (two key pairs) of one 8-token segment;
         // warp w handles tokens 8w .. 8w+7.  The reference token 31 is the last token of
         // segment 3, so segments 0-3 run backward from it and segments 4-7 forward.
@@ -390,11 +397,11 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             st_release_gpu(sa.ready + (size_t)pub_bh * RING + pub_c % RING, (unsigned)(pub_c + 1));
             pub_c = -1;
         };
-        auto stage_part = [&](int itx, int part) {
-            const int c2 = task_c(itx), b2 = p.head0 + task_bh(itx);     // global head
+        auto stage_part = [&](int tk, int part) {
+            const int c2 = tk / NH, b2 = p.head0 + tk % NH;     // global head
             const int bb = b2 / p.H, hh = b2 % p.H;
             if (part == 0) {
-                staged = itx + 1;
+                ++staged;
                 mbar_arrive_expect_tx(g_stage, 65536u);
                 tma_load_4d(gsb + G_KH, &tm.q, 0, hh, c2 * C, bb, g_stage);
             } else if (part == 1) {
@@ -406,14 +413,30 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
         };
         const uint32_t ID_KK = idesc_bf16(128, 64, 0, 0, 0), ID_MK = idesc_bf16(128, 64, 1, 0, 0);
 
-        if (MODE == 0 && ntasks > 0) prefetch(task_bh(0), task_c(0));
-        if (MODE == 1 && tid == 0 && ntasks > 0) {
-            stage_part(0, 0);
-            stage_part(0, 1);
-            stage_part(0, 2);
+        int task = 0, nxt = total;      // split: nxt, the claimed next task (thread 0)
+        int fixed_next = (MODE == 0) ? 0 : 2 * ((int)blockIdx.x - NH) + grp;   // static order
+        auto claim = [&]() -> int {
+            if (sa.dynamic) return (int)atomicAdd(sa.next_task, 1u);
+            const int t = fixed_next;
+            fixed_next += 2 * ((int)gridDim.x - NH);
+            return min(t, total);
+        };
+        if (MODE == 0 && total > 0) prefetch(bh, 0);
+        if (MODE == 1) {
+            if (tid == 0) {
+                nxt = claim();
+                *s_task = nxt;
+                if (nxt < total) {
+                    stage_part(nxt, 0);
+                    stage_part(nxt, 1);
+                    stage_part(nxt, 2);
+                }
+            }
+            named_bar(gbar, NPREP);
+            task = *s_task;
         }
-        for (int it = 0; it < ntasks; ++it) {
-            const int c = task_c(it), bhx = task_bh(it);
+        for (int it = 0; task < total; ++it) {
+            const int c = (MODE == 0) ? task : task / NH, bhx = (MODE == 0) ? bh : task % NH;
             const int Lc = chunk_len(c);
             const int bufi = (MODE == 0) ? (it & 1) : 0;      // split workers: single tile buffers
             float* vec = (MODE == 0) ? vecs(bufi) : reinterpret_cast<float*>(gb + G_VEC);
@@ -744,7 +767,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 }
             }
             if (MODE == 0) mbar_arrive(bar_rho + bufi);
-            if (MODE == 0 && it + 1 < ntasks) prefetch(task_bh(it + 1), task_c(it + 1));
+            if (MODE == 0 && task + 1 < total) prefetch(bh, task + 1);
 
             // ---- MMA1: [Ktil ; Qtil] Khat^T -> TMEM ------------------------------------
             tc_fence_after();
@@ -758,9 +781,14 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                 skip_commit = false;
             }
             if (!mma_wait()) break;
-            if (MODE == 1 && tid == 0 && it + 1 < ntasks) {     // MMA1 has read the operand tiles
-                stage_part(it + 1, 0);
-                stage_part(it + 1, 1);
+            if (MODE == 1 && tid == 0) {     // MMA1 has read the operand tiles
+                // claim the next task; the group reads it after this task's last barrier
+                nxt = claim();
+                *s_task = nxt;
+                if (nxt < total) {
+                    stage_part(nxt, 0);
+                    stage_part(nxt, 1);
+                }
             }
 
             // ---- solve: Tm = (I + A)^{-1}; Pm masked -> bf16 ---------------------------
@@ -927,7 +955,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     if (untied)
                         reinterpret_cast<uint4*>(ring + SL_TW)[tid + e * NPREP] = reinterpret_cast<const uint4*>(TW)[tid + e * NPREP];
                 }
-                if (tid == 0 && it + 1 < ntasks) stage_part(it + 1, 2);          // A and Tm done
+                if (tid == 0 && nxt < total) stage_part(nxt, 2);          // A and Tm done
             }
 
             if (MODE == 0) {
@@ -959,6 +987,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             }
             if (MODE == 0) mbar_arrive(bar_full + bufi);
             if (MODE == 1) { pub_c = c; pub_bh = bhx; }
+            task = (MODE == 0) ? task + 1 : *s_task;
         }
         if (MODE == 1 && tid == 32 && pub_c >= 0) publish_slot();
         if (bad) atomicExch(range_flag, 1);

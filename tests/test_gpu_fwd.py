@@ -214,17 +214,35 @@ def test_auto_picks_tensor_cores_for_bf16_d128(G):
         expect = "tcgen05_split" if 2 * B * H <= sms else "tcgen05"   # chains + prep workers
         assert G.resolved_algo(d) == expect
         if expect == "tcgen05_split":
-            assert G.workspace_bytes(d) >= B * H * 8 * 67840
+            assert G.workspace_bytes(d) >= B * H * 8 * 76288
     d = G.fwd_desc(16, 12, 4096, 128, 128, torch.bfloat16, torch.bfloat16)
     rem = (16 * 12) % sms if 16 * 12 > sms else 0
     expect = "tcgen05_waves" if 0 < rem and 2 * rem <= sms else "tcgen05"   # many heads
     assert G.resolved_algo(d) == expect
     if expect == "tcgen05_waves":
-        assert G.workspace_bytes(d) >= rem * 8 * 67840
+        assert G.workspace_bytes(d) >= rem * 8 * 76288
     d = G.fwd_desc(1, 1, 64, 64, 64, torch.bfloat16, torch.bfloat16)
     assert G.resolved_algo(d) == "simt"
     d = G.fwd_desc(1, 1, 64, 128, 128, torch.float32, torch.float32)
     assert G.resolved_algo(d) == "simt"
+
+
+@pytest.mark.parametrize("rotation", [False, True])
+def test_split_dynamic_task_order_parity(G, rotation):
+    """With 52 heads the split kernel's worker groups (2 per non-chain SM) fill at most half
+    of the ring's slots (8 per head), so the workers take their tasks from the global counter
+    instead of a fixed stride; six chunks with a ragged tail, against the oracle."""
+    import torch
+    B, H, T = 4, 13, 330
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if 2 * B * H > sms:
+        pytest.skip("needs 2*B*H <= SM count")
+    assert 2 * (sms - B * H) <= B * H * 8 // 2          # the counter order applies
+    p = I.make_fwd(B, T, H, 128, 128, dtype="bf16", seed=77 + int(rotation), s0_std=0.2, rotation=rotation)
+    o, S = U.run_gpu_fwd(p, "tcgen05_split")
+    assert G.query_device_status() == G.GDR_OK
+    o_ref, S_ref = U.oracle_fwd(p)
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref)
 
 
 @pytest.mark.parametrize("rotation", [False, True])
