@@ -285,61 +285,43 @@ def run_ours(args):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
 
     # ---- separate erase / write strengths (CARVE): the same workload with a write strength w ----
-    untied = None
+    def time_variant(step, v_bytes):
+        """Time one variant of the forward on the same workload (CUDA events, max over ranks)."""
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        n_v = max(3, min(args.steps, 10))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_v):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        v_ms = max_over_ranks(a.elapsed_time(b), dev)
+        v_tok = sum_over_ranks(float(tokens * n_v), dev)
+        v_gbs = v_bytes / (a.elapsed_time(b) / n_v * 1e-3) / 1e9
+        return {"value": round(v_tok / (v_ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s",
+                "ms_per_step": round(v_ms / n_v, 4), "steps": n_v, "kernel": kernel_name,
+                "roofline": {"bound": "hbm", "achieved": round(v_gbs, 1), "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(v_gbs / peaks["hbm_gbs"], 4),
+                             "algorithmic_bytes_per_launch": int(v_bytes)}}
+
+    def fwd_variant(**kw):
+        return lambda: gdr.chunk_fwd(dv_t["q"], dv_t["k"], dv_t["v"], dv_t["g"], dv_t["beta"], dv_t["theta"],
+                                     dv_t["S0"], gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o,
+                                     S_T=S_T, stream=stream, workspace=wsp, **kw)
+
+    untied = l2norm = cmean = None
     if not args.no_untied:
+        # ---- separate erase / write strengths (CARVE): the same workload with a write strength w ----
         w_dev = torch.from_numpy(I.make_write_strength(rank_seed(cfg["seed"], rank) + 17, (p.B, p.T, p.H))).to(dev)
-
-        def ustep():
-            gdr.chunk_fwd(dv_t["q"], dv_t["k"], dv_t["v"], dv_t["g"], dv_t["beta"], dv_t["theta"], dv_t["S0"],
-                          gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o, S_T=S_T, stream=stream,
-                          workspace=wsp, w=w_dev)
-
-        for _ in range(3):
-            ustep()
-        torch.cuda.synchronize()
-        n_u = max(3, min(args.steps, 10))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(n_u):
-            ustep()
-        b.record(stream)
-        torch.cuda.synchronize()
-        u_ms = max_over_ranks(a.elapsed_time(b), dev)
-        u_tok = sum_over_ranks(float(tokens * n_u), dev)
-        u_bytes = algo_bytes + p.B * p.T * p.H * 4            # plus w
-        u_gbs = u_bytes / (a.elapsed_time(b) / n_u * 1e-3) / 1e9
-        untied = {"value": round(u_tok / (u_ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s",
-                  "ms_per_step": round(u_ms / n_u, 4), "steps": n_u, "kernel": kernel_name,
-                  "roofline": {"bound": "hbm", "achieved": round(u_gbs, 1), "peak": peaks["hbm_gbs"],
-                               "unit": "GB/s", "frac": round(u_gbs / peaks["hbm_gbs"], 4),
-                               "algorithmic_bytes_per_launch": int(u_bytes)}}
-
-    # ---- fused L2 normalisation of q and k: the same workload with the prologue on ----
-    l2norm = None
-    if not args.no_untied:
-        def nstep():
-            gdr.chunk_fwd(dv_t["q"], dv_t["k"], dv_t["v"], dv_t["g"], dv_t["beta"], dv_t["theta"], dv_t["S0"],
-                          gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o, S_T=S_T, stream=stream,
-                          workspace=wsp, qk_l2norm=True)
-
-        for _ in range(3):
-            nstep()
-        torch.cuda.synchronize()
-        n_n = max(3, min(args.steps, 10))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(n_n):
-            nstep()
-        b.record(stream)
-        torch.cuda.synchronize()
-        n_ms = max_over_ranks(a.elapsed_time(b), dev)
-        n_tok = sum_over_ranks(float(tokens * n_n), dev)
-        n_gbs = algo_bytes / (a.elapsed_time(b) / n_n * 1e-3) / 1e9
-        l2norm = {"value": round(n_tok / (n_ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s",
-                  "ms_per_step": round(n_ms / n_n, 4), "steps": n_n, "kernel": kernel_name,
-                  "roofline": {"bound": "hbm", "achieved": round(n_gbs, 1), "peak": peaks["hbm_gbs"],
-                               "unit": "GB/s", "frac": round(n_gbs / peaks["hbm_gbs"], 4),
-                               "algorithmic_bytes_per_launch": int(algo_bytes)}}
+        untied = time_variant(fwd_variant(w=w_dev), algo_bytes + p.B * p.T * p.H * 4)     # plus w
+        # ---- fused L2 normalisation of q and k: the same workload with the prologue on ----
+        l2norm = time_variant(fwd_variant(qk_l2norm=True), algo_bytes)
+        # ---- chunk means of o (the content signal of CARVE's content-aware erase) ----
+        nc = (p.T + p.chunk - 1) // p.chunk
+        m_dev = torch.empty((p.B, nc, p.H, p.dv), dtype=torch.float32, device=dev)
+        cmean = time_variant(fwd_variant(chunk_mean=m_dev), algo_bytes + m_dev.numel() * 4)   # plus the means
 
     # ---- decode: 256 sequences x 16 heads, fp32 state, one launch per step ----
     decode = None
@@ -408,6 +390,7 @@ def run_ours(args):
         "decode": decode,
         "untied": untied,
         "qk_l2norm": l2norm,
+        "chunk_mean": cmean,
         "cpu_baseline": cpu,
         "clocks": clk.summary(),
     }
@@ -493,8 +476,8 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--no-untied", action="store_true", help="skip the separate-write-strength and "
-                    "fused-L2-norm measurements")
+    ap.add_argument("--no-untied", action="store_true", help="skip the separate-write-strength, "
+                    "fused-L2-norm and chunk-mean measurements")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

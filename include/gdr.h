@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define GDR_ABI_VERSION 2
+#define GDR_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define GDR_API __attribute__((visibility("default")))
@@ -184,7 +184,8 @@ GDR_API gdr_status gdr_decode_step(const gdr_dec_desc* desc,
  * gdr_decode_step are these calls with w = NULL.  Every kernel supports it; the chunk solver
  * is unchanged (A still uses beta), only U = (I + A)^{-1} diag(w) V changes.  The
  * content-aware erase of that page (beta modulated by the previous chunk's mean output)
- * is left to the caller, which passes the resulting beta.  Other arguments, layouts, errors
+ * is left to the caller, which passes the resulting beta; gdr_chunk_fwd_ex below also
+ * returns the chunk means it needs.  Other arguments, layouts, errors
  * and ownership as for gdr_chunk_fwd / gdr_decode_step.  (gdr_chunk_fwd_noalloc is tied only.)
  */
 GDR_API gdr_status gdr_chunk_fwd_untied(const gdr_fwd_desc* desc,
@@ -198,6 +199,30 @@ GDR_API gdr_status gdr_decode_step_untied(const gdr_dec_desc* desc,
                                           const float* g, const float* beta, const float* w,
                                           const float* theta, float* S, void* o,
                                           gdr_stream_t stream);
+
+/*
+ * gdr_chunk_fwd_untied with one more output: the mean of o over each chunk, the content
+ * signal of the content-aware erase ("CARVE" page, section 2.1: the chunk mean of the
+ * outputs the kernel already writes, fed through a zero-initialised low-rank projection
+ * into the next chunk's erase gate).
+ *
+ *   chunk_mean[b, c, h, :] = (1 / L_c) * sum over tokens t of chunk c of o[b, t, h, :]
+ *
+ * with chunks of desc->chunk (64) tokens and L_c the number of tokens of chunk c inside T
+ * (the last chunk may be shorter).  chunk_mean is fp32 [B, ceil(T/64), H, dv], 16-byte
+ * aligned, written whole; NULL = not computed (this call is then gdr_chunk_fwd_untied).  The
+ * kernels sum the fp32 outputs before rounding them to the output dtype, in the epilogue that
+ * writes o, so the only extra HBM traffic is the write of chunk_mean itself.  The projection
+ * and the gate (beta for chunk c + 1 from chunk_mean of chunk c) belong to the layer that
+ * produces beta.  Every kernel supports it.  Other arguments, layouts, errors and ownership
+ * as for gdr_chunk_fwd_untied.
+ */
+GDR_API gdr_status gdr_chunk_fwd_ex(const gdr_fwd_desc* desc,
+                                    const void* q, const void* k, const void* v,
+                                    const float* g, const float* beta, const float* w,
+                                    const float* theta, const float* S0, void* o, float* S_T,
+                                    float* chunk_mean, void* workspace, size_t workspace_bytes,
+                                    gdr_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word that

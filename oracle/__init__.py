@@ -97,6 +97,24 @@ def gdr_fwd(q, k, v, g, beta, theta=None, S0=None, gate_mode=GATE_LOGDECAY, scal
     return o, S_T
 
 
+def chunk_means(o, chunk=64):
+    """Mean of the outputs over each chunk ("CARVE" page, section 2.1: the chunk mean
+    m_c = (1/L) sum of o_t over chunk c, the content signal of its content-aware erase).
+
+    o: [B,T,H,dv].  Chunk c holds tokens c*chunk .. min((c+1)*chunk, T) - 1 and L is the
+    number of those tokens, so a short last chunk is averaged over its own tokens.
+    Returns [B, ceil(T/chunk), H, dv] float64.
+    """
+    o = np.asarray(o, dtype=np.float64)
+    B, T, H, dv = o.shape
+    nc = (T + chunk - 1) // chunk
+    m = np.zeros((B, nc, H, dv))
+    for c in range(nc):
+        t0, t1 = c * chunk, min((c + 1) * chunk, T)
+        m[:, c] = o[:, t0:t1].sum(axis=1) / (t1 - t0)
+    return m
+
+
 def gdr_decode_step(q, k, v, g, beta, S, theta=None, gate_mode=GATE_LOGDECAY, scale=1.0, w=None,
                     qk_l2norm=False):
     """One fp64 decode step (w: write strength [N,H] or None for w = beta).

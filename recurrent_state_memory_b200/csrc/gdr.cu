@@ -277,7 +277,7 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
 template <int MODE>
 static gdr_status dispatch_tc_mode(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws) {
     const bool ob = d->out_dtype == GDR_BF16;
-    if (p.w || p.qk_norm) {      // the kernel with the optional features
+    if (p.w || p.qk_norm || p.chunk_mean) {      // the kernel with the optional features
         if (d->rotation)
             return ob ? launch_tc<MODE, true, __nv_bfloat16, true>(p, st, ws) : launch_tc<MODE, true, float, true>(p, st, ws);
         return ob ? launch_tc<MODE, false, __nv_bfloat16, true>(p, st, ws) : launch_tc<MODE, false, float, true>(p, st, ws);
@@ -352,6 +352,14 @@ gdr_status gdr_chunk_fwd_untied(const gdr_fwd_desc* d, const void* q, const void
                                 const float* g, const float* beta, const float* w, const float* theta,
                                 const float* S0, void* o, float* S_T, void* workspace,
                                 size_t workspace_bytes, gdr_stream_t stream) {
+    return gdr_chunk_fwd_ex(d, q, k, v, g, beta, w, theta, S0, o, S_T, nullptr, workspace, workspace_bytes,
+                            stream);
+}
+
+gdr_status gdr_chunk_fwd_ex(const gdr_fwd_desc* d, const void* q, const void* k, const void* v,
+                            const float* g, const float* beta, const float* w, const float* theta,
+                            const float* S0, void* o, float* S_T, float* chunk_mean, void* workspace,
+                            size_t workspace_bytes, gdr_stream_t stream) {
     t_detail[0] = 0;
     gdr_status s = check_fwd_desc(d);
     if (s != GDR_OK) return s;
@@ -364,7 +372,7 @@ gdr_status gdr_chunk_fwd_untied(const gdr_fwd_desc* d, const void* q, const void
     }
     if (!d->rotation && theta) return fail(GDR_ERR_INVALID_ARG, "theta must be NULL without rotation%s");
     if ((theta && !aligned16(theta)) || (S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)) ||
-        (w && !aligned16(w)))
+        (w && !aligned16(w)) || (chunk_mean && !aligned16(chunk_mean)))
         return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
     const size_t need = gdr_chunk_fwd_workspace_bytes(d);
     if (need > 0 && (!workspace || workspace_bytes < need)) return fail(GDR_ERR_WORKSPACE, "workspace too small%s");
@@ -376,7 +384,7 @@ gdr_status gdr_chunk_fwd_untied(const gdr_fwd_desc* d, const void* q, const void
     p.gate_mode = (int)d->gate_mode;
     p.scale = d->scale;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.theta = theta;
-    p.S0 = S0; p.o = o; p.S_T = S_T;
+    p.S0 = S0; p.o = o; p.S_T = S_T; p.chunk_mean = chunk_mean;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d->T == 0 && !S_T) return GDR_OK;
     const gdr_algo algo = resolve_algo(d);
@@ -505,7 +513,7 @@ gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* d, const void* q, const voi
     p.gate_mode = (int)d->gate_mode;
     p.scale = d->scale;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = nullptr; p.theta = theta;
-    p.S0 = S0; p.o = o; p.S_T = S_T;
+    p.S0 = S0; p.o = o; p.S_T = S_T; p.chunk_mean = nullptr;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d->T == 0) return S_T ? dispatch_tc_mode<0>(d, p, st, nullptr) : GDR_OK;
     void* scratch = nullptr;

@@ -40,6 +40,7 @@ struct FwdParams {
     const float* S0;
     void* o;
     float* S_T;
+    float* chunk_mean;      // [B, ceil(T/64), H, dv] fp32 mean of o over each chunk, or nullptr
 };
 
 namespace simt {
@@ -288,12 +289,26 @@ __global__ void __launch_bounds__(NT) chunk_fwd_kernel(FwdParams p) {
         }
 
         // 7. O = QS + Pm E.
+        float msum = 0.f;     // chunk mean: this thread's column j = tid % DVT over its rows
         for (int idx = tid; idx < C * DVT; idx += NT) {
             const int r = idx / DVT, j = idx % DVT;
             if (r < Lc) {
                 float acc = QS[r * (DVT + 1) + j];
                 for (int i = 0; i <= r; ++i) acc = fmaf(Pm[r * (C + 1) + i], R[i * (DVT + 1) + j], acc);
                 st_from_f32(o + tok(r) * dv + j0 + j, acc);
+                msum += acc;
+            }
+        }
+        if (p.chunk_mean) {
+            // mean of this chunk's outputs (fp32, before rounding to the output type); QS is
+            // free once every thread is past step 7
+            __syncthreads();
+            QS[tid] = msum;
+            __syncthreads();
+            if (tid < DVT) {
+                float s = 0.f;
+                for (int w8 = 0; w8 < NT / DVT; ++w8) s += QS[w8 * DVT + tid];
+                p.chunk_mean[(((size_t)b * nchunks + c) * p.H + h) * dv + j0 + tid] = s / (float)Lc;
             }
         }
 

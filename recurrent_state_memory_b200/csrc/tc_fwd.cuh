@@ -266,6 +266,11 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
     const int nchunks = (p.T + C - 1) / C;
     const bool untied = EXT && p.w != nullptr;    // a write strength w separate from beta
     const bool qkn = EXT && p.qk_norm != 0;       // fused L2 normalisation of q and k
+    const bool cmean = EXT && p.chunk_mean != nullptr;   // per-chunk mean of o as a second output
+    // chunk_mean [B, nchunks, H, dv] fp32: element of (global head gx, chunk c, value row r)
+    auto cmean_at = [&](int gx, int c, int r) -> float* {
+        return p.chunk_mean + (((size_t)(gx / p.H) * nchunks + c) * p.H + gx % p.H) * D + r;
+    };
     auto chunk_len = [&](int c) -> int { return min(C, p.T - c * C); };
     auto tokh = [&](int bhx, int c, int r) -> size_t {      // bhx: local head
         const int gx = p.head0 + bhx;
@@ -1251,13 +1256,20 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     bulk_wait_read_all();           // the previous o store has read the staging
                 }
                 ebar();
+                float msum = 0.f;       // this value row's sum over the chunk's tokens
 #pragma unroll 1
                 for (int g = 0; g < 2; ++g) {
                     float vals[32];
                     tmem_ld32(tq + COL_O + g * 32, vals);
 #pragma unroll
                     for (int u = 0; u < 32; ++u) st_from_f32(stg + (g * 32 + u) * D + row, vals[u]);
+                    if (cmean) {
+                        const int Lg = chunk_len(c) - g * 32;    // tokens of this half inside T
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) msum += (u < Lg) ? vals[u] : 0.f;
+                    }
                 }
+                if (cmean) *cmean_at(gbh, c, row) = msum / (float)chunk_len(c);
                 tc_fence_before();
                 fence_proxy_async_smem();
                 ebar();
@@ -1325,10 +1337,15 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
             const int j8 = lane & 7, grp = lane >> 3;
             OT* obase = o + tok(c, 0) * D + quad * 32 + grp * 8;
             const size_t tstride = (size_t)p.H * D;
+            float msum = 0.f;           // this value row's sum over the chunk's tokens
 #pragma unroll 1
             for (int g = 0; g < 2; ++g) {
                 float vals[32];
                 tmem_ld32(tq + col + g * 32, vals);
+                if (cmean) {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) msum += (g * 32 + u < Lc) ? vals[u] : 0.f;
+                }
 #pragma unroll
                 for (int blk8 = 0; blk8 < 4; ++blk8) {
                     float v8[8];
@@ -1347,6 +1364,7 @@ __global__ void __launch_bounds__(nthreads<MODE>(), 1) chunk_fwd_tc_kernel(FwdPa
                     }
                 }
             }
+            if (cmean) *cmean_at(gbh, c, row) = msum / (float)Lc;
         };
 
         // Initial state, prescaled by the first chunk's reference decay.

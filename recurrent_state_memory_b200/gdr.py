@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_decode_step.argtypes = [ctypes.POINTER(DecDesc), vp, vp, vp, fp, fp, fp, fp, vp, vp]
         L.gdr_chunk_fwd_untied.restype = ctypes.c_int
         L.gdr_chunk_fwd_untied.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, fp, vp, sz, vp]
+        L.gdr_chunk_fwd_ex.restype = ctypes.c_int
+        L.gdr_chunk_fwd_ex.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, fp, fp, vp, sz, vp]
         L.gdr_decode_step_untied.restype = ctypes.c_int
         L.gdr_decode_step_untied.argtypes = [ctypes.POINTER(DecDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, vp]
         L.gdr_query_device_status.restype = ctypes.c_int
@@ -83,7 +85,7 @@ def lib() -> ctypes.CDLL:
         L.gdr_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp, vp]
         L.gdr_debug_set_tc_fault.restype = None
         L.gdr_debug_set_tc_fault.argtypes = [ctypes.c_int, ctypes.c_ulonglong]
-        if L.gdr_abi_version() != 2:
+        if L.gdr_abi_version() != 3:
             raise RuntimeError("libgdr.so ABI version mismatch")
         _lib = L
     return _lib
@@ -155,18 +157,22 @@ def workspace_bytes(desc: FwdDesc) -> int:
 
 def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
               algo="auto", out_dtype=None, want_state=True, o=None, S_T=None, workspace=None,
-              stream=None, chunk=64, w=None, qk_l2norm=False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Chunk-parallel forward.  Returns (o, S_T).
+              stream=None, chunk=64, w=None, qk_l2norm=False, want_chunk_mean=False,
+              chunk_mean=None):
+    """Chunk-parallel forward.  Returns (o, S_T), or (o, S_T, chunk_mean) when
+    want_chunk_mean is set or a chunk_mean tensor is passed.
 
     beta is the erase strength; w [B,T,H] (fp32) a separate write strength, or None for
-    the tied rule (w = beta).  With CUDA tensors the call is asynchronous on `stream`
+    the tied rule (w = beta).  chunk_mean [B, ceil(T/64), H, dv] (fp32) receives the mean
+    of o over each chunk.  With CUDA tensors the call is asynchronous on `stream`
     (default: the current stream).  With host tensors the inputs are copied to the current
-    device, the library is called, and o / S_T are copied back (synchronising).
+    device, the library is called, and the outputs are copied back (synchronising).
     """
     if not q.is_cuda:
         return _chunk_fwd_host(q, k, v, g, beta, theta, S0, gate_mode=gate_mode, scale=scale,
                                algo=algo, out_dtype=out_dtype, want_state=want_state, chunk=chunk, w=w,
-                               qk_l2norm=qk_l2norm)
+                               qk_l2norm=qk_l2norm,
+                               want_chunk_mean=want_chunk_mean or chunk_mean is not None)
     dev = q.device
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -200,11 +206,25 @@ def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTP
         S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
     if S_T is not None:
         _need(S_T, "S_T", torch.float32, dev)
+    with_mean = want_chunk_mean or chunk_mean is not None
+    if with_mean:
+        nc = (T + chunk - 1) // chunk
+        if chunk_mean is None:
+            chunk_mean = torch.empty((B, nc, H, dv), dtype=torch.float32, device=dev)
+        _need(chunk_mean, "chunk_mean", torch.float32, dev)
+        if tuple(chunk_mean.shape) != (B, nc, H, dv):
+            raise ValueError("chunk_mean has the wrong shape")
     desc = fwd_desc(B, H, T, dk, dv, q.dtype, out_dtype, gate_mode, rotation, scale, algo, chunk, qk_l2norm)
     need = workspace_bytes(desc)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if with_mean:
+        st = lib().gdr_chunk_fwd_ex(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                    _ptr(w), _ptr(theta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(chunk_mean),
+                                    _ptr(workspace), ws_bytes, _stream_handle(stream, dev))
+        _check(st, "gdr_chunk_fwd_ex")
+        return o, S_T, chunk_mean
     if w is None:
         st = lib().gdr_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                  _ptr(theta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
@@ -220,10 +240,8 @@ def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTP
 def _chunk_fwd_host(q, k, v, g, beta, theta, S0, w=None, **kw):
     dev = torch.device("cuda", torch.cuda.current_device())
     to = lambda t: None if t is None else t.to(dev, non_blocking=True)
-    o, S_T = chunk_fwd(to(q), to(k), to(v), to(g), to(beta), to(theta), to(S0), w=to(w), **kw)
-    o_h = o.to("cpu")
-    S_h = None if S_T is None else S_T.to("cpu")
-    return o_h, S_h
+    out = chunk_fwd(to(q), to(k), to(v), to(g), to(beta), to(theta), to(S0), w=to(w), **kw)
+    return tuple(None if t is None else t.to("cpu") for t in out)
 
 
 def decode_step(q, k, v, g, beta, S, theta=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,

@@ -111,6 +111,21 @@ def test_untied_entry_points_check_the_write_strength(G):
     assert st == G.GDR_ERR_INVALID_ARG
 
 
+def test_extended_entry_point_checks_the_chunk_mean_output(G):
+    """gdr_chunk_fwd_ex adds the chunk-mean output; a misaligned chunk_mean is rejected
+    before any launch, as is a misaligned w."""
+    L = G.lib()
+    d = _desc(G)
+    get = lambda n: ctypes.c_void_p(FAKE[n])
+    st = L.gdr_chunk_fwd_ex(ctypes.byref(d), get("q"), get("k"), get("v"), get("g"), get("beta"),
+                            None, None, None, get("o"), get("S_T"), ctypes.c_void_p(0x10004), None, 0, None)
+    assert st == G.GDR_ERR_INVALID_ARG
+    assert b"aligned" in L.gdr_last_error_detail()
+    st = L.gdr_chunk_fwd_ex(ctypes.byref(d), get("q"), get("k"), get("v"), get("g"), get("beta"),
+                            ctypes.c_void_p(0x10004), None, None, get("o"), get("S_T"), get("S_T"), None, 0, None)
+    assert st == G.GDR_ERR_INVALID_ARG
+
+
 def test_qk_l2norm_flag_is_checked(G):
     d = _desc(G)
     d.qk_l2norm = 2

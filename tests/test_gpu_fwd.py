@@ -309,6 +309,67 @@ def test_waves_split_remainder_parity(G, B, rotation):
     U.assert_fwd_parity(p, o, S, o_ref, S_ref)
 
 
+CMEAN_CASES = [
+    # (algo, dtype, B, H, T, rotation, s0, untied)
+    ("simt", "f32", 1, 2, 150, False, True, False),
+    ("simt", "bf16", 1, 2, 64, True, False, True),
+    ("tcgen05", "bf16", 2, 2, 257, False, True, False),
+    ("tcgen05", "bf16", 1, 3, 100, True, True, True),
+    ("tcgen05_split", "bf16", 2, 3, 333, False, True, True),
+    ("tcgen05_split", "bf16", 1, 2, 200, True, False, False),
+]
+
+
+@pytest.mark.parametrize("case", CMEAN_CASES, ids=lambda c: "{}_{}_B{}H{}T{}{}{}{}".format(
+    c[0], c[1], c[2], c[3], c[4], "_rot" if c[5] else "", "_s0" if c[6] else "", "_untied" if c[7] else ""))
+def test_chunk_mean_parity(G, case):
+    """The chunk means of o (the extended call's second output, the content signal of the
+    content-aware erase) against the oracle's chunk means of its fp64 o; ragged last chunks,
+    rotation, initial state, with and without a separate write strength."""
+    import torch
+    algo, dtype, B, H, T, rot, s0, untied = case
+    dk = 128 if algo != "simt" else 64
+    p = I.make_fwd(B, T, H, dk, dk, dtype=dtype, seed=1000 + T, rotation=rot, s0_std=0.2 if s0 else None)
+    w = I.make_write_strength(1001 + T, (B, T, H)) if untied else None
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "g", "beta", "theta", "S0")}
+    o, S, m = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["theta"], t["S0"], gate_mode=p.gate_mode,
+                          algo=algo, w=None if w is None else torch.from_numpy(w).cuda(), want_chunk_mean=True)
+    torch.cuda.synchronize()
+    assert G.query_device_status() == G.GDR_OK
+    o_ref, S_ref = oracle.gdr_fwd(p.widened("q"), p.widened("k"), p.widened("v"), p.widened("g"),
+                                  p.widened("beta"), p.widened("theta"), p.widened("S0"),
+                                  gate_mode=p.gate_mode, scale=p.scale,
+                                  w=None if w is None else w.astype(np.float64))
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref)
+    m_ref = oracle.chunk_means(o_ref, 64)
+    assert tuple(m.shape) == m_ref.shape
+    assert U.max_rel(m.cpu().numpy().astype(np.float64), m_ref) <= U.TOL_O[dtype]
+
+
+def test_chunk_mean_with_waves_and_on_host_buffers(G):
+    """More heads than SMs (fused waves plus a split remainder, heads offset into the batch)
+    with the chunk means requested; then the same call on host tensors returns the same
+    three outputs."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B, H, T = 1, sms + 13, 130
+    p = I.make_fwd(B, T, H, 128, 128, dtype="bf16", seed=1100, s0_std=0.2)
+    d = G.fwd_desc(B, H, T, 128, 128, torch.bfloat16, torch.bfloat16, p.gate_mode, False)
+    assert G.resolved_algo(d) == "tcgen05_waves"
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "g", "beta", "S0")}
+    o, S, m = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], None, t["S0"], gate_mode=p.gate_mode,
+                          want_chunk_mean=True)
+    torch.cuda.synchronize()
+    assert G.query_device_status() == G.GDR_OK
+    o_ref, S_ref = U.oracle_fwd(p)
+    U.assert_fwd_parity(p, o, S, o_ref, S_ref)
+    assert U.max_rel(m.cpu().numpy().astype(np.float64), oracle.chunk_means(o_ref, 64)) <= U.TOL_O["bf16"]
+    h = {key: val.cpu() for key, val in t.items()}
+    o_h, S_h, m_h = G.chunk_fwd(h["q"], h["k"], h["v"], h["g"], h["beta"], None, h["S0"], gate_mode=p.gate_mode,
+                                want_chunk_mean=True)
+    assert not o_h.is_cuda and torch.equal(o_h, o.cpu()) and torch.equal(S_h, S.cpu()) and torch.equal(m_h, m.cpu())
+
+
 L2NORM_CASES = [
     # (algo, dtype, B, H, T, rotation)
     ("simt", "f32", 1, 2, 150, False),

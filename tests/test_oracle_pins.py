@@ -468,3 +468,44 @@ def test_l2norm_prologue_keeps_zero_vectors_zero_and_decode_agrees():
                                         oracle.GATE_NEG_SOFTPLUS, qk_l2norm=True)
         assert _rel(o_t + 1e-300, o[:, t] + 1e-300) < 1e-12 or np.all(o[:, t] == o_t)
     assert _rel(S, S_f) < 1e-12
+
+
+# ---- chunk means of the output (the content signal of CARVE's content-aware erase) -------
+
+@pytest.mark.parametrize("T,chunk", [(150, 64), (64, 64), (37, 16), (1, 64)])
+def test_chunk_means_of_a_ramp_are_the_chunk_midpoints(T, chunk):
+    """o_t = t (every head and value row): the mean over tokens t0 .. t1-1 of a chunk is the
+    midpoint (t0 + t1 - 1) / 2 of an arithmetic series, the last chunk cut at T."""
+    o = np.broadcast_to(np.arange(T, dtype=np.float64)[None, :, None, None], (2, T, 3, 4)).copy()
+    m = oracle.chunk_means(o, chunk)
+    nc = -(-T // chunk)
+    assert m.shape == (2, nc, 3, 4)
+    for c in range(nc):
+        t0, t1 = c * chunk, min((c + 1) * chunk, T)
+        assert np.all(m[:, c] == (t0 + t1 - 1) / 2.0)
+
+
+def test_chunk_means_of_piecewise_constant_outputs_and_total_mass():
+    """o constant within each chunk returns that constant; and sum_c L_c m_c is the sum of
+    o over the whole sequence, for any o."""
+    rng = np.random.default_rng(91)
+    T, chunk = 200, 64
+    levels = rng.standard_normal((1, 4, 2, 5))
+    o = np.repeat(levels, chunk, axis=1)[:, :T]
+    assert _rel(oracle.chunk_means(o, chunk), levels) < 1e-14
+    o = rng.standard_normal((2, T, 3, 5))
+    m = oracle.chunk_means(o, chunk)
+    L = np.array([64, 64, 64, 8], dtype=np.float64)
+    assert _rel(np.einsum("bchd,c->bhd", m, L), o.sum(axis=1)) < 1e-13
+
+
+def test_chunk_means_of_a_full_write_are_the_value_means():
+    """beta = 1, unit keys, q_t = k_t: the readout returns v_t (S_t k_t = v_t), so the
+    chunk means of the recurrence's output are the chunk means of v, a closed form that
+    does not pass through the recurrence."""
+    rng = np.random.default_rng(92)
+    q, k, v, a, beta, theta, S0 = _rand_problem(rng, 1, 70, 2, 8, 6, rotation=True)
+    o, _ = oracle.gdr_fwd(k, k, v, a, np.ones_like(beta), theta, S0, oracle.GATE_NEG_SOFTPLUS)
+    m = oracle.chunk_means(o, 64)
+    assert _rel(m[:, 0], v[:, :64].mean(axis=1)) < 1e-12
+    assert _rel(m[:, 1], v[:, 64:].mean(axis=1)) < 1e-12
