@@ -261,13 +261,18 @@ def run_ours(args):
         h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
         d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
 
+        hdesc = gdr.fwd_desc(p.B, p.H, p.T, p.dk, p.dv, pinned["q"].dtype, o.dtype, p.gate_mode, p.theta is not None,
+                             p.scale, args.algo)
+        wsh = torch.empty(gdr.host_workspace_bytes(hdesc, S0=pinned.get("S0") is not None, S_T=True),
+                          dtype=torch.uint8, device=dev)
+
         def e2e_step():
-            d = {k: (None if t is None else dv_t[k].copy_(t, non_blocking=True)) for k, t in pinned.items()}
-            gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["theta"], d["S0"],
-                          gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o, S_T=S_T, stream=stream,
-                          workspace=wsp)
-            o_h.copy_(o, non_blocking=True)
-            S_h.copy_(S_T, non_blocking=True)
+            # the public call on host tensors: gdr_chunk_fwd_host copies each batch slice in,
+            # runs it and copies it out, overlapping neighbouring slices; returns when o and
+            # S_T are in host memory
+            gdr.chunk_fwd(pinned["q"], pinned["k"], pinned["v"], pinned["g"], pinned["beta"], pinned.get("theta"),
+                          pinned.get("S0"), gate_mode=p.gate_mode, scale=p.scale, algo=args.algo, o=o_h, S_T=S_h,
+                          stream=stream, workspace=wsh)
 
         for _ in range(2):
             e2e_step()

@@ -225,6 +225,44 @@ GDR_API gdr_status gdr_chunk_fwd_ex(const gdr_fwd_desc* desc,
                                     gdr_stream_t stream);
 
 /*
+ * gdr_chunk_fwd_ex on HOST buffers: q, k, v, g, beta, w, theta and S0 are read from host
+ * memory and o, S_T and chunk_mean are written to host memory; only the workspace is device
+ * memory.  Same arguments, layouts and results as gdr_chunk_fwd_ex (NULL = absent for w,
+ * theta, S0, S_T, chunk_mean), computed slice by slice over the batch: the B entries are cut
+ * into at most 8 slices of equal size (the last may be smaller), and each slice is one
+ * gdr_chunk_fwd_ex call with B = its entry count, so its kernel is the one AUTO (or
+ * desc->algo) picks for that B.
+ *
+ * Slice i's inputs are copied into device slot i % 2 on a copy stream of the library's, its
+ * forward runs on `stream`, and its outputs are copied back on a second copy stream, so the
+ * host-to-device copies, the device-to-host copies and the kernels of neighbouring slices
+ * overlap.  The copies run asynchronously (and overlap) only from page-locked host memory
+ * (cudaHostAlloc / cudaHostRegister); pageable buffers work but each copy then blocks the
+ * host thread.
+ *
+ * Ordering: the copies start after the work already queued on `stream`, and `stream` is
+ * complete only once every output is in host memory (synchronise it, or an event recorded
+ * on it, before reading o).  Host buffers must stay valid and unchanged until then.  The
+ * library's copy streams and events are created on a device's first call and kept until
+ * the process exits; calls from several host threads are enqueued one at a time.
+ *
+ * workspace: device memory of at least gdr_chunk_fwd_host_workspace_bytes(desc, ...) bytes,
+ * 16-byte aligned, given the same presence flags (non-zero when that argument is not NULL),
+ * else GDR_ERR_WORKSPACE.  It holds the split kernel's ring (if any) and two slots of
+ * per-slice inputs and outputs; like the ring it may be reused by later calls on the same
+ * stream.  Errors: as gdr_chunk_fwd_ex; GDR_ERR_CUDA if a copy cannot be queued (the outputs
+ * are then undefined).
+ */
+GDR_API size_t gdr_chunk_fwd_host_workspace_bytes(const gdr_fwd_desc* desc, int with_w, int with_S0,
+                                                  int with_S_T, int with_chunk_mean);
+GDR_API gdr_status gdr_chunk_fwd_host(const gdr_fwd_desc* desc,
+                                      const void* q, const void* k, const void* v,
+                                      const float* g, const float* beta, const float* w,
+                                      const float* theta, const float* S0, void* o, float* S_T,
+                                      float* chunk_mean, void* workspace, size_t workspace_bytes,
+                                      gdr_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that
  * kernels set when a bounded wait gives up (GDR_ERR_TIMEOUT) or when the tensor-core
  * kernel meets a decay outside its factored range (GDR_ERR_RANGE; the outputs of that

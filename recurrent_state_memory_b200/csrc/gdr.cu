@@ -309,6 +309,90 @@ static gdr_status decode_types(const gdr_dec_desc* d, const dec::DecParams& p, c
     return launch_decode<DK, ROT, float, float>(p, st);
 }
 
+// ---- host-buffer forward: batch slices through two device slots ----------------------------
+// gdr_chunk_fwd_host copies slice i's inputs into slot i % 2 on one copy stream, runs the
+// forward of that slice on the caller's stream and copies its outputs back on a second copy
+// stream, so the copies of neighbouring slices overlap each other and the compute.  The
+// streams and events are created once per device and kept for the life of the process.
+constexpr int HOST_MAX_DEVICES = 64;
+constexpr int HOST_MAX_SLICES = 8;
+struct HostPipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr;
+    cudaEvent_t loaded[2] = {}, computed[2] = {}, stored[2] = {};
+    bool ready = false;
+};
+static HostPipe s_pipe[HOST_MAX_DEVICES];
+static std::mutex s_pipe_mu;     // held while a call enqueues: the events are shared
+
+static gdr_status host_pipe(HostPipe** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= HOST_MAX_DEVICES) return fail(GDR_ERR_UNSUPPORTED, "device index out of range%s");
+    HostPipe& P = s_pipe[dev];
+    if (!P.ready) {
+        if ((e = cudaStreamCreateWithFlags(&P.h2d, cudaStreamNonBlocking)) != cudaSuccess ||
+            (e = cudaStreamCreateWithFlags(&P.d2h, cudaStreamNonBlocking)) != cudaSuccess ||
+            (e = cudaEventCreateWithFlags(&P.start, cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_fail(e, "host pipeline streams");
+        for (int i = 0; i < 2; ++i) {
+            if ((e = cudaEventCreateWithFlags(&P.loaded[i], cudaEventDisableTiming)) != cudaSuccess ||
+                (e = cudaEventCreateWithFlags(&P.computed[i], cudaEventDisableTiming)) != cudaSuccess ||
+                (e = cudaEventCreateWithFlags(&P.stored[i], cudaEventDisableTiming)) != cudaSuccess)
+                return cuda_fail(e, "host pipeline events");
+        }
+        P.ready = true;
+    }
+    *out = &P;
+    return GDR_OK;
+}
+
+// Bytes per batch entry of each tensor of the forward, in the order of HostTensor.
+enum HostTensor { HT_Q, HT_K, HT_V, HT_G, HT_BETA, HT_W, HT_THETA, HT_S0, HT_O, HT_ST, HT_CM, HT_COUNT };
+struct HostPlan {
+    size_t per_b[HT_COUNT];   // bytes of one batch entry (0: tensor absent)
+    size_t off[HT_COUNT];     // offset in a slot (256-byte aligned)
+    size_t slot_bytes;
+    size_t ring_bytes;        // split-kernel workspace at the start, rounded to 256
+    int bs, nslices;          // batch entries per slice, number of slices
+};
+static size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static void host_plan(const gdr_fwd_desc* d, bool w, bool S0, bool S_T, bool cm, HostPlan* P) {
+    const size_t T = (size_t)d->T, H = (size_t)d->H, dk = (size_t)d->dk, dv = (size_t)d->dv;
+    const size_t si = d->qkv_dtype == GDR_BF16 ? 2 : 4, so = d->out_dtype == GDR_BF16 ? 2 : 4;
+    const size_t ng = d->rotation ? dk / 2 : dk, nc = (T + 63) / 64;
+    P->per_b[HT_Q] = T * H * dk * si;
+    P->per_b[HT_K] = T * H * dk * si;
+    P->per_b[HT_V] = T * H * dv * si;
+    P->per_b[HT_G] = T * H * ng * 4;
+    P->per_b[HT_BETA] = T * H * 4;
+    P->per_b[HT_W] = w ? T * H * 4 : 0;
+    P->per_b[HT_THETA] = d->rotation ? T * H * (dk / 2) * 4 : 0;
+    P->per_b[HT_S0] = S0 ? H * dv * dk * 4 : 0;
+    P->per_b[HT_O] = T * H * dv * so;
+    P->per_b[HT_ST] = S_T ? H * dv * dk * 4 : 0;
+    P->per_b[HT_CM] = cm ? nc * H * dv * 4 : 0;
+    const int B = d->B > 0 ? d->B : 1;
+    const int ns = B < HOST_MAX_SLICES ? B : HOST_MAX_SLICES;
+    P->bs = (B + ns - 1) / ns;
+    P->nslices = (B + P->bs - 1) / P->bs;
+    size_t o = 0;
+    for (int t = 0; t < HT_COUNT; ++t) {
+        P->off[t] = o;
+        o += round256(P->per_b[t] * (size_t)P->bs);
+    }
+    P->slot_bytes = o;
+    // the slices have bs entries, the last one possibly fewer: the larger workspace of the two
+    gdr_fwd_desc sd = *d;
+    sd.B = P->bs;
+    size_t ring = gdr_chunk_fwd_workspace_bytes(&sd);
+    sd.B = B - (P->nslices - 1) * P->bs;
+    const size_t ring_last = gdr_chunk_fwd_workspace_bytes(&sd);
+    P->ring_bytes = round256(ring > ring_last ? ring : ring_last);
+}
+
 }  // namespace gdr
 
 using namespace gdr;
@@ -520,6 +604,97 @@ gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* d, const void* q, const voi
     s = noalloc_scratch(&scratch);
     if (s != GDR_OK) return s;
     return dispatch_tc_mode<1>(d, p, st, scratch);
+}
+
+size_t gdr_chunk_fwd_host_workspace_bytes(const gdr_fwd_desc* d, int with_w, int with_S0, int with_S_T,
+                                          int with_chunk_mean) {
+    if (check_fwd_desc(d) != GDR_OK || d->B == 0 || d->H == 0) return 0;
+    HostPlan P;
+    host_plan(d, with_w != 0, with_S0 != 0, with_S_T != 0, with_chunk_mean != 0, &P);
+    return P.ring_bytes + 2 * P.slot_bytes;
+}
+
+gdr_status gdr_chunk_fwd_host(const gdr_fwd_desc* d, const void* q, const void* k, const void* v,
+                              const float* g, const float* beta, const float* w, const float* theta,
+                              const float* S0, void* o, float* S_T, float* chunk_mean, void* workspace,
+                              size_t workspace_bytes, gdr_stream_t stream) {
+    t_detail[0] = 0;
+    gdr_status s = check_fwd_desc(d);
+    if (s != GDR_OK) return s;
+    if (d->B == 0 || d->H == 0) return GDR_OK;
+    if (d->T > 0 && (!q || !k || !v || !g || !beta || !o))
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta and o are required%s");
+    if (d->T > 0 && d->rotation && !theta) return fail(GDR_ERR_INVALID_ARG, "theta is required with rotation%s");
+    if (!d->rotation && theta) return fail(GDR_ERR_INVALID_ARG, "theta must be NULL without rotation%s");
+    HostPlan P;
+    host_plan(d, w != nullptr, S0 != nullptr, S_T != nullptr, chunk_mean != nullptr, &P);
+    if (!workspace || workspace_bytes < P.ring_bytes + 2 * P.slot_bytes)
+        return fail(GDR_ERR_WORKSPACE, "workspace too small (gdr_chunk_fwd_host_workspace_bytes)%s");
+    if (!aligned16(workspace)) return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned%s");
+    const void* host_in[HT_COUNT] = {q, k, v, g, beta, w, theta, S0, nullptr, nullptr, nullptr};
+    void* host_out[HT_COUNT] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                o, S_T, chunk_mean};
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+    std::lock_guard<std::mutex> lock(s_pipe_mu);
+    HostPipe* pp = nullptr;
+    s = host_pipe(&pp);
+    if (s != GDR_OK) return s;
+    HostPipe& H = *pp;
+    cudaError_t e;
+    // the copy streams start after the work already on the caller's stream
+    if ((e = cudaEventRecord(H.start, st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if ((e = cudaStreamWaitEvent(H.h2d, H.start, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(H.d2h, H.start, 0)) != cudaSuccess)
+        return cuda_fail(e, "cudaStreamWaitEvent");
+    for (int i = 0; i < P.nslices; ++i) {
+        const int j = i & 1;
+        const size_t b0 = (size_t)i * P.bs;
+        const int nb = (int)((size_t)d->B - b0 < (size_t)P.bs ? (size_t)d->B - b0 : (size_t)P.bs);
+        uint8_t* slot = ws + P.ring_bytes + (size_t)j * P.slot_bytes;
+        void* dptr[HT_COUNT];
+        for (int t = 0; t < HT_COUNT; ++t) dptr[t] = P.per_b[t] ? slot + P.off[t] : nullptr;
+        // inputs of slice i into slot j, once the slice two back has finished reading them
+        if (i >= 2 && (e = cudaStreamWaitEvent(H.h2d, H.computed[j], 0)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamWaitEvent");
+        for (int t = HT_Q; t <= HT_S0; ++t) {
+            const size_t n = P.per_b[t] * (size_t)nb;
+            if (n == 0 || !host_in[t]) continue;
+            e = cudaMemcpyAsync(dptr[t], static_cast<const uint8_t*>(host_in[t]) + P.per_b[t] * b0, n,
+                                cudaMemcpyHostToDevice, H.h2d);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (host to device)");
+        }
+        if ((e = cudaEventRecord(H.loaded[j], H.h2d)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+        // the forward of slice i on the caller's stream; its outputs overwrite slot j's, so it
+        // also waits for the slice two back to have been copied out
+        if ((e = cudaStreamWaitEvent(st, H.loaded[j], 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+        if (i >= 2 && (e = cudaStreamWaitEvent(st, H.stored[j], 0)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamWaitEvent");
+        gdr_fwd_desc sd = *d;
+        sd.B = nb;
+        s = gdr_chunk_fwd_ex(&sd, dptr[HT_Q], dptr[HT_K], dptr[HT_V], static_cast<const float*>(dptr[HT_G]),
+                             static_cast<const float*>(dptr[HT_BETA]), static_cast<const float*>(dptr[HT_W]),
+                             static_cast<const float*>(dptr[HT_THETA]), static_cast<const float*>(dptr[HT_S0]),
+                             dptr[HT_O], static_cast<float*>(dptr[HT_ST]), static_cast<float*>(dptr[HT_CM]),
+                             P.ring_bytes ? ws : nullptr, P.ring_bytes, stream);
+        if (s != GDR_OK) return s;
+        if ((e = cudaEventRecord(H.computed[j], st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+        // outputs of slice i back to the host
+        if ((e = cudaStreamWaitEvent(H.d2h, H.computed[j], 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+        for (int t = HT_O; t <= HT_CM; ++t) {
+            const size_t n = P.per_b[t] * (size_t)nb;
+            if (n == 0 || !host_out[t]) continue;
+            e = cudaMemcpyAsync(static_cast<uint8_t*>(host_out[t]) + P.per_b[t] * b0, dptr[t], n,
+                                cudaMemcpyDeviceToHost, H.d2h);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (device to host)");
+        }
+        if ((e = cudaEventRecord(H.stored[j], H.d2h)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    }
+    // the caller's stream completes once every output is in host memory
+    if ((e = cudaStreamWaitEvent(st, H.stored[(P.nslices - 1) & 1], 0)) != cudaSuccess)
+        return cuda_fail(e, "cudaStreamWaitEvent");
+    return GDR_OK;
 }
 
 void gdr_debug_set_tc_fault(int skip_first_commit, unsigned long long wait_limit_ns) {

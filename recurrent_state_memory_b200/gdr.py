@@ -12,7 +12,7 @@ from __future__ import annotations
 import ctypes
 import os
 import re
-from typing import Optional, Tuple
+from typing import Optional
 
 import torch
 
@@ -75,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.gdr_chunk_fwd_untied.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, fp, vp, sz, vp]
         L.gdr_chunk_fwd_ex.restype = ctypes.c_int
         L.gdr_chunk_fwd_ex.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, fp, fp, vp, sz, vp]
+        L.gdr_chunk_fwd_host.restype = ctypes.c_int
+        L.gdr_chunk_fwd_host.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, fp, fp, vp, sz, vp]
+        L.gdr_chunk_fwd_host_workspace_bytes.restype = sz
+        L.gdr_chunk_fwd_host_workspace_bytes.argtypes = [ctypes.POINTER(FwdDesc)] + [ctypes.c_int] * 4
         L.gdr_decode_step_untied.restype = ctypes.c_int
         L.gdr_decode_step_untied.argtypes = [ctypes.POINTER(DecDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, vp]
         L.gdr_query_device_status.restype = ctypes.c_int
@@ -155,6 +159,12 @@ def workspace_bytes(desc: FwdDesc) -> int:
     return int(lib().gdr_chunk_fwd_workspace_bytes(ctypes.byref(desc)))
 
 
+def host_workspace_bytes(desc: FwdDesc, w=False, S0=False, S_T=False, chunk_mean=False) -> int:
+    """Device workspace of gdr_chunk_fwd_host for this descriptor and these optional arguments."""
+    return int(lib().gdr_chunk_fwd_host_workspace_bytes(ctypes.byref(desc), int(bool(w)), int(bool(S0)),
+                                                        int(bool(S_T)), int(bool(chunk_mean))))
+
+
 def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
               algo="auto", out_dtype=None, want_state=True, o=None, S_T=None, workspace=None,
               stream=None, chunk=64, w=None, qk_l2norm=False, want_chunk_mean=False,
@@ -165,14 +175,12 @@ def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTP
     beta is the erase strength; w [B,T,H] (fp32) a separate write strength, or None for
     the tied rule (w = beta).  chunk_mean [B, ceil(T/64), H, dv] (fp32) receives the mean
     of o over each chunk.  With CUDA tensors the call is asynchronous on `stream`
-    (default: the current stream).  With host tensors the inputs are copied to the current
-    device, the library is called, and the outputs are copied back (synchronising).
+    (default: the current stream).  With host tensors it is one gdr_chunk_fwd_host call
+    (copies and kernels pipelined over batch slices inside the library; asynchronous copies
+    need page-locked tensors) on the current device, and it returns once the host outputs
+    are written; outputs it allocates are page-locked when q (or, for T = 0, S0) is.
     """
-    if not q.is_cuda:
-        return _chunk_fwd_host(q, k, v, g, beta, theta, S0, gate_mode=gate_mode, scale=scale,
-                               algo=algo, out_dtype=out_dtype, want_state=want_state, chunk=chunk, w=w,
-                               qk_l2norm=qk_l2norm,
-                               want_chunk_mean=want_chunk_mean or chunk_mean is not None)
+    host = not q.is_cuda
     dev = q.device
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -199,22 +207,37 @@ def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTP
         _need(S0, "S0", torch.float32, dev)
         if tuple(S0.shape) != (B, H, dv, dk):
             raise ValueError("S0 has the wrong shape")
+    # outputs it allocates are page-locked when the inputs are (asynchronous copies)
+    pin = host and any(t.is_pinned() for t in (q, S0) if t is not None and t.numel() > 0)
     if o is None:
-        o = torch.empty((B, T, H, dv), dtype=out_dtype, device=dev)
+        o = torch.empty((B, T, H, dv), dtype=out_dtype, device=dev, pin_memory=pin)
     _need(o, "o", out_dtype, dev)
     if S_T is None and want_state:
-        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev, pin_memory=pin)
     if S_T is not None:
         _need(S_T, "S_T", torch.float32, dev)
     with_mean = want_chunk_mean or chunk_mean is not None
     if with_mean:
         nc = (T + chunk - 1) // chunk
         if chunk_mean is None:
-            chunk_mean = torch.empty((B, nc, H, dv), dtype=torch.float32, device=dev)
+            chunk_mean = torch.empty((B, nc, H, dv), dtype=torch.float32, device=dev, pin_memory=pin)
         _need(chunk_mean, "chunk_mean", torch.float32, dev)
         if tuple(chunk_mean.shape) != (B, nc, H, dv):
             raise ValueError("chunk_mean has the wrong shape")
     desc = fwd_desc(B, H, T, dk, dv, q.dtype, out_dtype, gate_mode, rotation, scale, algo, chunk, qk_l2norm)
+    out = (o, S_T, chunk_mean) if with_mean else (o, S_T)
+    if host:
+        cdev = torch.device("cuda", torch.cuda.current_device())
+        need = host_workspace_bytes(desc, w is not None, S0 is not None, S_T is not None, with_mean)
+        if workspace is None and need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=cdev)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = lib().gdr_chunk_fwd_host(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                      _ptr(w), _ptr(theta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(chunk_mean),
+                                      _ptr(workspace), ws_bytes, _stream_handle(stream, cdev))
+        _check(st, "gdr_chunk_fwd_host")
+        (stream if stream is not None else torch.cuda.current_stream(cdev)).synchronize()
+        return out
     need = workspace_bytes(desc)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -224,24 +247,17 @@ def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTP
                                     _ptr(w), _ptr(theta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(chunk_mean),
                                     _ptr(workspace), ws_bytes, _stream_handle(stream, dev))
         _check(st, "gdr_chunk_fwd_ex")
-        return o, S_T, chunk_mean
-    if w is None:
+    elif w is None:
         st = lib().gdr_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                  _ptr(theta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
                                  _stream_handle(stream, dev))
+        _check(st, "gdr_chunk_fwd")
     else:
         st = lib().gdr_chunk_fwd_untied(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                         _ptr(w), _ptr(theta), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
                                         ws_bytes, _stream_handle(stream, dev))
-    _check(st, "gdr_chunk_fwd")
-    return o, S_T
-
-
-def _chunk_fwd_host(q, k, v, g, beta, theta, S0, w=None, **kw):
-    dev = torch.device("cuda", torch.cuda.current_device())
-    to = lambda t: None if t is None else t.to(dev, non_blocking=True)
-    out = chunk_fwd(to(q), to(k), to(v), to(g), to(beta), to(theta), to(S0), w=to(w), **kw)
-    return tuple(None if t is None else t.to("cpu") for t in out)
+        _check(st, "gdr_chunk_fwd_untied")
+    return out
 
 
 def decode_step(q, k, v, g, beta, S, theta=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,

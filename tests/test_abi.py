@@ -126,6 +126,25 @@ def test_extended_entry_point_checks_the_chunk_mean_output(G):
     assert st == G.GDR_ERR_INVALID_ARG
 
 
+def test_host_entry_workspace_and_argument_checks(G):
+    """gdr_chunk_fwd_host: the workspace holds two slots of one batch slice's inputs and
+    outputs (more with the optional tensors); a short workspace and a missing theta are
+    rejected before anything is queued."""
+    L = G.lib()
+    d = _desc(G, B=2, T=130)             # H=2 dk=dv=64 bf16: two slices of one entry
+    base = G.host_workspace_bytes(d)
+    per_slice = 130 * 2 * (3 * 64 * 2 + 64 * 4 + 4 + 64 * 2)
+    assert base >= 2 * per_slice
+    assert G.host_workspace_bytes(d, w=True, S0=True, S_T=True, chunk_mean=True) > base
+    get = lambda n: ctypes.c_void_p(FAKE[n])
+    args = [get("q"), get("k"), get("v"), get("g"), get("beta"), None, None, None, get("o"), None, None]
+    st = L.gdr_chunk_fwd_host(ctypes.byref(d), *args, ctypes.c_void_p(0x100000), base - 1, None)
+    assert st == G.GDR_ERR_WORKSPACE
+    d.rotation = 1
+    st = L.gdr_chunk_fwd_host(ctypes.byref(d), *args, ctypes.c_void_p(0x100000), 1 << 40, None)
+    assert st == G.GDR_ERR_INVALID_ARG
+
+
 def test_qk_l2norm_flag_is_checked(G):
     d = _desc(G)
     d.qk_l2norm = 2

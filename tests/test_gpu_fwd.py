@@ -142,6 +142,46 @@ def test_host_buffers_round_trip(G):
     U.assert_fwd_parity(p, o, S, o_ref, S_ref)
 
 
+@pytest.mark.parametrize("B,T,rot,algo", [(5, 200, True, "auto"), (11, 130, False, "auto"), (3, 100, False, "simt"),
+                                          (3, 0, False, "simt")])
+def test_host_entry_pipelines_batch_slices(G, B, T, rot, algo):
+    """gdr_chunk_fwd_host on page-locked host tensors (separate write strength, initial state,
+    chunk means): the batch runs in slices of ceil(B / min(B, 8)) entries, one device call
+    each, with the copies of neighbouring slices overlapped.  Every output equals the device
+    calls on the same slices bit for bit, and the oracle within tolerance."""
+    import torch
+    dk = 128 if algo != "simt" else 64
+    p = I.make_fwd(B, T, 2, dk, dk, dtype="bf16", seed=1200 + B + T, rotation=rot, s0_std=0.2)
+    w = I.make_write_strength(1201 + B, (B, T, 2))
+    keys = ("q", "k", "v", "g", "beta", "theta", "S0")
+    h = {key: (None if getattr(p, key) is None else U.to_torch(getattr(p, key), "cpu").pin_memory()) for key in keys}
+    wh = torch.from_numpy(w).pin_memory()
+    o_h, S_h, m_h = G.chunk_fwd(h["q"], h["k"], h["v"], h["g"], h["beta"], h["theta"], h["S0"],
+                                gate_mode=p.gate_mode, algo=algo, w=wh, want_chunk_mean=True)
+    assert not o_h.is_cuda and S_h.is_pinned()
+    assert T == 0 or (o_h.is_pinned() and m_h.is_pinned())     # (an empty tensor has no pinned storage)
+    assert G.query_device_status() == G.GDR_OK
+    d = {key: (None if val is None else val.cuda()) for key, val in h.items()}
+    wd = wh.cuda()
+    bs = -(-B // min(B, 8))
+    cut = lambda t, sl: None if t is None else t[sl].contiguous()
+    for b0 in range(0, B, bs):
+        sl = slice(b0, min(B, b0 + bs))
+        o_d, S_d, m_d = G.chunk_fwd(cut(d["q"], sl), cut(d["k"], sl), cut(d["v"], sl), cut(d["g"], sl),
+                                    cut(d["beta"], sl), cut(d["theta"], sl), cut(d["S0"], sl),
+                                    gate_mode=p.gate_mode, algo=algo, w=cut(wd, sl), want_chunk_mean=True)
+        torch.cuda.synchronize()
+        assert torch.equal(o_h[sl], o_d.cpu()) and torch.equal(S_h[sl], S_d.cpu()) and torch.equal(m_h[sl], m_d.cpu())
+    o_ref, S_ref = oracle.gdr_fwd(p.widened("q"), p.widened("k"), p.widened("v"), p.widened("g"),
+                                  p.widened("beta"), p.widened("theta"), p.widened("S0"),
+                                  gate_mode=p.gate_mode, scale=p.scale, w=w.astype(np.float64))
+    if T == 0:
+        assert o_h.numel() == 0 and m_h.shape[1] == 0 and torch.equal(S_h, h["S0"])
+        return
+    U.assert_fwd_parity(p, o_h, S_h, o_ref, S_ref)
+    assert U.max_rel(m_h.numpy().astype(np.float64), oracle.chunk_means(o_ref, 64)) <= U.TOL_O["bf16"]
+
+
 FULL = ["b4_h16_t4096_d128", "b16_h12_t4096_d128_slow_s0", "b2_h16_t8192_d128_rot"]
 
 
