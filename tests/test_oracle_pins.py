@@ -509,3 +509,38 @@ def test_chunk_means_of_a_full_write_are_the_value_means():
     m = oracle.chunk_means(o, 64)
     assert _rel(m[:, 0], v[:, :64].mean(axis=1)) < 1e-12
     assert _rel(m[:, 1], v[:, 64:].mean(axis=1)) < 1e-12
+
+
+def test_chunk_mean_pins_catch_planted_mistakes():
+    """The ramp closed form sees plausible mistakes in a chunk mean: a short last chunk divided
+    by the full chunk length, chunk boundaries off by one token, and the mean taken over the
+    wrong axis."""
+    T, chunk = 150, 64
+    # o[b, t, h, j] = t (j + 1): value rows carry different ramps, so the axis matters
+    o = np.arange(T, dtype=np.float64)[None, :, None, None] * np.arange(1, 4)[None, None, None, :]
+    o = np.broadcast_to(o, (1, T, 2, 3)).copy()
+    nc = -(-T // chunk)
+
+    def expect(c):
+        t0, t1 = c * chunk, min((c + 1) * chunk, T)
+        return o[:, t0:t1].sum(axis=1) / (t1 - t0)
+
+    def planted(variant):
+        m = np.zeros((1, nc, 2, 3))
+        for c in range(nc):
+            t0, t1 = c * chunk, min((c + 1) * chunk, T)
+            if variant == "full_divisor":
+                m[:, c] = o[:, t0:t1].sum(axis=1) / chunk
+            elif variant == "shifted":
+                m[:, c] = o[:, t0 + 1:t1 + 1].mean(axis=1)
+            elif variant == "wrong_axis":
+                m[:, c] = o[:, t0:t1].mean(axis=-1, keepdims=True).mean(axis=1)
+        return m
+
+    m = oracle.chunk_means(o, chunk)
+    for c in range(nc):
+        assert _rel(m[:, c], expect(c)) < 1e-15
+        assert np.all(m[0, c, 0, 0] == (c * chunk + min((c + 1) * chunk, T) - 1) / 2.0)
+    for variant in ("full_divisor", "shifted", "wrong_axis"):
+        bad = planted(variant)
+        assert max(_rel(bad[:, c], expect(c)) for c in range(nc)) > 1e-3, variant
