@@ -61,7 +61,7 @@ L2NORM_EPS = 1e-6
 
 def l2_normalise(x):
     """x / sqrt(sum x^2 + 1e-6) over the last axis, in fp64: the L2 normalisation of q and k
-    that the layer applies before the recurrence (task statement; CARVE / KDA mixers),
+    that gated-DeltaNet-family layers (CARVE, KDA) apply before the recurrence,
     with a small epsilon so that a zero vector stays zero."""
     x = np.asarray(x, dtype=np.float64)
     return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + L2NORM_EPS)

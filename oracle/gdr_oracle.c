@@ -20,8 +20,9 @@
  *     diag(alpha_t * exp(i theta_t)) is a direct sum of 2x2 rotation-decay blocks.
  *   - "CARVE" page, section 2.3: the decay is a key-axis exponential gate,
  *     D_t = diag(exp(g_t)) with g_t <= 0.
- *   - the readout o_t = S_t q_t uses the post-update state (the CARVE page
- *     writes S_{t-1} q_t in section 2.1; the benchmark spec fixes S_t).
+ *   - the readout o_t = S_t q_t uses the post-update state, so o_t sees the token's
+ *     own write (the convention of this library; the CARVE page writes S_{t-1} q_t in
+ *     section 2.1).
  *   - "CARVE" page, sections 2.1-2.2: an erase gate b_t and a separate scalar value
  *     write gate w_{h,t} per head and token.  Read here as the erase strength that
  *     multiplies the removal along k_t and the write strength that multiplies v_t k_t^T;

@@ -5,7 +5,7 @@ import numpy as np
 import oracle
 from recurrent_state_memory_b200 import inputs as I
 
-# Tolerances (the benchmark spec's parity bars):
+# Parity tolerances:
 #   o:   max|o - o_ref| / max|o_ref| <= 1e-4 (fp32 mode), <= 2e-2 (bf16 inputs)
 #   S_T: ||S_T - S_ref||_F / ||S_ref||_F <= 1e-2
 TOL_O = {"f32": 1e-4, "bf16": 2e-2}
