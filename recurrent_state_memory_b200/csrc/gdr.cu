@@ -643,6 +643,13 @@ gdr_status gdr_chunk_fwd_host(const gdr_fwd_desc* d, const void* q, const void* 
     if (s != GDR_OK) return s;
     HostPipe& H = *pp;
     cudaError_t e;
+    // On an error after copies were queued, the caller's stream still waits for the copy
+    // streams, so that host buffers are not released while a copy may still read or write them.
+    auto bail = [&](gdr_status err) -> gdr_status {
+        if (cudaEventRecord(H.loaded[0], H.h2d) == cudaSuccess) (void)cudaStreamWaitEvent(st, H.loaded[0], 0);
+        if (cudaEventRecord(H.stored[0], H.d2h) == cudaSuccess) (void)cudaStreamWaitEvent(st, H.stored[0], 0);
+        return err;
+    };
     // the copy streams start after the work already on the caller's stream
     if ((e = cudaEventRecord(H.start, st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     if ((e = cudaStreamWaitEvent(H.h2d, H.start, 0)) != cudaSuccess ||
@@ -657,20 +664,21 @@ gdr_status gdr_chunk_fwd_host(const gdr_fwd_desc* d, const void* q, const void* 
         for (int t = 0; t < HT_COUNT; ++t) dptr[t] = P.per_b[t] ? slot + P.off[t] : nullptr;
         // inputs of slice i into slot j, once the slice two back has finished reading them
         if (i >= 2 && (e = cudaStreamWaitEvent(H.h2d, H.computed[j], 0)) != cudaSuccess)
-            return cuda_fail(e, "cudaStreamWaitEvent");
+            return bail(cuda_fail(e, "cudaStreamWaitEvent"));
         for (int t = HT_Q; t <= HT_S0; ++t) {
             const size_t n = P.per_b[t] * (size_t)nb;
             if (n == 0 || !host_in[t]) continue;
             e = cudaMemcpyAsync(dptr[t], static_cast<const uint8_t*>(host_in[t]) + P.per_b[t] * b0, n,
                                 cudaMemcpyHostToDevice, H.h2d);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (host to device)");
+            if (e != cudaSuccess) return bail(cuda_fail(e, "cudaMemcpyAsync (host to device)"));
         }
-        if ((e = cudaEventRecord(H.loaded[j], H.h2d)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+        if ((e = cudaEventRecord(H.loaded[j], H.h2d)) != cudaSuccess) return bail(cuda_fail(e, "cudaEventRecord"));
         // the forward of slice i on the caller's stream; its outputs overwrite slot j's, so it
         // also waits for the slice two back to have been copied out
-        if ((e = cudaStreamWaitEvent(st, H.loaded[j], 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+        if ((e = cudaStreamWaitEvent(st, H.loaded[j], 0)) != cudaSuccess)
+            return bail(cuda_fail(e, "cudaStreamWaitEvent"));
         if (i >= 2 && (e = cudaStreamWaitEvent(st, H.stored[j], 0)) != cudaSuccess)
-            return cuda_fail(e, "cudaStreamWaitEvent");
+            return bail(cuda_fail(e, "cudaStreamWaitEvent"));
         gdr_fwd_desc sd = *d;
         sd.B = nb;
         s = gdr_chunk_fwd_ex(&sd, dptr[HT_Q], dptr[HT_K], dptr[HT_V], static_cast<const float*>(dptr[HT_G]),
@@ -678,22 +686,23 @@ gdr_status gdr_chunk_fwd_host(const gdr_fwd_desc* d, const void* q, const void* 
                              static_cast<const float*>(dptr[HT_THETA]), static_cast<const float*>(dptr[HT_S0]),
                              dptr[HT_O], static_cast<float*>(dptr[HT_ST]), static_cast<float*>(dptr[HT_CM]),
                              P.ring_bytes ? ws : nullptr, P.ring_bytes, stream);
-        if (s != GDR_OK) return s;
-        if ((e = cudaEventRecord(H.computed[j], st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+        if (s != GDR_OK) return bail(s);
+        if ((e = cudaEventRecord(H.computed[j], st)) != cudaSuccess) return bail(cuda_fail(e, "cudaEventRecord"));
         // outputs of slice i back to the host
-        if ((e = cudaStreamWaitEvent(H.d2h, H.computed[j], 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+        if ((e = cudaStreamWaitEvent(H.d2h, H.computed[j], 0)) != cudaSuccess)
+            return bail(cuda_fail(e, "cudaStreamWaitEvent"));
         for (int t = HT_O; t <= HT_CM; ++t) {
             const size_t n = P.per_b[t] * (size_t)nb;
             if (n == 0 || !host_out[t]) continue;
             e = cudaMemcpyAsync(static_cast<uint8_t*>(host_out[t]) + P.per_b[t] * b0, dptr[t], n,
                                 cudaMemcpyDeviceToHost, H.d2h);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (device to host)");
+            if (e != cudaSuccess) return bail(cuda_fail(e, "cudaMemcpyAsync (device to host)"));
         }
-        if ((e = cudaEventRecord(H.stored[j], H.d2h)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+        if ((e = cudaEventRecord(H.stored[j], H.d2h)) != cudaSuccess) return bail(cuda_fail(e, "cudaEventRecord"));
     }
     // the caller's stream completes once every output is in host memory
     if ((e = cudaStreamWaitEvent(st, H.stored[(P.nslices - 1) & 1], 0)) != cudaSuccess)
-        return cuda_fail(e, "cudaStreamWaitEvent");
+        return bail(cuda_fail(e, "cudaStreamWaitEvent"));
     return GDR_OK;
 }
 
