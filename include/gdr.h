@@ -251,7 +251,8 @@ GDR_API gdr_status gdr_chunk_fwd_ex(const gdr_fwd_desc* desc,
  * else GDR_ERR_WORKSPACE.  It holds the split kernel's ring (if any) and two slots of
  * per-slice inputs and outputs; like the ring it may be reused by later calls on the same
  * stream.  Errors: as gdr_chunk_fwd_ex; GDR_ERR_CUDA if a copy cannot be queued (the outputs
- * are then undefined).
+ * are then undefined, and `stream` still waits for the copies already queued, so host buffers
+ * may be released once it has completed).
  */
 GDR_API size_t gdr_chunk_fwd_host_workspace_bytes(const gdr_fwd_desc* desc, int with_w, int with_S0,
                                                   int with_S_T, int with_chunk_mean);
