@@ -9,7 +9,8 @@ library and its binding) never imports it.
 passages it follows).  ``chunk_wy`` and ``chunk_ut`` restate the chunk-parallel
 algebra in fp64 numpy so the tests can check it against the recurrence, as the
 "Semidirect Fourier Delta Attention" page reports doing in its results section
-(numerical verification against brute force).
+(numerical verification against brute force).  ``backward.gdr_bwd`` gives the fp64
+reverse-mode gradients of the same recurrence (the oracle of a backward pass).
 """
 import ctypes
 import os

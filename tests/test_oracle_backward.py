@@ -1,0 +1,151 @@
+"""Pins of the fp64 backward oracle (oracle/backward.py) against the forward oracle it
+differentiates (the C token recurrence): central finite differences of every input, exact
+adjoint identities for the inputs the outputs are linear in, and planted mistakes."""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import backward as bwd
+
+
+def _problem(rng, T, H, dk, dv, rotation, untied, gate_mode):
+    q = rng.standard_normal((1, T, H, dk))
+    k = rng.standard_normal((1, T, H, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((1, T, H, dv))
+    ng = dk // 2 if rotation else dk
+    g = rng.standard_normal((1, T, H, ng)) if gate_mode == 1 else -np.abs(rng.standard_normal((1, T, H, ng))) * 0.3
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((1, T, H))))
+    w = rng.uniform(0.2, 1.2, (1, T, H)) if untied else None
+    theta = rng.uniform(-np.pi, np.pi, (1, T, H, dk // 2)) if rotation else None
+    S0 = rng.standard_normal((1, H, dv, dk)) * 0.5
+    return dict(q=q, k=k, v=v, g=g, beta=beta, w=w, theta=theta, S0=S0)
+
+
+def _loss(x, gO, gS, gate_mode, scale):
+    o, S_T = oracle.gdr_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["theta"], x["S0"],
+                            gate_mode=gate_mode, scale=scale, w=x["w"])
+    return float(np.sum(gO * o) + np.sum(gS * S_T))
+
+
+@pytest.mark.parametrize("rotation,untied,gate_mode", [(False, False, 1), (False, True, 0), (True, False, 0),
+                                                       (True, True, 1)])
+def test_backward_matches_central_differences(rotation, untied, gate_mode):
+    """Every element of every input: (L(x + h) - L(x - h)) / 2h with L = <gO, o> + <gS, S_T>
+    computed by the C forward oracle, against the backward oracle's gradient."""
+    rng = np.random.default_rng(300 + 2 * rotation + untied)
+    T, H, dk, dv, scale = 6, 2, 4, 3, 0.7
+    x = _problem(rng, T, H, dk, dv, rotation, untied, gate_mode)
+    gO = rng.standard_normal((1, T, H, dv))
+    gS = rng.standard_normal((1, H, dv, dk))
+    o, S_T, grads = bwd.gdr_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["theta"], x["S0"], gO, gS,
+                                gate_mode=gate_mode, scale=scale, w=x["w"])
+    o_ref, S_ref = oracle.gdr_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["theta"], x["S0"],
+                                  gate_mode=gate_mode, scale=scale, w=x["w"])
+    assert np.max(np.abs(o - o_ref)) < 1e-12 and np.max(np.abs(S_T - S_ref)) < 1e-12
+    h = 1e-6
+    names = ["q", "k", "v", "g", "beta", "S0"] + (["w"] if untied else []) + (["theta"] if rotation else [])
+    for n in names:
+        fd = np.zeros_like(x[n])
+        for idx in np.ndindex(x[n].shape):
+            xp = {m: (None if a is None else a.copy()) for m, a in x.items()}
+            xm = {m: (None if a is None else a.copy()) for m, a in x.items()}
+            xp[n][idx] += h
+            xm[n][idx] -= h
+            fd[idx] = (_loss(xp, gO, gS, gate_mode, scale) - _loss(xm, gO, gS, gate_mode, scale)) / (2 * h)
+        err = np.max(np.abs(grads[n] - fd)) / max(np.max(np.abs(fd)), 1e-12)
+        assert err < 1e-6, (n, err)
+    assert (grads["w"] is None) == (not untied) and (grads["theta"] is None) == (not rotation)
+
+
+def test_backward_adjoint_identities_are_exact():
+    """o and S_T are linear in (S0, v): for any direction d, L(x + d) - L(x) equals
+    <grad, d> up to rounding, with no finite-difference error."""
+    rng = np.random.default_rng(310)
+    T, H, dk, dv = 9, 2, 6, 5
+    x = _problem(rng, T, H, dk, dv, True, True, 1)
+    gO = rng.standard_normal((1, T, H, dv))
+    gS = rng.standard_normal((1, H, dv, dk))
+    _, _, grads = bwd.gdr_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["theta"], x["S0"], gO, gS,
+                              gate_mode=1, w=x["w"])
+    L0 = _loss(x, gO, gS, 1, 1.0)
+    for n in ("S0", "v"):
+        d = rng.standard_normal(x[n].shape)
+        xd = dict(x)
+        xd[n] = x[n] + d
+        assert abs((_loss(xd, gO, gS, 1, 1.0) - L0) - np.sum(grads[n] * d)) < 1e-10 * max(1.0, abs(L0))
+
+
+def test_backward_catches_planted_mistakes():
+    """The finite-difference pin is sharp enough to see plausible mistakes in a backward: the
+    erase term's gradient dropped from dk, the rotation's adjoint taken with e^{+i theta}, and
+    the readout gradient taken from the pre-update state."""
+    rng = np.random.default_rng(320)
+    T, H, dk, dv = 5, 1, 4, 3
+    x = _problem(rng, T, H, dk, dv, True, False, 0)
+    gO = rng.standard_normal((1, T, H, dv))
+    gS = rng.standard_normal((1, H, dv, dk))
+    sel = lambda a: None if a is None else a[0, :, 0]
+    args = (sel(x["q"]), sel(x["k"]), sel(x["v"]), sel(x["g"]), sel(x["beta"]), sel(x["theta"]), x["S0"][0, 0],
+            sel(gO), gS[0, 0], 0, 1.0, None)
+    _, _, ok = bwd.gdr_bwd_head(*args)
+
+    def fd(n):
+        out = np.zeros_like(x[n])
+        for idx in np.ndindex(x[n].shape):
+            xp = {m: (None if a is None else a.copy()) for m, a in x.items()}
+            xm = {m: (None if a is None else a.copy()) for m, a in x.items()}
+            xp[n][idx] += 1e-6
+            xm[n][idx] -= 1e-6
+            out[idx] = (_loss(xp, gO, gS, 0, 1.0) - _loss(xm, gO, gS, 0, 1.0)) / 2e-6
+        return out[0, :, 0] if n != "S0" else out[0, 0]
+
+    ref = {n: fd(n) for n in ("k", "q", "S0")}
+    for n in ref:
+        assert np.max(np.abs(ok[n] - ref[n])) < 1e-6 * np.max(np.abs(ref[n])), n
+    q, k, v, g, beta, theta, S0 = args[:7]
+    S = S0.copy()                   # forward states X_t of this problem
+    Xs = []
+    for t in range(T):
+        al = np.exp(g[t])
+        c, s_ = np.cos(theta[t]), np.sin(theta[t])
+        X = bwd._decay(S, al, c, s_)
+        Xs.append(X)
+        e = beta[t] * (v[t] - X @ k[t])
+        S = X + np.outer(e, k[t])
+
+    def back(conj_sign):
+        """The state adjoint G = dL/dS_t run backwards; conj_sign = +1 multiplies by
+        alpha e^{-i theta} (the adjoint of the decay), -1 by alpha e^{+i theta} (a mistake).
+        Returns dS0 and the dk of the correct sweep without the erase term's -beta X^T ge."""
+        G = gS[0, 0].copy()
+        k_wo = np.zeros_like(k)
+        for t in range(T - 1, -1, -1):
+            G = G + np.outer(gO[0, t, 0], q[t])
+            ge = G @ k[t]
+            k_wo[t] = ok["k"][t] + beta[t] * (Xs[t].T @ ge)
+            gX = G - beta[t] * np.outer(ge, k[t])
+            al = np.exp(g[t])
+            c, s_ = np.cos(theta[t]), conj_sign * np.sin(theta[t])
+            Gn = np.empty_like(gX)
+            Gn[:, 0::2] = al * (c * gX[:, 0::2] + s_ * gX[:, 1::2])
+            Gn[:, 1::2] = al * (c * gX[:, 1::2] - s_ * gX[:, 0::2])
+            G = Gn
+        return G, k_wo
+
+    dS0_ok, bad_k = back(+1)
+    assert np.max(np.abs(dS0_ok - ref["S0"])) < 1e-6 * np.max(np.abs(ref["S0"]))     # the sweep is right
+    # (a) dk without the erase term's -beta X^T ge
+    assert np.max(np.abs(bad_k - ref["k"])) > 1e-3 * np.max(np.abs(ref["k"]))
+    # (b) the adjoint of the rotation with e^{+i theta}
+    dS0_bad, _ = back(-1)
+    assert np.max(np.abs(dS0_bad - ref["S0"])) > 1e-3 * np.max(np.abs(ref["S0"]))
+    # (c) dq from the pre-update state S_{t-1}
+    S = S0.copy()
+    bad_q = np.zeros_like(q)
+    for t in range(T):
+        bad_q[t] = S.T @ gO[0, t, 0]
+        al = np.exp(g[t])
+        X = bwd._decay(S, al, np.cos(theta[t]), np.sin(theta[t]))
+        S = X + np.outer(beta[t] * (v[t] - X @ k[t]), k[t])
+    assert np.max(np.abs(bad_q - ref["q"])) > 1e-3 * np.max(np.abs(ref["q"]))
