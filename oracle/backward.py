@@ -27,6 +27,9 @@ chain rule runs backwards over the tokens with the states recomputed forward and
     G <- gX D_t^T  (rotation: gX times alpha e^{-i theta} per pair);  dS0 = G after token 1
     dalpha = sum over rows of gX * dX/dalpha;  dtheta = sum over rows of (gX_b X_a - gX_a X_b)
     dg = dalpha * dalpha/dg  (alpha for gate mode 0; -alpha sigmoid(a) for gate mode 1)
+
+``chunk_bwd_head`` computes the same gradients by the chunk-parallel WY/UT algebra (real
+decay), the form a backward kernel takes; the tests hold it to the token-level sweep.
 """
 import numpy as np
 
@@ -137,3 +140,102 @@ def gdr_bwd(q, k, v, g, beta, theta=None, S0=None, gO=None, gS=None, gate_mode=0
                     out[n][b, :, h] = gr[n]
             out["S0"][b, h] = gr["S0"]
     return o, S_T, out
+
+
+def chunk_bwd_head(q, k, v, g, beta, S0, gO, gS, gate_mode, scale, w, chunk=64):
+    """The same gradients for one head (real decay), by the chunk-parallel WY/UT algebra that a
+    backward kernel follows, restated in fp64 ("CARVE" page, section 1 item 3: the WY-form
+    chunk solver; "Semidirect Fourier Delta Attention" page, *Constructive Chunk-WY Theorem*).
+
+    Forward of a chunk with start state S0 (dv x dk), gamma = in-chunk cumulative log decay:
+        Ktil = K e^{gamma},  Qtil = scale Q e^{gamma},  Khat = K e^{-gamma},  Kdec = K e^{gamma_L - gamma}
+        A = diag(beta) strict_lower(Ktil Khat^T),  P = incl_lower(Qtil Khat^T),  T = (I + A)^{-1}
+        R = diag(w) V - diag(beta) Ktil S0^T,  E = T R
+        O = Qtil S0^T + P E,  S_L = S0 diag(e^{gamma_L}) + E^T Kdec
+    The chunk-start states come from a forward sweep; the backward sweep runs the chunks in
+    reverse with dS_L of chunk c = dS0 of chunk c + 1 (gS for the last chunk).
+    Returns (o, S_T, grads) like ``gdr_bwd_head`` (no rotation).
+    """
+    T_, dk = q.shape
+    dv = v.shape[1]
+    wv = beta if w is None else w
+    nc = (T_ + chunk - 1) // chunk
+    al, dal = _alpha(g, gate_mode)
+    lg = np.log(al)            # log alpha per token and key dim
+    dlg = dal / al             # d log alpha / d (gate input)
+
+    def parts(c, S0c):
+        t0, t1 = c * chunk, min((c + 1) * chunk, T_)
+        K, Q, V = k[t0:t1], q[t0:t1], v[t0:t1]
+        gam = np.cumsum(lg[t0:t1], axis=0)
+        gl = gam[-1]
+        Kt, Qt, Kh, Kd = K * np.exp(gam), scale * Q * np.exp(gam), K * np.exp(-gam), K * np.exp(gl - gam)
+        L = t1 - t0
+        Ms, Mi = np.tril(np.ones((L, L)), -1), np.tril(np.ones((L, L)))
+        Ap = Kt @ Kh.T
+        A = beta[t0:t1, None] * (Ap * Ms)
+        P = (Qt @ Kh.T) * Mi
+        Tm = np.linalg.inv(np.eye(L) + A)
+        R = wv[t0:t1, None] * V - beta[t0:t1, None] * (Kt @ S0c.T)
+        E = Tm @ R
+        O = Qt @ S0c.T + P @ E
+        SL = S0c * np.exp(gl)[None, :] + E.T @ Kd
+        return dict(t0=t0, t1=t1, K=K, Q=Q, V=V, gam=gam, gl=gl, Kt=Kt, Qt=Qt, Kh=Kh, Kd=Kd, Ms=Ms,
+                    Mi=Mi, Ap=Ap, P=P, Tm=Tm, R=R, E=E, O=O, SL=SL, S0=S0c)
+
+    S = np.zeros((dv, dk)) if S0 is None else np.array(S0, dtype=np.float64)
+    fw = []
+    o = np.zeros((T_, dv))
+    for c in range(nc):
+        f = parts(c, S)
+        fw.append(f)
+        o[f["t0"]:f["t1"]] = f["O"]
+        S = f["SL"]
+    grads = {"q": np.zeros_like(q), "k": np.zeros_like(k), "v": np.zeros_like(v), "g": np.zeros_like(g),
+             "beta": np.zeros(T_), "w": None if w is None else np.zeros(T_), "theta": None}
+    dSL = np.zeros((dv, dk)) if gS is None else np.array(gS, dtype=np.float64)
+    for c in range(nc - 1, -1, -1):
+        f = fw[c]
+        t0, t1 = f["t0"], f["t1"]
+        dO = np.zeros((t1 - t0, dv)) if gO is None else gO[t0:t1]
+        S0c, E, P, Tm, R = f["S0"], f["E"], f["P"], f["Tm"], f["R"]
+        Kt, Qt, Kh, Kd, K, gam, gl = f["Kt"], f["Qt"], f["Kh"], f["Kd"], f["K"], f["gam"], f["gl"]
+        bt = beta[t0:t1]
+        # outputs: O = Qtil S0^T + P E ;  S_L = S0 diag(e^{gamma_L}) + E^T Kdec
+        dE = P.T @ dO + Kd @ dSL.T
+        dP = (dO @ E.T) * f["Mi"]
+        dQt = dO @ S0c + dP @ Kh
+        dKh = dP.T @ Qt
+        dS0 = dO.T @ Qt + dSL * np.exp(gl)[None, :]
+        dKd = E @ dSL
+        dgl = np.exp(gl) * np.sum(S0c * dSL, axis=0) + np.sum(dKd * Kd, axis=0)
+        # E = T R ;  T = (I + A)^{-1}
+        dR = Tm.T @ dE
+        dA = -Tm.T @ (dE @ R.T) @ Tm.T
+        # R = diag(w) V - diag(beta) Ktil S0^T
+        grads["v"][t0:t1] = wv[t0:t1, None] * dR
+        KS = Kt @ S0c.T
+        dbeta = -np.sum(dR * KS, axis=1)
+        if w is None:
+            dbeta += np.sum(dR * f["V"], axis=1)
+        else:
+            grads["w"][t0:t1] = np.sum(dR * f["V"], axis=1)
+        dKt = -(bt[:, None] * dR) @ S0c
+        dS0 -= (bt[:, None] * dR).T @ Kt
+        # A = diag(beta) strict_lower(Ktil Khat^T)
+        dbeta += np.sum(dA * f["Ap"] * f["Ms"], axis=1)
+        dAp = bt[:, None] * dA * f["Ms"]
+        dKt += dAp @ Kh
+        dKh += dAp.T @ Kt
+        grads["beta"][t0:t1] = dbeta
+        # factors of K, Q and the cumulative log decay gamma
+        eg = np.exp(gam)
+        grads["q"][t0:t1] = scale * dQt * eg
+        grads["k"][t0:t1] = dKt * eg + dKh / eg + dKd * np.exp(gl - gam)
+        dgam = dKt * Kt + dQt * Qt - dKh * Kh - dKd * Kd
+        dgam[-1] += dgl
+        dlog = np.cumsum(dgam[::-1], axis=0)[::-1]          # gamma = cumsum(log alpha)
+        grads["g"][t0:t1] = dlog * dlg[t0:t1]
+        dSL = dS0
+    grads["S0"] = dSL
+    return o, S, grads
