@@ -28,8 +28,8 @@ chain rule runs backwards over the tokens with the states recomputed forward and
     dalpha = sum over rows of gX * dX/dalpha;  dtheta = sum over rows of (gX_b X_a - gX_a X_b)
     dg = dalpha * dalpha/dg  (alpha for gate mode 0; -alpha sigmoid(a) for gate mode 1)
 
-``chunk_bwd_head`` computes the same gradients by the chunk-parallel WY/UT algebra (real
-decay), the form a backward kernel takes; the tests hold it to the token-level sweep.
+``chunk_bwd_head`` computes the same gradients by the chunk-parallel WY/UT algebra (real and
+rotation decay), the form a backward kernel takes; the tests hold it to the token-level sweep.
 """
 import numpy as np
 
@@ -142,34 +142,63 @@ def gdr_bwd(q, k, v, g, beta, theta=None, S0=None, gO=None, gS=None, gate_mode=0
     return o, S_T, out
 
 
-def chunk_bwd_head(q, k, v, g, beta, S0, gO, gS, gate_mode, scale, w, chunk=64):
-    """The same gradients for one head (real decay), by the chunk-parallel WY/UT algebra that a
-    backward kernel follows, restated in fp64 ("CARVE" page, section 1 item 3: the WY-form
-    chunk solver; "Semidirect Fourier Delta Attention" page, *Constructive Chunk-WY Theorem*).
+def _to_c(x):
+    """Key pairs (2j, 2j+1) of the last axis as complex numbers x_2j + i x_2j+1."""
+    return x[..., 0::2] + 1j * x[..., 1::2]
+
+
+def _to_r(z):
+    """Inverse of ``_to_c``."""
+    x = np.empty(z.shape[:-1] + (2 * z.shape[-1],))
+    x[..., 0::2], x[..., 1::2] = z.real, z.imag
+    return x
+
+
+def chunk_bwd_head(q, k, v, g, beta, S0, gO, gS, gate_mode, scale, w, chunk=64, theta=None):
+    """The same gradients for one head, by the chunk-parallel WY/UT algebra that a backward
+    kernel follows, restated in fp64 ("CARVE" page, section 1 item 3: the WY-form chunk
+    solver; "Semidirect Fourier Delta Attention" page, *Constructive Chunk-WY Theorem*).
 
     Forward of a chunk with start state S0 (dv x dk), gamma = in-chunk cumulative log decay:
         Ktil = K e^{gamma},  Qtil = scale Q e^{gamma},  Khat = K e^{-gamma},  Kdec = K e^{gamma_L - gamma}
         A = diag(beta) strict_lower(Ktil Khat^T),  P = incl_lower(Qtil Khat^T),  T = (I + A)^{-1}
         R = diag(w) V - diag(beta) Ktil S0^T,  E = T R
         O = Qtil S0^T + P E,  S_L = S0 diag(e^{gamma_L}) + E^T Kdec
-    The chunk-start states come from a forward sweep; the backward sweep runs the chunks in
-    reverse with dS_L of chunk c = dS0 of chunk c + 1 (gS for the last chunk).
-    Returns (o, S_T, grads) like ``gdr_bwd_head`` (no rotation).
+    Rotation (theta given): with key pairs as complex numbers and the cumulative factor
+    Lam_r = prod over the chunk's tokens t <= r of alpha_t e^{i theta_t} (per pair), the same
+    algebra holds with Ktil = K conj(Lam), Qtil = scale Q conj(Lam), Khat = K / Lam,
+    Kdec = K Lam_L / Lam and S0 Lam_L, every product of two tiles being the real dot product
+    of their (re, im) pairs.  The chunk-start states come from a forward sweep; the backward
+    sweep runs the chunks in reverse with dS_L of chunk c = dS0 of chunk c + 1 (gS for the
+    last chunk).  Returns (o, S_T, grads) like ``gdr_bwd_head``.
     """
     T_, dk = q.shape
     dv = v.shape[1]
+    rot = theta is not None
     wv = beta if w is None else w
     nc = (T_ + chunk - 1) // chunk
     al, dal = _alpha(g, gate_mode)
-    lg = np.log(al)            # log alpha per token and key dim
+    lg = np.log(al)            # log alpha per token and key dim (rotation: per pair)
     dlg = dal / al             # d log alpha / d (gate input)
 
     def parts(c, S0c):
         t0, t1 = c * chunk, min((c + 1) * chunk, T_)
         K, Q, V = k[t0:t1], q[t0:t1], v[t0:t1]
-        gam = np.cumsum(lg[t0:t1], axis=0)
-        gl = gam[-1]
-        Kt, Qt, Kh, Kd = K * np.exp(gam), scale * Q * np.exp(gam), K * np.exp(-gam), K * np.exp(gl - gam)
+        f = dict(t0=t0, t1=t1, K=K, Q=Q, V=V, S0=S0c)
+        if not rot:
+            gam = np.cumsum(lg[t0:t1], axis=0)
+            gl = gam[-1]
+            Kt, Qt, Kh, Kd = K * np.exp(gam), scale * Q * np.exp(gam), K * np.exp(-gam), K * np.exp(gl - gam)
+            S0dec = S0c * np.exp(gl)[None, :]
+            f.update(gam=gam, gl=gl)
+        else:
+            Lam = np.exp(np.cumsum(lg[t0:t1] + 1j * theta[t0:t1], axis=0))
+            LamL = Lam[-1]
+            Kc, Qc = _to_c(K), _to_c(Q)
+            Kt, Qt = _to_r(Kc * np.conj(Lam)), _to_r(scale * Qc * np.conj(Lam))
+            Kh, Kd = _to_r(Kc / Lam), _to_r(Kc * LamL / Lam)
+            S0dec = _to_r(_to_c(S0c) * LamL[None, :])
+            f.update(Lam=Lam, LamL=LamL, Kc=Kc, Qc=Qc)
         L = t1 - t0
         Ms, Mi = np.tril(np.ones((L, L)), -1), np.tril(np.ones((L, L)))
         Ap = Kt @ Kh.T
@@ -179,9 +208,9 @@ def chunk_bwd_head(q, k, v, g, beta, S0, gO, gS, gate_mode, scale, w, chunk=64):
         R = wv[t0:t1, None] * V - beta[t0:t1, None] * (Kt @ S0c.T)
         E = Tm @ R
         O = Qt @ S0c.T + P @ E
-        SL = S0c * np.exp(gl)[None, :] + E.T @ Kd
-        return dict(t0=t0, t1=t1, K=K, Q=Q, V=V, gam=gam, gl=gl, Kt=Kt, Qt=Qt, Kh=Kh, Kd=Kd, Ms=Ms,
-                    Mi=Mi, Ap=Ap, P=P, Tm=Tm, R=R, E=E, O=O, SL=SL, S0=S0c)
+        SL = S0dec + E.T @ Kd
+        f.update(Kt=Kt, Qt=Qt, Kh=Kh, Kd=Kd, Ms=Ms, Mi=Mi, Ap=Ap, P=P, Tm=Tm, R=R, E=E, O=O, SL=SL)
+        return f
 
     S = np.zeros((dv, dk)) if S0 is None else np.array(S0, dtype=np.float64)
     fw = []
@@ -192,23 +221,23 @@ def chunk_bwd_head(q, k, v, g, beta, S0, gO, gS, gate_mode, scale, w, chunk=64):
         o[f["t0"]:f["t1"]] = f["O"]
         S = f["SL"]
     grads = {"q": np.zeros_like(q), "k": np.zeros_like(k), "v": np.zeros_like(v), "g": np.zeros_like(g),
-             "beta": np.zeros(T_), "w": None if w is None else np.zeros(T_), "theta": None}
+             "beta": np.zeros(T_), "w": None if w is None else np.zeros(T_),
+             "theta": np.zeros_like(theta) if rot else None}
     dSL = np.zeros((dv, dk)) if gS is None else np.array(gS, dtype=np.float64)
     for c in range(nc - 1, -1, -1):
         f = fw[c]
         t0, t1 = f["t0"], f["t1"]
         dO = np.zeros((t1 - t0, dv)) if gO is None else gO[t0:t1]
         S0c, E, P, Tm, R = f["S0"], f["E"], f["P"], f["Tm"], f["R"]
-        Kt, Qt, Kh, Kd, K, gam, gl = f["Kt"], f["Qt"], f["Kh"], f["Kd"], f["K"], f["gam"], f["gl"]
+        Kt, Qt, Kh, Kd, K = f["Kt"], f["Qt"], f["Kh"], f["Kd"], f["K"]
         bt = beta[t0:t1]
-        # outputs: O = Qtil S0^T + P E ;  S_L = S0 diag(e^{gamma_L}) + E^T Kdec
+        # outputs: O = Qtil S0^T + P E ;  S_L = (S0 decayed over the chunk) + E^T Kdec
         dE = P.T @ dO + Kd @ dSL.T
         dP = (dO @ E.T) * f["Mi"]
         dQt = dO @ S0c + dP @ Kh
         dKh = dP.T @ Qt
-        dS0 = dO.T @ Qt + dSL * np.exp(gl)[None, :]
+        dS0 = dO.T @ Qt
         dKd = E @ dSL
-        dgl = np.exp(gl) * np.sum(S0c * dSL, axis=0) + np.sum(dKd * Kd, axis=0)
         # E = T R ;  T = (I + A)^{-1}
         dR = Tm.T @ dE
         dA = -Tm.T @ (dE @ R.T) @ Tm.T
@@ -228,14 +257,30 @@ def chunk_bwd_head(q, k, v, g, beta, S0, gO, gS, gate_mode, scale, w, chunk=64):
         dKt += dAp @ Kh
         dKh += dAp.T @ Kt
         grads["beta"][t0:t1] = dbeta
-        # factors of K, Q and the cumulative log decay gamma
-        eg = np.exp(gam)
-        grads["q"][t0:t1] = scale * dQt * eg
-        grads["k"][t0:t1] = dKt * eg + dKh / eg + dKd * np.exp(gl - gam)
-        dgam = dKt * Kt + dQt * Qt - dKh * Kh - dKd * Kd
-        dgam[-1] += dgl
-        dlog = np.cumsum(dgam[::-1], axis=0)[::-1]          # gamma = cumsum(log alpha)
-        grads["g"][t0:t1] = dlog * dlg[t0:t1]
+        # factors of K and Q, the chunk's decay of S0, and the cumulative decay
+        if not rot:
+            gam, gl = f["gam"], f["gl"]
+            eg = np.exp(gam)
+            dS0 += dSL * np.exp(gl)[None, :]
+            grads["q"][t0:t1] = scale * dQt * eg
+            grads["k"][t0:t1] = dKt * eg + dKh / eg + dKd * np.exp(gl - gam)
+            dgam = dKt * Kt + dQt * Qt - dKh * Kh - dKd * Kd
+            dgam[-1] += np.exp(gl) * np.sum(S0c * dSL, axis=0) + np.sum(dKd * Kd, axis=0)   # gamma_L terms
+            dlog = np.cumsum(dgam[::-1], axis=0)[::-1]          # gamma = cumsum(log alpha)
+            grads["g"][t0:t1] = dlog * dlg[t0:t1]
+        else:
+            # complex gradients g_z with dL = Re(conj(g_z) dz) per pair
+            Lam, LamL, Kc, Qc = f["Lam"], f["LamL"], f["Kc"], f["Qc"]
+            gKt, gQt, gKh, gKd, gSL = _to_c(dKt), _to_c(dQt), _to_c(dKh), _to_c(dKd), _to_c(dSL)
+            dS0 += _to_r(gSL * np.conj(LamL)[None, :])
+            grads["q"][t0:t1] = _to_r(scale * gQt * Lam)
+            grads["k"][t0:t1] = _to_r(gKt * Lam + gKh * np.conj(1.0 / Lam) + gKd * np.conj(LamL / Lam))
+            gLam = (np.conj(gKt) * Kc + scale * np.conj(gQt) * Qc - gKh * np.conj(Kc / Lam ** 2)
+                    - gKd * np.conj(Kc * LamL / Lam ** 2))
+            gLam[-1] += np.sum(gKd * np.conj(Kc / Lam), axis=0) + np.sum(gSL * np.conj(_to_c(S0c)), axis=0)
+            gz = np.cumsum((gLam * np.conj(Lam))[::-1], axis=0)[::-1]   # Lam = exp(cumsum(log alpha + i theta))
+            grads["g"][t0:t1] = gz.real * dlg[t0:t1]
+            grads["theta"][t0:t1] = gz.imag
         dSL = dS0
     grads["S0"] = dSL
     return o, S, grads

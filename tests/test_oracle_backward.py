@@ -151,21 +151,25 @@ def test_backward_catches_planted_mistakes():
     assert np.max(np.abs(bad_q - ref["q"])) > 1e-3 * np.max(np.abs(ref["q"]))
 
 
-@pytest.mark.parametrize("T,chunk,untied,gate_mode", [(70, 16, False, 1), (37, 8, True, 0), (64, 64, True, 1),
-                                                      (5, 64, False, 0)])
-def test_chunked_backward_equals_the_token_backward(T, chunk, untied, gate_mode):
+@pytest.mark.parametrize("T,chunk,untied,gate_mode,rotation", [(70, 16, False, 1, False), (37, 8, True, 0, False),
+                                                               (64, 64, True, 1, False), (5, 64, False, 0, False),
+                                                               (70, 16, True, 1, True), (37, 8, False, 0, True),
+                                                               (3, 64, True, 0, True)])
+def test_chunked_backward_equals_the_token_backward(T, chunk, untied, gate_mode, rotation):
     """The chunk-parallel WY/UT restatement of the backward (what a backward kernel computes,
     chunk by chunk with the state gradient carried backwards) against the token-level reverse
     sweep: outputs, final state and every gradient, several chunks and a ragged last one."""
     rng = np.random.default_rng(400 + T)
     dk, dv, scale = 8, 5, 0.8
-    x = _problem(rng, T, 1, dk, dv, False, untied, gate_mode)
+    x = _problem(rng, T, 1, dk, dv, rotation, untied, gate_mode)
     gO = rng.standard_normal((1, T, 1, dv))
     gS = rng.standard_normal((1, 1, dv, dk))
     sel = lambda a: None if a is None else a[0, :, 0]
     args = (sel(x["q"]), sel(x["k"]), sel(x["v"]), sel(x["g"]), sel(x["beta"]))
-    o1, S1, g1 = bwd.gdr_bwd_head(*args, None, x["S0"][0, 0], sel(gO), gS[0, 0], gate_mode, scale, sel(x["w"]))
-    o2, S2, g2 = bwd.chunk_bwd_head(*args, x["S0"][0, 0], sel(gO), gS[0, 0], gate_mode, scale, sel(x["w"]), chunk)
+    o1, S1, g1 = bwd.gdr_bwd_head(*args, sel(x["theta"]), x["S0"][0, 0], sel(gO), gS[0, 0], gate_mode, scale,
+                                  sel(x["w"]))
+    o2, S2, g2 = bwd.chunk_bwd_head(*args, x["S0"][0, 0], sel(gO), gS[0, 0], gate_mode, scale, sel(x["w"]), chunk,
+                                    theta=sel(x["theta"]))
     assert np.max(np.abs(o2 - o1)) < 1e-10 * np.max(np.abs(o1)) and np.max(np.abs(S2 - S1)) < 1e-10 * np.max(np.abs(S1))
-    for n in ("q", "k", "v", "g", "beta", "S0") + (("w",) if untied else ()):
+    for n in ("q", "k", "v", "g", "beta", "S0") + (("w",) if untied else ()) + (("theta",) if rotation else ()):
         assert np.max(np.abs(g2[n] - g1[n])) < 1e-9 * max(np.max(np.abs(g1[n])), 1e-12), n
