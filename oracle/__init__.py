@@ -98,6 +98,40 @@ def gdr_fwd(q, k, v, g, beta, theta=None, S0=None, gate_mode=GATE_LOGDECAY, scal
     return o, S_T
 
 
+def segment_scan(q, k, v, g, beta, theta=None, S0=None, segment=256, gate_mode=GATE_LOGDECAY, scale=1.0,
+                 w=None):
+    """The forward in sequence-parallel form, for one head: the affine transfer of the state
+    over a stretch of tokens ("Semidirect Fourier Delta Attention" page, *Main contributions*:
+    S_end = S_start A + B, exact) applied to segments of the sequence.
+
+    q, k [T,dk]; v [T,dv]; g, beta, w, theta per token as in ``gdr_fwd``; S0 [dv,dk] or None.
+    Each segment s (tokens s*segment .. end) is computed independently of the others, twice:
+      - from the zero state, giving its outputs o0_t and its write summary B_s = final state;
+      - from the identity state (dk x dk) with v = 0, giving o'_t = A_{s,t} (scale q_t) and its
+        transfer A_s = final state, with A_{s,t} the product of the segment's token transitions
+        D_t (I - beta_t k_t k_t^T) up to t.
+    Then a sequential scan over segments gives each start state, S_{s+1} = S_s A_s + B_s, and
+    the outputs are o_t = o0_t + S_s o'_t.  Returns (o [T,dv], S_T [dv,dk]).
+    """
+    q, k, v, g, beta, theta, S0, w = map(_f64, (q, k, v, g, beta, theta, S0, w))
+    T, dk = q.shape
+    dv = v.shape[1]
+    one = lambda a, t0, t1: None if a is None else a[None, t0:t1, None]
+    S = np.zeros((dv, dk)) if S0 is None else S0.copy()
+    o = np.zeros((T, dv))
+    for t0 in range(0, T, segment):
+        t1 = min(t0 + segment, T)
+        args = (one(q, t0, t1), one(k, t0, t1))
+        rest = (one(g, t0, t1), one(beta, t0, t1), one(theta, t0, t1))
+        o0, B_s = gdr_fwd(*args, one(v, t0, t1), *rest, None, gate_mode=gate_mode, scale=scale,
+                          w=one(w, t0, t1))
+        oI, A_s = gdr_fwd(*args, np.zeros((1, t1 - t0, 1, dk)), *rest, np.eye(dk)[None, None],
+                          gate_mode=gate_mode, scale=scale, w=one(w, t0, t1))
+        o[t0:t1] = o0[0, :, 0] + oI[0, :, 0] @ S.T
+        S = S @ A_s[0, 0] + B_s[0, 0]
+    return o, S
+
+
 def chunk_means(o, chunk=64):
     """Mean of the outputs over each chunk ("CARVE" page, section 2.1: the chunk mean
     m_c = (1/L) sum of o_t over chunk c, the content signal of its content-aware erase).

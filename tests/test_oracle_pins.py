@@ -544,3 +544,22 @@ def test_chunk_mean_pins_catch_planted_mistakes():
     for variant in ("full_divisor", "shifted", "wrong_axis"):
         bad = planted(variant)
         assert max(_rel(bad[:, c], expect(c)) for c in range(nc)) > 1e-3, variant
+
+
+# ---- sequence-parallel form: segments joined by the affine state transfer (NEXT-3) ---------
+
+@pytest.mark.parametrize("T,segment,rotation,untied", [(200, 64, False, False), (130, 50, True, True),
+                                                       (97, 256, True, False), (64, 1, False, True)])
+def test_segment_scan_equals_the_token_recurrence(T, segment, rotation, untied):
+    """Segments computed independently (from the zero state and from the identity), joined by
+    a sequential scan of S_{s+1} = S_s A_s + B_s and an output correction S_s A_{s,t} q_t,
+    reproduce the token recurrence: segment lengths that divide T, that do not, a single
+    segment and one-token segments."""
+    rng = np.random.default_rng(600 + T)
+    q, k, v, a, beta, theta, S0 = _rand_problem(rng, 1, T, 1, 8, 6, rotation)
+    w = _write_gate(rng, (1, T, 1)) if untied else None
+    sel = lambda x: None if x is None else x[0, :, 0]
+    o_ref, S_ref = oracle.gdr_fwd(q, k, v, a, beta, theta, S0, oracle.GATE_NEG_SOFTPLUS, w=w)
+    o, S = oracle.segment_scan(sel(q), sel(k), sel(v), sel(a), sel(beta), sel(theta), S0[0, 0], segment,
+                               oracle.GATE_NEG_SOFTPLUS, w=sel(w))
+    assert _rel(o, o_ref[0, :, 0]) < 1e-11 and _rel(S, S_ref[0, 0]) < 1e-11
