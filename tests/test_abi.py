@@ -145,6 +145,31 @@ def test_host_entry_workspace_and_argument_checks(G):
     assert st == G.GDR_ERR_INVALID_ARG
 
 
+def test_auto_resolution_and_workspace_sizes_without_a_device(G):
+    """With no device visible the library assumes a B200's 148 SMs.  AUTO's choice follows the
+    rules gdr.h states (split when 2 B*H <= SMs and T > 64; whole fused waves plus a split
+    remainder when B*H > SMs and the remainder fits that rule; fused otherwise; the CUDA-core
+    kernel for other shapes), and the split workspace is B*H*8 slots of 76,288 bytes plus
+    36 bytes of flags per head and one task counter."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("the 148-SM assumption holds only where no device is visible")
+    bf = torch.bfloat16
+    d = lambda B, H, T, dk=128: G.fwd_desc(B, H, T, dk, dk, bf, bf)
+    split = lambda nh: nh * 8 * 76288 + (nh * 8 + nh + 1) * 4
+    assert G.resolved_algo(d(4, 16, 4096)) == "tcgen05_split" and G.workspace_bytes(d(4, 16, 4096)) == split(64)
+    assert G.resolved_algo(d(2, 37, 4096)) == "tcgen05_split"            # 74 heads: exactly half
+    assert G.resolved_algo(d(1, 75, 4096)) == "tcgen05"                  # 75 heads: more than half
+    assert G.resolved_algo(d(4, 16, 64)) == "tcgen05"                    # a single chunk
+    assert G.resolved_algo(d(16, 12, 4096)) == "tcgen05_waves"           # 192 = 148 + 44
+    assert G.workspace_bytes(d(16, 12, 4096)) == split(44)
+    assert G.resolved_algo(d(2, 118, 4096)) == "tcgen05"                 # 236 = 148 + 88: 88 > 74
+    assert G.workspace_bytes(d(2, 118, 4096)) == 0
+    assert G.resolved_algo(d(4, 16, 4096, dk=64)) == "simt"
+    f32 = G.fwd_desc(4, 16, 4096, 128, 128, torch.float32, torch.float32)
+    assert G.resolved_algo(f32) == "simt" and G.workspace_bytes(f32) == 0
+
+
 def test_qk_l2norm_flag_is_checked(G):
     d = _desc(G)
     d.qk_l2norm = 2
