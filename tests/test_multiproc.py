@@ -54,3 +54,21 @@ def test_single_process_helpers_are_identity():
     assert bench.max_over_ranks(3.5) == 3.5
     assert bench.sum_over_ranks(2.0) == 2.0
     assert bench.rank_seed(4, 0) == 4
+
+
+def test_reference_arm_prints_one_contract_line(capsys):
+    """`bench.py --impl reference` (the fp64 oracle timed on the host cores) prints one JSON
+    line with the forward metric, impl "reference", an oracle cpu_baseline and an e2e object
+    with no host-device traffic; it needs no GPU."""
+    import json
+
+    import bench
+    bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"])
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "Mtokens/s"
+    assert d["value"] > 0 and d["higher_is_better"] and d["steps"] == 1 and d["gpu_launches"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "Mtokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"] == bench.WORKLOAD
