@@ -177,6 +177,14 @@ def fwd_flops_per_token_head(dk, dv, C=64):
     return 6 * dk * dv + C * (3 * dk + 2 * dv)
 
 
+def workload_config(name, p):
+    """The `config` object of the JSON line, identical in both arms for the same workload."""
+    return {"workload": name, "B": p.B, "H": p.H, "T": p.T, "dk": p.dk, "dv": p.dv, "chunk": p.chunk,
+            "inputs": "bf16 q/k/v, fp32 raw gate (-softplus fused) and beta" if p.dtype == "bf16" else
+                      "fp32 q/k/v, gate and beta",
+            "l2": f"inputs {p.nbytes_algorithmic / 1e6:.0f} MB vs L2 {L2_BYTES / 1e6:.0f} MB; no flush"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -383,11 +391,8 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if resolved.startswith("tcgen05") else "f32",
         "data": "synthetic (seeded SplitMix64; q,k L2-normalised, bf16)",
-        "config": {"workload": f"{args.workload}: B={p.B} H={p.H} T={p.T} dk={p.dk} dv={p.dv} chunk={p.chunk}, "
-                               "bf16 q/k/v, fp32 g (raw gate, -softplus fused) and beta, S0=0",
-                   "B": p.B, "H": p.H, "T": p.T, "dk": p.dk, "dv": p.dv, "chunk": p.chunk, "algo": resolved,
-                   "per_rank_batch": p.B, "parallelism": f"replicas x{ws} (independent batches)",
-                   "l2": f"inputs {algo_bytes / 1e6:.0f} MB > L2 {L2_BYTES / 1e6:.0f} MB; no flush"},
+        "config": workload_config(args.workload, p),
+        "algo": resolved, "per_rank_batch": p.B, "parallelism": f"replicas x{ws} (independent batches)",
         "tflops_algorithmic": round(tflops, 2),
         "roofline": roofline,
         "e2e": e2e,
@@ -403,29 +408,31 @@ def run_ours(args):
 
 
 def cpu_baseline(p, seconds: float):
-    """The oracle, as it stands, on a bounded sample of whole heads of the workload."""
+    """The oracle, as it stands, on a bounded sample of whole heads of the workload.  Each group
+    of heads is laid out for the oracle before its clock starts, so that only the oracle's own
+    run is timed (as in the reference arm)."""
     import oracle
-    t0 = time.time()
-    heads_done, tokens = 0, 0
+    heads_done, tokens, el = 0, 0, 0.0
     order = [(b, h) for b in range(p.B) for h in range(p.H)]
     batch = max(1, oracle.num_threads())
     i = 0
-    while i < len(order) and (time.time() - t0) < seconds:
+    while i < len(order) and el < seconds:
         grp = order[i:i + batch]
         sl = [p.head_slice(b, h) for (b, h) in grp]
-        # run the group as one oracle call so its OpenMP loop spreads over the cores
+        # the group as one oracle call, so that its OpenMP loop spreads over the cores
         cat = lambda key: None if getattr(sl[0], key) is None else np.concatenate([s.widened(key) for s in sl], axis=0)
-        oracle.gdr_fwd(cat("q"), cat("k"), cat("v"), cat("g"), cat("beta"), cat("theta"), cat("S0"),
-                       gate_mode=p.gate_mode, scale=p.scale)
+        arrs = [cat(key) for key in ("q", "k", "v", "g", "beta", "theta", "S0")]
+        t0 = time.perf_counter()
+        oracle.gdr_fwd(*arrs, gate_mode=p.gate_mode, scale=p.scale)
+        el += time.perf_counter() - t0
         heads_done += len(grp)
         tokens += len(grp) * p.T
         i += batch
-    el = time.time() - t0
     # per-head token throughput scaled to the workload's unit: tokens of B*T over all H heads
     value = (tokens / p.H) / el / 1e6
     return {"value": round(value, 6), "unit": "Mtokens/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{heads_done} whole heads (T={p.T}) of the workload, fp64 token recurrence, "
-                      f"{el:.1f} s; tokens counted as B*T over all H heads"}
+                      f"{el:.1f} s of oracle time; tokens counted as B*T over all H heads"}
 
 
 # ------------------------------------------------------- reference arm ----
@@ -459,8 +466,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded SplitMix64)", "impl": "reference",
-            "config": {"workload": args.workload, "B": p.B, "H": p.H, "T": p.T, "dk": p.dk, "dv": p.dv,
-                       "chunk": p.chunk},
+            "config": workload_config(args.workload, p),
             "cpu_baseline": {"value": round(value, 6), "unit": "Mtokens/s", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "Mtokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -290,7 +290,10 @@ GDR_API gdr_status gdr_query_device_status(gdr_stream_t stream);
  *     dk = dv = 128; B*H must not exceed GDR_NOALLOC_MAX_HEADS, else GDR_ERR_UNSUPPORTED with
  *     a message (nothing launched).  Other arguments as for gdr_chunk_fwd.
  *   - The first call on each device looks up the scratch array's device address
- *     (cudaGetSymbolAddress) and caches it; make that first call before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current) and caches it with the context's id;
+ *     a context destroyed and created again (cudaDeviceReset) is seen by its new id and the
+ *     address is looked up again.  Make the first call in each context before any stream
+ *     capture.
  *   - Every call shares the one scratch array, which keeps the last call's contents; each
  *     call clears the flags it needs on its own stream first.  Calls that overlap on the
  *     GPU (other streams, other host threads) race on the array and must be serialised by

@@ -124,10 +124,48 @@ constexpr size_t NOALLOC_BYTES =
     tcf::split_flag_words(NOALLOC_MAX_HEADS) * sizeof(unsigned int);
 static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_BYTES];
 
-// In host code g_noalloc_scratch names a host-side stand-in, not device memory; the device
-// address is looked up once per device (with that device current) and cached here.
+// The current context's unique id (the driver's cuCtxGetId), so that per-device caches can
+// tell a context that was destroyed and created again (cudaDeviceReset, a released primary
+// context) from the one they were filled in: module globals and streams of the old context are
+// gone with it.  The driver calls are looked up through the runtime so that the library does
+// not link libcuda itself.  *id is 0 when no context is current on this thread.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+static gdr_status current_ctx_id(unsigned long long* id) {
+    static std::mutex mu;
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!get_current || !get_id) {
+            void* p1 = nullptr;
+            void* p2 = nullptr;
+            cudaDriverEntryPointQueryResult q1 = cudaDriverEntryPointSymbolNotFound, q2 = q1;
+            cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &p1, cudaEnableDefault, &q1);
+            if (e == cudaSuccess) e = cudaGetDriverEntryPoint("cuCtxGetId", &p2, cudaEnableDefault, &q2);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetDriverEntryPoint(cuCtxGetCurrent / cuCtxGetId)");
+            if (q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !p1 || !p2)
+                return fail(GDR_ERR_CUDA, "the driver has no cuCtxGetCurrent / cuCtxGetId%s");
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p1);
+            get_id = reinterpret_cast<CtxGetIdFn>(p2);
+        }
+    }
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return fail(GDR_ERR_CUDA, "cuCtxGetCurrent failed%s");
+    *id = 0;
+    if (ctx && get_id(ctx, id) != CUDA_SUCCESS) return fail(GDR_ERR_CUDA, "cuCtxGetId failed%s");
+    return GDR_OK;
+}
+
+// In host code g_noalloc_scratch names a host-side stand-in, not device memory.  Its device
+// address is looked up with the device current (cudaGetSymbolAddress), once per device and
+// context, and cached; a context that has been destroyed and created again is seen by its new
+// id, and the address is looked up again.  The first call on a device (or in a new context)
+// does the lookup, so it should come before any stream capture.
 constexpr int NOALLOC_MAX_DEVICES = 64;
 static void* s_noalloc_ptr[NOALLOC_MAX_DEVICES] = {};
+static unsigned long long s_noalloc_ctx[NOALLOC_MAX_DEVICES] = {};
 static std::mutex s_noalloc_mu;
 
 static gdr_status noalloc_scratch(void** out) {
@@ -135,12 +173,18 @@ static gdr_status noalloc_scratch(void** out) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return fail(GDR_ERR_UNSUPPORTED, "device index too large%s");
+    unsigned long long ctx = 0;
+    gdr_status s = current_ctx_id(&ctx);
+    if (s != GDR_OK) return s;
     std::lock_guard<std::mutex> lock(s_noalloc_mu);
-    if (!s_noalloc_ptr[dev]) {
+    if (!s_noalloc_ptr[dev] || ctx == 0 || s_noalloc_ctx[dev] != ctx) {
         void* ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
         if (e != cudaSuccess || ptr == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+        // the lookup makes the device's primary context current if none was
+        if (ctx == 0 && (s = current_ctx_id(&ctx)) != GDR_OK) return s;
         s_noalloc_ptr[dev] = ptr;
+        s_noalloc_ctx[dev] = ctx;
     }
     *out = s_noalloc_ptr[dev];
     return GDR_OK;
@@ -321,6 +365,7 @@ struct HostPipe {
     cudaEvent_t start = nullptr;
     cudaEvent_t loaded[2] = {}, computed[2] = {}, stored[2] = {};
     bool ready = false;
+    unsigned long long ctx = 0;     // the context they were created in
 };
 static HostPipe s_pipe[HOST_MAX_DEVICES];
 static std::mutex s_pipe_mu;     // held while a call enqueues: the events are shared
@@ -331,6 +376,12 @@ static gdr_status host_pipe(HostPipe** out) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= HOST_MAX_DEVICES) return fail(GDR_ERR_UNSUPPORTED, "device index out of range%s");
     HostPipe& P = s_pipe[dev];
+    unsigned long long ctx = 0;
+    gdr_status s = current_ctx_id(&ctx);
+    if (s != GDR_OK) return s;
+    // Streams and events of a context that has since been destroyed are gone with it (and
+    // cannot be destroyed again); a new context gets new ones.
+    if (P.ready && ctx != 0 && P.ctx != ctx) P = HostPipe();
     if (!P.ready) {
         if ((e = cudaStreamCreateWithFlags(&P.h2d, cudaStreamNonBlocking)) != cudaSuccess ||
             (e = cudaStreamCreateWithFlags(&P.d2h, cudaStreamNonBlocking)) != cudaSuccess ||
@@ -342,6 +393,8 @@ static gdr_status host_pipe(HostPipe** out) {
                 (e = cudaEventCreateWithFlags(&P.stored[i], cudaEventDisableTiming)) != cudaSuccess)
                 return cuda_fail(e, "host pipeline events");
         }
+        if (ctx == 0 && (s = current_ctx_id(&ctx)) != GDR_OK) return s;
+        P.ctx = ctx;
         P.ready = true;
     }
     *out = &P;
@@ -420,7 +473,12 @@ size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc) {
     if (check_fwd_desc(desc) != GDR_OK) return 0;
     const gdr_algo a = resolve_algo(desc);
     if (a == GDR_ALGO_TCGEN05_SPLIT) return split_workspace_bytes(desc);
-    if (a == GDR_ALGO_TCGEN05_WAVES) return split_workspace_heads((size_t)waves_remainder(desc, device_sm_count()));
+    if (a == GDR_ALGO_TCGEN05_WAVES) {
+        // only a last partial wave that the split kernel runs needs the ring
+        const int sms = device_sm_count();
+        const long long rem = waves_remainder(desc, sms);
+        return (rem > 0 && split_fits_heads(rem, sms, desc->T)) ? split_workspace_heads((size_t)rem) : 0;
+    }
     return 0;
 }
 

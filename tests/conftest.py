@@ -26,3 +26,23 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """The achieved parity errors of the GPU tests (worst per test), beside the tolerances
+    they are held to: max-rel of o <= 1e-4 (fp32 mode) / 2e-2 (bf16), rel-L2 of S_T <= 1e-2."""
+    try:
+        import parity_util as U
+    except Exception:
+        return
+    if not U.MARGINS:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "achieved parity errors (worst per test)")
+    for test in sorted(U.MARGINS):
+        ent = U.MARGINS[test]
+        cols = "  ".join(f"{k}={v:.3e}" for k, v in sorted(ent.items()))
+        tr.write_line(f"{cols}  {test}")
+    path = os.environ.get("GDR_PARITY_LOG")
+    if path:
+        U.write_margins(path)

@@ -72,3 +72,6 @@ def test_reference_arm_prints_one_contract_line(capsys):
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "Mtokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == bench.WORKLOAD
+    # the GPU arm builds its config object with the same function from the same workload
+    from recurrent_state_memory_b200 import inputs as I
+    assert d["config"] == bench.workload_config(bench.WORKLOAD, I.make_config(bench.WORKLOAD))

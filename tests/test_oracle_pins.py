@@ -470,6 +470,52 @@ def test_l2norm_prologue_keeps_zero_vectors_zero_and_decode_agrees():
     assert _rel(S, S_f) < 1e-12
 
 
+def _l2norm_epsilon_pin_holds(normalise):
+    """The stated convention puts the 1e-6 inside the square root: for x = c u with a unit u,
+    the result is u c / sqrt(c^2 + 1e-6).  Choosing c^2 as a multiple of 1e-6 makes that
+    norm a known number: c^2 = 3e-6 gives sqrt(3)/2, c^2 = 1e-6 gives 1/sqrt(2), c^2 = 8e-6
+    gives sqrt(8)/3.  The direction of x is kept."""
+    rng = np.random.default_rng(91)
+    for mult, norm in ((3.0, np.sqrt(3.0) / 2.0), (1.0, 1.0 / np.sqrt(2.0)), (8.0, np.sqrt(8.0) / 3.0)):
+        u = rng.normal(size=(4, 16))
+        u /= np.linalg.norm(u, axis=-1, keepdims=True)
+        y = np.asarray(normalise(u * np.sqrt(mult * 1e-6)), dtype=np.float64)
+        if not np.allclose(np.linalg.norm(y, axis=-1), norm, rtol=1e-9, atol=0):
+            return False
+        if not np.allclose(y / np.linalg.norm(y, axis=-1, keepdims=True), u, rtol=1e-9, atol=1e-12):
+            return False
+    return True
+
+
+def test_l2norm_epsilon_sits_inside_the_root_with_value_1e_6():
+    assert _l2norm_epsilon_pin_holds(oracle.l2_normalise)
+
+
+def test_l2norm_epsilon_pin_catches_planted_mistakes():
+    planted = {
+        "epsilon outside the root": lambda x: x / (np.sqrt(np.sum(x * x, -1, keepdims=True)) + 1e-6),
+        "epsilon 1e-12": lambda x: x / np.sqrt(np.sum(x * x, -1, keepdims=True) + 1e-12),
+        "no epsilon": lambda x: x / np.sqrt(np.sum(x * x, -1, keepdims=True)),
+    }
+    for name, f in planted.items():
+        assert not _l2norm_epsilon_pin_holds(f), name
+
+
+def test_l2norm_epsilon_reaches_the_forward():
+    """One token from the zero state, q = k = c u with c^2 = 3e-6: S_1 = beta v khat^T and
+    o_1 = beta v (khat . qhat) = beta v c^2 / (c^2 + 1e-6) = 0.75 beta v, whatever the gate."""
+    rng = np.random.default_rng(92)
+    H, d = 3, 8
+    u = rng.normal(size=(1, 1, H, d))
+    u /= np.linalg.norm(u, axis=-1, keepdims=True)
+    q = k = u * np.sqrt(3e-6)
+    v = rng.normal(size=(1, 1, H, 5))
+    a = rng.normal(size=(1, 1, H, d))
+    beta = rng.uniform(0.2, 0.9, size=(1, 1, H))
+    o, _ = oracle.gdr_fwd(q, k, v, a, beta, None, None, oracle.GATE_NEG_SOFTPLUS, qk_l2norm=True)
+    assert np.allclose(o, 0.75 * beta[..., None] * v, rtol=1e-10, atol=0)
+
+
 # ---- chunk means of the output (the content signal of CARVE's content-aware erase) -------
 
 @pytest.mark.parametrize("T,chunk", [(150, 64), (64, 64), (37, 16), (1, 64)])

@@ -25,11 +25,11 @@ def G():
     return gdr
 
 
-def _call_noalloc(G, p, t, out_dtype):
+def _call_noalloc(G, p, t, out_dtype, qk_l2norm=False):
     import torch
     dev = t["q"].device
     desc = G.fwd_desc(p.B, p.H, p.T, p.dk, p.dv, t["q"].dtype, out_dtype, p.gate_mode, p.rotation,
-                      p.scale, "auto")
+                      p.scale, "auto", qk_l2norm=qk_l2norm)
     o = torch.empty((p.B, p.T, p.H, p.dv), dtype=out_dtype, device=dev)
     S_T = torch.empty((p.B, p.H, p.dv, p.dk), dtype=torch.float32, device=dev)
     st = G.lib().gdr_chunk_fwd_noalloc(ctypes.byref(desc), G._ptr(t["q"]), G._ptr(t["k"]), G._ptr(t["v"]),
@@ -39,22 +39,42 @@ def _call_noalloc(G, p, t, out_dtype):
     return o, S_T
 
 
-def test_noalloc_matches_workspace_entry_on_consecutive_calls(G):
+# Consecutive calls through the one shared scratch array: a 6-head call, the largest call the
+# array holds (32 heads), then smaller calls after it (4 heads with the fused L2
+# normalisation, 10 heads with a single chunk), so that flags left behind by a larger call
+# meet a later, smaller one; then a call with no tokens at all (S_T = S0).
+CASES = [dict(B=2, T=333, H=3, seed=71, rotation=True, s0_std=0.2, out="bf16"),
+         dict(B=4, T=200, H=8, seed=72, rotation=False, s0_std=None, out="f32"),
+         dict(B=1, T=150, H=4, seed=73, rotation=False, s0_std=0.1, out="bf16", l2=True),
+         dict(B=2, T=64, H=5, seed=74, rotation=True, s0_std=None, out="bf16"),
+         dict(B=3, T=0, H=2, seed=75, rotation=False, s0_std=0.3, out="f32")]
+
+
+def test_noalloc_matches_oracle_and_workspace_entry_on_consecutive_calls(G):
     import torch
-    cases = [dict(B=2, T=333, H=3, seed=71, rotation=True, s0_std=0.2, out=torch.bfloat16),
-             dict(B=4, T=200, H=8, seed=72, rotation=False, s0_std=None, out=torch.float32)]
-    for cs in cases:                     # two calls in a row, through the shared scratch
+    import oracle
+    for cs in CASES:
+        out = torch.bfloat16 if cs["out"] == "bf16" else torch.float32
+        l2 = cs.get("l2", False)
         p = I.make_fwd(cs["B"], cs["T"], cs["H"], 128, 128, dtype="bf16", seed=cs["seed"],
                        rotation=cs["rotation"], s0_std=cs["s0_std"])
         t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "g", "beta", "theta", "S0")}
-        o_ref, S_ref = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["theta"], t["S0"],
-                                   gate_mode=p.gate_mode, algo="tcgen05_split", out_dtype=cs["out"])
-        o, S = _call_noalloc(G, p, t, cs["out"])
+        o, S = _call_noalloc(G, p, t, out, qk_l2norm=l2)
         torch.cuda.synchronize()
         assert G.query_device_status() == G.GDR_OK
-        assert U.max_rel(U.o_to_f64(o), U.o_to_f64(o_ref)) <= U.TOL_O["bf16"]
-        assert U.rel_l2(S.cpu().numpy(), S_ref.cpu().numpy()) <= U.TOL_S
-        assert torch.equal(o, o_ref) and torch.equal(S, S_ref)      # the same kernel and inputs
+        o_ref, S_ref = oracle.gdr_fwd(p.widened("q"), p.widened("k"), p.widened("v"), p.widened("g"),
+                                      p.widened("beta"), p.widened("theta"), p.widened("S0"),
+                                      gate_mode=p.gate_mode, scale=p.scale, qk_l2norm=l2)
+        if p.T == 0:
+            assert torch.equal(S, t["S0"])                 # no tokens: the state passes through
+        else:
+            U.assert_fwd_parity(p, o, S, o_ref, S_ref)
+        # the workspace entry with the same (split) kernel gives the same bytes
+        if p.T > 0:
+            o_w, S_w = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["theta"], t["S0"],
+                                   gate_mode=p.gate_mode, algo="tcgen05_split", out_dtype=out, qk_l2norm=l2)
+            torch.cuda.synchronize()
+            assert torch.equal(o, o_w) and torch.equal(S, S_w)
 
 
 def test_noalloc_rejects_more_heads_than_its_scratch_holds(G):
