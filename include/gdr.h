@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define GDR_ABI_VERSION 3
+#define GDR_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define GDR_API __attribute__((visibility("default")))
@@ -71,21 +71,28 @@ typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
 typedef enum { GDR_GATE_LOGDECAY = 0, GDR_GATE_NEG_SOFTPLUS = 1 } gdr_gate_mode;
 
 typedef enum {
-    GDR_ALGO_AUTO = 0,    /* tensor-core chunk kernel when supported (the split one when
-                             2*B*H <= SM count and T > 64, the waves mix when B*H exceeds the SM
-                             count and its remainder would take the split kernel), else SIMT */
+    GDR_ALGO_AUTO = 0,    /* the split tensor-core kernel for bf16 q/k/v, dk = dv = 128 and
+                             T > 64 (any number of heads), in its sequence-parallel form
+                             (GDR_ALGO_TCGEN05_SEGMENTS) when a few heads have long sequences,
+                             so that one chain per head would be the bound; the fused kernel for
+                             a single chunk; the CUDA-core kernel for every other shape and for
+                             fp32 mode */
     GDR_ALGO_SIMT = 1,    /* fp32 CUDA-core chunk-WY kernel (every supported shape) */
     GDR_ALGO_TCGEN05 = 2, /* tcgen05/TMEM chunk-WY kernel, one CTA per (batch, head):
                              bf16 q/k/v, dk = dv = 128 */
-    GDR_ALGO_TCGEN05_SPLIT = 3 /* same method; one CTA per head runs only the state chain
-                             while every other SM prepares chunks (two at a time), handed
-                             over through a ring in the workspace (needs B*H < SM count;
-                             cooperative launch); results agree with GDR_ALGO_TCGEN05 to
+    GDR_ALGO_TCGEN05_SPLIT = 3 /* same method on a cooperative grid of one CTA per SM:
+                             nc CTAs run the state chains (heads in waves of nc, one after
+                             another), every other SM prepares chunks, handed over through a
+                             ring in the workspace; results agree with GDR_ALGO_TCGEN05 to
                              rounding */,
-    GDR_ALGO_TCGEN05_WAVES = 4 /* more heads than SMs: the fused kernel for whole waves of
-                             SM-count heads, then the split kernel for the last partial wave
-                             when it is at most half the SM count (else fused throughout);
-                             workspace for the split part */
+    GDR_ALGO_TCGEN05_WAVES = 4 /* the fused kernel for whole waves of SM-count heads, then the
+                             split kernel for the heads of a last partial wave (workspace for
+                             that part) */,
+    GDR_ALGO_TCGEN05_SEGMENTS = 5 /* sequence-parallel: each head's sequence is cut into
+                             desc->segments segments (0: chosen by the library) that run as
+                             separate chains, from the zero state and from the identity; an
+                             affine scan over the segments and an output correction combine
+                             them (see gdr_chunk_fwd) */
 } gdr_algo;
 
 /* Shape and mode of one chunked forward call. */
@@ -101,6 +108,8 @@ typedef struct {
     gdr_algo algo;
     int qk_l2norm;        /* 1: the kernels L2-normalise q_t and k_t per token and head first,
                              x / sqrt(sum x^2 + 1e-6) in fp32, before the scale (0: as given) */
+    int segments;         /* GDR_ALGO_TCGEN05_SEGMENTS: number of segments per sequence (>= 2; 0
+                             lets the library choose); ignored by the other algorithms */
 } gdr_fwd_desc;
 
 /* Shape and mode of one decode step over N independent sequences. */
@@ -126,10 +135,11 @@ GDR_API const char* gdr_last_error_detail(void);
 
 /* Bytes of device workspace gdr_chunk_fwd needs for this descriptor (0 = none;
  * the workspace argument may then be NULL).  Returns 0 for an invalid desc.  The split
- * tensor-core kernel needs B*H*8 ring slots of 76,288 bytes plus 36 bytes of flags per
- * head and one 4-byte task counter; it resets the flags itself (on the call's stream) and the buffer may be reused
- * by later calls on the same stream.  Uses the current device's SM count when
- * desc->algo is GDR_ALGO_AUTO. */
+ * tensor-core kernel needs, for each of its nc state chains (1 <= nc <= min(B*H, SMs / 2),
+ * chosen from B*H, T and the SM count), a ring of 8 slots of 91,136 bytes plus 36 bytes of
+ * flags, and one 4-byte task counter; it resets the flags itself (on the call's stream) and
+ * the buffer may be reused by later calls on the same stream.  Uses the current device's
+ * SM count. */
 GDR_API size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc);
 
 /*
@@ -152,7 +162,18 @@ GDR_API size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc);
  *
  * Numerical range: the kernels factor exp(Gamma_r - Gamma_i) through per-chunk
  * reference points; a key dim whose log-decay over 32 consecutive tokens is
- * below -80 may overflow the factored form (GDR_ALGO_TCGEN05 only).
+ * below -80 may overflow the factored form (tensor-core kernels; reported as
+ * GDR_ERR_RANGE by gdr_query_device_status).
+ *
+ * GDR_ALGO_TCGEN05_SEGMENTS (sequence parallelism; "Semidirect Fourier Delta Attention"
+ * page, "Main contributions": the exact affine transfer S_end = S_start A + B): each
+ * sequence is cut into segments of a whole number of chunks (the last one may be shorter).
+ * Every segment runs from the zero state (segment 0 from S0), giving o0 and its end state
+ * B, and segments 1.. also from the identity with zero values, giving y_t = A q_t and the
+ * transition A; a scan over the segments forms their true start states St (fp32) and S_T,
+ * and o_t = o0_t + St y_t (tf32 products) for t in segments 1..  The workspace
+ * (gdr_chunk_fwd_workspace_bytes) then also holds the per-segment states and y (4 bytes per
+ * token, head and key dim) and must be 256-byte aligned.
  */
 GDR_API gdr_status gdr_chunk_fwd(const gdr_fwd_desc* desc,
                          const void* q, const void* k, const void* v,
@@ -283,9 +304,9 @@ GDR_API gdr_status gdr_query_device_status(gdr_stream_t stream);
  *
  * It runs the split tensor-core kernel (same arithmetic and results as
  * gdr_chunk_fwd with GDR_ALGO_TCGEN05_SPLIT) with the kernel's hand-off ring in a scratch
- * array compiled into the library: GDR_NOALLOC_MAX_HEADS * 8 slots of 76,288 bytes plus
- * flags (about 18.6 MiB), which every GPU that loads the library holds until the process
- * exits.
+ * array compiled into the library: at most GDR_NOALLOC_MAX_HEADS rings of 8 slots of 91,136
+ * bytes plus flags (about 22.3 MiB), which every GPU that loads the library holds until the
+ * process exits.
  *   - desc->algo must be GDR_ALGO_AUTO or GDR_ALGO_TCGEN05_SPLIT; q, k, v must be bf16 with
  *     dk = dv = 128; B*H must not exceed GDR_NOALLOC_MAX_HEADS, else GDR_ERR_UNSUPPORTED with
  *     a message (nothing launched).  Other arguments as for gdr_chunk_fwd.

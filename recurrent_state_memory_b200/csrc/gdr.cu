@@ -11,6 +11,8 @@
 #include "simt_fwd.cuh"
 #include "decode.cuh"
 #include "tc_fwd.cuh"
+#include "split_fwd.cuh"
+#include "seg_combine.cuh"
 
 namespace gdr {
 
@@ -79,49 +81,70 @@ static int device_sm_count() {
     return n;
 }
 
-// The split kernel gives each head one chain CTA and shares the remaining SMs among prep
-// workers; with more than half of the SMs taken by chains, too few workers are left and the
-// fused kernel (prep and chain of a head in one CTA) is faster.
-static bool split_fits_heads(long long nh, int sms, int T) { return nh >= 1 && 2 * nh <= (long long)sms && T > 64; }
+// The split kernel runs the state chains on `nc` SMs and prepares chunks on the others; with
+// more heads than chains, each chain runs its heads one after another (waves of nc heads).
+// nc balances the two sides with a cost model measured on B200: a chain needs about
+// CHAIN_CYCLES per chunk, a worker SM about WORKER_CYCLES per chunk of one head.
+constexpr double CHAIN_CYCLES = 1500.0, WORKER_CYCLES = 2600.0;
+static double split_cost(long long nv, long long nchunks, int nc, int sms) {
+    const long long waves = (nv + nc - 1) / nc;
+    const double t_chain = (double)waves * nchunks * CHAIN_CYCLES;
+    const double t_work = (double)nv * nchunks * WORKER_CYCLES / (double)(sms - nc);
+    return t_chain > t_work ? t_chain : t_work;
+}
+static int plan_chains(long long nv, long long nchunks, int sms) {
+    if (nv <= 0 || nchunks <= 0) return 1;
+    int best = 1;
+    double best_t = 1e300;
+    const int max_nc = (int)(nv < sms / 2 ? nv : sms / 2);
+    for (int nc = 1; nc <= max_nc; ++nc) {
+        const double t = split_cost(nv, nchunks, nc, sms);
+        if (t < best_t * 0.999) { best_t = t; best = nc; }
+    }
+    return best;
+}
+// Virtual heads (chains) and chunks per virtual head of one split-kernel launch.
+static void split_geometry(const FwdParams& p, long long* nv, long long* nchunks) {
+    const long long ns = p.nseg > 1 ? p.nseg - p.seg0 : 1;
+    *nv = (long long)p.nheads * ns;
+    *nchunks = p.nseg > 1 ? p.seg_len / 64 : (p.T + 63) / 64;
+}
+static bool split_fits_heads(long long nh, int sms, int T) { return nh >= 1 && sms >= 2 && T > 64; }
 static bool split_fits(const gdr_fwd_desc* d, int sms) {
     return split_fits_heads((long long)d->B * d->H, sms, d->T);
 }
-// More heads than SMs: the fused kernel runs whole waves of SM-count heads; a last partial
-// wave that would leave more than half of the SMs idle goes to the split kernel instead.
+// GDR_ALGO_TCGEN05_WAVES: the fused kernel for whole waves of SM-count heads and the split
+// kernel for the heads of a last partial wave.
 static long long waves_remainder(const gdr_fwd_desc* d, int sms) {
     const long long nh = (long long)d->B * d->H;
     return nh > sms ? nh % sms : 0;
 }
-static bool waves_fit(const gdr_fwd_desc* d, int sms) {
-    const long long rem = waves_remainder(d, sms);
-    return rem > 0 && split_fits_heads(rem, sms, d->T);
-}
 
-// The algorithm a descriptor runs with: AUTO takes a tensor-core kernel when it supports
-// the shape and dtype, the split one when the heads leave room for prep workers, the waves
-// mix when a partial last wave would leave most SMs idle.
+static bool segments_pay(long long nh, long long T, int sms);
+
+// The algorithm a descriptor runs with: AUTO takes the split tensor-core kernel when it
+// supports the shape and dtype and the sequence has more than one chunk, the fused one for a
+// single chunk, the CUDA-core kernel otherwise.
 static gdr_algo resolve_algo(const gdr_fwd_desc* d) {
     if (d->algo == GDR_ALGO_AUTO) {
         if (!tc_supported(d)) return GDR_ALGO_SIMT;
         const int sms = device_sm_count();
-        if (split_fits(d, sms)) return GDR_ALGO_TCGEN05_SPLIT;
-        return waves_fit(d, sms) ? GDR_ALGO_TCGEN05_WAVES : GDR_ALGO_TCGEN05;
+        if (!split_fits(d, sms)) return GDR_ALGO_TCGEN05;
+        return segments_pay((long long)d->B * d->H, d->T, sms) ? GDR_ALGO_TCGEN05_SEGMENTS : GDR_ALGO_TCGEN05_SPLIT;
     }
     return d->algo;
 }
 
-static size_t split_workspace_heads(size_t nh) {
-    return nh * tcf::RING * tcf::SLOT_BYTES + tcf::split_flag_words(nh) * sizeof(unsigned int);
+static size_t split_workspace_heads(size_t nh, int T) {
+    return spl::workspace_bytes((size_t)plan_chains((long long)nh, (T + 63) / 64, device_sm_count()));
 }
-static size_t split_workspace_bytes(const gdr_fwd_desc* d) { return split_workspace_heads((size_t)d->B * d->H); }
+static size_t split_workspace_bytes(const gdr_fwd_desc* d) { return split_workspace_heads((size_t)d->B * d->H, d->T); }
 
 // ---- scratch for gdr_chunk_fwd_noalloc ---------------------------------------------------
 // The split kernel's ring and flags for at most NOALLOC_MAX_HEADS heads, as a file-scope
 // device array: every GPU that loads this library holds these bytes until the process exits.
 constexpr int NOALLOC_MAX_HEADS = GDR_NOALLOC_MAX_HEADS;
-constexpr size_t NOALLOC_BYTES =
-    (size_t)NOALLOC_MAX_HEADS * tcf::RING * tcf::SLOT_BYTES +
-    tcf::split_flag_words(NOALLOC_MAX_HEADS) * sizeof(unsigned int);
+constexpr size_t NOALLOC_BYTES = spl::workspace_bytes(NOALLOC_MAX_HEADS);
 static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_BYTES];
 
 // The current context's unique id (the driver's cuCtxGetId), so that per-device caches can
@@ -202,10 +225,13 @@ static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
     if (d->rotation != 0 && d->rotation != 1) return fail(GDR_ERR_INVALID_ARG, "rotation must be 0 or 1%s");
     if (d->qk_l2norm != 0 && d->qk_l2norm != 1) return fail(GDR_ERR_INVALID_ARG, "qk_l2norm must be 0 or 1%s");
     if (d->algo != GDR_ALGO_AUTO && d->algo != GDR_ALGO_SIMT && d->algo != GDR_ALGO_TCGEN05 &&
-        d->algo != GDR_ALGO_TCGEN05_SPLIT && d->algo != GDR_ALGO_TCGEN05_WAVES)
+        d->algo != GDR_ALGO_TCGEN05_SPLIT && d->algo != GDR_ALGO_TCGEN05_WAVES && d->algo != GDR_ALGO_TCGEN05_SEGMENTS)
         return fail(GDR_ERR_INVALID_ARG, "bad algo%s");
+    if (d->segments < 0 || d->segments == 1 || d->segments > 4096)
+        return fail(GDR_ERR_INVALID_ARG, "segments must be 0 (library's choice) or 2 .. 4096%s");
     if ((long long)d->B * d->H > 0x7fffffffLL) return fail(GDR_ERR_INVALID_ARG, "B*H too large%s");
-    if ((d->algo == GDR_ALGO_TCGEN05 || d->algo == GDR_ALGO_TCGEN05_SPLIT || d->algo == GDR_ALGO_TCGEN05_WAVES) &&
+    if ((d->algo == GDR_ALGO_TCGEN05 || d->algo == GDR_ALGO_TCGEN05_SPLIT || d->algo == GDR_ALGO_TCGEN05_WAVES ||
+         d->algo == GDR_ALGO_TCGEN05_SEGMENTS) &&
         !tc_supported(d))
         return fail(GDR_ERR_UNSUPPORTED, "the tcgen05 kernels need bf16 q/k/v and dk = dv = 128%s");
     return GDR_OK;
@@ -255,27 +281,26 @@ static gdr_status encode_bthd(EncodeTiledFn fn, CUtensorMap* m, const void* base
     return GDR_OK;
 }
 
-template <bool ROT, typename OT>
-static gdr_status encode_split_maps(const FwdParams& p, tcf::TmaMaps* tm) {
+template <bool ROT>
+static gdr_status encode_split_maps(const FwdParams& p, spl::Maps* tm) {
     EncodeTiledFn fn = nullptr;
     gdr_status s = encode_fn(&fn);
     if (s != GDR_OK) return s;
     const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    const int D = tcf::D, NG = ROT ? tcf::D / 2 : tcf::D;
+    const int D = spl::D, NG = ROT ? spl::D / 2 : spl::D;
     if ((s = encode_bthd(fn, &tm->q, p.q, bf, 2, p, D, D, false)) != GDR_OK) return s;
     if ((s = encode_bthd(fn, &tm->k, p.k, bf, 2, p, D, D, false)) != GDR_OK) return s;
     if ((s = encode_bthd(fn, &tm->g, p.g, f32, 4, p, NG, NG, false)) != GDR_OK) return s;
     if (ROT && (s = encode_bthd(fn, &tm->th, p.theta, f32, 4, p, NG, NG, false)) != GDR_OK) return s;
-    if ((s = encode_bthd(fn, &tm->v, p.v, bf, 2, p, D, 64, true)) != GDR_OK) return s;
-    const bool ob = sizeof(OT) == 2;
-    return encode_bthd(fn, &tm->o, p.o, ob ? bf : f32, sizeof(OT), p, D, D, false);
+    if (p.v && (s = encode_bthd(fn, &tm->v, p.v, bf, 2, p, D, 64, true)) != GDR_OK) return s;   // NULL: zero values
+    return GDR_OK;
 }
 
-template <int MODE, bool ROT, typename OT, bool EXT>
-static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
-    auto kern = tcf::chunk_fwd_tc_kernel<MODE, ROT, OT, EXT>;
-    constexpr int nt = tcf::nthreads<MODE>();
-    constexpr uint32_t smem = tcf::smem_bytes<MODE>();
+template <bool ROT, typename OT, bool EXT>
+static gdr_status launch_tc(const FwdParams& p, cudaStream_t st) {
+    auto kern = tcf::chunk_fwd_tc_kernel<0, ROT, OT, EXT>;
+    constexpr int nt = tcf::nthreads<0>();
+    constexpr uint32_t smem = tcf::smem_bytes<0>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tcgen05 chunk kernel)");
     tcf::TcExtra x;
@@ -284,51 +309,188 @@ static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
     tcf::SplitArgs sa{nullptr, nullptr, nullptr};
     tcf::TmaMaps tm;
     memset(&tm, 0, sizeof(tm));
-    if (MODE == 0) {
-        kern<<<p.nheads, nt, smem, st>>>(p, x, sa, tm);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
-        return GDR_OK;
-    }
-    // Split: the whole grid must be resident at once (one CTA per SM), which a cooperative
-    // launch guarantees or refuses.
-    const int nh = p.nheads;
-    const int sms = device_sm_count();
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-    const int grid = sms * (per_sm < 1 ? 1 : per_sm > 1 ? 1 : per_sm);
-    if (per_sm < 1 || grid <= nh) return fail(GDR_ERR_UNSUPPORTED, "split kernel: B*H must be below the SM count%s");
-    gdr_status s = encode_split_maps<ROT, OT>(p, &tm);
-    if (s != GDR_OK) return s;
-    const size_t nring = (size_t)nh * tcf::RING * tcf::SLOT_BYTES;
-    sa.ring = static_cast<uint8_t*>(ws);
-    sa.ready = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + nring);
-    sa.consumed = sa.ready + (size_t)nh * tcf::RING;
-    sa.next_task = sa.consumed + nh;
-    // Worker order: from the counter while the worker groups fill at most half the ring's
-    // slots (the workers are then the bound and the counter evens out their load); at a
-    // fixed stride otherwise (measured faster there: it paces each group to the chains).
-    sa.dynamic = (2 * (grid - nh) <= nh * tcf::RING / 2) ? 1 : 0;
-    e = cudaMemsetAsync(sa.ready, 0, tcf::split_flag_words(nh) * sizeof(unsigned int), st);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split flags)");
-    void* args[] = {const_cast<FwdParams*>(&p), &x, &sa, &tm};
-    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(nt), args, smem, st);
-    if (e != cudaSuccess) return cuda_fail(e, "cooperative launch(tcgen05 split kernel)");
+    kern<<<p.nheads, nt, smem, st>>>(p, x, sa, tm);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
     return GDR_OK;
 }
 
-template <int MODE>
-static gdr_status dispatch_tc_mode(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws) {
+template <bool ROT, typename OT, bool EXT>
+static gdr_status launch_split(const FwdParams& p, cudaStream_t st, void* ws) {
+    auto kern = spl::split_fwd_kernel<ROT, OT, EXT>;
+    constexpr uint32_t smem = spl::SMEM_BYTES;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(split chunk kernel)");
+    // The whole grid must be resident at once (one CTA per SM), which a cooperative launch
+    // guarantees or refuses.
+    long long nv = 0, nchunks = 0;
+    split_geometry(p, &nv, &nchunks);
+    const int sms = device_sm_count();
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, spl::NT, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (per_sm < 1) return fail(GDR_ERR_UNSUPPORTED, "split kernel: does not fit on an SM%s");
+    const int grid = sms;
+    const int nc = plan_chains(nv, nchunks, sms);
+    if (nc < 1 || nc >= grid) return fail(GDR_ERR_UNSUPPORTED, "split kernel: no SM left for prep workers%s");
+    spl::Maps tm;
+    memset(&tm, 0, sizeof(tm));
+    gdr_status s = encode_split_maps<ROT>(p, &tm);
+    if (s != GDR_OK) return s;
+    spl::Cfg cf;
+    cf.ring = static_cast<uint8_t*>(ws);
+    cf.ready = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + (size_t)nc * spl::RING * spl::SLOT_BYTES);
+    cf.consumed = cf.ready + (size_t)nc * spl::RING;
+    cf.next_task = cf.consumed + nc;
+    cf.nc = nc;
+    // Task order: from the counter while the prep workers are the bound (few chains, so a worker
+    // that ran fast takes the next task); at a fixed stride otherwise, which paces each worker
+    // to the chains.
+    const long long waves = (nv + nc - 1) / nc;
+    const double t_chain = (double)waves * nchunks * CHAIN_CYCLES;
+    const double t_work = (double)nv * nchunks * WORKER_CYCLES / (double)(grid - nc);
+    cf.dynamic = t_work >= t_chain ? 1 : 0;
+    cf.wait_limit_ns = s_wait_limit_ns;
+    cf.fault_skip_commit = s_fault_skip_commit;
+    e = cudaMemsetAsync(cf.ready, 0, spl::flag_words((size_t)nc) * sizeof(unsigned int), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split flags)");
+    void* args[] = {const_cast<FwdParams*>(&p), &cf, &tm};
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(spl::NT), args, smem, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cooperative launch(split chunk kernel)");
+    return GDR_OK;
+}
+
+// The kernel instantiation with the optional features (a separate write strength, the fused L2
+// normalisation, the chunk means of o) runs only when one of them is asked for.
+static gdr_status dispatch_fused(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st) {
     const bool ob = d->out_dtype == GDR_BF16;
-    if (p.w || p.qk_norm || p.chunk_mean) {      // the kernel with the optional features
-        if (d->rotation)
-            return ob ? launch_tc<MODE, true, __nv_bfloat16, true>(p, st, ws) : launch_tc<MODE, true, float, true>(p, st, ws);
-        return ob ? launch_tc<MODE, false, __nv_bfloat16, true>(p, st, ws) : launch_tc<MODE, false, float, true>(p, st, ws);
+    if (p.w || p.qk_norm || p.chunk_mean) {
+        if (d->rotation) return ob ? launch_tc<true, __nv_bfloat16, true>(p, st) : launch_tc<true, float, true>(p, st);
+        return ob ? launch_tc<false, __nv_bfloat16, true>(p, st) : launch_tc<false, float, true>(p, st);
     }
-    if (d->rotation)
-        return ob ? launch_tc<MODE, true, __nv_bfloat16, false>(p, st, ws) : launch_tc<MODE, true, float, false>(p, st, ws);
-    return ob ? launch_tc<MODE, false, __nv_bfloat16, false>(p, st, ws) : launch_tc<MODE, false, float, false>(p, st, ws);
+    if (d->rotation) return ob ? launch_tc<true, __nv_bfloat16, false>(p, st) : launch_tc<true, float, false>(p, st);
+    return ob ? launch_tc<false, __nv_bfloat16, false>(p, st) : launch_tc<false, float, false>(p, st);
+}
+
+static gdr_status dispatch_split(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws,
+                                 bool f32_out = false) {
+    const bool ob = d->out_dtype == GDR_BF16 && !f32_out;
+    if (p.w || p.qk_norm || p.chunk_mean) {
+        if (d->rotation) return ob ? launch_split<true, __nv_bfloat16, true>(p, st, ws) : launch_split<true, float, true>(p, st, ws);
+        return ob ? launch_split<false, __nv_bfloat16, true>(p, st, ws) : launch_split<false, float, true>(p, st, ws);
+    }
+    if (d->rotation) return ob ? launch_split<true, __nv_bfloat16, false>(p, st, ws) : launch_split<true, float, false>(p, st, ws);
+    return ob ? launch_split<false, __nv_bfloat16, false>(p, st, ws) : launch_split<false, float, false>(p, st, ws);
+}
+
+// ---- sequence-parallel forward (segments) ---------------------------------------------------
+// Each head's sequence is cut into nseg segments of seg_len tokens (a multiple of 64; the last
+// one may be shorter).  Pass 1 runs every segment from the zero state (segment 0 from S0): o0
+// into o, chunk means of o0, end states Bz.  Pass 2 runs segments 1.. from the identity with
+// zero values: y_t = A_{start->t} q_t (fp32) and the transitions A.  The scan kernel forms the
+// start states St of segments 1.. and S_T; the correction kernel adds St y to o (and to the
+// chunk means).
+struct SegPlan {
+    int nseg = 1, seg_len = 0;
+    size_t off_bz = 0, off_a = 0, off_st = 0, off_y = 0, total = 0;
+};
+constexpr double HBM_BYTES_PER_CYCLE = 3300.0;   // about 6.5 TB/s at 1.965 GHz
+static double seg_cost(long long nh, long long T, int nseg, int sms) {
+    const long long seg_len = ((T + nseg - 1) / nseg + 63) / 64 * 64;
+    const long long ns = (T + seg_len - 1) / seg_len, sc = seg_len / 64;
+    double t = split_cost(nh * ns, sc, plan_chains(nh * ns, sc, sms), sms);
+    if (ns > 1) {
+        t += split_cost(nh * (ns - 1), sc, plan_chains(nh * (ns - 1), sc, sms), sms);
+        t += (double)(ns - 1) * 3000.0;                                                // scan steps
+        t += (double)nh * T * (ns - 1) / ns * 1024.0 / HBM_BYTES_PER_CYCLE;           // y, o traffic
+    }
+    return t;
+}
+static int choose_segments(long long nh, long long T, int sms) {
+    double best = 1e300;
+    int bn = 2;
+    for (int n = 2; n <= 64; n *= 2) {
+        if (T < 128LL * n) break;
+        const double t = seg_cost(nh, T, n, sms);
+        if (t < best) { best = t; bn = n; }
+    }
+    return bn;
+}
+// AUTO takes the segments when the model puts them well ahead of one chain per head.
+static bool segments_pay(long long nh, long long T, int sms) {
+    if (T < 256) return false;
+    const long long nchunks = (T + 63) / 64;
+    const double t_plain = split_cost(nh, nchunks, plan_chains(nh, nchunks, sms), sms);
+    return seg_cost(nh, T, choose_segments(nh, T, sms), sms) < 0.75 * t_plain;
+}
+static size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+static void seg_plan(const gdr_fwd_desc* d, int sms, SegPlan* P) {
+    const long long nh = (long long)d->B * d->H, T = d->T;
+    const int want = d->segments > 0 ? d->segments : choose_segments(nh, T, sms);
+    const long long seg_len = ((T + want - 1) / want + 63) / 64 * 64;
+    const long long ns = seg_len > 0 ? (T + seg_len - 1) / seg_len : 1, sc = seg_len / 64;
+    P->nseg = (int)ns;
+    P->seg_len = (int)seg_len;
+    int nc = plan_chains(nh * ns, sc, sms);
+    if (ns > 1) {
+        const int nc2 = plan_chains(nh * (ns - 1), sc, sms);
+        if (nc2 > nc) nc = nc2;
+    }
+    const size_t DD4 = (size_t)spl::D * spl::D * 4;
+    size_t o = round256(spl::workspace_bytes((size_t)nc));
+    P->off_bz = o;  o += round256((size_t)nh * ns * DD4);
+    P->off_a = o;   o += round256((size_t)nh * (ns - 1) * DD4);
+    P->off_st = o;  o += round256((size_t)nh * (ns - 1) * DD4);
+    P->off_y = o;   o += round256(ns > 1 ? (size_t)d->B * T * d->H * spl::D * 4 : 0);
+    P->total = o;
+}
+
+template <typename OT>
+static gdr_status launch_correct(const seg::CorrParams& cp, const CUtensorMap& ymap, int nblocks, cudaStream_t st) {
+    auto kern = seg::seg_correct_kernel<OT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)seg::CORR_SMEM);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(segment correction kernel)");
+    kern<<<nblocks, seg::CORR_NT, seg::CORR_SMEM, st>>>(cp, ymap, s_wait_limit_ns);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launch(segment correction kernel)");
+    return GDR_OK;
+}
+
+static gdr_status run_segments(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws) {
+    SegPlan P;
+    seg_plan(d, device_sm_count(), &P);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    FwdParams p1 = p;
+    if (P.nseg <= 1) return dispatch_split(d, p1, st, ws);
+    float* Bz = reinterpret_cast<float*>(w + P.off_bz);
+    float* A = reinterpret_cast<float*>(w + P.off_a);
+    float* St = reinterpret_cast<float*>(w + P.off_st);
+    float* y = reinterpret_cast<float*>(w + P.off_y);
+    p1.nseg = P.nseg; p1.seg_len = P.seg_len; p1.seg0 = 0; p1.s0_identity = 0;
+    p1.S_T = Bz;
+    gdr_status s = dispatch_split(d, p1, st, w);                   // o0, chunk means of o0, Bz
+    if (s != GDR_OK) return s;
+    FwdParams p2 = p1;
+    p2.seg0 = 1; p2.s0_identity = 1;
+    p2.v = nullptr; p2.w = nullptr; p2.S0 = nullptr; p2.chunk_mean = nullptr;
+    p2.o = y; p2.S_T = A;
+    s = dispatch_split(d, p2, st, w, true);                        // y (fp32), A
+    if (s != GDR_OK) return s;
+    seg::ScanParams sp{p.nheads, P.nseg, Bz, A, St, p.S_T};
+    cudaError_t e = cudaFuncSetAttribute(seg::seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)seg::SCAN_SMEM);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(segment scan kernel)");
+    seg::seg_scan_kernel<<<dim3(p.nheads, seg::D / seg::RB), seg::SCAN_NT, seg::SCAN_SMEM, st>>>(sp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch(segment scan kernel)");
+    EncodeTiledFn fn = nullptr;
+    if ((s = encode_fn(&fn)) != GDR_OK) return s;
+    CUtensorMap ymap;
+    memset(&ymap, 0, sizeof(ymap));
+    if ((s = encode_bthd(fn, &ymap, y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p, spl::D, 32, true)) != GDR_OK) return s;
+    seg::CorrParams cp{p.B, p.H, p.T, P.nseg, P.seg_len, p.head0, St, p.o, p.chunk_mean};
+    const int nblocks = p.nheads * (P.nseg - 1) * (P.seg_len / seg::TOK);
+    return d->out_dtype == GDR_BF16 ? launch_correct<__nv_bfloat16>(cp, ymap, nblocks, st)
+                                    : launch_correct<float>(cp, ymap, nblocks, st);
 }
 
 // ----------------------------------------------------------------- decode ----
@@ -410,7 +572,6 @@ struct HostPlan {
     size_t ring_bytes;        // split-kernel workspace at the start, rounded to 256
     int bs, nslices;          // batch entries per slice, number of slices
 };
-static size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 static void host_plan(const gdr_fwd_desc* d, bool w, bool S0, bool S_T, bool cm, HostPlan* P) {
     const size_t T = (size_t)d->T, H = (size_t)d->H, dk = (size_t)d->dk, dv = (size_t)d->dv;
@@ -473,11 +634,17 @@ size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc) {
     if (check_fwd_desc(desc) != GDR_OK) return 0;
     const gdr_algo a = resolve_algo(desc);
     if (a == GDR_ALGO_TCGEN05_SPLIT) return split_workspace_bytes(desc);
+    if (a == GDR_ALGO_TCGEN05_SEGMENTS) {
+        if (desc->T <= 0) return 0;
+        SegPlan P;
+        seg_plan(desc, device_sm_count(), &P);
+        return P.total;
+    }
     if (a == GDR_ALGO_TCGEN05_WAVES) {
         // only a last partial wave that the split kernel runs needs the ring
         const int sms = device_sm_count();
         const long long rem = waves_remainder(desc, sms);
-        return (rem > 0 && split_fits_heads(rem, sms, desc->T)) ? split_workspace_heads((size_t)rem) : 0;
+        return (rem > 0 && split_fits_heads(rem, sms, desc->T)) ? split_workspace_heads((size_t)rem, desc->T) : 0;
     }
     return 0;
 }
@@ -527,12 +694,18 @@ gdr_status gdr_chunk_fwd_ex(const gdr_fwd_desc* d, const void* q, const void* k,
     p.scale = d->scale;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.theta = theta;
     p.S0 = S0; p.o = o; p.S_T = S_T; p.chunk_mean = chunk_mean;
+    p.nseg = 1; p.seg_len = 0; p.seg0 = 0; p.s0_identity = 0;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (d->T == 0 && !S_T) return GDR_OK;
     const gdr_algo algo = resolve_algo(d);
     if (algo == GDR_ALGO_TCGEN05_SPLIT && d->T > 0) {
         if (!aligned16(workspace)) return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned%s");
-        return dispatch_tc_mode<1>(d, p, st, workspace);
+        return dispatch_split(d, p, st, workspace);
+    }
+    if (algo == GDR_ALGO_TCGEN05_SEGMENTS && d->T > 0) {
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+            return fail(GDR_ERR_INVALID_ARG, "workspace must be 256-byte aligned for GDR_ALGO_TCGEN05_SEGMENTS%s");
+        return run_segments(d, p, st, workspace);
     }
     if (algo == GDR_ALGO_TCGEN05_WAVES && d->T > 0) {
         const long long rem = waves_remainder(d, device_sm_count());
@@ -542,14 +715,15 @@ gdr_status gdr_chunk_fwd_ex(const gdr_fwd_desc* d, const void* q, const void* k,
             pf.nheads = (int)(p.nheads - rem);
             ps.head0 = pf.nheads;
             ps.nheads = (int)rem;
-            s = dispatch_tc_mode<0>(d, pf, st, nullptr);           // whole waves, fused
+            s = dispatch_fused(d, pf, st);                    // whole waves, fused
             if (s != GDR_OK) return s;
-            return dispatch_tc_mode<1>(d, ps, st, workspace);      // the last partial wave, split
+            return dispatch_split(d, ps, st, workspace);      // the last partial wave, split
         }
-        return dispatch_tc_mode<0>(d, p, st, nullptr);
+        return dispatch_fused(d, p, st);
     }
-    if (algo == GDR_ALGO_TCGEN05 || algo == GDR_ALGO_TCGEN05_SPLIT || algo == GDR_ALGO_TCGEN05_WAVES)
-        return dispatch_tc_mode<0>(d, p, st, nullptr);
+    if (algo == GDR_ALGO_TCGEN05 || algo == GDR_ALGO_TCGEN05_SPLIT || algo == GDR_ALGO_TCGEN05_WAVES ||
+        algo == GDR_ALGO_TCGEN05_SEGMENTS)
+        return dispatch_fused(d, p, st);
     return d->rotation ? dispatch_simt_dk<true>(d, p, st) : dispatch_simt_dk<false>(d, p, st);
 }
 
@@ -656,12 +830,13 @@ gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* d, const void* q, const voi
     p.scale = d->scale;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = nullptr; p.theta = theta;
     p.S0 = S0; p.o = o; p.S_T = S_T; p.chunk_mean = nullptr;
+    p.nseg = 1; p.seg_len = 0; p.seg0 = 0; p.s0_identity = 0;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (d->T == 0) return S_T ? dispatch_tc_mode<0>(d, p, st, nullptr) : GDR_OK;
+    if (d->T == 0) return S_T ? dispatch_fused(d, p, st) : GDR_OK;
     void* scratch = nullptr;
     s = noalloc_scratch(&scratch);
     if (s != GDR_OK) return s;
-    return dispatch_tc_mode<1>(d, p, st, scratch);
+    return dispatch_split(d, p, st, scratch);
 }
 
 size_t gdr_chunk_fwd_host_workspace_bytes(const gdr_fwd_desc* d, int with_w, int with_S0, int with_S_T,
@@ -763,6 +938,17 @@ gdr_status gdr_chunk_fwd_host(const gdr_fwd_desc* d, const void* q, const void* 
         return bail(cuda_fail(e, "cudaStreamWaitEvent"));
     return GDR_OK;
 }
+
+#ifdef GDR_TIMELINE
+// Profiling builds only: copy the split kernel's event timeline to host memory (see split_fwd.cuh).
+GDR_API int gdr_debug_timeline(unsigned long long* host, size_t n) {
+    return cudaMemcpyFromSymbol(host, g_timeline, n * sizeof(unsigned long long)) == cudaSuccess ? 0 : -1;
+}
+GDR_API int gdr_debug_timeline_clear(void) {
+    static unsigned long long zero[148 * TL_ITERS * TL_EVENTS];
+    return cudaMemcpyToSymbol(g_timeline, zero, sizeof(zero)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 void gdr_debug_set_tc_fault(int skip_first_commit, unsigned long long wait_limit_ns) {
     s_fault_skip_commit = skip_first_commit ? 1 : 0;

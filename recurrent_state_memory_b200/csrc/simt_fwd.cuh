@@ -41,6 +41,12 @@ struct FwdParams {
     void* o;
     float* S_T;
     float* chunk_mean;      // [B, ceil(T/64), H, dv] fp32 mean of o over each chunk, or nullptr
+    // Split tensor-core kernel only: with nseg > 1 each head's sequence runs as segments of
+    // seg_len tokens (a multiple of 64), segments seg0 .. nseg-1, each as its own chain (a
+    // "virtual head"): segment 0 starts from S0 (or zero), the others from zero, or every one
+    // from the identity when s0_identity is set (dk = dv); S_T then holds one state per virtual
+    // head.  v == nullptr means zero values.
+    int nseg, seg_len, seg0, s0_identity;
 };
 
 namespace simt {

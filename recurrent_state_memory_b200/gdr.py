@@ -24,7 +24,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gdr.h")
  GDR_ERR_RANGE) = range(7)
 GDR_F32, GDR_BF16 = 0, 1
 GATE_LOGDECAY, GATE_NEG_SOFTPLUS = 0, 1
-ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_split": 3, "tcgen05_waves": 4}
+ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_split": 3, "tcgen05_waves": 4, "tcgen05_segments": 5}
 ALGO_NAMES = {v: k for k, v in ALGOS.items()}
 
 
@@ -33,7 +33,8 @@ class FwdDesc(ctypes.Structure):
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("chunk", ctypes.c_int),
                 ("qkv_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
                 ("gate_mode", ctypes.c_int), ("rotation", ctypes.c_int),
-                ("scale", ctypes.c_float), ("algo", ctypes.c_int), ("qk_l2norm", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("algo", ctypes.c_int), ("qk_l2norm", ctypes.c_int),
+                ("segments", ctypes.c_int)]
 
 
 class DecDesc(ctypes.Structure):
@@ -89,7 +90,7 @@ def lib() -> ctypes.CDLL:
         L.gdr_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp, vp]
         L.gdr_debug_set_tc_fault.restype = None
         L.gdr_debug_set_tc_fault.argtypes = [ctypes.c_int, ctypes.c_ulonglong]
-        if L.gdr_abi_version() != 3:
+        if L.gdr_abi_version() != 4:
             raise RuntimeError("libgdr.so ABI version mismatch")
         _lib = L
     return _lib
@@ -137,9 +138,10 @@ def _need(t: torch.Tensor, name: str, dtype=None, device=None):
 
 
 def fwd_desc(B, H, T, dk, dv, qkv_dtype, out_dtype, gate_mode=GATE_NEG_SOFTPLUS, rotation=False,
-             scale=1.0, algo="auto", chunk=64, qk_l2norm=False) -> FwdDesc:
+             scale=1.0, algo="auto", chunk=64, qk_l2norm=False, segments=0) -> FwdDesc:
     return FwdDesc(B, H, T, dk, dv, chunk, _dtype_code(qkv_dtype), _dtype_code(out_dtype),
-                   int(gate_mode), int(bool(rotation)), float(scale), ALGOS[algo], int(bool(qk_l2norm)))
+                   int(gate_mode), int(bool(rotation)), float(scale), ALGOS[algo], int(bool(qk_l2norm)),
+                   int(segments))
 
 
 def resolved_algo(desc: FwdDesc) -> str:
@@ -168,9 +170,12 @@ def host_workspace_bytes(desc: FwdDesc, w=False, S0=False, S_T=False, chunk_mean
 def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
               algo="auto", out_dtype=None, want_state=True, o=None, S_T=None, workspace=None,
               stream=None, chunk=64, w=None, qk_l2norm=False, want_chunk_mean=False,
-              chunk_mean=None):
+              chunk_mean=None, segments=0):
     """Chunk-parallel forward.  Returns (o, S_T), or (o, S_T, chunk_mean) when
     want_chunk_mean is set or a chunk_mean tensor is passed.
+
+    algo "tcgen05_segments" cuts each sequence into `segments` pieces that run as separate
+    chains and are combined exactly (0: the library chooses the number).
 
     beta is the erase strength; w [B,T,H] (fp32) a separate write strength, or None for
     the tied rule (w = beta).  chunk_mean [B, ceil(T/64), H, dv] (fp32) receives the mean
@@ -224,7 +229,8 @@ def chunk_fwd(q, k, v, g, beta, theta=None, S0=None, *, gate_mode=GATE_NEG_SOFTP
         _need(chunk_mean, "chunk_mean", torch.float32, dev)
         if tuple(chunk_mean.shape) != (B, nc, H, dv):
             raise ValueError("chunk_mean has the wrong shape")
-    desc = fwd_desc(B, H, T, dk, dv, q.dtype, out_dtype, gate_mode, rotation, scale, algo, chunk, qk_l2norm)
+    desc = fwd_desc(B, H, T, dk, dv, q.dtype, out_dtype, gate_mode, rotation, scale, algo, chunk, qk_l2norm,
+                    segments)
     out = (o, S_T, chunk_mean) if with_mean else (o, S_T)
     if host:
         cdev = torch.device("cuda", torch.cuda.current_device())
