@@ -298,18 +298,15 @@ static gdr_status encode_split_maps(const FwdParams& p, spl::Maps* tm) {
 
 template <bool ROT, typename OT, bool EXT>
 static gdr_status launch_tc(const FwdParams& p, cudaStream_t st) {
-    auto kern = tcf::chunk_fwd_tc_kernel<0, ROT, OT, EXT>;
-    constexpr int nt = tcf::nthreads<0>();
-    constexpr uint32_t smem = tcf::smem_bytes<0>();
+    auto kern = tcf::chunk_fwd_tc_kernel<ROT, OT, EXT>;
+    constexpr int nt = tcf::NT;
+    constexpr uint32_t smem = tcf::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tcgen05 chunk kernel)");
     tcf::TcExtra x;
     x.wait_limit_ns = s_wait_limit_ns;
     x.fault_skip_commit = s_fault_skip_commit;
-    tcf::SplitArgs sa{nullptr, nullptr, nullptr};
-    tcf::TmaMaps tm;
-    memset(&tm, 0, sizeof(tm));
-    kern<<<p.nheads, nt, smem, st>>>(p, x, sa, tm);
+    kern<<<p.nheads, nt, smem, st>>>(p, x);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
     return GDR_OK;

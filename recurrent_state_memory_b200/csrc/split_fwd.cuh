@@ -658,10 +658,12 @@ __device__ __forceinline__ void worker_producer(const FwdParams& p, const Cfg& c
         return min(t, total);
     };
     int staged = 0;
+    bool gave_up = false;
     int t = claim();
     for (int i = 0;; ++i) {
         if (i >= 1 && !mbar_wait_bounded(b_infree, (uint32_t)((i - 1) & 1), lim)) {
             atomicExch(abort_f, 1);
+            gave_up = true;
             break;
         }
         tk_ring[i & 3] = t;
@@ -680,12 +682,13 @@ __device__ __forceinline__ void worker_producer(const FwdParams& p, const Cfg& c
         ++staged;
         t = claim();                    // the next claim overlaps these copies
     }
-    // copies still in flight land before the CTA ends
-    if (staged > 0) (void)mbar_wait_bounded(b_in, (uint32_t)((staged - 1) & 1), lim);
+    // After giving up, copies still in flight land before the CTA ends.  (Otherwise the
+    // elementwise group has waited for every one of them.)
+    if (gave_up && staged > 0) (void)mbar_wait_bounded(b_in, (uint32_t)((staged - 1) & 1), lim);
 }
 
-// Publisher (one thread): once the solve group has staged a task's tiles, copies Qtil, Pm, Wm^T
-// and Tw (Tb) into the task's ring slot with bulk copies, waits until they are written, and
+// Publisher (one thread): once the solve group has staged a task's tiles, copies Pm, Wm2^T and
+// Tw (Tb) into the task's ring slot with bulk copies, waits until they are written, and
 // publishes the slot with a release store (the elementwise group's stores to the slot happened
 // before, through the task's barriers).
 template <bool EXT>
