@@ -7,9 +7,12 @@ A step is one chunked forward pass over the whole workload: B=4, H=16, T=4096,
 dk=dv=128, chunk 64, bf16 q/k/v, fp32 gates (seeded synthetic inputs, resident in
 HBM).  The inputs (408 MB) are larger than the 126 MB L2, so no flush is needed
 between steps.  Decode (256 sequences x 16 heads, fp32 state) is measured in the
-same run and reported in the "decode" object.  Under torchrun every rank runs its
-own independent batch (weak scaling, no data-path collective); the time is the
-max over ranks.  Rank 0 prints one JSON line.
+same run and reported in the "decode" object, and the two other forward
+workloads (B=16, H=12, T=4096 with slow decay and a random initial state; the
+block-rotation variant at B=2, H=16, T=8192) each get an object of their own in
+"workloads", timed the same way with their own roofline and clock record.  Under
+torchrun every rank runs its own independent batch (weak scaling, no data-path
+collective); the time is the max over ranks.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -30,6 +33,9 @@ if ROOT not in sys.path:
 
 METRIC = "gated delta-rule fwd Mtokens/s and % roofline at H=16,dk=dv=128; decode GB/s"
 WORKLOAD = "b4_h16_t4096_d128"
+# every forward workload of the benchmark: the headline one, the 1.3B-layer training shape with
+# slow decay and a random initial state, the block-rotation variant
+FWD_WORKLOADS = ("b4_h16_t4096_d128", "b16_h12_t4096_d128_slow_s0", "b2_h16_t8192_d128_rot")
 L2_BYTES = 126e6
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -81,8 +87,9 @@ def load_peaks():
 KERNEL_SOURCES = {
     "gdr_chunk_fwd_simt": ["simt_fwd.cuh", "common.cuh"],
     "gdr_chunk_fwd_tcgen05": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
-    "gdr_chunk_fwd_tcgen05_split": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
-    "gdr_chunk_fwd_tcgen05_waves": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
+    "gdr_chunk_fwd_tcgen05_split": ["split_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
+    "gdr_chunk_fwd_tcgen05_waves": ["tc_fwd.cuh", "split_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
+    "gdr_chunk_fwd_tcgen05_segments": ["split_fwd.cuh", "seg_combine.cuh", "tc_ptx.cuh", "common.cuh"],
     "gdr_decode_step": ["decode.cuh", "common.cuh"],
 }
 
@@ -185,30 +192,29 @@ def workload_config(name, p):
             "l2": f"inputs {p.nbytes_algorithmic / 1e6:.0f} MB vs L2 {L2_BYTES / 1e6:.0f} MB; no flush"}
 
 
-def run_ours(args):
+def _to_torch(a):
+    import torch
+    if a is None:
+        return None
+    return torch.from_numpy(a.copy()).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+
+
+def time_fwd(name, args, dev, stream, rank, ws, steps):
+    """One forward workload: seeded inputs resident in HBM, W untimed warm-up launches, then
+    `steps` launches timed with CUDA events on the launching stream (barrier + synchronize on
+    both sides, max over ranks), with the SM clocks sampled meanwhile."""
     import torch
     import torch.distributed as dist
     from recurrent_state_memory_b200 import gdr
     from recurrent_state_memory_b200 import inputs as I
 
-    ws, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if ws > 1:
-        import datetime
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
-
-    gdr.lib()
-    cfg = dict(I.FWD_CONFIGS[args.workload])
+    cfg = dict(I.FWD_CONFIGS[name])
     cfg["seed"] = rank_seed(cfg["seed"], rank)
-    p = I.make_fwd(name=args.workload, **cfg)
-    to = lambda a: None if a is None else (
-        torch.from_numpy(a.copy()).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a))
-    host = {k: to(getattr(p, k)) for k in ("q", "k", "v", "g", "beta", "theta", "S0")}
+    p = I.make_fwd(name=name, **cfg)
+    host = {k: _to_torch(getattr(p, k)) for k in ("q", "k", "v", "g", "beta", "theta", "S0")}
     dv_t = {k: (None if t is None else t.to(dev)) for k, t in host.items()}
     o = torch.empty((p.B, p.T, p.H, p.dv), dtype=dv_t["q"].dtype, device=dev)
     S_T = torch.empty((p.B, p.H, p.dv, p.dk), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
     desc = gdr.fwd_desc(p.B, p.H, p.T, p.dk, p.dv, dv_t["q"].dtype, o.dtype, p.gate_mode, p.rotation,
                         p.scale, args.algo)
     ws_bytes = gdr.workspace_bytes(desc)
@@ -225,12 +231,11 @@ def run_ours(args):
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
-
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     t_all0, t_all1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index) as clk:
         t_all0.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             evs[i][0].record(stream)
             step()
             evs[i][1].record(stream)
@@ -240,10 +245,9 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     per_launch_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = t_all0.elapsed_time(t_all1)
-    total_ms_max = max_over_ranks(total_ms, dev)
+    total_ms_max = max_over_ranks(t_all0.elapsed_time(t_all1), dev)
     tokens = p.B * p.T
-    tokens_all = sum_over_ranks(float(tokens * args.steps), dev)
+    tokens_all = sum_over_ranks(float(tokens * steps), dev)
     value = tokens_all / (total_ms_max * 1e-3) / 1e6
 
     peaks, peak_src = load_peaks()
@@ -254,11 +258,48 @@ def run_ours(args):
     kernel_name = "gdr_chunk_fwd_" + resolved
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
-                "traffic": stored_traffic(kernel_name, args.workload),
+                "traffic": stored_traffic(kernel_name, name),
                 "peak_source": f"{peak_src} HBM copy bandwidth",
                 "algorithmic_bytes_per_launch": algo_bytes, "kernel": kernel_name}
     flops = fwd_flops_per_token_head(p.dk, p.dv) * tokens * p.H
-    tflops = flops / avg_launch_s / 1e12
+    return {"p": p, "host": host, "dv_t": dv_t, "o": o, "S_T": S_T, "wsp": wsp, "desc": desc,
+            "resolved": resolved, "kernel_name": kernel_name, "value": value, "total_ms_max": total_ms_max,
+            "tokens": tokens, "peaks": peaks, "roofline": roofline, "tflops": flops / avg_launch_s / 1e12,
+            "launches": gdr.kernel_launches(desc) * steps, "clocks": clk.summary(), "steps": steps}
+
+
+def workload_summary(name, r):
+    """The object a secondary forward workload gets in the JSON line."""
+    return {"value": round(r["value"], 3), "unit": "Mtokens/s", "ms_per_step": round(r["total_ms_max"] / r["steps"], 4),
+            "steps": r["steps"], "config": workload_config(name, r["p"]), "algo": r["resolved"],
+            "tflops_algorithmic": round(r["tflops"], 2), "roofline": r["roofline"], "gpu_launches": r["launches"],
+            "clocks": r["clocks"]}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from recurrent_state_memory_b200 import gdr
+    from recurrent_state_memory_b200 import inputs as I
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    gdr.lib()
+    stream = torch.cuda.current_stream(dev)
+    main = time_fwd(args.workload, args, dev, stream, rank, ws, args.steps)
+    p, host, dv_t, o, S_T, wsp = main["p"], main["host"], main["dv_t"], main["o"], main["S_T"], main["wsp"]
+    cfg = dict(I.FWD_CONFIGS[args.workload])
+    cfg["seed"] = rank_seed(cfg["seed"], rank)
+    to = _to_torch
+    value, total_ms_max, tokens = main["value"], main["total_ms_max"], main["tokens"]
+    peaks, roofline, tflops = main["peaks"], main["roofline"], main["tflops"]
+    resolved, kernel_name = main["resolved"], main["kernel_name"]
+    algo_bytes = p.nbytes_algorithmic
 
     # ---- end to end through the public API with pinned host buffers ----
     e2e = None
@@ -376,6 +417,18 @@ def run_ours(args):
                                "traffic": stored_traffic("gdr_decode_step", "decode_n256_h16_d128"),
                                "kernel": "gdr_decode_step"}}
 
+    # ---- the other forward workloads, each timed the same way on its own inputs ----
+    workloads = None
+    if not args.no_workloads:
+        workloads = {}
+        for name in FWD_WORKLOADS:
+            if name == args.workload:
+                continue
+            r = time_fwd(name, args, dev, stream, rank, ws, min(args.steps, 10))
+            workloads[name] = workload_summary(name, r)
+            del r
+            torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
         cpu = cpu_baseline(p, args.cpu_seconds)
@@ -396,13 +449,14 @@ def run_ours(args):
         "tflops_algorithmic": round(tflops, 2),
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": args.steps * (2 if resolved == "tcgen05_waves" else 1),
+        "gpu_launches": main["launches"],
         "decode": decode,
         "untied": untied,
         "qk_l2norm": l2norm,
         "chunk_mean": cmean,
         "cpu_baseline": cpu,
-        "clocks": clk.summary(),
+        "clocks": main["clocks"],
+        "workloads": workloads,
     }
     print(json.dumps(line), flush=True)
 
@@ -481,12 +535,14 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
-    ap.add_argument("--algo", choices=["auto", "simt", "tcgen05", "tcgen05_split", "tcgen05_waves"], default="auto")
+    ap.add_argument("--algo", choices=["auto", "simt", "tcgen05", "tcgen05_split", "tcgen05_waves",
+                                       "tcgen05_segments"], default="auto")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the other forward workloads")
     ap.add_argument("--no-untied", action="store_true", help="skip the separate-write-strength, "
                     "fused-L2-norm and chunk-mean measurements")
     args = ap.parse_args(argv)

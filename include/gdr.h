@@ -331,6 +331,15 @@ GDR_API gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* desc,
  * descriptor is invalid.  No GPU work. */
 GDR_API int gdr_chunk_fwd_algo(const gdr_fwd_desc* desc);
 
+/* The number of kernels one forward call with this descriptor launches on the stream
+ * (the zeroing of the split kernel's flags by cudaMemsetAsync not counted): 1 for the
+ * SIMT, fused and split kernels, 2 for TCGEN05_WAVES with a partial last wave, 4 for
+ * TCGEN05_SEGMENTS with more than one segment (two split passes, the scan and the
+ * correction), 0 when B or H is 0; a call with T = 0 counts 1 (it writes S_T).  -1 if
+ * the descriptor is invalid.  No GPU work (the segment plan reads the device's SM
+ * count). */
+GDR_API int gdr_chunk_fwd_kernel_launches(const gdr_fwd_desc* desc);
+
 /*
  * Test hook for the bounded waits of the tensor-core kernel (process-wide, not
  * thread-safe).  wait_limit_ns bounds every mbarrier wait (0 restores the 2 s

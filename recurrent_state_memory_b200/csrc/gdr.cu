@@ -793,6 +793,24 @@ int gdr_chunk_fwd_algo(const gdr_fwd_desc* desc) {
     return (int)resolve_algo(desc);
 }
 
+int gdr_chunk_fwd_kernel_launches(const gdr_fwd_desc* d) {
+    if (check_fwd_desc(d) != GDR_OK) return -1;
+    if (d->B == 0 || d->H == 0) return 0;
+    const gdr_algo a = resolve_algo(d);
+    if (d->T == 0) return 1;
+    if (a == GDR_ALGO_TCGEN05_SEGMENTS) {
+        SegPlan P;
+        seg_plan(d, device_sm_count(), &P);
+        return P.nseg <= 1 ? 1 : 4;         // two split passes, the scan, the correction
+    }
+    if (a == GDR_ALGO_TCGEN05_WAVES) {
+        const int sms = device_sm_count();
+        const long long rem = waves_remainder(d, sms);
+        return (rem > 0 && split_fits_heads(rem, sms, d->T)) ? 2 : 1;
+    }
+    return 1;
+}
+
 gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* d, const void* q, const void* k, const void* v,
                                  const float* g, const float* beta, const float* theta, const float* S0,
                                  void* o, float* S_T, gdr_stream_t stream) {

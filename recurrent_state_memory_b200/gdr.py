@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_query_device_status.argtypes = [vp]
         L.gdr_chunk_fwd_algo.restype = ctypes.c_int
         L.gdr_chunk_fwd_algo.argtypes = [ctypes.POINTER(FwdDesc)]
+        L.gdr_chunk_fwd_kernel_launches.restype = ctypes.c_int
+        L.gdr_chunk_fwd_kernel_launches.argtypes = [ctypes.POINTER(FwdDesc)]
         L.gdr_chunk_fwd_noalloc.restype = ctypes.c_int
         L.gdr_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp, vp]
         L.gdr_debug_set_tc_fault.restype = None
@@ -150,6 +152,14 @@ def resolved_algo(desc: FwdDesc) -> str:
     if a < 0:
         raise ValueError("invalid descriptor")
     return ALGO_NAMES[a]
+
+
+def kernel_launches(desc: FwdDesc) -> int:
+    """How many kernels one forward call with this descriptor launches."""
+    n = int(lib().gdr_chunk_fwd_kernel_launches(ctypes.byref(desc)))
+    if n < 0:
+        raise ValueError("invalid descriptor")
+    return n
 
 
 def debug_set_tc_fault(skip_first_commit: bool, wait_limit_ns: int = 0):

@@ -185,3 +185,22 @@ def test_qk_l2norm_flag_is_checked(G):
     assert _call_fwd(G, d, FAKE) == G.GDR_ERR_INVALID_ARG
     d.qk_l2norm = 1
     assert G.lib().gdr_chunk_fwd_workspace_bytes(ctypes.byref(d)) == 0     # SIMT shape here
+
+
+def test_kernel_launch_count_without_a_device(G):
+    """The number of kernels a forward call launches: one for the SIMT, fused and split kernels,
+    four for the sequence-parallel form with several segments (two split passes, the scan and
+    the correction), none for an empty batch."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("the 148-SM assumption holds only where no device is visible")
+    bf = torch.bfloat16
+    d = lambda B, H, T, dk=128, **kw: G.fwd_desc(B, H, T, dk, dk, bf, bf, **kw)
+    assert G.kernel_launches(d(4, 16, 4096)) == 1                      # split
+    assert G.kernel_launches(d(4, 16, 64)) == 1                        # fused, one chunk
+    assert G.kernel_launches(d(4, 16, 4096, dk=64)) == 1               # SIMT
+    assert G.kernel_launches(d(1, 1, 4096)) == 4                       # segments
+    assert G.kernel_launches(d(1, 1, 64, algo="tcgen05_segments", segments=2)) == 1   # one segment
+    assert G.kernel_launches(d(0, 16, 4096)) == 0
+    with pytest.raises(ValueError):
+        G.kernel_launches(G.fwd_desc(1, 1, 64, 48, 48, bf, bf))
