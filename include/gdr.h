@@ -341,6 +341,46 @@ GDR_API int gdr_chunk_fwd_algo(const gdr_fwd_desc* desc);
 GDR_API int gdr_chunk_fwd_kernel_launches(const gdr_fwd_desc* desc);
 
 /*
+ * Backward pass of gdr_chunk_fwd: the gradients of a loss L with respect to every input, given
+ * dO = dL/do and dS_T = dL/dS_T (the training use that the "CARVE" page, section 4, measures).
+ * It follows the chain rule through the chunk-WY algebra ("CARVE" page, section 1 item 3;
+ * "Semidirect Fourier Delta Attention" page, "Constructive Chunk-WY Theorem"): one CTA per
+ * (batch, head) keeps each chunk's start state from a forward sweep, then runs the chunks in
+ * reverse, the gradient of each chunk's end state flowing into the one before.  fp32 throughout
+ * (tensor-core products with split-tf32 operands).
+ *
+ *   desc            as for gdr_chunk_fwd; dk = dv (32, 64 or 128), rotation = 0, qk_l2norm = 0
+ *                   (else GDR_ERR_UNSUPPORTED); algo and segments are ignored.  dO has the
+ *                   dtype desc->out_dtype; q, k, v desc->qkv_dtype.
+ *   q, k, v, g, beta, w, S0   the forward's inputs, layouts as in gdr_chunk_fwd (w may be NULL:
+ *                   w = beta; S0 may be NULL: zero).
+ *   dO [B,T,H,dv]   gradient of o, or NULL (zero).
+ *   dS_T [B,H,dv,dk] fp32 gradient of the final state, or NULL (zero).
+ *   dq, dk [B,T,H,dk], dv [B,T,H,dv], dg [B,T,H,dk] (of the gate input as given: g itself with
+ *                   GDR_GATE_LOGDECAY, the raw gate a with GDR_GATE_NEG_SOFTPLUS), dbeta [B,T,H]:
+ *                   fp32 outputs, required when T > 0.
+ *   dw [B,T,H]      fp32, required exactly when w is given (then dbeta is the erase strength's
+ *                   gradient alone).
+ *   dS0 [B,H,dv,dk] fp32 gradient of S0, or NULL (not written).
+ *   workspace       device memory of gdr_chunk_bwd_workspace_bytes(desc) bytes, 16-byte aligned
+ *                   (the chunk start states and each head's chunk matrices; about
+ *                   (1 MB + 64 KB per chunk) per head at d = 128).
+ * All pointers are device pointers, 16-byte aligned, owned by the caller; the call is
+ * asynchronous on `stream` and allocates nothing.  With T = 0, dS0 = dS_T.  Errors: argument
+ * checks return before any launch; a decay too strong for the factored form over half a chunk
+ * (a factor above 3e38) sets the device status word's range bit (gdr_query_device_status ->
+ * GDR_ERR_RANGE).
+ */
+GDR_API size_t gdr_chunk_bwd_workspace_bytes(const gdr_fwd_desc* desc);
+GDR_API gdr_status gdr_chunk_bwd(const gdr_fwd_desc* desc,
+                                 const void* q, const void* k, const void* v,
+                                 const float* g, const float* beta, const float* w,
+                                 const float* S0, const void* dO, const float* dS_T,
+                                 float* dq, float* dk, float* dv, float* dg, float* dbeta,
+                                 float* dw, float* dS0,
+                                 void* workspace, size_t workspace_bytes, gdr_stream_t stream);
+
+/*
  * Test hook for the bounded waits of the tensor-core kernel (process-wide, not
  * thread-safe).  wait_limit_ns bounds every mbarrier wait (0 restores the 2 s
  * default).  With skip_first_commit != 0, each later launch never signals its first

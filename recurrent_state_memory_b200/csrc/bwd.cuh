@@ -1,0 +1,402 @@
+// bwd.cuh -- gradients of the chunk-WY forward (the backward pass of training).
+//
+// The chain rule through the chunk-parallel WY/UT algebra of the forward ("CARVE" page, section
+// 1 item 3, the WY-form chunk solver; "Semidirect Fourier Delta Attention" page, "Constructive
+// Chunk-WY Theorem" and the exact affine chunk transfer).  Per chunk of C = 64 tokens with start
+// state S0 (dv x dk), in-chunk cumulative log-decay gam (per token and key dim) and the
+// reference token m = 31 (so that no factor exceeds the decay of half a chunk):
+//   Kt = K e^{gam - gam_m},  Qt = scale Q e^{gam - gam_m},  Kh = K e^{-(gam - gam_m)},
+//   Kd = K e^{gam_L - gam},  S0p = S0 e^{gam_m}                           (column scalings)
+//   Ap = Kt Kh^T,  A = diag(beta) strict_lower(Ap),  P = incl_lower(Qt Kh^T),  T = (I + A)^{-1}
+//   KS = Kt S0p^T,  R = diag(w) V - diag(beta) KS,  E = T R
+//   O = Qt S0p^T + P E,  S_L = S0 e^{gam_L} + E^T Kd
+// and, backwards, with dO the chunk's output gradient and dS_L that of its end state:
+//   dE = P^T dO + Kd dS_L^T,  dP = incl_lower(dO E^T),  dR = T^T dE,  dA = -T^T (dE R^T) T^T
+//   dQt = dO S0p + dP Kh,  dKh = dP^T Qt + dAp^T Kt,  dKt = -(diag(beta) dR) S0p + dAp Kh,
+//   dKd = E dS_L,  dAp = diag(beta) strict_lower(dA)
+//   dS0 = (dO^T Qt - (diag(beta) dR)^T Kt) e^{gam_m} + dS_L e^{gam_L}
+//   dv = diag(w) dR,  dbeta = -rowsum(dR . KS) + rowsum(strict_lower(dA . Ap)) [+ rowsum(dR . V)
+//   when w = beta],  dw = rowsum(dR . V)
+//   dq = scale dQt e^{gam - gam_m},  dk = dKt e^{gam - gam_m} + dKh e^{-(gam - gam_m)} + dKd e^{gam_L - gam}
+//   dgam = dKt . Kt + dQt . Qt - dKh . Kh - dKd . Kd, plus, at the last token,
+//          e^{gam_L} colsum(S0 . dS_L) + colsum(dKd . Kd);   dg = (reverse cumsum of dgam) dlogalpha/dg
+// (the reference token cancels out of every product, so it leaves the gradients unchanged).
+//
+// One CTA per (batch, head).  A forward sweep over the chunks keeps each chunk's start state
+// (checkpoints in the workspace); the backward sweep then runs the chunks in reverse, each
+// recomputing its forward quantities from its checkpoint, with dS_L of chunk c the dS0 of chunk
+// c + 1 (the caller's dS_T for the last one).  The matrix products are warp-level tf32 tensor-core
+// MMAs with each operand split into a tf32 high part and a tf32 remainder (three products per
+// step), which keeps fp32 accuracy; the per-chunk matrices live in a per-head region of the
+// workspace (they stay in L1/L2).  Real decay only; the rotation variant's gradients exist in the
+// oracle.  Tokens past T are zero padding (k = q = v = 0, beta = w = 0, log-decay 0): exact
+// identity transitions whose gradients are not written.
+#pragma once
+
+#include "common.cuh"
+
+namespace gdr {
+namespace bwd {
+
+constexpr int C = 64;
+constexpr int NT = 512;
+constexpr int NW = NT / 32;
+constexpr unsigned STATUS_RANGE = 2u;
+
+struct BwdParams {
+    int B, H, T, gate_mode;
+    float scale;
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    const float* w;          // write strength [B,T,H] or nullptr (w = beta)
+    const float* S0;         // [B,H,dv,dk] or nullptr (zero)
+    const void* dO;          // [B,T,H,dv] (the output's dtype) or nullptr (zero)
+    const float* dS_T;       // [B,H,dv,dk] or nullptr (zero)
+    float* dq;               // [B,T,H,dk]
+    float* dk;               // [B,T,H,dk]
+    float* dv;               // [B,T,H,dv]
+    float* dg;               // [B,T,H,dk]
+    float* dbeta;            // [B,T,H]
+    float* dw;               // [B,T,H] (with w) or nullptr
+    float* dS0;              // [B,H,dv,dk] or nullptr
+    float* ws;               // per head: head_floats floats
+    size_t head_floats;
+};
+
+// Per-head workspace layout (floats).
+template <int DK, int DV>
+struct Lay {
+    static constexpr int K = 0, Q = K + C * DK, V = Q + C * DK, DO = V + C * DV;
+    static constexpr int EG = DO + C * DV;          // e^{gam - gam_m}
+    static constexpr int EGI = EG + C * DK;         // e^{-(gam - gam_m)}
+    static constexpr int DLG = EGI + C * DK;        // d log alpha / d gate input
+    static constexpr int KT = DLG + C * DK, KH = KT + C * DK, QT = KH + C * DK, KD = QT + C * DK;
+    static constexpr int AP = KD + C * DK, PM = AP + C * C, TM = PM + C * C, X1 = TM + C * C, X2 = X1 + C * C;
+    static constexpr int DA = X2 + C * C, DPM = DA + C * C;
+    static constexpr int KS = DPM + C * C, R = KS + C * DV, E = R + C * DV, DE = E + C * DV, DR = DE + C * DV;
+    static constexpr int DQT = DR + C * DV, DKH = DQT + C * DK, DKD = DKH + C * DK, DKT = DKD + C * DK;
+    static constexpr int DGAM = DKT + C * DK;
+    static constexpr int BT = DGAM + C * DK, WT = BT + C;
+    static constexpr int E31 = WT + C, EGL = E31 + DK, ED = EGL + DK, CS = ED + DK;   // column vectors
+    static constexpr int S0P = CS + DK, SC = S0P + DV * DK, DSL = SC + DV * DK, DS0 = DSL + DV * DK;
+    static constexpr int CKPT = DS0 + DV * DK;      // nchunks x (dv x dk): chunk start states
+    static constexpr size_t floats(int nchunks) { return (size_t)CKPT + (size_t)nchunks * DV * DK; }
+};
+
+__device__ __forceinline__ uint32_t tf32_hi(float x) { return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u; }
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Cm (M x N, row stride ldc) = alpha op(A) op(B) (+ Cm when acc), with op(A)(i, k) = A[i][k]
+// (TA: A[k][i]) and op(B)(k, j) = B[k][j] (TB: B[j][k]).  M, N multiples of 16, K of 8.  All
+// warps of the CTA take part; the caller synchronises before and after.
+template <bool TA, bool TB>
+__device__ void mm(float* Cm, int ldc, const float* A, int lda, const float* Bm, int ldb, int M, int N, int K,
+                   float alpha, bool acc) {
+    const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+    const int tn = N / 16, ntiles = (M / 16) * tn;
+    auto a_ = [&](int i, int k) -> float { return TA ? A[(size_t)k * lda + i] : A[(size_t)i * lda + k]; };
+    auto b_ = [&](int k, int j) -> float { return TB ? Bm[(size_t)j * ldb + k] : Bm[(size_t)k * ldb + j]; };
+    for (int t = warp; t < ntiles; t += NW) {
+        const int r0 = (t / tn) * 16, c0 = (t % tn) * 16;
+        float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        for (int k0 = 0; k0 < K; k0 += 8) {
+            const float af[4] = {a_(r0 + gid, k0 + tig), a_(r0 + gid + 8, k0 + tig), a_(r0 + gid, k0 + tig + 4),
+                                 a_(r0 + gid + 8, k0 + tig + 4)};
+            uint32_t ah[4], al[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ah[e] = tf32_hi(af[e]);
+                al[e] = tf32_hi(af[e] - __uint_as_float(ah[e]));
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float bf[2] = {b_(k0 + tig, c0 + 8 * h + gid), b_(k0 + tig + 4, c0 + 8 * h + gid)};
+                uint32_t bh[2], bl[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    bh[e] = tf32_hi(bf[e]);
+                    bl[e] = tf32_hi(bf[e] - __uint_as_float(bh[e]));
+                }
+                mma_tf32(d[h], al, bh);
+                mma_tf32(d[h], ah, bl);
+                mma_tf32(d[h], ah, bh);
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int row = r0 + gid + ((e >> 1) << 3), col = c0 + 8 * h + 2 * tig + (e & 1);
+                float x = alpha * d[h][e];
+                if (acc) x += Cm[(size_t)row * ldc + col];
+                Cm[(size_t)row * ldc + col] = x;
+            }
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ float ldx(const T* p, size_t i) {
+    return ld_f32<T>(p + i);
+}
+
+// One chunk's inputs and forward quantities up to E (every thread; ends synchronised).
+// S0 is the chunk's start state (dv x dk, row-major).
+template <int DK, int DV, typename QT, typename OT>
+__device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0, const float* S0, bool want_dO,
+                              int* range_f) {
+    using L = Lay<DK, DV>;
+    const int tid = (int)threadIdx.x;
+    const QT* q = static_cast<const QT*>(p.q);
+    const QT* k = static_cast<const QT*>(p.k);
+    const QT* v = static_cast<const QT*>(p.v);
+    auto tok = [&](int r) -> size_t { return ((size_t)b * p.T + (t0 + r)) * p.H + h; };
+    // raw inputs of the chunk, zero past T
+    for (int i = tid; i < C * DK; i += NT) {
+        const int r = i / DK, d = i % DK;
+        const bool ok = t0 + r < p.T;
+        W[L::K + i] = ok ? ldx(k, tok(r) * DK + d) : 0.f;
+        W[L::Q + i] = ok ? ldx(q, tok(r) * DK + d) : 0.f;
+        float lg = 0.f, dl = 0.f;
+        if (ok) {
+            const float a = p.g[tok(r) * DK + d];
+            lg = log_decay(a, p.gate_mode);
+            dl = p.gate_mode == 1 ? -1.f / (1.f + expf(-a)) : 1.f;      // d(-softplus a)/da = -sigmoid(a)
+        }
+        W[L::EG + i] = lg;               // log alpha for now
+        W[L::DLG + i] = dl;
+    }
+    for (int i = tid; i < C * DV; i += NT) {
+        const int r = i / DV, d = i % DV;
+        const bool ok = t0 + r < p.T;
+        W[L::V + i] = ok ? ldx(v, tok(r) * DV + d) : 0.f;
+        if (want_dO) W[L::DO + i] = (ok && p.dO) ? ldx(static_cast<const OT*>(p.dO), tok(r) * DV + d) : 0.f;
+    }
+    if (tid < C) {
+        const bool ok = t0 + tid < p.T;
+        const float bt = ok ? p.beta[tok(tid)] : 0.f;
+        W[L::BT + tid] = bt;
+        W[L::WT + tid] = ok ? (p.w ? p.w[tok(tid)] : bt) : 0.f;
+    }
+    __syncthreads();
+    // cumulative log-decay per key dim, relative to token m = 31, and the column decays
+    if (tid < DK) {
+        const int d = tid;
+        float gam = 0.f, g31 = 0.f;
+        for (int r = 0; r < C; ++r) {
+            gam += W[L::EG + r * DK + d];
+            W[L::EG + r * DK + d] = gam;
+            if (r == 31) g31 = gam;
+        }
+        const float gl = gam;
+        W[L::E31 + d] = expf(g31);
+        W[L::EGL + d] = expf(gl);
+        W[L::ED + d] = expf(gl - g31);
+        bool bad = false;
+        for (int r = 0; r < C; ++r) {
+            const float x = W[L::EG + r * DK + d] - g31;
+            const float e = expf(x), ei = expf(-x);
+            if (!(e < 3e38f) || !(ei < 3e38f)) bad = true;
+            W[L::EG + r * DK + d] = e;
+            W[L::EGI + r * DK + d] = ei;
+        }
+        if (bad) atomicExch(range_f, 1);
+    }
+    __syncthreads();
+    for (int i = tid; i < C * DK; i += NT) {
+        const int d = i % DK;
+        const float kk = W[L::K + i];
+        W[L::KT + i] = kk * W[L::EG + i];
+        W[L::KH + i] = kk * W[L::EGI + i];
+        W[L::QT + i] = p.scale * W[L::Q + i] * W[L::EG + i];
+        W[L::KD + i] = kk * W[L::EGI + i] * W[L::ED + d];
+    }
+    for (int i = tid; i < DV * DK; i += NT) W[L::S0P + i] = S0[i] * W[L::E31 + i % DK];
+    __syncthreads();
+    mm<false, true>(W + L::AP, C, W + L::KT, DK, W + L::KH, DK, C, C, DK, 1.f, false);      // Ap = Kt Kh^T
+    mm<false, true>(W + L::PM, C, W + L::QT, DK, W + L::KH, DK, C, C, DK, 1.f, false);      // Qt Kh^T
+    mm<false, true>(W + L::KS, DV, W + L::KT, DK, W + L::S0P, DK, C, DV, DK, 1.f, false);   // KS = Kt S0p^T
+    __syncthreads();
+    // masks; R = diag(w) V - diag(beta) KS; T = (I + A)^{-1} by forward substitution, eight
+    // threads per column
+    for (int i = tid; i < C * C; i += NT) {
+        const int r = i / C, c = i % C;
+        if (c > r) W[L::PM + i] = 0.f;
+    }
+    for (int i = tid; i < C * DV; i += NT) {
+        const int r = i / DV;
+        W[L::R + i] = W[L::WT + r] * W[L::V + i] - W[L::BT + r] * W[L::KS + i];
+    }
+    {
+        const int j = tid >> 3, part = tid & 7;            // column j, eighth of the sum
+        float* Tm = W + L::TM;
+        for (int r = 0; r < C; ++r) {
+            float s = 0.f;
+            if (r > j) {
+                const float br = W[L::BT + r];
+                for (int i = j + part; i < r; i += 8) s += br * W[L::AP + r * C + i] * Tm[i * C + j];
+            }
+#pragma unroll
+            for (int off = 4; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            if (part == 0) Tm[r * C + j] = (r == j) ? 1.f : (r > j ? -s : 0.f);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    mm<false, false>(W + L::E, DV, W + L::TM, C, W + L::R, DV, C, DV, C, 1.f, false);       // E = T R
+    __syncthreads();
+}
+
+template <int DK, int DV, typename QT, typename OT>
+__global__ void __launch_bounds__(NT, 1) chunk_bwd_kernel(BwdParams p) {
+    using L = Lay<DK, DV>;
+    __shared__ int range_f;
+    const int tid = (int)threadIdx.x;
+    const int head = (int)blockIdx.x, b = head / p.H, h = head % p.H;
+    const int nc = (p.T + C - 1) / C;
+    float* W = p.ws + (size_t)head * p.head_floats;
+    if (tid == 0) range_f = 0;
+    // ---- forward sweep: chunk start states ---------------------------------------------------
+    for (int i = tid; i < DV * DK; i += NT) W[L::SC + i] = p.S0 ? p.S0[(size_t)head * DV * DK + i] : 0.f;
+    __syncthreads();
+    for (int c = 0; c < nc; ++c) {
+        float* ck = W + L::CKPT + (size_t)c * DV * DK;
+        for (int i = tid; i < DV * DK; i += NT) ck[i] = W[L::SC + i];
+        __syncthreads();
+        chunk_forward<DK, DV, QT, OT>(p, W, b, h, c * C, ck, false, &range_f);
+        // S_L = S0 e^{gam_L} + E^T Kd
+        for (int i = tid; i < DV * DK; i += NT) W[L::SC + i] = ck[i] * W[L::EGL + i % DK];
+        __syncthreads();
+        mm<true, false>(W + L::SC, DK, W + L::E, DV, W + L::KD, DK, DV, DK, C, 1.f, true);
+        __syncthreads();
+    }
+    // ---- backward sweep --------------------------------------------------------------------------
+    for (int i = tid; i < DV * DK; i += NT) W[L::DSL + i] = p.dS_T ? p.dS_T[(size_t)head * DV * DK + i] : 0.f;
+    __syncthreads();
+    for (int c = nc - 1; c >= 0; --c) {
+        const int t0 = c * C;
+        const float* S0c = W + L::CKPT + (size_t)c * DV * DK;
+        chunk_forward<DK, DV, QT, OT>(p, W, b, h, t0, S0c, true, &range_f);
+        // dE = P^T dO + Kd dSL^T ; dP = incl_lower(dO E^T) ; dKd = E dSL ; dS0 = dO^T Qt
+        mm<true, false>(W + L::DE, DV, W + L::PM, C, W + L::DO, DV, C, DV, C, 1.f, false);
+        mm<false, true>(W + L::DPM, C, W + L::DO, DV, W + L::E, DV, C, C, DV, 1.f, false);
+        mm<false, false>(W + L::DKD, DK, W + L::E, DV, W + L::DSL, DK, C, DK, DV, 1.f, false);
+        mm<true, false>(W + L::DS0, DK, W + L::DO, DV, W + L::QT, DK, DV, DK, C, 1.f, false);
+        __syncthreads();
+        mm<false, true>(W + L::DE, DV, W + L::KD, DK, W + L::DSL, DK, C, DV, DK, 1.f, true);
+        for (int i = tid; i < C * C; i += NT) {
+            const int r = i / C, cc = i % C;
+            if (cc > r) W[L::DPM + i] = 0.f;
+        }
+        __syncthreads();
+        // dR = T^T dE ; X1 = dE R^T ; dQt = dO S0p + dP Kh ; dKh = dP^T Qt
+        mm<true, false>(W + L::DR, DV, W + L::TM, C, W + L::DE, DV, C, DV, C, 1.f, false);
+        mm<false, true>(W + L::X1, C, W + L::DE, DV, W + L::R, DV, C, C, DV, 1.f, false);
+        mm<false, false>(W + L::DQT, DK, W + L::DO, DV, W + L::S0P, DK, C, DK, DV, 1.f, false);
+        mm<true, false>(W + L::DKH, DK, W + L::DPM, C, W + L::QT, DK, C, DK, C, 1.f, false);
+        __syncthreads();
+        mm<false, false>(W + L::DQT, DK, W + L::DPM, C, W + L::KH, DK, C, DK, C, 1.f, true);
+        mm<true, false>(W + L::X2, C, W + L::TM, C, W + L::X1, C, C, C, C, 1.f, false);      // T^T X1
+        // beta dR (in place) after dv, dw and the dR parts of dbeta
+        __syncthreads();
+        mm<false, true>(W + L::DA, C, W + L::X2, C, W + L::TM, C, C, C, C, -1.f, false);     // dA = -X2 T^T
+        if (tid < C * 8) {
+            // per token r (eight threads each): dbeta and dw parts from dR
+            const int r = tid >> 3, part = tid & 7;
+            float sks = 0.f, sv = 0.f;
+            for (int j = part; j < DV; j += 8) {
+                const float dr = W[L::DR + r * DV + j];
+                sks += dr * W[L::KS + r * DV + j];
+                sv += dr * W[L::V + r * DV + j];
+            }
+#pragma unroll
+            for (int off = 4; off >= 1; off >>= 1) {
+                sks += __shfl_xor_sync(0xffffffffu, sks, off);
+                sv += __shfl_xor_sync(0xffffffffu, sv, off);
+            }
+            if (part == 0) {
+                W[L::DGAM + r] = -sks + (p.w ? 0.f : sv);        // dbeta so far (DGAM used as scratch)
+                if (p.dw && t0 + r < p.T) p.dw[((size_t)b * p.T + t0 + r) * p.H + h] = sv;
+            }
+        }
+        for (int i = tid; i < C * DV; i += NT) {
+            const int r = i / DV, j = i % DV;
+            if (t0 + r < p.T) p.dv[(((size_t)b * p.T + t0 + r) * p.H + h) * DV + j] = W[L::WT + r] * W[L::DR + i];
+        }
+        __syncthreads();
+        // dAp = diag(beta) strict_lower(dA) (in place, after the dA . Ap part of dbeta)
+        if (tid < C * 8) {
+            const int r = tid >> 3, part = tid & 7;
+            float s = 0.f;
+            for (int i = part; i < r; i += 8) s += W[L::DA + r * C + i] * W[L::AP + r * C + i];
+#pragma unroll
+            for (int off = 4; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            if (part == 0 && t0 + r < p.T)
+                p.dbeta[((size_t)b * p.T + t0 + r) * p.H + h] = W[L::DGAM + r] + s;
+        }
+        __syncthreads();
+        for (int i = tid; i < C * C; i += NT) {
+            const int r = i / C, cc = i % C;
+            W[L::DA + i] = cc < r ? W[L::BT + r] * W[L::DA + i] : 0.f;
+        }
+        for (int i = tid; i < C * DV; i += NT) W[L::DR + i] *= W[L::BT + i / DV];
+        __syncthreads();
+        // dKt = -(beta dR) S0p + dAp Kh ; dKh += dAp^T Kt ; dS0 -= (beta dR)^T Kt
+        mm<false, false>(W + L::DKT, DK, W + L::DR, DV, W + L::S0P, DK, C, DK, DV, -1.f, false);
+        mm<true, false>(W + L::DKH, DK, W + L::DA, C, W + L::KT, DK, C, DK, C, 1.f, true);
+        mm<true, false>(W + L::DS0, DK, W + L::DR, DV, W + L::KT, DK, DV, DK, C, -1.f, true);
+        __syncthreads();
+        mm<false, false>(W + L::DKT, DK, W + L::DA, C, W + L::KH, DK, C, DK, C, 1.f, true);
+        __syncthreads();
+        // dq, dk; dgam; dS0 = dS0 e^{gam_m} + dSL e^{gam_L}
+        for (int i = tid; i < C * DK; i += NT) {
+            const int r = i / DK, d = i % DK;
+            const float eg = W[L::EG + i], egi = W[L::EGI + i];
+            const float gkt = W[L::DKT + i], gkh = W[L::DKH + i], gqt = W[L::DQT + i], gkd = W[L::DKD + i];
+            if (t0 + r < p.T) {
+                const size_t o = (((size_t)b * p.T + t0 + r) * p.H + h) * DK + d;
+                p.dq[o] = p.scale * gqt * eg;
+                p.dk[o] = gkt * eg + gkh * egi + gkd * egi * W[L::ED + d];
+            }
+            W[L::DGAM + i] = gkt * W[L::KT + i] + gqt * W[L::QT + i] - gkh * W[L::KH + i] - gkd * W[L::KD + i];
+        }
+        if (tid < DK) {     // column sums for the last token's decay terms
+            const int d = tid;
+            float s0 = 0.f, sd = 0.f;
+            for (int i = 0; i < DV; ++i) s0 += S0c[i * DK + d] * W[L::DSL + i * DK + d];
+            for (int r = 0; r < C; ++r) sd += W[L::DKD + r * DK + d] * W[L::KD + r * DK + d];
+            W[L::CS + d] = W[L::EGL + d] * s0 + sd;
+        }
+        __syncthreads();
+        if (tid < DK) {     // reverse cumulative sum over the chunk's tokens
+            const int d = tid;
+            float acc = W[L::CS + d];
+            for (int r = C - 1; r >= 0; --r) {
+                acc += W[L::DGAM + r * DK + d];
+                if (t0 + r < p.T)
+                    p.dg[(((size_t)b * p.T + t0 + r) * p.H + h) * DK + d] = acc * W[L::DLG + r * DK + d];
+            }
+        }
+        for (int i = tid; i < DV * DK; i += NT) {
+            const int d = i % DK;
+            W[L::DS0 + i] = W[L::DS0 + i] * W[L::E31 + d] + W[L::DSL + i] * W[L::EGL + d];
+        }
+        __syncthreads();
+        for (int i = tid; i < DV * DK; i += NT) W[L::DSL + i] = W[L::DS0 + i];
+        __syncthreads();
+    }
+    if (p.dS0)
+        for (int i = tid; i < DV * DK; i += NT) p.dS0[(size_t)head * DV * DK + i] = W[L::DSL + i];
+    if (tid == 0 && range_f) atomicOr(&g_device_status, STATUS_RANGE);
+}
+
+}  // namespace bwd
+}  // namespace gdr

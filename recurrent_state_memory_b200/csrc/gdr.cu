@@ -13,6 +13,7 @@
 #include "tc_fwd.cuh"
 #include "split_fwd.cuh"
 #include "seg_combine.cuh"
+#include "bwd.cuh"
 
 namespace gdr {
 
@@ -604,6 +605,42 @@ static void host_plan(const gdr_fwd_desc* d, bool w, bool S0, bool S_T, bool cm,
     P->ring_bytes = round256(ring > ring_last ? ring : ring_last);
 }
 
+// ---- backward ------------------------------------------------------------------------------
+static gdr_status check_bwd_desc(const gdr_fwd_desc* d) {
+    gdr_status s = check_fwd_desc(d);
+    if (s != GDR_OK) return s;
+    if (d->dk != d->dv) return fail(GDR_ERR_UNSUPPORTED, "the backward needs dk = dv%s");
+    if (d->rotation) return fail(GDR_ERR_UNSUPPORTED, "the backward has no rotation form (real decay only)%s");
+    if (d->qk_l2norm) return fail(GDR_ERR_UNSUPPORTED, "the backward takes q and k as given (no qk_l2norm)%s");
+    return GDR_OK;
+}
+
+static size_t bwd_head_floats(int d, int T) {
+    const int nc = (T + 63) / 64;
+    switch (d) {
+        case 32: return bwd::Lay<32, 32>::floats(nc);
+        case 64: return bwd::Lay<64, 64>::floats(nc);
+        default: return bwd::Lay<128, 128>::floats(nc);
+    }
+}
+
+template <int D, typename QT, typename OT>
+static gdr_status launch_bwd(const bwd::BwdParams& p, int nh, cudaStream_t st) {
+    bwd::chunk_bwd_kernel<D, D, QT, OT><<<(unsigned)nh, bwd::NT, 0, st>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? GDR_OK : cuda_fail(e, "launch(backward kernel)");
+}
+
+template <int D>
+static gdr_status dispatch_bwd_d(const gdr_fwd_desc* d, const bwd::BwdParams& p, cudaStream_t st) {
+    const int nh = d->B * d->H;
+    const bool qb = d->qkv_dtype == GDR_BF16, ob = d->out_dtype == GDR_BF16;
+    if (qb && ob) return launch_bwd<D, __nv_bfloat16, __nv_bfloat16>(p, nh, st);
+    if (qb) return launch_bwd<D, __nv_bfloat16, float>(p, nh, st);
+    if (ob) return launch_bwd<D, float, __nv_bfloat16>(p, nh, st);
+    return launch_bwd<D, float, float>(p, nh, st);
+}
+
 }  // namespace gdr
 
 using namespace gdr;
@@ -809,6 +846,50 @@ int gdr_chunk_fwd_kernel_launches(const gdr_fwd_desc* d) {
         return (rem > 0 && split_fits_heads(rem, sms, d->T)) ? 2 : 1;
     }
     return 1;
+}
+
+size_t gdr_chunk_bwd_workspace_bytes(const gdr_fwd_desc* d) {
+    if (check_bwd_desc(d) != GDR_OK) return 0;
+    if (d->B == 0 || d->H == 0 || d->T == 0) return 0;
+    return (size_t)d->B * d->H * bwd_head_floats(d->dk, d->T) * sizeof(float);
+}
+
+gdr_status gdr_chunk_bwd(const gdr_fwd_desc* d, const void* q, const void* k, const void* v, const float* g,
+                         const float* beta, const float* w, const float* S0, const void* dO, const float* dS_T,
+                         float* dq, float* dk, float* dv, float* dg, float* dbeta, float* dw, float* dS0,
+                         void* workspace, size_t workspace_bytes, gdr_stream_t stream) {
+    t_detail[0] = 0;
+    gdr_status s = check_bwd_desc(d);
+    if (s != GDR_OK) return s;
+    if (d->B == 0 || d->H == 0) return GDR_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t sbytes = (size_t)d->B * d->H * d->dv * d->dk * sizeof(float);
+    if (d->T == 0) {    // no tokens: the gradient of S0 is that of S_T
+        if (!dS0) return GDR_OK;
+        if (!aligned16(dS0) || (dS_T && !aligned16(dS_T))) return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
+        const cudaError_t e = dS_T ? cudaMemcpyAsync(dS0, dS_T, sbytes, cudaMemcpyDeviceToDevice, st)
+                                   : cudaMemsetAsync(dS0, 0, sbytes, st);
+        return e == cudaSuccess ? GDR_OK : cuda_fail(e, "copy(dS0)");
+    }
+    if (!q || !k || !v || !g || !beta || !dq || !dk || !dv || !dg || !dbeta)
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta, dq, dk, dv, dg and dbeta are required%s");
+    if ((w == nullptr) != (dw == nullptr)) return fail(GDR_ERR_INVALID_ARG, "dw is required exactly when w is given%s");
+    const void* ptrs[] = {q, k, v, g, beta, w, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dw, dS0, workspace};
+    for (const void* x : ptrs)
+        if (x && !aligned16(x)) return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
+    const size_t need = gdr_chunk_bwd_workspace_bytes(d);
+    if (!workspace || workspace_bytes < need) return fail(GDR_ERR_WORKSPACE, "workspace too small%s");
+    bwd::BwdParams p;
+    p.B = d->B; p.H = d->H; p.T = d->T; p.gate_mode = (int)d->gate_mode; p.scale = d->scale;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.S0 = S0; p.dO = dO; p.dS_T = dS_T;
+    p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.dbeta = dbeta; p.dw = dw; p.dS0 = dS0;
+    p.ws = static_cast<float*>(workspace);
+    p.head_floats = bwd_head_floats(d->dk, d->T);
+    switch (d->dk) {
+        case 32: return dispatch_bwd_d<32>(d, p, st);
+        case 64: return dispatch_bwd_d<64>(d, p, st);
+        default: return dispatch_bwd_d<128>(d, p, st);
+    }
 }
 
 gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* d, const void* q, const void* k, const void* v,

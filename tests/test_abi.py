@@ -204,3 +204,31 @@ def test_kernel_launch_count_without_a_device(G):
     assert G.kernel_launches(d(0, 16, 4096)) == 0
     with pytest.raises(ValueError):
         G.kernel_launches(G.fwd_desc(1, 1, 64, 48, 48, bf, bf))
+
+
+def test_backward_checks_its_arguments_without_launching(G):
+    """gdr_chunk_bwd: the shapes it does not take are refused before any launch, a missing
+    output or a w without its dw is an argument error, and the workspace size follows the
+    per-head layout (chunk start states plus the chunk matrices)."""
+    import ctypes
+    import torch
+    L = G.lib()
+    bf = torch.bfloat16
+    d = lambda B, H, T, dk=128, dv=128, **kw: G.fwd_desc(B, H, T, dk, dv, bf, bf, **kw)
+    call = lambda desc, ptrs, ws=None, wsb=0: L.gdr_chunk_bwd(ctypes.byref(desc), *ptrs, ws, wsb, None)
+    fake = ctypes.c_void_p(1 << 20)        # never dereferenced: every call below fails its checks first
+    full = [fake] * 16                     # q, k, v, g, beta, w, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dw, dS0
+    assert call(d(1, 1, 64, rotation=True), full) == G.GDR_ERR_UNSUPPORTED
+    assert call(d(1, 1, 64, dk=64, dv=128), full) == G.GDR_ERR_UNSUPPORTED
+    assert call(d(1, 1, 64, qk_l2norm=True), full) == G.GDR_ERR_UNSUPPORTED
+    no_dw = list(full)
+    no_dw[14] = None
+    assert call(d(1, 1, 64), no_dw) == G.GDR_ERR_INVALID_ARG
+    no_dq = list(full)
+    no_dq[9] = None
+    assert call(d(1, 1, 64), no_dq) == G.GDR_ERR_INVALID_ARG
+    assert call(d(1, 1, 64), full, None, 0) == G.GDR_ERR_WORKSPACE
+    assert G.bwd_workspace_bytes(d(1, 1, 64, rotation=True)) == 0
+    per_head = lambda nc: 4 * (64 * 128 * 21 + 64 * 64 * 7 + 64 * 2 + 128 * 4 + 4 * 128 * 128 + nc * 128 * 128)
+    assert G.bwd_workspace_bytes(d(2, 3, 1000)) == 6 * per_head(16)
+    assert G.bwd_workspace_bytes(d(2, 3, 0)) == 0

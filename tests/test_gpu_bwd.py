@@ -1,0 +1,117 @@
+"""GPU parity of the backward pass (gdr_chunk_bwd) against the fp64 oracle's reverse-mode sweep
+of the token recurrence (oracle/backward.py): every input gradient, element by element.
+
+Tolerance: the kernel computes in fp32 (split-tf32 tensor-core products, fp32 elsewhere) on the
+same bf16/fp32 input values the oracle widens, so its error is fp32 rounding accumulated along
+the chunk chain; each gradient must satisfy max|d - d_ref| / max|d_ref| <= 1e-3."""
+import numpy as np
+import pytest
+
+from oracle.backward import gdr_bwd
+from recurrent_state_memory_b200 import inputs as I
+
+import parity_util as U
+
+pytestmark = pytest.mark.gpu
+
+TOL_BWD = 1e-3
+
+
+@pytest.fixture(scope="module")
+def G():
+    from recurrent_state_memory_b200 import gdr
+    gdr.lib()
+    return gdr
+
+
+BWD_CASES = [
+    # (B, H, T, d, dtype, gate_mode, untied w, S0, dO, dS_T, gate recipe)
+    (1, 2, 128, 128, "bf16", 1, False, False, True, True, "normal"),
+    (2, 1, 100, 64, "f32", 0, False, True, True, False, "normal"),       # ragged, log-decay gates
+    (1, 3, 200, 32, "bf16", 1, True, True, True, True, "normal"),        # ragged, separate w
+    (1, 1, 64, 128, "f32", 1, False, True, False, True, "normal"),       # only dS_T
+    (2, 2, 257, 128, "bf16", 1, False, True, True, True, "normal"),      # one-token tail
+    (1, 1, 512, 128, "bf16", 1, False, True, True, True, "slow"),        # slow decay, 8 chunks
+]
+
+
+def _case_id(c):
+    B, H, T, d, dt, gm, w, s0, do, ds, gate = c
+    return f"B{B}H{H}T{T}d{d}_{dt}_g{gm}" + ("_w" if w else "") + ("_s0" if s0 else "") + \
+        ("_dO" if do else "") + ("_dS" if ds else "") + ("_slow" if gate == "slow" else "")
+
+
+def _inputs(case, seed):
+    B, H, T, d, dt, gm, untied, s0, with_dO, with_dS, gate = case
+    p = I.make_fwd(B, T, H, d, d, dtype=dt, seed=seed, gate=gate, s0_std=0.3 if s0 else None)
+    g = p.g if gm == 1 else (-np.logaddexp(0.0, p.g.astype(np.float64))).astype(np.float32)   # log-decay values
+    w = I.make_write_strength(seed + 1, (B, T, H)) if untied else None
+    dO = I.normal(seed, "dO", (B, T, H, d)).astype(np.float32) if with_dO else None
+    if dO is not None and dt == "bf16":
+        dO = I.to_bf16_bits(dO)
+    dS = I.normal(seed, "dS_T", (B, H, d, d), std=0.5).astype(np.float32) if with_dS else None
+    return p, g, w, dO, dS
+
+
+def _widen(a):
+    if a is None:
+        return None
+    return (I.bf16_bits_to_f32(a) if a.dtype == np.uint16 else a).astype(np.float64)
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=_case_id)
+def test_backward_parity(G, case):
+    import torch
+    p, g, w, dO, dS = _inputs(case, 700 + case[2] + case[3])
+    gm = case[5]
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "beta", "S0")}
+    gt = U.to_torch(g, "cuda")
+    wt, dOt, dSt = U.to_torch(w, "cuda"), U.to_torch(dO, "cuda"), U.to_torch(dS, "cuda")
+    grads = G.chunk_bwd(t["q"], t["k"], t["v"], gt, t["beta"], t["S0"], dOt, dSt, gate_mode=gm, w=wt,
+                        out_dtype=t["q"].dtype)
+    torch.cuda.synchronize()
+    assert G.query_device_status() == G.GDR_OK
+    _, _, ref = gdr_bwd(p.widened("q"), p.widened("k"), p.widened("v"), g.astype(np.float64),
+                        p.widened("beta"), None, p.widened("S0"), _widen(dO), _widen(dS), gate_mode=gm,
+                        scale=p.scale, w=None if w is None else w.astype(np.float64))
+    names = ["q", "k", "v", "g", "beta", "S0"] + (["w"] if w is not None else [])
+    for n in names:
+        got = grads[n].cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(got)), f"non-finite d{n}"
+        e = U.max_rel(got, ref[n])
+        assert e <= TOL_BWD, f"d{n}: max-rel error {e:.3e} > {TOL_BWD:.0e}"
+
+
+def test_backward_without_tokens_passes_the_state_gradient(G):
+    import torch
+    q = torch.zeros((1, 0, 2, 64), dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros((1, 0, 2, 64), dtype=torch.bfloat16, device="cuda")
+    g = torch.zeros((1, 0, 2, 64), dtype=torch.float32, device="cuda")
+    beta = torch.zeros((1, 0, 2), dtype=torch.float32, device="cuda")
+    dS = torch.from_numpy(I.normal(5, "dS_T", (1, 2, 64, 64)).astype(np.float32)).cuda()
+    grads = G.chunk_bwd(q, q, v, g, beta, None, None, dS)
+    torch.cuda.synchronize()
+    assert torch.equal(grads["S0"], dS)
+
+
+def test_backward_matches_a_finite_difference_of_the_forward_kernel(G):
+    """The backward kernel against the forward kernel itself: the directional derivative of
+    <dO, o> + <dS_T, S_T> along a random direction of beta, by central differences of two
+    fp32 forward launches, equals <dbeta, direction>."""
+    import torch
+    B, H, T, d = 1, 2, 130, 64
+    p = I.make_fwd(B, T, H, d, d, dtype="f32", seed=771, s0_std=0.2)
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "g", "beta", "S0")}
+    dO = torch.from_numpy(I.normal(772, "dO", (B, T, H, d)).astype(np.float32)).cuda()
+    dS = torch.from_numpy(I.normal(773, "dS_T", (B, H, d, d)).astype(np.float32)).cuda()
+    dirn = torch.from_numpy(I.normal(774, "dir", (B, T, H)).astype(np.float32)).cuda()
+    grads = G.chunk_bwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], dO, dS)
+    h = 1e-3
+
+    def loss(beta):
+        o, S = G.chunk_fwd(t["q"], t["k"], t["v"], t["g"], beta, None, t["S0"], algo="simt")
+        return float((o.double() * dO.double()).sum() + (S.double() * dS.double()).sum())
+
+    fd = (loss(t["beta"] + h * dirn) - loss(t["beta"] - h * dirn)) / (2 * h)
+    an = float((grads["beta"].double() * dirn.double()).sum())
+    assert abs(fd - an) <= 2e-3 * max(1.0, abs(an)), (fd, an)
