@@ -95,16 +95,38 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// Shared-memory floats the products need: both operands with padded rows.
+constexpr int SMEM_FLOATS = 128 * 132 + 128 * 136;
+constexpr size_t SMEM_BYTES = sizeof(float) * SMEM_FLOATS;
+
+// rows x cols floats (global, row stride ld, 16-byte aligned rows) -> shared memory with row
+// stride ls, float4 at a time
+__device__ __forceinline__ void stage(float* dst, int ls, const float* src, int ld, int rows, int cols) {
+    const int c4 = cols >> 2;
+    for (int i = (int)threadIdx.x; i < rows * c4; i += NT) {
+        const int r = i / c4, c = (i % c4) * 4;
+        *reinterpret_cast<float4*>(dst + r * ls + c) = *reinterpret_cast<const float4*>(src + (size_t)r * ld + c);
+    }
+}
+
 // Cm (M x N, row stride ldc) = alpha op(A) op(B) (+ Cm when acc), with op(A)(i, k) = A[i][k]
-// (TA: A[k][i]) and op(B)(k, j) = B[k][j] (TB: B[j][k]).  M, N multiples of 16, K of 8.  All
-// warps of the CTA take part; the caller synchronises before and after.
+// (TA: A[k][i]) and op(B)(k, j) = B[k][j] (TB: B[j][k]).  M, N multiples of 16, K of 8, all at
+// most 128.  Both operands are first staged in shared memory `sm`, with row strides padded so
+// that the fragment loads hit 32 distinct banks.  All threads of the CTA take part; the caller
+// synchronises before (the operands are written) and after (Cm is read).
 template <bool TA, bool TB>
 __device__ void mm(float* Cm, int ldc, const float* A, int lda, const float* Bm, int ldb, int M, int N, int K,
-                   float alpha, bool acc) {
+                   float alpha, bool acc, float* sm) {
     const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
     const int tn = N / 16, ntiles = (M / 16) * tn;
-    auto a_ = [&](int i, int k) -> float { return TA ? A[(size_t)k * lda + i] : A[(size_t)i * lda + k]; };
-    auto b_ = [&](int k, int j) -> float { return TB ? Bm[(size_t)j * ldb + k] : Bm[(size_t)k * ldb + j]; };
+    const int sa = TA ? M + 8 : K + 4, sbs = TB ? K + 4 : N + 8;
+    float* sA = sm;
+    float* sB = sm + 128 * 132;
+    stage(sA, sa, A, lda, TA ? K : M, TA ? M : K);
+    stage(sB, sbs, Bm, ldb, TB ? N : K, TB ? K : N);
+    __syncthreads();
+    auto a_ = [&](int i, int k) -> float { return TA ? sA[k * sa + i] : sA[i * sa + k]; };
+    auto b_ = [&](int k, int j) -> float { return TB ? sB[j * sbs + k] : sB[k * sbs + j]; };
     for (int t = warp; t < ntiles; t += NW) {
         const int r0 = (t / tn) * 16, c0 = (t % tn) * 16;
         float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -141,6 +163,7 @@ __device__ void mm(float* Cm, int ldc, const float* A, int lda, const float* Bm,
                 Cm[(size_t)row * ldc + col] = x;
             }
     }
+    __syncthreads();     // the staged operands may be overwritten by the next product
 }
 
 template <typename T>
@@ -152,33 +175,38 @@ __device__ __forceinline__ float ldx(const T* p, size_t i) {
 // S0 is the chunk's start state (dv x dk, row-major).
 template <int DK, int DV, typename QT, typename OT>
 __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0, const float* S0, bool want_dO,
-                              int* range_f) {
+                              int* range_f, float* sm) {
     using L = Lay<DK, DV>;
     const int tid = (int)threadIdx.x;
     const QT* q = static_cast<const QT*>(p.q);
     const QT* k = static_cast<const QT*>(p.k);
     const QT* v = static_cast<const QT*>(p.v);
     auto tok = [&](int r) -> size_t { return ((size_t)b * p.T + (t0 + r)) * p.H + h; };
-    // raw inputs of the chunk, zero past T
-    for (int i = tid; i < C * DK; i += NT) {
-        const int r = i / DK, d = i % DK;
+    // raw inputs of the chunk, zero past T (four loads in flight per thread); the log-decays go
+    // to shared memory for the scan below
+    float* sg = sm;                       // [C][DK] log alpha, then gam
+    float* sg31 = sm + C * DK;            // [DK]
+    constexpr int NK = C * DK / NT, NV = C * DV / NT;
+#pragma unroll
+    for (int u = 0; u < NK; ++u) {
+        const int i = tid + u * NT, r = i / DK, d = i % DK;
         const bool ok = t0 + r < p.T;
-        W[L::K + i] = ok ? ldx(k, tok(r) * DK + d) : 0.f;
-        W[L::Q + i] = ok ? ldx(q, tok(r) * DK + d) : 0.f;
-        float lg = 0.f, dl = 0.f;
-        if (ok) {
-            const float a = p.g[tok(r) * DK + d];
-            lg = log_decay(a, p.gate_mode);
-            dl = p.gate_mode == 1 ? -1.f / (1.f + expf(-a)) : 1.f;      // d(-softplus a)/da = -sigmoid(a)
-        }
-        W[L::EG + i] = lg;               // log alpha for now
-        W[L::DLG + i] = dl;
+        const size_t o = tok(r) * DK + d;
+        const float kk = ok ? ldx(k, o) : 0.f, qq = ok ? ldx(q, o) : 0.f, a = ok ? p.g[o] : 0.f;
+        W[L::K + i] = kk;
+        W[L::Q + i] = qq;
+        sg[i] = ok ? log_decay(a, p.gate_mode) : 0.f;
+        W[L::DLG + i] = ok ? (p.gate_mode == 1 ? -1.f / (1.f + expf(-a)) : 1.f) : 0.f;   // d(-softplus a)/da = -sigmoid(a)
     }
-    for (int i = tid; i < C * DV; i += NT) {
-        const int r = i / DV, d = i % DV;
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int i = tid + u * NT, r = i / DV, d = i % DV;
         const bool ok = t0 + r < p.T;
-        W[L::V + i] = ok ? ldx(v, tok(r) * DV + d) : 0.f;
-        if (want_dO) W[L::DO + i] = (ok && p.dO) ? ldx(static_cast<const OT*>(p.dO), tok(r) * DV + d) : 0.f;
+        const size_t o = tok(r) * DV + d;
+        const float vv = ok ? ldx(v, o) : 0.f;
+        const float dd = (want_dO && ok && p.dO) ? ldx(static_cast<const OT*>(p.dO), o) : 0.f;
+        W[L::V + i] = vv;
+        if (want_dO) W[L::DO + i] = dd;
     }
     if (tid < C) {
         const bool ok = t0 + tid < p.T;
@@ -192,21 +220,25 @@ __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0
         const int d = tid;
         float gam = 0.f, g31 = 0.f;
         for (int r = 0; r < C; ++r) {
-            gam += W[L::EG + r * DK + d];
-            W[L::EG + r * DK + d] = gam;
+            gam += sg[r * DK + d];
+            sg[r * DK + d] = gam;
             if (r == 31) g31 = gam;
         }
         const float gl = gam;
+        sg31[d] = g31;
         W[L::E31 + d] = expf(g31);
         W[L::EGL + d] = expf(gl);
         W[L::ED + d] = expf(gl - g31);
+    }
+    __syncthreads();
+    {
         bool bad = false;
-        for (int r = 0; r < C; ++r) {
-            const float x = W[L::EG + r * DK + d] - g31;
+        for (int i = tid; i < C * DK; i += NT) {
+            const float x = sg[i] - sg31[i % DK];
             const float e = expf(x), ei = expf(-x);
             if (!(e < 3e38f) || !(ei < 3e38f)) bad = true;
-            W[L::EG + r * DK + d] = e;
-            W[L::EGI + r * DK + d] = ei;
+            W[L::EG + i] = e;
+            W[L::EGI + i] = ei;
         }
         if (bad) atomicExch(range_f, 1);
     }
@@ -221,9 +253,9 @@ __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0
     }
     for (int i = tid; i < DV * DK; i += NT) W[L::S0P + i] = S0[i] * W[L::E31 + i % DK];
     __syncthreads();
-    mm<false, true>(W + L::AP, C, W + L::KT, DK, W + L::KH, DK, C, C, DK, 1.f, false);      // Ap = Kt Kh^T
-    mm<false, true>(W + L::PM, C, W + L::QT, DK, W + L::KH, DK, C, C, DK, 1.f, false);      // Qt Kh^T
-    mm<false, true>(W + L::KS, DV, W + L::KT, DK, W + L::S0P, DK, C, DV, DK, 1.f, false);   // KS = Kt S0p^T
+    mm<false, true>(W + L::AP, C, W + L::KT, DK, W + L::KH, DK, C, C, DK, 1.f, false, sm);      // Ap = Kt Kh^T
+    mm<false, true>(W + L::PM, C, W + L::QT, DK, W + L::KH, DK, C, C, DK, 1.f, false, sm);      // Qt Kh^T
+    mm<false, true>(W + L::KS, DV, W + L::KT, DK, W + L::S0P, DK, C, DV, DK, 1.f, false, sm);   // KS = Kt S0p^T
     __syncthreads();
     // masks; R = diag(w) V - diag(beta) KS; T = (I + A)^{-1} by forward substitution, eight
     // threads per column
@@ -235,29 +267,37 @@ __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0
         const int r = i / DV;
         W[L::R + i] = W[L::WT + r] * W[L::V + i] - W[L::BT + r] * W[L::KS + i];
     }
-    {
+    {   // A = diag(beta) strict_lower(Ap) and T in shared memory (row stride C + 1)
+        float* sAm = sm;
+        float* sT = sm + C * (C + 1);
+        for (int i = tid; i < C * C; i += NT) {
+            const int r = i / C, c = i % C;
+            sAm[r * (C + 1) + c] = W[L::BT + r] * W[L::AP + i];
+        }
+        __syncthreads();
         const int j = tid >> 3, part = tid & 7;            // column j, eighth of the sum
-        float* Tm = W + L::TM;
         for (int r = 0; r < C; ++r) {
             float s = 0.f;
-            if (r > j) {
-                const float br = W[L::BT + r];
-                for (int i = j + part; i < r; i += 8) s += br * W[L::AP + r * C + i] * Tm[i * C + j];
-            }
+            if (r > j)
+                for (int i = j + part; i < r; i += 8) s += sAm[r * (C + 1) + i] * sT[i * (C + 1) + j];
 #pragma unroll
             for (int off = 4; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-            if (part == 0) Tm[r * C + j] = (r == j) ? 1.f : (r > j ? -s : 0.f);
+            if (part == 0) sT[r * (C + 1) + j] = (r == j) ? 1.f : (r > j ? -s : 0.f);
             __syncwarp();
         }
+        __syncthreads();
+        for (int i = tid; i < C * C; i += NT) W[L::TM + i] = sT[(i / C) * (C + 1) + i % C];
     }
     __syncthreads();
-    mm<false, false>(W + L::E, DV, W + L::TM, C, W + L::R, DV, C, DV, C, 1.f, false);       // E = T R
+    mm<false, false>(W + L::E, DV, W + L::TM, C, W + L::R, DV, C, DV, C, 1.f, false, sm);       // E = T R
     __syncthreads();
 }
 
 template <int DK, int DV, typename QT, typename OT>
 __global__ void __launch_bounds__(NT, 1) chunk_bwd_kernel(BwdParams p) {
     using L = Lay<DK, DV>;
+    extern __shared__ float4 sm4[];
+    float* sm = reinterpret_cast<float*>(sm4);
     __shared__ int range_f;
     const int tid = (int)threadIdx.x;
     const int head = (int)blockIdx.x, b = head / p.H, h = head % p.H;
@@ -271,11 +311,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_kernel(BwdParams p) {
         float* ck = W + L::CKPT + (size_t)c * DV * DK;
         for (int i = tid; i < DV * DK; i += NT) ck[i] = W[L::SC + i];
         __syncthreads();
-        chunk_forward<DK, DV, QT, OT>(p, W, b, h, c * C, ck, false, &range_f);
+        chunk_forward<DK, DV, QT, OT>(p, W, b, h, c * C, ck, false, &range_f, sm);
         // S_L = S0 e^{gam_L} + E^T Kd
         for (int i = tid; i < DV * DK; i += NT) W[L::SC + i] = ck[i] * W[L::EGL + i % DK];
         __syncthreads();
-        mm<true, false>(W + L::SC, DK, W + L::E, DV, W + L::KD, DK, DV, DK, C, 1.f, true);
+        mm<true, false>(W + L::SC, DK, W + L::E, DV, W + L::KD, DK, DV, DK, C, 1.f, true, sm);
         __syncthreads();
     }
     // ---- backward sweep --------------------------------------------------------------------------
@@ -284,30 +324,30 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_kernel(BwdParams p) {
     for (int c = nc - 1; c >= 0; --c) {
         const int t0 = c * C;
         const float* S0c = W + L::CKPT + (size_t)c * DV * DK;
-        chunk_forward<DK, DV, QT, OT>(p, W, b, h, t0, S0c, true, &range_f);
+        chunk_forward<DK, DV, QT, OT>(p, W, b, h, t0, S0c, true, &range_f, sm);
         // dE = P^T dO + Kd dSL^T ; dP = incl_lower(dO E^T) ; dKd = E dSL ; dS0 = dO^T Qt
-        mm<true, false>(W + L::DE, DV, W + L::PM, C, W + L::DO, DV, C, DV, C, 1.f, false);
-        mm<false, true>(W + L::DPM, C, W + L::DO, DV, W + L::E, DV, C, C, DV, 1.f, false);
-        mm<false, false>(W + L::DKD, DK, W + L::E, DV, W + L::DSL, DK, C, DK, DV, 1.f, false);
-        mm<true, false>(W + L::DS0, DK, W + L::DO, DV, W + L::QT, DK, DV, DK, C, 1.f, false);
+        mm<true, false>(W + L::DE, DV, W + L::PM, C, W + L::DO, DV, C, DV, C, 1.f, false, sm);
+        mm<false, true>(W + L::DPM, C, W + L::DO, DV, W + L::E, DV, C, C, DV, 1.f, false, sm);
+        mm<false, false>(W + L::DKD, DK, W + L::E, DV, W + L::DSL, DK, C, DK, DV, 1.f, false, sm);
+        mm<true, false>(W + L::DS0, DK, W + L::DO, DV, W + L::QT, DK, DV, DK, C, 1.f, false, sm);
         __syncthreads();
-        mm<false, true>(W + L::DE, DV, W + L::KD, DK, W + L::DSL, DK, C, DV, DK, 1.f, true);
+        mm<false, true>(W + L::DE, DV, W + L::KD, DK, W + L::DSL, DK, C, DV, DK, 1.f, true, sm);
         for (int i = tid; i < C * C; i += NT) {
             const int r = i / C, cc = i % C;
             if (cc > r) W[L::DPM + i] = 0.f;
         }
         __syncthreads();
         // dR = T^T dE ; X1 = dE R^T ; dQt = dO S0p + dP Kh ; dKh = dP^T Qt
-        mm<true, false>(W + L::DR, DV, W + L::TM, C, W + L::DE, DV, C, DV, C, 1.f, false);
-        mm<false, true>(W + L::X1, C, W + L::DE, DV, W + L::R, DV, C, C, DV, 1.f, false);
-        mm<false, false>(W + L::DQT, DK, W + L::DO, DV, W + L::S0P, DK, C, DK, DV, 1.f, false);
-        mm<true, false>(W + L::DKH, DK, W + L::DPM, C, W + L::QT, DK, C, DK, C, 1.f, false);
+        mm<true, false>(W + L::DR, DV, W + L::TM, C, W + L::DE, DV, C, DV, C, 1.f, false, sm);
+        mm<false, true>(W + L::X1, C, W + L::DE, DV, W + L::R, DV, C, C, DV, 1.f, false, sm);
+        mm<false, false>(W + L::DQT, DK, W + L::DO, DV, W + L::S0P, DK, C, DK, DV, 1.f, false, sm);
+        mm<true, false>(W + L::DKH, DK, W + L::DPM, C, W + L::QT, DK, C, DK, C, 1.f, false, sm);
         __syncthreads();
-        mm<false, false>(W + L::DQT, DK, W + L::DPM, C, W + L::KH, DK, C, DK, C, 1.f, true);
-        mm<true, false>(W + L::X2, C, W + L::TM, C, W + L::X1, C, C, C, C, 1.f, false);      // T^T X1
+        mm<false, false>(W + L::DQT, DK, W + L::DPM, C, W + L::KH, DK, C, DK, C, 1.f, true, sm);
+        mm<true, false>(W + L::X2, C, W + L::TM, C, W + L::X1, C, C, C, C, 1.f, false, sm);      // T^T X1
         // beta dR (in place) after dv, dw and the dR parts of dbeta
         __syncthreads();
-        mm<false, true>(W + L::DA, C, W + L::X2, C, W + L::TM, C, C, C, C, -1.f, false);     // dA = -X2 T^T
+        mm<false, true>(W + L::DA, C, W + L::X2, C, W + L::TM, C, C, C, C, -1.f, false, sm);     // dA = -X2 T^T
         if (tid < C * 8) {
             // per token r (eight threads each): dbeta and dw parts from dR
             const int r = tid >> 3, part = tid & 7;
@@ -350,13 +390,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_kernel(BwdParams p) {
         for (int i = tid; i < C * DV; i += NT) W[L::DR + i] *= W[L::BT + i / DV];
         __syncthreads();
         // dKt = -(beta dR) S0p + dAp Kh ; dKh += dAp^T Kt ; dS0 -= (beta dR)^T Kt
-        mm<false, false>(W + L::DKT, DK, W + L::DR, DV, W + L::S0P, DK, C, DK, DV, -1.f, false);
-        mm<true, false>(W + L::DKH, DK, W + L::DA, C, W + L::KT, DK, C, DK, C, 1.f, true);
-        mm<true, false>(W + L::DS0, DK, W + L::DR, DV, W + L::KT, DK, DV, DK, C, -1.f, true);
+        mm<false, false>(W + L::DKT, DK, W + L::DR, DV, W + L::S0P, DK, C, DK, DV, -1.f, false, sm);
+        mm<true, false>(W + L::DKH, DK, W + L::DA, C, W + L::KT, DK, C, DK, C, 1.f, true, sm);
+        mm<true, false>(W + L::DS0, DK, W + L::DR, DV, W + L::KT, DK, DV, DK, C, -1.f, true, sm);
         __syncthreads();
-        mm<false, false>(W + L::DKT, DK, W + L::DA, C, W + L::KH, DK, C, DK, C, 1.f, true);
+        mm<false, false>(W + L::DKT, DK, W + L::DA, C, W + L::KH, DK, C, DK, C, 1.f, true, sm);
         __syncthreads();
-        // dq, dk; dgam; dS0 = dS0 e^{gam_m} + dSL e^{gam_L}
+        // dq, dk; dgam (shared memory); dS0 = dS0 e^{gam_m} + dSL e^{gam_L}
+        float* sdg = sm;                  // [C][DK] dgam, then dg
+        float* sdl = sm + C * DK;         // [C][DK] d log alpha / d gate input
+        float* scs = sm + 2 * C * DK;     // [NT / DK][DK] column-sum parts
         for (int i = tid; i < C * DK; i += NT) {
             const int r = i / DK, d = i % DK;
             const float eg = W[L::EG + i], egi = W[L::EGI + i];
@@ -366,24 +409,31 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_kernel(BwdParams p) {
                 p.dq[o] = p.scale * gqt * eg;
                 p.dk[o] = gkt * eg + gkh * egi + gkd * egi * W[L::ED + d];
             }
-            W[L::DGAM + i] = gkt * W[L::KT + i] + gqt * W[L::QT + i] - gkh * W[L::KH + i] - gkd * W[L::KD + i];
+            sdg[i] = gkt * W[L::KT + i] + gqt * W[L::QT + i] - gkh * W[L::KH + i] - gkd * W[L::KD + i];
+            sdl[i] = W[L::DLG + i];
         }
-        if (tid < DK) {     // column sums for the last token's decay terms
-            const int d = tid;
+        {   // column sums for the last token's decay terms: NT / DK threads per key dim
+            constexpr int NP = NT / DK;
+            const int d = tid % DK, part = tid / DK;
             float s0 = 0.f, sd = 0.f;
-            for (int i = 0; i < DV; ++i) s0 += S0c[i * DK + d] * W[L::DSL + i * DK + d];
-            for (int r = 0; r < C; ++r) sd += W[L::DKD + r * DK + d] * W[L::KD + r * DK + d];
-            W[L::CS + d] = W[L::EGL + d] * s0 + sd;
+            for (int i = part; i < DV; i += NP) s0 += S0c[i * DK + d] * W[L::DSL + i * DK + d];
+            for (int r = part; r < C; r += NP) sd += W[L::DKD + r * DK + d] * W[L::KD + r * DK + d];
+            scs[part * DK + d] = W[L::EGL + d] * s0 + sd;
         }
         __syncthreads();
         if (tid < DK) {     // reverse cumulative sum over the chunk's tokens
             const int d = tid;
-            float acc = W[L::CS + d];
+            float acc = 0.f;
+            for (int pp = 0; pp < NT / DK; ++pp) acc += scs[pp * DK + d];
             for (int r = C - 1; r >= 0; --r) {
-                acc += W[L::DGAM + r * DK + d];
-                if (t0 + r < p.T)
-                    p.dg[(((size_t)b * p.T + t0 + r) * p.H + h) * DK + d] = acc * W[L::DLG + r * DK + d];
+                acc += sdg[r * DK + d];
+                sdg[r * DK + d] = acc * sdl[r * DK + d];
             }
+        }
+        __syncthreads();
+        for (int i = tid; i < C * DK; i += NT) {
+            const int r = i / DK, d = i % DK;
+            if (t0 + r < p.T) p.dg[(((size_t)b * p.T + t0 + r) * p.H + h) * DK + d] = sdg[i];
         }
         for (int i = tid; i < DV * DK; i += NT) {
             const int d = i % DK;

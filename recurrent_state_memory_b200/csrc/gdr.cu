@@ -626,8 +626,11 @@ static size_t bwd_head_floats(int d, int T) {
 
 template <int D, typename QT, typename OT>
 static gdr_status launch_bwd(const bwd::BwdParams& p, int nh, cudaStream_t st) {
-    bwd::chunk_bwd_kernel<D, D, QT, OT><<<(unsigned)nh, bwd::NT, 0, st>>>(p);
-    const cudaError_t e = cudaGetLastError();
+    auto kern = bwd::chunk_bwd_kernel<D, D, QT, OT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(backward kernel)");
+    kern<<<(unsigned)nh, bwd::NT, bwd::SMEM_BYTES, st>>>(p);
+    e = cudaGetLastError();
     return e == cudaSuccess ? GDR_OK : cuda_fail(e, "launch(backward kernel)");
 }
 
