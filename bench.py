@@ -10,7 +10,9 @@ between steps.  Decode (256 sequences x 16 heads, fp32 state) is measured in the
 same run and reported in the "decode" object, and the two other forward
 workloads (B=16, H=12, T=4096 with slow decay and a random initial state; the
 block-rotation variant at B=2, H=16, T=8192) each get an object of their own in
-"workloads", timed the same way with their own roofline and clock record.  Under
+"workloads", timed the same way with their own roofline and clock record; the
+backward pass (gradients of every input) on the headline workload is the "backward"
+object.  Under
 torchrun every rank runs its own independent batch (weak scaling, no data-path
 collective); the time is the max over ranks.  Rank 0 prints one JSON line.
 """
@@ -87,8 +89,9 @@ def load_peaks():
 KERNEL_SOURCES = {
     "gdr_chunk_fwd_simt": ["simt_fwd.cuh", "common.cuh"],
     "gdr_chunk_fwd_tcgen05": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
-    "gdr_chunk_fwd_tcgen05_split": ["split_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
-    "gdr_chunk_fwd_tcgen05_waves": ["tc_fwd.cuh", "split_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
+    "gdr_chunk_fwd_tcgen05_split": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
+    "gdr_chunk_fwd_tcgen05_waves": ["tc_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
+    "gdr_chunk_fwd_tcgen05_chains": ["split_fwd.cuh", "tc_ptx.cuh", "common.cuh"],
     "gdr_chunk_fwd_tcgen05_segments": ["split_fwd.cuh", "seg_combine.cuh", "tc_ptx.cuh", "common.cuh"],
     "gdr_decode_step": ["decode.cuh", "common.cuh"],
 }
@@ -417,6 +420,41 @@ def run_ours(args):
                                "traffic": stored_traffic("gdr_decode_step", "decode_n256_h16_d128"),
                                "kernel": "gdr_decode_step"}}
 
+    # ---- backward pass (gradients of every input) on the same workload ----
+    bwd = None
+    if not args.no_bwd and not p.rotation and p.dk == p.dv:
+        dO_dev = torch.from_numpy(I.normal(rank_seed(cfg["seed"], rank) + 31, "dO", (p.B, p.T, p.H, p.dv))
+                                  .astype(np.float32)).to(dev).to(o.dtype)
+        dS_dev = torch.from_numpy(I.normal(rank_seed(cfg["seed"], rank) + 32, "dS_T", (p.B, p.H, p.dv, p.dk))
+                                  .astype(np.float32)).to(dev)
+        bdesc = gdr.fwd_desc(p.B, p.H, p.T, p.dk, p.dv, dv_t["q"].dtype, o.dtype, p.gate_mode, False, p.scale)
+        bws = torch.empty(gdr.bwd_workspace_bytes(bdesc), dtype=torch.uint8, device=dev)
+
+        def bstep():
+            return gdr.chunk_bwd(dv_t["q"], dv_t["k"], dv_t["v"], dv_t["g"], dv_t["beta"], dv_t["S0"], dO_dev, dS_dev,
+                                 gate_mode=p.gate_mode, scale=p.scale, workspace=bws, stream=stream)
+
+        bstep()
+        torch.cuda.synchronize()
+        n_b = max(1, min(args.steps, 3))
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_b):
+            bstep()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        b_ms = max_over_ranks(a.elapsed_time(b_) / n_b, dev)
+        # bytes a backward must move: q, k, v, gates, beta and dO in; dq, dk, dv, dg (fp32), dbeta out
+        esz = dv_t["q"].element_size()
+        b_bytes = p.B * p.T * p.H * (3 * p.dk * esz + p.dk * 4 + 4 + p.dv * o.element_size() + 4 * p.dk * 4 + 4)
+        b_gbs = b_bytes / (b_ms * 1e-3) / 1e9
+        bwd = {"value": round(tokens / (b_ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s", "ms_per_step": round(b_ms, 3),
+               "steps": n_b, "kernel": "gdr_chunk_bwd",
+               "train_step_mtokens_s": round(tokens / ((b_ms + total_ms_max / args.steps) * 1e-3) / 1e6, 3),
+               "roofline": {"bound": "hbm", "achieved": round(b_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": round(b_gbs / peaks["hbm_gbs"], 4), "algorithmic_bytes_per_launch": int(b_bytes)}}
+        del bws
+
     # ---- the other forward workloads, each timed the same way on its own inputs ----
     workloads = None
     if not args.no_workloads:
@@ -451,6 +489,7 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": main["launches"],
         "decode": decode,
+        "backward": bwd,
         "untied": untied,
         "qk_l2norm": l2norm,
         "chunk_mean": cmean,
@@ -536,13 +575,14 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--algo", choices=["auto", "simt", "tcgen05", "tcgen05_split", "tcgen05_waves",
-                                       "tcgen05_segments"], default="auto")
+                                       "tcgen05_segments", "tcgen05_chains"], default="auto")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-workloads", action="store_true", help="skip the other forward workloads")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward pass")
     ap.add_argument("--no-untied", action="store_true", help="skip the separate-write-strength, "
                     "fused-L2-norm and chunk-mean measurements")
     args = ap.parse_args(argv)

@@ -63,7 +63,8 @@ typedef enum {
     GDR_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
     GDR_ERR_TIMEOUT = 4,     /* a kernel gave up on a bounded wait (device status word) */
     GDR_ERR_WORKSPACE = 5,   /* workspace pointer NULL or smaller than required */
-    GDR_ERR_RANGE = 6        /* a decay factor left the factored range (device status word) */
+    GDR_ERR_RANGE = 6,       /* a decay factor left the factored range (device status word) */
+    GDR_ERR_BOUNDS = 7       /* an index check of the debug build failed (device status word) */
 } gdr_status;
 
 typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
@@ -71,28 +72,35 @@ typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
 typedef enum { GDR_GATE_LOGDECAY = 0, GDR_GATE_NEG_SOFTPLUS = 1 } gdr_gate_mode;
 
 typedef enum {
-    GDR_ALGO_AUTO = 0,    /* the split tensor-core kernel for bf16 q/k/v, dk = dv = 128 and
-                             T > 64 (any number of heads), in its sequence-parallel form
-                             (GDR_ALGO_TCGEN05_SEGMENTS) when a few heads have long sequences,
-                             so that one chain per head would be the bound; the fused kernel for
-                             a single chunk; the CUDA-core kernel for every other shape and for
-                             fp32 mode */
+    GDR_ALGO_AUTO = 0,    /* for bf16 q/k/v and dk = dv = 128: the fused kernel for a single
+                             chunk; the sequence-parallel form (GDR_ALGO_TCGEN05_SEGMENTS) when a
+                             few heads have long sequences, so that one chain per head would be
+                             the bound; else the split kernel when 2*B*H <= SM count, the waves
+                             mix when B*H exceeds the SM count and its remainder would take the
+                             split kernel, the fused kernel otherwise.  The CUDA-core kernel for
+                             every other shape and for fp32 mode */
     GDR_ALGO_SIMT = 1,    /* fp32 CUDA-core chunk-WY kernel (every supported shape) */
     GDR_ALGO_TCGEN05 = 2, /* tcgen05/TMEM chunk-WY kernel, one CTA per (batch, head):
                              bf16 q/k/v, dk = dv = 128 */
-    GDR_ALGO_TCGEN05_SPLIT = 3 /* same method on a cooperative grid of one CTA per SM:
-                             nc CTAs run the state chains (heads in waves of nc, one after
-                             another), every other SM prepares chunks, handed over through a
-                             ring in the workspace; results agree with GDR_ALGO_TCGEN05 to
+    GDR_ALGO_TCGEN05_SPLIT = 3 /* same method; one CTA per head runs only the state chain
+                             while every other SM prepares chunks (two at a time), handed
+                             over through a ring in the workspace (needs B*H < SM count;
+                             cooperative launch); results agree with GDR_ALGO_TCGEN05 to
                              rounding */,
-    GDR_ALGO_TCGEN05_WAVES = 4 /* the fused kernel for whole waves of SM-count heads, then the
-                             split kernel for the heads of a last partial wave (workspace for
-                             that part) */,
+    GDR_ALGO_TCGEN05_WAVES = 4 /* more heads than SMs: the fused kernel for whole waves of
+                             SM-count heads, then the split kernel for the last partial wave
+                             when it is at most half the SM count (else fused throughout);
+                             workspace for the split part */,
     GDR_ALGO_TCGEN05_SEGMENTS = 5 /* sequence-parallel: each head's sequence is cut into
                              desc->segments segments (0: chosen by the library) that run as
                              separate chains, from the zero state and from the identity; an
                              affine scan over the segments and an output correction combine
-                             them (see gdr_chunk_fwd) */
+                             them (see gdr_chunk_fwd) */,
+    GDR_ALGO_TCGEN05_CHAINS = 6 /* the chain kernel the segments run on, for any number of
+                             heads: a cooperative grid of one CTA per SM, nc of them state chains
+                             (heads in waves of nc, one after another, nc from a cost model) and
+                             every other SM a prep worker whose elementwise and solve warp groups
+                             work on consecutive chunks; T > 64 */
 } gdr_algo;
 
 /* Shape and mode of one chunked forward call. */
@@ -388,6 +396,13 @@ GDR_API gdr_status gdr_chunk_bwd(const gdr_fwd_desc* desc,
  * memory and returns, and gdr_query_device_status reports GDR_ERR_TIMEOUT.  Outputs of
  * such a launch are not valid.  Nothing faults or traps.
  */
+/* Debug build (libgdr_debug.so, compiled with -DGDR_BOUNDS_CHECK): every kernel tests the
+ * index of each global-memory access that it computes (ring slots and flags, outputs, the
+ * states, beta) before making it; a failing test skips the access, records its site number and
+ * sets the status word's bounds bit (gdr_query_device_status -> GDR_ERR_BOUNDS).  Returns and
+ * clears the first failing site (0: none), or -1 in the default build, which has no checks. */
+GDR_API int gdr_debug_bounds_site(void);
+
 GDR_API void gdr_debug_set_tc_fault(int skip_first_commit, unsigned long long wait_limit_ns);
 
 #ifdef __cplusplus

@@ -302,6 +302,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_kernel(BwdParams p) {
     const int tid = (int)threadIdx.x;
     const int head = (int)blockIdx.x, b = head / p.H, h = head % p.H;
     const int nc = (p.T + C - 1) / C;
+    if (!GDR_INB(head < p.B * p.H, 401)) return;     // (the whole CTA)
     float* W = p.ws + (size_t)head * p.head_floats;
     if (tid == 0) range_f = 0;
     // ---- forward sweep: chunk start states ---------------------------------------------------

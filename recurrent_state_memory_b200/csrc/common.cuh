@@ -12,6 +12,25 @@ namespace gdr {
 // cleared by gdr_query_device_status.  (All kernels live in one translation unit.)
 __device__ unsigned int g_device_status = 0;
 
+// Index checks of the debug build (compiled with -DGDR_BOUNDS_CHECK).  GDR_INB(cond, site)
+// guards one global-memory access: when cond fails, the site number goes to g_bounds_site (the
+// first failure is kept), bit 2 of the status word is set and the access is skipped.  In the
+// default build the macro is the constant true and costs nothing.
+constexpr unsigned STATUS_BOUNDS = 4u;
+__device__ unsigned int g_bounds_site = 0;
+#ifdef GDR_BOUNDS_CHECK
+__device__ __forceinline__ bool in_bounds(bool c, unsigned site) {
+    if (!c) {
+        atomicCAS(&g_bounds_site, 0u, site);
+        atomicOr(&g_device_status, STATUS_BOUNDS);
+    }
+    return c;
+}
+#define GDR_INB(cond, site) ::gdr::in_bounds((cond), (site))
+#else
+#define GDR_INB(cond, site) true
+#endif
+
 // Element loads/stores with the storage type chosen at compile time.
 template <typename T> __device__ __forceinline__ float ld_f32(const T* p);
 template <> __device__ __forceinline__ float ld_f32<float>(const float* p) { return *p; }

@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_kernel(DecParams p) {
     const QT* q = static_cast<const QT*>(p.q) + (size_t)nh * DK;
     const QT* k = static_cast<const QT*>(p.k) + (size_t)nh * DK;
     const QT* v = static_cast<const QT*>(p.v) + (size_t)nh * p.dv;
+    if (!GDR_INB(nh < p.N * p.H, 301)) return;      // (the whole CTA: nh is the same for all its threads)
     OT* o = static_cast<OT*>(p.o) + (size_t)nh * p.dv;
     float* S = p.S + (size_t)nh * p.dv * DK;
 

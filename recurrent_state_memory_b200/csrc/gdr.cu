@@ -110,42 +110,62 @@ static void split_geometry(const FwdParams& p, long long* nv, long long* nchunks
     *nv = (long long)p.nheads * ns;
     *nchunks = p.nseg > 1 ? p.seg_len / 64 : (p.T + 63) / 64;
 }
-static bool split_fits_heads(long long nh, int sms, int T) { return nh >= 1 && sms >= 2 && T > 64; }
+// The split kernel (tcf, one chain CTA per head) shares the SMs without a chain among prep
+// workers; with more than half of the SMs taken by chains, too few workers are left and the
+// fused kernel (prep and chain of a head in one CTA) is faster.
+static bool split_fits_heads(long long nh, int sms, int T) { return nh >= 1 && 2 * nh <= (long long)sms && T > 64; }
 static bool split_fits(const gdr_fwd_desc* d, int sms) {
     return split_fits_heads((long long)d->B * d->H, sms, d->T);
 }
-// GDR_ALGO_TCGEN05_WAVES: the fused kernel for whole waves of SM-count heads and the split
-// kernel for the heads of a last partial wave.
+// More heads than SMs: the fused kernel runs whole waves of SM-count heads; a last partial
+// wave that would leave more than half of the SMs idle goes to the split kernel instead.
 static long long waves_remainder(const gdr_fwd_desc* d, int sms) {
     const long long nh = (long long)d->B * d->H;
     return nh > sms ? nh % sms : 0;
 }
+static bool waves_fit(const gdr_fwd_desc* d, int sms) {
+    const long long rem = waves_remainder(d, sms);
+    return rem > 0 && split_fits_heads(rem, sms, d->T);
+}
+// The chains kernel (spl) takes any number of heads (each chain runs its heads one after
+// another) and the segments of the sequence-parallel form.
+static bool chains_fit(const gdr_fwd_desc* d, int sms) { return (long long)d->B * d->H >= 1 && sms >= 2 && d->T > 64; }
 
 static bool segments_pay(long long nh, long long T, int sms);
 
-// The algorithm a descriptor runs with: AUTO takes the split tensor-core kernel when it
-// supports the shape and dtype and the sequence has more than one chunk, the fused one for a
-// single chunk, the CUDA-core kernel otherwise.
+// The algorithm a descriptor runs with.  AUTO: the CUDA-core kernel for shapes and dtypes the
+// tensor-core kernels do not take; the fused kernel for a single chunk; the sequence-parallel
+// form when its model puts it well ahead (few heads, long sequences); else the split kernel when
+// the heads leave room for prep workers, the waves mix when a partial last wave would leave
+// most SMs idle, the fused kernel otherwise.
 static gdr_algo resolve_algo(const gdr_fwd_desc* d) {
     if (d->algo == GDR_ALGO_AUTO) {
         if (!tc_supported(d)) return GDR_ALGO_SIMT;
         const int sms = device_sm_count();
-        if (!split_fits(d, sms)) return GDR_ALGO_TCGEN05;
-        return segments_pay((long long)d->B * d->H, d->T, sms) ? GDR_ALGO_TCGEN05_SEGMENTS : GDR_ALGO_TCGEN05_SPLIT;
+        if (d->T <= 64) return GDR_ALGO_TCGEN05;
+        if (segments_pay((long long)d->B * d->H, d->T, sms)) return GDR_ALGO_TCGEN05_SEGMENTS;
+        if (split_fits(d, sms)) return GDR_ALGO_TCGEN05_SPLIT;
+        return waves_fit(d, sms) ? GDR_ALGO_TCGEN05_WAVES : GDR_ALGO_TCGEN05;
     }
     return d->algo;
 }
 
-static size_t split_workspace_heads(size_t nh, int T) {
-    return spl::workspace_bytes((size_t)plan_chains((long long)nh, (T + 63) / 64, device_sm_count()));
+static size_t split_workspace_heads(size_t nh) {
+    return nh * tcf::RING * tcf::SLOT_BYTES + tcf::split_flag_words(nh) * sizeof(unsigned int);
 }
-static size_t split_workspace_bytes(const gdr_fwd_desc* d) { return split_workspace_heads((size_t)d->B * d->H, d->T); }
+static size_t split_workspace_bytes(const gdr_fwd_desc* d) { return split_workspace_heads((size_t)d->B * d->H); }
+static size_t chains_workspace_bytes(const gdr_fwd_desc* d) {
+    const long long nh = (long long)d->B * d->H;
+    return spl::workspace_bytes((size_t)plan_chains(nh, (d->T + 63) / 64, device_sm_count()));
+}
 
 // ---- scratch for gdr_chunk_fwd_noalloc ---------------------------------------------------
 // The split kernel's ring and flags for at most NOALLOC_MAX_HEADS heads, as a file-scope
 // device array: every GPU that loads this library holds these bytes until the process exits.
 constexpr int NOALLOC_MAX_HEADS = GDR_NOALLOC_MAX_HEADS;
-constexpr size_t NOALLOC_BYTES = spl::workspace_bytes(NOALLOC_MAX_HEADS);
+constexpr size_t NOALLOC_BYTES =
+    (size_t)NOALLOC_MAX_HEADS * tcf::RING * tcf::SLOT_BYTES +
+    tcf::split_flag_words(NOALLOC_MAX_HEADS) * sizeof(unsigned int);
 static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_BYTES];
 
 // The current context's unique id (the driver's cuCtxGetId), so that per-device caches can
@@ -226,13 +246,14 @@ static gdr_status check_fwd_desc(const gdr_fwd_desc* d) {
     if (d->rotation != 0 && d->rotation != 1) return fail(GDR_ERR_INVALID_ARG, "rotation must be 0 or 1%s");
     if (d->qk_l2norm != 0 && d->qk_l2norm != 1) return fail(GDR_ERR_INVALID_ARG, "qk_l2norm must be 0 or 1%s");
     if (d->algo != GDR_ALGO_AUTO && d->algo != GDR_ALGO_SIMT && d->algo != GDR_ALGO_TCGEN05 &&
-        d->algo != GDR_ALGO_TCGEN05_SPLIT && d->algo != GDR_ALGO_TCGEN05_WAVES && d->algo != GDR_ALGO_TCGEN05_SEGMENTS)
+        d->algo != GDR_ALGO_TCGEN05_SPLIT && d->algo != GDR_ALGO_TCGEN05_WAVES && d->algo != GDR_ALGO_TCGEN05_SEGMENTS &&
+        d->algo != GDR_ALGO_TCGEN05_CHAINS)
         return fail(GDR_ERR_INVALID_ARG, "bad algo%s");
     if (d->segments < 0 || d->segments == 1 || d->segments > 4096)
         return fail(GDR_ERR_INVALID_ARG, "segments must be 0 (library's choice) or 2 .. 4096%s");
     if ((long long)d->B * d->H > 0x7fffffffLL) return fail(GDR_ERR_INVALID_ARG, "B*H too large%s");
     if ((d->algo == GDR_ALGO_TCGEN05 || d->algo == GDR_ALGO_TCGEN05_SPLIT || d->algo == GDR_ALGO_TCGEN05_WAVES ||
-         d->algo == GDR_ALGO_TCGEN05_SEGMENTS) &&
+         d->algo == GDR_ALGO_TCGEN05_SEGMENTS || d->algo == GDR_ALGO_TCGEN05_CHAINS) &&
         !tc_supported(d))
         return fail(GDR_ERR_UNSUPPORTED, "the tcgen05 kernels need bf16 q/k/v and dk = dv = 128%s");
     return GDR_OK;
@@ -297,24 +318,85 @@ static gdr_status encode_split_maps(const FwdParams& p, spl::Maps* tm) {
     return GDR_OK;
 }
 
-template <bool ROT, typename OT, bool EXT>
-static gdr_status launch_tc(const FwdParams& p, cudaStream_t st) {
-    auto kern = tcf::chunk_fwd_tc_kernel<ROT, OT, EXT>;
-    constexpr int nt = tcf::NT;
-    constexpr uint32_t smem = tcf::SMEM_BYTES;
+template <bool ROT, typename OT>
+static gdr_status encode_tc_maps(const FwdParams& p, tcf::TmaMaps* tm) {
+    EncodeTiledFn fn = nullptr;
+    gdr_status s = encode_fn(&fn);
+    if (s != GDR_OK) return s;
+    const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const int D = tcf::D, NG = ROT ? tcf::D / 2 : tcf::D;
+    if ((s = encode_bthd(fn, &tm->q, p.q, bf, 2, p, D, D, false)) != GDR_OK) return s;
+    if ((s = encode_bthd(fn, &tm->k, p.k, bf, 2, p, D, D, false)) != GDR_OK) return s;
+    if ((s = encode_bthd(fn, &tm->g, p.g, f32, 4, p, NG, NG, false)) != GDR_OK) return s;
+    if (ROT && (s = encode_bthd(fn, &tm->th, p.theta, f32, 4, p, NG, NG, false)) != GDR_OK) return s;
+    if ((s = encode_bthd(fn, &tm->v, p.v, bf, 2, p, D, 64, true)) != GDR_OK) return s;
+    const bool ob = sizeof(OT) == 2;
+    return encode_bthd(fn, &tm->o, p.o, ob ? bf : f32, sizeof(OT), p, D, D, false);
+}
+
+template <int MODE, bool ROT, typename OT, bool EXT>
+static gdr_status launch_tc(const FwdParams& p, cudaStream_t st, void* ws) {
+    auto kern = tcf::chunk_fwd_tc_kernel<MODE, ROT, OT, EXT>;
+    constexpr int nt = tcf::nthreads<MODE>();
+    constexpr uint32_t smem = tcf::smem_bytes<MODE>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tcgen05 chunk kernel)");
     tcf::TcExtra x;
     x.wait_limit_ns = s_wait_limit_ns;
     x.fault_skip_commit = s_fault_skip_commit;
-    kern<<<p.nheads, nt, smem, st>>>(p, x);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
+    tcf::SplitArgs sa{nullptr, nullptr, nullptr};
+    tcf::TmaMaps tm;
+    memset(&tm, 0, sizeof(tm));
+    if (MODE == 0) {
+        kern<<<p.nheads, nt, smem, st>>>(p, x, sa, tm);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "launch(tcgen05 chunk kernel)");
+        return GDR_OK;
+    }
+    // Split: the whole grid must be resident at once (one CTA per SM), which a cooperative
+    // launch guarantees or refuses.
+    const int nh = p.nheads;
+    const int sms = device_sm_count();
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    const int grid = sms * (per_sm < 1 ? 1 : per_sm > 1 ? 1 : per_sm);
+    if (per_sm < 1 || grid <= nh) return fail(GDR_ERR_UNSUPPORTED, "split kernel: B*H must be below the SM count%s");
+    gdr_status s = encode_tc_maps<ROT, OT>(p, &tm);
+    if (s != GDR_OK) return s;
+    const size_t nring = (size_t)nh * tcf::RING * tcf::SLOT_BYTES;
+    sa.ring = static_cast<uint8_t*>(ws);
+    sa.ready = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + nring);
+    sa.consumed = sa.ready + (size_t)nh * tcf::RING;
+    sa.next_task = sa.consumed + nh;
+    // Worker order: from the counter while the worker groups fill at most half the ring's
+    // slots (the workers are then the bound and the counter evens out their load); at a
+    // fixed stride otherwise (measured faster there: it paces each group to the chains).
+    sa.dynamic = (2 * (grid - nh) <= nh * tcf::RING / 2) ? 1 : 0;
+    sa.discard = (reinterpret_cast<uintptr_t>(ws) & 127u) == 0 ? 1 : 0;
+    e = cudaMemsetAsync(sa.ready, 0, tcf::split_flag_words(nh) * sizeof(unsigned int), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split flags)");
+    void* args[] = {const_cast<FwdParams*>(&p), &x, &sa, &tm};
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(nt), args, smem, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cooperative launch(tcgen05 split kernel)");
     return GDR_OK;
 }
 
+template <int MODE>
+static gdr_status dispatch_tc_mode(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws) {
+    const bool ob = d->out_dtype == GDR_BF16;
+    if (p.w || p.qk_norm || p.chunk_mean) {      // the kernel with the optional features
+        if (d->rotation)
+            return ob ? launch_tc<MODE, true, __nv_bfloat16, true>(p, st, ws) : launch_tc<MODE, true, float, true>(p, st, ws);
+        return ob ? launch_tc<MODE, false, __nv_bfloat16, true>(p, st, ws) : launch_tc<MODE, false, float, true>(p, st, ws);
+    }
+    if (d->rotation)
+        return ob ? launch_tc<MODE, true, __nv_bfloat16, false>(p, st, ws) : launch_tc<MODE, true, float, false>(p, st, ws);
+    return ob ? launch_tc<MODE, false, __nv_bfloat16, false>(p, st, ws) : launch_tc<MODE, false, float, false>(p, st, ws);
+}
+
 template <bool ROT, typename OT, bool EXT>
-static gdr_status launch_split(const FwdParams& p, cudaStream_t st, void* ws) {
+static gdr_status launch_chains(const FwdParams& p, cudaStream_t st, void* ws) {
     auto kern = spl::split_fwd_kernel<ROT, OT, EXT>;
     constexpr uint32_t smem = spl::SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -350,6 +432,7 @@ static gdr_status launch_split(const FwdParams& p, cudaStream_t st, void* ws) {
     cf.dynamic = t_work >= t_chain ? 1 : 0;
     cf.wait_limit_ns = s_wait_limit_ns;
     cf.fault_skip_commit = s_fault_skip_commit;
+    cf.discard = (reinterpret_cast<uintptr_t>(ws) & 127u) == 0 ? 1 : 0;
     e = cudaMemsetAsync(cf.ready, 0, spl::flag_words((size_t)nc) * sizeof(unsigned int), st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split flags)");
     void* args[] = {const_cast<FwdParams*>(&p), &cf, &tm};
@@ -358,27 +441,25 @@ static gdr_status launch_split(const FwdParams& p, cudaStream_t st, void* ws) {
     return GDR_OK;
 }
 
-// The kernel instantiation with the optional features (a separate write strength, the fused L2
-// normalisation, the chunk means of o) runs only when one of them is asked for.
 static gdr_status dispatch_fused(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st) {
-    const bool ob = d->out_dtype == GDR_BF16;
-    if (p.w || p.qk_norm || p.chunk_mean) {
-        if (d->rotation) return ob ? launch_tc<true, __nv_bfloat16, true>(p, st) : launch_tc<true, float, true>(p, st);
-        return ob ? launch_tc<false, __nv_bfloat16, true>(p, st) : launch_tc<false, float, true>(p, st);
-    }
-    if (d->rotation) return ob ? launch_tc<true, __nv_bfloat16, false>(p, st) : launch_tc<true, float, false>(p, st);
-    return ob ? launch_tc<false, __nv_bfloat16, false>(p, st) : launch_tc<false, float, false>(p, st);
+    return dispatch_tc_mode<0>(d, p, st, nullptr);
+}
+static gdr_status dispatch_split(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws) {
+    return dispatch_tc_mode<1>(d, p, st, ws);
 }
 
-static gdr_status dispatch_split(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws,
-                                 bool f32_out = false) {
+// The chains kernel; f32_out writes o in fp32 whatever the descriptor's output dtype (the
+// segments' second pass).  The instantiation with the optional features runs only when one of
+// them is asked for.
+static gdr_status dispatch_chains(const gdr_fwd_desc* d, const FwdParams& p, cudaStream_t st, void* ws,
+                                  bool f32_out = false) {
     const bool ob = d->out_dtype == GDR_BF16 && !f32_out;
     if (p.w || p.qk_norm || p.chunk_mean) {
-        if (d->rotation) return ob ? launch_split<true, __nv_bfloat16, true>(p, st, ws) : launch_split<true, float, true>(p, st, ws);
-        return ob ? launch_split<false, __nv_bfloat16, true>(p, st, ws) : launch_split<false, float, true>(p, st, ws);
+        if (d->rotation) return ob ? launch_chains<true, __nv_bfloat16, true>(p, st, ws) : launch_chains<true, float, true>(p, st, ws);
+        return ob ? launch_chains<false, __nv_bfloat16, true>(p, st, ws) : launch_chains<false, float, true>(p, st, ws);
     }
-    if (d->rotation) return ob ? launch_split<true, __nv_bfloat16, false>(p, st, ws) : launch_split<true, float, false>(p, st, ws);
-    return ob ? launch_split<false, __nv_bfloat16, false>(p, st, ws) : launch_split<false, float, false>(p, st, ws);
+    if (d->rotation) return ob ? launch_chains<true, __nv_bfloat16, false>(p, st, ws) : launch_chains<true, float, false>(p, st, ws);
+    return ob ? launch_chains<false, __nv_bfloat16, false>(p, st, ws) : launch_chains<false, float, false>(p, st, ws);
 }
 
 // ---- sequence-parallel forward (segments) ---------------------------------------------------
@@ -459,20 +540,20 @@ static gdr_status run_segments(const gdr_fwd_desc* d, const FwdParams& p, cudaSt
     seg_plan(d, device_sm_count(), &P);
     uint8_t* w = static_cast<uint8_t*>(ws);
     FwdParams p1 = p;
-    if (P.nseg <= 1) return dispatch_split(d, p1, st, ws);
+    if (P.nseg <= 1) return dispatch_chains(d, p1, st, ws);
     float* Bz = reinterpret_cast<float*>(w + P.off_bz);
     float* A = reinterpret_cast<float*>(w + P.off_a);
     float* St = reinterpret_cast<float*>(w + P.off_st);
     float* y = reinterpret_cast<float*>(w + P.off_y);
     p1.nseg = P.nseg; p1.seg_len = P.seg_len; p1.seg0 = 0; p1.s0_identity = 0;
     p1.S_T = Bz;
-    gdr_status s = dispatch_split(d, p1, st, w);                   // o0, chunk means of o0, Bz
+    gdr_status s = dispatch_chains(d, p1, st, w);                  // o0, chunk means of o0, Bz
     if (s != GDR_OK) return s;
     FwdParams p2 = p1;
     p2.seg0 = 1; p2.s0_identity = 1;
     p2.v = nullptr; p2.w = nullptr; p2.S0 = nullptr; p2.chunk_mean = nullptr;
     p2.o = y; p2.S_T = A;
-    s = dispatch_split(d, p2, st, w, true);                        // y (fp32), A
+    s = dispatch_chains(d, p2, st, w, true);                       // y (fp32), A
     if (s != GDR_OK) return s;
     seg::ScanParams sp{p.nheads, P.nseg, Bz, A, St, p.S_T};
     cudaError_t e = cudaFuncSetAttribute(seg::seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -661,6 +742,7 @@ const char* gdr_status_string(gdr_status s) {
         case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
         case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE";
         case GDR_ERR_RANGE: return "GDR_ERR_RANGE";
+        case GDR_ERR_BOUNDS: return "GDR_ERR_BOUNDS";
     }
     return "GDR_ERR_UNKNOWN";
 }
@@ -671,6 +753,7 @@ size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc) {
     if (check_fwd_desc(desc) != GDR_OK) return 0;
     const gdr_algo a = resolve_algo(desc);
     if (a == GDR_ALGO_TCGEN05_SPLIT) return split_workspace_bytes(desc);
+    if (a == GDR_ALGO_TCGEN05_CHAINS) return desc->T > 64 ? chains_workspace_bytes(desc) : 0;
     if (a == GDR_ALGO_TCGEN05_SEGMENTS) {
         if (desc->T <= 0) return 0;
         SegPlan P;
@@ -681,7 +764,7 @@ size_t gdr_chunk_fwd_workspace_bytes(const gdr_fwd_desc* desc) {
         // only a last partial wave that the split kernel runs needs the ring
         const int sms = device_sm_count();
         const long long rem = waves_remainder(desc, sms);
-        return (rem > 0 && split_fits_heads(rem, sms, desc->T)) ? split_workspace_heads((size_t)rem, desc->T) : 0;
+        return (rem > 0 && split_fits_heads(rem, sms, desc->T)) ? split_workspace_heads((size_t)rem) : 0;
     }
     return 0;
 }
@@ -739,6 +822,10 @@ gdr_status gdr_chunk_fwd_ex(const gdr_fwd_desc* d, const void* q, const void* k,
         if (!aligned16(workspace)) return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned%s");
         return dispatch_split(d, p, st, workspace);
     }
+    if (algo == GDR_ALGO_TCGEN05_CHAINS && d->T > 64) {
+        if (!aligned16(workspace)) return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned%s");
+        return dispatch_chains(d, p, st, workspace);
+    }
     if (algo == GDR_ALGO_TCGEN05_SEGMENTS && d->T > 0) {
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
             return fail(GDR_ERR_INVALID_ARG, "workspace must be 256-byte aligned for GDR_ALGO_TCGEN05_SEGMENTS%s");
@@ -759,7 +846,7 @@ gdr_status gdr_chunk_fwd_ex(const gdr_fwd_desc* d, const void* q, const void* k,
         return dispatch_fused(d, p, st);
     }
     if (algo == GDR_ALGO_TCGEN05 || algo == GDR_ALGO_TCGEN05_SPLIT || algo == GDR_ALGO_TCGEN05_WAVES ||
-        algo == GDR_ALGO_TCGEN05_SEGMENTS)
+        algo == GDR_ALGO_TCGEN05_SEGMENTS || algo == GDR_ALGO_TCGEN05_CHAINS)
         return dispatch_fused(d, p, st);
     return d->rotation ? dispatch_simt_dk<true>(d, p, st) : dispatch_simt_dk<false>(d, p, st);
 }
@@ -823,9 +910,24 @@ gdr_status gdr_query_device_status(gdr_stream_t stream) {
         e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(status)");
         snprintf(t_detail, sizeof(t_detail), "device status word 0x%08x", word);
-        return (word & tcf::STATUS_TIMEOUT) ? GDR_ERR_TIMEOUT : GDR_ERR_RANGE;
+        if (word & tcf::STATUS_TIMEOUT) return GDR_ERR_TIMEOUT;
+        return (word & STATUS_BOUNDS) ? GDR_ERR_BOUNDS : GDR_ERR_RANGE;
     }
     return GDR_OK;
+}
+
+int gdr_debug_bounds_site(void) {
+#ifdef GDR_BOUNDS_CHECK
+    unsigned int site = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&site, g_bounds_site, sizeof(site)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_bounds_site, &zero, sizeof(zero)) != cudaSuccess) {
+        cudaGetLastError();
+        return -2;
+    }
+    return (int)site;
+#else
+    return -1;
+#endif
 }
 
 int gdr_chunk_fwd_algo(const gdr_fwd_desc* desc) {

@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(SCAN_NT) seg_scan_kernel(ScanParams sp) {
         for (int u = 0; u < 8; ++u) sS[rr * D + cb + u] = acc[u];
         __syncthreads();
     }
-    if (sp.S_T) {
+    if (sp.S_T && GDR_INB(h < sp.nheads && r0 + RB <= D, 201)) {
         for (int e = t; e < RB * D; e += SCAN_NT) sp.S_T[(size_t)h * DD + (size_t)(r0 + e / D) * D + e % D] = sS[e];
     }
 }
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(CORR_NT, 1) seg_correct_kernel(CorrParams cp, 
                     for (int e = 0; e < 8; ++e) v8[e] = vals[blk8 * 8 + e];
                     transpose8x8(v8, j8);
                     const int r = g * 32 + blk8 * 8 + j8;
-                    if (t0 + r < cp.T) {
+                    if (t0 + r < cp.T && GDR_INB(gx < cp.B * cp.H, 204)) {
                         OT* dst = obase + (size_t)r * tstride;
                         if constexpr (sizeof(OT) == 2) {
                             const uint4 cur = *reinterpret_cast<const uint4*>(dst);

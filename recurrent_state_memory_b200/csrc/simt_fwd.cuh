@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(NT) chunk_fwd_kernel(FwdParams p) {
             if (r < Lc) {
                 float acc = QS[r * (DVT + 1) + j];
                 for (int i = 0; i <= r; ++i) acc = fmaf(Pm[r * (C + 1) + i], R[i * (DVT + 1) + j], acc);
-                st_from_f32(o + tok(r) * dv + j0 + j, acc);
+                if (GDR_INB(t0 + r < p.T && bh < p.B * p.H && j0 + j < dv, 501)) st_from_f32(o + tok(r) * dv + j0 + j, acc);
                 msum += acc;
             }
         }
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(NT) chunk_fwd_kernel(FwdParams p) {
         }
     }
     __syncthreads();
-    if (p.S_T) {
+    if (p.S_T && GDR_INB(bh < p.B * p.H && j0 + DVT <= dv, 502)) {
         for (int idx = tid; idx < DVT * DK; idx += NT) {
             const int j = idx / DK, d = idx % DK;
             p.S_T[((size_t)bh * dv + j0 + j) * DK + d] = S[j * KS + d];

@@ -131,6 +131,7 @@ struct Cfg {
     int dynamic;               // 1: tasks from the counter; 0: worker w takes w, w + W, ...
     unsigned long long wait_limit_ns;
     int fault_skip_commit;     // test hook: the first MMA completion of each worker is never signalled
+    int discard;               // 1: the ring is 128-byte aligned, so consumed slots are dropped from L2
 };
 
 // Flag words after the ring (zeroed before every launch): ready, consumed, next_task.
@@ -320,8 +321,9 @@ __device__ __forceinline__ void worker_elementwise(const FwdParams& p, const Cfg
         const int tc0 = vh_t0(p, geo, tk.gh) + tk.c * C;     // first token of the chunk
         const int Lc = vh_chunk_len(p, geo, tk.gh, tk.c);
         uint8_t* slot = cf.ring + ((size_t)tk.j * RING + tk.s % RING) * SLOT_BYTES;
+        const bool slot_ok = GDR_INB(tk.j >= 0 && tk.j < NC && tk.s >= 0, 101);
         float beta_r = 0.f, w_r = 0.f;
-        if (tid < Lc) {
+        if (tid < Lc && GDR_INB(gx < p.B * p.H && tc0 + tid < p.T, 102)) {
             beta_r = __ldg(p.beta + tok_row(p, gx, tc0 + tid));
             w_r = untied ? __ldg(p.w + tok_row(p, gx, tc0 + tid)) : beta_r;
         }
@@ -416,7 +418,8 @@ __device__ __forceinline__ void worker_elementwise(const FwdParams& p, const Cfg
 
         // ---- reference decays: P_m (tokens 0..31) and P_m^{-1} P_C (tokens 32..63) -> ring ----
         float* rvec = reinterpret_cast<float*>(slot + SL_VEC);
-        if (!ROT) {
+        if (!slot_ok) {
+        } else if (!ROT) {
             if (tid < 128) {
                 const int d = tid;
                 float lo = 1.f, hi = 1.f;
@@ -503,7 +506,7 @@ __device__ __forceinline__ void worker_elementwise(const FwdParams& p, const Cfg
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const uint32_t d = (uint32_t)(4 * dg + e);
-                    *reinterpret_cast<float4*>(slot + SL_H + kb2 * 16384u + sw128_off(d, c16)) =
+                    if (slot_ok) *reinterpret_cast<float4*>(slot + SL_H + kb2 * 16384u + sw128_off(d, c16)) =
                         make_float4(khb[0][e], khb[1][e], khb[2][e], khb[3][e]);
                 }
             };
@@ -712,6 +715,10 @@ __device__ __forceinline__ void worker_publisher(const FwdParams& p, const Cfg& 
         const Task tk = decode_task(task, NC, NV, nchunks);
         uint8_t* slot = cf.ring + ((size_t)tk.j * RING + tk.s % RING) * SLOT_BYTES;
         const uint32_t kq = sb + WK_KQ + (uint32_t)pb * 32768u;
+        if (!GDR_INB(tk.j >= 0 && tk.j < NC && tk.s >= 0, 104)) {      // neither copy nor publish
+            mbar_arrive(b_pubread + pb);
+            continue;
+        }
         bulk_s2g(slot + SL_Q, kq + 8192u, 8192u);                  // Qtil, dk 0..63
         bulk_s2g(slot + SL_Q + 8192u, kq + 16384u + 8192u, 8192u); // Qtil, dk 64..127
         bulk_s2g(slot + SL_P, sb + WK_PMS, 16384u);
@@ -1042,7 +1049,8 @@ __device__ __forceinline__ void chain_role(const FwdParams& p, const Cfg& cf, co
             }
             if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
             // the slot's bytes are here: its L2 lines are dead, drop them without write-back
-            for (uint32_t off = (uint32_t)lane * 128u; off < SLOT_BYTES; off += 32u * 128u) discard_l2_line(src + off);
+            if (cf.discard)
+                for (uint32_t off = (uint32_t)lane * 128u; off < SLOT_BYTES; off += 32u * 128u) discard_l2_line(src + off);
             __syncwarp();
             if (lane == 0) st_release_gpu(cf.consumed + j, (unsigned)(s + 1));
         }
@@ -1194,7 +1202,7 @@ __device__ __forceinline__ void chain_role(const FwdParams& p, const Cfg& cf, co
                     for (int e = 0; e < 8; ++e) v8[e] = vals[blk8 * 8 + e];
                     transpose8(v8, j8);
                     const int r = g * 32 + blk8 * 8 + j8;
-                    if (r < Lc) {
+                    if (r < Lc && GDR_INB(gx < p.B * p.H && t0 + r < p.T, 109)) {
                         OT* dst = obase + (size_t)r * tstride;
                         if constexpr (sizeof(OT) == 2) {
                             *reinterpret_cast<uint4*>(dst) = pack8(v8);
@@ -1205,7 +1213,7 @@ __device__ __forceinline__ void chain_role(const FwdParams& p, const Cfg& cf, co
                     }
                 }
             }
-            if (cmean && Lc > 0) {    // the chunk index within the whole sequence
+            if (cmean && Lc > 0 && GDR_INB(gx < p.B * p.H && t0 < p.T, 110)) {    // the chunk index within the whole sequence
                 const int nct = (p.T + C - 1) / C, cg = t0 / C;
                 p.chunk_mean[(((size_t)(gx / p.H) * nct + cg) * p.H + gx % p.H) * D + row] = msum / (float)Lc;
             }
@@ -1256,7 +1264,7 @@ __device__ __forceinline__ void chain_role(const FwdParams& p, const Cfg& cf, co
             if (p.s0_identity) {
 #pragma unroll
                 for (int u = 0; u < 64; ++u) v[u] = (c0 + u == row) ? 1.f : 0.f;
-            } else if (from_s0) {
+            } else if (from_s0 && GDR_INB(gx < p.B * p.H, 112)) {
                 const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)gx * D + row) * D + c0);
 #pragma unroll
                 for (int u4 = 0; u4 < 16; ++u4) {
@@ -1309,7 +1317,7 @@ __device__ __forceinline__ void chain_role(const FwdParams& p, const Cfg& cf, co
             } else {
                 // S_T: one per head, or one per virtual head when segments run separately
                 const int sx = p.nseg > 1 ? vh_of(s) : head_of(s);
-                if (p.S_T) {
+                if (p.S_T && GDR_INB(sx < (p.nseg > 1 ? geo.nv : p.B * p.H), 111)) {
                     float4* dst = reinterpret_cast<float4*>(p.S_T + ((size_t)sx * D + row) * D + c0);
 #pragma unroll
                     for (int u4 = 0; u4 < 16; ++u4)

@@ -21,10 +21,11 @@ LIB_PATH = os.path.join(_HERE, "libgdr.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gdr.h")
 
 (GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_CUDA, GDR_ERR_TIMEOUT, GDR_ERR_WORKSPACE,
- GDR_ERR_RANGE) = range(7)
+ GDR_ERR_RANGE, GDR_ERR_BOUNDS) = range(8)
 GDR_F32, GDR_BF16 = 0, 1
 GATE_LOGDECAY, GATE_NEG_SOFTPLUS = 0, 1
-ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_split": 3, "tcgen05_waves": 4, "tcgen05_segments": 5}
+ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_split": 3, "tcgen05_waves": 4, "tcgen05_segments": 5,
+         "tcgen05_chains": 6}
 ALGO_NAMES = {v: k for k, v in ALGOS.items()}
 
 
@@ -88,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_chunk_fwd_algo.argtypes = [ctypes.POINTER(FwdDesc)]
         L.gdr_chunk_fwd_kernel_launches.restype = ctypes.c_int
         L.gdr_chunk_fwd_kernel_launches.argtypes = [ctypes.POINTER(FwdDesc)]
+        L.gdr_debug_bounds_site.restype = ctypes.c_int
+        L.gdr_debug_bounds_site.argtypes = []
         L.gdr_chunk_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.gdr_chunk_bwd_workspace_bytes.argtypes = [ctypes.POINTER(FwdDesc)]
         L.gdr_chunk_bwd.restype = ctypes.c_int
@@ -165,6 +168,19 @@ def kernel_launches(desc: FwdDesc) -> int:
     if n < 0:
         raise ValueError("invalid descriptor")
     return n
+
+
+def use_library(path: str) -> None:
+    """Load the library from `path` from now on (the debug build with index checks,
+    libgdr_debug.so, for example); the next call loads it."""
+    global LIB_PATH, _lib
+    LIB_PATH = path
+    _lib = None
+
+
+def debug_bounds_site() -> int:
+    """First failing index check of the debug build (0: none), cleared; -1 in the default build."""
+    return int(lib().gdr_debug_bounds_site())
 
 
 def debug_set_tc_fault(skip_first_commit: bool, wait_limit_ns: int = 0):

@@ -147,33 +147,38 @@ def test_host_entry_workspace_and_argument_checks(G):
 
 def test_auto_resolution_and_workspace_sizes_without_a_device(G):
     """With no device visible the library assumes a B200's 148 SMs.  AUTO's choice follows the
-    rules gdr.h states (the split kernel for bf16, dk = dv = 128 and T > 64, whatever the number
-    of heads, or its sequence-parallel form when a few heads have long sequences; the fused
-    kernel for a single chunk; the CUDA-core kernel for other shapes).  The
-    split workspace is nc rings of 8 slots of 91,136 bytes plus 36 bytes of flags per chain and
-    one task counter, with nc chains (1 <= nc <= min(B*H, 74)); 64 heads get one chain each."""
+    rules gdr.h states: the fused kernel for a single chunk; the sequence-parallel form for one
+    head with a long sequence; split when 2 B*H <= SMs and T > 64; whole fused waves plus a split
+    remainder when B*H > SMs and the remainder fits that rule; fused otherwise; the CUDA-core
+    kernel for other shapes.  The split workspace is B*H*8 slots of 76,288 bytes plus 36 bytes of
+    flags per head and one task counter; the chains kernel's is nc rings of 8 slots of 91,136
+    bytes plus 36 bytes of flags and one counter, with 1 <= nc <= min(B*H, 74)."""
     import torch
     if torch.cuda.is_available():
         pytest.skip("the 148-SM assumption holds only where no device is visible")
     bf = torch.bfloat16
-    d = lambda B, H, T, dk=128: G.fwd_desc(B, H, T, dk, dk, bf, bf)
-    per_chain = 8 * 91136 + 9 * 4
-
-    def chains(desc):
-        n, rem = divmod(G.workspace_bytes(desc) - 4, per_chain)
-        assert rem == 0
-        return n
-
-    assert G.resolved_algo(d(4, 16, 4096)) == "tcgen05_split" and chains(d(4, 16, 4096)) == 64
-    for B, H in ((2, 37), (1, 75), (16, 12), (2, 118)):
-        assert G.resolved_algo(d(B, H, 4096)) == "tcgen05_split"
-        assert 1 <= chains(d(B, H, 4096)) <= min(B * H, 74)
+    d = lambda B, H, T, dk=128, **kw: G.fwd_desc(B, H, T, dk, dk, bf, bf, **kw)
+    split = lambda nh: nh * 8 * 76288 + (nh * 8 + nh + 1) * 4
+    assert G.resolved_algo(d(4, 16, 4096)) == "tcgen05_split" and G.workspace_bytes(d(4, 16, 4096)) == split(64)
+    assert G.resolved_algo(d(2, 37, 4096)) == "tcgen05_split"            # 74 heads: exactly half
+    assert G.resolved_algo(d(1, 75, 4096)) == "tcgen05"                  # 75 heads: more than half
+    assert G.resolved_algo(d(4, 16, 64)) == "tcgen05"                    # a single chunk
+    assert G.resolved_algo(d(4, 16, 65)) == "tcgen05_split"              # two chunks
+    assert G.resolved_algo(d(16, 12, 4096)) == "tcgen05_waves"           # 192 = 148 + 44
+    assert G.workspace_bytes(d(16, 12, 4096)) == split(44)
+    assert G.resolved_algo(d(2, 118, 4096)) == "tcgen05"                 # 236 = 148 + 88: 88 > 74
+    assert G.workspace_bytes(d(2, 118, 4096)) == 0
     # one head with a long sequence: its chain alone would be the bound, so the sequence is cut
-    # into segments; the workspace then also holds y (fp32, one dk-vector per token)
+    # into segments (on the chains kernel); the workspace then also holds y (fp32 per token)
     assert G.resolved_algo(d(1, 1, 4096)) == "tcgen05_segments"
     assert G.workspace_bytes(d(1, 1, 4096)) >= 4096 * 128 * 4
-    assert G.resolved_algo(d(4, 16, 65)) == "tcgen05_split"              # two chunks
-    assert G.resolved_algo(d(4, 16, 64)) == "tcgen05" and G.workspace_bytes(d(4, 16, 64)) == 0   # one chunk
+    # the chains kernel on request, for any number of heads
+    per_chain = 8 * 91136 + 9 * 4
+    for B, H in ((4, 16), (2, 37), (1, 75), (16, 12), (2, 118)):
+        desc = d(B, H, 4096, algo="tcgen05_chains")
+        assert G.resolved_algo(desc) == "tcgen05_chains"
+        n, rem = divmod(G.workspace_bytes(desc) - 4, per_chain)
+        assert rem == 0 and 1 <= n <= min(B * H, 74)
     assert G.resolved_algo(d(4, 16, 4096, dk=64)) == "simt"
     f32 = G.fwd_desc(4, 16, 4096, 128, 128, torch.float32, torch.float32)
     assert G.resolved_algo(f32) == "simt" and G.workspace_bytes(f32) == 0
@@ -232,3 +237,10 @@ def test_backward_checks_its_arguments_without_launching(G):
     per_head = lambda nc: 4 * (64 * 128 * 21 + 64 * 64 * 7 + 64 * 2 + 128 * 4 + 4 * 128 * 128 + nc * 128 * 128)
     assert G.bwd_workspace_bytes(d(2, 3, 1000)) == 6 * per_head(16)
     assert G.bwd_workspace_bytes(d(2, 3, 0)) == 0
+
+
+def test_default_build_has_no_index_checks(G):
+    """The index checks exist only in the debug build (libgdr_debug.so); the default build
+    answers -1 without touching a device."""
+    assert G.debug_bounds_site() == -1
+    assert G.status_string(G.GDR_ERR_BOUNDS) == "GDR_ERR_BOUNDS"

@@ -18,7 +18,7 @@ def G():
     gdr.debug_set_tc_fault(False, 0)
 
 
-@pytest.mark.parametrize("algo", ["tcgen05", "tcgen05_split"])
+@pytest.mark.parametrize("algo", ["tcgen05", "tcgen05_split", "tcgen05_chains"])
 def test_bounded_wait_gives_up_and_reports(G, algo):
     """A barrier that nothing signals: the wait runs out after 5 ms, the kernel frees
     its tensor memory and returns, the status word says GDR_ERR_TIMEOUT; the next

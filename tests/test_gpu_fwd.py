@@ -9,13 +9,17 @@ import parity_util as U
 
 pytestmark = pytest.mark.gpu
 
-ALGOS_ALL = ["simt", "tcgen05", "tcgen05_split"]
-TC_ALGOS = ["tcgen05", "tcgen05_split"]
+ALGOS_ALL = ["simt", "tcgen05", "tcgen05_split", "tcgen05_chains"]
+TC_ALGOS = ["tcgen05", "tcgen05_split", "tcgen05_chains"]
 
 
 def _skip_unsupported(algo, dtype, dk, dv, nh=1):
     if algo.startswith("tcgen05") and not (dtype == "bf16" and dk == 128 and dv == 128):
         pytest.skip("tcgen05 kernels: bf16 q/k/v with dk = dv = 128 only")
+    if algo == "tcgen05_split":
+        import torch
+        if nh >= torch.cuda.get_device_properties(0).multi_processor_count:
+            pytest.skip("split kernel: B*H must be below the SM count (the chains kernel takes any number)")
 
 
 @pytest.fixture(scope="module")
@@ -244,10 +248,17 @@ def test_auto_picks_tensor_cores_for_bf16_d128(G):
     import torch
     d = G.fwd_desc(1, 1, 64, 128, 128, torch.bfloat16, torch.bfloat16)
     assert G.resolved_algo(d) == "tcgen05"                    # a single chunk: fused
-    for B, H, T in ((2, 16, 8192), (4, 16, 4096), (16, 12, 4096), (1, 1, 65)):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for B, H, T in ((2, 16, 8192), (4, 16, 4096), (1, 1, 65)):
         d = G.fwd_desc(B, H, T, 128, 128, torch.bfloat16, torch.bfloat16)
-        assert G.resolved_algo(d) == "tcgen05_split"          # state chains + prep workers, any head count
-        assert G.workspace_bytes(d) >= 8 * 91136
+        expect = "tcgen05_split" if 2 * B * H <= sms else "tcgen05"   # chains + prep workers
+        assert G.resolved_algo(d) == expect
+        if expect == "tcgen05_split":
+            assert G.workspace_bytes(d) >= B * H * 8 * 76288
+    d = G.fwd_desc(16, 12, 4096, 128, 128, torch.bfloat16, torch.bfloat16)
+    rem = (16 * 12) % sms if 16 * 12 > sms else 0
+    expect = "tcgen05_waves" if 0 < rem and 2 * rem <= sms else "tcgen05"   # many heads
+    assert G.resolved_algo(d) == expect
     d = G.fwd_desc(1, 1, 64, 64, 64, torch.bfloat16, torch.bfloat16)
     assert G.resolved_algo(d) == "simt"
     d = G.fwd_desc(1, 1, 64, 128, 128, torch.float32, torch.float32)
@@ -255,14 +266,15 @@ def test_auto_picks_tensor_cores_for_bf16_d128(G):
 
 
 @pytest.mark.parametrize("rotation", [False, True])
-@pytest.mark.parametrize("B,H", [(4, 13), (2, 100)])
-def test_split_many_heads_parity(G, rotation, B, H):
-    """52 heads (one per chain) and 200 heads (more than the SMs: each chain runs several heads
-    one after another, in waves); six chunks with a ragged tail, initial state, against the
-    oracle on every head."""
+@pytest.mark.parametrize("algo,B,H", [("tcgen05_split", 4, 13), ("tcgen05_chains", 4, 13),
+                                      ("tcgen05_chains", 2, 100)])
+def test_split_many_heads_parity(G, rotation, algo, B, H):
+    """52 heads (one chain each, both split kernels) and 200 heads (more than the SMs: each of
+    the chains kernel's chains runs several heads one after another, in waves); six chunks with a
+    ragged tail, initial state, against the oracle on every head."""
     B_, T = B, 330
     p = I.make_fwd(B_, T, H, 128, 128, dtype="bf16", seed=77 + int(rotation) + H, s0_std=0.2, rotation=rotation)
-    o, S = U.run_gpu_fwd(p, "tcgen05_split")
+    o, S = U.run_gpu_fwd(p, algo)
     assert G.query_device_status() == G.GDR_OK
     o_ref, S_ref = U.oracle_fwd(p)
     U.assert_fwd_parity(p, o, S, o_ref, S_ref)
