@@ -352,10 +352,11 @@ GDR_API int gdr_chunk_fwd_kernel_launches(const gdr_fwd_desc* desc);
  * Backward pass of gdr_chunk_fwd: the gradients of a loss L with respect to every input, given
  * dO = dL/do and dS_T = dL/dS_T (the training use that the "CARVE" page, section 4, measures).
  * It follows the chain rule through the chunk-WY algebra ("CARVE" page, section 1 item 3;
- * "Semidirect Fourier Delta Attention" page, "Constructive Chunk-WY Theorem"): one CTA per
- * (batch, head) keeps each chunk's start state from a forward sweep, then runs the chunks in
- * reverse, the gradient of each chunk's end state flowing into the one before.  fp32 throughout
- * (tensor-core products with split-tf32 operands).
+ * "Semidirect Fourier Delta Attention" page, "Constructive Chunk-WY Theorem" and the exact
+ * affine chunk transfer) in three launches: every chunk's transfer coefficients in parallel
+ * (S_L = S0 A_c + B_c and dS0 = G_c + dS_L A_c^T need no state), one short chain per (batch,
+ * head) for the chunk start states and the end-state gradients, then every chunk's gradients in
+ * parallel.  fp32 throughout (tensor-core products with split-tf32 operands).
  *
  *   desc            as for gdr_chunk_fwd; dk = dv (32, 64 or 128), rotation = 0, qk_l2norm = 0
  *                   (else GDR_ERR_UNSUPPORTED); algo and segments are ignored.  dO has the
@@ -371,8 +372,8 @@ GDR_API int gdr_chunk_fwd_kernel_launches(const gdr_fwd_desc* desc);
  *                   gradient alone).
  *   dS0 [B,H,dv,dk] fp32 gradient of S0, or NULL (not written).
  *   workspace       device memory of gdr_chunk_bwd_workspace_bytes(desc) bytes, 16-byte aligned
- *                   (the chunk start states and each head's chunk matrices; about
- *                   (1 MB + 64 KB per chunk) per head at d = 128).
+ *                   (five dk x dv fp32 matrices per chunk, two per head, and about 1 MB of
+ *                   chunk matrices per SM at d = 128: 1.48 GB at B=4, H=16, T=4096).
  * All pointers are device pointers, 16-byte aligned, owned by the caller; the call is
  * asynchronous on `stream` and allocates nothing.  With T = 0, dS0 = dS_T.  Errors: argument
  * checks return before any launch; a decay too strong for the factored form over half a chunk

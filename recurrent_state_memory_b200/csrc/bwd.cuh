@@ -62,14 +62,20 @@ struct BwdParams {
     float* dbeta;            // [B,T,H]
     float* dw;               // [B,T,H] (with w) or nullptr
     float* dS0;              // [B,H,dv,dk] or nullptr
-    float* ws;               // per head: head_floats floats
-    size_t head_floats;
+    // workspace parts (floats)
+    float* coef;             // [B*H][nc][3][dv*dk]: A_c (dk x dk, in a dv x dk slot), B_c, G_c
+    float* ckpt;             // [B*H][nc][dv*dk]: the state at each chunk start
+    float* dsl;              // [B*H][nc][dv*dk]: the gradient of each chunk's end state
+    float* chain;            // [B*H][2][dv*dk]: the chain's two buffers
+    float* scratch;          // [grid][scratch_floats]: each CTA's chunk matrices
+    size_t scratch_floats;
 };
 
-// Per-head workspace layout (floats).
+// Scratch layout of one CTA of the parallel passes (floats): one chunk's matrices.  The raw k
+// and q tiles share storage with dKt and dKh, which are written only after k and q are done with.
 template <int DK, int DV>
 struct Lay {
-    static constexpr int K = 0, Q = K + C * DK, V = Q + C * DK, DO = V + C * DV;
+    static constexpr int V = 0, DO = V + C * DV;
     static constexpr int EG = DO + C * DV;          // e^{gam - gam_m}
     static constexpr int EGI = EG + C * DK;         // e^{-(gam - gam_m)}
     static constexpr int DLG = EGI + C * DK;        // d log alpha / d gate input
@@ -78,12 +84,11 @@ struct Lay {
     static constexpr int DA = X2 + C * C, DPM = DA + C * C;
     static constexpr int KS = DPM + C * C, R = KS + C * DV, E = R + C * DV, DE = E + C * DV, DR = DE + C * DV;
     static constexpr int DQT = DR + C * DV, DKH = DQT + C * DK, DKD = DKH + C * DK, DKT = DKD + C * DK;
-    static constexpr int DGAM = DKT + C * DK;
-    static constexpr int BT = DGAM + C * DK, WT = BT + C;
-    static constexpr int E31 = WT + C, EGL = E31 + DK, ED = EGL + DK, CS = ED + DK;   // column vectors
-    static constexpr int S0P = CS + DK, SC = S0P + DV * DK, DSL = SC + DV * DK, DS0 = DSL + DV * DK;
-    static constexpr int CKPT = DS0 + DV * DK;      // nchunks x (dv x dk): chunk start states
-    static constexpr size_t floats(int nchunks) { return (size_t)CKPT + (size_t)nchunks * DV * DK; }
+    static constexpr int K = DKT, Q = DKH;          // raw k and q (chunk_forward only)
+    static constexpr int BT = DKT + C * DK, WT = BT + C, DBS = WT + C;   // beta, w, dbeta parts
+    static constexpr int E31 = DBS + C, EGL = E31 + DK, ED = EGL + DK;   // column vectors
+    static constexpr int S0P = ED + DK;
+    static constexpr size_t floats() { return (size_t)S0P + (size_t)DV * DK; }
 };
 
 __device__ __forceinline__ uint32_t tf32_hi(float x) { return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u; }
@@ -129,10 +134,15 @@ __device__ void mm(float* Cm, int ldc, const float* A, int lda, const float* Bm,
     auto b_ = [&](int k, int j) -> float { return TB ? sB[j * sbs + k] : sB[k * sbs + j]; };
     for (int t = warp; t < ntiles; t += NW) {
         const int r0 = (t / tn) * 16, c0 = (t % tn) * 16;
-        float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // three accumulators per 8-column half (high x high, high x low, low x high), so that
+        // six independent MMA chains run side by side; summed at the end, small parts first
+        float dhh[2][4] = {}, dhl[2][4] = {}, dlh[2][4] = {};
+#pragma unroll 2
         for (int k0 = 0; k0 < K; k0 += 8) {
             const float af[4] = {a_(r0 + gid, k0 + tig), a_(r0 + gid + 8, k0 + tig), a_(r0 + gid, k0 + tig + 4),
                                  a_(r0 + gid + 8, k0 + tig + 4)};
+            const float bf[2][2] = {{b_(k0 + tig, c0 + gid), b_(k0 + tig + 4, c0 + gid)},
+                                    {b_(k0 + tig, c0 + 8 + gid), b_(k0 + tig + 4, c0 + 8 + gid)}};
             uint32_t ah[4], al[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -141,16 +151,15 @@ __device__ void mm(float* Cm, int ldc, const float* A, int lda, const float* Bm,
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const float bf[2] = {b_(k0 + tig, c0 + 8 * h + gid), b_(k0 + tig + 4, c0 + 8 * h + gid)};
                 uint32_t bh[2], bl[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    bh[e] = tf32_hi(bf[e]);
-                    bl[e] = tf32_hi(bf[e] - __uint_as_float(bh[e]));
+                    bh[e] = tf32_hi(bf[h][e]);
+                    bl[e] = tf32_hi(bf[h][e] - __uint_as_float(bh[e]));
                 }
-                mma_tf32(d[h], al, bh);
-                mma_tf32(d[h], ah, bl);
-                mma_tf32(d[h], ah, bh);
+                mma_tf32(dlh[h], al, bh);
+                mma_tf32(dhl[h], ah, bl);
+                mma_tf32(dhh[h], ah, bh);
             }
         }
 #pragma unroll
@@ -158,7 +167,7 @@ __device__ void mm(float* Cm, int ldc, const float* A, int lda, const float* Bm,
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int row = r0 + gid + ((e >> 1) << 3), col = c0 + 8 * h + 2 * tig + (e & 1);
-                float x = alpha * d[h][e];
+                float x = alpha * ((dlh[h][e] + dhl[h][e]) + dhh[h][e]);
                 if (acc) x += Cm[(size_t)row * ldc + col];
                 Cm[(size_t)row * ldc + col] = x;
             }
@@ -251,11 +260,12 @@ __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0
         W[L::QT + i] = p.scale * W[L::Q + i] * W[L::EG + i];
         W[L::KD + i] = kk * W[L::EGI + i] * W[L::ED + d];
     }
-    for (int i = tid; i < DV * DK; i += NT) W[L::S0P + i] = S0[i] * W[L::E31 + i % DK];
+    if (S0)
+        for (int i = tid; i < DV * DK; i += NT) W[L::S0P + i] = S0[i] * W[L::E31 + i % DK];
     __syncthreads();
     mm<false, true>(W + L::AP, C, W + L::KT, DK, W + L::KH, DK, C, C, DK, 1.f, false, sm);      // Ap = Kt Kh^T
     mm<false, true>(W + L::PM, C, W + L::QT, DK, W + L::KH, DK, C, C, DK, 1.f, false, sm);      // Qt Kh^T
-    mm<false, true>(W + L::KS, DV, W + L::KT, DK, W + L::S0P, DK, C, DV, DK, 1.f, false, sm);   // KS = Kt S0p^T
+    if (S0) mm<false, true>(W + L::KS, DV, W + L::KT, DK, W + L::S0P, DK, C, DV, DK, 1.f, false, sm);   // KS = Kt S0p^T
     __syncthreads();
     // masks; R = diag(w) V - diag(beta) KS; T = (I + A)^{-1} by forward substitution, eight
     // threads per column
@@ -263,10 +273,11 @@ __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0
         const int r = i / C, c = i % C;
         if (c > r) W[L::PM + i] = 0.f;
     }
-    for (int i = tid; i < C * DV; i += NT) {
-        const int r = i / DV;
-        W[L::R + i] = W[L::WT + r] * W[L::V + i] - W[L::BT + r] * W[L::KS + i];
-    }
+    if (S0)
+        for (int i = tid; i < C * DV; i += NT) {
+            const int r = i / DV;
+            W[L::R + i] = W[L::WT + r] * W[L::V + i] - W[L::BT + r] * W[L::KS + i];
+        }
     {   // A = diag(beta) strict_lower(Ap) and T in shared memory (row stride C + 1)
         float* sAm = sm;
         float* sT = sm + C * (C + 1);
@@ -289,163 +300,335 @@ __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0
         for (int i = tid; i < C * C; i += NT) W[L::TM + i] = sT[(i / C) * (C + 1) + i % C];
     }
     __syncthreads();
-    mm<false, false>(W + L::E, DV, W + L::TM, C, W + L::R, DV, C, DV, C, 1.f, false, sm);       // E = T R
+    if (S0) mm<false, false>(W + L::E, DV, W + L::TM, C, W + L::R, DV, C, DV, C, 1.f, false, sm);   // E = T R
     __syncthreads();
 }
 
+// The gradients of one chunk, every thread taking part, after chunk_forward on the chunk's start
+// state S0c (its quantities are in W); dSL is the gradient of the chunk's end state.
 template <int DK, int DV, typename QT, typename OT>
-__global__ void __launch_bounds__(NT, 1) chunk_bwd_kernel(BwdParams p) {
+__device__ void chunk_grads(const BwdParams& p, float* W, int b, int h, int t0, const float* S0c, const float* dSL,
+                            float* sm) {
+    using L = Lay<DK, DV>;
+    const int tid = (int)threadIdx.x;
+    // dE = P^T dO + Kd dSL^T ; dP = incl_lower(dO E^T) ; dKd = E dSL
+    mm<true, false>(W + L::DE, DV, W + L::PM, C, W + L::DO, DV, C, DV, C, 1.f, false, sm);
+    mm<false, true>(W + L::DPM, C, W + L::DO, DV, W + L::E, DV, C, C, DV, 1.f, false, sm);
+    mm<false, false>(W + L::DKD, DK, W + L::E, DV, dSL, DK, C, DK, DV, 1.f, false, sm);
+    __syncthreads();
+    mm<false, true>(W + L::DE, DV, W + L::KD, DK, dSL, DK, C, DV, DK, 1.f, true, sm);
+    for (int i = tid; i < C * C; i += NT) {
+        const int r = i / C, cc = i % C;
+        if (cc > r) W[L::DPM + i] = 0.f;
+    }
+    __syncthreads();
+    // dR = T^T dE ; X1 = dE R^T ; dQt = dO S0p + dP Kh ; dKh = dP^T Qt
+    mm<true, false>(W + L::DR, DV, W + L::TM, C, W + L::DE, DV, C, DV, C, 1.f, false, sm);
+    mm<false, true>(W + L::X1, C, W + L::DE, DV, W + L::R, DV, C, C, DV, 1.f, false, sm);
+    mm<false, false>(W + L::DQT, DK, W + L::DO, DV, W + L::S0P, DK, C, DK, DV, 1.f, false, sm);
+    mm<true, false>(W + L::DKH, DK, W + L::DPM, C, W + L::QT, DK, C, DK, C, 1.f, false, sm);
+    __syncthreads();
+    mm<false, false>(W + L::DQT, DK, W + L::DPM, C, W + L::KH, DK, C, DK, C, 1.f, true, sm);
+    mm<true, false>(W + L::X2, C, W + L::TM, C, W + L::X1, C, C, C, C, 1.f, false, sm);      // T^T X1
+    // beta dR (in place) after dv, dw and the dR parts of dbeta
+    __syncthreads();
+    mm<false, true>(W + L::DA, C, W + L::X2, C, W + L::TM, C, C, C, C, -1.f, false, sm);     // dA = -X2 T^T
+    if (tid < C * 8) {
+        // per token r (eight threads each): dbeta and dw parts from dR
+        const int r = tid >> 3, part = tid & 7;
+        float sks = 0.f, sv = 0.f;
+        for (int j = part; j < DV; j += 8) {
+            const float dr = W[L::DR + r * DV + j];
+            sks += dr * W[L::KS + r * DV + j];
+            sv += dr * W[L::V + r * DV + j];
+        }
+#pragma unroll
+        for (int off = 4; off >= 1; off >>= 1) {
+            sks += __shfl_xor_sync(0xffffffffu, sks, off);
+            sv += __shfl_xor_sync(0xffffffffu, sv, off);
+        }
+        if (part == 0) {
+            W[L::DBS + r] = -sks + (p.w ? 0.f : sv);         // dbeta so far
+            if (p.dw && t0 + r < p.T) p.dw[((size_t)b * p.T + t0 + r) * p.H + h] = sv;
+        }
+    }
+    for (int i = tid; i < C * DV; i += NT) {
+        const int r = i / DV, j = i % DV;
+        if (t0 + r < p.T) p.dv[(((size_t)b * p.T + t0 + r) * p.H + h) * DV + j] = W[L::WT + r] * W[L::DR + i];
+    }
+    __syncthreads();
+    // dAp = diag(beta) strict_lower(dA) (in place, after the dA . Ap part of dbeta)
+    if (tid < C * 8) {
+        const int r = tid >> 3, part = tid & 7;
+        float s = 0.f;
+        for (int i = part; i < r; i += 8) s += W[L::DA + r * C + i] * W[L::AP + r * C + i];
+#pragma unroll
+        for (int off = 4; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (part == 0 && t0 + r < p.T)
+            p.dbeta[((size_t)b * p.T + t0 + r) * p.H + h] = W[L::DBS + r] + s;
+    }
+    __syncthreads();
+    for (int i = tid; i < C * C; i += NT) {
+        const int r = i / C, cc = i % C;
+        W[L::DA + i] = cc < r ? W[L::BT + r] * W[L::DA + i] : 0.f;
+    }
+    for (int i = tid; i < C * DV; i += NT) W[L::DR + i] *= W[L::BT + i / DV];
+    __syncthreads();
+    // dKt = -(beta dR) S0p + dAp Kh ; dKh += dAp^T Kt
+    mm<false, false>(W + L::DKT, DK, W + L::DR, DV, W + L::S0P, DK, C, DK, DV, -1.f, false, sm);
+    mm<true, false>(W + L::DKH, DK, W + L::DA, C, W + L::KT, DK, C, DK, C, 1.f, true, sm);
+    __syncthreads();
+    mm<false, false>(W + L::DKT, DK, W + L::DA, C, W + L::KH, DK, C, DK, C, 1.f, true, sm);
+    __syncthreads();
+    // dq, dk; dgam (shared memory)
+    float* sdg = sm;                  // [C][DK] dgam, then dg
+    float* sdl = sm + C * DK;         // [C][DK] d log alpha / d gate input
+    float* scs = sm + 2 * C * DK;     // [NT / DK][DK] column-sum parts
+    for (int i = tid; i < C * DK; i += NT) {
+        const int r = i / DK, d = i % DK;
+        const float eg = W[L::EG + i], egi = W[L::EGI + i];
+        const float gkt = W[L::DKT + i], gkh = W[L::DKH + i], gqt = W[L::DQT + i], gkd = W[L::DKD + i];
+        if (t0 + r < p.T) {
+            const size_t o = (((size_t)b * p.T + t0 + r) * p.H + h) * DK + d;
+            p.dq[o] = p.scale * gqt * eg;
+            p.dk[o] = gkt * eg + gkh * egi + gkd * egi * W[L::ED + d];
+        }
+        sdg[i] = gkt * W[L::KT + i] + gqt * W[L::QT + i] - gkh * W[L::KH + i] - gkd * W[L::KD + i];
+        sdl[i] = W[L::DLG + i];
+    }
+    {   // column sums for the last token's decay terms: NT / DK threads per key dim
+        constexpr int NP = NT / DK;
+        const int d = tid % DK, part = tid / DK;
+        float s0 = 0.f, sd = 0.f;
+        for (int i = part; i < DV; i += NP) s0 += S0c[i * DK + d] * dSL[i * DK + d];
+        for (int r = part; r < C; r += NP) sd += W[L::DKD + r * DK + d] * W[L::KD + r * DK + d];
+        scs[part * DK + d] = W[L::EGL + d] * s0 + sd;
+    }
+    __syncthreads();
+    if (tid < DK) {     // reverse cumulative sum over the chunk's tokens
+        const int d = tid;
+        float acc = 0.f;
+        for (int pp = 0; pp < NT / DK; ++pp) acc += scs[pp * DK + d];
+        for (int r = C - 1; r >= 0; --r) {
+            acc += sdg[r * DK + d];
+            sdg[r * DK + d] = acc * sdl[r * DK + d];
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < C * DK; i += NT) {
+        const int r = i / DK, d = i % DK;
+        if (t0 + r < p.T) p.dg[(((size_t)b * p.T + t0 + r) * p.H + h) * DK + d] = sdg[i];
+    }
+    __syncthreads();
+}
+
+// Tasks of the two parallel passes: chunk c of head hd, as t = hd * nc + c; each CTA takes
+// tasks blockIdx.x, blockIdx.x + gridDim.x, ... with its own region of the scratch.
+
+// Pass 1: each chunk's transfer coefficients, which need no state:
+//   M = T^T Kd,  A_c = diag(e^{gam_L}) - diag(e^{gam_m}) Kt^T diag(beta) M     (dk x dk)
+//   B_c = (T diag(w) V)^T Kd                                                  (dv x dk)
+//   G_c = dO^T (Qt - P T diag(beta) Kt) diag(e^{gam_m})                        (dv x dk)
+// so that a chunk's end state is S_L = S0 A_c + B_c and its start state's gradient is
+// dS0 = G_c + dS_L A_c^T.
+template <int DK, int DV, typename QT, typename OT>
+__global__ void __launch_bounds__(NT, 1) bwd_coef_kernel(BwdParams p) {
     using L = Lay<DK, DV>;
     extern __shared__ float4 sm4[];
     float* sm = reinterpret_cast<float*>(sm4);
     __shared__ int range_f;
     const int tid = (int)threadIdx.x;
-    const int head = (int)blockIdx.x, b = head / p.H, h = head % p.H;
-    const int nc = (p.T + C - 1) / C;
-    if (!GDR_INB(head < p.B * p.H, 401)) return;     // (the whole CTA)
-    float* W = p.ws + (size_t)head * p.head_floats;
+    const int nc = (p.T + C - 1) / C, ntask = p.B * p.H * nc;
+    float* W = p.scratch + (size_t)blockIdx.x * p.scratch_floats;
     if (tid == 0) range_f = 0;
-    // ---- forward sweep: chunk start states ---------------------------------------------------
-    for (int i = tid; i < DV * DK; i += NT) W[L::SC + i] = p.S0 ? p.S0[(size_t)head * DV * DK + i] : 0.f;
-    __syncthreads();
-    for (int c = 0; c < nc; ++c) {
-        float* ck = W + L::CKPT + (size_t)c * DV * DK;
-        for (int i = tid; i < DV * DK; i += NT) ck[i] = W[L::SC + i];
+    for (int t = (int)blockIdx.x; t < ntask; t += (int)gridDim.x) {
+        const int hd = t / nc, c = t % nc, b = hd / p.H, h = hd % p.H;
+        if (!GDR_INB(hd < p.B * p.H, 402)) break;
+        chunk_forward<DK, DV, QT, OT>(p, W, b, h, c * C, nullptr, true, &range_f, sm);
+        float* A = p.coef + ((size_t)t * 3 + 0) * DV * DK;
+        float* Bc = p.coef + ((size_t)t * 3 + 1) * DV * DK;
+        float* G = p.coef + ((size_t)t * 3 + 2) * DV * DK;
+        // M = T^T Kd (in DQT); diag(w) V (in V); diag(beta) Kt (in DKT)
+        mm<true, false>(W + L::DQT, DK, W + L::TM, C, W + L::KD, DK, C, DK, C, 1.f, false, sm);
+        for (int i = tid; i < C * DV; i += NT) W[L::V + i] *= W[L::WT + i / DV];
+        for (int i = tid; i < C * DK; i += NT) W[L::DKT + i] = W[L::BT + i / DK] * W[L::KT + i];
         __syncthreads();
-        chunk_forward<DK, DV, QT, OT>(p, W, b, h, c * C, ck, false, &range_f, sm);
-        // S_L = S0 e^{gam_L} + E^T Kd
-        for (int i = tid; i < DV * DK; i += NT) W[L::SC + i] = ck[i] * W[L::EGL + i % DK];
+        // N = (diag(beta) Kt)^T M (into A); E0 = T diag(w) V (in E); W1 = T diag(beta) Kt (in DKH)
+        mm<true, false>(A, DK, W + L::DKT, DK, W + L::DQT, DK, DK, DK, C, 1.f, false, sm);
+        mm<false, false>(W + L::E, DV, W + L::TM, C, W + L::V, DV, C, DV, C, 1.f, false, sm);
+        mm<false, false>(W + L::DKH, DK, W + L::TM, C, W + L::DKT, DK, C, DK, C, 1.f, false, sm);
         __syncthreads();
-        mm<true, false>(W + L::SC, DK, W + L::E, DV, W + L::KD, DK, DV, DK, C, 1.f, true, sm);
+        // A_c = diag(e^{gam_L}) - diag(e^{gam_m}) N ; B_c = E0^T Kd ; X = P W1 (in DKD)
+        for (int i = tid; i < DK * DK; i += NT) {
+            const int r = i / DK, cc = i % DK;
+            A[i] = (r == cc ? W[L::EGL + r] : 0.f) - W[L::E31 + r] * A[i];
+        }
+        mm<true, false>(Bc, DK, W + L::E, DV, W + L::KD, DK, DV, DK, C, 1.f, false, sm);
+        mm<false, false>(W + L::DKD, DK, W + L::PM, C, W + L::DKH, DK, C, DK, C, 1.f, false, sm);
+        __syncthreads();
+        // G_c = dO^T (Qt - X) diag(e^{gam_m})
+        for (int i = tid; i < C * DK; i += NT) W[L::DKD + i] = W[L::QT + i] - W[L::DKD + i];
+        __syncthreads();
+        mm<true, false>(G, DK, W + L::DO, DV, W + L::DKD, DK, DV, DK, C, 1.f, false, sm);
+        for (int i = tid; i < DV * DK; i += NT) G[i] *= W[L::E31 + i % DK];
         __syncthreads();
     }
-    // ---- backward sweep --------------------------------------------------------------------------
-    for (int i = tid; i < DV * DK; i += NT) W[L::DSL + i] = p.dS_T ? p.dS_T[(size_t)head * DV * DK + i] : 0.f;
-    __syncthreads();
-    for (int c = nc - 1; c >= 0; --c) {
-        const int t0 = c * C;
-        const float* S0c = W + L::CKPT + (size_t)c * DV * DK;
-        chunk_forward<DK, DV, QT, OT>(p, W, b, h, t0, S0c, true, &range_f, sm);
-        // dE = P^T dO + Kd dSL^T ; dP = incl_lower(dO E^T) ; dKd = E dSL ; dS0 = dO^T Qt
-        mm<true, false>(W + L::DE, DV, W + L::PM, C, W + L::DO, DV, C, DV, C, 1.f, false, sm);
-        mm<false, true>(W + L::DPM, C, W + L::DO, DV, W + L::E, DV, C, C, DV, 1.f, false, sm);
-        mm<false, false>(W + L::DKD, DK, W + L::E, DV, W + L::DSL, DK, C, DK, DV, 1.f, false, sm);
-        mm<true, false>(W + L::DS0, DK, W + L::DO, DV, W + L::QT, DK, DV, DK, C, 1.f, false, sm);
-        __syncthreads();
-        mm<false, true>(W + L::DE, DV, W + L::KD, DK, W + L::DSL, DK, C, DV, DK, 1.f, true, sm);
-        for (int i = tid; i < C * C; i += NT) {
-            const int r = i / C, cc = i % C;
-            if (cc > r) W[L::DPM + i] = 0.f;
+    if (tid == 0 && range_f) atomicOr(&g_device_status, STATUS_RANGE);
+}
+
+// 16-byte copy global -> shared that completes asynchronously (cp.async, L2 only).
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Pass 2, one CTA per head: the chunk start states S_{c+1} = S_c A_c + B_c (kept for pass 3),
+// then, backwards, the end-state gradients dS_L(c-1) = G_c + dS_L(c) A_c^T (kept), and the
+// gradient of S0.  The carried matrix stays in shared memory; the next chunk's A_c is fetched
+// with asynchronous copies while the current product runs, and B_c / G_c are loaded into
+// registers at the start of the step.
+template <int D>
+__global__ void __launch_bounds__(NT, 1) bwd_chain_kernel(BwdParams p) {
+    extern __shared__ float4 sm4[];
+    float* sm = reinterpret_cast<float*>(sm4);
+    constexpr int SS = D + 4;                  // row stride of the carried matrix (the A operand)
+    constexpr int SA = D + 8;                  // row stride of A_c read as it is (forwards)
+    constexpr int SAT = D + 4;                 // row stride of A_c read transposed (backwards)
+    constexpr int DD = D * D;
+    constexpr int TN = D / 16, NTILE = TN * TN, TPW = (NTILE + NW - 1) / NW;   // 16x16 tiles per warp
+    float* S = sm;                             // [D][SS]
+    float* Abuf[2] = {sm + D * SS, sm + D * SS + D * SA};
+    const int tid = (int)threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+    const int hd = (int)blockIdx.x, nc = (p.T + C - 1) / C;
+    if (!GDR_INB(hd < p.B * p.H, 403)) return;     // (the whole CTA)
+    auto coef = [&](int c, int k) -> const float* { return p.coef + (((size_t)hd * nc + c) * 3 + k) * DD; };
+    auto prefetch_A = [&](int c, int buf, int stride) {
+        for (int i = tid; i < DD / 4; i += NT) {
+            const int r = (4 * i) / D, cc = (4 * i) % D;
+            cp_async16(Abuf[buf] + r * stride + cc, coef(c, 0) + 4 * i);
         }
-        __syncthreads();
-        // dR = T^T dE ; X1 = dE R^T ; dQt = dO S0p + dP Kh ; dKh = dP^T Qt
-        mm<true, false>(W + L::DR, DV, W + L::TM, C, W + L::DE, DV, C, DV, C, 1.f, false, sm);
-        mm<false, true>(W + L::X1, C, W + L::DE, DV, W + L::R, DV, C, C, DV, 1.f, false, sm);
-        mm<false, false>(W + L::DQT, DK, W + L::DO, DV, W + L::S0P, DK, C, DK, DV, 1.f, false, sm);
-        mm<true, false>(W + L::DKH, DK, W + L::DPM, C, W + L::QT, DK, C, DK, C, 1.f, false, sm);
-        __syncthreads();
-        mm<false, false>(W + L::DQT, DK, W + L::DPM, C, W + L::KH, DK, C, DK, C, 1.f, true, sm);
-        mm<true, false>(W + L::X2, C, W + L::TM, C, W + L::X1, C, C, C, C, 1.f, false, sm);      // T^T X1
-        // beta dR (in place) after dv, dw and the dR parts of dbeta
-        __syncthreads();
-        mm<false, true>(W + L::DA, C, W + L::X2, C, W + L::TM, C, C, C, C, -1.f, false, sm);     // dA = -X2 T^T
-        if (tid < C * 8) {
-            // per token r (eight threads each): dbeta and dw parts from dR
-            const int r = tid >> 3, part = tid & 7;
-            float sks = 0.f, sv = 0.f;
-            for (int j = part; j < DV; j += 8) {
-                const float dr = W[L::DR + r * DV + j];
-                sks += dr * W[L::KS + r * DV + j];
-                sv += dr * W[L::V + r * DV + j];
-            }
+        cp_async_commit();
+    };
+    // n steps of the chain from chunk c0 in direction dc: S <- coef(c, add_k) + S op(A_c); the new
+    // S of chunk c is also stored at keep + (hd * nc + c + shift) * DD unless keep is null
+    auto run = [&](bool fwd, int c0, int dc, int n, float* keep, int shift, int add_k) {
+        const int stride = fwd ? SA : SAT;
+        if (n > 0) prefetch_A(c0, 0, stride);
+        for (int st = 0; st < n; ++st) {
+            const int c = c0 + st * dc, buf = st & 1;
+            const float* addp = coef(c, add_k);
+            float res[TPW][8];
 #pragma unroll
-            for (int off = 4; off >= 1; off >>= 1) {
-                sks += __shfl_xor_sync(0xffffffffu, sks, off);
-                sv += __shfl_xor_sync(0xffffffffu, sv, off);
-            }
-            if (part == 0) {
-                W[L::DGAM + r] = -sks + (p.w ? 0.f : sv);        // dbeta so far (DGAM used as scratch)
-                if (p.dw && t0 + r < p.T) p.dw[((size_t)b * p.T + t0 + r) * p.H + h] = sv;
-            }
-        }
-        for (int i = tid; i < C * DV; i += NT) {
-            const int r = i / DV, j = i % DV;
-            if (t0 + r < p.T) p.dv[(((size_t)b * p.T + t0 + r) * p.H + h) * DV + j] = W[L::WT + r] * W[L::DR + i];
-        }
-        __syncthreads();
-        // dAp = diag(beta) strict_lower(dA) (in place, after the dA . Ap part of dbeta)
-        if (tid < C * 8) {
-            const int r = tid >> 3, part = tid & 7;
-            float s = 0.f;
-            for (int i = part; i < r; i += 8) s += W[L::DA + r * C + i] * W[L::AP + r * C + i];
+            for (int u = 0; u < TPW; ++u) {
+                const int t = warp + u * NW, r0 = (t / TN) * 16, col0 = (t % TN) * 16;
 #pragma unroll
-            for (int off = 4; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-            if (part == 0 && t0 + r < p.T)
-                p.dbeta[((size_t)b * p.T + t0 + r) * p.H + h] = W[L::DGAM + r] + s;
-        }
-        __syncthreads();
-        for (int i = tid; i < C * C; i += NT) {
-            const int r = i / C, cc = i % C;
-            W[L::DA + i] = cc < r ? W[L::BT + r] * W[L::DA + i] : 0.f;
-        }
-        for (int i = tid; i < C * DV; i += NT) W[L::DR + i] *= W[L::BT + i / DV];
-        __syncthreads();
-        // dKt = -(beta dR) S0p + dAp Kh ; dKh += dAp^T Kt ; dS0 -= (beta dR)^T Kt
-        mm<false, false>(W + L::DKT, DK, W + L::DR, DV, W + L::S0P, DK, C, DK, DV, -1.f, false, sm);
-        mm<true, false>(W + L::DKH, DK, W + L::DA, C, W + L::KT, DK, C, DK, C, 1.f, true, sm);
-        mm<true, false>(W + L::DS0, DK, W + L::DR, DV, W + L::KT, DK, DV, DK, C, -1.f, true, sm);
-        __syncthreads();
-        mm<false, false>(W + L::DKT, DK, W + L::DA, C, W + L::KH, DK, C, DK, C, 1.f, true, sm);
-        __syncthreads();
-        // dq, dk; dgam (shared memory); dS0 = dS0 e^{gam_m} + dSL e^{gam_L}
-        float* sdg = sm;                  // [C][DK] dgam, then dg
-        float* sdl = sm + C * DK;         // [C][DK] d log alpha / d gate input
-        float* scs = sm + 2 * C * DK;     // [NT / DK][DK] column-sum parts
-        for (int i = tid; i < C * DK; i += NT) {
-            const int r = i / DK, d = i % DK;
-            const float eg = W[L::EG + i], egi = W[L::EGI + i];
-            const float gkt = W[L::DKT + i], gkh = W[L::DKH + i], gqt = W[L::DQT + i], gkd = W[L::DKD + i];
-            if (t0 + r < p.T) {
-                const size_t o = (((size_t)b * p.T + t0 + r) * p.H + h) * DK + d;
-                p.dq[o] = p.scale * gqt * eg;
-                p.dk[o] = gkt * eg + gkh * egi + gkd * egi * W[L::ED + d];
+                for (int e = 0; e < 8; ++e) {
+                    const int row = r0 + gid + (((e >> 1) & 1) << 3), col = col0 + 8 * (e >> 2) + 2 * tig + (e & 1);
+                    res[u][e] = t < NTILE ? addp[row * D + col] : 0.f;
+                }
             }
-            sdg[i] = gkt * W[L::KT + i] + gqt * W[L::QT + i] - gkh * W[L::KH + i] - gkd * W[L::KD + i];
-            sdl[i] = W[L::DLG + i];
-        }
-        {   // column sums for the last token's decay terms: NT / DK threads per key dim
-            constexpr int NP = NT / DK;
-            const int d = tid % DK, part = tid / DK;
-            float s0 = 0.f, sd = 0.f;
-            for (int i = part; i < DV; i += NP) s0 += S0c[i * DK + d] * W[L::DSL + i * DK + d];
-            for (int r = part; r < C; r += NP) sd += W[L::DKD + r * DK + d] * W[L::KD + r * DK + d];
-            scs[part * DK + d] = W[L::EGL + d] * s0 + sd;
-        }
-        __syncthreads();
-        if (tid < DK) {     // reverse cumulative sum over the chunk's tokens
-            const int d = tid;
-            float acc = 0.f;
-            for (int pp = 0; pp < NT / DK; ++pp) acc += scs[pp * DK + d];
-            for (int r = C - 1; r >= 0; --r) {
-                acc += sdg[r * DK + d];
-                sdg[r * DK + d] = acc * sdl[r * DK + d];
+            cp_async_wait_all();
+            __syncthreads();                                   // A_c landed; S is the current matrix
+            if (st + 1 < n) prefetch_A(c + dc, buf ^ 1, stride);
+            const float* Ab = Abuf[buf];
+#pragma unroll
+            for (int u = 0; u < TPW; ++u) {
+                const int t = warp + u * NW, r0 = (t / TN) * 16, col0 = (t % TN) * 16;
+                if (t >= NTILE) continue;
+                float dhh[2][4] = {}, dhl[2][4] = {}, dlh[2][4] = {};
+#pragma unroll 2
+                for (int k0 = 0; k0 < D; k0 += 8) {
+                    const float af[4] = {S[(r0 + gid) * SS + k0 + tig], S[(r0 + gid + 8) * SS + k0 + tig],
+                                         S[(r0 + gid) * SS + k0 + tig + 4], S[(r0 + gid + 8) * SS + k0 + tig + 4]};
+                    uint32_t ah[4], al[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        ah[e] = tf32_hi(af[e]);
+                        al[e] = tf32_hi(af[e] - __uint_as_float(ah[e]));
+                    }
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int j = col0 + 8 * hh + gid;
+                        // op(A_c)(k, j): A_c[k][j] forwards, A_c[j][k] backwards
+                        const float bf[2] = {fwd ? Ab[(k0 + tig) * SA + j] : Ab[j * SAT + k0 + tig],
+                                             fwd ? Ab[(k0 + tig + 4) * SA + j] : Ab[j * SAT + k0 + tig + 4]};
+                        uint32_t bh[2], bl[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            bh[e] = tf32_hi(bf[e]);
+                            bl[e] = tf32_hi(bf[e] - __uint_as_float(bh[e]));
+                        }
+                        mma_tf32(dlh[hh], al, bh);
+                        mma_tf32(dhl[hh], ah, bl);
+                        mma_tf32(dhh[hh], ah, bh);
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    res[u][e] += (dlh[e >> 2][e & 3] + dhl[e >> 2][e & 3]) + dhh[e >> 2][e & 3];
+            }
+            __syncthreads();                                   // every read of S is done
+            float* kp = keep ? keep + ((size_t)hd * nc + c + shift) * DD : nullptr;
+#pragma unroll
+            for (int u = 0; u < TPW; ++u) {
+                const int t = warp + u * NW, r0 = (t / TN) * 16, col0 = (t % TN) * 16;
+                if (t >= NTILE) continue;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int row = r0 + gid + (((e >> 1) & 1) << 3), col = col0 + 8 * (e >> 2) + 2 * tig + (e & 1);
+                    S[row * SS + col] = res[u][e];
+                    if (kp) kp[row * D + col] = res[u][e];
+                }
             }
         }
         __syncthreads();
-        for (int i = tid; i < C * DK; i += NT) {
-            const int r = i / DK, d = i % DK;
-            if (t0 + r < p.T) p.dg[(((size_t)b * p.T + t0 + r) * p.H + h) * DK + d] = sdg[i];
-        }
-        for (int i = tid; i < DV * DK; i += NT) {
-            const int d = i % DK;
-            W[L::DS0 + i] = W[L::DS0 + i] * W[L::E31 + d] + W[L::DSL + i] * W[L::EGL + d];
-        }
-        __syncthreads();
-        for (int i = tid; i < DV * DK; i += NT) W[L::DSL + i] = W[L::DS0 + i];
-        __syncthreads();
+    };
+    // forward: S_0 kept at ckpt[0]; S_{c+1} = B_c + S_c A_c kept at ckpt[c + 1], c = 0 .. nc-2
+    for (int i = tid; i < DD; i += NT) {
+        const float x = p.S0 ? p.S0[(size_t)hd * DD + i] : 0.f;
+        S[(i / D) * SS + i % D] = x;
+        p.ckpt[(size_t)hd * nc * DD + i] = x;
     }
+    __syncthreads();
+    run(true, 0, 1, nc - 1, p.ckpt, 1, 1);
+    // backward: dS_L(nc-1) = dS_T kept at dsl[nc-1]; dS_L(c-1) = G_c + dS_L(c) A_c^T kept at
+    // dsl[c-1], c = nc-1 .. 1; then dS0 = G_0 + dS_L(0) A_0^T
+    for (int i = tid; i < DD; i += NT) {
+        const float x = p.dS_T ? p.dS_T[(size_t)hd * DD + i] : 0.f;
+        S[(i / D) * SS + i % D] = x;
+        p.dsl[((size_t)hd * nc + nc - 1) * DD + i] = x;
+    }
+    __syncthreads();
+    run(false, nc - 1, -1, nc - 1, p.dsl, -1, 2);
+    run(false, 0, -1, 1, nullptr, 0, 2);
     if (p.dS0)
-        for (int i = tid; i < DV * DK; i += NT) p.dS0[(size_t)head * DV * DK + i] = W[L::DSL + i];
+        for (int i = tid; i < DD; i += NT) p.dS0[(size_t)hd * DD + i] = S[(i / D) * SS + i % D];
+}
+
+// Shared memory of the chain kernel: the carried matrix and two buffers of A_c.
+template <int D>
+constexpr size_t chain_smem_bytes() { return sizeof(float) * ((size_t)D * (D + 4) + 2 * (size_t)D * (D + 8)); }
+
+// Pass 3: every chunk's gradients from its start state and its end state's gradient.
+template <int DK, int DV, typename QT, typename OT>
+__global__ void __launch_bounds__(NT, 1) bwd_grad_kernel(BwdParams p) {
+    extern __shared__ float4 sm4[];
+    float* sm = reinterpret_cast<float*>(sm4);
+    __shared__ int range_f;
+    const int tid = (int)threadIdx.x;
+    const int nc = (p.T + C - 1) / C, ntask = p.B * p.H * nc;
+    float* W = p.scratch + (size_t)blockIdx.x * p.scratch_floats;
+    if (tid == 0) range_f = 0;
+    for (int t = (int)blockIdx.x; t < ntask; t += (int)gridDim.x) {
+        const int hd = t / nc, c = t % nc, b = hd / p.H, h = hd % p.H;
+        if (!GDR_INB(hd < p.B * p.H, 404)) break;
+        const float* S0c = p.ckpt + (size_t)t * DV * DK;
+        const float* dSL = p.dsl + (size_t)t * DV * DK;
+        chunk_forward<DK, DV, QT, OT>(p, W, b, h, c * C, S0c, true, &range_f, sm);
+        chunk_grads<DK, DV, QT, OT>(p, W, b, h, c * C, S0c, dSL, sm);
+    }
     if (tid == 0 && range_f) atomicOr(&g_device_status, STATUS_RANGE);
 }
 

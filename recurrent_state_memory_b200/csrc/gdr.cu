@@ -696,23 +696,45 @@ static gdr_status check_bwd_desc(const gdr_fwd_desc* d) {
     return GDR_OK;
 }
 
-static size_t bwd_head_floats(int d, int T) {
-    const int nc = (T + 63) / 64;
+// Backward workspace (floats): the chunk coefficients (3 per chunk), the chunk start states and
+// end-state gradients (1 each per chunk), the chains' two buffers per head, and one scratch
+// region per CTA of the two parallel passes (one CTA per SM).
+static size_t bwd_scratch_floats(int d) {
     switch (d) {
-        case 32: return bwd::Lay<32, 32>::floats(nc);
-        case 64: return bwd::Lay<64, 64>::floats(nc);
-        default: return bwd::Lay<128, 128>::floats(nc);
+        case 32: return bwd::Lay<32, 32>::floats();
+        case 64: return bwd::Lay<64, 64>::floats();
+        default: return bwd::Lay<128, 128>::floats();
     }
+}
+static int bwd_grid(long long nh, int T) {
+    const long long tasks = nh * ((T + 63) / 64), sms = device_sm_count();
+    return (int)(tasks < sms ? tasks : sms);
+}
+static size_t bwd_workspace_floats(const gdr_fwd_desc* d) {
+    const size_t nh = (size_t)d->B * d->H, nc = (size_t)(d->T + 63) / 64, dd = (size_t)d->dk * d->dv;
+    return nh * nc * 5 * dd + nh * 2 * dd + (size_t)bwd_grid((long long)nh, d->T) * bwd_scratch_floats(d->dk);
+}
+
+template <typename K>
+static gdr_status launch_bwd_kernel(K kern, int grid, size_t smem, const bwd::BwdParams& p, cudaStream_t st,
+                                   const char* what) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(backward kernel)");
+    kern<<<(unsigned)grid, bwd::NT, smem, st>>>(p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? GDR_OK : cuda_fail(e, what);
 }
 
 template <int D, typename QT, typename OT>
 static gdr_status launch_bwd(const bwd::BwdParams& p, int nh, cudaStream_t st) {
-    auto kern = bwd::chunk_bwd_kernel<D, D, QT, OT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(backward kernel)");
-    kern<<<(unsigned)nh, bwd::NT, bwd::SMEM_BYTES, st>>>(p);
-    e = cudaGetLastError();
-    return e == cudaSuccess ? GDR_OK : cuda_fail(e, "launch(backward kernel)");
+    const int grid = bwd_grid(nh, p.T);
+    gdr_status s = launch_bwd_kernel(bwd::bwd_coef_kernel<D, D, QT, OT>, grid, bwd::SMEM_BYTES, p, st,
+                                     "launch(backward coefficients)");
+    if (s != GDR_OK) return s;
+    s = launch_bwd_kernel(bwd::bwd_chain_kernel<D>, nh, bwd::chain_smem_bytes<D>(), p, st, "launch(backward chains)");
+    if (s != GDR_OK) return s;
+    return launch_bwd_kernel(bwd::bwd_grad_kernel<D, D, QT, OT>, grid, bwd::SMEM_BYTES, p, st,
+                             "launch(backward gradients)");
 }
 
 template <int D>
@@ -956,7 +978,7 @@ int gdr_chunk_fwd_kernel_launches(const gdr_fwd_desc* d) {
 size_t gdr_chunk_bwd_workspace_bytes(const gdr_fwd_desc* d) {
     if (check_bwd_desc(d) != GDR_OK) return 0;
     if (d->B == 0 || d->H == 0 || d->T == 0) return 0;
-    return (size_t)d->B * d->H * bwd_head_floats(d->dk, d->T) * sizeof(float);
+    return bwd_workspace_floats(d) * sizeof(float);
 }
 
 gdr_status gdr_chunk_bwd(const gdr_fwd_desc* d, const void* q, const void* k, const void* v, const float* g,
@@ -988,8 +1010,16 @@ gdr_status gdr_chunk_bwd(const gdr_fwd_desc* d, const void* q, const void* k, co
     p.B = d->B; p.H = d->H; p.T = d->T; p.gate_mode = (int)d->gate_mode; p.scale = d->scale;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.S0 = S0; p.dO = dO; p.dS_T = dS_T;
     p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.dbeta = dbeta; p.dw = dw; p.dS0 = dS0;
-    p.ws = static_cast<float*>(workspace);
-    p.head_floats = bwd_head_floats(d->dk, d->T);
+    {
+        const size_t nh = (size_t)d->B * d->H, nc = (size_t)(d->T + 63) / 64, dd = (size_t)d->dk * d->dv;
+        float* w = static_cast<float*>(workspace);
+        p.coef = w;
+        p.ckpt = p.coef + nh * nc * 3 * dd;
+        p.dsl = p.ckpt + nh * nc * dd;
+        p.chain = p.dsl + nh * nc * dd;
+        p.scratch = p.chain + nh * 2 * dd;
+        p.scratch_floats = bwd_scratch_floats(d->dk);
+    }
     switch (d->dk) {
         case 32: return dispatch_bwd_d<32>(d, p, st);
         case 64: return dispatch_bwd_d<64>(d, p, st);

@@ -234,8 +234,13 @@ def test_backward_checks_its_arguments_without_launching(G):
     assert call(d(1, 1, 64), no_dq) == G.GDR_ERR_INVALID_ARG
     assert call(d(1, 1, 64), full, None, 0) == G.GDR_ERR_WORKSPACE
     assert G.bwd_workspace_bytes(d(1, 1, 64, rotation=True)) == 0
-    per_head = lambda nc: 4 * (64 * 128 * 21 + 64 * 64 * 7 + 64 * 2 + 128 * 4 + 4 * 128 * 128 + nc * 128 * 128)
-    assert G.bwd_workspace_bytes(d(2, 3, 1000)) == 6 * per_head(16)
+    # five d x d fp32 matrices per chunk (three coefficients, the start state, the end state's
+    # gradient), two per head for the chains, and one scratch region per CTA of the parallel
+    # passes (one per SM, at most one per chunk)
+    scratch = 64 * 128 * 18 + 64 * 64 * 7 + 64 * 3 + 128 * 3 + 128 * 128
+    dd = 128 * 128
+    assert G.bwd_workspace_bytes(d(2, 3, 1000)) == 4 * (6 * 16 * 5 * dd + 6 * 2 * dd + 96 * scratch)
+    assert G.bwd_workspace_bytes(d(4, 16, 4096)) == 4 * (64 * 64 * 5 * dd + 64 * 2 * dd + 148 * scratch)
     assert G.bwd_workspace_bytes(d(2, 3, 0)) == 0
 
 
