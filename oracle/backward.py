@@ -114,12 +114,33 @@ def gdr_bwd_head(q, k, v, g, beta, theta, S0, gO, gS, gate_mode, scale, w):
     return o, S, grads
 
 
-def gdr_bwd(q, k, v, g, beta, theta=None, S0=None, gO=None, gS=None, gate_mode=0, scale=1.0, w=None):
+def l2_normalise_bwd(x, gy):
+    """Gradient with respect to x of y = x / sqrt(sum x^2 + eps) over the last axis (the
+    normalisation of ``oracle.l2_normalise``), given gy = dL/dy:
+    dL/dx = (gy - y (y . gy)) / sqrt(sum x^2 + eps)."""
+    from . import L2NORM_EPS
+    x = np.asarray(x, dtype=np.float64)
+    r = 1.0 / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + L2NORM_EPS)
+    y = x * r
+    return (gy - y * np.sum(y * gy, axis=-1, keepdims=True)) * r
+
+
+def gdr_bwd(q, k, v, g, beta, theta=None, S0=None, gO=None, gS=None, gate_mode=0, scale=1.0, w=None,
+            qk_l2norm=False):
     """Whole-batch gradients, head by head (layouts as ``oracle.gdr_fwd``; gO like o, gS like
     S_T).  Returns (o, S_T, grads) with grads a dict of arrays shaped like the inputs
-    ("q", "k", "v", "g", "beta", "w" or None, "theta" or None, "S0")."""
+    ("q", "k", "v", "g", "beta", "w" or None, "theta" or None, "S0").  With qk_l2norm, q and k
+    are L2-normalised per token and head first (as ``oracle.gdr_fwd`` does), and their gradients
+    are taken through the normalisation."""
     f = lambda a: None if a is None else np.asarray(a, dtype=np.float64)
     q, k, v, g, beta, theta, S0, gO, gS, w = map(f, (q, k, v, g, beta, theta, S0, gO, gS, w))
+    if qk_l2norm:
+        from . import l2_normalise
+        o, S_T, out = gdr_bwd(l2_normalise(q), l2_normalise(k), v, g, beta, theta, S0, gO, gS, gate_mode,
+                              scale, w)
+        out["q"] = l2_normalise_bwd(q, out["q"])
+        out["k"] = l2_normalise_bwd(k, out["k"])
+        return o, S_T, out
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     o = np.zeros((B, T, H, dv))

@@ -22,9 +22,9 @@ def _problem(rng, T, H, dk, dv, rotation, untied, gate_mode):
     return dict(q=q, k=k, v=v, g=g, beta=beta, w=w, theta=theta, S0=S0)
 
 
-def _loss(x, gO, gS, gate_mode, scale):
+def _loss(x, gO, gS, gate_mode, scale, qk_l2norm=False):
     o, S_T = oracle.gdr_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["theta"], x["S0"],
-                            gate_mode=gate_mode, scale=scale, w=x["w"])
+                            gate_mode=gate_mode, scale=scale, w=x["w"], qk_l2norm=qk_l2norm)
     return float(np.sum(gO * o) + np.sum(gS * S_T))
 
 
@@ -56,6 +56,38 @@ def test_backward_matches_central_differences(rotation, untied, gate_mode):
         err = np.max(np.abs(grads[n] - fd)) / max(np.max(np.abs(fd)), 1e-12)
         assert err < 1e-6, (n, err)
     assert (grads["w"] is None) == (not untied) and (grads["theta"] is None) == (not rotation)
+
+
+@pytest.mark.parametrize("rotation", [False, True])
+def test_backward_through_the_l2_normalisation_matches_central_differences(rotation):
+    """With qk_l2norm the forward oracle normalises q and k itself; the backward oracle's dq and
+    dk (through the normalisation) against central differences of that forward, on raw q and k
+    of norms far from 1 and one q row near the epsilon's scale."""
+    rng = np.random.default_rng(330 + rotation)
+    T, H, dk, dv, scale = 5, 1, 4, 3, 0.6
+    x = _problem(rng, T, H, dk, dv, rotation, False, 1)
+    x["q"] *= 3.0
+    x["k"] = x["k"] * rng.uniform(0.2, 4.0, (1, T, H, 1))
+    x["q"][0, 2, 0] *= 1e-3                       # |q| ~ 5e-3: the epsilon matters
+    gO = rng.standard_normal((1, T, H, dv))
+    gS = rng.standard_normal((1, H, dv, dk))
+    _, _, grads = bwd.gdr_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["theta"], x["S0"], gO, gS,
+                              gate_mode=1, scale=scale, qk_l2norm=True)
+    h = 1e-7
+    for n in ("q", "k", "beta"):
+        fd = np.zeros_like(x[n])
+        for idx in np.ndindex(x[n].shape):
+            xp = {m: (None if a is None else a.copy()) for m, a in x.items()}
+            xm = {m: (None if a is None else a.copy()) for m, a in x.items()}
+            xp[n][idx] += h
+            xm[n][idx] -= h
+            fd[idx] = (_loss(xp, gO, gS, 1, scale, True) - _loss(xm, gO, gS, 1, scale, True)) / (2 * h)
+        err = np.max(np.abs(grads[n] - fd)) / max(np.max(np.abs(fd)), 1e-12)
+        assert err < 1e-5, (n, err)
+    # the un-normalised gradient is a different vector (the pin sees a missing projection)
+    _, _, raw = bwd.gdr_bwd(oracle.l2_normalise(x["q"]), oracle.l2_normalise(x["k"]), x["v"], x["g"], x["beta"],
+                            x["theta"], x["S0"], gO, gS, gate_mode=1, scale=scale)
+    assert np.max(np.abs(raw["k"] - grads["k"])) > 1e-2 * np.max(np.abs(grads["k"]))
 
 
 def test_backward_adjoint_identities_are_exact():
