@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define GDR_ABI_VERSION 4
+#define GDR_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define GDR_API __attribute__((visibility("default")))
@@ -356,24 +356,31 @@ GDR_API int gdr_chunk_fwd_kernel_launches(const gdr_fwd_desc* desc);
  * affine chunk transfer) in three launches: every chunk's transfer coefficients in parallel
  * (S_L = S0 A_c + B_c and dS0 = G_c + dS_L A_c^T need no state), one short chain per (batch,
  * head) for the chunk start states and the end-state gradients, then every chunk's gradients in
- * parallel.  fp32 throughout (tensor-core products with split-tf32 operands).
+ * parallel.  fp32 throughout (tensor-core products with split-tf32 operands).  With rotation
+ * ("Semidirect Fourier Delta Attention" page, "Core architecture", 2x2 rotation-decay blocks) the
+ * key pairs are complex numbers and the adjoints of the complex decay products are their
+ * conjugates; with qk_l2norm the gradients of q and k are taken through the normalisation
+ * x / sqrt(sum x^2 + 1e-6).
  *
- *   desc            as for gdr_chunk_fwd; dk = dv (32, 64 or 128), rotation = 0, qk_l2norm = 0
- *                   (else GDR_ERR_UNSUPPORTED); algo and segments are ignored.  dO has the
- *                   dtype desc->out_dtype; q, k, v desc->qkv_dtype.
- *   q, k, v, g, beta, w, S0   the forward's inputs, layouts as in gdr_chunk_fwd (w may be NULL:
- *                   w = beta; S0 may be NULL: zero).
+ *   desc            as for gdr_chunk_fwd; dk = dv (32, 64 or 128), else GDR_ERR_UNSUPPORTED;
+ *                   rotation, qk_l2norm, gate_mode and scale as in the forward; algo and
+ *                   segments are ignored.  dO has the dtype desc->out_dtype; q, k, v
+ *                   desc->qkv_dtype.
+ *   q, k, v, g, beta, w, theta, S0   the forward's inputs, layouts as in gdr_chunk_fwd (w may be
+ *                   NULL: w = beta; theta [B,T,H,dk/2] exactly with rotation; S0 may be NULL:
+ *                   zero).
  *   dO [B,T,H,dv]   gradient of o, or NULL (zero).
  *   dS_T [B,H,dv,dk] fp32 gradient of the final state, or NULL (zero).
- *   dq, dk [B,T,H,dk], dv [B,T,H,dv], dg [B,T,H,dk] (of the gate input as given: g itself with
- *                   GDR_GATE_LOGDECAY, the raw gate a with GDR_GATE_NEG_SOFTPLUS), dbeta [B,T,H]:
- *                   fp32 outputs, required when T > 0.
+ *   dq, dk [B,T,H,dk], dv [B,T,H,dv], dg [B,T,H,dk] (rotation: [B,T,H,dk/2]; of the gate input
+ *                   as given: g itself with GDR_GATE_LOGDECAY, the raw gate a with
+ *                   GDR_GATE_NEG_SOFTPLUS), dbeta [B,T,H]: fp32 outputs, required when T > 0.
  *   dw [B,T,H]      fp32, required exactly when w is given (then dbeta is the erase strength's
  *                   gradient alone).
+ *   dtheta [B,T,H,dk/2]  fp32, required exactly with rotation (when T > 0).
  *   dS0 [B,H,dv,dk] fp32 gradient of S0, or NULL (not written).
  *   workspace       device memory of gdr_chunk_bwd_workspace_bytes(desc) bytes, 16-byte aligned
- *                   (five dk x dv fp32 matrices per chunk, two per head, and about 1 MB of
- *                   chunk matrices per SM at d = 128: 1.48 GB at B=4, H=16, T=4096).
+ *                   (five dk x dv fp32 matrices per chunk and about 1 MB of chunk matrices per
+ *                   SM at d = 128: 1.47 GB at B=4, H=16, T=4096).
  * All pointers are device pointers, 16-byte aligned, owned by the caller; the call is
  * asynchronous on `stream` and allocates nothing.  With T = 0, dS0 = dS_T.  Errors: argument
  * checks return before any launch; a decay too strong for the factored form over half a chunk
@@ -384,9 +391,9 @@ GDR_API size_t gdr_chunk_bwd_workspace_bytes(const gdr_fwd_desc* desc);
 GDR_API gdr_status gdr_chunk_bwd(const gdr_fwd_desc* desc,
                                  const void* q, const void* k, const void* v,
                                  const float* g, const float* beta, const float* w,
-                                 const float* S0, const void* dO, const float* dS_T,
-                                 float* dq, float* dk, float* dv, float* dg, float* dbeta,
-                                 float* dw, float* dS0,
+                                 const float* theta, const float* S0, const void* dO,
+                                 const float* dS_T, float* dq, float* dk, float* dv, float* dg,
+                                 float* dbeta, float* dw, float* dtheta, float* dS0,
                                  void* workspace, size_t workspace_bytes, gdr_stream_t stream);
 
 /*

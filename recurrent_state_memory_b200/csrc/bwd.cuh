@@ -28,9 +28,23 @@
 // c + 1 (the caller's dS_T for the last one).  The matrix products are warp-level tf32 tensor-core
 // MMAs with each operand split into a tf32 high part and a tf32 remainder (three products per
 // step), which keeps fp32 accuracy; the per-chunk matrices live in a per-head region of the
-// workspace (they stay in L1/L2).  Real decay only; the rotation variant's gradients exist in the
-// oracle.  Tokens past T are zero padding (k = q = v = 0, beta = w = 0, log-decay 0): exact
-// identity transitions whose gradients are not written.
+// workspace (they stay in L1/L2).  Tokens past T are zero padding (k = q = v = 0, beta = w = 0,
+// log-decay 0): exact identity transitions whose gradients are not written.
+//
+// Rotation ("Semidirect Fourier Delta Attention" page, "Core architecture", real implementation:
+// 2x2 rotation-decay blocks).  Key pair j of a row is the complex number x + i y and the chunk's
+// cumulative factor is Lam_r = e^{rho_r + i phi_r} (rho, phi: in-chunk sums of log alpha and of
+// theta).  Every tile factor becomes a complex multiplier per pair: Kt = K F, Qt = scale Q F,
+// Kh = K Fh, Kd = K Fh (Lam_L / Lam_m), S0p = S0 Lam_m with F = conj(Lam_r / Lam_m) and
+// Fh = Lam_m / Lam_r (same phase, inverse magnitude); the products stay real (the dot product of
+// the (re, im) pairs).  Backwards the multipliers are conjugated (the adjoint of a complex
+// product), dg takes drho and dtheta takes dphi, each summed in reverse over the chunk:
+//   drho = Re(conj(dKt) Kt + conj(dQt) Qt - conj(dKh) Kh - conj(dKd) Kd)
+//   dphi = Im(conj(dKt) Kt + conj(dQt) Qt + conj(dKh) Kh + conj(dKd) Kd)
+// plus, at the last token, Re / -Im of sum_rows conj(dS_L) S0 Lam_L and sum_r conj(dKd) Kd.
+//
+// L2 normalisation (qk_l2norm): the chunk algebra runs on qn = q / sqrt(|q|^2 + 1e-6) and kn;
+// dq = (dqn - qn (qn . dqn)) / sqrt(|q|^2 + 1e-6), and the same for k.
 #pragma once
 
 #include "common.cuh"
@@ -40,6 +54,7 @@ namespace bwd {
 
 constexpr int C = 64;
 constexpr int NT = 512;
+static_assert(NT == C * 8, "eight threads per token in the per-token reductions");
 constexpr int NW = NT / 32;
 constexpr unsigned STATUS_RANGE = 2u;
 
@@ -52,6 +67,7 @@ struct BwdParams {
     const float* g;
     const float* beta;
     const float* w;          // write strength [B,T,H] or nullptr (w = beta)
+    const float* theta;      // rotation angles [B,T,H,dk/2] (rot) or nullptr
     const float* S0;         // [B,H,dv,dk] or nullptr (zero)
     const void* dO;          // [B,T,H,dv] (the output's dtype) or nullptr (zero)
     const float* dS_T;       // [B,H,dv,dk] or nullptr (zero)
@@ -62,11 +78,13 @@ struct BwdParams {
     float* dbeta;            // [B,T,H]
     float* dw;               // [B,T,H] (with w) or nullptr
     float* dS0;              // [B,H,dv,dk] or nullptr
+    float* dtheta;           // [B,T,H,dk/2] (rot) or nullptr
+    int rot;                 // 1: 2x2 rotation-decay blocks (g and theta have dk/2 entries per token)
+    int norm;                // 1: q and k L2-normalised per token first
     // workspace parts (floats)
     float* coef;             // [B*H][nc][3][dv*dk]: A_c (dk x dk, in a dv x dk slot), B_c, G_c
     float* ckpt;             // [B*H][nc][dv*dk]: the state at each chunk start
     float* dsl;              // [B*H][nc][dv*dk]: the gradient of each chunk's end state
-    float* chain;            // [B*H][2][dv*dk]: the chain's two buffers
     float* scratch;          // [grid][scratch_floats]: each CTA's chunk matrices
     size_t scratch_floats;
 };
@@ -86,8 +104,10 @@ struct Lay {
     static constexpr int DQT = DR + C * DV, DKH = DQT + C * DK, DKD = DKH + C * DK, DKT = DKD + C * DK;
     static constexpr int K = DKT, Q = DKH;          // raw k and q (chunk_forward only)
     static constexpr int BT = DKT + C * DK, WT = BT + C, DBS = WT + C;   // beta, w, dbeta parts
-    static constexpr int E31 = DBS + C, EGL = E31 + DK, ED = EGL + DK;   // column vectors
-    static constexpr int S0P = ED + DK;
+    static constexpr int E31 = DBS + C, EGL = E31 + DK, ED = EGL + DK;   // column vectors (rotation:
+                                                                         // (re, im) per key pair)
+    static constexpr int NQV = ED + DK, NKV = NQV + C;   // per-token 1/|q|, 1/|k| (qk_l2norm)
+    static constexpr int S0P = NKV + C;
     static constexpr size_t floats() { return (size_t)S0P + (size_t)DV * DK; }
 };
 
@@ -194,19 +214,33 @@ __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0
     auto tok = [&](int r) -> size_t { return ((size_t)b * p.T + (t0 + r)) * p.H + h; };
     // raw inputs of the chunk, zero past T (four loads in flight per thread); the log-decays go
     // to shared memory for the scan below
+    // (rotation: column 2j holds log alpha of pair j, column 2j + 1 its angle theta)
     float* sg = sm;                       // [C][DK] log alpha, then gam
-    float* sg31 = sm + C * DK;            // [DK]
+    float* sg31 = sm + C * DK;            // [DK] gam at the reference token
+    float* sgl = sg31 + DK;               // [DK] gam at the last token
+    const int ng = p.rot ? DK / 2 : DK;   // gate entries per token
     constexpr int NK = C * DK / NT, NV = C * DV / NT;
 #pragma unroll
     for (int u = 0; u < NK; ++u) {
         const int i = tid + u * NT, r = i / DK, d = i % DK;
         const bool ok = t0 + r < p.T;
         const size_t o = tok(r) * DK + d;
-        const float kk = ok ? ldx(k, o) : 0.f, qq = ok ? ldx(q, o) : 0.f, a = ok ? p.g[o] : 0.f;
+        const float kk = ok ? ldx(k, o) : 0.f, qq = ok ? ldx(q, o) : 0.f;
         W[L::K + i] = kk;
         W[L::Q + i] = qq;
-        sg[i] = ok ? log_decay(a, p.gate_mode) : 0.f;
-        W[L::DLG + i] = ok ? (p.gate_mode == 1 ? -1.f / (1.f + expf(-a)) : 1.f) : 0.f;   // d(-softplus a)/da = -sigmoid(a)
+        float lg = 0.f, dl = 0.f;
+        if (ok) {
+            if (p.rot && (d & 1)) {
+                lg = p.theta[tok(r) * ng + (d >> 1)];          // d phi / d theta = 1
+                dl = 1.f;
+            } else {
+                const float a = p.g[tok(r) * ng + (p.rot ? d >> 1 : d)];
+                lg = log_decay(a, p.gate_mode);
+                dl = p.gate_mode == 1 ? -1.f / (1.f + expf(-a)) : 1.f;   // d(-softplus a)/da = -sigmoid(a)
+            }
+        }
+        sg[i] = lg;
+        W[L::DLG + i] = dl;
     }
 #pragma unroll
     for (int u = 0; u < NV; ++u) {
@@ -225,7 +259,26 @@ __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0
         W[L::WT + tid] = ok ? (p.w ? p.w[tok(tid)] : bt) : 0.f;
     }
     __syncthreads();
-    // cumulative log-decay per key dim, relative to token m = 31, and the column decays
+    // qk_l2norm: 1/|k| and 1/|q| per token, eight threads a token
+    if (p.norm) {
+        const int r = tid >> 3, part = tid & 7;
+        float sk = 0.f, sq = 0.f;
+        for (int d = part; d < DK; d += 8) {
+            const float a = W[L::K + r * DK + d], c = W[L::Q + r * DK + d];
+            sk += a * a;
+            sq += c * c;
+        }
+#pragma unroll
+        for (int off = 4; off >= 1; off >>= 1) {
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        }
+        if (part == 0) {
+            W[L::NKV + r] = rsqrtf(sk + 1e-6f);
+            W[L::NQV + r] = rsqrtf(sq + 1e-6f);
+        }
+    }
+    // cumulative log-decay (rotation: and angle) per key dim, the reference token m = 31
     if (tid < DK) {
         const int d = tid;
         float gam = 0.f, g31 = 0.f;
@@ -234,19 +287,52 @@ __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0
             sg[r * DK + d] = gam;
             if (r == 31) g31 = gam;
         }
-        const float gl = gam;
         sg31[d] = g31;
-        W[L::E31 + d] = expf(g31);
-        W[L::EGL + d] = expf(gl);
-        W[L::ED + d] = expf(gl - g31);
+        sgl[d] = gam;
     }
     __syncthreads();
+    // column factors e^{gam_m}, e^{gam_L}, e^{gam_L - gam_m} (rotation: Lam_m, Lam_L, Lam_L / Lam_m
+    // as (re, im) per pair) and the tile multipliers EG = e^{gam - gam_m}, EGI = e^{-(gam - gam_m)}
+    // (rotation: F and Fh per pair)
+    if (tid < DK) {
+        const int d = tid;
+        if (!p.rot) {
+            W[L::E31 + d] = expf(sg31[d]);
+            W[L::EGL + d] = expf(sgl[d]);
+            W[L::ED + d] = expf(sgl[d] - sg31[d]);
+        } else {
+            const int e = d & ~1;
+            const bool im = d & 1;
+            auto cs = [&](float ang) -> float {
+                float sn, c;
+                sincosf(ang, &sn, &c);
+                return im ? sn : c;
+            };
+            W[L::E31 + d] = expf(sg31[e]) * cs(sg31[e + 1]);
+            W[L::EGL + d] = expf(sgl[e]) * cs(sgl[e + 1]);
+            W[L::ED + d] = expf(sgl[e] - sg31[e]) * cs(sgl[e + 1] - sg31[e + 1]);
+        }
+    }
     {
         bool bad = false;
         for (int i = tid; i < C * DK; i += NT) {
-            const float x = sg[i] - sg31[i % DK];
-            const float e = expf(x), ei = expf(-x);
-            if (!(e < 3e38f) || !(ei < 3e38f)) bad = true;
+            const int d = i % DK;
+            float e, ei;
+            if (!p.rot) {
+                const float x = sg[i] - sg31[d];
+                e = expf(x);
+                ei = expf(-x);
+                if (!(e < 3e38f) || !(ei < 3e38f)) bad = true;
+            } else {
+                const int i0 = i & ~1, d0 = d & ~1;
+                const float x = sg[i0] - sg31[d0];
+                float sn, c;
+                sincosf(sg[i0 + 1] - sg31[d0 + 1], &sn, &c);
+                const float m = expf(x), mi = expf(-x), f = (d & 1) ? -sn : c;    // e^{-i dphi}
+                if (!(m < 3e38f) || !(mi < 3e38f)) bad = true;
+                e = m * f;
+                ei = mi * f;
+            }
             W[L::EG + i] = e;
             W[L::EGI + i] = ei;
         }
@@ -254,15 +340,39 @@ __device__ void chunk_forward(const BwdParams& p, float* W, int b, int h, int t0
     }
     __syncthreads();
     for (int i = tid; i < C * DK; i += NT) {
-        const int d = i % DK;
-        const float kk = W[L::K + i];
-        W[L::KT + i] = kk * W[L::EG + i];
-        W[L::KH + i] = kk * W[L::EGI + i];
-        W[L::QT + i] = p.scale * W[L::Q + i] * W[L::EG + i];
-        W[L::KD + i] = kk * W[L::EGI + i] * W[L::ED + d];
+        const int r = i / DK, d = i % DK;
+        const float nk = p.norm ? W[L::NKV + r] : 1.f, nq = p.norm ? p.scale * W[L::NQV + r] : p.scale;
+        if (!p.rot) {
+            const float kk = W[L::K + i] * nk;
+            W[L::KT + i] = kk * W[L::EG + i];
+            W[L::KH + i] = kk * W[L::EGI + i];
+            W[L::QT + i] = nq * W[L::Q + i] * W[L::EG + i];
+            W[L::KD + i] = kk * W[L::EGI + i] * W[L::ED + d];
+        } else {
+            // complex products per pair: component im of (ar + i ai)(br + i bi)
+            const int i0 = i & ~1, d0 = d & ~1;
+            const bool im = d & 1;
+            auto cm = [im](float ar, float ai, float br, float bi) { return im ? ar * bi + ai * br : ar * br - ai * bi; };
+            const float kx = W[L::K + i0] * nk, ky = W[L::K + i0 + 1] * nk;
+            const float qx = W[L::Q + i0] * nq, qy = W[L::Q + i0 + 1] * nq;
+            const float fr = W[L::EG + i0], fi = W[L::EG + i0 + 1], hr = W[L::EGI + i0], hi = W[L::EGI + i0 + 1];
+            const float dr = W[L::ED + d0], di = W[L::ED + d0 + 1];
+            W[L::KT + i] = cm(kx, ky, fr, fi);
+            W[L::KH + i] = cm(kx, ky, hr, hi);
+            W[L::QT + i] = cm(qx, qy, fr, fi);
+            W[L::KD + i] = cm(kx, ky, hr * dr - hi * di, hr * di + hi * dr);
+        }
     }
     if (S0)
-        for (int i = tid; i < DV * DK; i += NT) W[L::S0P + i] = S0[i] * W[L::E31 + i % DK];
+        for (int i = tid; i < DV * DK; i += NT) {
+            if (!p.rot) {
+                W[L::S0P + i] = S0[i] * W[L::E31 + i % DK];
+            } else {
+                const int i0 = i & ~1, d0 = i0 % DK;
+                const float x = S0[i0], y = S0[i0 + 1], mr = W[L::E31 + d0], mi = W[L::E31 + d0 + 1];
+                W[L::S0P + i] = (i & 1) ? x * mi + y * mr : x * mr - y * mi;
+            }
+        }
     __syncthreads();
     mm<false, true>(W + L::AP, C, W + L::KT, DK, W + L::KH, DK, C, C, DK, 1.f, false, sm);      // Ap = Kt Kh^T
     mm<false, true>(W + L::PM, C, W + L::QT, DK, W + L::KH, DK, C, C, DK, 1.f, false, sm);      // Qt Kh^T
@@ -381,29 +491,75 @@ __device__ void chunk_grads(const BwdParams& p, float* W, int b, int h, int t0, 
     __syncthreads();
     mm<false, false>(W + L::DKT, DK, W + L::DA, C, W + L::KH, DK, C, DK, C, 1.f, true, sm);
     __syncthreads();
-    // dq, dk; dgam (shared memory)
+    // dq, dk (qk_l2norm: those of the normalised q and k, in X1.. and DA.., C x DK each); dgam
+    // (rotation: drho in column 2j, dphi in column 2j + 1) in shared memory
     float* sdg = sm;                  // [C][DK] dgam, then dg
-    float* sdl = sm + C * DK;         // [C][DK] d log alpha / d gate input
+    float* sdl = sm + C * DK;         // [C][DK] d log alpha / d gate input (rotation: 1 for the angle)
     float* scs = sm + 2 * C * DK;     // [NT / DK][DK] column-sum parts
+    float* gqn = W + L::X1;
+    float* gkn = W + L::DA;
+    static_assert(L::X2 == L::X1 + C * C && L::DPM == L::DA + C * C && DK <= 2 * C, "C x DK over two C x C tiles");
     for (int i = tid; i < C * DK; i += NT) {
         const int r = i / DK, d = i % DK;
-        const float eg = W[L::EG + i], egi = W[L::EGI + i];
-        const float gkt = W[L::DKT + i], gkh = W[L::DKH + i], gqt = W[L::DQT + i], gkd = W[L::DKD + i];
-        if (t0 + r < p.T) {
-            const size_t o = (((size_t)b * p.T + t0 + r) * p.H + h) * DK + d;
-            p.dq[o] = p.scale * gqt * eg;
-            p.dk[o] = gkt * eg + gkh * egi + gkd * egi * W[L::ED + d];
+        float gq, gk, dgm;
+        if (!p.rot) {
+            const float eg = W[L::EG + i], egi = W[L::EGI + i];
+            const float gkt = W[L::DKT + i], gkh = W[L::DKH + i], gqt = W[L::DQT + i], gkd = W[L::DKD + i];
+            gq = p.scale * gqt * eg;
+            gk = gkt * eg + gkh * egi + gkd * egi * W[L::ED + d];
+            dgm = gkt * W[L::KT + i] + gqt * W[L::QT + i] - gkh * W[L::KH + i] - gkd * W[L::KD + i];
+        } else {
+            const int i0 = i & ~1, d0 = d & ~1;
+            const bool im = d & 1;
+            // component im of a conj(b); Re and Im of conj(a) b over the pair at offset o
+            auto cmc = [im](float ar, float ai, float br, float bi) { return im ? ai * br - ar * bi : ar * br + ai * bi; };
+            auto pr = [&](int ga, int x) {
+                const float ar = W[ga + i0], ai = W[ga + i0 + 1], br = W[x + i0], bi = W[x + i0 + 1];
+                return im ? ar * bi - ai * br : ar * br + ai * bi;
+            };
+            const float fr = W[L::EG + i0], fi = W[L::EG + i0 + 1], hr = W[L::EGI + i0], hi = W[L::EGI + i0 + 1];
+            const float dr = W[L::ED + d0], di = W[L::ED + d0 + 1];
+            const float gr = hr * dr - hi * di, gi = hr * di + hi * dr;       // Fh Lam_L / Lam_m
+            gq = p.scale * cmc(W[L::DQT + i0], W[L::DQT + i0 + 1], fr, fi);
+            gk = cmc(W[L::DKT + i0], W[L::DKT + i0 + 1], fr, fi) + cmc(W[L::DKH + i0], W[L::DKH + i0 + 1], hr, hi) +
+                 cmc(W[L::DKD + i0], W[L::DKD + i0 + 1], gr, gi);
+            const float sgn = im ? 1.f : -1.f;       // Kh and Kd: -Re for drho, +Im for dphi
+            dgm = pr(L::DKT, L::KT) + pr(L::DQT, L::QT) + sgn * (pr(L::DKH, L::KH) + pr(L::DKD, L::KD));
         }
-        sdg[i] = gkt * W[L::KT + i] + gqt * W[L::QT + i] - gkh * W[L::KH + i] - gkd * W[L::KD + i];
+        if (p.norm) {
+            gqn[i] = gq;
+            gkn[i] = gk;
+        } else if (t0 + r < p.T) {
+            const size_t o = (((size_t)b * p.T + t0 + r) * p.H + h) * DK + d;
+            p.dq[o] = gq;
+            p.dk[o] = gk;
+        }
+        sdg[i] = dgm;
         sdl[i] = W[L::DLG + i];
     }
     {   // column sums for the last token's decay terms: NT / DK threads per key dim
         constexpr int NP = NT / DK;
         const int d = tid % DK, part = tid / DK;
         float s0 = 0.f, sd = 0.f;
-        for (int i = part; i < DV; i += NP) s0 += S0c[i * DK + d] * dSL[i * DK + d];
-        for (int r = part; r < C; r += NP) sd += W[L::DKD + r * DK + d] * W[L::KD + r * DK + d];
-        scs[part * DK + d] = W[L::EGL + d] * s0 + sd;
+        if (!p.rot) {
+            for (int i = part; i < DV; i += NP) s0 += S0c[i * DK + d] * dSL[i * DK + d];
+            for (int r = part; r < C; r += NP) sd += W[L::DKD + r * DK + d] * W[L::KD + r * DK + d];
+            scs[part * DK + d] = W[L::EGL + d] * s0 + sd;
+        } else {
+            // drho_L: Re sum conj(dS_L) S0 Lam_L + Re sum conj(dKd) Kd; dphi_L: -Im of the same
+            const int d0 = d & ~1;
+            const bool im = d & 1;
+            const float lr = W[L::EGL + d0], li = W[L::EGL + d0 + 1];
+            auto pr = [im](float ar, float ai, float br, float bi) { return im ? -(ar * bi - ai * br) : ar * br + ai * bi; };
+            for (int i = part; i < DV; i += NP) {
+                const float x = S0c[i * DK + d0], y = S0c[i * DK + d0 + 1];
+                s0 += pr(dSL[i * DK + d0], dSL[i * DK + d0 + 1], x * lr - y * li, x * li + y * lr);
+            }
+            for (int r = part; r < C; r += NP)
+                sd += pr(W[L::DKD + r * DK + d0], W[L::DKD + r * DK + d0 + 1], W[L::KD + r * DK + d0],
+                         W[L::KD + r * DK + d0 + 1]);
+            scs[part * DK + d] = s0 + sd;
+        }
     }
     __syncthreads();
     if (tid < DK) {     // reverse cumulative sum over the chunk's tokens
@@ -416,9 +572,44 @@ __device__ void chunk_grads(const BwdParams& p, float* W, int b, int h, int t0, 
         }
     }
     __syncthreads();
+    const int ng = p.rot ? DK / 2 : DK;
     for (int i = tid; i < C * DK; i += NT) {
         const int r = i / DK, d = i % DK;
-        if (t0 + r < p.T) p.dg[(((size_t)b * p.T + t0 + r) * p.H + h) * DK + d] = sdg[i];
+        if (t0 + r >= p.T) continue;
+        const size_t tk = ((size_t)b * p.T + t0 + r) * p.H + h;
+        if (!p.rot) p.dg[tk * DK + d] = sdg[i];
+        else (d & 1 ? p.dtheta : p.dg)[tk * ng + (d >> 1)] = sdg[i];
+    }
+    if (p.norm) {
+        // through the normalisation, per token (eight threads each; rows past T are computed
+        // from the zero padding and not written): d x = r (dxn - xn (xn . dxn)), r = 1 / |x|
+        const QT* q = static_cast<const QT*>(p.q);
+        const QT* k = static_cast<const QT*>(p.k);
+        const int r = tid >> 3, part = tid & 7;
+        const bool ok = t0 + r < p.T;
+        const size_t ob = (((size_t)b * p.T + (ok ? t0 + r : 0)) * p.H + h) * DK;
+        float sk = 0.f, sq = 0.f, pk = 0.f, pq = 0.f;
+        for (int d = part; d < DK; d += 8) {
+            const float kk = ok ? ldx(k, ob + d) : 0.f, qq = ok ? ldx(q, ob + d) : 0.f;
+            sk += kk * kk;
+            sq += qq * qq;
+            pk += kk * gkn[r * DK + d];
+            pq += qq * gqn[r * DK + d];
+        }
+#pragma unroll
+        for (int off = 4; off >= 1; off >>= 1) {
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            pk += __shfl_xor_sync(0xffffffffu, pk, off);
+            pq += __shfl_xor_sync(0xffffffffu, pq, off);
+        }
+        const float rk = rsqrtf(sk + 1e-6f), rq = rsqrtf(sq + 1e-6f);
+        const float ck = rk * rk * rk * pk, cq = rq * rq * rq * pq;
+        if (ok)
+            for (int d = part; d < DK; d += 8) {
+                p.dk[ob + d] = rk * gkn[r * DK + d] - ck * ldx(k, ob + d);
+                p.dq[ob + d] = rq * gqn[r * DK + d] - cq * ldx(q, ob + d);
+            }
     }
     __syncthreads();
 }
@@ -460,10 +651,19 @@ __global__ void __launch_bounds__(NT, 1) bwd_coef_kernel(BwdParams p) {
         mm<false, false>(W + L::DKH, DK, W + L::TM, C, W + L::DKT, DK, C, DK, C, 1.f, false, sm);
         __syncthreads();
         // A_c = diag(e^{gam_L}) - diag(e^{gam_m}) N ; B_c = E0^T Kd ; X = P W1 (in DKD)
-        for (int i = tid; i < DK * DK; i += NT) {
-            const int r = i / DK, cc = i % DK;
-            A[i] = (r == cc ? W[L::EGL + r] : 0.f) - W[L::E31 + r] * A[i];
-        }
+        if (!p.rot)
+            for (int i = tid; i < DK * DK; i += NT) {
+                const int r = i / DK, cc = i % DK;
+                A[i] = (r == cc ? W[L::EGL + r] : 0.f) - W[L::E31 + r] * A[i];
+            }
+        else    // the 2x2 blocks of right-multiplication by Lam_L and Lam_m: [[re, im], [-im, re]]
+            for (int i = tid; i < DK / 2 * DK; i += NT) {
+                const int r0 = 2 * (i / DK), cc = i % DK;
+                const float n0 = A[r0 * DK + cc], n1 = A[(r0 + 1) * DK + cc];
+                const float lr = W[L::EGL + r0], li = W[L::EGL + r0 + 1], mr = W[L::E31 + r0], mi = W[L::E31 + r0 + 1];
+                A[r0 * DK + cc] = (cc == r0 ? lr : cc == r0 + 1 ? li : 0.f) - (mr * n0 + mi * n1);
+                A[(r0 + 1) * DK + cc] = (cc == r0 ? -li : cc == r0 + 1 ? lr : 0.f) - (mr * n1 - mi * n0);
+            }
         mm<true, false>(Bc, DK, W + L::E, DV, W + L::KD, DK, DV, DK, C, 1.f, false, sm);
         mm<false, false>(W + L::DKD, DK, W + L::PM, C, W + L::DKH, DK, C, DK, C, 1.f, false, sm);
         __syncthreads();
@@ -471,7 +671,14 @@ __global__ void __launch_bounds__(NT, 1) bwd_coef_kernel(BwdParams p) {
         for (int i = tid; i < C * DK; i += NT) W[L::DKD + i] = W[L::QT + i] - W[L::DKD + i];
         __syncthreads();
         mm<true, false>(G, DK, W + L::DO, DV, W + L::DKD, DK, DV, DK, C, 1.f, false, sm);
-        for (int i = tid; i < DV * DK; i += NT) G[i] *= W[L::E31 + i % DK];
+        if (!p.rot)
+            for (int i = tid; i < DV * DK; i += NT) G[i] *= W[L::E31 + i % DK];
+        else    // rows times conj(Lam_m): the transpose of the right-multiplication by Lam_m
+            for (int i = 2 * tid; i < DV * DK; i += 2 * NT) {
+                const float x = G[i], y = G[i + 1], mr = W[L::E31 + i % DK], mi = W[L::E31 + i % DK + 1];
+                G[i] = x * mr + y * mi;
+                G[i + 1] = y * mr - x * mi;
+            }
         __syncthreads();
     }
     if (tid == 0 && range_f) atomicOr(&g_device_status, STATUS_RANGE);

@@ -691,14 +691,12 @@ static gdr_status check_bwd_desc(const gdr_fwd_desc* d) {
     gdr_status s = check_fwd_desc(d);
     if (s != GDR_OK) return s;
     if (d->dk != d->dv) return fail(GDR_ERR_UNSUPPORTED, "the backward needs dk = dv%s");
-    if (d->rotation) return fail(GDR_ERR_UNSUPPORTED, "the backward has no rotation form (real decay only)%s");
-    if (d->qk_l2norm) return fail(GDR_ERR_UNSUPPORTED, "the backward takes q and k as given (no qk_l2norm)%s");
     return GDR_OK;
 }
 
 // Backward workspace (floats): the chunk coefficients (3 per chunk), the chunk start states and
-// end-state gradients (1 each per chunk), the chains' two buffers per head, and one scratch
-// region per CTA of the two parallel passes (one CTA per SM).
+// end-state gradients (1 each per chunk), and one scratch region per CTA of the two parallel
+// passes (one CTA per SM).
 static size_t bwd_scratch_floats(int d) {
     switch (d) {
         case 32: return bwd::Lay<32, 32>::floats();
@@ -712,7 +710,7 @@ static int bwd_grid(long long nh, int T) {
 }
 static size_t bwd_workspace_floats(const gdr_fwd_desc* d) {
     const size_t nh = (size_t)d->B * d->H, nc = (size_t)(d->T + 63) / 64, dd = (size_t)d->dk * d->dv;
-    return nh * nc * 5 * dd + nh * 2 * dd + (size_t)bwd_grid((long long)nh, d->T) * bwd_scratch_floats(d->dk);
+    return nh * nc * 5 * dd + (size_t)bwd_grid((long long)nh, d->T) * bwd_scratch_floats(d->dk);
 }
 
 template <typename K>
@@ -982,9 +980,9 @@ size_t gdr_chunk_bwd_workspace_bytes(const gdr_fwd_desc* d) {
 }
 
 gdr_status gdr_chunk_bwd(const gdr_fwd_desc* d, const void* q, const void* k, const void* v, const float* g,
-                         const float* beta, const float* w, const float* S0, const void* dO, const float* dS_T,
-                         float* dq, float* dk, float* dv, float* dg, float* dbeta, float* dw, float* dS0,
-                         void* workspace, size_t workspace_bytes, gdr_stream_t stream) {
+                         const float* beta, const float* w, const float* theta, const float* S0, const void* dO,
+                         const float* dS_T, float* dq, float* dk, float* dv, float* dg, float* dbeta, float* dw,
+                         float* dtheta, float* dS0, void* workspace, size_t workspace_bytes, gdr_stream_t stream) {
     t_detail[0] = 0;
     gdr_status s = check_bwd_desc(d);
     if (s != GDR_OK) return s;
@@ -1001,23 +999,26 @@ gdr_status gdr_chunk_bwd(const gdr_fwd_desc* d, const void* q, const void* k, co
     if (!q || !k || !v || !g || !beta || !dq || !dk || !dv || !dg || !dbeta)
         return fail(GDR_ERR_INVALID_ARG, "q, k, v, g, beta, dq, dk, dv, dg and dbeta are required%s");
     if ((w == nullptr) != (dw == nullptr)) return fail(GDR_ERR_INVALID_ARG, "dw is required exactly when w is given%s");
-    const void* ptrs[] = {q, k, v, g, beta, w, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dw, dS0, workspace};
+    if (d->rotation ? (!theta || !dtheta) : (theta || dtheta))
+        return fail(GDR_ERR_INVALID_ARG, "theta and dtheta are required exactly with rotation%s");
+    const void* ptrs[] = {q, k, v, g, beta, w, theta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dw, dtheta, dS0, workspace};
     for (const void* x : ptrs)
         if (x && !aligned16(x)) return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
     const size_t need = gdr_chunk_bwd_workspace_bytes(d);
     if (!workspace || workspace_bytes < need) return fail(GDR_ERR_WORKSPACE, "workspace too small%s");
     bwd::BwdParams p;
     p.B = d->B; p.H = d->H; p.T = d->T; p.gate_mode = (int)d->gate_mode; p.scale = d->scale;
-    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.S0 = S0; p.dO = dO; p.dS_T = dS_T;
-    p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.dbeta = dbeta; p.dw = dw; p.dS0 = dS0;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.w = w; p.theta = theta; p.S0 = S0; p.dO = dO; p.dS_T = dS_T;
+    p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.dbeta = dbeta; p.dw = dw; p.dS0 = dS0; p.dtheta = dtheta;
+    p.rot = d->rotation ? 1 : 0;
+    p.norm = d->qk_l2norm ? 1 : 0;
     {
         const size_t nh = (size_t)d->B * d->H, nc = (size_t)(d->T + 63) / 64, dd = (size_t)d->dk * d->dv;
         float* w = static_cast<float*>(workspace);
         p.coef = w;
         p.ckpt = p.coef + nh * nc * 3 * dd;
         p.dsl = p.ckpt + nh * nc * dd;
-        p.chain = p.dsl + nh * nc * dd;
-        p.scratch = p.chain + nh * 2 * dd;
+        p.scratch = p.dsl + nh * nc * dd;
         p.scratch_floats = bwd_scratch_floats(d->dk);
     }
     switch (d->dk) {

@@ -94,13 +94,13 @@ def lib() -> ctypes.CDLL:
         L.gdr_chunk_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.gdr_chunk_bwd_workspace_bytes.argtypes = [ctypes.POINTER(FwdDesc)]
         L.gdr_chunk_bwd.restype = ctypes.c_int
-        L.gdr_chunk_bwd.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp,
-                                    fp, fp, fp, fp, fp, fp, fp, vp, ctypes.c_size_t, vp]
+        L.gdr_chunk_bwd.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, fp,
+                                    fp, fp, fp, fp, fp, fp, fp, fp, vp, ctypes.c_size_t, vp]
         L.gdr_chunk_fwd_noalloc.restype = ctypes.c_int
         L.gdr_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp, vp]
         L.gdr_debug_set_tc_fault.restype = None
         L.gdr_debug_set_tc_fault.argtypes = [ctypes.c_int, ctypes.c_ulonglong]
-        if L.gdr_abi_version() != 4:
+        if L.gdr_abi_version() != 5:
             raise RuntimeError("libgdr.so ABI version mismatch")
         _lib = L
     return _lib
@@ -302,23 +302,28 @@ def bwd_workspace_bytes(desc: FwdDesc) -> int:
 
 
 def chunk_bwd(q, k, v, g, beta, S0=None, dO=None, dS_T=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
-              w=None, out_dtype=None, want_dS0=True, workspace=None, stream=None, chunk=64):
-    """Backward of ``chunk_fwd`` (real decay, dk = dv): the gradients of every input given dO
-    (like o, dtype out_dtype, default q's) and dS_T (fp32 like S_T); either may be None (zero).
-    Returns a dict of fp32 tensors "q", "k", "v", "g", "beta", "w" (None without w) and "S0"
-    (None unless want_dS0).  Asynchronous on `stream` (default: the current stream)."""
+              w=None, theta=None, qk_l2norm=False, out_dtype=None, want_dS0=True, workspace=None, stream=None,
+              chunk=64):
+    """Backward of ``chunk_fwd`` (dk = dv): the gradients of every input given dO (like o, dtype
+    out_dtype, default q's) and dS_T (fp32 like S_T); either may be None (zero).  theta (rotation)
+    and qk_l2norm as in the forward.  Returns a dict of fp32 tensors "q", "k", "v", "g", "beta",
+    "w" (None without w), "theta" (None without rotation) and "S0" (None unless want_dS0).
+    Asynchronous on `stream` (default: the current stream)."""
     dev = q.device
     B, T, H, dk = q.shape
     dv = v.shape[-1]
+    rotation = theta is not None
+    ng = dk // 2 if rotation else dk
     out_dtype = out_dtype or (dO.dtype if dO is not None else q.dtype)
     _need(q, "q", device=dev)
     _need(k, "k", q.dtype, dev)
     _need(v, "v", q.dtype, dev)
     _need(g, "g", torch.float32, dev)
     _need(beta, "beta", torch.float32, dev)
-    if tuple(k.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv) or tuple(g.shape) != (B, T, H, dk):
+    if tuple(k.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv) or tuple(g.shape) != (B, T, H, ng):
         raise ValueError("q, k, v, g shapes disagree")
-    for t, n, shp in ((w, "w", (B, T, H)), (S0, "S0", (B, H, dv, dk)), (dS_T, "dS_T", (B, H, dv, dk))):
+    for t, n, shp in ((w, "w", (B, T, H)), (S0, "S0", (B, H, dv, dk)), (dS_T, "dS_T", (B, H, dv, dk)),
+                      (theta, "theta", (B, T, H, dk // 2))):
         if t is not None:
             _need(t, n, torch.float32, dev)
             if tuple(t.shape) != shp:
@@ -329,18 +334,21 @@ def chunk_bwd(q, k, v, g, beta, S0=None, dO=None, dS_T=None, *, gate_mode=GATE_N
             raise ValueError("dO has the wrong shape")
     f32 = dict(dtype=torch.float32, device=dev)
     grads = {"q": torch.empty((B, T, H, dk), **f32), "k": torch.empty((B, T, H, dk), **f32),
-             "v": torch.empty((B, T, H, dv), **f32), "g": torch.empty((B, T, H, dk), **f32),
+             "v": torch.empty((B, T, H, dv), **f32), "g": torch.empty((B, T, H, ng), **f32),
              "beta": torch.empty((B, T, H), **f32), "w": None if w is None else torch.empty((B, T, H), **f32),
+             "theta": torch.empty((B, T, H, dk // 2), **f32) if rotation else None,
              "S0": torch.empty((B, H, dv, dk), **f32) if want_dS0 else None}
-    desc = fwd_desc(B, H, T, dk, dv, q.dtype, out_dtype, gate_mode, False, scale, "auto", chunk)
+    desc = fwd_desc(B, H, T, dk, dv, q.dtype, out_dtype, gate_mode, rotation, scale, "auto", chunk,
+                    qk_l2norm=qk_l2norm)
     need = bwd_workspace_bytes(desc)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().gdr_chunk_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(w),
-                             _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(grads["q"]), _ptr(grads["k"]), _ptr(grads["v"]),
-                             _ptr(grads["g"]), _ptr(grads["beta"]), _ptr(grads["w"]), _ptr(grads["S0"]),
-                             _ptr(workspace), ws_bytes, _stream_handle(stream, dev))
+                             _ptr(theta), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(grads["q"]), _ptr(grads["k"]),
+                             _ptr(grads["v"]), _ptr(grads["g"]), _ptr(grads["beta"]), _ptr(grads["w"]),
+                             _ptr(grads["theta"]), _ptr(grads["S0"]), _ptr(workspace), ws_bytes,
+                             _stream_handle(stream, dev))
     _check(st, "gdr_chunk_bwd")
     return grads
 

@@ -213,8 +213,9 @@ def test_kernel_launch_count_without_a_device(G):
 
 def test_backward_checks_its_arguments_without_launching(G):
     """gdr_chunk_bwd: the shapes it does not take are refused before any launch, a missing
-    output or a w without its dw is an argument error, and the workspace size follows the
-    per-head layout (chunk start states plus the chunk matrices)."""
+    output, a w without its dw or a theta that does not match the rotation flag is an argument
+    error, and the workspace size follows the layout (per chunk: three coefficients, the start
+    state, the end state's gradient; one scratch region per CTA of the parallel passes)."""
     import ctypes
     import torch
     L = G.lib()
@@ -222,25 +223,31 @@ def test_backward_checks_its_arguments_without_launching(G):
     d = lambda B, H, T, dk=128, dv=128, **kw: G.fwd_desc(B, H, T, dk, dv, bf, bf, **kw)
     call = lambda desc, ptrs, ws=None, wsb=0: L.gdr_chunk_bwd(ctypes.byref(desc), *ptrs, ws, wsb, None)
     fake = ctypes.c_void_p(1 << 20)        # never dereferenced: every call below fails its checks first
-    full = [fake] * 16                     # q, k, v, g, beta, w, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dw, dS0
-    assert call(d(1, 1, 64, rotation=True), full) == G.GDR_ERR_UNSUPPORTED
+    # q, k, v, g, beta, w, theta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dw, dtheta, dS0
+    rot = [fake] * 18
+    full = list(rot)
+    full[6] = full[16] = None              # no theta / dtheta without rotation
     assert call(d(1, 1, 64, dk=64, dv=128), full) == G.GDR_ERR_UNSUPPORTED
-    assert call(d(1, 1, 64, qk_l2norm=True), full) == G.GDR_ERR_UNSUPPORTED
+    assert call(d(1, 1, 64, rotation=True), full) == G.GDR_ERR_INVALID_ARG      # rotation without theta
+    assert call(d(1, 1, 64), rot) == G.GDR_ERR_INVALID_ARG                      # theta without rotation
+    no_dtheta = list(rot)
+    no_dtheta[16] = None
+    assert call(d(1, 1, 64, rotation=True), no_dtheta) == G.GDR_ERR_INVALID_ARG
     no_dw = list(full)
-    no_dw[14] = None
+    no_dw[15] = None
     assert call(d(1, 1, 64), no_dw) == G.GDR_ERR_INVALID_ARG
     no_dq = list(full)
-    no_dq[9] = None
+    no_dq[10] = None
     assert call(d(1, 1, 64), no_dq) == G.GDR_ERR_INVALID_ARG
     assert call(d(1, 1, 64), full, None, 0) == G.GDR_ERR_WORKSPACE
-    assert G.bwd_workspace_bytes(d(1, 1, 64, rotation=True)) == 0
-    # five d x d fp32 matrices per chunk (three coefficients, the start state, the end state's
-    # gradient), two per head for the chains, and one scratch region per CTA of the parallel
-    # passes (one per SM, at most one per chunk)
-    scratch = 64 * 128 * 18 + 64 * 64 * 7 + 64 * 3 + 128 * 3 + 128 * 128
+    assert call(d(1, 1, 64, rotation=True), rot, None, 0) == G.GDR_ERR_WORKSPACE
+    assert call(d(1, 1, 64, qk_l2norm=True), full, None, 0) == G.GDR_ERR_WORKSPACE
+    # scratch per CTA: 18 C x d tiles, 7 C x C tiles, 5 per-token and 3 per-key vectors, S0p
+    scratch = 64 * 128 * 18 + 64 * 64 * 7 + 64 * 5 + 128 * 3 + 128 * 128
     dd = 128 * 128
-    assert G.bwd_workspace_bytes(d(2, 3, 1000)) == 4 * (6 * 16 * 5 * dd + 6 * 2 * dd + 96 * scratch)
-    assert G.bwd_workspace_bytes(d(4, 16, 4096)) == 4 * (64 * 64 * 5 * dd + 64 * 2 * dd + 148 * scratch)
+    assert G.bwd_workspace_bytes(d(2, 3, 1000)) == 4 * (6 * 16 * 5 * dd + 96 * scratch)
+    assert G.bwd_workspace_bytes(d(4, 16, 4096)) == 4 * (64 * 64 * 5 * dd + 148 * scratch)
+    assert G.bwd_workspace_bytes(d(4, 16, 4096, rotation=True)) == G.bwd_workspace_bytes(d(4, 16, 4096))
     assert G.bwd_workspace_bytes(d(2, 3, 0)) == 0
 
 

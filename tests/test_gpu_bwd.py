@@ -25,25 +25,35 @@ def G():
 
 
 BWD_CASES = [
-    # (B, H, T, d, dtype, gate_mode, untied w, S0, dO, dS_T, gate recipe)
-    (1, 2, 128, 128, "bf16", 1, False, False, True, True, "normal"),
-    (2, 1, 100, 64, "f32", 0, False, True, True, False, "normal"),       # ragged, log-decay gates
-    (1, 3, 200, 32, "bf16", 1, True, True, True, True, "normal"),        # ragged, separate w
-    (1, 1, 64, 128, "f32", 1, False, True, False, True, "normal"),       # only dS_T
-    (2, 2, 257, 128, "bf16", 1, False, True, True, True, "normal"),      # one-token tail
-    (1, 1, 512, 128, "bf16", 1, False, True, True, True, "slow"),        # slow decay, 8 chunks
+    # (B, H, T, d, dtype, gate_mode, untied w, S0, dO, dS_T, gate recipe, rotation, qk_l2norm)
+    (1, 2, 128, 128, "bf16", 1, False, False, True, True, "normal", False, False),
+    (2, 1, 100, 64, "f32", 0, False, True, True, False, "normal", False, False),      # ragged, log-decay gates
+    (1, 3, 200, 32, "bf16", 1, True, True, True, True, "normal", False, False),       # ragged, separate w
+    (1, 1, 64, 128, "f32", 1, False, True, False, True, "normal", False, False),      # only dS_T
+    (2, 2, 257, 128, "bf16", 1, False, True, True, True, "normal", False, False),     # one-token tail
+    (1, 1, 512, 128, "bf16", 1, False, True, True, True, "slow", False, False),       # slow decay, 8 chunks
+    (1, 2, 200, 128, "bf16", 1, False, True, True, True, "normal", True, False),      # rotation, ragged
+    (2, 1, 130, 64, "f32", 0, True, True, True, True, "normal", True, False),         # rotation, log-decay, w
+    (1, 2, 150, 128, "bf16", 1, False, True, True, True, "normal", False, True),      # qk_l2norm
+    (1, 1, 100, 32, "f32", 1, True, True, True, True, "slow", True, True),            # rotation + qk_l2norm
 ]
 
 
 def _case_id(c):
-    B, H, T, d, dt, gm, w, s0, do, ds, gate = c
+    B, H, T, d, dt, gm, w, s0, do, ds, gate, rot, nrm = c
     return f"B{B}H{H}T{T}d{d}_{dt}_g{gm}" + ("_w" if w else "") + ("_s0" if s0 else "") + \
-        ("_dO" if do else "") + ("_dS" if ds else "") + ("_slow" if gate == "slow" else "")
+        ("_dO" if do else "") + ("_dS" if ds else "") + ("_slow" if gate == "slow" else "") + \
+        ("_rot" if rot else "") + ("_l2" if nrm else "")
 
 
 def _inputs(case, seed):
-    B, H, T, d, dt, gm, untied, s0, with_dO, with_dS, gate = case
-    p = I.make_fwd(B, T, H, d, d, dtype=dt, seed=seed, gate=gate, s0_std=0.3 if s0 else None)
+    B, H, T, d, dt, gm, untied, s0, with_dO, with_dS, gate, rot, nrm = case
+    p = I.make_fwd(B, T, H, d, d, dtype=dt, seed=seed, gate=gate, s0_std=0.3 if s0 else None, rotation=rot)
+    if nrm:     # raw q and k of norms far from one (the kernel normalises them)
+        for n in ("q", "k"):
+            x = I.normal(seed, n + "_raw", (B, T, H, d)).astype(np.float32) * \
+                (0.5 + 3.0 * I.uniform(seed, n + "_len", B * T * H).reshape(B, T, H, 1)).astype(np.float32)
+            setattr(p, n, I.to_bf16_bits(x) if dt == "bf16" else x)
     g = p.g if gm == 1 else (-np.logaddexp(0.0, p.g.astype(np.float64))).astype(np.float32)   # log-decay values
     w = I.make_write_strength(seed + 1, (B, T, H)) if untied else None
     dO = I.normal(seed, "dO", (B, T, H, d)).astype(np.float32) if with_dO else None
@@ -63,18 +73,19 @@ def _widen(a):
 def test_backward_parity(G, case):
     import torch
     p, g, w, dO, dS = _inputs(case, 700 + case[2] + case[3])
-    gm = case[5]
-    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "beta", "S0")}
+    gm, rot, nrm = case[5], case[11], case[12]
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "beta", "S0", "theta")}
     gt = U.to_torch(g, "cuda")
     wt, dOt, dSt = U.to_torch(w, "cuda"), U.to_torch(dO, "cuda"), U.to_torch(dS, "cuda")
     grads = G.chunk_bwd(t["q"], t["k"], t["v"], gt, t["beta"], t["S0"], dOt, dSt, gate_mode=gm, w=wt,
-                        out_dtype=t["q"].dtype)
+                        theta=t["theta"], qk_l2norm=nrm, out_dtype=t["q"].dtype)
     torch.cuda.synchronize()
     assert G.query_device_status() == G.GDR_OK
     _, _, ref = gdr_bwd(p.widened("q"), p.widened("k"), p.widened("v"), g.astype(np.float64),
-                        p.widened("beta"), None, p.widened("S0"), _widen(dO), _widen(dS), gate_mode=gm,
-                        scale=p.scale, w=None if w is None else w.astype(np.float64))
-    names = ["q", "k", "v", "g", "beta", "S0"] + (["w"] if w is not None else [])
+                        p.widened("beta"), None if not rot else p.theta.astype(np.float64), p.widened("S0"),
+                        _widen(dO), _widen(dS), gate_mode=gm, scale=p.scale,
+                        w=None if w is None else w.astype(np.float64), qk_l2norm=nrm)
+    names = ["q", "k", "v", "g", "beta", "S0"] + (["w"] if w is not None else []) + (["theta"] if rot else [])
     for n in names:
         got = grads[n].cpu().numpy().astype(np.float64)
         assert np.all(np.isfinite(got)), f"non-finite d{n}"

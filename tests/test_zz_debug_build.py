@@ -1,6 +1,7 @@
 """The debug build (libgdr_debug.so, -DGDR_BOUNDS_CHECK): every kernel tests the index of each
 global-memory access it computes before making it.  On small and ragged shapes through every
-kernel (split, waves, segments, fused, CUDA-core forward, decode, backward) no test fails, and
+kernel (split, waves, segments, fused, CUDA-core forward, decode, backward with and without
+rotation and the L2 normalisation) no test fails, and
 the outputs equal the default build's (the checks change no arithmetic; the compiler may still
 contract a product differently around the added branches, so one rounding step of the output
 type is allowed)."""
@@ -81,6 +82,8 @@ def test_debug_build_decode_and_backward(G):
     gdr, default, dbg = G
     dc = I.make_decode(N=4, H=4, dk=128, dv=128, steps=2, dtype="bf16", seed=9, s_std=0.1)   # 16-byte aligned per step
     p = I.make_fwd(1, 130, 2, 64, 64, dtype="bf16", seed=10, s0_std=0.2)
+    pr = I.make_fwd(2, 77, 1, 32, 32, dtype="f32", seed=12, s0_std=0.2, rotation=True)      # rotation, ragged
+    dS = torch.from_numpy(I.normal(13, "dS_T", (2, 1, 32, 32)).astype(np.float32)).cuda()
     res = {}
     for name, path in (("default", default), ("debug", dbg)):
         gdr.use_library(path)
@@ -91,14 +94,18 @@ def test_debug_build_decode_and_backward(G):
         t = {k: U.to_torch(getattr(p, k), "cuda") for k in ("q", "k", "v", "g", "beta", "S0")}
         dO = torch.from_numpy(I.normal(11, "dO", (1, 130, 2, 64)).astype(np.float32)).cuda().to(torch.bfloat16)
         grads = gdr.chunk_bwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], dO, None)
+        tr = {k: U.to_torch(getattr(pr, k), "cuda") for k in ("q", "k", "v", "g", "beta", "S0", "theta")}
+        grads_r = gdr.chunk_bwd(tr["q"], tr["k"], tr["v"], tr["g"], tr["beta"], tr["S0"], None, dS,
+                                theta=tr["theta"], qk_l2norm=True)
         torch.cuda.synchronize()
         assert gdr.query_device_status() == gdr.GDR_OK
         if name == "debug":
             assert gdr.debug_bounds_site() == 0
-        res[name] = (S, o, grads)
-    Sd, od, gd = res["debug"]
-    S0_, o0, g0 = res["default"]
+        res[name] = (S, o, grads, grads_r)
+    Sd, od, gd, grd = res["debug"]
+    S0_, o0, g0, gr0 = res["default"]
     assert _same(Sd, S0_) and all(_same(a, b) for a, b in zip(od, o0))
-    for n, x in g0.items():
-        if x is not None:
-            assert _same(gd[n], x)
+    for a, b in ((gd, g0), (grd, gr0)):
+        for n, x in b.items():
+            if x is not None:
+                assert _same(a[n], x)
