@@ -397,6 +397,57 @@ GDR_API gdr_status gdr_chunk_bwd(const gdr_fwd_desc* desc,
                                  void* workspace, size_t workspace_bytes, gdr_stream_t stream);
 
 /*
+ * Raven's routed slot memory ("Raven: High-Recall Sequence Modeling with Sparse Memory Routing"
+ * page, section 2.1, routing slot memories, and section 2.2, the Raven architecture): per
+ * (batch, head) a key state Sk and a value state Sv of M = 64 slots (rows) of d values.  Token t:
+ *   - the router keeps the top K of the logits z_t (ties to the lower slot index), takes the
+ *     sigmoid m of the kept ones and normalises them, r_t[i] = m_i / sum of the kept m (zero on the
+ *     other slots); the logits are an input (the projection W x_t belongs to the layer);
+ *   - only the chosen slots decay and are written: with a_t the log-decay of the gate g_t
+ *     (g itself for GDR_GATE_LOGDECAY, -softplus(g) for GDR_GATE_NEG_SOFTPLUS),
+ *     S[i] <- e^{a_t r_t[i]} S[i] + (1 - e^{a_t r_t[i]}) x_t, x = k_t for Sk and v_t for Sv;
+ *     an unchosen slot (r = 0) stays as it is;
+ *   - the readout is softmax attention over the slots of the updated states,
+ *     o_t = sum_i softmax_i(scale q_t . Sk[i]) Sv[i] (with a one-hot router that cycles through
+ *     the slots and a decay that empties the chosen slot, exactly sliding-window attention over
+ *     the last M tokens, the special case the page's section 2.1 names).
+ * The library runs it in chunks of 32 tokens (per-slot cumulative decays, bf16 tensor-core
+ * products, the chunk's writes as sums over the tokens that chose each slot, fp32 states), and
+ * splits long sequences into segments whose start states it composes from the earlier segments'
+ * end states (the chunk transition is diagonal in the slots).
+ */
+typedef struct {
+    int B, H, T;          /* batch, heads, tokens (T >= 0) */
+    int d;                /* head dim of q, k, v and the slot states: 64 or 128 */
+    int slots;            /* M: must be 64 */
+    int topk;             /* K: 1 .. 16 */
+    gdr_dtype qkv_dtype;  /* must be GDR_BF16 */
+    gdr_dtype out_dtype;  /* GDR_BF16 or GDR_F32 */
+    gdr_gate_mode gate_mode;
+    float scale;          /* multiplies q . Sk[i] inside the softmax */
+    int segments;         /* 0: the library chooses; n >= 1: n segments per sequence (at most one
+                             per 32-token chunk) */
+} gdr_raven_desc;
+
+/* Segments per sequence a descriptor runs with, or -1 if it is invalid.  No GPU work. */
+GDR_API int gdr_raven_fwd_segments(const gdr_raven_desc* desc);
+/* Device workspace for gdr_raven_fwd: (B*H) * (segments - 1) * (2*64*d + 64) floats (zero with
+ * one segment), or 0 for an invalid descriptor. */
+GDR_API size_t gdr_raven_fwd_workspace_bytes(const gdr_raven_desc* desc);
+/*
+ *   q, k, v [B,T,H,d] bf16;  z [B,T,H,64] fp32 router logits (finite or -inf);  g [B,T,H] fp32;
+ *   S0k, S0v [B,H,64,d] fp32 initial states or NULL (zero);  o [B,T,H,d] out_dtype;
+ *   Sk_T, Sv_T [B,H,64,d] fp32 final states or NULL (not written).
+ * All device pointers, 16-byte aligned, owned by the caller; asynchronous on `stream`; nothing
+ * is allocated.  Errors: GDR_ERR_INVALID_ARG / GDR_ERR_UNSUPPORTED / GDR_ERR_WORKSPACE before any
+ * launch.  One launch with one segment, two otherwise (the segment states, then the outputs).
+ */
+GDR_API gdr_status gdr_raven_fwd(const gdr_raven_desc* desc, const void* q, const void* k, const void* v,
+                                 const float* z, const float* g, const float* S0k, const float* S0v,
+                                 void* o, float* Sk_T, float* Sv_T, void* workspace,
+                                 size_t workspace_bytes, gdr_stream_t stream);
+
+/*
  * Test hook for the bounded waits of the tensor-core kernel (process-wide, not
  * thread-safe).  wait_limit_ns bounds every mbarrier wait (0 restores the 2 s
  * default).  With skip_first_commit != 0, each later launch never signals its first

@@ -14,6 +14,7 @@
 #include "split_fwd.cuh"
 #include "seg_combine.cuh"
 #include "bwd.cuh"
+#include "raven.cuh"
 
 namespace gdr {
 
@@ -745,6 +746,66 @@ static gdr_status dispatch_bwd_d(const gdr_fwd_desc* d, const bwd::BwdParams& p,
     return launch_bwd<D, float, float>(p, nh, st);
 }
 
+// ---- Raven (routed slot memory) ------------------------------------------------------------
+static gdr_status check_raven_desc(const gdr_raven_desc* d) {
+    if (!d) return fail(GDR_ERR_INVALID_ARG, "descriptor is NULL%s");
+    if (d->B < 0 || d->H < 0 || d->T < 0) return fail(GDR_ERR_INVALID_ARG, "B, H, T must be >= 0%s");
+    if (d->d != 64 && d->d != 128) return fail(GDR_ERR_UNSUPPORTED, "Raven head dim must be 64 or 128%s");
+    if (d->slots != rvn::M) return fail(GDR_ERR_UNSUPPORTED, "Raven needs 64 slots%s");
+    if (d->topk < 1 || d->topk > rvn::KMAX) return fail(GDR_ERR_INVALID_ARG, "topk must be in 1..16%s");
+    if (d->qkv_dtype != GDR_BF16) return fail(GDR_ERR_UNSUPPORTED, "Raven takes bf16 q, k, v%s");
+    if (!dtype_ok(d->out_dtype)) return fail(GDR_ERR_INVALID_ARG, "bad out dtype%s");
+    if (d->gate_mode != GDR_GATE_LOGDECAY && d->gate_mode != GDR_GATE_NEG_SOFTPLUS)
+        return fail(GDR_ERR_INVALID_ARG, "bad gate mode%s");
+    if (d->segments < 0) return fail(GDR_ERR_INVALID_ARG, "segments must be >= 0%s");
+    return GDR_OK;
+}
+
+// Segments per sequence: enough CTAs to cover the SMs, at least 8 chunks per segment, unless
+// the caller fixes the number.
+static void raven_plan(const gdr_raven_desc* d, int* nseg, int* seg_chunks) {
+    const int nc = (d->T + rvn::C - 1) / rvn::C;
+    const long long nh = (long long)d->B * d->H;
+    long long want = d->segments;
+    if (want <= 0) {
+        want = nh > 0 ? device_sm_count() / nh : 1;
+        if (want > nc / 8) want = nc / 8;
+    }
+    if (want < 1) want = 1;
+    if (want > nc) want = nc > 0 ? nc : 1;
+    const int per = nc > 0 ? (int)((nc + want - 1) / want) : 1;
+    *seg_chunks = per;
+    *nseg = nc > 0 ? (nc + per - 1) / per : 1;
+}
+
+static size_t raven_workspace_floats(const gdr_raven_desc* d) {
+    int nseg, per;
+    raven_plan(d, &nseg, &per);
+    const size_t nh = (size_t)d->B * d->H;
+    return nseg > 1 ? nh * (nseg - 1) * (2 * (size_t)rvn::M * d->d + rvn::M) : 0;
+}
+
+template <int D, bool FULL, typename OT>
+static gdr_status launch_raven_kernel(const rvn::RavenParams& p, int grid, cudaStream_t st) {
+    auto kern = rvn::raven_fwd_kernel<D, FULL, OT>;
+    const size_t smem = rvn::Sm<D>::BYTES;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(raven kernel)");
+    kern<<<(unsigned)grid, rvn::NT, smem, st>>>(p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? GDR_OK : cuda_fail(e, FULL ? "launch(raven outputs)" : "launch(raven segment states)");
+}
+
+template <int D, typename OT>
+static gdr_status launch_raven(const rvn::RavenParams& p, cudaStream_t st) {
+    const int nh = p.B * p.H;
+    if (p.nseg > 1) {
+        const gdr_status s = launch_raven_kernel<D, false, OT>(p, nh * (p.nseg - 1), st);
+        if (s != GDR_OK) return s;
+    }
+    return launch_raven_kernel<D, true, OT>(p, nh * p.nseg, st);
+}
+
 }  // namespace gdr
 
 using namespace gdr;
@@ -1026,6 +1087,58 @@ gdr_status gdr_chunk_bwd(const gdr_fwd_desc* d, const void* q, const void* k, co
         case 64: return dispatch_bwd_d<64>(d, p, st);
         default: return dispatch_bwd_d<128>(d, p, st);
     }
+}
+
+int gdr_raven_fwd_segments(const gdr_raven_desc* d) {
+    if (check_raven_desc(d) != GDR_OK) return -1;
+    int nseg, per;
+    raven_plan(d, &nseg, &per);
+    return nseg;
+}
+
+size_t gdr_raven_fwd_workspace_bytes(const gdr_raven_desc* d) {
+    if (check_raven_desc(d) != GDR_OK) return 0;
+    return raven_workspace_floats(d) * sizeof(float);
+}
+
+gdr_status gdr_raven_fwd(const gdr_raven_desc* d, const void* q, const void* k, const void* v, const float* z,
+                         const float* g, const float* S0k, const float* S0v, void* o, float* Sk_T, float* Sv_T,
+                         void* workspace, size_t workspace_bytes, gdr_stream_t stream) {
+    t_detail[0] = 0;
+    gdr_status s = check_raven_desc(d);
+    if (s != GDR_OK) return s;
+    if (d->B == 0 || d->H == 0) return GDR_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const void* ptrs[] = {q, k, v, z, g, S0k, S0v, o, Sk_T, Sv_T, workspace};
+    for (const void* x : ptrs)
+        if (x && !aligned16(x)) return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned%s");
+    const size_t sbytes = (size_t)d->B * d->H * rvn::M * d->d * sizeof(float);
+    if (d->T == 0) {    // no tokens: the final states are the initial ones
+        float* outs[2] = {Sk_T, Sv_T};
+        const float* ins[2] = {S0k, S0v};
+        for (int j = 0; j < 2; ++j) {
+            if (!outs[j]) continue;
+            const cudaError_t e = ins[j] ? cudaMemcpyAsync(outs[j], ins[j], sbytes, cudaMemcpyDeviceToDevice, st)
+                                         : cudaMemsetAsync(outs[j], 0, sbytes, st);
+            if (e != cudaSuccess) return cuda_fail(e, "copy(S_T)");
+        }
+        return GDR_OK;
+    }
+    if (!q || !k || !v || !z || !g || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, z, g and o are required%s");
+    const size_t need = gdr_raven_fwd_workspace_bytes(d);
+    if (need && (!workspace || workspace_bytes < need)) return fail(GDR_ERR_WORKSPACE, "workspace too small%s");
+    rvn::RavenParams p;
+    p.B = d->B; p.H = d->H; p.T = d->T; p.K = d->topk; p.gate_mode = (int)d->gate_mode; p.scale = d->scale;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.k = static_cast<const __nv_bfloat16*>(k);
+    p.v = static_cast<const __nv_bfloat16*>(v);
+    p.z = z; p.g = g; p.S0k = S0k; p.S0v = S0v; p.o = o; p.SkT = Sk_T; p.SvT = Sv_T;
+    raven_plan(d, &p.nseg, &p.seg_chunks);
+    p.segW = static_cast<float*>(workspace);
+    p.segL = p.nseg > 1 ? p.segW + (size_t)d->B * d->H * (p.nseg - 1) * 2 * rvn::M * d->d : nullptr;
+    const bool ob = d->out_dtype == GDR_BF16;
+    if (d->d == 64) return ob ? launch_raven<64, __nv_bfloat16>(p, st) : launch_raven<64, float>(p, st);
+    return ob ? launch_raven<128, __nv_bfloat16>(p, st) : launch_raven<128, float>(p, st);
 }
 
 gdr_status gdr_chunk_fwd_noalloc(const gdr_fwd_desc* d, const void* q, const void* k, const void* v,

@@ -45,6 +45,13 @@ class DecDesc(ctypes.Structure):
                 ("qk_l2norm", ctypes.c_int)]
 
 
+class RavenDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("d", ctypes.c_int),
+                ("slots", ctypes.c_int), ("topk", ctypes.c_int), ("qkv_dtype", ctypes.c_int),
+                ("out_dtype", ctypes.c_int), ("gate_mode", ctypes.c_int), ("scale", ctypes.c_float),
+                ("segments", ctypes.c_int)]
+
+
 class GdrError(RuntimeError):
     def __init__(self, status: int, where: str, detail: str):
         super().__init__(f"{where}: {status_string(status)} ({detail})")
@@ -96,6 +103,13 @@ def lib() -> ctypes.CDLL:
         L.gdr_chunk_bwd.restype = ctypes.c_int
         L.gdr_chunk_bwd.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, fp, vp, fp,
                                     fp, fp, fp, fp, fp, fp, fp, fp, vp, ctypes.c_size_t, vp]
+        L.gdr_raven_fwd_segments.restype = ctypes.c_int
+        L.gdr_raven_fwd_segments.argtypes = [ctypes.POINTER(RavenDesc)]
+        L.gdr_raven_fwd_workspace_bytes.restype = ctypes.c_size_t
+        L.gdr_raven_fwd_workspace_bytes.argtypes = [ctypes.POINTER(RavenDesc)]
+        L.gdr_raven_fwd.restype = ctypes.c_int
+        L.gdr_raven_fwd.argtypes = [ctypes.POINTER(RavenDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp, fp, vp,
+                                    ctypes.c_size_t, vp]
         L.gdr_chunk_fwd_noalloc.restype = ctypes.c_int
         L.gdr_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(FwdDesc), vp, vp, vp, fp, fp, fp, fp, vp, fp, vp]
         L.gdr_debug_set_tc_fault.restype = None
@@ -351,6 +365,58 @@ def chunk_bwd(q, k, v, g, beta, S0=None, dO=None, dS_T=None, *, gate_mode=GATE_N
                              _stream_handle(stream, dev))
     _check(st, "gdr_chunk_bwd")
     return grads
+
+
+def raven_desc(B, H, T, d, topk, out_dtype=torch.bfloat16, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0, segments=0,
+               slots=64) -> RavenDesc:
+    return RavenDesc(B, H, T, d, slots, topk, _dtype_code(torch.bfloat16), _dtype_code(out_dtype), int(gate_mode),
+                     float(scale), int(segments))
+
+
+def raven_segments(desc: RavenDesc) -> int:
+    n = int(lib().gdr_raven_fwd_segments(ctypes.byref(desc)))
+    if n < 0:
+        raise ValueError("invalid Raven descriptor")
+    return n
+
+
+def raven_workspace_bytes(desc: RavenDesc) -> int:
+    return int(lib().gdr_raven_fwd_workspace_bytes(ctypes.byref(desc)))
+
+
+def raven_fwd(q, k, v, z, g, S0k=None, S0v=None, *, topk, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,
+              out_dtype=None, segments=0, want_state=True, workspace=None, stream=None):
+    """Raven's routed slot memory forward (``gdr_raven_fwd``): q, k, v [B,T,H,d] bf16, router
+    logits z [B,T,H,64] fp32, decay gate g [B,T,H] fp32, optional start states S0k, S0v
+    [B,H,64,d] fp32.  Returns (o [B,T,H,d], Sk_T, Sv_T) (the states None unless want_state)."""
+    dev = q.device
+    B, T, H, d = q.shape
+    out_dtype = out_dtype or q.dtype
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k, "k", torch.bfloat16, dev)
+    _need(v, "v", torch.bfloat16, dev)
+    _need(z, "z", torch.float32, dev)
+    _need(g, "g", torch.float32, dev)
+    if tuple(k.shape) != (B, T, H, d) or tuple(v.shape) != (B, T, H, d) or tuple(z.shape) != (B, T, H, 64) \
+            or tuple(g.shape) != (B, T, H):
+        raise ValueError("q, k, v, z, g shapes disagree")
+    for t, n in ((S0k, "S0k"), (S0v, "S0v")):
+        if t is not None:
+            _need(t, n, torch.float32, dev)
+            if tuple(t.shape) != (B, H, 64, d):
+                raise ValueError(f"{n} has the wrong shape")
+    o = torch.empty((B, T, H, d), dtype=out_dtype, device=dev)
+    SkT = torch.empty((B, H, 64, d), dtype=torch.float32, device=dev) if want_state else None
+    SvT = torch.empty((B, H, 64, d), dtype=torch.float32, device=dev) if want_state else None
+    desc = raven_desc(B, H, T, d, topk, out_dtype, gate_mode, scale, segments)
+    need = raven_workspace_bytes(desc)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().gdr_raven_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(g), _ptr(S0k), _ptr(S0v),
+                             _ptr(o), _ptr(SkT), _ptr(SvT), _ptr(workspace), ws_bytes, _stream_handle(stream, dev))
+    _check(st, "gdr_raven_fwd")
+    return o, SkT, SvT
 
 
 def decode_step(q, k, v, g, beta, S, theta=None, *, gate_mode=GATE_NEG_SOFTPLUS, scale=1.0,

@@ -274,3 +274,63 @@ def make_decode(N, H, dk, dv, steps, dtype="bf16", seed=4, s_std=0.02, rotation=
         q, k, v = to_bf16_bits(q), to_bf16_bits(k), to_bf16_bits(v)
     return DecodeInputs(N, H, dk, dv, dtype, GATE_NEG_SOFTPLUS, rotation, q, k, v, a, beta,
                         theta, S, scale)
+
+
+@dataclass
+class RavenInputs:
+    """One problem of Raven's routed slot memory (arrays host numpy, q / k / v bf16 bit patterns)."""
+    B: int
+    T: int
+    H: int
+    d: int
+    K: int
+    gate_mode: int
+    q: np.ndarray               # [B,T,H,d] bf16 bits
+    k: np.ndarray
+    v: np.ndarray
+    z: np.ndarray               # [B,T,H,M] float32 router logits
+    g: np.ndarray               # [B,T,H] float32 decay gate
+    S0k: Optional[np.ndarray]   # [B,H,M,d] float32 or None
+    S0v: Optional[np.ndarray]
+    scale: float
+    name: str = ""
+
+    def widened(self, key: str) -> Optional[np.ndarray]:
+        a = getattr(self, key)
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return bf16_bits_to_f32(a).astype(np.float64)
+        return a.astype(np.float64)
+
+
+def make_raven(B, T, H, d, K=8, seed=5, gate_mode=GATE_NEG_SOFTPLUS, s0_std: Optional[float] = None, M=64,
+               scale: Optional[float] = None, name="") -> RavenInputs:
+    """Random Raven problem: q, k, v ~ N(0,1) rounded to bf16, router logits z ~ N(0,1) per slot,
+    the gate ~ N(0,1) (a raw gate for GATE_NEG_SOFTPLUS) or -|N(0,1)| (a log-decay for
+    GATE_LOGDECAY), start states N(0, s0_std^2) or none, scale 1/sqrt(d) unless given."""
+    q = to_bf16_bits(normal(seed, "rq", (B, T, H, d)))
+    k = to_bf16_bits(normal(seed, "rk", (B, T, H, d)))
+    v = to_bf16_bits(normal(seed, "rv", (B, T, H, d)))
+    z = normal(seed, "rz", (B, T, H, M)).astype(np.float32)
+    g = normal(seed, "rg", (B, T, H))
+    g = (g if gate_mode == GATE_NEG_SOFTPLUS else -np.abs(g)).astype(np.float32)
+    S0k = S0v = None
+    if s0_std is not None:
+        S0k = normal(seed, "rS0k", (B, H, M, d), std=s0_std).astype(np.float32)
+        S0v = normal(seed, "rS0v", (B, H, M, d), std=s0_std).astype(np.float32)
+    return RavenInputs(B, T, H, d, K, gate_mode, q, k, v, z, g, S0k, S0v,
+                       float(d ** -0.5 if scale is None else scale), name)
+
+
+# Raven's workload: the headline forward's shape (B=4, H=16, T=4096, d=128) with 64 slots and
+# top-8 routing (the page fixes neither number).
+RAVEN_CONFIGS = {
+    "raven_b4_h16_t4096_d128": dict(B=4, T=4096, H=16, d=128, K=8, seed=5),
+}
+
+
+def make_raven_config(name: str, **overrides) -> RavenInputs:
+    kw = dict(RAVEN_CONFIGS[name])
+    kw.update(overrides)
+    return make_raven(name=name, **kw)

@@ -256,3 +256,38 @@ def test_default_build_has_no_index_checks(G):
     answers -1 without touching a device."""
     assert G.debug_bounds_site() == -1
     assert G.status_string(G.GDR_ERR_BOUNDS) == "GDR_ERR_BOUNDS"
+
+
+def test_raven_checks_its_arguments_and_plans_segments(G):
+    """gdr_raven_fwd: unsupported shapes and types are refused before any launch, missing
+    inputs are argument errors, the segment plan covers the SMs with at least 8 chunks of 32
+    tokens per segment, and the workspace holds the earlier segments' end states."""
+    import torch
+    L = G.lib()
+    d = lambda B, H, T, dd=128, K=8, **kw: G.raven_desc(B, H, T, dd, K, **kw)
+    fake = ctypes.c_void_p(1 << 20)        # never dereferenced
+    call = lambda desc, ptrs, ws=None, wsb=0: L.gdr_raven_fwd(ctypes.byref(desc), *ptrs, ws, wsb, None)
+    full = [fake] * 10                     # q, k, v, z, g, S0k, S0v, o, Sk_T, Sv_T
+    assert call(d(1, 1, 64, dd=32), full) == G.GDR_ERR_UNSUPPORTED
+    assert call(d(1, 1, 64, slots=32), full) == G.GDR_ERR_UNSUPPORTED
+    assert call(d(1, 1, 64, K=0), full) == G.GDR_ERR_INVALID_ARG
+    assert call(d(1, 1, 64, K=17), full) == G.GDR_ERR_INVALID_ARG
+    bad = d(1, 1, 64)
+    bad.qkv_dtype = 0
+    assert call(bad, full) == G.GDR_ERR_UNSUPPORTED
+    no_z = list(full)
+    no_z[3] = None
+    assert call(d(1, 1, 64), no_z) == G.GDR_ERR_INVALID_ARG
+    mis = list(full)
+    mis[0] = ctypes.c_void_p((1 << 20) + 8)
+    assert call(d(1, 1, 64), mis) == G.GDR_ERR_INVALID_ARG
+    # 64 heads of 128 chunks: two segments on 148 SMs; one head of 128 chunks: 16 of 8 chunks
+    assert G.raven_segments(d(4, 16, 4096)) == 2
+    assert G.raven_segments(d(1, 1, 4096)) == 16
+    assert G.raven_segments(d(1, 1, 100)) == 1
+    assert G.raven_segments(d(1, 1, 100, segments=3)) == 2          # 4 chunks: 2 per segment
+    assert G.raven_segments(d(2, 3, 1000, segments=5)) == 5
+    assert G.raven_workspace_bytes(d(4, 16, 4096)) == 4 * 64 * 1 * (2 * 64 * 128 + 64)
+    assert G.raven_workspace_bytes(d(1, 1, 100)) == 0
+    assert call(d(4, 16, 4096), full, None, 0) == G.GDR_ERR_WORKSPACE
+    assert G.raven_workspace_bytes(d(1, 1, 64, dd=32)) == 0
