@@ -455,6 +455,43 @@ def run_ours(args):
                             "frac": round(b_gbs / peaks["hbm_gbs"], 4), "algorithmic_bytes_per_launch": int(b_bytes)}}
         del bws
 
+    # ---- Raven's routed slot memory (a second recurrence) at the headline shape ----
+    raven = None
+    if not args.no_raven:
+        rcfg = dict(I.RAVEN_CONFIGS["raven_b4_h16_t4096_d128"])
+        rcfg["seed"] = rank_seed(rcfg["seed"], rank)
+        rp = I.make_raven(name="raven_b4_h16_t4096_d128", **rcfg)
+        rt = {n: to(getattr(rp, n)).to(dev) for n in ("q", "k", "v", "z", "g")}
+        rdesc = gdr.raven_desc(rp.B, rp.H, rp.T, rp.d, rp.K, scale=rp.scale)
+        rws = torch.empty(max(16, gdr.raven_workspace_bytes(rdesc)), dtype=torch.uint8, device=dev)
+
+        def rstep():
+            return gdr.raven_fwd(rt["q"], rt["k"], rt["v"], rt["z"], rt["g"], topk=rp.K, scale=rp.scale,
+                                 workspace=rws, stream=stream)
+
+        for _ in range(max(3, args.warmup)):
+            rstep()
+        torch.cuda.synchronize()
+        n_r = max(1, min(args.steps, 10))
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_r):
+            rstep()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        r_ms = max_over_ranks(a.elapsed_time(b_) / n_r, dev)
+        r_tok = rp.B * rp.T * rp.H
+        # q, k, v bf16, 64 router logits fp32, the gate fp32 in; o bf16 out; the final states
+        r_bytes = r_tok * (3 * rp.d * 2 + 64 * 4 + 4 + rp.d * 2) + rp.B * rp.H * 2 * 64 * rp.d * 4
+        r_gbs = r_bytes / (r_ms * 1e-3) / 1e9
+        raven = {"value": round(r_tok / (r_ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s", "us_per_step": round(r_ms * 1e3, 1),
+                 "steps": n_r, "kernel": "gdr_raven_fwd", "workload": "raven_b4_h16_t4096_d128 (64 slots, top-8)",
+                 "segments": gdr.raven_segments(rdesc), "launches_per_step": 2 if gdr.raven_segments(rdesc) > 1 else 1,
+                 "roofline": {"bound": "hbm", "achieved": round(r_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": round(r_gbs / peaks["hbm_gbs"], 4), "algorithmic_bytes_per_launch": int(r_bytes)}}
+        del rt, rws
+        torch.cuda.empty_cache()
+
     # ---- the other forward workloads, each timed the same way on its own inputs ----
     workloads = None
     if not args.no_workloads:
@@ -490,6 +527,7 @@ def run_ours(args):
         "gpu_launches": main["launches"],
         "decode": decode,
         "backward": bwd,
+        "raven": raven,
         "untied": untied,
         "qk_l2norm": l2norm,
         "chunk_mean": cmean,
@@ -583,6 +621,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-workloads", action="store_true", help="skip the other forward workloads")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward pass")
+    ap.add_argument("--no-raven", action="store_true", help="skip the Raven slot-memory forward")
     ap.add_argument("--no-untied", action="store_true", help="skip the separate-write-strength, "
                     "fused-L2-norm and chunk-mean measurements")
     args = ap.parse_args(argv)

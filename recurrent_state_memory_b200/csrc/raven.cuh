@@ -14,8 +14,10 @@
 //   P = softmax over the slots;  PE = P e^{lam};  Bm[t,s] = sum_{i chosen at s} P[t,i] c_s[i] e^{lam_t[i] - lam_s[i]}
 //   O = PE Sv0 + Bm V                                                          (tensor cores)
 //   S_L[i] = e^{lam_L[i]} S0[i] + sum_{s chose i} c_s[i] e^{lam_L[i] - lam_s[i]} x_s   (fp32, sparse)
-// Every exponent is <= 0.  The sums over the chunk's writes follow per-slot token lists built
-// in token order, so the results do not depend on thread timing.
+// Every exponent is <= 0.  The sums over the chunk's writes run over each slot's tokens in
+// token order (a 32-bit mask per slot: bit t set when token t chose the slot), so the results
+// do not depend on thread timing; the per-token tables are kept slot-major so that a warp reads
+// a slot's tokens from one row.
 //
 // Sequence parallelism: the transition of a chunk is diagonal in the slots, so a segment of
 // chunks maps its start state to e^{Lam_seg} S + W_seg (per slot).  A state pass runs every
@@ -37,7 +39,7 @@ constexpr int M = 64;          // slots
 constexpr int KMAX = 16;       // largest top-K
 constexpr int NT = 512;
 constexpr int NW = NT / 32;
-static_assert(NT == C * M / 4 && NT == 8 * M && NW == C / 2, "thread mappings below");
+static_assert(NT == C * M / 4 && NT == 8 * M && NW == C / 2 && C == 32, "thread mappings below (a token per lane)");
 
 struct RavenParams {
     int B, H, T, K, gate_mode;
@@ -70,18 +72,17 @@ struct Sm {
     static constexpr size_t VT = KT + 2ull * C * DP * 2;
     static constexpr size_t ZT = VT + 2ull * C * DP * 2;   // fp32 [2][C][M]
     static constexpr size_t GT = ZT + 2ull * C * M * 4;    // fp32 [2][C]
-    static constexpr size_t LAM = GT + 2ull * C * 4;       // fp32 [C][M]: a r, then lam
-    static constexpr size_t CD = LAM + (size_t)C * M * 4;  // fp32 [C][M]: c (zero where not chosen)
-    static constexpr size_t SC = CD + (size_t)C * M * 4;   // fp32 [C][M + 4]: scores, then P
+    static constexpr int CS = C + 1;                       // row stride of the slot-major tables
+    static constexpr size_t LAMT = GT + 2ull * C * 4;      // fp32 [M][CS]: a r, then lam (slot-major)
+    static constexpr size_t CT = LAMT + (size_t)M * CS * 4;     // fp32 [M][CS]: c (valid where chosen)
+    static constexpr size_t SC = CT + (size_t)M * CS * 4;  // fp32 [C][M + 4]: scores, then P
     static constexpr size_t AB = SC + (size_t)C * (M + 4) * 4;   // fp32 [C][C + 4]: A
     static constexpr size_t PEB = AB + (size_t)C * (C + 4) * 4;  // bf16 [C][M + 8]: P e^{lam}
     static constexpr size_t BB = PEB + (size_t)C * (M + 8) * 2;  // bf16 [C][C + 8]: Bm
     static constexpr size_t PS = BB + (size_t)C * (C + 8) * 2;   // fp32 [8][M]: scan parts
-    static constexpr size_t LST = PS + 8ull * M * 4;             // u8 [M][C]: tokens that chose the slot
-    static constexpr size_t NLS = LST + (size_t)M * C;           // int [M]: their number
-    static constexpr size_t SEL = NLS + (size_t)M * 4;           // u8 [C][KMAX]: chosen slots per token
-    static constexpr size_t CH = SEL + (size_t)C * KMAX;         // u8 [C][M]: chosen flags
-    static constexpr size_t LTOT = CH + (size_t)C * M;           // fp32 [M]: summed log-decay (state pass)
+    static constexpr size_t MSK = PS + 8ull * M * 4;             // u32 [2][M]: tokens that chose the slot
+    static constexpr size_t SEL = MSK + 2ull * M * 4;            // u8 [C][KMAX]: chosen slots per token
+    static constexpr size_t LTOT = SEL + (size_t)C * KMAX;       // fp32 [M]: summed log-decay (state pass)
     static constexpr size_t BYTES = LTOT + (size_t)M * 4;
 };
 
@@ -194,17 +195,16 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
     float* Svf = reinterpret_cast<float*>(sm + L::SVF);
     __nv_bfloat16* Skb = reinterpret_cast<__nv_bfloat16*>(sm + L::SKB);
     __nv_bfloat16* Svb = reinterpret_cast<__nv_bfloat16*>(sm + L::SVB);
-    float* lam = reinterpret_cast<float*>(sm + L::LAM);
-    float* cd = reinterpret_cast<float*>(sm + L::CD);
+    float* lamT = reinterpret_cast<float*>(sm + L::LAMT);
+    float* cT = reinterpret_cast<float*>(sm + L::CT);
+    uint32_t* mskb = reinterpret_cast<uint32_t*>(sm + L::MSK);
+    constexpr int CS = L::CS;
     float* sc = reinterpret_cast<float*>(sm + L::SC);
     float* ab = reinterpret_cast<float*>(sm + L::AB);
     __nv_bfloat16* peb = reinterpret_cast<__nv_bfloat16*>(sm + L::PEB);
     __nv_bfloat16* bb = reinterpret_cast<__nv_bfloat16*>(sm + L::BB);
     float* ps = reinterpret_cast<float*>(sm + L::PS);
-    unsigned char* lst = sm + L::LST;
-    int* nls = reinterpret_cast<int*>(sm + L::NLS);
     unsigned char* sel = sm + L::SEL;
-    unsigned char* ch = sm + L::CH;
     float* ltot = reinterpret_cast<float*>(sm + L::LTOT);
     constexpr int SCS = M + 4, ABS = C + 4, PES = M + 8, BBS = C + 8;
 
@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
         V::stb(Svb + i * DP + c0, av);
     }
     if (tid < M) ltot[tid] = 0.f;
+    if (tid < 2 * M) mskb[tid] = 0u;
 
     // ---- chunk inputs: asynchronous copies into buffer `buf` ----
     auto load_chunk = [&](int c, int buf) {
@@ -272,7 +273,12 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
             cp_async16(zd + r * M + pc, p.z + (ok ? tokrow(t0 + r) : 0) * M + pc, ok);
         }
         float* gd = reinterpret_cast<float*>(sm + L::GT) + (size_t)buf * C;
-        if (tid < C) gd[tid] = t0 + tid < p.T ? p.g[tokrow(t0 + tid)] : 0.f;
+        if (tid < C) {      // one gate per token (stride H floats): 4-byte asynchronous copies
+            const bool ok = t0 + tid < p.T;
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(gd + tid)),
+                         "l"(p.g + (ok ? tokrow(t0 + tid) : 0)), "r"(ok ? 4u : 0u)
+                         : "memory");
+        }
         cp_commit();
     };
 
@@ -288,15 +294,11 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
         const float* zt = reinterpret_cast<const float*>(sm + L::ZT) + (size_t)buf * C * M;
         const float* gt = reinterpret_cast<const float*>(sm + L::GT) + (size_t)buf * C;
 
+        // Slot i's tokens: bit t of msk[i]; its tables lamT[i][t], cT[i][t] hold values only there.
+        uint32_t* msk = mskb + buf * M;
+        if (tid < M) mskb[(buf ^ 1) * M + tid] = 0u;               // for chunk c + 1
         // ---- router: one warp per token (two tokens per warp) ----
         for (int t = warp; t < C; t += NW) {
-            lam[t * M + lane] = 0.f;
-            lam[t * M + lane + 32] = 0.f;
-            cd[t * M + lane] = 0.f;
-            cd[t * M + lane + 32] = 0.f;
-            ch[t * M + lane] = 0;
-            ch[t * M + lane + 32] = 0;
-            __syncwarp();
             if (t0 + t >= p.T) continue;                            // padding: chooses nothing
             // K rounds of a warp-wide maximum of order keys (one redux), the lowest slot index
             // among equal keys taken by two ballots (slots lane < slots lane + 32)
@@ -313,40 +315,45 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
                 if (win == lane + 32) u1 = 0u;
                 if (lane == j) my_i = win;
             }
-            const float my_z = zt[t * M + my_i];
-            const float m = lane < p.K ? 1.f / (1.f + expf(-my_z)) : 0.f;
-            float sum = m;
+            const bool ch0 = u0 == 0u, ch1 = u1 == 0u;             // the lane's slots were chosen
+            const float m0 = ch0 ? 1.f / (1.f + expf(-zt[t * M + lane])) : 0.f;
+            const float m1 = ch1 ? 1.f / (1.f + expf(-zt[t * M + lane + 32])) : 0.f;
+            float sum = m0 + m1;
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            if (lane < p.K) {
-                const float lr = log_decay(gt[t], p.gate_mode) * (m / sum);
-                lam[t * M + my_i] = lr;
-                cd[t * M + my_i] = -expm1f(lr);
-                ch[t * M + my_i] = 1;
-                sel[t * KMAX + lane] = (unsigned char)my_i;
+            const float a = log_decay(gt[t], p.gate_mode);
+            if (ch0) {
+                const float lr = a * (m0 / sum);
+                lamT[lane * CS + t] = lr;
+                cT[lane * CS + t] = -expm1f(lr);
+                atomicOr(&msk[lane], 1u << t);
             }
+            if (ch1) {
+                const float lr = a * (m1 / sum);
+                lamT[(lane + 32) * CS + t] = lr;
+                cT[(lane + 32) * CS + t] = -expm1f(lr);
+                atomicOr(&msk[lane + 32], 1u << t);
+            }
+            if (lane < p.K) sel[t * KMAX + lane] = (unsigned char)my_i;
         }
         __syncthreads();
-        // ---- cumulative log-decay per slot (8 parts of 4 tokens) and the per-slot token lists ----
+        // ---- cumulative log-decay per slot (8 parts of 4 tokens) ----
         {
             const int i = tid & (M - 1), part = tid >> 6;
+            const uint32_t mk = msk[i];
             float run = 0.f;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) run += lam[(part * 4 + u) * M + i];
+            for (int u = 0; u < 4; ++u)
+                if ((mk >> (part * 4 + u)) & 1u) run += lamT[i * CS + part * 4 + u];
             ps[part * M + i] = run;
-            if (tid < M) {
-                int n = 0;
-                for (int s = 0; s < C; ++s)
-                    if (ch[s * M + tid]) lst[tid * C + n++] = (unsigned char)s;
-                nls[tid] = n;
-            }
             __syncthreads();
             float acc = 0.f;
             for (int pp = 0; pp < part; ++pp) acc += ps[pp * M + i];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                acc += lam[(part * 4 + u) * M + i];
-                lam[(part * 4 + u) * M + i] = acc;
+                const int t = part * 4 + u;
+                if ((mk >> t) & 1u) acc += lamT[i * CS + t];
+                lamT[i * CS + t] = acc;
             }
         }
         __syncthreads();
@@ -365,22 +372,22 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
                     for (int e = 0; e < 4; ++e) {
                         const int r = tm * 16 + gid + ((e >> 1) << 3), col = tn * 16 + hh * 8 + 2 * tig + (e & 1);
                         if (isA) ab[r * ABS + col] = p.scale * acc[hh][e];
-                        else sc[r * SCS + col] = p.scale * acc[hh][e] * expf(lam[r * M + col]);
+                        else sc[r * SCS + col] = p.scale * acc[hh][e] * __expf(lamT[col * CS + r]);
                     }
             }
             __syncthreads();
             // ---- the chunk's own writes in the scores ----
             {
-                const int i = tid & (M - 1), tq = tid >> 6, n = nls[i];
+                const int i = tid & (M - 1), tq = tid >> 6;
+                const uint32_t mk = msk[i];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int t = tq + 8 * u;
-                    const float lt = lam[t * M + i];
+                    const float lt = lamT[i * CS + t];
                     float acc = 0.f;
-                    for (int e = 0; e < n; ++e) {
-                        const int s = lst[i * C + e];
-                        if (s > t) break;
-                        acc += ab[t * ABS + s] * cd[s * M + i] * expf(lt - lam[s * M + i]);
+                    for (uint32_t m = mk & ((2u << t) - 1u); m; m &= m - 1u) {      // tokens s <= t
+                        const int s = __ffs(m) - 1;
+                        acc += ab[t * ABS + s] * cT[i * CS + s] * __expf(lt - lamT[i * CS + s]);
                     }
                     sc[t * SCS + i] += acc;
                 }
@@ -399,8 +406,8 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
                 const float p0 = e0 / s, p1 = e1 / s;
                 sc[t * SCS + lane] = p0;
                 sc[t * SCS + lane + 32] = p1;
-                peb[t * PES + lane] = __float2bfloat16_rn(p0 * expf(lam[t * M + lane]));
-                peb[t * PES + lane + 32] = __float2bfloat16_rn(p1 * expf(lam[t * M + lane + 32]));
+                peb[t * PES + lane] = __float2bfloat16_rn(p0 * __expf(lamT[lane * CS + t]));
+                peb[t * PES + lane + 32] = __float2bfloat16_rn(p1 * __expf(lamT[(lane + 32) * CS + t]));
             }
             __syncthreads();
             // ---- Bm[t,s] over the K slots token s chose ----
@@ -413,7 +420,7 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
                     if (s <= t && t0 + s < p.T)
                         for (int j = 0; j < p.K; ++j) {
                             const int i = sel[s * KMAX + j];
-                            acc += sc[t * SCS + i] * cd[s * M + i] * expf(lam[t * M + i] - lam[s * M + i]);
+                            acc += sc[t * SCS + i] * cT[i * CS + s] * __expf(lamT[i * CS + t] - lamT[i * CS + s]);
                         }
                     bb[t * BBS + s] = __float2bfloat16_rn(acc);
                 }
@@ -445,7 +452,10 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
         // ---- state update (fp32) ----
         for (int si = 0; si < M / NW; ++si) {
             const int i = warp + NW * si;
-            const float lL = lam[(C - 1) * M + i], dL = expf(lL);
+            const uint32_t mk = msk[i];
+            const float lL = lamT[i * CS + C - 1], dL = __expf(lL);
+            // this lane's token: its weight in the slot's end state (zero unless it chose the slot)
+            const float fl = ((mk >> lane) & 1u) ? cT[i * CS + lane] * __expf(lL - lamT[i * CS + lane]) : 0.f;
             float ak[CPL], av[CPL];
             V::ld(ak, Skf + i * D + c0);
             V::ld(av, Svf + i * D + c0);
@@ -454,10 +464,9 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
                 ak[u] *= dL;
                 av[u] *= dL;
             }
-            const int n = nls[i];
-            for (int e = 0; e < n; ++e) {
-                const int s = lst[i * C + e];
-                const float f = cd[s * M + i] * expf(lL - lam[s * M + i]);
+            for (uint32_t m = mk; m; m &= m - 1u) {
+                const int s = __ffs(m) - 1;
+                const float f = __shfl_sync(0xffffffffu, fl, s);
                 float xk[CPL], xv[CPL];
                 V::ldb(xk, kt + s * DP + c0);
                 V::ldb(xv, vt + s * DP + c0);
