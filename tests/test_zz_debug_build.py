@@ -1,7 +1,7 @@
 """The debug build (libgdr_debug.so, -DGDR_BOUNDS_CHECK): every kernel tests the index of each
 global-memory access it computes before making it.  On small and ragged shapes through every
 kernel (split, waves, segments, fused, CUDA-core forward, decode, backward with and without
-rotation and the L2 normalisation) no test fails, and
+rotation and the L2 normalisation, Raven's slot memory) no test fails, and
 the outputs equal the default build's (the checks change no arithmetic; the compiler may still
 contract a product differently around the added branches, so one rounding step of the output
 type is allowed)."""
@@ -75,6 +75,25 @@ def test_debug_build_forward(G, case):
     for a, b in zip(got, ref):
         if a is not None:
             assert _same(a, b)
+
+
+def test_debug_build_raven(G):
+    """Raven's two passes (three segments, a ragged tail) on the debug build."""
+    import torch
+    p = I.make_raven(2, 200, 2, 64, K=4, seed=14, s0_std=0.3)
+    t = {n: U.to_torch(getattr(p, n), "cuda") for n in ("q", "k", "v", "z", "g", "S0k", "S0v")}
+    res = {}
+    for name, path in (("default", G[1]), ("debug", G[2])):
+        G[0].use_library(path)
+        out = G[0].raven_fwd(t["q"], t["k"], t["v"], t["z"], t["g"], t["S0k"], t["S0v"], topk=p.K, scale=p.scale,
+                             segments=3)
+        torch.cuda.synchronize()
+        assert G[0].query_device_status() == G[0].GDR_OK
+        if name == "debug":
+            assert G[0].debug_bounds_site() == 0
+        res[name] = [x.clone() for x in out]
+    for a, b in zip(res["debug"], res["default"]):
+        assert _same(a, b)
 
 
 def test_debug_build_decode_and_backward(G):
