@@ -480,11 +480,12 @@ def run_ours(args):
         b_.record(stream)
         torch.cuda.synchronize()
         r_ms = max_over_ranks(a.elapsed_time(b_) / n_r, dev)
-        r_tok = rp.B * rp.T * rp.H
+        r_th = rp.B * rp.T * rp.H          # token-heads (the bytes); tokens are B*T, as in the headline
         # q, k, v bf16, 64 router logits fp32, the gate fp32 in; o bf16 out; the final states
-        r_bytes = r_tok * (3 * rp.d * 2 + 64 * 4 + 4 + rp.d * 2) + rp.B * rp.H * 2 * 64 * rp.d * 4
+        r_bytes = r_th * (3 * rp.d * 2 + 64 * 4 + 4 + rp.d * 2) + rp.B * rp.H * 2 * 64 * rp.d * 4
         r_gbs = r_bytes / (r_ms * 1e-3) / 1e9
-        raven = {"value": round(r_tok / (r_ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s", "us_per_step": round(r_ms * 1e3, 1),
+        raven = {"value": round(rp.B * rp.T / (r_ms * 1e-3) / 1e6, 3), "unit": "Mtokens/s",
+                 "us_per_step": round(r_ms * 1e3, 1),
                  "steps": n_r, "kernel": "gdr_raven_fwd", "workload": "raven_b4_h16_t4096_d128 (64 slots, top-8)",
                  "segments": gdr.raven_segments(rdesc), "launches_per_step": 2 if gdr.raven_segments(rdesc) > 1 else 1,
                  "roofline": {"bound": "hbm", "achieved": round(r_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
