@@ -126,3 +126,31 @@ def test_backward_matches_a_finite_difference_of_the_forward_kernel(G):
     fd = (loss(t["beta"] + h * dirn) - loss(t["beta"] - h * dirn)) / (2 * h)
     an = float((grads["beta"].double() * dirn.double()).sum())
     assert abs(fd - an) <= 2e-3 * max(1.0, abs(an)), (fd, an)
+
+
+def test_backward_full_size_sampled_heads(G):
+    """The bench workload (B=4 H=16 T=4096 d=128, bf16) with dO and dS_T: every gradient of
+    three sampled heads against the oracle's chunked restatement of the reverse sweep
+    (oracle/backward.py::chunk_bwd_head, pinned to the token sweep on the CPU)."""
+    import torch
+    from oracle.backward import chunk_bwd_head
+    p = I.make_config("b4_h16_t4096_d128")
+    t = {key: U.to_torch(getattr(p, key), "cuda") for key in ("q", "k", "v", "g", "beta")}
+    dO = I.to_bf16_bits(I.normal(780, "dO", (p.B, p.T, p.H, p.dv)).astype(np.float32))
+    dS = I.normal(781, "dS_T", (p.B, p.H, p.dv, p.dk), std=0.5).astype(np.float32)
+    grads = G.chunk_bwd(t["q"], t["k"], t["v"], t["g"], t["beta"], None, U.to_torch(dO, "cuda"),
+                        U.to_torch(dS, "cuda"), gate_mode=p.gate_mode, scale=p.scale, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert G.query_device_status() == G.GDR_OK
+    dO64 = I.bf16_bits_to_f32(dO).astype(np.float64)
+    for (b, h) in ((0, 0), (2, 9), (3, 15)):
+        sel = lambda a: a[b, :, h]
+        _, _, ref = chunk_bwd_head(sel(p.widened("q")), sel(p.widened("k")), sel(p.widened("v")),
+                                   sel(p.widened("g")), sel(p.widened("beta")), None, sel(dO64),
+                                   dS[b, h].astype(np.float64), p.gate_mode, p.scale, None)
+        for n in ("q", "k", "v", "g", "beta"):
+            got = grads[n][b, :, h].cpu().numpy().astype(np.float64)
+            e = U.max_rel(got, ref[n])
+            assert e <= TOL_BWD, f"d{n} of head ({b},{h}): max-rel error {e:.3e}"
+        e = U.max_rel(grads["S0"][b, h].cpu().numpy().astype(np.float64), ref["S0"])
+        assert e <= TOL_BWD, f"dS0 of head ({b},{h}): max-rel error {e:.3e}"
