@@ -431,8 +431,10 @@ typedef struct {
 
 /* Segments per sequence a descriptor runs with, or -1 if it is invalid.  No GPU work. */
 GDR_API int gdr_raven_fwd_segments(const gdr_raven_desc* desc);
-/* Device workspace for gdr_raven_fwd: (B*H) * (segments - 1) * (2*64*d + 64) floats (zero with
- * one segment), or 0 for an invalid descriptor. */
+/* Device workspace for gdr_raven_fwd: (B*H) * units * (2*64*d + 64) floats, where the units are
+ * the pieces (a divisor of the segment length, at least 4 chunks of 32 tokens, short enough for
+ * about two waves of CTAs) of the chunks before the last segment whose end states the first
+ * launch computes; zero with one segment, or for an invalid descriptor. */
 GDR_API size_t gdr_raven_fwd_workspace_bytes(const gdr_raven_desc* desc);
 /*
  *   q, k, v [B,T,H,d] bf16;  z [B,T,H,64] fp32 router logits (finite or -inf);  g [B,T,H] fp32;

@@ -778,11 +778,31 @@ static void raven_plan(const gdr_raven_desc* d, int* nseg, int* seg_chunks) {
     *nseg = nc > 0 ? (nc + per - 1) / per : 1;
 }
 
+// State units of the state pass: the chunks before the last segment, in units of a divisor of
+// the segment length, halved while a unit keeps at least the length that gives about two waves
+// of state CTAs (and at least 4 chunks).
+static void raven_units(const gdr_raven_desc* d, int nseg, int seg_chunks, int* nsub, int* sub_chunks) {
+    if (nseg <= 1) {
+        *nsub = 0;
+        *sub_chunks = seg_chunks;
+        return;
+    }
+    const long long nh = (long long)d->B * d->H;
+    long long want = (2LL * device_sm_count() + nh - 1) / nh;          // units per sequence
+    if (want < nseg - 1) want = nseg - 1;
+    const long long target = ((long long)(nseg - 1) * seg_chunks + want - 1) / want;
+    int sub = seg_chunks;
+    while (sub % 2 == 0 && sub / 2 >= target && sub / 2 >= 4) sub /= 2;
+    *sub_chunks = sub;
+    *nsub = (nseg - 1) * (seg_chunks / sub);
+}
+
 static size_t raven_workspace_floats(const gdr_raven_desc* d) {
-    int nseg, per;
+    int nseg, per, nsub, sub;
     raven_plan(d, &nseg, &per);
+    raven_units(d, nseg, per, &nsub, &sub);
     const size_t nh = (size_t)d->B * d->H;
-    return nseg > 1 ? nh * (nseg - 1) * (2 * (size_t)rvn::M * d->d + rvn::M) : 0;
+    return nh * (size_t)nsub * (2 * (size_t)rvn::M * d->d + rvn::M);
 }
 
 template <int D, bool FULL, typename OT>
@@ -799,8 +819,8 @@ static gdr_status launch_raven_kernel(const rvn::RavenParams& p, int grid, cudaS
 template <int D, typename OT>
 static gdr_status launch_raven(const rvn::RavenParams& p, cudaStream_t st) {
     const int nh = p.B * p.H;
-    if (p.nseg > 1) {
-        const gdr_status s = launch_raven_kernel<D, false, OT>(p, nh * (p.nseg - 1), st);
+    if (p.nsub > 0) {
+        const gdr_status s = launch_raven_kernel<D, false, OT>(p, nh * p.nsub, st);
         if (s != GDR_OK) return s;
     }
     return launch_raven_kernel<D, true, OT>(p, nh * p.nseg, st);
@@ -1134,8 +1154,9 @@ gdr_status gdr_raven_fwd(const gdr_raven_desc* d, const void* q, const void* k, 
     p.v = static_cast<const __nv_bfloat16*>(v);
     p.z = z; p.g = g; p.S0k = S0k; p.S0v = S0v; p.o = o; p.SkT = Sk_T; p.SvT = Sv_T;
     raven_plan(d, &p.nseg, &p.seg_chunks);
+    raven_units(d, p.nseg, p.seg_chunks, &p.nsub, &p.sub_chunks);
     p.segW = static_cast<float*>(workspace);
-    p.segL = p.nseg > 1 ? p.segW + (size_t)d->B * d->H * (p.nseg - 1) * 2 * rvn::M * d->d : nullptr;
+    p.segL = p.nsub > 0 ? p.segW + (size_t)d->B * d->H * p.nsub * 2 * rvn::M * d->d : nullptr;
     const bool ob = d->out_dtype == GDR_BF16;
     if (d->d == 64) return ob ? launch_raven<64, __nv_bfloat16>(p, st) : launch_raven<64, float>(p, st);
     return ob ? launch_raven<128, __nv_bfloat16>(p, st) : launch_raven<128, float>(p, st);

@@ -19,10 +19,11 @@
 // do not depend on thread timing; the per-token tables are kept slot-major so that a warp reads
 // a slot's tokens from one row.
 //
-// Sequence parallelism: the transition of a chunk is diagonal in the slots, so a segment of
-// chunks maps its start state to e^{Lam_seg} S + W_seg (per slot).  A state pass runs every
-// segment but the last from the zero state (W_seg, Lam_seg into the workspace); the output pass
-// then starts segment g from S0 composed with the segments before it.
+// Sequence parallelism: the transition of a chunk is diagonal in the slots, so a run of chunks
+// maps its start state to e^{Lam} S + W (per slot).  A state pass runs the chunks before the
+// last output segment, cut into units shorter than a segment (so that its CTAs fill the SMs),
+// each from the zero state (W, Lam into the workspace); the output pass then starts segment g
+// from S0 composed, in order, with every unit before it.
 //
 // One 512-thread CTA per (head, segment) and about 208 KB of shared memory at D = 128: the fp32
 // states, their bf16 copies (the MMA operands), double-buffered q / k / v / z tiles of the next
@@ -54,9 +55,11 @@ struct RavenParams {
     void* o;                  // [B,T,H,D]
     float* SkT;               // [B,H,M,D] or nullptr
     float* SvT;               // [B,H,M,D] or nullptr
-    int nseg, seg_chunks;     // segments per sequence, chunks per segment
-    float* segW;              // [B*H][nseg-1][2][M][D]: each segment's end states from zero
-    float* segL;              // [B*H][nseg-1][M]: each segment's total log-decay per slot
+    int nseg, seg_chunks;     // output segments per sequence, chunks per segment
+    int nsub, sub_chunks;     // state units per sequence (covering the segments before the last),
+                              // chunks per unit (a divisor of seg_chunks)
+    float* segW;              // [B*H][nsub][2][M][D]: each unit's end states from zero
+    float* segL;              // [B*H][nsub][M]: each unit's total log-decay per slot
 };
 
 // Shared-memory layout (byte offsets).
@@ -209,12 +212,13 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
     constexpr int SCS = M + 4, ABS = C + 4, PES = M + 8, BBS = C + 8;
 
     const int tid = (int)threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nsegw = FULL ? p.nseg : p.nseg - 1;
+    const int nsegw = FULL ? p.nseg : p.nsub;
     const int hd = (int)blockIdx.x / nsegw, seg = (int)blockIdx.x % nsegw;
     const int b = hd / p.H, h = hd % p.H;
     if (!GDR_INB(hd < p.B * p.H, 701)) return;
     const int nc = (p.T + C - 1) / C;
-    const int c_begin = seg * p.seg_chunks, c_end = min(nc, c_begin + p.seg_chunks);
+    const int span = FULL ? p.seg_chunks : p.sub_chunks;
+    const int c_begin = seg * span, c_end = min(nc, c_begin + span);
     const size_t MD = (size_t)M * D;
     auto tokrow = [&](int t) -> size_t { return ((size_t)b * p.T + t) * p.H + h; };
 
@@ -231,8 +235,8 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
         if (FULL && p.S0k) V::ld(ak, p.S0k + (size_t)hd * MD + (size_t)i * D + c0);
         if (FULL && p.S0v) V::ld(av, p.S0v + (size_t)hd * MD + (size_t)i * D + c0);
         if (FULL)
-            for (int s2 = 0; s2 < seg; ++s2) {
-                const size_t base = ((size_t)hd * (p.nseg - 1) + s2);
+            for (int s2 = 0; s2 < seg * (p.seg_chunks / p.sub_chunks); ++s2) {
+                const size_t base = ((size_t)hd * p.nsub + s2);
                 const float dk = expf(p.segL[base * M + i]);
                 float wk[CPL], wv[CPL];
                 V::ld(wk, p.segW + base * 2 * MD + (size_t)i * D + c0);
@@ -492,7 +496,7 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
         V::ld(ak, Skf + i * D + c0);
         V::ld(av, Svf + i * D + c0);
         if (!FULL) {
-            const size_t base = (size_t)hd * (p.nseg - 1) + seg;
+            const size_t base = (size_t)hd * p.nsub + seg;
             V::st(p.segW + base * 2 * MD + (size_t)i * D + c0, ak);
             V::st(p.segW + base * 2 * MD + MD + (size_t)i * D + c0, av);
             if (lane == 0) p.segL[base * M + i] = ltot[i];
