@@ -48,6 +48,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace gdr {
 namespace bwd {
@@ -813,6 +814,204 @@ __global__ void __launch_bounds__(NT, 1) bwd_chain_kernel(BwdParams p) {
     run(false, 0, -1, 1, nullptr, 0, 2);
     if (p.dS0)
         for (int i = tid; i < DD; i += NT) p.dS0[(size_t)hd * DD + i] = S[(i / D) * SS + i % D];
+}
+
+// Pass 2 on the tensor cores (d = 128): the same chains, one step S <- X_c + S op(A_c) as
+// tcgen05 kind::tf32 MMAs (M = N = 128) with each operand split into a tf32 high part and
+// remainder (hi hi + hi lo + lo hi: fp32 accuracy).  S (hi, lo) is the A operand in tensor memory
+// (lane = row), op(A_c) (hi, lo) the B operand in shared memory (K-major, 128-byte swizzle), and
+// the accumulator starts as X_c (B_c forwards, G_c backwards).  Warps 0-3 own the TMEM rows
+// (X_c in, the new S out to the workspace and back into TMEM as hi / lo); the other warps split
+// A_c into the B operand; thread 0 issues the MMAs; the next A_c is fetched asynchronously
+// while the MMAs run.
+constexpr uint32_t TC_BHI = 0, TC_BLO = 65536, TC_RAW = 131072;     // byte offsets (1024-aligned base)
+constexpr int TC_RS = 132;                                            // row stride of the raw A_c (floats)
+constexpr uint32_t TC_BAR = TC_RAW + 128u * TC_RS * 4u;
+constexpr size_t TC_SMEM_BYTES = TC_BAR + 64 + 1024;                 // + barrier, TMEM slot, alignment
+constexpr uint32_t TC_COL_D = 0, TC_COL_HI = 128, TC_COL_LO = 256;   // TMEM columns
+
+// byte offset of element (row n, k) of a 128 x 128 tf32 operand, K-major, 128-byte swizzle
+__device__ __forceinline__ uint32_t tf32_koff(uint32_t n, uint32_t k) {
+    return (k >> 5) * 16384u + tc::sw128_off(n, (k & 31u) >> 2) + (k & 3u) * 4u;
+}
+
+__global__ void __launch_bounds__(NT, 1) bwd_chain_tc_kernel(BwdParams p) {
+    using namespace tc;
+    constexpr int D = 128;
+    constexpr int DD = D * D;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
+    uint8_t* base = smem_raw + (sb - raw_u32);
+    float* raw = reinterpret_cast<float*>(base + TC_RAW);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(base + TC_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + TC_BAR + 16);
+    int* fail = reinterpret_cast<int*>(base + TC_BAR + 20);
+    const int tid = (int)threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int hd = (int)blockIdx.x, nc = (p.T + C - 1) / C;
+    const uint64_t limit = 2000000000ull;
+    if (!GDR_INB(hd < p.B * p.H, 405)) return;     // (the whole CTA)
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        *fail = 0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tq = tbase + ((uint32_t)((warp & 3) * 32) << 16);
+    const int row = (warp & 3) * 32 + lane;          // warps 0-3: this thread's row of S
+    auto coef = [&](int c, int k) -> const float* { return p.coef + (((size_t)hd * nc + c) * 3 + k) * DD; };
+    auto prefetch = [&](int c) {
+        for (int i = tid; i < DD / 4; i += NT) {
+            const int r = (4 * i) / D, cc = (4 * i) % D;
+            cp_async16(raw + r * TC_RS + cc, coef(c, 0) + 4 * i);
+        }
+        cp_async_commit();
+    };
+    // row `row` of S (fp32, 128 values) -> TMEM hi / lo columns; also to `keep` (a workspace row)
+    auto put_rows = [&](const float (&v)[32], int g) {
+        float hi[32], lo[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            hi[u] = __uint_as_float(tf32_hi(v[u]));
+            lo[u] = v[u] - hi[u];
+        }
+        tmem_st16(tq + TC_COL_HI + g * 32, *reinterpret_cast<const float(*)[16]>(hi));
+        tmem_st16(tq + TC_COL_HI + g * 32 + 16, *reinterpret_cast<const float(*)[16]>(hi + 16));
+        tmem_st16(tq + TC_COL_LO + g * 32, *reinterpret_cast<const float(*)[16]>(lo));
+        tmem_st16(tq + TC_COL_LO + g * 32 + 16, *reinterpret_cast<const float(*)[16]>(lo + 16));
+    };
+    // the start matrix (S0 forwards, dS_T backwards) into TMEM and kept at `keep`
+    auto start = [&](const float* src, float* keep) {
+        if (warp < 4) {
+#pragma unroll 1
+            for (int g = 0; g < 4; ++g) {
+                float v[32];
+#pragma unroll
+                for (int u4 = 0; u4 < 8; ++u4) {
+                    const float4 x = src ? *reinterpret_cast<const float4*>(src + (size_t)row * D + g * 32 + 4 * u4)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[4 * u4] = x.x; v[4 * u4 + 1] = x.y; v[4 * u4 + 2] = x.z; v[4 * u4 + 3] = x.w;
+                }
+                put_rows(v, g);
+                if (keep) {
+#pragma unroll
+                    for (int u4 = 0; u4 < 8; ++u4)
+                        *reinterpret_cast<float4*>(keep + (size_t)row * D + g * 32 + 4 * u4) =
+                            make_float4(v[4 * u4], v[4 * u4 + 1], v[4 * u4 + 2], v[4 * u4 + 3]);
+                }
+            }
+            tmem_wait_st();
+        }
+    };
+    uint32_t phase = 0;
+    // n steps from chunk c0 in direction dc: S <- coef(c, add_k) + S op(A_c), kept at
+    // keep + (hd * nc + c + shift) * DD unless keep is null; returns false on a timeout
+    auto run = [&](bool fwd, int c0, int dc, int n, float* keep, int shift, int add_k, float* last_out) -> bool {
+        if (n > 0) prefetch(c0);
+        for (int st = 0; st < n; ++st) {
+            const int c = c0 + st * dc;
+            cp_async_wait_all();
+            __syncthreads();                          // A_c landed; the last step's MMAs are done
+            if (warp >= 4) {                          // A_c -> B operand (hi, lo)
+                const int t = tid - 128;
+                for (int e = t; e < DD; e += NT - 128) {
+                    // B(n, k) = A_c[k][n] forwards, A_c[n][k] backwards; consecutive threads take
+                    // consecutive k, so that the swizzled stores are conflict-free
+                    const int nn = e / D, kk = e % D;
+                    const float x = fwd ? raw[kk * TC_RS + nn] : raw[nn * TC_RS + kk];
+                    const float hi = __uint_as_float(tf32_hi(x));
+                    const uint32_t off = tf32_koff((uint32_t)nn, (uint32_t)kk);
+                    *reinterpret_cast<float*>(base + TC_BHI + off) = hi;
+                    *reinterpret_cast<float*>(base + TC_BLO + off) = x - hi;
+                }
+            } else {                                   // X_c -> the accumulator
+                const float* xs = coef(c, add_k);
+#pragma unroll 1
+                for (int g = 0; g < 4; ++g) {
+                    float v[32];
+#pragma unroll
+                    for (int u4 = 0; u4 < 8; ++u4) {
+                        const float4 x = *reinterpret_cast<const float4*>(xs + (size_t)row * D + g * 32 + 4 * u4);
+                        v[4 * u4] = x.x; v[4 * u4 + 1] = x.y; v[4 * u4 + 2] = x.z; v[4 * u4 + 3] = x.w;
+                    }
+                    tmem_st16(tq + TC_COL_D + g * 32, *reinterpret_cast<const float(*)[16]>(v));
+                    tmem_st16(tq + TC_COL_D + g * 32 + 16, *reinterpret_cast<const float(*)[16]>(v + 16));
+                }
+                tmem_wait_st();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();                          // B operand and accumulator ready; raw is free
+            tc_fence_after();
+            if (st + 1 < n) prefetch(c + dc);
+            if (tid == 0) {
+                const uint32_t id = idesc_tf32(128, 128);
+#pragma unroll 1
+                for (int term = 0; term < 3; ++term) {      // hi hi, lo hi, hi lo
+                    const uint32_t acol = term == 1 ? TC_COL_LO : TC_COL_HI;
+                    const uint32_t boff = term == 2 ? TC_BLO : TC_BHI;
+#pragma unroll
+                    for (int ks = 0; ks < 16; ++ks) {
+                        const uint32_t kb = ks >> 2, kin = (ks & 3) * 32;
+                        mma_tf32_ts(tbase + TC_COL_D, tbase + acol + ks * 8,
+                                    sdesc_sw128(sb + boff + kb * 16384 + kin, 16, 1024), id, 1);
+                    }
+                }
+                mma_commit(bar);
+                if (!mbar_wait_bounded(bar, phase, limit)) *fail = 1;
+            }
+            phase ^= 1u;
+            __syncthreads();
+            tc_fence_after();
+            if (*fail) return false;
+            if (warp < 4) {                            // the new S: kept, and back into TMEM
+                float* kp = keep ? keep + ((size_t)hd * nc + c + shift) * DD : last_out;
+#pragma unroll 1
+                for (int g = 0; g < 4; ++g) {
+                    float v[32];
+                    tmem_ld32(tq + TC_COL_D + g * 32, v);
+                    if (kp) {
+#pragma unroll
+                        for (int u4 = 0; u4 < 8; ++u4)
+                            *reinterpret_cast<float4*>(kp + (size_t)row * D + g * 32 + 4 * u4) =
+                                make_float4(v[4 * u4], v[4 * u4 + 1], v[4 * u4 + 2], v[4 * u4 + 3]);
+                    }
+                    put_rows(v, g);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+        }
+        return true;
+    };
+    bool ok = true;
+    // forward: S_0 kept at ckpt[0]; S_{c+1} = B_c + S_c A_c kept at ckpt[c + 1], c = 0 .. nc-2
+    start(p.S0 ? p.S0 + (size_t)hd * DD : nullptr, p.ckpt + (size_t)hd * nc * DD);
+    ok = run(true, 0, 1, nc - 1, p.ckpt, 1, 1, nullptr);
+    // backward: dS_L(nc-1) = dS_T kept at dsl[nc-1]; dS_L(c-1) = G_c + dS_L(c) A_c^T kept at
+    // dsl[c-1], c = nc-1 .. 1; then dS0 = G_0 + dS_L(0) A_0^T
+    if (ok) {
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        start(p.dS_T ? p.dS_T + (size_t)hd * DD : nullptr, p.dsl + ((size_t)hd * nc + nc - 1) * DD);
+        ok = run(false, nc - 1, -1, nc - 1, p.dsl, -1, 2, nullptr);
+    }
+    if (ok) ok = run(false, 0, -1, 1, nullptr, 0, 2, p.dS0 ? p.dS0 + (size_t)hd * DD : nullptr);
+    if (!ok && tid == 0) atomicOr(&g_device_status, 1u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 512);
+    }
 }
 
 // Shared memory of the chain kernel: the carried matrix and two buffers of A_c.

@@ -730,7 +730,10 @@ static gdr_status launch_bwd(const bwd::BwdParams& p, int nh, cudaStream_t st) {
     gdr_status s = launch_bwd_kernel(bwd::bwd_coef_kernel<D, D, QT, OT>, grid, bwd::SMEM_BYTES, p, st,
                                      "launch(backward coefficients)");
     if (s != GDR_OK) return s;
-    s = launch_bwd_kernel(bwd::bwd_chain_kernel<D>, nh, bwd::chain_smem_bytes<D>(), p, st, "launch(backward chains)");
+    if constexpr (D == 128)    // the chains on tcgen05 (tf32, three-way split)
+        s = launch_bwd_kernel(bwd::bwd_chain_tc_kernel, nh, bwd::TC_SMEM_BYTES, p, st, "launch(backward chains)");
+    else
+        s = launch_bwd_kernel(bwd::bwd_chain_kernel<D>, nh, bwd::chain_smem_bytes<D>(), p, st, "launch(backward chains)");
     if (s != GDR_OK) return s;
     return launch_bwd_kernel(bwd::bwd_grad_kernel<D, D, QT, OT>, grid, bwd::SMEM_BYTES, p, st,
                              "launch(backward gradients)");
