@@ -355,8 +355,8 @@ GDR_API int gdr_chunk_fwd_kernel_launches(const gdr_fwd_desc* desc);
  * "Semidirect Fourier Delta Attention" page, "Constructive Chunk-WY Theorem" and the exact
  * affine chunk transfer) in three launches: every chunk's transfer coefficients in parallel
  * (S_L = S0 A_c + B_c and dS0 = G_c + dS_L A_c^T need no state), one short chain per (batch,
- * head) for the chunk start states and the end-state gradients, then every chunk's gradients in
- * parallel.  fp32 throughout (tensor-core products with split-tf32 operands).  With rotation
+ * head) for the chunk start states and the end-state gradients (on tcgen05 at d = 128), then
+ * every chunk's gradients in parallel.  fp32 throughout (tensor-core products with split-tf32 operands).  With rotation
  * ("Semidirect Fourier Delta Attention" page, "Core architecture", 2x2 rotation-decay blocks) the
  * key pairs are complex numbers and the adjoints of the complex decay products are their
  * conjugates; with qk_l2norm the gradients of q and k are taken through the normalisation
