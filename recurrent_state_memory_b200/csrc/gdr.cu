@@ -577,9 +577,13 @@ static gdr_status run_segments(const gdr_fwd_desc* d, const FwdParams& p, cudaSt
 
 template <int DK, bool ROT, typename QT, typename OT>
 static gdr_status launch_decode(const dec::DecParams& p, cudaStream_t st) {
-    const int row_blocks = (p.dv + dec::ROWS_PER_CTA - 1) / dec::ROWS_PER_CTA;
-    const long long grid = (long long)p.N * p.H * row_blocks;
-    if (grid > 0x7fffffffLL) return fail(GDR_ERR_INVALID_ARG, "N*H too large%s");
+    // persistent: at most CTAS_PER_SM CTAs per SM, each warp walking 16-row work items
+    const long long items = (long long)p.N * p.H * (p.dv / dec::RI);
+    if (items > 0x7fffffffLL) return fail(GDR_ERR_INVALID_ARG, "N*H too large%s");
+    const long long need = (items + dec::WARPS - 1) / dec::WARPS;
+    const long long cap = (long long)device_sm_count() * dec::CTAS_PER_SM;
+    const long long grid = need < cap ? need : cap;
+    if (grid <= 0) return GDR_OK;
     dec::decode_kernel<DK, ROT, QT, OT><<<(unsigned)grid, dec::WARPS * 32, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launch(decode kernel)");
