@@ -128,10 +128,6 @@ static bool waves_fit(const gdr_fwd_desc* d, int sms) {
     const long long rem = waves_remainder(d, sms);
     return rem > 0 && split_fits_heads(rem, sms, d->T);
 }
-// The chains kernel (spl) takes any number of heads (each chain runs its heads one after
-// another) and the segments of the sequence-parallel form.
-static bool chains_fit(const gdr_fwd_desc* d, int sms) { return (long long)d->B * d->H >= 1 && sms >= 2 && d->T > 64; }
-
 static bool segments_pay(long long nh, long long T, int sms);
 
 // The algorithm a descriptor runs with.  AUTO: the CUDA-core kernel for shapes and dtypes the
