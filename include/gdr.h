@@ -431,10 +431,11 @@ typedef struct {
 
 /* Segments per sequence a descriptor runs with, or -1 if it is invalid.  No GPU work. */
 GDR_API int gdr_raven_fwd_segments(const gdr_raven_desc* desc);
-/* Device workspace for gdr_raven_fwd: (B*H) * units * (2*64*d + 64) floats, where the units are
- * the pieces (a divisor of the segment length, at least 4 chunks of 32 tokens, short enough for
- * about two waves of CTAs) of the chunks before the last segment whose end states the first
- * launch computes; zero with one segment, or for an invalid descriptor. */
+/* Device workspace for gdr_raven_fwd: every token's routing record (B*T*H * 144 bytes, rounded up
+ * to 256), then (B*H) * units * (2*64*d + 64) floats, where the units are the pieces (a divisor of
+ * the segment length, at least 4 chunks of 32 tokens, short enough for about two waves of CTAs)
+ * of the chunks before the last segment whose end states the state pass computes; 0 when
+ * B, H or T is 0, or for an invalid descriptor. */
 GDR_API size_t gdr_raven_fwd_workspace_bytes(const gdr_raven_desc* desc);
 /*
  *   q, k, v [B,T,H,d] bf16;  z [B,T,H,64] fp32 router logits (finite or -inf);  g [B,T,H] fp32;
@@ -442,7 +443,8 @@ GDR_API size_t gdr_raven_fwd_workspace_bytes(const gdr_raven_desc* desc);
  *   Sk_T, Sv_T [B,H,64,d] fp32 final states or NULL (not written).
  * All device pointers, 16-byte aligned, owned by the caller; asynchronous on `stream`; nothing
  * is allocated.  Errors: GDR_ERR_INVALID_ARG / GDR_ERR_UNSUPPORTED / GDR_ERR_WORKSPACE before any
- * launch.  One launch with one segment, two otherwise (the segment states, then the outputs).
+ * launch.  Two launches with one segment (the router for every token, then the outputs), three
+ * otherwise (the router, the state units, the outputs).
  */
 GDR_API gdr_status gdr_raven_fwd(const gdr_raven_desc* desc, const void* q, const void* k, const void* v,
                                  const float* z, const float* g, const float* S0k, const float* S0v,

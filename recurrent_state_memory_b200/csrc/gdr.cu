@@ -800,12 +800,16 @@ static void raven_units(const gdr_raven_desc* d, int nseg, int seg_chunks, int* 
     *nsub = (nseg - 1) * (seg_chunks / sub);
 }
 
-static size_t raven_workspace_floats(const gdr_raven_desc* d) {
+// Workspace: every token's routing record (rounded up to 256 bytes), then the state units.
+static size_t raven_route_bytes(const gdr_raven_desc* d) {
+    return ((size_t)d->B * d->T * d->H * rvn::ROUTE_BYTES + 255) / 256 * 256;
+}
+static size_t raven_workspace_bytes_(const gdr_raven_desc* d) {
     int nseg, per, nsub, sub;
     raven_plan(d, &nseg, &per);
     raven_units(d, nseg, per, &nsub, &sub);
     const size_t nh = (size_t)d->B * d->H;
-    return nh * (size_t)nsub * (2 * (size_t)rvn::M * d->d + rvn::M);
+    return raven_route_bytes(d) + nh * (size_t)nsub * (2 * (size_t)rvn::M * d->d + rvn::M) * sizeof(float);
 }
 
 template <int D, bool FULL, typename OT>
@@ -822,6 +826,13 @@ static gdr_status launch_raven_kernel(const rvn::RavenParams& p, int grid, cudaS
 template <int D, typename OT>
 static gdr_status launch_raven(const rvn::RavenParams& p, cudaStream_t st) {
     const int nh = p.B * p.H;
+    {   // the router, one warp per (token, head)
+        const long long n_tok = (long long)p.B * p.T * p.H;
+        const long long blocks = (n_tok + 7) / 8, cap = (long long)device_sm_count() * 8;
+        rvn::raven_route_kernel<<<(unsigned)(blocks < cap ? blocks : cap), 256, 0, st>>>(p);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "launch(raven router)");
+    }
     if (p.nsub > 0) {
         const gdr_status s = launch_raven_kernel<D, false, OT>(p, nh * p.nsub, st);
         if (s != GDR_OK) return s;
@@ -1121,7 +1132,8 @@ int gdr_raven_fwd_segments(const gdr_raven_desc* d) {
 
 size_t gdr_raven_fwd_workspace_bytes(const gdr_raven_desc* d) {
     if (check_raven_desc(d) != GDR_OK) return 0;
-    return raven_workspace_floats(d) * sizeof(float);
+    if (d->B == 0 || d->H == 0 || d->T == 0) return 0;
+    return raven_workspace_bytes_(d);
 }
 
 gdr_status gdr_raven_fwd(const gdr_raven_desc* d, const void* q, const void* k, const void* v, const float* z,
@@ -1149,7 +1161,7 @@ gdr_status gdr_raven_fwd(const gdr_raven_desc* d, const void* q, const void* k, 
     }
     if (!q || !k || !v || !z || !g || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, z, g and o are required%s");
     const size_t need = gdr_raven_fwd_workspace_bytes(d);
-    if (need && (!workspace || workspace_bytes < need)) return fail(GDR_ERR_WORKSPACE, "workspace too small%s");
+    if (!workspace || workspace_bytes < need) return fail(GDR_ERR_WORKSPACE, "workspace too small%s");
     rvn::RavenParams p;
     p.B = d->B; p.H = d->H; p.T = d->T; p.K = d->topk; p.gate_mode = (int)d->gate_mode; p.scale = d->scale;
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -1158,7 +1170,8 @@ gdr_status gdr_raven_fwd(const gdr_raven_desc* d, const void* q, const void* k, 
     p.z = z; p.g = g; p.S0k = S0k; p.S0v = S0v; p.o = o; p.SkT = Sk_T; p.SvT = Sv_T;
     raven_plan(d, &p.nseg, &p.seg_chunks);
     raven_units(d, p.nseg, p.seg_chunks, &p.nsub, &p.sub_chunks);
-    p.segW = static_cast<float*>(workspace);
+    p.route = static_cast<unsigned char*>(workspace);
+    p.segW = reinterpret_cast<float*>(p.route + raven_route_bytes(d));
     p.segL = p.nsub > 0 ? p.segW + (size_t)d->B * d->H * p.nsub * 2 * rvn::M * d->d : nullptr;
     const bool ob = d->out_dtype == GDR_BF16;
     if (d->d == 64) return ob ? launch_raven<64, __nv_bfloat16>(p, st) : launch_raven<64, float>(p, st);

@@ -25,9 +25,11 @@
 // each from the zero state (W, Lam into the workspace); the output pass then starts segment g
 // from S0 composed, in order, with every unit before it.
 //
-// One 512-thread CTA per (head, segment) and about 208 KB of shared memory at D = 128: the fp32
-// states, their bf16 copies (the MMA operands), double-buffered q / k / v / z tiles of the next
-// chunk (cp.async, zero-filled past T), and the chunk's tables.
+// The router runs first, for every token at once (`raven_route_kernel`: one warp per token and
+// head, the whole GPU busy), and leaves each token's chosen slots and weights in the workspace.
+// Then one 512-thread CTA per (head, segment) and about 205 KB of shared memory at D = 128: the
+// fp32 states, their bf16 copies (the MMA operands), double-buffered q / k / v tiles and routing
+// records of the next chunk (cp.async, zero-filled past T), and the chunk's tables.
 #pragma once
 
 #include "common.cuh"
@@ -60,7 +62,13 @@ struct RavenParams {
                               // chunks per unit (a divisor of seg_chunks)
     float* segW;              // [B*H][nsub][2][M][D]: each unit's end states from zero
     float* segL;              // [B*H][nsub][M]: each unit's total log-decay per slot
+    unsigned char* route;     // [B*T*H][ROUTE_BYTES]: each token's chosen slots and weights
 };
+
+// A token's routing record: the chosen slots (in the order chosen), then a_t r_t[i] and
+// c = 1 - e^{a_t r_t[i]} for each of them.
+constexpr int ROUTE_BYTES = KMAX + 2 * 4 * KMAX;     // 144
+constexpr int ROUTE_LR = KMAX, ROUTE_C = KMAX + 4 * KMAX;
 
 // Shared-memory layout (byte offsets).
 template <int D>
@@ -73,10 +81,9 @@ struct Sm {
     static constexpr size_t QT = SVB + (size_t)M * DP * 2; // bf16 [2][C][DP]
     static constexpr size_t KT = QT + 2ull * C * DP * 2;
     static constexpr size_t VT = KT + 2ull * C * DP * 2;
-    static constexpr size_t ZT = VT + 2ull * C * DP * 2;   // fp32 [2][C][M]
-    static constexpr size_t GT = ZT + 2ull * C * M * 4;    // fp32 [2][C]
+    static constexpr size_t RT = VT + 2ull * C * DP * 2;   // [2][C][ROUTE_BYTES] routing records
     static constexpr int CS = C + 1;                       // row stride of the slot-major tables
-    static constexpr size_t LAMT = GT + 2ull * C * 4;      // fp32 [M][CS]: a r, then lam (slot-major)
+    static constexpr size_t LAMT = RT + 2ull * C * ROUTE_BYTES;   // fp32 [M][CS]: a r, then lam (slot-major)
     static constexpr size_t CT = LAMT + (size_t)M * CS * 4;     // fp32 [M][CS]: c (valid where chosen)
     static constexpr size_t SC = CT + (size_t)M * CS * 4;  // fp32 [C][M + 4]: scores, then P
     static constexpr size_t AB = SC + (size_t)C * (M + 4) * 4;   // fp32 [C][C + 4]: A
@@ -186,6 +193,43 @@ __device__ __forceinline__ void tile_nn(float (&acc)[2][4], const __nv_bfloat16*
     }
 }
 
+// The router of every token, one warp per (token, head), before the chunked passes: K rounds of
+// a warp-wide maximum of order-preserving keys of the fp32 logits (one redux each), the lowest
+// slot index among equal keys taken by two ballots (slots lane < slots lane + 32); then the
+// kept sigmoid scores normalised, a_t r_t and c = 1 - e^{a_t r_t} per chosen slot.
+__global__ void __launch_bounds__(256) raven_route_kernel(RavenParams p) {
+    const int lane = (int)threadIdx.x & 31;
+    const long long n_tok = (long long)p.B * p.T * p.H;
+    const long long W = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long n = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < n_tok; n += W) {
+        const float* zr = p.z + n * M;
+        uint32_t u0 = order_key(zr[lane]), u1 = order_key(zr[lane + 32]);
+        int my_i = 0;
+        for (int j = 0; j < p.K; ++j) {
+            const bool first = u0 >= u1;
+            const uint32_t cand = first ? u0 : u1;
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, cand);
+            const uint32_t b0 = __ballot_sync(0xffffffffu, cand == mx && first);
+            const uint32_t b1 = __ballot_sync(0xffffffffu, cand == mx && !first);
+            const int win = b0 ? __ffs(b0) - 1 : 32 + __ffs(b1) - 1;
+            if (win == lane) u0 = 0u;
+            if (win == lane + 32) u1 = 0u;
+            if (lane == j) my_i = win;
+        }
+        const float m = lane < p.K ? 1.f / (1.f + expf(-zr[my_i])) : 0.f;
+        float sum = m;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane < p.K && GDR_INB(n < n_tok, 703)) {
+            unsigned char* rec = p.route + n * ROUTE_BYTES;
+            const float lr = log_decay(p.g[n], p.gate_mode) * (m / sum);
+            rec[lane] = (unsigned char)my_i;
+            reinterpret_cast<float*>(rec + ROUTE_LR)[lane] = lr;
+            reinterpret_cast<float*>(rec + ROUTE_C)[lane] = -expm1f(lr);
+        }
+    }
+}
+
 // FULL = false: the state pass (segment from the zero state; end state and summed log-decay to
 // the workspace).  FULL = true: the output pass.
 template <int D, bool FULL, typename OT>
@@ -270,18 +314,11 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
             cp_async16(kd + r * DP + pc, p.k + src, ok);
             cp_async16(vd + r * DP + pc, p.v + src, ok);
         }
-        float* zd = reinterpret_cast<float*>(sm + L::ZT) + (size_t)buf * C * M;
-        for (int i = tid; i < C * M / 4; i += NT) {
-            const int r = i / (M / 4), pc = (i % (M / 4)) * 4;
+        unsigned char* rd = sm + L::RT + (size_t)buf * C * ROUTE_BYTES;
+        for (int i = tid; i < C * (ROUTE_BYTES / 16); i += NT) {
+            const int r = i / (ROUTE_BYTES / 16), pc = (i % (ROUTE_BYTES / 16)) * 16;
             const bool ok = t0 + r < p.T;
-            cp_async16(zd + r * M + pc, p.z + (ok ? tokrow(t0 + r) : 0) * M + pc, ok);
-        }
-        float* gd = reinterpret_cast<float*>(sm + L::GT) + (size_t)buf * C;
-        if (tid < C) {      // one gate per token (stride H floats): 4-byte asynchronous copies
-            const bool ok = t0 + tid < p.T;
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(gd + tid)),
-                         "l"(p.g + (ok ? tokrow(t0 + tid) : 0)), "r"(ok ? 4u : 0u)
-                         : "memory");
+            cp_async16(rd + r * ROUTE_BYTES + pc, p.route + (ok ? tokrow(t0 + r) : 0) * ROUTE_BYTES + pc, ok);
         }
         cp_commit();
     };
@@ -295,50 +332,22 @@ __global__ void __launch_bounds__(NT, 1) raven_fwd_kernel(RavenParams p) {
         const __nv_bfloat16* qt = reinterpret_cast<const __nv_bfloat16*>(sm + L::QT) + (size_t)buf * C * DP;
         const __nv_bfloat16* kt = reinterpret_cast<const __nv_bfloat16*>(sm + L::KT) + (size_t)buf * C * DP;
         const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(sm + L::VT) + (size_t)buf * C * DP;
-        const float* zt = reinterpret_cast<const float*>(sm + L::ZT) + (size_t)buf * C * M;
-        const float* gt = reinterpret_cast<const float*>(sm + L::GT) + (size_t)buf * C;
+        const unsigned char* rt = sm + L::RT + (size_t)buf * C * ROUTE_BYTES;
 
         // Slot i's tokens: bit t of msk[i]; its tables lamT[i][t], cT[i][t] hold values only there.
         uint32_t* msk = mskb + buf * M;
         if (tid < M) mskb[(buf ^ 1) * M + tid] = 0u;               // for chunk c + 1
-        // ---- router: one warp per token (two tokens per warp) ----
-        for (int t = warp; t < C; t += NW) {
-            if (t0 + t >= p.T) continue;                            // padding: chooses nothing
-            // K rounds of a warp-wide maximum of order keys (one redux), the lowest slot index
-            // among equal keys taken by two ballots (slots lane < slots lane + 32)
-            uint32_t u0 = order_key(zt[t * M + lane]), u1 = order_key(zt[t * M + lane + 32]);
-            int my_i = 0;
-            for (int j = 0; j < p.K; ++j) {
-                const bool first = u0 >= u1;
-                const uint32_t cand = first ? u0 : u1;
-                const uint32_t mx = __reduce_max_sync(0xffffffffu, cand);
-                const uint32_t b0 = __ballot_sync(0xffffffffu, cand == mx && first);
-                const uint32_t b1 = __ballot_sync(0xffffffffu, cand == mx && !first);
-                const int win = b0 ? __ffs(b0) - 1 : 32 + __ffs(b1) - 1;
-                if (win == lane) u0 = 0u;
-                if (win == lane + 32) u1 = 0u;
-                if (lane == j) my_i = win;
+        // ---- the chunk's routing (computed by raven_route_kernel): into the slot-major tables ----
+        {
+            const int t = tid >> 4, j = tid & 15;                   // 32 tokens x 16 entries
+            if (j < p.K && t0 + t < p.T) {                          // padding chooses nothing
+                const unsigned char* rr = rt + t * ROUTE_BYTES;
+                const int i = rr[j];
+                lamT[i * CS + t] = reinterpret_cast<const float*>(rr + ROUTE_LR)[j];
+                cT[i * CS + t] = reinterpret_cast<const float*>(rr + ROUTE_C)[j];
+                atomicOr(&msk[i], 1u << t);
+                sel[t * KMAX + j] = (unsigned char)i;
             }
-            const bool ch0 = u0 == 0u, ch1 = u1 == 0u;             // the lane's slots were chosen
-            const float m0 = ch0 ? 1.f / (1.f + expf(-zt[t * M + lane])) : 0.f;
-            const float m1 = ch1 ? 1.f / (1.f + expf(-zt[t * M + lane + 32])) : 0.f;
-            float sum = m0 + m1;
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            const float a = log_decay(gt[t], p.gate_mode);
-            if (ch0) {
-                const float lr = a * (m0 / sum);
-                lamT[lane * CS + t] = lr;
-                cT[lane * CS + t] = -expm1f(lr);
-                atomicOr(&msk[lane], 1u << t);
-            }
-            if (ch1) {
-                const float lr = a * (m1 / sum);
-                lamT[(lane + 32) * CS + t] = lr;
-                cT[(lane + 32) * CS + t] = -expm1f(lr);
-                atomicOr(&msk[lane + 32], 1u << t);
-            }
-            if (lane < p.K) sel[t * KMAX + lane] = (unsigned char)my_i;
         }
         __syncthreads();
         // ---- cumulative log-decay per slot (8 parts of 4 tokens) ----

@@ -289,8 +289,12 @@ def test_raven_checks_its_arguments_and_plans_segments(G):
     assert G.raven_segments(d(2, 3, 1000, segments=5)) == 5
     # the state units: 64 chunks before the last segment, cut to 16-chunk units (4 x 64 heads
     # = 256 state CTAs, about two waves on 148 SMs)
-    assert G.raven_workspace_bytes(d(4, 16, 4096)) == 4 * 64 * 4 * (2 * 64 * 128 + 64)
-    assert G.raven_workspace_bytes(d(1, 1, 4096)) == 4 * 1 * 30 * (2 * 64 * 128 + 64)   # 16 segments of 8, units of 4
-    assert G.raven_workspace_bytes(d(1, 1, 100)) == 0
+    # every token's routing record (144 bytes, the total rounded up to 256), then the state units
+    route = lambda n: (n * 144 + 255) // 256 * 256
+    assert G.raven_workspace_bytes(d(4, 16, 4096)) == route(4 * 4096 * 16) + 4 * 64 * 4 * (2 * 64 * 128 + 64)
+    assert G.raven_workspace_bytes(d(1, 1, 4096)) == route(4096) + 4 * 1 * 30 * (2 * 64 * 128 + 64)   # 16 segments of 8, units of 4
+    assert G.raven_workspace_bytes(d(1, 1, 100)) == route(100)
+    assert G.raven_workspace_bytes(d(1, 1, 0)) == 0
     assert call(d(4, 16, 4096), full, None, 0) == G.GDR_ERR_WORKSPACE
+    assert call(d(1, 1, 100), full, None, 0) == G.GDR_ERR_WORKSPACE
     assert G.raven_workspace_bytes(d(1, 1, 64, dd=32)) == 0
