@@ -129,7 +129,7 @@ constexpr size_t SMEM_BYTES = sizeof(float) * SMEM_FLOATS;
 // stride ls, float4 at a time
 __device__ __forceinline__ void stage(float* dst, int ls, const float* src, int ld, int rows, int cols) {
     const int c4 = cols >> 2;
-#pragma unroll 4
+#pragma unroll 16
     for (int i = (int)threadIdx.x; i < rows * c4; i += NT) {
         const int r = i / c4, c = (i % c4) * 4;
         *reinterpret_cast<float4*>(dst + r * ls + c) = *reinterpret_cast<const float4*>(src + (size_t)r * ld + c);
